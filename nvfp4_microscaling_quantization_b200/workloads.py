@@ -1,0 +1,179 @@
+"""Seeded synthetic input generators for the quantization workloads.
+
+This module holds no quantization arithmetic: it only draws bf16 tensors
+with the shapes and value distributions of the linear-layer tensors that
+block-scaled NVFP4 training quantizes (weights, activations, gradients), and
+names the calls each workload makes.  Both the CUDA path (through bench.py and
+the GPU tests) and the CPU oracle (through the tests) read the same tensors
+from here.
+
+Every tensor is drawn on the host with a torch CPU generator seeded by the
+workload seed, in float32, then rounded to bf16 (round-to-nearest-even).  The
+draws happen in the order written below, so a (workload, seed) pair always
+gives the same bits.
+
+Distributions (the pages' workloads are the weight, activation and gradient
+tensors of LLM linear layers, quantized forward with RTN / 4-over-6 / IF4 and
+backward with SR / MS-EDEN):
+  normal(std)        : std * N(0, 1)
+  outlier_normal     : std * N(0, 1), then 1% of entries (Bernoulli mask) x10
+  student_t3(std)    : N(0,1) / sqrt(chi2_3 / 3), chi2_3 = sum of 3 squared
+                       N(0,1) draws, times std / sqrt(3) (t_3 has variance 3)
+  laplace_channels   : Laplace(0, 1) (inverse CDF of U(-1/2, 1/2)) times a
+                       per-column scale 10^U(-1, 1) (log-uniform in [0.1, 10])
+"""
+from dataclasses import dataclass, field
+from typing import Dict, List, Tuple
+
+import torch
+
+ROWWISE, TRANSPOSED = 0, 1
+RTN, SR, MS_EDEN, IF4, FOUR_OVER_SIX = 0, 1, 2, 3, 4
+MODE_NAMES = {RTN: "rtn", SR: "sr", MS_EDEN: "ms_eden", IF4: "if4", FOUR_OVER_SIX: "4over6"}
+LAYOUT_NAMES = {ROWWISE: "rowwise", TRANSPOSED: "transposed"}
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return g
+
+
+def normal(shape, std: float, gen: torch.Generator) -> torch.Tensor:
+    return (torch.randn(shape, generator=gen, dtype=torch.float32) * std).to(torch.bfloat16)
+
+
+def outlier_normal(shape, std: float, frac: float, factor: float, gen: torch.Generator) -> torch.Tensor:
+    x = torch.randn(shape, generator=gen, dtype=torch.float32) * std
+    mask = torch.rand(shape, generator=gen, dtype=torch.float32) < frac
+    x = torch.where(mask, x * factor, x)
+    return x.to(torch.bfloat16)
+
+
+def student_t3(shape, std: float, gen: torch.Generator) -> torch.Tensor:
+    z = torch.randn(shape, generator=gen, dtype=torch.float32)
+    chi2 = torch.zeros(shape, dtype=torch.float32)
+    for _ in range(3):
+        n = torch.randn(shape, generator=gen, dtype=torch.float32)
+        chi2.addcmul_(n, n)
+    t = z / torch.sqrt(chi2 / 3.0)
+    return (t * (std / 3.0 ** 0.5)).to(torch.bfloat16)
+
+
+def laplace_channels(shape, gen: torch.Generator) -> torch.Tensor:
+    rows, cols = shape
+    u = torch.rand(shape, generator=gen, dtype=torch.float32) - 0.5
+    lap = -torch.sign(u) * torch.log1p(-2.0 * u.abs())
+    col_scale = torch.pow(10.0, torch.rand((1, cols), generator=gen, dtype=torch.float32) * 2.0 - 1.0)
+    return (lap * col_scale).to(torch.bfloat16)
+
+
+@dataclass(frozen=True)
+class Call:
+    """One quantization call of a workload: which tensor, layout, mode, RHT group."""
+    tensor: str
+    layout: int
+    mode: int
+    rht_group: int
+
+    @property
+    def name(self) -> str:
+        g = f"g{self.rht_group}" if self.rht_group else "norht"
+        return f"{self.tensor}.{LAYOUT_NAMES[self.layout]}.{MODE_NAMES[self.mode]}.{g}"
+
+
+@dataclass
+class Workload:
+    name: str
+    seed: int
+    shapes: Dict[str, Tuple[int, int]]
+    calls: List[Call] = field(default_factory=list)
+    description: str = ""
+
+    def tensors(self) -> Dict[str, torch.Tensor]:
+        return _GENERATORS[self.name](self)
+
+    def elements(self, call: Call) -> int:
+        r, c = self.shapes[call.tensor]
+        return r * c
+
+
+def _small(w):
+    g = _gen(w.seed)
+    return {"x": normal(w.shapes["x"], 1.0, g)}
+
+
+def _weight(w):
+    g = _gen(w.seed)
+    return {"w": outlier_normal(w.shapes["w"], 0.02, 0.01, 10.0, g)}
+
+
+def _gradient(w):
+    g = _gen(w.seed)
+    return {"g": student_t3(w.shapes["g"], 1e-3, g)}
+
+
+def _activation(w):
+    g = _gen(w.seed)
+    return {"a": laplace_channels(w.shapes["a"], g)}
+
+
+def _mlp_up(w):
+    g = _gen(w.seed)
+    x = normal(w.shapes["x"], 1.0, g)
+    wt = normal(w.shapes["w"], 0.02, g)
+    dy = student_t3(w.shapes["dy"], 1e-4, g)
+    return {"x": x, "w": wt, "dy": dy}
+
+
+_GENERATORS = {"small": _small, "weight": _weight, "gradient": _gradient,
+               "activation": _activation, "mlp_up": _mlp_up}
+
+
+def small(rows=256, cols=256) -> Workload:
+    """256x256 N(0,1), seed 0: RTN and SR with and without a 128-point RHT, MS-EDEN with it."""
+    calls = [Call("x", ROWWISE, RTN, 0), Call("x", ROWWISE, RTN, 128),
+             Call("x", ROWWISE, SR, 0), Call("x", ROWWISE, SR, 128),
+             Call("x", ROWWISE, MS_EDEN, 128)]
+    return Workload("small", 0, {"x": (rows, cols)}, calls, "256x256 N(0,1)")
+
+
+def weight(rows=4096, cols=4096) -> Workload:
+    """Weight-like 4096x4096 N(0, 0.02^2) with 1% outliers x10, seed 1: RTN and 4/6 row-wise."""
+    calls = [Call("w", ROWWISE, RTN, 0), Call("w", ROWWISE, FOUR_OVER_SIX, 0)]
+    return Workload("weight", 1, {"w": (rows, cols)}, calls, "4096x4096 N(0,0.02) + 1% x10 outliers")
+
+
+def gradient(rows=8192, cols=4096) -> Workload:
+    """Gradient-like 8192x4096 Student-t3 with std 1e-3, seed 2: MS-EDEN and SR, g=128, both layouts."""
+    calls = [Call("g", lay, mode, 128) for mode in (MS_EDEN, SR) for lay in (ROWWISE, TRANSPOSED)]
+    return Workload("gradient", 2, {"g": (rows, cols)}, calls, "8192x4096 Student-t3 std 1e-3")
+
+
+def activation(rows=16384, cols=8192) -> Workload:
+    """Activation-like 16384x8192 Laplace(0,1) x per-channel 10^U(-1,1), seed 3: IF4 with and without RHT."""
+    calls = [Call("a", ROWWISE, IF4, 0), Call("a", ROWWISE, IF4, 128)]
+    return Workload("activation", 3, {"a": (rows, cols)}, calls, "16384x8192 Laplace x log-uniform channel scale")
+
+
+def mlp_up(tokens=16384, d_model=4096, d_ff=14336) -> Workload:
+    """One Llama-style MLP up-projection training step, seed 4.
+
+    X [tokens, d_model] N(0,1), W [d_ff, d_model] N(0, 0.02^2), dY [tokens, d_ff]
+    Student-t3 std 1e-4.  Forward Y = X W^T: RTN on X and W along d_model.
+    Backward dX = dY W: MS-EDEN along d_ff on dY (row-wise) and W (transposed);
+    dW = dY^T X: MS-EDEN along tokens on dY (transposed) and X (transposed).
+    """
+    calls = [Call("x", ROWWISE, RTN, 0), Call("w", ROWWISE, RTN, 0),
+             Call("dy", ROWWISE, MS_EDEN, 128), Call("w", TRANSPOSED, MS_EDEN, 128),
+             Call("dy", TRANSPOSED, MS_EDEN, 128), Call("x", TRANSPOSED, MS_EDEN, 128)]
+    return Workload("mlp_up", 4, {"x": (tokens, d_model), "w": (d_ff, d_model), "dy": (tokens, d_ff)},
+                    calls, "MLP up-projection step: X 16384x4096, W 14336x4096, dY 16384x14336")
+
+
+ALL = {"small": small, "weight": weight, "gradient": gradient, "activation": activation, "mlp_up": mlp_up}
+
+
+def bf16_bits(t: torch.Tensor):
+    """bf16 tensor (CPU) -> numpy uint16 array of its bit patterns (no copy of semantics)."""
+    return t.contiguous().view(torch.int16).numpy().view("uint16")

@@ -1,0 +1,230 @@
+"""CPU oracle for block-scaled NVFP4 quantization -- TEST INFRASTRUCTURE ONLY.
+
+A ctypes wrapper over oracle/nvfp4_oracle.c (plain C99, binary32 round-to-
+nearest-even, no contraction).  Only tests/, __graft_entry__.smoke() and the
+CPU-baseline leg of bench.py may import this package; the CUDA library and its
+Python binding never do.
+
+Every function takes and returns numpy arrays on the host.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+ROWWISE, TRANSPOSED = 0, 1
+RTN, SR, MS_EDEN, IF4, FOUR_OVER_SIX = 0, 1, 2, 3, 4
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        _lib = ctypes.CDLL(path)
+        _declare(_lib)
+    return _lib
+
+
+def _declare(L):
+    P = ctypes.c_void_p
+    i64, u64, i32, f32 = ctypes.c_int64, ctypes.c_uint64, ctypes.c_int, ctypes.c_float
+    L.oracle_philox4x32_10.argtypes = [P, P, P]
+    L.oracle_philox4x32_10.restype = None
+    L.oracle_uniform_element.argtypes = [u64, u64]
+    L.oracle_uniform_element.restype = f32
+    L.oracle_uniform_block.argtypes = [u64, u64]
+    L.oracle_uniform_block.restype = f32
+    L.oracle_rht_sign.argtypes = [u64, i32]
+    L.oracle_rht_sign.restype = f32
+    L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+    L.oracle_e2m1_decode.restype = f32
+    L.oracle_e2m1_rtn.argtypes = [f32]
+    L.oracle_e2m1_rtn.restype = ctypes.c_uint8
+    L.oracle_e2m1_sr.argtypes = [f32, f32]
+    L.oracle_e2m1_sr.restype = ctypes.c_uint8
+    L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.oracle_e4m3_decode.restype = f32
+    L.oracle_e4m3_rne_sat.argtypes = [f32]
+    L.oracle_e4m3_rne_sat.restype = ctypes.c_uint8
+    L.oracle_e4m3_ru_sat.argtypes = [f32]
+    L.oracle_e4m3_ru_sat.restype = ctypes.c_uint8
+    L.oracle_e4m3_sr.argtypes = [f32, f32]
+    L.oracle_e4m3_sr.restype = ctypes.c_uint8
+    L.oracle_rht_scale.argtypes = [i32]
+    L.oracle_rht_scale.restype = f32
+    L.oracle_rht_rows.argtypes = [P, i64, i64, i32, u64, i32, P]
+    L.oracle_rht_rows.restype = i32
+    L.oracle_amax.argtypes = [P, i64, i64, i64, i32, i32, u64, P]
+    L.oracle_amax.restype = i32
+    L.oracle_global_scale.argtypes = [f32, i32]
+    L.oracle_global_scale.restype = f32
+    L.oracle_quantize_rows.argtypes = [P, i64, i64, i64, i32, i32, i32, u64, P, i64, i64, P, P, P]
+    L.oracle_quantize_rows.restype = i32
+    L.oracle_quantize.argtypes = [P, i64, i64, i64, i32, i32, i32, u64, P, P, P, P]
+    L.oracle_quantize.restype = i32
+    L.oracle_dequantize.argtypes = [P, P, f32, i64, i64, i32, i32, u64, i32, P]
+    L.oracle_dequantize.restype = i32
+    L.oracle_rht_view.argtypes = [P, i64, i64, i64, i32, i32, u64, P]
+    L.oracle_rht_view.restype = i32
+    L.oracle_if4_constants.argtypes = [P, P]
+    L.oracle_if4_constants.restype = None
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _check(st):
+    if st != 0:
+        raise OracleError(f"oracle status {st}")
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _as_bf16_bits(x):
+    """Accept a uint16 array of bf16 bit patterns (2-D, row-major, may have ld > cols)."""
+    x = np.asarray(x)
+    if x.dtype != np.uint16:
+        raise TypeError("oracle takes bf16 as uint16 bit patterns")
+    return x
+
+
+def view_shape(rows, cols, layout):
+    return (rows, cols) if layout == ROWWISE else (cols, rows)
+
+
+def philox(ctr, key):
+    c = np.ascontiguousarray(ctr, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    out = np.zeros(4, dtype=np.uint32)
+    lib().oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def uniform_element(seed, e):
+    return lib().oracle_uniform_element(seed, e)
+
+
+def uniform_block(seed, b):
+    return lib().oracle_uniform_block(seed, b)
+
+
+def rht_signs(seed, g):
+    return np.array([lib().oracle_rht_sign(seed, j) for j in range(g)], dtype=np.float32)
+
+
+def rht_scale(g):
+    return lib().oracle_rht_scale(g)
+
+
+def e2m1_rtn(y):
+    return lib().oracle_e2m1_rtn(float(y))
+
+
+def e2m1_sr(y, u):
+    return lib().oracle_e2m1_sr(float(y), float(u))
+
+
+def e2m1_decode(code):
+    return lib().oracle_e2m1_decode(int(code))
+
+
+def e4m3_decode(code):
+    return lib().oracle_e4m3_decode(int(code))
+
+
+def e4m3_rne_sat(v):
+    return lib().oracle_e4m3_rne_sat(float(v))
+
+
+def e4m3_ru_sat(v):
+    return lib().oracle_e4m3_ru_sat(float(v))
+
+
+def e4m3_sr(t, u):
+    return lib().oracle_e4m3_sr(float(t), float(u))
+
+
+def if4_constants():
+    k = np.zeros(2, dtype=np.float32)
+    lib().oracle_if4_constants(_ptr(k[0:1]), _ptr(k[1:2]))
+    return float(k[0]), float(k[1])
+
+
+def global_scale(amax, mode):
+    return lib().oracle_global_scale(float(amax), mode)
+
+
+def rht_rows(v, g, seed, inverse=False):
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    rows, cols = v.shape
+    out = np.empty_like(v)
+    _check(lib().oracle_rht_rows(_ptr(v), rows, cols, g, seed, int(inverse), _ptr(out)))
+    return out
+
+
+def rht_view(x_bits, layout, g, seed, cols=None):
+    x = _as_bf16_bits(x_bits)
+    rows, ld = x.shape
+    cols = ld if cols is None else cols
+    vr, vc = view_shape(rows, cols, layout)
+    out = np.empty((vr, vc), dtype=np.float32)
+    _check(lib().oracle_rht_view(_ptr(np.ascontiguousarray(x)), rows, cols, ld, layout, g, seed,
+                                 _ptr(out)))
+    return out
+
+
+def amax(x_bits, layout, g, seed, cols=None):
+    x = np.ascontiguousarray(_as_bf16_bits(x_bits))
+    rows, ld = x.shape
+    cols = ld if cols is None else cols
+    a = np.zeros(1, dtype=np.float32)
+    _check(lib().oracle_amax(_ptr(x), rows, cols, ld, layout, g, seed, _ptr(a)))
+    return float(a[0])
+
+
+def quantize(x_bits, layout, mode, g, seed, amax_in=None, cols=None, row_range=None):
+    """Returns (codes uint8 [vr, vc/2], scales uint8 [vr, vc/16], global_scale float).
+
+    x_bits: uint16 [rows, ld] bf16 patterns; cols (<= ld) is the logical width.
+    row_range: optional (begin, end) of view rows to compute; other rows stay 0.
+    """
+    x = np.ascontiguousarray(_as_bf16_bits(x_bits))
+    rows, ld = x.shape
+    cols = ld if cols is None else cols
+    vr, vc = view_shape(rows, cols, layout)
+    codes = np.zeros((vr, vc // 2), dtype=np.uint8)
+    scales = np.zeros((vr, max(vc // 16, 0)), dtype=np.uint8)
+    gs = np.zeros(1, dtype=np.float32)
+    a = None if amax_in is None else np.array([amax_in], dtype=np.float32)
+    b, e = (0, vr) if row_range is None else row_range
+    _check(lib().oracle_quantize_rows(_ptr(x), rows, cols, ld, layout, mode, g, seed,
+                                      None if a is None else _ptr(a), b, e, _ptr(codes),
+                                      _ptr(scales), _ptr(gs)))
+    return codes, scales, float(gs[0])
+
+
+def dequantize(codes, scales, gscale, mode, g, seed, inverse_rht=False):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    vr, half = codes.shape
+    vc = half * 2
+    out = np.empty((vr, vc), dtype=np.float32)
+    _check(lib().oracle_dequantize(_ptr(codes), _ptr(scales), float(gscale), vr, vc, mode, g,
+                                   seed, int(inverse_rht), _ptr(out)))
+    return out
+
+
+def unpack_codes(codes):
+    """Split packed bytes into one 4-bit code per element (low nibble first)."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    out = np.empty(codes.shape[:-1] + (codes.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = codes & 15
+    out[..., 1::2] = codes >> 4
+    return out

@@ -1,0 +1,28 @@
+"""Build the CPU oracle (test infrastructure) into oracle/liboracle.so.
+
+The oracle is plain C99 compiled with contraction and fast-math off, so every
+binary32 operation in it is one IEEE round-to-nearest-even step.
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "nvfp4_oracle.c")
+OUT = os.path.join(HERE, "liboracle.so")
+
+CFLAGS = ["-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+          "-fno-unsafe-math-optimizations", "-Wall", "-Wextra"]
+
+
+def build(force: bool = False) -> str:
+    if not force and os.path.exists(OUT) and os.path.getmtime(OUT) >= os.path.getmtime(SRC):
+        return OUT
+    cmd = ["gcc", *CFLAGS, SRC, "-o", OUT + ".tmp", "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(OUT + ".tmp", OUT)
+    return OUT
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv))

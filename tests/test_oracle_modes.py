@@ -1,0 +1,342 @@
+"""Pins the oracle's quantization modes to what the pages and the mathematics fix.
+
+* SR is unbiased when nothing clips, with error E[(y-l)(u-y)] per value
+  ("Comparing INT4 and NVFP4 Palettes on Real Gradient Tensors", section "The
+  two corners, and what the palette does to them"): Monte-Carlo mean within 4
+  sigma, and the empirical error equals the closed form.
+* MS-EDEN is unbiased in expectation and has lower error than SR (Quartet II
+  abstract: "more than 2x lower quantization error than SR"; article list
+  "Kerninnovationen"): Monte-Carlo mean within 4 sigma after the inverse
+  rotation, and the MSE ordering RTN < MS-EDEN < SR on Gaussian data.
+* IF4 keeps the lower-error option of FP4 and scaled INT4 and flags INT4 in
+  the scale's sign bit (IF4 paper page, abstract, Figure 1 and Figure 3).
+* 4/6 keeps the lower-error of the two block scales (Quartet II article,
+  "Quantisierung im Vorwaertsdurchlauf"; IF4 page Table 1, scale max 256).
+* Structural properties: transposed view = row-wise quantization of X^T,
+  leading dimension, amax_in, zero tensor and zero blocks, nibble order.
+"""
+import numpy as np
+import pytest
+import torch
+
+from nvfp4_microscaling_quantization_b200 import workloads as W
+
+ROW, TR = 0, 1
+RTN, SR, EDEN, IF4, FO6 = 0, 1, 2, 3, 4
+GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def bits_of(t):
+    return W.bf16_bits(t)
+
+
+def bf16(a):
+    return torch.from_numpy(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def f32(a):
+    return np.float32(a)
+
+
+def deq(orc, codes, scales, gs, mode, g, seed, inverse=False):
+    return orc.dequantize(codes, scales, gs, mode, g, seed, inverse_rht=inverse).astype(np.float64)
+
+
+# ----------------------------------------------------------------------------- SR
+def test_sr_monte_carlo_unbiased_and_closed_form_error(orc):
+    """4096 identical rows: same scales, independent uniforms per row (element index)."""
+    rng = np.random.default_rng(0)
+    row = bf16(rng.standard_normal(256))
+    T = 4096
+    x = row[None, :].repeat(T, 1)
+    codes, scales, gs = orc.quantize(bits_of(x), ROW, SR, 0, 42)
+    assert np.all(scales == scales[0:1])  # every row gets the same block scales
+    q = deq(orc, codes, scales, gs, SR, 0, 42)
+    xv = row.float().numpy().astype(np.float64)
+    # closed form per element: d^2 (y-l)(u-y) with y the scaled value
+    d = np.array([np.float32(orc.e4m3_decode(s)) * np.float32(gs) for s in scales[0]], dtype=np.float32)
+    dd = np.repeat(d, 16)
+    r = (np.float32(1.0) / dd).astype(np.float32)
+    y = np.abs((xv.astype(np.float32) * r).astype(np.float32)).astype(np.float64)
+    y = np.minimum(y, 6.0)
+    lo = GRID[np.searchsorted(GRID, y, side="right") - 1]
+    hi = GRID[np.minimum(np.searchsorted(GRID, y, side="right"), 7)]
+    var = dd.astype(np.float64) ** 2 * (y - lo) * (hi - y)
+    mean = q.mean(axis=0)
+    sd = np.sqrt(var / T)
+    z = np.abs(mean - xv) / np.maximum(sd, 1e-30)
+    z[var == 0] = 0.0
+    assert np.all(np.abs(mean - xv)[var == 0] < 1e-6 * np.abs(xv).max())  # exact values stay exact
+    # unbiased: every element within 4 sigma (+ the 2^-16 resolution of the uniforms)
+    slack = dd.astype(np.float64) * (hi - lo) * 2.0 ** -16
+    assert np.all(np.abs(mean - xv) <= 4 * sd + slack)
+    # empirical MSE equals the closed form within its sampling error
+    emp = ((q - xv[None, :]) ** 2).mean(axis=0).sum()
+    assert abs(emp - var.sum()) <= 0.05 * var.sum()
+
+
+def test_sr_never_exceeds_block_range(orc):
+    """Round-up scales: |Q(x)| <= block absmax rounded up, never clipped."""
+    rng = np.random.default_rng(1)
+    x = bf16(rng.standard_t(3, size=(64, 256)))
+    codes, scales, gs = orc.quantize(bits_of(x), ROW, SR, 0, 3)
+    q = deq(orc, codes, scales, gs, SR, 0, 3)
+    xv = x.float().numpy().astype(np.float64)
+    d = np.vectorize(lambda s: np.float32(orc.e4m3_decode(int(s))) * np.float32(gs))(scales).astype(np.float64)
+    assert np.all(np.abs(q) <= 6 * np.repeat(d, 16, axis=1) * (1 + 1e-6))
+    # the block's largest element is never rounded away from its interval
+    assert np.all(np.abs(q - xv) <= np.repeat(d, 16, axis=1) * 2.0 + 1e-12)
+
+
+# ------------------------------------------------------------------------- MS-EDEN
+def _eden_trials(orc, x_row, T, g=128):
+    bits = bits_of(x_row[None, :])
+    outs = []
+    for s in range(T):
+        seed = 1000 + s
+        codes, scales, gs = orc.quantize(bits, ROW, EDEN, g, seed)
+        outs.append(deq(orc, codes, scales, gs, EDEN, g, seed, inverse=True)[0])
+    return np.array(outs)
+
+
+def test_ms_eden_monte_carlo_unbiased(orc):
+    rng = np.random.default_rng(2)
+    x = bf16(rng.standard_normal(256))
+    xv = x.float().numpy().astype(np.float64)
+    T = 3000
+    q = _eden_trials(orc, x, T)
+    mean = q.mean(axis=0)
+    sd = q.std(axis=0, ddof=1) / np.sqrt(T)
+    z = (mean - xv) / sd
+    # 4-sigma per element, and the whole vector's chi-square within 4 sigma of its mean
+    assert np.max(np.abs(z)) < 4.0 + 0.5  # 256 elements: max |N(0,1)| rarely exceeds 4
+    n = len(z)
+    assert abs(np.sum(z ** 2) - n) < 4 * np.sqrt(2 * n)
+
+
+def _mse(orc, x, mode, g, seeds):
+    bits = bits_of(x)
+    xv = x.float().numpy().astype(np.float64)
+    tot = 0.0
+    for s in seeds:
+        codes, scales, gs = orc.quantize(bits, ROW, mode, g, s)
+        q = deq(orc, codes, scales, gs, mode, g, s, inverse=g > 0)
+        tot += np.mean((q - xv) ** 2)
+    return tot / len(seeds)
+
+
+def test_mse_ordering_rtn_eden_sr(orc):
+    """RTN < MS-EDEN < SR on N(0,1) blocks, all with the 128-point RHT; SR/EDEN reported."""
+    rng = np.random.default_rng(4)
+    x = bf16(rng.standard_normal((64, 512)))
+    seeds = list(range(8))
+    m_rtn = _mse(orc, x, RTN, 128, seeds)
+    m_eden = _mse(orc, x, EDEN, 128, seeds)
+    m_sr = _mse(orc, x, SR, 128, seeds)
+    print(f"\nMSE  RTN {m_rtn:.5f}  MS-EDEN {m_eden:.5f}  SR {m_sr:.5f}  SR/EDEN {m_sr / m_eden:.2f}")
+    assert m_rtn < m_eden < m_sr
+    assert m_sr / m_eden > 1.5  # the pages claim "more than 2x"; the ratio is reported above
+
+
+def test_ms_eden_codes_are_rtn_codes(orc):
+    """Randomness lives only on the scale: codes equal RTN's (same view, same block scale choice)."""
+    rng = np.random.default_rng(5)
+    x = bf16(rng.standard_normal((32, 256)))
+    # MS-EDEN maps the amax to 6 x 256 and RTN to 6 x 448: amax 4 and 7 give the same s_g
+    c_e, s_e, g_e = orc.quantize(bits_of(x), ROW, EDEN, 128, 9, amax_in=4.0)
+    c_r, s_r, g_r = orc.quantize(bits_of(x), ROW, RTN, 128, 9, amax_in=7.0)
+    assert g_e == g_r
+    assert np.array_equal(c_e, c_r)
+    # scales differ from RTN's by at most one E4M3 step after the correction (c near 1)
+    se = np.vectorize(lambda s: orc.e4m3_decode(int(s)))(s_e)
+    sr = np.vectorize(lambda s: orc.e4m3_decode(int(s)))(s_r)
+    assert np.all(np.abs(se / sr - 1) < 0.3)
+    assert np.mean(s_e != s_r) > 0.05
+
+
+# --------------------------------------------------------------------------- IF4
+def _block_views(orc, x_bits, layout, mode, g, seed):
+    codes, scales, gs = orc.quantize(x_bits, layout, mode, g, seed)
+    z = orc.rht_view(x_bits, layout, g, seed) if g else \
+        torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    if layout == TR and not g:
+        z = np.ascontiguousarray(z.T)
+    return codes, scales, gs, z.astype(np.float32)
+
+
+@pytest.mark.parametrize("g", [0, 128])
+def test_if4_picks_lower_error_option(orc, g):
+    wl = W.activation(rows=32, cols=512)
+    a = wl.tensors()["a"]
+    bits = bits_of(a)
+    codes, scales, gs, z = _block_views(orc, bits, ROW, IF4, g, 3)
+    k1, k2 = orc.if4_constants()
+    cu = orc.unpack_codes(codes)
+    n_int = 0
+    for r in range(z.shape[0]):
+        for b in range(z.shape[1] // 16):
+            S = int(scales[r, b])
+            d = f32(f32(orc.e4m3_decode(S & 0x7F)) * f32(gs))
+            if d == 0:
+                continue
+            y = (z[r, 16 * b:16 * b + 16] * f32(f32(1.0) / d)).astype(np.float32)
+            fp = np.array([orc.e2m1_decode(orc.e2m1_rtn(float(v))) for v in y], dtype=np.float64)
+            k = np.clip(np.round((y * f32(k1)).astype(np.float32)), -7, 7)
+            it = (k * f32(k2)).astype(np.float32).astype(np.float64)
+            e_fp = np.sum((y - fp) ** 2)
+            e_int = np.sum((y - it) ** 2)
+            flag = bool(S & 0x80)
+            n_int += flag
+            chosen, other = (e_int, e_fp) if flag else (e_fp, e_int)
+            assert chosen <= other * (1 + 1e-5) + 1e-12, (r, b)
+            # codes are those of the chosen option
+            c = cu[r, 16 * b:16 * b + 16]
+            if flag:
+                kk = np.where(c & 8, -(c & 7).astype(int), (c & 7).astype(int))
+                assert np.array_equal(kk, k.astype(int))
+            else:
+                assert np.allclose([orc.e2m1_decode(int(v)) for v in c], fp)
+    print(f"\nIF4 g={g}: INT4 picked for {n_int} of {z.size // 16} blocks")
+
+
+def test_if4_fp4_blocks_equal_rtn(orc):
+    """An IF4 block with the flag clear is byte-identical to RTN NVFP4 (flag 1 = INT4 reading)."""
+    wl = W.activation(rows=64, cols=256)
+    bits = bits_of(wl.tensors()["a"])
+    c_i, s_i, g_i = orc.quantize(bits, ROW, IF4, 0, 3)
+    c_r, s_r, g_r = orc.quantize(bits, ROW, RTN, 0, 3)
+    assert g_i == g_r
+    fp = (s_i & 0x80) == 0
+    assert np.array_equal(s_i[fp], s_r[fp])
+    assert np.array_equal((s_i & 0x7F), s_r)
+    cb_i = orc.unpack_codes(c_i).reshape(c_i.shape[0], -1, 16)
+    cb_r = orc.unpack_codes(c_r).reshape(c_r.shape[0], -1, 16)
+    assert np.array_equal(cb_i[fp], cb_r[fp])
+    assert 0 < np.mean(~fp) < 1
+
+
+def test_if4_rht_raises_int4_share(orc):
+    """Reported: the share of INT4 blocks with and without the rotation (IF4 page, Figure 5)."""
+    wl = W.activation(rows=64, cols=1024)
+    bits = bits_of(wl.tensors()["a"])
+    _, s0, _ = orc.quantize(bits, ROW, IF4, 0, 3)
+    _, s1, _ = orc.quantize(bits, ROW, IF4, 128, 3)
+    f0, f1 = np.mean(s0 >= 0x80), np.mean(s1 >= 0x80)
+    print(f"\nIF4 INT4 share: no RHT {f0:.3f}, RHT {f1:.3f}")
+    assert f1 > f0
+
+
+# --------------------------------------------------------------------------- 4/6
+def test_four_over_six_picks_lower_error(orc):
+    wl = W.weight(rows=32, cols=512)
+    bits = bits_of(wl.tensors()["w"])
+    codes, scales, gs, z = _block_views(orc, bits, ROW, FO6, 0, 1)
+    A = np.abs(z).max()
+    assert gs == orc.global_scale(A, FO6)
+    cand = {}
+    for r in range(z.shape[0]):
+        for b in range(z.shape[1] // 16):
+            zb = z[r, 16 * b:16 * b + 16]
+            ab = f32(np.abs(zb).max())
+            errs, Ss = [], []
+            for m in (6.0, 4.0):
+                S = orc.e4m3_rne_sat(f32(ab / f32(f32(m) * f32(gs))))
+                d = f32(f32(orc.e4m3_decode(S)) * f32(gs))
+                y = (zb * f32(f32(1.0) / d)).astype(np.float32)
+                v = np.array([orc.e2m1_decode(orc.e2m1_rtn(float(t))) for t in y], dtype=np.float32)
+                errs.append(np.sum((zb.astype(np.float64) - (v * d).astype(np.float32)) ** 2))
+                Ss.append(S)
+            S = int(scales[r, b])
+            assert S in Ss
+            chosen = errs[Ss.index(S)] if Ss[0] != Ss[1] else errs[0]
+            assert chosen <= min(errs) * (1 + 1e-5) + 1e-30
+            cand[(r, b)] = Ss.index(S)
+    frac4 = np.mean([v == 1 for v in cand.values()])
+    print(f"\n4/6: scale-to-4 chosen for {frac4:.3f} of blocks")
+    assert 0 < frac4 < 1
+
+
+def test_four_over_six_not_worse_than_rtn(orc):
+    wl = W.weight(rows=64, cols=1024)
+    x = wl.tensors()["w"]
+    m_rtn = _mse(orc, x, RTN, 0, [0])
+    m_46 = _mse(orc, x, FO6, 0, [0])
+    print(f"\nweight-like MSE: RTN {m_rtn:.3e}  4/6 {m_46:.3e}")
+    assert m_46 <= m_rtn
+
+
+# ------------------------------------------------------------------- structural
+@pytest.mark.parametrize("mode,g", [(RTN, 0), (SR, 0), (EDEN, 128), (IF4, 0), (FO6, 0), (SR, 32)])
+def test_transposed_is_rowwise_of_transpose(orc, mode, g):
+    rng = np.random.default_rng(6)
+    x = bf16(rng.standard_normal((256, 64)))
+    a = orc.quantize(bits_of(x), TR, mode, g, 17)
+    b = orc.quantize(bits_of(x.t().contiguous()), ROW, mode, g, 17)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1]) and a[2] == b[2]
+
+
+def test_leading_dimension_and_amax_in(orc):
+    rng = np.random.default_rng(7)
+    full = bf16(rng.standard_normal((64, 160)))
+    bits = bits_of(full)
+    cols = 128
+    dense = bits_of(full[:, :cols].contiguous())
+    for layout in (ROW, TR):
+        a = orc.quantize(bits, layout, EDEN, 32, 5, cols=cols)
+        b = orc.quantize(dense, layout, EDEN, 32, 5)
+        assert all(np.array_equal(u, v) for u, v in zip(a[:2], b[:2])) and a[2] == b[2]
+        A = orc.amax(dense, layout, 32, 5)
+        c = orc.quantize(dense, layout, EDEN, 32, 5, amax_in=A)
+        assert all(np.array_equal(u, v) for u, v in zip(b[:2], c[:2])) and b[2] == c[2]
+
+
+@pytest.mark.parametrize("mode", [RTN, SR, EDEN, IF4, FO6])
+def test_zero_tensor_and_zero_block(orc, mode):
+    g = 16 if mode == EDEN else 0
+    z = np.zeros((4, 64), dtype=np.uint16)
+    codes, scales, gs = orc.quantize(z, ROW, mode, g, 1)
+    assert gs == 1.0 and not codes.any() and not scales.any()
+    x = np.zeros((4, 64), dtype=np.float32)
+    x[1, 20] = 3.0
+    codes, scales, gs = orc.quantize(bits_of(bf16(x)), ROW, mode, 0 if mode != EDEN else 16, 1)
+    assert scales[1, 1] != 0 and scales[0].sum() == 0 and scales[1, [0, 2, 3]].sum() == 0
+
+
+def test_nibble_order_and_scale_layout(orc):
+    x = np.zeros((2, 32), dtype=np.float32)
+    x[0, 0] = 6.0   # element 0 -> low nibble of byte 0
+    x[0, 3] = -3.0  # element 3 -> high nibble of byte 1
+    x[1, 31] = 1.0  # last element -> high nibble of byte 15, scale index 1
+    codes, scales, gs = orc.quantize(bits_of(bf16(x)), ROW, RTN, 0, 0)
+    assert gs == np.float32(6.0) / np.float32(2688.0)
+    assert codes[0, 0] & 15 == 7 and codes[0, 0] >> 4 == 0
+    assert codes[0, 1] >> 4 == 8 | 5 and codes[0, 1] & 15 == 0
+    assert codes[1, 15] >> 4 == 7 and scales[1, 0] == 0 and scales[1, 1] != 0
+    assert scales.shape == (2, 2) and codes.shape == (2, 16)
+
+
+def test_rtn_error_bound(orc):
+    rng = np.random.default_rng(9)
+    x = bf16(rng.standard_normal((32, 256)) * np.exp(rng.uniform(-4, 4, size=(32, 1))))
+    for g in (0, 64):
+        codes, scales, gs = orc.quantize(bits_of(x), ROW, RTN, g, 2)
+        q = deq(orc, codes, scales, gs, RTN, g, 2)
+        z = orc.rht_view(bits_of(x), ROW, g, 2) if g else x.float().numpy()
+        d = np.vectorize(lambda s: np.float32(orc.e4m3_decode(int(s))) * np.float32(gs))(scales)
+        dd = np.repeat(d, 16, axis=1).astype(np.float64)
+        y = np.abs(z) / dd
+        bound = np.where(y > 6, y - 6, 1.0) * dd * (1 + 1e-5)
+        assert np.all(np.abs(q - z) <= bound)
+
+
+def test_gaussian_top_interval_share_reported(orc):
+    """Soft reproduction: about 19.3% of Gaussian values land in [4, 6] under absmax-to-6 SR scaling
+    (palettes post, interval decomposition); reported, loosely bounded."""
+    rng = np.random.default_rng(10)
+    x = bf16(rng.standard_normal((256, 1024)))
+    codes, scales, gs = orc.quantize(bits_of(x), ROW, SR, 0, 0)
+    d = np.vectorize(lambda s: np.float32(orc.e4m3_decode(int(s))) * np.float32(gs))(scales)
+    y = np.abs(x.float().numpy()) / np.repeat(d, 16, axis=1)
+    share = np.mean(y >= 4.0)
+    print(f"\nshare of |y| in [4,6]: {share:.4f}")
+    assert 0.15 < share < 0.21
