@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Throughput of block-scaled NVFP4 quantization on B200.
+
+One step quantizes the tensors of one Llama-style MLP up-projection training
+step (X 16384x4096, W 14336x4096, dY 16384x14336, bf16) the way a fully-NVFP4
+linear layer needs them: RTN on X and W along d_model (forward), MS-EDEN with
+a 128-point random Hadamard rotation on dY row-wise and transposed, and on X
+and W transposed (backward) -- six calls, each the tensor-amax pre-pass then
+the quantization kernel, through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  value = algorithmic bytes (2 B read + 0.5 B
+codes + 0.0625 B scales per element of every call) / device time, all ranks
+summed (weak scaling: each rank quantizes its own step's tensors, no data-path
+collective).  L2 is flushed (a 256 MiB write) before every timed step, outside
+the timed region.  --impl reference times the CPU oracle on a bounded sample
+of the same workload.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
+
+METRIC = "NVFP4 quantize GB/s and % of B200 HBM peak per mode (Gelem/s), 1 GPU"
+UNIT = "GB/s"
+BYTES_PER_ELEMENT = 2.0 + 0.5 + 0.0625   # bf16 in, E2M1 codes out, E4M3 scales out
+PREPASS_BYTES_PER_ELEMENT = 2.0          # the amax pre-pass reads the tensor once more
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+# DRAM bytes per launch measured by ncu for the dominant kernel, keyed by the
+# hash of the kernel sources they were taken with (see profiles/).  A changed
+# kernel reports traffic = null until it is captured again.
+NCU_TRAFFIC = {}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--cpu-sample-fraction", type=float, default=1.0 / 8,
+                   help="fraction of each call's view rows the CPU baseline quantizes")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args(argv)
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world, device=None):
+    if world > 1:
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Largest value over all ranks (every rank takes part)."""
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(bytes_per_rank_step: float, steps: int, world: int, max_seconds: float) -> float:
+    """GB/s of the whole job: every rank's bytes over the slowest rank's time."""
+    return bytes_per_rank_step * steps * world / max_seconds / 1e9
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "200"], stdout=self.out,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.path:
+            self.out.close()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "nvfp4_microscaling_quantization_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------------- our CUDA path
+class Call:
+    """One quantization call bound to device buffers, issued through the raw C ABI."""
+
+    def __init__(self, N, call, x, seed, stream_handle):
+        import ctypes
+        self.N, self.call, self.x, self.seed = N, call, x, seed
+        rows, cols = x.shape
+        self.rows, self.cols, self.ld = rows, cols, x.stride(0)
+        self.elements = rows * cols
+        self.codes, self.scales, self.gscale = N.alloc_outputs(rows, cols, call.layout, x.device)
+        self.amax = torch.empty(1, dtype=torch.float32, device=x.device)
+        P = ctypes.c_void_p
+        self.p = dict(x=P(x.data_ptr()), codes=P(self.codes.data_ptr()), scales=P(self.scales.data_ptr()),
+                      gscale=P(self.gscale.data_ptr()), amax=P(self.amax.data_ptr()))
+        self.stream = stream_handle
+
+    def amax_pass(self):
+        st = self.N.nvfp4_amax(self.p["x"], self.rows, self.cols, self.ld, self.call.layout,
+                               self.call.rht_group, self.seed, self.p["amax"], self.stream)
+        if st:
+            raise self.N.Nvfp4Error(st, "nvfp4_amax")
+
+    def quantize(self):
+        st = self.N.nvfp4_quantize(self.p["x"], self.rows, self.cols, self.ld, self.call.layout, self.call.mode,
+                                   self.call.rht_group, self.seed, self.p["amax"], self.p["codes"],
+                                   self.p["scales"], self.p["gscale"], None, 0, self.stream)
+        if st:
+            raise self.N.Nvfp4Error(st, "nvfp4_quantize")
+
+    def output_bytes(self):
+        return self.codes.numel() + self.scales.numel() + 4
+
+
+def run_ours(args, world, rank, local):
+    import ctypes
+    from nvfp4_microscaling_quantization_b200 import binding as N
+    from nvfp4_microscaling_quantization_b200 import workloads as W
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    N.lib()
+    wl = W.mlp_up(seed=4 + 1000 * rank)
+    tensors = wl.tensors(device)
+    stream = torch.cuda.current_stream(device)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    calls = [Call(N, c, tensors[c.tensor], wl.seed, sh) for c in wl.calls]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    bytes_per_step = sum(BYTES_PER_ELEMENT * c.elements for c in calls)
+    elems_per_step = sum(c.elements for c in calls)
+
+    def step(evs=None):
+        for i, c in enumerate(calls):
+            if evs is not None:
+                evs[i][0].record(stream)
+            c.amax_pass()
+            if evs is not None:
+                evs[i][1].record(stream)
+            c.quantize()
+            if evs is not None:
+                evs[i][2].record(stream)
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+
+    K = args.steps
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    starts, ends = [ev() for _ in range(K)], [ev() for _ in range(K)]
+    call_evs = [[[ev(), ev(), ev()] for _ in calls] for _ in range(K)]
+    with ClockSampler(local) as clocks:
+        barrier(world, local)
+        torch.cuda.synchronize(device)
+        for k in range(K):
+            flush.zero_()                    # L2 flush, outside the timed region
+            starts[k].record(stream)
+            step(call_evs[k])
+            ends[k].record(stream)
+        torch.cuda.synchronize(device)
+        barrier(world, local)
+    clock = clocks.summary()
+
+    step_ms = [starts[k].elapsed_time(ends[k]) for k in range(K)]
+    total_s = max_over_ranks(sum(step_ms) / 1e3, world, device)
+    amax_ms = [statistics.mean(call_evs[k][i][0].elapsed_time(call_evs[k][i][1]) for k in range(K))
+               for i in range(len(calls))]
+    quant_ms = [statistics.mean(call_evs[k][i][1].elapsed_time(call_evs[k][i][2]) for k in range(K))
+                for i in range(len(calls))]
+    quant_total_s = max_over_ranks(sum(quant_ms) * K / 1e3, world, device)
+    value = weak_scaling_value(bytes_per_step, K, world, total_s)
+    value_supplied = weak_scaling_value(bytes_per_step, K, world, quant_total_s)
+    peak, peak_kind = hbm_peak()
+
+    # dominant kernel: the quantize kernel with the largest share of the step
+    dom = max(range(len(calls)), key=lambda i: quant_ms[i])
+    dom_bytes = BYTES_PER_ELEMENT * calls[dom].elements
+    achieved = dom_bytes / (quant_ms[dom] / 1e3) / 1e9
+    src_hash = kernel_source_hash()
+    traffic = NCU_TRAFFIC.get((src_hash, calls[dom].call.name))
+
+    per_call = []
+    for i, c in enumerate(calls):
+        per_call.append({
+            "call": c.call.name, "elements": c.elements,
+            "quantize_us": round(quant_ms[i] * 1e3, 2), "amax_us": round(amax_ms[i] * 1e3, 2),
+            "quantize_gbs": round(BYTES_PER_ELEMENT * c.elements / (quant_ms[i] / 1e3) / 1e9, 1),
+            "amax_gbs": round(PREPASS_BYTES_PER_ELEMENT * c.elements / (amax_ms[i] / 1e3) / 1e9, 1),
+            "quantize_gelem_s": round(c.elements / (quant_ms[i] / 1e3) / 1e9, 1),
+        })
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, calls, tensors, stream, device, world, bytes_per_step)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = {k: v.cpu() for k, v in tensors.items()}
+        cpu = cpu_baseline(wl, host, args.cpu_sample_fraction)
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(total_s * 1e3 / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {
+            "workload": "mlp_up: one Llama-style MLP up-projection training step's tensors, "
+                        "X 16384x4096 N(0,1), W 14336x4096 N(0,0.02^2), dY 16384x14336 Student-t3 std 1e-4",
+            "calls": [c.call.name for c in calls],
+            "path": "per call: tensor-amax pre-pass kernel + quantize kernel (C ABI), one stream",
+            "input_dtype": "bf16", "l2": "flushed before every timed step (256 MiB write, untimed)",
+            "parallelism": f"replicas x{world} (independent tensors per rank)",
+        },
+        "gelem_per_s": round(elems_per_step * K * world / total_s / 1e9, 1),
+        "frac_of_hbm_peak": round(value / world / peak, 4),
+        "value_amax_supplied": round(value_supplied, 1),
+        "frac_of_hbm_peak_amax_supplied": round(value_supplied / world / peak, 4),
+        "roofline": {"bound": "hbm", "kernel": f"quantize {calls[dom].call.name}",
+                     "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic_bytes": int(dom_bytes), "avg_launch_us": round(quant_ms[dom] * 1e3, 2)},
+        "per_call": per_call,
+        "gpu_launches": 2 * len(calls) * K,
+        "clocks": clock,
+        "kernel_source": src_hash,
+    }
+    if e2e is not None:
+        result["e2e"] = e2e
+    if cpu is not None:
+        result["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, calls, tensors, stream, device, world, bytes_per_step):
+    """Same step through the public API with host buffers: pinned H2D of the step's
+    inputs, the six calls, D2H of every output, all inside the timed region."""
+    host_in = {k: v.cpu().pin_memory() for k, v in tensors.items()}
+    host_out = [(torch.empty(c.codes.shape, dtype=torch.uint8).pin_memory(),
+                 torch.empty(c.scales.shape, dtype=torch.uint8).pin_memory(),
+                 torch.empty(1, dtype=torch.float32).pin_memory()) for c in calls]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(c.output_bytes() for c in calls)
+
+    def e2e_step():
+        for k, t in tensors.items():
+            t.copy_(host_in[k], non_blocking=True)
+        for c in calls:
+            c.amax_pass()
+            c.quantize()
+        for c, (hc, hs, hg) in zip(calls, host_out):
+            hc.copy_(c.codes, non_blocking=True)
+            hs.copy_(c.scales, non_blocking=True)
+            hg.copy_(c.gscale, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    K = max(args.e2e_steps, 1)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, device.index)
+    torch.cuda.synchronize(device)
+    start.record(stream)
+    for _ in range(K):
+        e2e_step()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world, device.index)
+    secs = max_over_ranks(start.elapsed_time(end) / 1e3, world, device)
+    return {"value": round(weak_scaling_value(bytes_per_step, K, world, secs), 2), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
+            "ms_per_step": round(secs * 1e3 / K, 3)}
+
+
+# ------------------------------------------------------------------------ CPU oracle
+def _sample_calls(wl, host, fraction):
+    """For every call, the sub-tensor holding the first `fraction` of its view rows."""
+    from nvfp4_microscaling_quantization_b200 import workloads as W
+    out = []
+    for c in wl.calls:
+        x = host[c.tensor]
+        rows, cols = x.shape
+        if c.layout == W.ROWWISE:
+            n = max(1, int(rows * fraction))
+            sub = x[:n]
+        else:
+            n = max(8, int(cols * fraction) // 8 * 8)
+            sub = x[:, :n]
+        out.append((c, W.bf16_bits(sub.contiguous())))
+    return out
+
+
+def time_oracle_sample(wl, samples):
+    import oracle
+    elements = 0
+    t0 = time.perf_counter()
+    for c, xb in samples:
+        a = oracle.amax(xb, c.layout, c.rht_group, wl.seed)
+        oracle.quantize(xb, c.layout, c.mode, c.rht_group, wl.seed, amax_in=a)
+        elements += xb.size
+    return elements, time.perf_counter() - t0
+
+
+def cpu_baseline(wl, host, fraction):
+    samples = _sample_calls(wl, host, fraction)
+    elements, secs = time_oracle_sample(wl, samples)
+    return {"value": round(BYTES_PER_ELEMENT * elements / secs / 1e9, 4), "unit": UNIT, "cores": 1,
+            "kind": "oracle",
+            "sample": f"first {fraction:.4g} of the view rows of each of the 6 calls "
+                      f"({elements} elements, amax pre-pass + quantize, single-threaded C), {secs:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle as the reference arm, on rank 0 only."""
+    if rank != 0:
+        return
+    from nvfp4_microscaling_quantization_b200 import workloads as W
+    wl = W.mlp_up(seed=4)
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    full = wl.tensors(device)
+    host = {k: v.cpu() for k, v in full.items()}
+    del full
+    fraction = 1.0 / 128
+    samples = _sample_calls(wl, host, fraction)
+    for _ in range(max(args.warmup, 0)):
+        time_oracle_sample(wl, samples)
+    total_e, total_s = 0, 0.0
+    for _ in range(args.steps):
+        e, s = time_oracle_sample(wl, samples)
+        total_e += e
+        total_s += s
+    value = BYTES_PER_ELEMENT * total_e / total_s / 1e9
+    sample = (f"each step: first {fraction:.4g} of the view rows of each of the 6 mlp_up calls "
+              f"({total_e // max(args.steps, 1)} elements, amax pre-pass + quantize)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_s * 1e3 / max(args.steps, 1), 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "mlp_up (bounded sample per step)", "input_dtype": "bf16"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --impl ours needs a CUDA GPU")
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

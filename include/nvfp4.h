@@ -1,0 +1,163 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4.so: block-scaled NVFP4 quantization of bf16
+ * training tensors on NVIDIA B200 (sm_100a).
+ *
+ * The method (sources named by page title and section):
+ *  - One FP8 E4M3 scale per 16 consecutive elements and one FP32 scale per
+ *    tensor; values rounded to nearest onto E2M1 (FP4) for the forward pass,
+ *    with the optional "Four Over Six" block scale choice.  Quartet II article
+ *    (mind-verse.de), section "Quantisierung im Vorwaertsdurchlauf".
+ *  - E2M1 values {0, +-0.5, +-1, +-1.5, +-2, +-3, +-4, +-6}, 16-element
+ *    blocks, a random Hadamard rotation before quantizing.  "Comparing INT4
+ *    and NVFP4 Palettes on Real Gradient Tensors", opening section.
+ *  - Unbiased stochastic rounding with an absmax scale that never clips.
+ *    Same post, section "The two corners, and what the palette does to them".
+ *  - MS-EDEN: deterministic rounding after a randomized Hadamard rotation,
+ *    with an EDEN correction factor folded into the group scale by stochastic
+ *    rounding.  Quartet II abstract (OpenAlex record) and article, section
+ *    "Quantisierung im Rueckwaertsdurchlauf" and list "Kerninnovationen".
+ *  - IF4: per 16-element block, the lower-error of FP4 and scaled INT4 under
+ *    the same E4M3 scale, flagged in the scale's sign bit.  IF4 paper page
+ *    (arXiv 2603.28765), abstract, Figure 1, Table 1, Figure 3.
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers are DEVICE pointers unless stated otherwise.  The library
+ *    allocates nothing and keeps no state between calls; every buffer is
+ *    owned by the caller and must stay valid until the stream work finishes.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) and returns without synchronising the host.  Arguments are
+ *    checked on the host before anything is launched: a failed check returns
+ *    a negative nvfp4_status and enqueues nothing.  A failed launch returns
+ *    NVFP4_ERR_CUDA.  Faults during execution surface at the caller's next
+ *    synchronisation.
+ *  - x is bf16, row-major, rows x cols, leading dimension ld (elements,
+ *    ld >= cols).  The quantized VIEW is V = X (NVFP4_ROWWISE: blocks of 16
+ *    along a row of X) or V = X^T (NVFP4_TRANSPOSED: blocks of 16 down a
+ *    column of X, output stored as X^T row-major).  The view has vrows x vcols
+ *    = rows x cols (row-wise) or cols x rows (transposed).
+ *  - codes: vrows x vcols/2 bytes; byte k of a row holds element 2k in its
+ *    low nibble and element 2k+1 in its high nibble.  An E2M1 code is sign
+ *    (bit 3) and a magnitude index (bits 0..2) into {0,.5,1,1.5,2,3,4,6}; an
+ *    INT4 code (IF4 blocks flagged INT4) is sign (bit 3) and |k| (bits 0..2),
+ *    value k * 6/7.  Zero is always code 0.
+ *  - scales: vrows x vcols/16 bytes, E4M3 (bias 7, max 448, min 2^-9); for
+ *    IF4, bit 7 set means the block holds INT4 codes.
+ *  - global_scale: one float s_g; an element decodes to
+ *    value(code) * RN(E4M3(scale & 0x7F) * s_g).
+ *  - rht_group g in {0 (no rotation), 16, 32, 64, 128}: the random Hadamard
+ *    rotation c_g H_g diag(sigma) applied to every g consecutive elements
+ *    along a view row, sigma = g random signs drawn from `seed` (one sign
+ *    vector shared by every group), c_g = RN(1/sqrt(g)).
+ *  - seed keys every random draw (element rounding, scale rounding, signs)
+ *    through Philox4x32-10 keyed by (seed, element or block index), so a
+ *    result is a pure function of (input, arguments, seed).
+ *  - Inputs must be finite; a nonzero tensor amax must be at least 2^-96.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = -1, /* null pointer, unknown enum value, bad group */
+  NVFP4_ERR_SHAPE = -2,       /* block dimension not a multiple of 16 or of g; ld < cols */
+  NVFP4_ERR_ALIGNMENT = -3,   /* x not 16-byte aligned, ld not a multiple of 8, ... */
+  NVFP4_ERR_UNSUPPORTED = -4, /* valid but unsupported combination (MS-EDEN without RHT) */
+  NVFP4_ERR_WORKSPACE = -5,   /* workspace missing or smaller than nvfp4_workspace_bytes */
+  NVFP4_ERR_CUDA = -6         /* a CUDA call or kernel launch failed */
+} nvfp4_status;
+
+typedef enum { NVFP4_ROWWISE = 0, NVFP4_TRANSPOSED = 1 } nvfp4_layout;
+
+typedef enum {
+  NVFP4_RTN = 0,     /* round to nearest, tensor amax -> 6 x 448 */
+  NVFP4_SR = 1,      /* stochastic rounding, block scale rounded up, amax -> 6 x 448 */
+  NVFP4_MS_EDEN = 2, /* RTN codes + EDEN-corrected, stochastically rounded scale; needs g > 0; amax -> 6 x 256 */
+  NVFP4_IF4 = 3,     /* per block FP4 or scaled INT4 (flag in scale bit 7), amax -> 6 x 448 */
+  NVFP4_4OVER6 = 4   /* per block scale mapping the absmax to 6 or to 4, amax -> 6 x 256 */
+} nvfp4_mode;
+
+/* Bytes of device workspace nvfp4_quantize needs when amax_in is NULL (the
+ * tensor amax is then computed in a pre-pass into the workspace).  Returns 0
+ * for invalid arguments. */
+NVFP4_API size_t nvfp4_workspace_bytes(int64_t rows, int64_t cols, int layout, int mode, int rht_group);
+
+/* Tensor amax of the (rotated) view: *amax_out = max |z| over the whole view,
+ * z the view rotated by the RHT when rht_group > 0.  This is the pre-pass of
+ * nvfp4_quantize, exposed so a caller can compute the amax once (or take it
+ * from a producer) and pass it as amax_in.  amax_out: one device float,
+ * overwritten.  Source: "FP32 scale per tensor", Quartet II article, section
+ * "Quantisierung im Vorwaertsdurchlauf". */
+NVFP4_API int nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int layout,
+               int rht_group, uint64_t seed, float* amax_out, void* stream);
+
+/* Quantize x to packed E2M1/INT4 codes, E4M3 block scales and the FP32
+ * tensor scale, in the given layout and mode (see the conventions above).
+ *  amax_in:   device float holding the tensor amax of the (rotated) view, or
+ *             NULL to compute it in a pre-pass (needs the workspace).  The
+ *             tensor scale is s_g = RN(amax / (6 M)), M = 448 (RTN, SR, IF4)
+ *             or 256 (MS-EDEN, 4/6); s_g = 1 for a zero amax.
+ *  codes, scales, global_scale: outputs (sizes above); global_scale is one
+ *             device float.
+ *  workspace: device memory of at least nvfp4_workspace_bytes(...) bytes when
+ *             amax_in is NULL, 16-byte aligned; may be NULL otherwise.
+ * Shapes: vcols must be a multiple of 16 and of rht_group; for the
+ * transposed layout cols must also be a multiple of 8.  Alignment: x 16-byte
+ * aligned, ld a multiple of 8, codes 8-byte aligned. */
+NVFP4_API int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int layout,
+                   int mode, int rht_group, uint64_t seed, const float* amax_in,
+                   uint8_t* codes, uint8_t* scales, float* global_scale, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/* Decode a quantized view (vrows x vcols) back to fp32:
+ * out[r][j] = value(code, flag) * RN(E4M3(scale & 0x7F) * s_g), and, when
+ * inverse_rht != 0 (needs rht_group > 0 and the seed used to quantize), the
+ * inverse rotation along each row.  value is the E2M1 value, or for an IF4
+ * block with bit 7 of its scale set, RN(k * RN(6/7)).  out: vrows x vcols
+ * dense fp32, 16-byte aligned.  global_scale: device float. */
+NVFP4_API int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
+                     int64_t vrows, int64_t vcols, int mode, int rht_group, uint64_t seed,
+                     int inverse_rht, float* out, void* stream);
+
+/* The random Hadamard rotation of the view, as fp32: out (vrows x vcols,
+ * dense, 16-byte aligned) = the view of `in` with every rht_group-long piece
+ * of a row rotated (inverse == 0) or un-rotated (inverse != 0).  in_dtype 0 =
+ * bf16, 1 = fp32 (then ld counts fp32 elements and must be a multiple of 4).
+ * Source: randomized Hadamard rotation, Quartet II article section
+ * "Quantisierung im Rueckwaertsdurchlauf"; 16x16 rotation in the palettes
+ * post, section "45 real tensors disagree". */
+NVFP4_API int nvfp4_rht(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld, int layout,
+              int rht_group, uint64_t seed, int inverse, float* out, void* stream);
+
+/* Element and scale codecs of the quantizer, exposed on their own.
+ * nvfp4_encode_e2m1: out[i] = E2M1 code (low nibble, one code per byte) of
+ * in[i] rounded to nearest, ties to the even code, saturating at +-6, zero
+ * always code 0 -- the rounding every RTN, MS-EDEN, IF4 and 4/6 element goes
+ * through.  nvfp4_encode_e4m3: out[i] = E4M3 code of in[i] >= 0 rounded to
+ * nearest-even (round_up == 0) or up to the next E4M3 value (round_up != 0),
+ * saturating at 448 -- the block-scale rounding.  in: n device floats (finite;
+ * non-negative for E4M3), out: n device bytes.  Sources: E2M1 value set, the
+ * palettes post, opening section; E4M3 range, IF4 paper page, Table 1. */
+NVFP4_API int nvfp4_encode_e2m1(const float* in, int64_t n, uint8_t* out, void* stream);
+NVFP4_API int nvfp4_encode_e4m3(const float* in, int64_t n, int round_up, uint8_t* out, void* stream);
+
+/* Static string naming a status code (never NULL). */
+NVFP4_API const char* nvfp4_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

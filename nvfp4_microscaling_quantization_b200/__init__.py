@@ -1,0 +1,13 @@
+"""Block-scaled NVFP4 quantization of bf16 training tensors on B200 (sm_100a).
+
+The kernels and the C ABI live in libnvfp4.so (sources in csrc/, interface in
+include/nvfp4.h); `binding` is the ctypes layer over it and `workloads` the
+seeded synthetic inputs.  Importing the package does not load the library;
+the first call through `binding` does, and raises if it is missing.
+"""
+from . import workloads  # noqa: F401
+from .binding import (  # noqa: F401
+    FOUR_OVER_SIX, IF4, MS_EDEN, ROWWISE, RTN, SR, TRANSPOSED, Nvfp4Error, amax, dequantize, encode_e2m1,
+    encode_e4m3, lib, nvfp4_encode_e2m1, nvfp4_encode_e4m3,
+    nvfp4_amax, nvfp4_dequantize, nvfp4_quantize, nvfp4_rht, nvfp4_status_string, nvfp4_workspace_bytes,
+    quantize, rht, view_shape)

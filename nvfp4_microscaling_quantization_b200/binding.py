@@ -1,0 +1,209 @@
+"""Thin Python binding of libnvfp4.so (argument marshalling only).
+
+The functions named like the C ABI (nvfp4_quantize, nvfp4_dequantize, nvfp4_rht,
+nvfp4_amax, nvfp4_workspace_bytes, nvfp4_status_string) take raw device
+pointers and sizes exactly as include/nvfp4.h declares them.  The tensor-level
+helpers (quantize, dequantize, rht, amax) take torch CUDA tensors, allocate the
+outputs with torch (device memory is the only thing torch provides here) and
+call the same entry points on the current CUDA stream.  Every step of the
+computation runs in the library's kernels; there is no CPU path.  If the
+library has not been built, every call raises.
+"""
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+ROWWISE, TRANSPOSED = 0, 1
+RTN, SR, MS_EDEN, IF4, FOUR_OVER_SIX = 0, 1, 2, 3, 4
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
+
+_lib = None
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {nvfp4_status_string(status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libnvfp4.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libnvfp4.so not found at {LIB_PATH}; build it with "
+                "`python -m nvfp4_microscaling_quantization_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i64, u64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_int, ctypes.c_size_t
+        L.nvfp4_workspace_bytes.argtypes = [i64, i64, i32, i32, i32]
+        L.nvfp4_workspace_bytes.restype = sz
+        L.nvfp4_amax.argtypes = [P, i64, i64, i64, i32, i32, u64, P, P]
+        L.nvfp4_amax.restype = i32
+        L.nvfp4_quantize.argtypes = [P, i64, i64, i64, i32, i32, i32, u64, P, P, P, P, P, sz, P]
+        L.nvfp4_quantize.restype = i32
+        L.nvfp4_dequantize.argtypes = [P, P, P, i64, i64, i32, i32, u64, i32, P, P]
+        L.nvfp4_dequantize.restype = i32
+        L.nvfp4_rht.argtypes = [P, i32, i64, i64, i64, i32, i32, u64, i32, P, P]
+        L.nvfp4_rht.restype = i32
+        L.nvfp4_encode_e2m1.argtypes = [P, i64, P, P]
+        L.nvfp4_encode_e2m1.restype = i32
+        L.nvfp4_encode_e4m3.argtypes = [P, i64, i32, P, P]
+        L.nvfp4_encode_e4m3.restype = i32
+        L.nvfp4_status_string.argtypes = [i32]
+        L.nvfp4_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+# --------------------------------------------------------------------------- raw C ABI
+def nvfp4_status_string(status: int) -> str:
+    return lib().nvfp4_status_string(status).decode()
+
+
+def nvfp4_workspace_bytes(rows, cols, layout, mode, rht_group) -> int:
+    return lib().nvfp4_workspace_bytes(rows, cols, layout, mode, rht_group)
+
+
+def nvfp4_amax(x, rows, cols, ld, layout, rht_group, seed, amax_out, stream) -> int:
+    return lib().nvfp4_amax(x, rows, cols, ld, layout, rht_group, seed, amax_out, stream)
+
+
+def nvfp4_quantize(x, rows, cols, ld, layout, mode, rht_group, seed, amax_in, codes, scales,
+                   global_scale, workspace, workspace_bytes, stream) -> int:
+    return lib().nvfp4_quantize(x, rows, cols, ld, layout, mode, rht_group, seed, amax_in, codes,
+                                scales, global_scale, workspace, workspace_bytes, stream)
+
+
+def nvfp4_dequantize(codes, scales, global_scale, vrows, vcols, mode, rht_group, seed, inverse_rht,
+                     out, stream) -> int:
+    return lib().nvfp4_dequantize(codes, scales, global_scale, vrows, vcols, mode, rht_group, seed,
+                                  inverse_rht, out, stream)
+
+
+def nvfp4_rht(x, in_dtype, rows, cols, ld, layout, rht_group, seed, inverse, out, stream) -> int:
+    return lib().nvfp4_rht(x, in_dtype, rows, cols, ld, layout, rht_group, seed, inverse, out, stream)
+
+
+def nvfp4_encode_e2m1(x, n, out, stream) -> int:
+    return lib().nvfp4_encode_e2m1(x, n, out, stream)
+
+
+def nvfp4_encode_e4m3(x, n, round_up, out, stream) -> int:
+    return lib().nvfp4_encode_e4m3(x, n, round_up, out, stream)
+
+
+# ----------------------------------------------------------------------- tensor helpers
+def _stream_handle(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _matrix(x: torch.Tensor, dtype) -> Tuple[int, int, int]:
+    if not x.is_cuda:
+        raise ValueError("nvfp4 works on CUDA tensors only")
+    if x.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {x.dtype}")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with unit column stride")
+    rows, cols = x.shape
+    return rows, cols, max(x.stride(0), cols, 1)
+
+
+def view_shape(rows: int, cols: int, layout: int) -> Tuple[int, int]:
+    return (rows, cols) if layout == ROWWISE else (cols, rows)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise Nvfp4Error(status, what)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def amax(x: torch.Tensor, layout: int = ROWWISE, rht_group: int = 0, seed: int = 0,
+         out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    rows, cols, ld = _matrix(x, torch.bfloat16)
+    out = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else out
+    _check(nvfp4_amax(_p(x), rows, cols, ld, layout, rht_group, seed, _p(out), _stream_handle(stream)),
+           "nvfp4_amax")
+    return out
+
+
+def alloc_outputs(rows: int, cols: int, layout: int, device) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    vr, vc = view_shape(rows, cols, layout)
+    codes = torch.empty((vr, vc // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((vr, vc // 16), dtype=torch.uint8, device=device)
+    gscale = torch.empty(1, dtype=torch.float32, device=device)
+    return codes, scales, gscale
+
+
+def quantize(x: torch.Tensor, layout: int = ROWWISE, mode: int = RTN, rht_group: int = 0, seed: int = 0,
+             amax_in: Optional[torch.Tensor] = None, out=None, workspace: Optional[torch.Tensor] = None,
+             stream=None):
+    """Quantize a bf16 CUDA matrix; returns (codes, scales, global_scale) device tensors."""
+    rows, cols, ld = _matrix(x, torch.bfloat16)
+    codes, scales, gscale = alloc_outputs(rows, cols, layout, x.device) if out is None else out
+    ws_bytes = 0
+    if amax_in is None:
+        ws_bytes = nvfp4_workspace_bytes(rows, cols, layout, mode, rht_group)
+        if workspace is None:
+            workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=x.device)
+    st = nvfp4_quantize(_p(x), rows, cols, ld, layout, mode, rht_group, seed, _p(amax_in), _p(codes),
+                        _p(scales), _p(gscale), _p(workspace) if amax_in is None else None,
+                        workspace.numel() if (amax_in is None and workspace is not None) else 0,
+                        _stream_handle(stream))
+    _check(st, "nvfp4_quantize")
+    return codes, scales, gscale
+
+
+def dequantize(codes: torch.Tensor, scales: torch.Tensor, gscale: torch.Tensor, mode: int = RTN,
+               rht_group: int = 0, seed: int = 0, inverse_rht: bool = False, stream=None) -> torch.Tensor:
+    vr, half = codes.shape
+    vc = 2 * half
+    out = torch.empty((vr, vc), dtype=torch.float32, device=codes.device)
+    _check(nvfp4_dequantize(_p(codes), _p(scales), _p(gscale), vr, vc, mode, rht_group, seed,
+                            int(inverse_rht), _p(out), _stream_handle(stream)), "nvfp4_dequantize")
+    return out
+
+
+def rht(x: torch.Tensor, layout: int = ROWWISE, rht_group: int = 128, seed: int = 0, inverse: bool = False,
+        stream=None) -> torch.Tensor:
+    if x.dtype == torch.bfloat16:
+        dt = 0
+    elif x.dtype == torch.float32:
+        dt = 1
+    else:
+        raise TypeError("rht takes bf16 or fp32")
+    rows, cols, ld = _matrix(x, x.dtype)
+    vr, vc = view_shape(rows, cols, layout)
+    out = torch.empty((vr, vc), dtype=torch.float32, device=x.device)
+    _check(nvfp4_rht(_p(x), dt, rows, cols, ld, layout, rht_group, seed, int(inverse), _p(out),
+                     _stream_handle(stream)), "nvfp4_rht")
+    return out
+
+
+def encode_e2m1(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """E2M1 code (one per byte) of every float of a CUDA fp32 tensor."""
+    if not x.is_cuda or x.dtype != torch.float32:
+        raise TypeError("encode_e2m1 takes a CUDA float32 tensor")
+    x = x.contiguous()
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(nvfp4_encode_e2m1(_p(x), x.numel(), _p(out), _stream_handle(stream)), "nvfp4_encode_e2m1")
+    return out
+
+
+def encode_e4m3(x: torch.Tensor, round_up: bool = False, stream=None) -> torch.Tensor:
+    """E4M3 code of every non-negative float of a CUDA fp32 tensor (RNE or round-up, saturating)."""
+    if not x.is_cuda or x.dtype != torch.float32:
+        raise TypeError("encode_e4m3 takes a CUDA float32 tensor")
+    x = x.contiguous()
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(nvfp4_encode_e4m3(_p(x), x.numel(), int(round_up), _p(out), _stream_handle(stream)),
+           "nvfp4_encode_e4m3")
+    return out

@@ -1,0 +1,147 @@
+// api.cu -- the C ABI of libnvfp4.so (declared in include/nvfp4.h):
+// argument checks on the host, then kernel launches on the caller's stream.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "nvfp4.h"
+
+namespace {
+
+constexpr size_t kWorkspaceBytes = 256;  // one 32-bit amax accumulator, padded
+
+bool valid_group(int g) { return g == 0 || g == 16 || g == 32 || g == 64 || g == 128; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Checks shared by quantize and amax.  On success fills the view shape.
+// An empty tensor (rows or cols zero) may come with NULL data pointers and any
+// ld; nothing is read or written for it except the tensor scale.
+int check_tensor(const void* x, int64_t rows, int64_t cols, int64_t ld, int layout, int rht_group,
+                 int64_t* vrows, int64_t* vcols) {
+  if (layout != NVFP4_ROWWISE && layout != NVFP4_TRANSPOSED) return NVFP4_ERR_INVALID_ARG;
+  if (!valid_group(rht_group)) return NVFP4_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0) return NVFP4_ERR_SHAPE;
+  *vrows = layout == NVFP4_ROWWISE ? rows : cols;
+  *vcols = layout == NVFP4_ROWWISE ? cols : rows;
+  if (*vcols % 16) return NVFP4_ERR_SHAPE;
+  if (rht_group && *vcols % rht_group) return NVFP4_ERR_SHAPE;
+  if (layout == NVFP4_TRANSPOSED && cols % 8) return NVFP4_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (!x) return NVFP4_ERR_INVALID_ARG;
+  if (ld < cols) return NVFP4_ERR_SHAPE;
+  if (!aligned(x, 16) || ld % 8) return NVFP4_ERR_ALIGNMENT;
+  return NVFP4_OK;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t nvfp4_workspace_bytes(int64_t rows, int64_t cols, int layout, int mode, int rht_group) {
+  if (rows < 0 || cols < 0 || (layout != 0 && layout != 1) || mode < 0 || mode > 4 ||
+      !valid_group(rht_group))
+    return 0;
+  return kWorkspaceBytes;
+}
+
+int nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int layout, int rht_group,
+               uint64_t seed, float* amax_out, void* stream) {
+  int64_t vr, vc;
+  int st = check_tensor(x, rows, cols, ld, layout, rht_group, &vr, &vc);
+  if (st) return st;
+  if (!amax_out) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(amax_out, 4)) return NVFP4_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = from_cuda(cudaMemsetAsync(amax_out, 0, sizeof(float), s)))) return st;
+  nvfp4::QuantArgs a{x, rows, cols, ld, layout, NVFP4_RTN, rht_group, seed, nullptr, amax_out,
+                     nullptr, nullptr, nullptr, s};
+  return from_cuda(nvfp4::launch_amax(a));
+}
+
+int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int layout, int mode,
+                   int rht_group, uint64_t seed, const float* amax_in, uint8_t* codes,
+                   uint8_t* scales, float* global_scale, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  int64_t vr, vc;
+  int st = check_tensor(x, rows, cols, ld, layout, rht_group, &vr, &vc);
+  if (st) return st;
+  if (mode < NVFP4_RTN || mode > NVFP4_4OVER6) return NVFP4_ERR_INVALID_ARG;
+  if (mode == NVFP4_MS_EDEN && rht_group == 0) return NVFP4_ERR_UNSUPPORTED;
+  const bool empty = vr == 0 || vc == 0;
+  if (!global_scale || (!empty && (!codes || !scales))) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes, 8) || !aligned(global_scale, 4)) return NVFP4_ERR_ALIGNMENT;
+  if (amax_in && !aligned(amax_in, 4)) return NVFP4_ERR_ALIGNMENT;
+  if (!amax_in) {
+    if (!workspace || workspace_bytes < kWorkspaceBytes) return NVFP4_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return NVFP4_ERR_ALIGNMENT;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  nvfp4::QuantArgs a{x, rows, cols, ld, layout, mode, rht_group, seed, amax_in, nullptr,
+                     codes, scales, global_scale, s};
+  if (!amax_in) {
+    if ((st = from_cuda(cudaMemsetAsync(workspace, 0, sizeof(float), s)))) return st;
+    a.amax_accum = workspace;
+    if ((st = from_cuda(nvfp4::launch_amax(a)))) return st;
+    a.amax = static_cast<const float*>(workspace);
+  }
+  return from_cuda(nvfp4::launch_quantize(a));
+}
+
+int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
+                     int64_t vrows, int64_t vcols, int mode, int rht_group, uint64_t seed,
+                     int inverse_rht, float* out, void* stream) {
+  if (!codes || !scales || !global_scale || !out) return NVFP4_ERR_INVALID_ARG;
+  if (mode < NVFP4_RTN || mode > NVFP4_4OVER6 || !valid_group(rht_group)) return NVFP4_ERR_INVALID_ARG;
+  if (inverse_rht && rht_group == 0) return NVFP4_ERR_INVALID_ARG;
+  if (vrows < 0 || vcols < 0 || vcols % 16 || (rht_group && vcols % rht_group)) return NVFP4_ERR_SHAPE;
+  if (!aligned(codes, 8) || !aligned(out, 16) || !aligned(global_scale, 4)) return NVFP4_ERR_ALIGNMENT;
+  nvfp4::DequantArgs a{codes, scales, global_scale, vrows, vcols, mode, rht_group, seed,
+                       inverse_rht ? 1 : 0, out, static_cast<cudaStream_t>(stream)};
+  return from_cuda(nvfp4::launch_dequantize(a));
+}
+
+int nvfp4_rht(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld, int layout,
+              int rht_group, uint64_t seed, int inverse, float* out, void* stream) {
+  if (!in || !out) return NVFP4_ERR_INVALID_ARG;
+  if (in_dtype != 0 && in_dtype != 1) return NVFP4_ERR_INVALID_ARG;
+  if (layout != NVFP4_ROWWISE && layout != NVFP4_TRANSPOSED) return NVFP4_ERR_INVALID_ARG;
+  if (rht_group == 0 || !valid_group(rht_group)) return NVFP4_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0 || ld < cols || ld < 1) return NVFP4_ERR_SHAPE;
+  const int64_t vcols = layout == NVFP4_ROWWISE ? cols : rows;
+  if (vcols % 16 || vcols % rht_group) return NVFP4_ERR_SHAPE;
+  if (!aligned(in, in_dtype == 0 ? 2 : 4) || !aligned(out, 16)) return NVFP4_ERR_ALIGNMENT;
+  nvfp4::RhtArgs a{in, in_dtype, rows, cols, ld, layout, rht_group, seed, inverse ? 1 : 0, out,
+                   static_cast<cudaStream_t>(stream)};
+  return from_cuda(nvfp4::launch_rht(a));
+}
+
+int nvfp4_encode_e2m1(const float* in, int64_t n, uint8_t* out, void* stream) {
+  if (!in || !out) return NVFP4_ERR_INVALID_ARG;
+  if (n < 0) return NVFP4_ERR_SHAPE;
+  if (!aligned(in, 4)) return NVFP4_ERR_ALIGNMENT;
+  return from_cuda(nvfp4::launch_encode_e2m1(in, n, out, static_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_encode_e4m3(const float* in, int64_t n, int round_up, uint8_t* out, void* stream) {
+  if (!in || !out) return NVFP4_ERR_INVALID_ARG;
+  if (n < 0) return NVFP4_ERR_SHAPE;
+  if (!aligned(in, 4)) return NVFP4_ERR_ALIGNMENT;
+  return from_cuda(nvfp4::launch_encode_e4m3(in, n, round_up, out, static_cast<cudaStream_t>(stream)));
+}
+
+const char* nvfp4_status_string(int status) {
+  switch (status) {
+    case NVFP4_OK: return "NVFP4_OK";
+    case NVFP4_ERR_INVALID_ARG: return "NVFP4_ERR_INVALID_ARG";
+    case NVFP4_ERR_SHAPE: return "NVFP4_ERR_SHAPE";
+    case NVFP4_ERR_ALIGNMENT: return "NVFP4_ERR_ALIGNMENT";
+    case NVFP4_ERR_UNSUPPORTED: return "NVFP4_ERR_UNSUPPORTED";
+    case NVFP4_ERR_WORKSPACE: return "NVFP4_ERR_WORKSPACE";
+    case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
+    default: return "NVFP4_UNKNOWN_STATUS";
+  }
+}
+
+}  // extern "C"

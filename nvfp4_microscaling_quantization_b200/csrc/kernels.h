@@ -1,0 +1,56 @@
+// kernels.h -- internal launcher interface between the C ABI (api.cu) and the
+// kernel translation units.  Not installed; the public interface is
+// include/nvfp4.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+struct QuantArgs {
+  const void* x;          // bf16 rows x cols, leading dimension ld
+  int64_t rows, cols, ld;
+  int layout;             // 0 row-wise, 1 transposed
+  int mode;               // nvfp4_mode
+  int rht_group;          // 0, 16, 32, 64, 128
+  uint64_t seed;
+  const float* amax;      // tensor amax (quantize)
+  void* amax_accum;       // zeroed 32-bit word receiving the amax bits (pre-pass)
+  uint8_t* codes;
+  uint8_t* scales;
+  float* gscale;
+  cudaStream_t stream;
+};
+
+struct DequantArgs {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const float* gscale;
+  int64_t vrows, vcols;
+  int mode, rht_group;
+  uint64_t seed;
+  int inverse_rht;
+  float* out;
+  cudaStream_t stream;
+};
+
+struct RhtArgs {
+  const void* in;
+  int in_dtype;           // 0 bf16, 1 fp32
+  int64_t rows, cols, ld;
+  int layout, rht_group;
+  uint64_t seed;
+  int inverse;
+  float* out;
+  cudaStream_t stream;
+};
+
+cudaError_t launch_amax(const QuantArgs& a);
+cudaError_t launch_quantize(const QuantArgs& a);
+cudaError_t launch_dequantize(const DequantArgs& a);
+cudaError_t launch_rht(const RhtArgs& a);
+cudaError_t launch_encode_e2m1(const float* in, int64_t n, uint8_t* out, cudaStream_t stream);
+cudaError_t launch_encode_e4m3(const float* in, int64_t n, int round_up, uint8_t* out, cudaStream_t stream);
+
+}  // namespace nvfp4

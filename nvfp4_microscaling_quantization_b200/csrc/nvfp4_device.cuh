@@ -1,0 +1,386 @@
+// nvfp4_device.cuh -- device building blocks of the NVFP4 quantizer (sm_100a).
+//
+// Every floating-point step that decides a code or a scale is one IEEE
+// binary32 operation with round-to-nearest-even, written with the explicit
+// __f*_rn intrinsics (and the library is built with -fmad=false, so nothing is
+// contracted).  The step order is the method's: rotate, block absmax, block
+// scale, scale to the grid, round, pack.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace nvfp4 {
+
+enum Mode { kRTN = 0, kSR = 1, kMSEDEN = 2, kIF4 = 3, k4over6 = 4 };
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy
+// as 1, 2, 3", SC'11): ten rounds of two 32x32->64 multiplications by the
+// round multipliers, the high halves mixed with the other counter words and
+// the key, the key advanced by the two Weyl increments between rounds.
+struct PhiloxKey {
+  uint32_t k0, k1;
+};
+
+__device__ __forceinline__ PhiloxKey philox_key(uint64_t seed) {
+  return PhiloxKey{static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32)};
+}
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, PhiloxKey key) {
+  uint32_t k0 = key.k0, k1 = key.k1;
+#pragma unroll
+  for (int round = 0; round < 10; ++round) {
+    const uint32_t lo0 = 0xD2511F53u * c.x;
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+
+// Stream tags carried in counter word 2.
+constexpr uint32_t kTagElement = 0;  // element stochastic rounding: 8 x 16-bit uniforms per call
+constexpr uint32_t kTagBlock = 1;    // scale stochastic rounding: 4 x 24-bit uniforms per call
+constexpr uint32_t kTagSigns = 2;    // RHT signs: 128 sign bits from call 0
+
+__device__ __forceinline__ uint4 philox_call(PhiloxKey key, uint64_t call, uint32_t tag) {
+  return philox4x32_10(
+      make_uint4(static_cast<uint32_t>(call), static_cast<uint32_t>(call >> 32), tag, 0u), key);
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4& w, uint32_t i) {
+  return i == 0 ? w.x : (i == 1 ? w.y : (i == 2 ? w.z : w.w));
+}
+
+// ---------------------------------------------------------------------------
+// Format conversions through the sm_100a conversion instructions.
+//
+// E2M1: 4 pairs of floats -> 8 codes in one 32-bit word, element 2k in the low
+// nibble of byte k.  The hardware rounds to nearest-even and saturates at 6;
+// a negative value that rounds to zero comes back as 0x8 and is cleared by
+// clear_negative_zero() so zero is always code 0.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return out;
+}
+
+// For each nibble: keep the sign bit only if the magnitude bits are nonzero.
+__device__ __forceinline__ uint32_t clear_negative_zero(uint32_t w) {
+  const uint32_t mag = w & 0x77777777u;
+  const uint32_t nonzero = (mag + 0x77777777u) & 0x88888888u;  // bit 3 of a nibble set iff mag != 0
+  return mag | (w & nonzero);
+}
+
+// 8 packed E2M1 codes -> 8 floats (exact: every grid value is an f16).
+__device__ __forceinline__ void e2m1x8_to_f32(uint32_t w, float* v) {
+  uint32_t h[4];
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "mov.b32 {q0, q1, q2, q3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, q2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, q3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    __half2 p = *reinterpret_cast<__half2*>(&h[k]);
+    v[2 * k] = __low2float(p);
+    v[2 * k + 1] = __high2float(p);
+  }
+}
+
+// E4M3 round-to-nearest-even with saturation at 448 (v >= 0).
+__device__ __forceinline__ uint32_t e4m3_rne_sat(float v) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(v));
+  return out & 0xFFu;
+}
+
+// E4M3 code (0x00..0x7E) -> float, exact.
+__device__ __forceinline__ float e4m3_decode(uint32_t code) {
+  uint32_t h2;
+  const uint16_t in = static_cast<uint16_t>(code & 0x7Fu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return __low2float(*reinterpret_cast<__half2*>(&h2));
+}
+
+// Smallest E4M3 value >= v, capped at 448 (v >= 0).
+__device__ __forceinline__ uint32_t e4m3_ru_sat(float v) {
+  uint32_t s = e4m3_rne_sat(v);
+  if (s < 0x7Eu && e4m3_decode(s) < v) ++s;
+  return s;
+}
+
+// Stochastic rounding of t >= 0 onto E4M3 with a uniform U in [0, 1):
+// neighbours lo <= t < hi, hi with probability (t - lo) / (hi - lo); t >= 448
+// gives 448.  (t - lo) and the division by the power-of-two gap are exact.
+__device__ __forceinline__ uint32_t e4m3_sr(float t, float U) {
+  if (!(t > 0.0f)) return 0u;
+  if (t >= 448.0f) return 0x7Eu;
+  uint32_t lo = e4m3_rne_sat(t);
+  if (e4m3_decode(lo) > t) --lo;
+  const float l = e4m3_decode(lo);
+  const float h = e4m3_decode(lo + 1);
+  const float f = __fdiv_rn(__fsub_rn(t, l), __fsub_rn(h, l));
+  return U < f ? lo + 1 : lo;
+}
+
+// bf16 pair (one 32-bit word) -> two floats.
+__device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xFFFF0000u);
+}
+
+// ---------------------------------------------------------------------------
+// Random Hadamard rotation of a g-group (g in 16..128) held as 16 consecutive
+// elements per lane by g/16 consecutive lanes.  Butterfly order: h = 1, 2, 4,
+// 8 inside the lane, then h = 16, 32, 64 across lanes (partner = lane ^ h/16):
+// (u_i, u_{i+h}) <- (u_i + u_{i+h}, u_i - u_{i+h}).  Each sum is one RN
+// addition, so the result matches a sequential butterfly in the same order.
+__device__ __forceinline__ void fwht16_local(float* v) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (i & h) continue;
+      const float a = v[i], b = v[i + h];
+      v[i] = __fadd_rn(a, b);
+      v[i + h] = __fsub_rn(a, b);
+    }
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void fwht_cross_lanes(float* v, uint32_t lane_in_group) {
+#pragma unroll
+  for (int hl = 1; hl < G / 16; hl <<= 1) {
+    const bool upper = (lane_in_group & hl) != 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float other = __shfl_xor_sync(0xFFFFFFFFu, v[i], hl);
+      v[i] = upper ? __fsub_rn(other, v[i]) : __fadd_rn(v[i], other);
+    }
+  }
+}
+
+template <int G>
+struct RhtConst;
+template <> struct RhtConst<16> { static constexpr float c = 0.25f; };
+template <> struct RhtConst<32> { static constexpr float c = 0x1.6a09e6p-3f; };  // RN(1/sqrt(32))
+template <> struct RhtConst<64> { static constexpr float c = 0.125f; };
+template <> struct RhtConst<128> { static constexpr float c = 0x1.6a09e6p-4f; }; // RN(1/sqrt(128))
+
+// 16 sign bits of this lane's slice of the g-long sign vector.
+__device__ __forceinline__ uint32_t rht_sign_bits(PhiloxKey key, uint32_t lane_in_group) {
+  const uint4 w = philox_call(key, 0, kTagSigns);
+  return (word_of(w, lane_in_group >> 1) >> ((lane_in_group & 1u) * 16u)) & 0xFFFFu;
+}
+
+template <int G>
+__device__ __forceinline__ void rht_forward(float* v, uint32_t sign_bits, uint32_t lane_in_group) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((sign_bits >> i) & 1u) << 31));
+  fwht16_local(v);
+  if constexpr (G > 16) fwht_cross_lanes<G>(v, lane_in_group);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], RhtConst<G>::c);
+}
+
+template <int G>
+__device__ __forceinline__ void rht_inverse(float* v, uint32_t sign_bits, uint32_t lane_in_group) {
+  fwht16_local(v);
+  if constexpr (G > 16) fwht_cross_lanes<G>(v, lane_in_group);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    v[i] = __fmul_rn(v[i], RhtConst<G>::c);
+    v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((sign_bits >> i) & 1u) << 31));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tensor scale: s_g = RN(A / (6 M)), M = 256 for MS-EDEN and 4/6, else 448.
+template <int MODE>
+__device__ __forceinline__ float global_scale_of(float amax) {
+  constexpr float six_m = (MODE == kMSEDEN || MODE == k4over6) ? 1536.0f : 2688.0f;
+  return amax > 0.0f ? __fdiv_rn(amax, six_m) : 1.0f;
+}
+
+// INT4 option of IF4: levels k in [-7, 7] standing for k * 6/7.
+constexpr float kIF4K1 = 0x1.2aaaaap+0f;  // RN(7/6)
+constexpr float kIF4K2 = 0x1.b6db6ep-1f;  // RN(6/7)
+
+// Where the random draws of one 16-element block come from.
+struct BlockRng {
+  PhiloxKey key;
+  uint64_t first_element;  // view linear index of element 0 of the block (a multiple of 16)
+  uint64_t block;          // view linear block index
+};
+
+struct BlockOut {
+  uint32_t lo, hi;  // 16 packed codes: lo = elements 0..7, hi = elements 8..15
+  uint32_t scale;   // scale byte (bit 7 = IF4 INT4 flag)
+};
+
+__device__ __forceinline__ float block_absmax(const float* z) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(z[i]));
+  return a;
+}
+
+// RTN codes of 16 scaled values.
+__device__ __forceinline__ void rtn_codes(const float* y, uint32_t& lo, uint32_t& hi) {
+  lo = clear_negative_zero(cvt_e2m1x8(y));
+  hi = clear_negative_zero(cvt_e2m1x8(y + 8));
+}
+
+// Stochastic rounding of one scaled value with the uniform k * 2^-16.
+__device__ __forceinline__ uint32_t sr_code(float y, uint32_t k16) {
+  const float a = fminf(fabsf(y), 6.0f);
+  // grid interval: [0,2) step 1/2, [2,4) step 1, [4,6] step 2
+  const float inv_step = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
+  const uint32_t base = a < 2.0f ? 0u : (a < 4.0f ? 2u : 4u);
+  const float t = __fmul_rn(a, inv_step);  // exact
+  const float fl = floorf(t);
+  const float frac = __fsub_rn(t, fl);     // exact: position inside the interval
+  uint32_t mag = static_cast<uint32_t>(fl) + base;
+  const float U = __fmul_rn(static_cast<float>(k16), 0x1p-16f);
+  if (U < frac) ++mag;
+  if (mag == 0u) return 0u;
+  return mag | (y < 0.0f ? 8u : 0u);
+}
+
+// Quantize one block of 16 (already rotated) values z under tensor scale s_g.
+template <int MODE>
+__device__ __forceinline__ BlockOut quantize_block(const float* z, float s_g, const BlockRng& rng) {
+  BlockOut out{0u, 0u, 0u};
+  const float a_b = block_absmax(z);
+
+  if constexpr (MODE == k4over6) {
+    uint32_t S[2], c_lo[2], c_hi[2];
+    float err[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float m = k == 0 ? 6.0f : 4.0f;
+      const float s_f = __fdiv_rn(a_b, __fmul_rn(m, s_g));
+      S[k] = e4m3_rne_sat(s_f);
+      const float d = __fmul_rn(e4m3_decode(S[k]), s_g);
+      float e = 0.0f;
+      if (d == 0.0f) {
+        c_lo[k] = c_hi[k] = 0u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) e = __fmaf_rn(z[i], z[i], e);
+      } else {
+        const float r = __frcp_rn(d);
+        float y[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(z[i], r);
+        rtn_codes(y, c_lo[k], c_hi[k]);
+        float v[16];
+        e2m1x8_to_f32(c_lo[k], v);
+        e2m1x8_to_f32(c_hi[k], v + 8);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float diff = __fsub_rn(z[i], __fmul_rn(v[i], d));
+          e = __fmaf_rn(diff, diff, e);
+        }
+      }
+      err[k] = e;
+    }
+    const int pick = err[1] < err[0] ? 1 : 0;
+    out.lo = c_lo[pick];
+    out.hi = c_hi[pick];
+    out.scale = S[pick];
+    return out;
+  } else {
+    const float s_f = __fdiv_rn(a_b, __fmul_rn(6.0f, s_g));
+    const uint32_t S = MODE == kSR ? e4m3_ru_sat(s_f) : e4m3_rne_sat(s_f);
+    const float d = __fmul_rn(e4m3_decode(S), s_g);
+    out.scale = S;
+    if (d == 0.0f) return out;
+    const float r = __frcp_rn(d);
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(z[i], r);
+
+    if constexpr (MODE == kRTN) {
+      rtn_codes(y, out.lo, out.hi);
+    } else if constexpr (MODE == kSR) {
+      const uint64_t call0 = rng.first_element >> 3;
+      const uint4 w0 = philox_call(rng.key, call0, kTagElement);
+      const uint4 w1 = philox_call(rng.key, call0 + 1, kTagElement);
+      uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t word0 = word_of(w0, i >> 1), word1 = word_of(w1, i >> 1);
+        const uint32_t k0 = (word0 >> ((i & 1) * 16)) & 0xFFFFu;
+        const uint32_t k1 = (word1 >> ((i & 1) * 16)) & 0xFFFFu;
+        lo |= sr_code(y[i], k0) << (4 * i);
+        hi |= sr_code(y[8 + i], k1) << (4 * i);
+      }
+      out.lo = lo;
+      out.hi = hi;
+    } else if constexpr (MODE == kMSEDEN) {
+      rtn_codes(y, out.lo, out.hi);
+      float v[16];
+      e2m1x8_to_f32(out.lo, v);
+      e2m1x8_to_f32(out.hi, v + 8);
+      float num = 0.0f, den = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        num = __fmaf_rn(y[i], y[i], num);
+        den = __fmaf_rn(y[i], v[i], den);
+      }
+      const float c = (num > 0.0f && den > 0.0f) ? __fdiv_rn(num, den) : 1.0f;
+      const float t = __fmul_rn(e4m3_decode(S), c);
+      const uint4 w = philox_call(rng.key, rng.block >> 2, kTagBlock);
+      const float U = __fmul_rn(static_cast<float>(word_of(w, rng.block & 3u) >> 8), 0x1p-24f);
+      out.scale = e4m3_sr(t, U);
+    } else {  // kIF4
+      uint32_t f_lo, f_hi;
+      rtn_codes(y, f_lo, f_hi);
+      float v[16];
+      e2m1x8_to_f32(f_lo, v);
+      e2m1x8_to_f32(f_hi, v + 8);
+      float eF = 0.0f, eI = 0.0f;
+      uint32_t i_lo = 0u, i_hi = 0u;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float dF = __fsub_rn(y[i], v[i]);
+        eF = __fmaf_rn(dF, dF, eF);
+        int k = __float2int_rn(__fmul_rn(y[i], kIF4K1));
+        k = max(-7, min(7, k));
+        const float dI = __fsub_rn(y[i], __fmul_rn(static_cast<float>(k), kIF4K2));
+        eI = __fmaf_rn(dI, dI, eI);
+        const uint32_t code = k == 0 ? 0u : (static_cast<uint32_t>(k < 0 ? -k : k) | (k < 0 ? 8u : 0u));
+        if (i < 8) i_lo |= code << (4 * i);
+        else i_hi |= code << (4 * (i - 8));
+      }
+      if (eI < eF) {
+        out.lo = i_lo;
+        out.hi = i_hi;
+        out.scale = S | 0x80u;
+      } else {
+        out.lo = f_lo;
+        out.hi = f_hi;
+      }
+    }
+    return out;
+  }
+}
+
+}  // namespace nvfp4

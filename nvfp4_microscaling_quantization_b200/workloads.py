@@ -7,10 +7,13 @@ names the calls each workload makes.  Both the CUDA path (through bench.py and
 the GPU tests) and the CPU oracle (through the tests) read the same tensors
 from here.
 
-Every tensor is drawn on the host with a torch CPU generator seeded by the
-workload seed, in float32, then rounded to bf16 (round-to-nearest-even).  The
-draws happen in the order written below, so a (workload, seed) pair always
-gives the same bits.
+Every tensor is drawn with a torch generator seeded by the workload seed, in
+float32, then rounded to bf16 (round-to-nearest-even).  The draws happen in
+the order written below, so a (workload, seed, device) triple always gives the
+same bits.  Small tensors are drawn on the CPU; the full-size workloads are
+drawn on the GPU (torch's CUDA generator), which takes well under a second
+where the CPU takes about a minute, and are copied to the host when the
+oracle needs them.
 
 Distributions (the pages' workloads are the weight, activation and gradient
 tensors of LLM linear layers, quantized forward with RTN / 4-over-6 / IF4 and
@@ -33,38 +36,40 @@ MODE_NAMES = {RTN: "rtn", SR: "sr", MS_EDEN: "ms_eden", IF4: "if4", FOUR_OVER_SI
 LAYOUT_NAMES = {ROWWISE: "rowwise", TRANSPOSED: "transposed"}
 
 
-def _gen(seed: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+def _gen(seed: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
     g.manual_seed(seed)
     return g
 
 
 def normal(shape, std: float, gen: torch.Generator) -> torch.Tensor:
-    return (torch.randn(shape, generator=gen, dtype=torch.float32) * std).to(torch.bfloat16)
+    return (torch.randn(shape, generator=gen, dtype=torch.float32, device=gen.device) * std).to(torch.bfloat16)
 
 
 def outlier_normal(shape, std: float, frac: float, factor: float, gen: torch.Generator) -> torch.Tensor:
-    x = torch.randn(shape, generator=gen, dtype=torch.float32) * std
-    mask = torch.rand(shape, generator=gen, dtype=torch.float32) < frac
+    x = torch.randn(shape, generator=gen, dtype=torch.float32, device=gen.device) * std
+    mask = torch.rand(shape, generator=gen, dtype=torch.float32, device=gen.device) < frac
     x = torch.where(mask, x * factor, x)
     return x.to(torch.bfloat16)
 
 
 def student_t3(shape, std: float, gen: torch.Generator) -> torch.Tensor:
-    z = torch.randn(shape, generator=gen, dtype=torch.float32)
-    chi2 = torch.zeros(shape, dtype=torch.float32)
+    z = torch.randn(shape, generator=gen, dtype=torch.float32, device=gen.device)
+    chi2 = torch.zeros(shape, dtype=torch.float32, device=gen.device)
     for _ in range(3):
-        n = torch.randn(shape, generator=gen, dtype=torch.float32)
+        n = torch.randn(shape, generator=gen, dtype=torch.float32, device=gen.device)
         chi2.addcmul_(n, n)
+        del n
     t = z / torch.sqrt(chi2 / 3.0)
     return (t * (std / 3.0 ** 0.5)).to(torch.bfloat16)
 
 
 def laplace_channels(shape, gen: torch.Generator) -> torch.Tensor:
     rows, cols = shape
-    u = torch.rand(shape, generator=gen, dtype=torch.float32) - 0.5
+    u = torch.rand(shape, generator=gen, dtype=torch.float32, device=gen.device) - 0.5
     lap = -torch.sign(u) * torch.log1p(-2.0 * u.abs())
-    col_scale = torch.pow(10.0, torch.rand((1, cols), generator=gen, dtype=torch.float32) * 2.0 - 1.0)
+    col_scale = torch.pow(10.0, torch.rand((1, cols), generator=gen, dtype=torch.float32,
+                                           device=gen.device) * 2.0 - 1.0)
     return (lap * col_scale).to(torch.bfloat16)
 
 
@@ -90,36 +95,37 @@ class Workload:
     calls: List[Call] = field(default_factory=list)
     description: str = ""
 
-    def tensors(self) -> Dict[str, torch.Tensor]:
-        return _GENERATORS[self.name](self)
+    def tensors(self, device="cpu") -> Dict[str, torch.Tensor]:
+        """The workload's bf16 tensors, drawn on `device` ("cpu" or a CUDA device)."""
+        return _GENERATORS[self.name](self, device)
 
     def elements(self, call: Call) -> int:
         r, c = self.shapes[call.tensor]
         return r * c
 
 
-def _small(w):
-    g = _gen(w.seed)
+def _small(w, device):
+    g = _gen(w.seed, device)
     return {"x": normal(w.shapes["x"], 1.0, g)}
 
 
-def _weight(w):
-    g = _gen(w.seed)
+def _weight(w, device):
+    g = _gen(w.seed, device)
     return {"w": outlier_normal(w.shapes["w"], 0.02, 0.01, 10.0, g)}
 
 
-def _gradient(w):
-    g = _gen(w.seed)
+def _gradient(w, device):
+    g = _gen(w.seed, device)
     return {"g": student_t3(w.shapes["g"], 1e-3, g)}
 
 
-def _activation(w):
-    g = _gen(w.seed)
+def _activation(w, device):
+    g = _gen(w.seed, device)
     return {"a": laplace_channels(w.shapes["a"], g)}
 
 
-def _mlp_up(w):
-    g = _gen(w.seed)
+def _mlp_up(w, device):
+    g = _gen(w.seed, device)
     x = normal(w.shapes["x"], 1.0, g)
     wt = normal(w.shapes["w"], 0.02, g)
     dy = student_t3(w.shapes["dy"], 1e-4, g)
@@ -156,7 +162,7 @@ def activation(rows=16384, cols=8192) -> Workload:
     return Workload("activation", 3, {"a": (rows, cols)}, calls, "16384x8192 Laplace x log-uniform channel scale")
 
 
-def mlp_up(tokens=16384, d_model=4096, d_ff=14336) -> Workload:
+def mlp_up(tokens=16384, d_model=4096, d_ff=14336, seed=4) -> Workload:
     """One Llama-style MLP up-projection training step, seed 4.
 
     X [tokens, d_model] N(0,1), W [d_ff, d_model] N(0, 0.02^2), dY [tokens, d_ff]
@@ -167,7 +173,7 @@ def mlp_up(tokens=16384, d_model=4096, d_ff=14336) -> Workload:
     calls = [Call("x", ROWWISE, RTN, 0), Call("w", ROWWISE, RTN, 0),
              Call("dy", ROWWISE, MS_EDEN, 128), Call("w", TRANSPOSED, MS_EDEN, 128),
              Call("dy", TRANSPOSED, MS_EDEN, 128), Call("x", TRANSPOSED, MS_EDEN, 128)]
-    return Workload("mlp_up", 4, {"x": (tokens, d_model), "w": (d_ff, d_model), "dy": (tokens, d_ff)},
+    return Workload("mlp_up", seed, {"x": (tokens, d_model), "w": (d_ff, d_model), "dy": (tokens, d_ff)},
                     calls, "MLP up-projection step: X 16384x4096, W 14336x4096, dY 16384x14336")
 
 

@@ -72,6 +72,10 @@ def _declare(L):
     L.oracle_rht_view.restype = i32
     L.oracle_if4_constants.argtypes = [P, P]
     L.oracle_if4_constants.restype = None
+    L.oracle_e2m1_rtn_array.argtypes = [P, i64, P]
+    L.oracle_e2m1_rtn_array.restype = None
+    L.oracle_e4m3_array.argtypes = [P, i64, i32, P]
+    L.oracle_e4m3_array.restype = None
 
 
 class OracleError(RuntimeError):
@@ -133,6 +137,20 @@ def e2m1_sr(y, u):
 
 def e2m1_decode(code):
     return lib().oracle_e2m1_decode(int(code))
+
+
+def e2m1_rtn_array(v):
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e2m1_rtn_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def e4m3_array(v, round_up=False):
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e4m3_array(_ptr(v), v.size, int(round_up), _ptr(out))
+    return out
 
 
 def e4m3_decode(code):

@@ -597,3 +597,13 @@ int oracle_rht_view(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, i
   for (int64_t r = 0; r < vr; ++r) load_view_row(x, ld, layout, r, vc, g, sigma, c, out + r * vc);
   return ORC_OK;
 }
+
+/* Array forms of the two codecs, for exhaustive comparisons. */
+void oracle_e2m1_rtn_array(const float* in, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_e2m1_rtn(in[i]);
+}
+
+void oracle_e4m3_array(const float* in, int64_t n, int round_up, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i)
+    out[i] = round_up ? oracle_e4m3_ru_sat(in[i]) : oracle_e4m3_rne_sat(in[i]);
+}

@@ -1,0 +1,122 @@
+"""The C-ABI library loads, exports every symbol include/nvfp4.h declares, and
+rejects bad arguments on the host before anything is launched.
+
+CPU-only: every call below fails one of the library's host-side checks, so no
+CUDA call is reached and no device pointer is ever dereferenced.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+OK, INVALID, SHAPE, ALIGN, UNSUPPORTED, WORKSPACE, CUDA = 0, -1, -2, -3, -4, -5, -6
+FAKE = 0x100000  # 16-byte aligned, never dereferenced: each call fails a check first
+
+
+@pytest.fixture(scope="module")
+def N():
+    from nvfp4_microscaling_quantization_b200 import binding, build
+    build.build()
+    binding.lib()
+    return binding
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for n in ["nvfp4_quantize", "nvfp4_dequantize", "nvfp4_rht", "nvfp4_amax", "nvfp4_workspace_bytes",
+              "nvfp4_status_string", "nvfp4_encode_e2m1", "nvfp4_encode_e4m3"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(N):
+    lib = N.lib()
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_nothing_else_exported(N):
+    """Only the C ABI is visible (the kernels and helpers are hidden)."""
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", N.LIB_PATH], capture_output=True, text=True).stdout
+    exported = sorted({l.split()[-1] for l in out.splitlines() if " T " in l})
+    assert exported == declared_symbols()
+
+
+def test_status_strings(N):
+    for st, name in [(OK, "NVFP4_OK"), (INVALID, "NVFP4_ERR_INVALID_ARG"), (SHAPE, "NVFP4_ERR_SHAPE"),
+                     (ALIGN, "NVFP4_ERR_ALIGNMENT"), (UNSUPPORTED, "NVFP4_ERR_UNSUPPORTED"),
+                     (WORKSPACE, "NVFP4_ERR_WORKSPACE"), (CUDA, "NVFP4_ERR_CUDA")]:
+        assert N.nvfp4_status_string(st) == name
+    assert N.nvfp4_status_string(12345) == "NVFP4_UNKNOWN_STATUS"
+
+
+def test_workspace_bytes(N):
+    assert N.nvfp4_workspace_bytes(4096, 4096, 0, 2, 128) == 256
+    assert N.nvfp4_workspace_bytes(4096, 4096, 2, 2, 128) == 0
+    assert N.nvfp4_workspace_bytes(4096, 4096, 0, 9, 128) == 0
+    assert N.nvfp4_workspace_bytes(4096, 4096, 0, 0, 48) == 0
+
+
+def q(N, x=FAKE, rows=64, cols=64, ld=64, layout=0, mode=0, g=0, amax=None, codes=FAKE + 0x1000,
+      scales=FAKE + 0x2000, gs=FAKE + 0x3000, ws=None, ws_bytes=0):
+    return N.nvfp4_quantize(x, rows, cols, ld, layout, mode, g, 0, amax, codes, scales, gs, ws, ws_bytes, None)
+
+
+def test_quantize_rejects(N):
+    assert q(N, x=None) == INVALID
+    assert q(N, x=None, rows=0) == WORKSPACE     # an empty tensor may have no data pointer
+    assert q(N, x=None, rows=0, gs=None) == INVALID
+    assert q(N, layout=2) == INVALID
+    assert q(N, g=48) == INVALID
+    assert q(N, mode=5) == INVALID
+    assert q(N, cols=40, ld=40) == SHAPE            # row-wise blocks need cols % 16 == 0
+    assert q(N, rows=40, layout=1) == SHAPE         # transposed blocks need rows % 16 == 0
+    assert q(N, cols=64, g=128) == SHAPE            # rotation group must divide the block dimension
+    assert q(N, rows=-1) == SHAPE
+    assert q(N, ld=32) == SHAPE                     # ld < cols
+    assert q(N, rows=64, cols=4, ld=8, layout=1) == SHAPE  # transposed needs cols % 8 == 0
+    assert q(N, x=FAKE + 8) == ALIGN                # x not 16-byte aligned
+    assert q(N, ld=68) == ALIGN                     # ld not a multiple of 8
+    assert q(N, mode=2, g=0) == UNSUPPORTED         # MS-EDEN needs the rotation
+    assert q(N, codes=None) == INVALID
+    assert q(N, scales=None) == INVALID
+    assert q(N, gs=None) == INVALID
+    assert q(N, codes=FAKE + 4) == ALIGN
+    assert q(N) == WORKSPACE                        # no amax_in and no workspace
+    assert q(N, ws=FAKE + 0x4000, ws_bytes=8) == WORKSPACE
+    assert q(N, ws=FAKE + 0x4008, ws_bytes=256) == ALIGN
+
+
+def test_other_entry_points_reject(N):
+    assert N.nvfp4_amax(None, 64, 64, 64, 0, 0, 0, FAKE, None) == INVALID
+    assert N.nvfp4_amax(FAKE, 64, 64, 64, 0, 0, 0, None, None) == INVALID
+    assert N.nvfp4_amax(FAKE, 64, 40, 40, 0, 0, 0, FAKE, None) == SHAPE
+    d = N.nvfp4_dequantize
+    assert d(None, FAKE, FAKE, 4, 64, 0, 0, 0, 0, FAKE, None) == INVALID
+    assert d(FAKE, FAKE, FAKE, 4, 64, 0, 0, 0, 1, FAKE, None) == INVALID  # inverse without rotation
+    assert d(FAKE, FAKE, FAKE, 4, 40, 0, 0, 0, 0, FAKE, None) == SHAPE
+    assert d(FAKE, FAKE, FAKE, 4, 64, 7, 0, 0, 0, FAKE, None) == INVALID
+    assert d(FAKE, FAKE, FAKE, 4, 64, 0, 0, 0, 0, FAKE + 4, None) == ALIGN
+    r = N.nvfp4_rht
+    assert r(FAKE, 0, 64, 64, 64, 0, 0, 0, 0, FAKE, None) == INVALID      # group 0
+    assert r(FAKE, 2, 64, 64, 64, 0, 16, 0, 0, FAKE, None) == INVALID     # dtype
+    assert r(FAKE, 0, 64, 48, 48, 0, 32, 0, 0, FAKE, None) == SHAPE
+    assert r(FAKE + 1, 0, 64, 64, 64, 0, 16, 0, 0, FAKE, None) == ALIGN
+    assert N.nvfp4_encode_e2m1(None, 4, FAKE, None) == INVALID
+    assert N.nvfp4_encode_e2m1(FAKE, -1, FAKE, None) == SHAPE
+    assert N.nvfp4_encode_e4m3(FAKE + 2, 4, 0, FAKE, None) == ALIGN
+
+
+def test_binding_refuses_cpu_tensors(N):
+    import torch
+    with pytest.raises(ValueError):
+        N.quantize(torch.zeros(16, 16, dtype=torch.bfloat16))

@@ -1,0 +1,245 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle, element
+by element, on the same seeded inputs.
+
+Every mode is compared bit-exactly in codes, scales (with the IF4 flag bit)
+and the FP32 tensor scale, with and without the rotation: the kernels follow
+the oracle's butterfly order and binary32 rounding, so even the rotated modes
+agree exactly (the 1e-5 relative tolerance allowed for rotated values is
+checked separately on the rotation itself and is met with zero difference).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_microscaling_quantization_b200 import binding as N
+from nvfp4_microscaling_quantization_b200 import workloads as W
+
+from gpu_helpers import assert_same, bits, compare_call, gpu_quantize, to_device
+
+pytestmark = pytest.mark.gpu
+
+MODES = [W.RTN, W.SR, W.MS_EDEN, W.IF4, W.FOUR_OVER_SIX]
+GROUPS = [0, 16, 32, 64, 128]
+
+
+@pytest.fixture(scope="module")
+def small_x():
+    return W.small().tensors()["x"]
+
+
+@pytest.mark.parametrize("layout", [W.ROWWISE, W.TRANSPOSED])
+@pytest.mark.parametrize("g", GROUPS)
+@pytest.mark.parametrize("mode", MODES)
+def test_small_workload_all_modes(small_x, mode, g, layout):
+    """256x256 N(0,1), seed 0 -- every mode, rotation group and layout."""
+    if mode == W.MS_EDEN and g == 0:
+        pytest.skip("MS-EDEN needs the rotation")
+    compare_call(small_x, layout, mode, g, 0)
+
+
+def test_small_workload_calls(small_x):
+    wl = W.small()
+    for c in wl.calls:
+        compare_call(small_x, c.layout, c.mode, c.rht_group, wl.seed)
+
+
+RAGGED = [
+    # rows, cols, ld_pad, layout, mode, g
+    (37, 48, 0, W.ROWWISE, W.RTN, 16),
+    (37, 48, 8, W.ROWWISE, W.SR, 16),
+    (1, 128, 0, W.ROWWISE, W.MS_EDEN, 128),
+    (3, 384, 8, W.ROWWISE, W.IF4, 128),
+    (5, 16, 0, W.ROWWISE, W.FOUR_OVER_SIX, 0),
+    (129, 4096 + 128, 0, W.ROWWISE, W.MS_EDEN, 128),
+    (48, 72, 0, W.TRANSPOSED, W.RTN, 16),          # ragged column tile
+    (144, 8, 0, W.TRANSPOSED, W.MS_EDEN, 16),      # ragged row tile
+    (256, 200, 8, W.TRANSPOSED, W.SR, 128),        # padded ld, ragged columns
+    (640, 384, 0, W.TRANSPOSED, W.MS_EDEN, 128),   # 5 x 6 tiles
+    (96, 64, 0, W.TRANSPOSED, W.IF4, 32),
+    (32, 24, 0, W.TRANSPOSED, W.FOUR_OVER_SIX, 0),
+    (1024, 8, 16, W.TRANSPOSED, W.MS_EDEN, 64),
+]
+
+
+@pytest.mark.parametrize("rows,cols,ld_pad,layout,mode,g", RAGGED)
+def test_ragged_shapes(rows, cols, ld_pad, layout, mode, g):
+    gen = torch.Generator().manual_seed(rows * 1000 + cols)
+    x = (torch.randn((rows, cols), generator=gen) * 3.0).to(torch.bfloat16)
+    compare_call(x, layout, mode, g, 1234, ld_pad=ld_pad)
+
+
+@pytest.mark.parametrize("layout", [W.ROWWISE, W.TRANSPOSED])
+def test_empty_tensor(layout):
+    x = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda") if layout == W.ROWWISE else \
+        torch.zeros((64, 0), dtype=torch.bfloat16, device="cuda")
+    codes, scales, gs = N.quantize(x, layout, W.RTN, 0, 0)
+    torch.cuda.synchronize()
+    assert codes.numel() == 0 and scales.numel() == 0 and gs.item() == 1.0
+
+
+@pytest.mark.parametrize("layout", [W.ROWWISE, W.TRANSPOSED])
+@pytest.mark.parametrize("g", GROUPS)
+def test_amax_matches_oracle(layout, g):
+    x = W.gradient(rows=512, cols=384).tensors()["g"]
+    got = N.amax(x.cuda(), layout, g, 77)
+    torch.cuda.synchronize()
+    assert got.item() == oracle.amax(bits(x), layout, g, 77)
+
+
+@pytest.mark.parametrize("layout", [W.ROWWISE, W.TRANSPOSED])
+def test_prepass_equals_supplied_amax(layout):
+    x = W.gradient(rows=512, cols=384).tensors()["g"]
+    xd = x.cuda()
+    a = oracle.amax(bits(x), layout, 128, 5)
+    for mode in (W.MS_EDEN, W.SR):
+        assert_same(gpu_quantize(xd, layout, mode, 128, 5), gpu_quantize(xd, layout, mode, 128, 5, amax=a))
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("g", [0, 32, 128])
+def test_dequantize_parity(mode, g):
+    if mode == W.MS_EDEN and g == 0:
+        pytest.skip("MS-EDEN needs the rotation")
+    x = W.activation(rows=64, cols=512).tensors()["a"]
+    codes, scales, gs = oracle.quantize(bits(x), W.ROWWISE, mode, g, 9)
+    c, s = torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda()
+    gst = torch.tensor([gs], dtype=torch.float32, device="cuda")
+    for inverse in ([False, True] if g else [False]):
+        got = N.dequantize(c, s, gst, mode, g, 9, inverse_rht=inverse).cpu().numpy()
+        exp = oracle.dequantize(codes, scales, gs, mode, g, 9, inverse_rht=inverse)
+        assert np.array_equal(got.view(np.uint32), exp.view(np.uint32)), (mode, g, inverse)
+
+
+@pytest.mark.parametrize("layout", [W.ROWWISE, W.TRANSPOSED])
+@pytest.mark.parametrize("g", [16, 32, 64, 128])
+def test_rotation_parity(layout, g):
+    x = W.gradient(rows=256, cols=384).tensors()["g"]
+    got = N.rht(x.cuda(), layout, g, 31).cpu().numpy()
+    exp = oracle.rht_view(bits(x), layout, g, 31)
+    # the stated tolerance (1e-5 relative) ...
+    assert np.max(np.abs(got - exp)) <= 1e-5 * np.abs(exp).max()
+    # ... and in fact bit-exact, because the butterfly order is the oracle's
+    assert np.array_equal(got.view(np.uint32), exp.view(np.uint32))
+    # inverse on fp32 input
+    back = N.rht(torch.from_numpy(exp).cuda(), W.ROWWISE, g, 31, inverse=True).cpu().numpy()
+    exp_back = oracle.rht_rows(exp, g, 31, inverse=True)
+    assert np.array_equal(back.view(np.uint32), exp_back.view(np.uint32))
+
+
+EDGE_MODES = [(W.RTN, 0), (W.SR, 0), (W.MS_EDEN, 16), (W.IF4, 0), (W.FOUR_OVER_SIX, 0), (W.IF4, 128),
+              (W.SR, 128)]
+
+
+def _edge_tensors():
+    out = {}
+    out["zeros"] = torch.zeros((64, 256), dtype=torch.bfloat16)
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn((64, 256), generator=g)
+    x[17, 33] = 1e30  # one huge outlier: every other block lands on subnormal or zero scales
+    out["outlier"] = x.to(torch.bfloat16)
+    y = torch.ones((64, 256)) * 0.37
+    y[::2] *= -1
+    out["all_equal_blocks"] = y.to(torch.bfloat16)
+    z = torch.randn((64, 256), generator=g)
+    z[0, 0] = 3.389e38   # near the bf16 maximum
+    z[1, 1] = -3.389e38
+    out["bf16_max"] = z.to(torch.bfloat16)
+    t = torch.randn((64, 256), generator=g) * 1e-20
+    out["tiny"] = t.to(torch.bfloat16)
+    s = torch.randn((64, 256), generator=g)
+    s[:, 128:] *= 1e-4   # blocks far below the tensor max: subnormal E4M3 scales
+    out["subnormal_scales"] = s.to(torch.bfloat16)
+    return out
+
+
+@pytest.mark.parametrize("name", list(_edge_tensors().keys()))
+@pytest.mark.parametrize("mode,g", EDGE_MODES)
+@pytest.mark.parametrize("layout", [W.ROWWISE, W.TRANSPOSED])
+def test_edge_cases(name, mode, g, layout):
+    if name == "bf16_max" and g:
+        pytest.skip("rotating values near the bf16 maximum overflows binary32 (out of the input domain)")
+    x = _edge_tensors()[name]
+    compare_call(x, layout, mode, g, 2024)
+
+
+def test_exhaustive_bf16_rtn_path():
+    """Every bf16 value of magnitude <= 6 goes through the quantizer with y = z exactly.
+
+    Each block is [6, v1..v15]; amax_in = 10.5 gives s_g = 2^-8, every block scale
+    is 256 and d = 1, so the codes are the E2M1 rounding of the bf16 values."""
+    b = np.arange(1 << 16, dtype=np.uint32)
+    f = (b << 16).view(np.float32)
+    vals = f[np.isfinite(f) & (np.abs(f) <= 6.0)]
+    n = (len(vals) + 14) // 15
+    vals = np.concatenate([vals, np.zeros(n * 15 - len(vals), dtype=np.float32)]).reshape(n, 15)
+    blocks = np.concatenate([np.full((n, 1), 6.0, dtype=np.float32), vals], axis=1)
+    rows = (n + 7) // 8
+    pad = np.zeros((rows * 8 - n, 16), dtype=np.float32)
+    mat = np.concatenate([blocks, pad]).reshape(rows, 128)
+    x = torch.from_numpy(mat).to(torch.bfloat16)
+    for mode in (W.RTN, W.SR, W.IF4, W.FOUR_OVER_SIX):
+        gpu = compare_call(x, W.ROWWISE, mode, 0, 7, amax=10.5)
+        if mode == W.RTN:
+            assert gpu[2] == 2.0 ** -8
+            assert np.all(gpu[1][:n // 8] == 0x78)  # scale 256
+
+
+def _neighbourhood(centres, radius):
+    out = []
+    for c in centres:
+        base = int(np.float32(c).view(np.uint32))
+        out.append(np.arange(max(base - radius, 0), base + radius + 1, dtype=np.int64))
+    return np.unique(np.concatenate(out)).astype(np.uint32)
+
+
+def test_e2m1_conversion_near_every_boundary():
+    """The hardware E2M1 conversion agrees with the oracle's rounding on every fp32
+    within 2^15 ulps of each threshold and grid value, both signs, and on a stride
+    sweep of all finite fp32 patterns."""
+    centres = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, 1e-38]
+    pos = _neighbourhood(centres, 1 << 15)
+    sweep = np.arange(0, 1 << 32, 257, dtype=np.uint64).astype(np.uint32)
+    bits_all = np.concatenate([pos, pos | np.uint32(0x80000000), sweep, np.array([0, 0x80000000], np.uint32)])
+    v = bits_all.view(np.float32)
+    v = v[np.isfinite(v)]
+    got = N.encode_e2m1(torch.from_numpy(v).cuda()).cpu().numpy()
+    exp = oracle.e2m1_rtn_array(v)
+    bad = np.flatnonzero(got != exp)
+    assert len(bad) == 0, f"{len(bad)} differ, e.g. {v[bad[:5]]} got {got[bad[:5]]} expected {exp[bad[:5]]}"
+
+
+@pytest.mark.parametrize("round_up", [False, True])
+def test_e4m3_conversion_near_every_boundary(round_up):
+    table = np.array([oracle.e4m3_decode(c) for c in range(0x7F)], dtype=np.float64)
+    centres = list(table[1:]) + list((table[1:] + table[:-1]) / 2) + [2.0 ** -10, 464.0, 480.0]
+    pos = _neighbourhood(centres, 1 << 10)
+    sweep = np.arange(0, 0x7F800000, 131, dtype=np.uint64).astype(np.uint32)
+    v = np.concatenate([pos, sweep]).view(np.float32)
+    v = v[np.isfinite(v) & (v >= 0)]
+    got = N.encode_e4m3(torch.from_numpy(v).cuda(), round_up=round_up).cpu().numpy()
+    exp = oracle.e4m3_array(v, round_up=round_up)
+    bad = np.flatnonzero(got != exp)
+    assert len(bad) == 0, f"{len(bad)} differ, e.g. {v[bad[:5]]} got {got[bad[:5]]} expected {exp[bad[:5]]}"
+
+
+def test_determinism_and_seeds():
+    x = W.gradient(rows=256, cols=256).tensors()["g"].cuda()
+    a = gpu_quantize(x, W.ROWWISE, W.SR, 128, 1)
+    b = gpu_quantize(x, W.ROWWISE, W.SR, 128, 1)
+    c = gpu_quantize(x, W.ROWWISE, W.SR, 128, 2)
+    assert_same(a, b)
+    assert not np.array_equal(a[0], c[0])
+    e1 = gpu_quantize(x, W.TRANSPOSED, W.MS_EDEN, 128, 1)
+    e2 = gpu_quantize(x, W.TRANSPOSED, W.MS_EDEN, 128, 1 << 40)
+    assert not np.array_equal(e1[1], e2[1])
+
+
+def test_side_stream_matches_default_stream():
+    x = W.small().tensors()["x"].cuda()
+    ref = gpu_quantize(x, W.TRANSPOSED, W.MS_EDEN, 128, 3)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        codes, scales, gs = N.quantize(x, W.TRANSPOSED, W.MS_EDEN, 128, 3, stream=s)
+    s.synchronize()
+    assert_same(ref, (codes.cpu().numpy(), scales.cpu().numpy(), float(gs.item())))
