@@ -407,17 +407,16 @@ def cpu_baseline(wl, host, fraction):
                       f"({elements} elements, amax pre-pass + quantize, single-threaded C), {secs:.1f} s"}
 
 
-def run_reference(args, world, rank):
-    """The CPU oracle as the reference arm, on rank 0 only."""
+def run_reference(args, world, rank, wl=None, fraction=1.0 / 128):
+    """The CPU oracle as the reference arm, on rank 0 only (the other ranks return at once)."""
     if rank != 0:
-        return
+        return None
     from nvfp4_microscaling_quantization_b200 import workloads as W
-    wl = W.mlp_up(seed=4)
+    wl = W.mlp_up(seed=4) if wl is None else wl
     device = "cuda" if torch.cuda.is_available() else "cpu"
     full = wl.tensors(device)
     host = {k: v.cpu() for k, v in full.items()}
     del full
-    fraction = 1.0 / 128
     samples = _sample_calls(wl, host, fraction)
     for _ in range(max(args.warmup, 0)):
         time_oracle_sample(wl, samples)
@@ -427,16 +426,18 @@ def run_reference(args, world, rank):
         total_e += e
         total_s += s
     value = BYTES_PER_ELEMENT * total_e / total_s / 1e9
-    sample = (f"each step: first {fraction:.4g} of the view rows of each of the 6 mlp_up calls "
+    sample = (f"each step: first {fraction:.4g} of the view rows of each of the {wl.name} calls "
               f"({total_e // max(args.steps, 1)} elements, amax pre-pass + quantize)")
-    print(json.dumps({
+    line = json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_s * 1e3 / max(args.steps, 1), 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "mlp_up (bounded sample per step)", "input_dtype": "bf16"},
+        "config": {"workload": f"{wl.name} (bounded sample per step)", "input_dtype": "bf16"},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }), flush=True)
+    })
+    print(line, flush=True)
+    return line
 
 
 def main(argv=None):

@@ -133,21 +133,21 @@ EDGE_MODES = [(W.RTN, 0), (W.SR, 0), (W.MS_EDEN, 16), (W.IF4, 0), (W.FOUR_OVER_S
 
 def _edge_tensors():
     out = {}
-    out["zeros"] = torch.zeros((64, 256), dtype=torch.bfloat16)
+    out["zeros"] = torch.zeros((128, 256), dtype=torch.bfloat16)
     g = torch.Generator().manual_seed(3)
-    x = torch.randn((64, 256), generator=g)
+    x = torch.randn((128, 256), generator=g)
     x[17, 33] = 1e30  # one huge outlier: every other block lands on subnormal or zero scales
     out["outlier"] = x.to(torch.bfloat16)
-    y = torch.ones((64, 256)) * 0.37
+    y = torch.ones((128, 256)) * 0.37
     y[::2] *= -1
     out["all_equal_blocks"] = y.to(torch.bfloat16)
-    z = torch.randn((64, 256), generator=g)
+    z = torch.randn((128, 256), generator=g)
     z[0, 0] = 3.389e38   # near the bf16 maximum
     z[1, 1] = -3.389e38
     out["bf16_max"] = z.to(torch.bfloat16)
-    t = torch.randn((64, 256), generator=g) * 1e-20
+    t = torch.randn((128, 256), generator=g) * 1e-20
     out["tiny"] = t.to(torch.bfloat16)
-    s = torch.randn((64, 256), generator=g)
+    s = torch.randn((128, 256), generator=g)
     s[:, 128:] *= 1e-4   # blocks far below the tensor max: subnormal E4M3 scales
     out["subnormal_scales"] = s.to(torch.bfloat16)
     return out
