@@ -141,6 +141,33 @@ NVFP4_API int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, cons
 NVFP4_API int nvfp4_rht(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld, int layout,
               int rht_group, uint64_t seed, int inverse, float* out, void* stream);
 
+/* nvfp4_quantize for callers that cannot give the library any device memory
+ * beyond their tensors.  The paper has no counterpart to this entry point.
+ *
+ * nvfp4_quantize needs a workspace when it computes the tensor amax itself
+ * (amax_in == NULL).  Some callers cannot provide one: an engine plugin that
+ * is handed only its input and output buffers, or a process whose framework
+ * has reserved all device memory in its own caching pool, where a fresh
+ * cudaMalloc would fail or stall the host until the device is idle.  This
+ * variant takes the same arguments minus the workspace and uses instead a
+ * fixed 256-byte array of device memory compiled into the library (every GPU
+ * that loads the library keeps those bytes until the process exits).  It
+ * allocates nothing and calls no allocating routine.
+ *  - The first call on a device looks up that array's device address (with
+ *    the device current); make that first call before any stream capture.
+ *  - All calls on a device share the one array.  Each call clears the part
+ *    that must start at zero on its own stream, but two calls that overlap
+ *    on the GPU (different streams, or different host threads) race on it
+ *    and may produce wrong tensor scales: serialise them.
+ *  - A call whose workspace need (nvfp4_workspace_bytes) exceeds 256 bytes is
+ *    rejected with NVFP4_ERR_WORKSPACE; with amax_in supplied no scratch is
+ *    used at all.
+ * Results are identical to nvfp4_quantize's for the same arguments. */
+NVFP4_API int nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                     int layout, int mode, int rht_group, uint64_t seed,
+                                     const float* amax_in, uint8_t* codes, uint8_t* scales,
+                                     float* global_scale, void* stream);
+
 /* Element and scale codecs of the quantizer, exposed on their own.
  * nvfp4_encode_e2m1: out[i] = E2M1 code (low nibble, one code per byte) of
  * in[i] rounded to nearest, ties to the even code, saturating at +-6, zero

@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_encode_e2m1.restype = i32
         L.nvfp4_encode_e4m3.argtypes = [P, i64, i32, P, P]
         L.nvfp4_encode_e4m3.restype = i32
+        L.nvfp4_quantize_noalloc.argtypes = [P, i64, i64, i64, i32, i32, i32, u64, P, P, P, P, P]
+        L.nvfp4_quantize_noalloc.restype = i32
         L.nvfp4_status_string.argtypes = [i32]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -86,6 +88,12 @@ def nvfp4_dequantize(codes, scales, global_scale, vrows, vcols, mode, rht_group,
 
 def nvfp4_rht(x, in_dtype, rows, cols, ld, layout, rht_group, seed, inverse, out, stream) -> int:
     return lib().nvfp4_rht(x, in_dtype, rows, cols, ld, layout, rht_group, seed, inverse, out, stream)
+
+
+def nvfp4_quantize_noalloc(x, rows, cols, ld, layout, mode, rht_group, seed, amax_in, codes, scales,
+                           global_scale, stream) -> int:
+    return lib().nvfp4_quantize_noalloc(x, rows, cols, ld, layout, mode, rht_group, seed, amax_in, codes,
+                                        scales, global_scale, stream)
 
 
 def nvfp4_encode_e2m1(x, n, out, stream) -> int:

@@ -33,7 +33,7 @@ def declared_symbols():
 def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ["nvfp4_quantize", "nvfp4_dequantize", "nvfp4_rht", "nvfp4_amax", "nvfp4_workspace_bytes",
-              "nvfp4_status_string", "nvfp4_encode_e2m1", "nvfp4_encode_e4m3"]:
+              "nvfp4_status_string", "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_quantize_noalloc"]:
         assert n in names
 
 
@@ -94,6 +94,13 @@ def test_quantize_rejects(N):
     assert q(N) == WORKSPACE                        # no amax_in and no workspace
     assert q(N, ws=FAKE + 0x4000, ws_bytes=8) == WORKSPACE
     assert q(N, ws=FAKE + 0x4008, ws_bytes=256) == ALIGN
+
+
+def test_noalloc_rejects_like_quantize(N):
+    nq = N.nvfp4_quantize_noalloc
+    assert nq(FAKE, 64, 64, 64, 2, 0, 0, 0, None, FAKE, FAKE, FAKE, None) == INVALID   # layout
+    assert nq(FAKE, 64, 64, 64, 0, 0, 48, 0, None, FAKE, FAKE, FAKE, None) == INVALID  # group
+    assert nq(FAKE, 64, 64, 64, 0, 9, 0, 0, None, FAKE, FAKE, FAKE, None) == INVALID   # mode
 
 
 def test_other_entry_points_reject(N):
