@@ -48,6 +48,13 @@ struct RhtArgs {
 
 cudaError_t launch_amax(const QuantArgs& a);
 cudaError_t launch_quantize(const QuantArgs& a);
+
+// The TMA-tiled kernels (quantize_tma.cu) take every shape they can tile;
+// launch_amax / launch_quantize route there and fall back to the one-block-
+// per-thread kernels for the rest (narrow or short tensors).
+bool tma_path_applies(const QuantArgs& a);
+cudaError_t launch_amax_tma(const QuantArgs& a);
+cudaError_t launch_quantize_tma(const QuantArgs& a);
 cudaError_t launch_dequantize(const DequantArgs& a);
 cudaError_t launch_rht(const RhtArgs& a);
 cudaError_t launch_encode_e2m1(const float* in, int64_t n, uint8_t* out, cudaStream_t stream);

@@ -9,6 +9,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace nvfp4 {
 
@@ -134,8 +135,9 @@ __device__ __forceinline__ uint32_t e4m3_sr(float t, float U) {
   if (e4m3_decode(lo) > t) --lo;
   const float l = e4m3_decode(lo);
   const float h = e4m3_decode(lo + 1);
-  const float f = __fdiv_rn(__fsub_rn(t, l), __fsub_rn(h, l));
-  return U < f ? lo + 1 : lo;
+  // U < (t - l) / (h - l)  <=>  U * (h - l) < t - l: h - l is a power of two, so
+  // both products and the difference are exact and the comparison is the same.
+  return __fmul_rn(U, __fsub_rn(h, l)) < __fsub_rn(t, l) ? lo + 1 : lo;
 }
 
 // bf16 pair (one 32-bit word) -> two floats.
@@ -380,6 +382,233 @@ __device__ __forceinline__ BlockOut quantize_block(const float* z, float s_g, co
       }
     }
     return out;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Two blocks at once.  The tiled kernels hold their data as float2 pairs whose
+// .x and .y belong to two different 16-element blocks (two blocks of a row, or
+// the same rows of two columns), so every per-element step of two blocks is
+// one packed f32x2 instruction.  Each lane of a packed operation is one
+// binary32 RN operation, so the per-block results, including the sequential
+// per-block dot products, are exactly those of quantize_block.
+struct PairRng {
+  PhiloxKey key;
+  uint64_t elem_a, elem_b;  // view index of element 0 of block a / b (multiples of 16)
+  float u_a, u_b;           // scale uniforms of block a / b (MS-EDEN)
+};
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// a - b per lane: the negation is exact, so each lane is the one RN subtraction.
+__device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) { return __fadd2_rn(a, f2(-b.x, -b.y)); }
+
+// E4M3 RNE of two non-negative floats in one conversion: .x -> bits 0..7, .y -> bits 8..15.
+__device__ __forceinline__ uint32_t e4m3x2_rne_sat(float a, float b) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(b), "f"(a));
+  return out;
+}
+
+// Two E4M3 codes (bits 0..7 and 8..15, each < 0x7F) -> two floats.
+__device__ __forceinline__ float2 e4m3x2_decode(uint32_t codes) {
+  uint32_t h2;
+  const uint16_t in = static_cast<uint16_t>(codes & 0x7F7Fu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  const __half2 p = *reinterpret_cast<const __half2*>(&h2);
+  return f2(__low2float(p), __high2float(p));
+}
+
+// Stochastic rounding of one block of 16 scaled values; elem = view index of element 0.
+__device__ __forceinline__ void sr_block(const float (&y)[16], PhiloxKey key, uint64_t elem, uint32_t& lo,
+                                         uint32_t& hi) {
+  const uint64_t call0 = elem >> 3;
+  const uint4 w0 = philox_call(key, call0, kTagElement);
+  const uint4 w1 = philox_call(key, call0 + 1, kTagElement);
+  lo = 0u;
+  hi = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t k0 = (word_of(w0, i >> 1) >> ((i & 1) * 16)) & 0xFFFFu;
+    const uint32_t k1 = (word_of(w1, i >> 1) >> ((i & 1) * 16)) & 0xFFFFu;
+    lo |= sr_code(y[i], k0) << (4 * i);
+    hi |= sr_code(y[8 + i], k1) << (4 * i);
+  }
+}
+
+// max |z| of each of the two blocks of a pair, as a tree (exact in any order).
+__device__ __forceinline__ void absmax_pair(const float2 (&z)[16], float& aa, float& ab) {
+  float ma[8], mb[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    ma[i] = fmaxf(fabsf(z[2 * i].x), fabsf(z[2 * i + 1].x));
+    mb[i] = fmaxf(fabsf(z[2 * i].y), fabsf(z[2 * i + 1].y));
+  }
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      ma[i] = fmaxf(ma[i], ma[i + w]);
+      mb[i] = fmaxf(mb[i], mb[i + w]);
+    }
+  aa = ma[0];
+  ab = mb[0];
+}
+
+template <int MODE>
+__device__ __forceinline__ void quantize_pair(const float2 (&z)[16], float s_g, float q6, float q4,
+                                              const PairRng& rng, BlockOut& oa, BlockOut& ob) {
+  float aa, ab;
+  absmax_pair(z, aa, ab);
+  const float2 sg2 = f2(s_g, s_g);
+
+  if constexpr (MODE == k4over6) {
+    uint32_t S[2], ca_lo[2], ca_hi[2], cb_lo[2], cb_hi[2];
+    float2 err[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float q = k == 0 ? q6 : q4;
+      S[k] = e4m3x2_rne_sat(__fdiv_rn(aa, q), __fdiv_rn(ab, q));
+      const float2 d = __fmul2_rn(e4m3x2_decode(S[k]), sg2);
+      const float2 r = f2(d.x != 0.0f ? __frcp_rn(d.x) : 0.0f, d.y != 0.0f ? __frcp_rn(d.y) : 0.0f);
+      float ya[16], yb[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 y = __fmul2_rn(z[i], r);
+        ya[i] = y.x;
+        yb[i] = y.y;
+      }
+      rtn_codes(ya, ca_lo[k], ca_hi[k]);
+      rtn_codes(yb, cb_lo[k], cb_hi[k]);
+      float va[16], vb[16];
+      e2m1x8_to_f32(ca_lo[k], va);
+      e2m1x8_to_f32(ca_hi[k], va + 8);
+      e2m1x8_to_f32(cb_lo[k], vb);
+      e2m1x8_to_f32(cb_hi[k], vb + 8);
+      float2 e = f2(0.0f, 0.0f);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 diff = sub2_rn(z[i], __fmul2_rn(f2(va[i], vb[i]), d));
+        e = __ffma2_rn(diff, diff, e);
+      }
+      err[k] = e;
+    }
+    const bool pa = err[1].x < err[0].x, pb = err[1].y < err[0].y;
+    oa.lo = pa ? ca_lo[1] : ca_lo[0];
+    oa.hi = pa ? ca_hi[1] : ca_hi[0];
+    oa.scale = (pa ? S[1] : S[0]) & 0xFFu;
+    ob.lo = pb ? cb_lo[1] : cb_lo[0];
+    ob.hi = pb ? cb_hi[1] : cb_hi[0];
+    ob.scale = ((pb ? S[1] : S[0]) >> 8) & 0xFFu;
+    return;
+  } else {
+    uint32_t S2 = e4m3x2_rne_sat(__fdiv_rn(aa, q6), __fdiv_rn(ab, q6));
+    uint32_t Sa = S2 & 0xFFu, Sb = S2 >> 8;
+    float2 dS = e4m3x2_decode(S2);
+    if constexpr (MODE == kSR) {
+      const float sfa = __fdiv_rn(aa, q6), sfb = __fdiv_rn(ab, q6);
+      if (Sa < 0x7Eu && dS.x < sfa) ++Sa;
+      if (Sb < 0x7Eu && dS.y < sfb) ++Sb;
+      S2 = Sa | (Sb << 8);
+      dS = e4m3x2_decode(S2);
+    }
+    oa.scale = Sa;
+    ob.scale = Sb;
+    const float2 d = __fmul2_rn(dS, sg2);
+    const float2 r = f2(d.x != 0.0f ? __frcp_rn(d.x) : 0.0f, d.y != 0.0f ? __frcp_rn(d.y) : 0.0f);
+    float ya[16], yb[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 y = __fmul2_rn(z[i], r);
+      ya[i] = y.x;
+      yb[i] = y.y;
+    }
+    if constexpr (MODE == kRTN) {
+      rtn_codes(ya, oa.lo, oa.hi);
+      rtn_codes(yb, ob.lo, ob.hi);
+    } else if constexpr (MODE == kSR) {
+      sr_block(ya, rng.key, rng.elem_a, oa.lo, oa.hi);
+      sr_block(yb, rng.key, rng.elem_b, ob.lo, ob.hi);
+    } else if constexpr (MODE == kMSEDEN) {
+      rtn_codes(ya, oa.lo, oa.hi);
+      rtn_codes(yb, ob.lo, ob.hi);
+      float va[16], vb[16];
+      e2m1x8_to_f32(oa.lo, va);
+      e2m1x8_to_f32(oa.hi, va + 8);
+      e2m1x8_to_f32(ob.lo, vb);
+      e2m1x8_to_f32(ob.hi, vb + 8);
+      float2 num = f2(0.0f, 0.0f), den = f2(0.0f, 0.0f);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 y = f2(ya[i], yb[i]);
+        num = __ffma2_rn(y, y, num);
+        den = __ffma2_rn(y, f2(va[i], vb[i]), den);
+      }
+      const float ca = (num.x > 0.0f && den.x > 0.0f) ? __fdiv_rn(num.x, den.x) : 1.0f;
+      const float cb = (num.y > 0.0f && den.y > 0.0f) ? __fdiv_rn(num.y, den.y) : 1.0f;
+      const float2 t = __fmul2_rn(dS, f2(ca, cb));
+      oa.scale = e4m3_sr(t.x, rng.u_a);
+      ob.scale = e4m3_sr(t.y, rng.u_b);
+    } else {  // kIF4
+      uint32_t fa_lo, fa_hi, fb_lo, fb_hi;
+      rtn_codes(ya, fa_lo, fa_hi);
+      rtn_codes(yb, fb_lo, fb_hi);
+      float va[16], vb[16];
+      e2m1x8_to_f32(fa_lo, va);
+      e2m1x8_to_f32(fa_hi, va + 8);
+      e2m1x8_to_f32(fb_lo, vb);
+      e2m1x8_to_f32(fb_hi, vb + 8);
+      float2 eF = f2(0.0f, 0.0f), eI = f2(0.0f, 0.0f);
+      uint32_t ia_lo = 0u, ia_hi = 0u, ib_lo = 0u, ib_hi = 0u;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 y = f2(ya[i], yb[i]);
+        const float2 dF = sub2_rn(y, f2(va[i], vb[i]));
+        eF = __ffma2_rn(dF, dF, eF);
+        const float2 t = __fmul2_rn(y, f2(kIF4K1, kIF4K1));
+        const int ka = max(-7, min(7, __float2int_rn(t.x)));
+        const int kb = max(-7, min(7, __float2int_rn(t.y)));
+        const float2 vi = __fmul2_rn(f2(static_cast<float>(ka), static_cast<float>(kb)), f2(kIF4K2, kIF4K2));
+        const float2 dI = sub2_rn(y, vi);
+        eI = __ffma2_rn(dI, dI, eI);
+        const uint32_t codea = ka == 0 ? 0u : (static_cast<uint32_t>(ka < 0 ? -ka : ka) | (ka < 0 ? 8u : 0u));
+        const uint32_t codeb = kb == 0 ? 0u : (static_cast<uint32_t>(kb < 0 ? -kb : kb) | (kb < 0 ? 8u : 0u));
+        if (i < 8) {
+          ia_lo |= codea << (4 * i);
+          ib_lo |= codeb << (4 * i);
+        } else {
+          ia_hi |= codea << (4 * (i - 8));
+          ib_hi |= codeb << (4 * (i - 8));
+        }
+      }
+      const bool inta = eI.x < eF.x, intb = eI.y < eF.y;
+      oa.lo = inta ? ia_lo : fa_lo;
+      oa.hi = inta ? ia_hi : fa_hi;
+      ob.lo = intb ? ib_lo : fb_lo;
+      ob.hi = intb ? ib_hi : fb_hi;
+      if (inta) oa.scale |= 0x80u;
+      if (intb) ob.scale |= 0x80u;
+    }
+  }
+}
+
+// Scale uniforms of four consecutive view blocks b0..b0+3 (MS-EDEN): one
+// Philox call when b0 is a multiple of 4, two otherwise.
+__device__ __forceinline__ void block_uniforms4(PhiloxKey key, uint64_t b0, float (&u)[4]) {
+  const uint4 w0 = philox_call(key, b0 >> 2, kTagBlock);
+  if ((b0 & 3u) == 0) {
+    u[0] = __fmul_rn(static_cast<float>(w0.x >> 8), 0x1p-24f);
+    u[1] = __fmul_rn(static_cast<float>(w0.y >> 8), 0x1p-24f);
+    u[2] = __fmul_rn(static_cast<float>(w0.z >> 8), 0x1p-24f);
+    u[3] = __fmul_rn(static_cast<float>(w0.w >> 8), 0x1p-24f);
+  } else {
+    const uint4 w1 = philox_call(key, (b0 >> 2) + 1, kTagBlock);
+#pragma unroll
+    for (uint32_t k = 0; k < 4; ++k) {
+      const uint64_t b = b0 + k;
+      const uint32_t word = (b >> 2) == (b0 >> 2) ? word_of(w0, b & 3u) : word_of(w1, b & 3u);
+      u[k] = __fmul_rn(static_cast<float>(word >> 8), 0x1p-24f);
+    }
   }
 }
 

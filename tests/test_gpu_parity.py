@@ -59,6 +59,18 @@ RAGGED = [
     (96, 64, 0, W.TRANSPOSED, W.IF4, 32),
     (32, 24, 0, W.TRANSPOSED, W.FOUR_OVER_SIX, 0),
     (1024, 8, 16, W.TRANSPOSED, W.MS_EDEN, 64),
+    # shapes the tiled (TMA) kernels take, with partial row and column tiles
+    (40, 176, 8, W.ROWWISE, W.RTN, 16),
+    (40, 176, 8, W.ROWWISE, W.MS_EDEN, 16),        # odd blocks per row: scale uniforms straddle calls
+    (16, 80, 0, W.ROWWISE, W.SR, 16),
+    (19, 96, 0, W.ROWWISE, W.FOUR_OVER_SIX, 32),
+    (33, 1536, 0, W.ROWWISE, W.IF4, 128),
+    (176, 136, 0, W.TRANSPOSED, W.RTN, 16),
+    (208, 72, 8, W.TRANSPOSED, W.IF4, 0),          # odd scale pitch: byte stores
+    (208, 72, 8, W.TRANSPOSED, W.MS_EDEN, 16),
+    (384, 192, 0, W.TRANSPOSED, W.SR, 64),
+    (256, 64, 0, W.TRANSPOSED, W.FOUR_OVER_SIX, 128),
+    (1280, 640, 0, W.TRANSPOSED, W.MS_EDEN, 128),
 ]
 
 
@@ -243,3 +255,28 @@ def test_side_stream_matches_default_stream():
         codes, scales, gs = N.quantize(x, W.TRANSPOSED, W.MS_EDEN, 128, 3, stream=s)
     s.synchronize()
     assert_same(ref, (codes.cpu().numpy(), scales.cpu().numpy(), float(gs.item())))
+
+
+@pytest.mark.parametrize("layout,mode,g", [(W.ROWWISE, W.MS_EDEN, 128), (W.TRANSPOSED, W.SR, 32),
+                                           (W.ROWWISE, W.RTN, 0), (W.TRANSPOSED, W.FOUR_OVER_SIX, 0)])
+def test_outputs_at_8_byte_offsets(layout, mode, g):
+    """Code and scale buffers that are only 8- (codes) or 1-byte (scales) aligned, as the ABI allows."""
+    import ctypes
+    x = W.gradient(rows=256, cols=512).tensors()["g"]
+    xd = x.cuda()
+    rows, cols = x.shape
+    vr, vc = N.view_shape(rows, cols, layout)
+    cbuf = torch.zeros(vr * vc // 2 + 64, dtype=torch.uint8, device="cuda")
+    sbuf = torch.zeros(vr * vc // 16 + 64, dtype=torch.uint8, device="cuda")
+    gs = torch.zeros(1, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    P = ctypes.c_void_p
+    st = N.nvfp4_quantize(P(xd.data_ptr()), rows, cols, cols, layout, mode, g, 21, None,
+                          P(cbuf.data_ptr() + 8), P(sbuf.data_ptr() + 1), P(gs.data_ptr()), P(ws.data_ptr()), 256,
+                          P(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    got_c = cbuf[8:8 + vr * vc // 2].cpu().numpy().reshape(vr, vc // 2)
+    got_s = sbuf[1:1 + vr * vc // 16].cpu().numpy().reshape(vr, vc // 16)
+    oc, osc, og = oracle.quantize(bits(x), layout, mode, g, 21)
+    assert_same((got_c, got_s, float(gs.item())), (oc, osc, og))
