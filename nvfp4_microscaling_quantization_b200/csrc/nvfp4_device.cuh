@@ -128,11 +128,12 @@ __device__ __forceinline__ uint32_t e4m3_ru_sat(float v) {
 // Stochastic rounding of t >= 0 onto E4M3 with a uniform U in [0, 1):
 // neighbours lo <= t < hi, hi with probability (t - lo) / (hi - lo); t >= 448
 // gives 448.  (t - lo) and the division by the power-of-two gap are exact.
+// Written without branches: for t >= 448 the RNE code is 0x7E and the code
+// above it (0x7F) decodes to NaN, so the comparison fails and 0x7E stays; for
+// t = 0 the code is 0 and nothing rounds up.
 __device__ __forceinline__ uint32_t e4m3_sr(float t, float U) {
-  if (!(t > 0.0f)) return 0u;
-  if (t >= 448.0f) return 0x7Eu;
   uint32_t lo = e4m3_rne_sat(t);
-  if (e4m3_decode(lo) > t) --lo;
+  lo = e4m3_decode(lo) > t ? lo - 1 : lo;
   const float l = e4m3_decode(lo);
   const float h = e4m3_decode(lo + 1);
   // U < (t - l) / (h - l)  <=>  U * (h - l) < t - l: h - l is a power of two, so
@@ -455,6 +456,13 @@ __device__ __forceinline__ void absmax_pair(const float2 (&z)[16], float& aa, fl
   ab = mb[0];
 }
 
+// RN(1/d) per lane, 0 for a zero scale (a zero block): computed unconditionally
+// and selected, so the reciprocal sits on no branch.
+__device__ __forceinline__ float2 rcp_or_zero(float2 d) {
+  const float ra = __frcp_rn(d.x), rb = __frcp_rn(d.y);
+  return f2(d.x != 0.0f ? ra : 0.0f, d.y != 0.0f ? rb : 0.0f);
+}
+
 template <int MODE>
 __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], float s_g, float q6, float q4,
                                               const PairRng& rng, BlockOut& oa, BlockOut& ob) {
@@ -470,7 +478,7 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], float s_g, 
       const float q = k == 0 ? q6 : q4;
       S[k] = e4m3x2_rne_sat(__fdiv_rn(aa, q), __fdiv_rn(ab, q));
       const float2 d = __fmul2_rn(e4m3x2_decode(S[k]), sg2);
-      const float2 r = f2(d.x != 0.0f ? __frcp_rn(d.x) : 0.0f, d.y != 0.0f ? __frcp_rn(d.y) : 0.0f);
+      const float2 r = rcp_or_zero(d);
       float ya[16], yb[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -515,7 +523,7 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], float s_g, 
     oa.scale = Sa;
     ob.scale = Sb;
     const float2 d = __fmul2_rn(dS, sg2);
-    const float2 r = f2(d.x != 0.0f ? __frcp_rn(d.x) : 0.0f, d.y != 0.0f ? __frcp_rn(d.y) : 0.0f);
+    const float2 r = rcp_or_zero(d);
     float ya[16], yb[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -544,8 +552,9 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], float s_g, 
         num = __ffma2_rn(y, y, num);
         den = __ffma2_rn(y, f2(va[i], vb[i]), den);
       }
-      const float ca = (num.x > 0.0f && den.x > 0.0f) ? __fdiv_rn(num.x, den.x) : 1.0f;
-      const float cb = (num.y > 0.0f && den.y > 0.0f) ? __fdiv_rn(num.y, den.y) : 1.0f;
+      const float qa = __fdiv_rn(num.x, den.x), qb = __fdiv_rn(num.y, den.y);
+      const float ca = (num.x > 0.0f && den.x > 0.0f) ? qa : 1.0f;
+      const float cb = (num.y > 0.0f && den.y > 0.0f) ? qb : 1.0f;
       const float2 t = __fmul2_rn(dS, f2(ca, cb));
       oa.scale = e4m3_sr(t.x, rng.u_a);
       ob.scale = e4m3_sr(t.y, rng.u_b);

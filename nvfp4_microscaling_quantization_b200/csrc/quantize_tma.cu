@@ -2,10 +2,11 @@
 //
 // A persistent CTA of 128 threads streams tiles of X through a ring of
 // shared-memory stages filled by TMA (cp.async.bulk.tensor 2-D, 128-byte
-// swizzle, no multicast).  Thread 0 keeps the ring full: it refills the stage
-// every thread released on the previous iteration (its "empty" mbarrier
-// counts the 128 releases) and arms the stage's "full" mbarrier with the
-// tile's byte count.  Every thread owns 64 elements = four 16-element blocks
+// swizzle, no multicast).  Each warp releases a stage once it has read its
+// part (one arrival on the stage's "empty" mbarrier) and takes a ticket; the
+// warp that takes the last ticket refills the stage with the CTA's tile that
+// many stages ahead and arms the stage's "full" mbarrier with the tile's byte
+// count, so no thread ever waits to refill.  Every thread owns 64 elements = four 16-element blocks
 // of one view row, held as two float2[16] pairs (block 0 | block 1, block 2 |
 // block 3), so each per-element step of two blocks is one packed f32x2
 // instruction.
@@ -30,8 +31,16 @@ namespace nvfp4 {
 
 namespace {
 
-constexpr int kNT = 128;         // threads per CTA
-constexpr int kStages = 3;       // ring depth
+#ifndef NVFP4_TMA_STAGES
+#define NVFP4_TMA_STAGES 3
+#endif
+#ifndef NVFP4_TMA_MIN_BLOCKS
+#define NVFP4_TMA_MIN_BLOCKS 4
+#endif
+
+constexpr int kNT = 128;                   // threads per CTA
+constexpr int kStages = NVFP4_TMA_STAGES;  // ring depth
+constexpr int kMinBlocks = NVFP4_TMA_MIN_BLOCKS;
 constexpr uint32_t kStageBytes = 16384;
 
 // row-wise: 8 boxes of 16 rows x 64 columns
@@ -48,16 +57,40 @@ __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
 }
 
 // ---------------------------------------------------------------- the ring
+constexpr int kWarps = kNT / 32;
+
 struct Ring {
   uint64_t full[kStages];
   uint64_t empty[kStages];
+  unsigned int tickets[kStages];
+  unsigned int issued_mask;   // stages that ever received a load
+  unsigned int last_parity;   // bit s: phase parity of the last load issued into stage s
   int abort_flag;
 };
 
+// (tile row, tile column) of the tiles a CTA visits: blockIdx.x, then every
+// gridDim.x-th tile, advanced without a division per step.
+struct TileCursor {
+  int64_t t, rt, ct;
+  __device__ __forceinline__ void start(int64_t t0, int64_t n_ct) {
+    t = t0;
+    rt = t0 / n_ct;
+    ct = t0 - rt * n_ct;
+  }
+  __device__ __forceinline__ void advance(int64_t step, int64_t drt, int64_t dct, int64_t n_ct) {
+    t += step;
+    rt += drt;
+    ct += dct;
+    if (ct >= n_ct) {
+      ct -= n_ct;
+      ++rt;
+    }
+  }
+};
+
 template <bool ROWWISE>
-__device__ __forceinline__ void issue_tile(const CUtensorMap* map, uint8_t* stage, uint64_t* full, int64_t t,
-                                           int64_t n_ct) {
-  const int64_t rt = t / n_ct, ct = t - rt * n_ct;
+__device__ __forceinline__ void issue_tile(const CUtensorMap* map, uint8_t* stage, uint64_t* full, int64_t rt,
+                                           int64_t ct) {
   mbar_arrive_expect_tx(full, kStageBytes);
   if constexpr (ROWWISE) {
     const int32_t x = static_cast<int32_t>(ct * kRowTileCols), y = static_cast<int32_t>(rt * kRowBoxRows);
@@ -177,7 +210,7 @@ __device__ __forceinline__ void quantize_store64(const float2 (&z)[2][16], const
 
 // -------------------------------------------------------------- the kernel
 template <int MODE, int G, bool AMAX_ONLY, bool ROWWISE>
-__global__ void __launch_bounds__(kNT)
+__global__ void __launch_bounds__(kNT, kMinBlocks)
 quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed,
                     const float* __restrict__ amax, unsigned int* __restrict__ amax_accum,
                     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, float* __restrict__ gscale) {
@@ -195,8 +228,11 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&ring.full[s], 1);
-      mbar_init(&ring.empty[s], kNT);
+      mbar_init(&ring.empty[s], kWarps);
+      ring.tickets[s] = 0;
     }
+    ring.issued_mask = 0;
+    ring.last_parity = 0;
     ring.abort_flag = 0;
     fence_barrier_init();
   }
@@ -212,12 +248,21 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
     }
   }
   __syncthreads();
+  const int64_t step = gridDim.x, drt = step / n_ct, dct = step - drt * n_ct;
+  // load the CTA's k-th tile (sequence index) into stage k mod kStages
+  auto load = [&](int64_t kseq) {
+    const int64_t tn = blockIdx.x + kseq * step;
+    if (tn >= n_tiles) return;
+    const int st = static_cast<int>(kseq % kStages);
+    const int64_t rt = tn / n_ct;
+    issue_tile<ROWWISE>(&tmap, stages + st * kStageBytes, &ring.full[st], rt, tn - rt * n_ct);
+    atomicOr(&ring.issued_mask, 1u << st);
+    if ((kseq / kStages) & 1) atomicOr(&ring.last_parity, 1u << st);
+    else atomicAnd(&ring.last_parity, ~(1u << st));
+  };
   if (tid == 0) {
     prefetch_tensormap(&tmap);
-    for (int k = 0; k < kStages; ++k) {
-      const int64_t t = blockIdx.x + int64_t(k) * gridDim.x;
-      if (t < n_tiles) issue_tile<ROWWISE>(&tmap, stages + k * kStageBytes, &ring.full[k], t, n_ct);
-    }
+    for (int k = 0; k < kStages; ++k) load(k);
   }
 
   ScaleCtx sc{1.0f, 0.0f, 0.0f};
@@ -235,23 +280,27 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
   const bool codes_aligned16 = ((vcols / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes) % 16) == 0;
   const bool scales_aligned4 = ((vcols / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales) % 4) == 0;
   float local_max = 0.0f;
-  int64_t issued_upto = kStages;  // tiles k < issued_upto have been issued (or do not exist)
-
-  int k = 0;
-  for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++k) {
-    const int s = k % kStages;
-    // thread 0 refills the stage released on the previous iteration
-    if (tid == 0 && k >= 1) {
-      const int sp = (k - 1) % kStages;
-      const int64_t tn = blockIdx.x + int64_t(k - 1 + kStages) * gridDim.x;
-      if (tn < n_tiles) {
-        if (mbar_wait(&ring.empty[sp], ((k - 1) / kStages) & 1u))
-          issue_tile<ROWWISE>(&tmap, stages + sp * kStageBytes, &ring.full[sp], tn, n_ct);
-        else
-          atomicExch(&ring.abort_flag, 1);
-        issued_upto = k - 1 + kStages + 1;
+  const uint32_t lane = tid & 31u;
+  // A warp is done with stage s: release it, and refill it if it was the last.
+  auto release = [&](int s, int k) {
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&ring.empty[s]);
+      if (atomicAdd(&ring.tickets[s], 1u) == kWarps - 1) {
+        atomicExch(&ring.tickets[s], 0u);
+        if (blockIdx.x + int64_t(k + kStages) * step < n_tiles) {
+          if (mbar_wait(&ring.empty[s], (k / kStages) & 1u)) load(k + kStages);
+          else atomicExch(&ring.abort_flag, 1);
+        }
       }
     }
+  };
+
+  TileCursor cur;
+  cur.start(blockIdx.x, n_ct);
+  int k = 0;
+  for (; cur.t < n_tiles; cur.advance(step, drt, dct, n_ct), ++k) {
+    const int s = k % kStages;
     if (!mbar_wait(&ring.full[s], (k / kStages) & 1u)) {
       atomicExch(&ring.abort_flag, 1);
       break;
@@ -263,7 +312,7 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
       uint4 ch[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) ch[c] = *reinterpret_cast<const uint4*>(rowp + swizzle128(j * 128u + c * 16u));
-      mbar_arrive(&ring.empty[s]);
+      release(s, k);
       const uint32_t* masks = sign_tab + 32 * (piece & 1u);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -290,7 +339,7 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
 #pragma unroll
       for (int e = 0; e < 64; ++e)
         v[e] = *reinterpret_cast<const uint16_t*>(colp + e * 128u + ((((col >> 3) ^ (e & 7)) & 7u) << 4));
-      mbar_arrive(&ring.empty[s]);
+      release(s, k);
       const uint32_t* masks = sign_tab + 64 * half;
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
@@ -309,7 +358,7 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
 
     if constexpr (G > 0) rotate64<G>(z, upper_half);
 
-    const int64_t rt = t / n_ct, ct = t - rt * n_ct;
+    const int64_t rt = cur.rt, ct = cur.ct;
     if constexpr (AMAX_ONLY) {
       local_max = fmaxf(local_max, absmax64(z));
     } else if constexpr (ROWWISE) {
@@ -323,18 +372,16 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
     }
   }
 
-  // After a failed wait: let every load still in flight land before the CTA exits.
-  if (tid == 0 && *reinterpret_cast<volatile int*>(&ring.abort_flag)) {
-    for (int64_t kk = k; kk < issued_upto; ++kk) {
-      const int64_t tt = blockIdx.x + kk * gridDim.x;
-      if (tt < n_tiles) mbar_wait(&ring.full[kk % kStages], (kk / kStages) & 1u);
-    }
-  }
   if constexpr (AMAX_ONLY) {
     const unsigned int bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(local_max));
     if ((tid & 31u) == 0) warp_max[tid >> 5] = bits;
   }
   __syncthreads();
+  // After a failed wait: let every load still in flight land before the CTA exits.
+  if (tid == 0 && *reinterpret_cast<volatile int*>(&ring.abort_flag)) {
+    for (int st = 0; st < kStages; ++st)
+      if ((ring.issued_mask >> st) & 1u) mbar_wait(&ring.full[st], (ring.last_parity >> st) & 1u);
+  }
   if (tid == 0) {
     const bool failed = *reinterpret_cast<volatile int*>(&ring.abort_flag) != 0;
     if constexpr (AMAX_ONLY) {

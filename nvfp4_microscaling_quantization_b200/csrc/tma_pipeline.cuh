@@ -2,11 +2,14 @@
 // TMA tile loads (cp.async.bulk.tensor, no multicast) completing on mbarriers,
 // consumer release through a second mbarrier per stage, and bounded waits.
 //
-// Every wait polls at most kMaxPolls times.  A wait that runs out (which only
-// a broken device or driver could cause) raises the CTA's abort flag; the
-// kernel then stops issuing loads, waits (again bounded) for the loads it has
-// in flight, reports the failure through a NaN in its scalar output and
-// returns, so the context stays usable.
+// Every wait is bounded: after one plain poll it sleeps on the barrier in
+// slices of at most kSuspendNs nanoseconds (the thread wakes as soon as the
+// phase completes) until kWaitLimitNs of wall time (%globaltimer) have passed.
+// A wait
+// that runs out (which only a broken device or driver could cause) raises the
+// CTA's abort flag; the kernel then stops issuing loads, waits (again bounded)
+// for the loads it has in flight, reports the failure through a NaN in its
+// scalar output and returns, so the context stays usable.
 #pragma once
 
 #include <cstdint>
@@ -14,7 +17,14 @@
 
 namespace nvfp4 {
 
-constexpr uint32_t kMaxPolls = 1u << 24;
+constexpr uint32_t kSuspendNs = 1u << 16;            // ~65 us per sleep
+constexpr uint64_t kWaitLimitNs = 2000000000ull;     // 2 s in all
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -49,11 +59,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-// Wait for the phase with the given parity to complete; false after kMaxPolls polls.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+      : "memory");
+  return done != 0;
+}
+
+// Wait for the phase with the given parity to complete; false if it has not
+// completed within kWaitLimitNs.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
+  const uint64_t start = global_timer_ns();
+  do {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+  } while (global_timer_ns() - start < kWaitLimitNs);
+  return mbar_try_wait(bar, parity);
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kMaxPolls; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity);
 }
 
 // 2-D tiled TMA load of one box into shared memory; x is the innermost
