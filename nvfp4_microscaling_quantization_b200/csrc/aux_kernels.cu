@@ -171,6 +171,13 @@ cudaError_t launch_encode_e4m3(const float* in, int64_t n, int round_up, uint8_t
 }
 
 cudaError_t launch_rht(const RhtArgs& a) {
+  if (!a.inverse && a.in_dtype == 0) {
+    // the forward rotation of a bf16 tensor is the quantizer's own: on the
+    // tensor cores whenever the quantizer would use them
+    QuantArgs q{a.in, a.rows, a.cols, a.ld, a.layout, kRTN, a.rht_group, a.seed, nullptr, nullptr,
+                nullptr, nullptr, nullptr, a.stream};
+    if (mma_path_applies(q)) return launch_rotate_mma(q, a.out);
+  }
   switch (a.rht_group * 2 + (a.inverse ? 1 : 0)) {
     case 32: return rht_one<16, false>(a);
     case 33: return rht_one<16, true>(a);

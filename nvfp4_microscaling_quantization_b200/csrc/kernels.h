@@ -55,6 +55,14 @@ cudaError_t launch_quantize(const QuantArgs& a);
 bool tma_path_applies(const QuantArgs& a);
 cudaError_t launch_amax_tma(const QuantArgs& a);
 cudaError_t launch_quantize_tma(const QuantArgs& a);
+
+// With a rotation (g > 0) and both dimensions at least 128, the rotation runs
+// on the tensor cores (rotate_mma.cu); launch_rotate_mma writes the rotated
+// view as dense fp32 (the forward nvfp4_rht of a bf16 tensor).
+bool mma_path_applies(const QuantArgs& a);
+cudaError_t launch_amax_mma(const QuantArgs& a);
+cudaError_t launch_quantize_mma(const QuantArgs& a);
+cudaError_t launch_rotate_mma(const QuantArgs& a, float* zout);
 cudaError_t launch_dequantize(const DequantArgs& a);
 cudaError_t launch_rht(const RhtArgs& a);
 cudaError_t launch_encode_e2m1(const float* in, int64_t n, uint8_t* out, cudaStream_t stream);

@@ -239,11 +239,13 @@ cudaError_t dispatch_group(const QuantArgs& a) {
 }  // namespace
 
 cudaError_t launch_amax(const QuantArgs& a) {
+  if (mma_path_applies(a)) return launch_amax_mma(a);
   if (tma_path_applies(a)) return launch_amax_tma(a);
   return dispatch_group<kRTN, true>(a);
 }
 
 cudaError_t launch_quantize(const QuantArgs& a) {
+  if (mma_path_applies(a)) return launch_quantize_mma(a);
   if (tma_path_applies(a)) return launch_quantize_tma(a);
   switch (a.mode) {
     case kRTN: return dispatch_group<kRTN, false>(a);

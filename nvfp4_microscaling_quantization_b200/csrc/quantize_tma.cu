@@ -25,6 +25,7 @@
 
 #include "kernels.h"
 #include "nvfp4_device.cuh"
+#include "quant_core.cuh"
 #include "tma_pipeline.cuh"
 
 namespace nvfp4 {
@@ -153,59 +154,6 @@ __device__ __forceinline__ void rotate64(float2 (&z)[2][16], bool upper_half) {
   for (int p = 0; p < 2; ++p)
 #pragma unroll
     for (int i = 0; i < 16; ++i) z[p][i] = __fmul2_rn(z[p][i], c2);
-}
-
-__device__ __forceinline__ float absmax64(const float2 (&z)[2][16]) {
-  float m[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-    m[i] = fmaxf(fmaxf(fabsf(z[0][i].x), fabsf(z[0][i].y)), fmaxf(fabsf(z[1][i].x), fabsf(z[1][i].y)));
-#pragma unroll
-  for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
-  return m[0];
-}
-
-struct ScaleCtx {
-  float s_g, q6, q4;
-};
-
-// Quantize the four blocks of view row `vrow` starting at view column `vcol0`
-// and store their codes and scales (blocks at or beyond vcols are skipped).
-template <int MODE>
-__device__ __forceinline__ void quantize_store64(const float2 (&z)[2][16], const ScaleCtx& sc, PhiloxKey key,
-                                                 int64_t vrow, int64_t vcol0, int64_t vcols, uint8_t* codes,
-                                                 uint8_t* scales, bool codes_aligned16, bool scales_aligned4) {
-  const uint64_t e0 = static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols) + static_cast<uint64_t>(vcol0);
-  float u[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  if constexpr (MODE == kMSEDEN) block_uniforms4(key, e0 >> 4, u);
-  BlockOut o[4];
-#pragma unroll
-  for (int p = 0; p < 2; ++p) {
-    const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, u[2 * p], u[2 * p + 1]};
-    quantize_pair<MODE>(z[p], sc.s_g, sc.q6, sc.q4, rng, o[2 * p], o[2 * p + 1]);
-  }
-  const int64_t left = (vcols - vcol0) / 16;
-  const int nvalid = left < 4 ? static_cast<int>(left) : 4;
-  uint8_t* cdst = codes + vrow * (vcols / 2) + vcol0 / 2;
-  uint8_t* sdst = scales + vrow * (vcols / 16) + vcol0 / 16;
-  if (nvalid == 4 && codes_aligned16) {
-    reinterpret_cast<uint4*>(cdst)[0] = make_uint4(o[0].lo, o[0].hi, o[1].lo, o[1].hi);
-    reinterpret_cast<uint4*>(cdst)[1] = make_uint4(o[2].lo, o[2].hi, o[3].lo, o[3].hi);
-  } else {
-#pragma unroll
-    for (int b = 0; b < 4; ++b)
-      if (b < nvalid) reinterpret_cast<uint2*>(cdst)[b] = make_uint2(o[b].lo, o[b].hi);
-  }
-  if (nvalid == 4 && scales_aligned4) {
-    *reinterpret_cast<uint32_t*>(sdst) = (o[0].scale & 0xFFu) | ((o[1].scale & 0xFFu) << 8) |
-                                         ((o[2].scale & 0xFFu) << 16) | ((o[3].scale & 0xFFu) << 24);
-  } else {
-#pragma unroll
-    for (int b = 0; b < 4; ++b)
-      if (b < nvalid) sdst[b] = static_cast<uint8_t>(o[b].scale);
-  }
 }
 
 // -------------------------------------------------------------- the kernel

@@ -2,7 +2,7 @@
 // TMA tile loads (cp.async.bulk.tensor, no multicast) completing on mbarriers,
 // consumer release through a second mbarrier per stage, and bounded waits.
 //
-// Every wait is bounded: after one plain poll it sleeps on the barrier in
+// Every wait is bounded: after a few plain polls it sleeps on the barrier in
 // slices of at most kSuspendNs nanoseconds (the thread wakes as soon as the
 // phase completes) until kWaitLimitNs of wall time (%globaltimer) have passed.
 // A wait
@@ -73,7 +73,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 
 // Wait for the phase with the given parity to complete; false if it has not
 // completed within kWaitLimitNs.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
   const uint64_t start = global_timer_ns();
   do {
     if (mbar_try_wait_sleep(bar, parity)) return true;
@@ -82,7 +82,10 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
 }
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity);
+#pragma unroll 1
+  for (int i = 0; i < 32; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity);
 }
 
 // 2-D tiled TMA load of one box into shared memory; x is the innermost

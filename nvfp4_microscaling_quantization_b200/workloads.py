@@ -22,8 +22,10 @@ backward with SR / MS-EDEN):
   outlier_normal     : std * N(0, 1), then 1% of entries (Bernoulli mask) x10
   student_t3(std)    : N(0,1) / sqrt(chi2_3 / 3), chi2_3 = sum of 3 squared
                        N(0,1) draws, times std / sqrt(3) (t_3 has variance 3)
-  laplace_channels   : Laplace(0, 1) (inverse CDF of U(-1/2, 1/2)) times a
-                       per-column scale 10^U(-1, 1) (log-uniform in [0.1, 10])
+  laplace_channels   : Laplace(0, 1) (inverse CDF of U(-1/2, 1/2), tail cut
+                       at |x| = 24 ln 2 so that a uniform draw of exactly 0
+                       gives a finite value) times a per-column scale
+                       10^U(-1, 1) (log-uniform in [0.1, 10])
 """
 from dataclasses import dataclass, field
 from typing import Dict, List, Tuple
@@ -67,7 +69,9 @@ def student_t3(shape, std: float, gen: torch.Generator) -> torch.Tensor:
 def laplace_channels(shape, gen: torch.Generator) -> torch.Tensor:
     rows, cols = shape
     u = torch.rand(shape, generator=gen, dtype=torch.float32, device=gen.device) - 0.5
-    lap = -torch.sign(u) * torch.log1p(-2.0 * u.abs())
+    # inverse CDF; torch.rand can return exactly 0 (u = -0.5), whose image is
+    # -inf, so the tail is cut at 2|u| = 1 - 2^-24 (|lap| <= 24 ln 2)
+    lap = -torch.sign(u) * torch.log1p(-(2.0 * u.abs()).clamp_max(1.0 - 2.0 ** -24))
     col_scale = torch.pow(10.0, torch.rand((1, cols), generator=gen, dtype=torch.float32,
                                            device=gen.device) * 2.0 - 1.0)
     return (lap * col_scale).to(torch.bfloat16)

@@ -72,6 +72,8 @@ def _declare(L):
     L.oracle_rht_view.restype = i32
     L.oracle_if4_constants.argtypes = [P, P]
     L.oracle_if4_constants.restype = None
+    L.oracle_quantize_rotated.argtypes = [P, i64, i64, i64, i32, u64, f32, P, P, P]
+    L.oracle_quantize_rotated.restype = i32
     L.oracle_e2m1_rtn_array.argtypes = [P, i64, P]
     L.oracle_e2m1_rtn_array.restype = None
     L.oracle_e4m3_array.argtypes = [P, i64, i32, P]
@@ -225,6 +227,21 @@ def quantize(x_bits, layout, mode, g, seed, amax_in=None, cols=None, row_range=N
     _check(lib().oracle_quantize_rows(_ptr(x), rows, cols, ld, layout, mode, g, seed,
                                       None if a is None else _ptr(a), b, e, _ptr(codes),
                                       _ptr(scales), _ptr(gs)))
+    return codes, scales, float(gs[0])
+
+
+def quantize_rotated(z, mode, seed, amax, row0=0):
+    """Quantize an already rotated fp32 view z [vr, vc] with the given tensor amax.
+
+    z holds view rows row0 .. row0+vr-1 of the full view; the random streams
+    follow the full view's element and block numbers."""
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    vr, vc = z.shape
+    codes = np.zeros((vr, vc // 2), dtype=np.uint8)
+    scales = np.zeros((vr, vc // 16), dtype=np.uint8)
+    gs = np.zeros(1, dtype=np.float32)
+    _check(lib().oracle_quantize_rotated(_ptr(z), row0, vr, vc, mode, seed, float(amax), _ptr(codes), _ptr(scales),
+                                         _ptr(gs)))
     return codes, scales, float(gs[0])
 
 

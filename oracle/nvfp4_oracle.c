@@ -607,3 +607,27 @@ void oracle_e4m3_array(const float* in, int64_t n, int round_up, uint8_t* out) {
   for (int64_t i = 0; i < n; ++i)
     out[i] = round_up ? oracle_e4m3_ru_sat(in[i]) : oracle_e4m3_rne_sat(in[i]);
 }
+
+/* Quantize an already rotated view z with a given tensor amax: steps 2 onward
+ * of oracle_quantize_rows, for checking a quantizer on rotated values it
+ * computed itself.  z holds the vr view rows row0 .. row0+vr-1 (vc fp32 each,
+ * dense); the random streams are indexed by the full view's element and block
+ * numbers, so a slice of rows gives those rows of the full result. */
+int oracle_quantize_rotated(const float* z, int64_t row0, int64_t vr, int64_t vc, int mode,
+                            uint64_t seed, float amax, uint8_t* codes, uint8_t* scales,
+                            float* global_scale) {
+  if (mode < ORC_RTN || mode > ORC_4OVER6) return ORC_ERR_ARG;
+  if (row0 < 0 || vr < 0 || vc < 0 || vc % 16) return ORC_ERR_SHAPE;
+  float s_g = oracle_global_scale(amax, mode);
+  *global_scale = s_g;
+  for (int64_t r = 0; r < vr; ++r) {
+    for (int64_t bc = 0; bc < vc / 16; ++bc) {
+      uint8_t code[16];
+      uint8_t S = quantize_block(z + r * vc + bc * 16, mode, s_g, seed, row0 + r, vc, bc, code);
+      scales[r * (vc / 16) + bc] = S;
+      for (int k = 0; k < 8; ++k)
+        codes[r * (vc / 2) + bc * 8 + k] = (uint8_t)(code[2 * k] | (code[2 * k + 1] << 4));
+    }
+  }
+  return ORC_OK;
+}

@@ -18,3 +18,14 @@ def orc():
     import oracle
     oracle.lib()
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Report the end-to-end differences of the rotated modes against the oracle."""
+    helpers = sys.modules.get("gpu_helpers")
+    if helpers is None or not helpers.ROTATED_MISMATCH[1]:
+        return
+    cb, c, sb, s = helpers.ROTATED_MISMATCH
+    terminalreporter.write_line(
+        f"rotated modes, end to end against the oracle: {cb} of {c} codes ({cb / c:.2e}) and "
+        f"{sb} of {s} scales ({sb / s:.2e}) differ")

@@ -340,3 +340,19 @@ def test_gaussian_top_interval_share_reported(orc):
     share = np.mean(y >= 4.0)
     print(f"\nshare of |y| in [4,6]: {share:.4f}")
     assert 0.15 < share < 0.21
+
+
+@pytest.mark.parametrize("mode", [RTN, SR, EDEN, IF4, FO6])
+def test_quantize_rotated_equals_quantize(orc, mode):
+    """Quantizing the oracle's own rotated view gives the oracle's quantization."""
+    rng = np.random.default_rng(12)
+    x = bf16(rng.standard_normal((128, 256)))
+    for layout in (ROW, TR):
+        z = orc.rht_view(bits_of(x), layout, 128, 8)
+        a = orc.amax(bits_of(x), layout, 128, 8)
+        ref = orc.quantize(bits_of(x), layout, mode, 128, 8)
+        got = orc.quantize_rotated(z, mode, 8, a)
+        assert np.array_equal(ref[0], got[0]) and np.array_equal(ref[1], got[1]) and ref[2] == got[2]
+        # a slice of view rows gives those rows of the full result
+        part = orc.quantize_rotated(z[37:41], mode, 8, a, row0=37)
+        assert np.array_equal(part[0], ref[0][37:41]) and np.array_equal(part[1], ref[1][37:41])
