@@ -24,6 +24,7 @@
 #include <cudaTypedefs.h>
 
 #include "kernels.h"
+#include "launch_config.h"
 #include "nvfp4_device.cuh"
 #include "quant_core.cuh"
 #include "tma_pipeline.cuh"
@@ -384,9 +385,8 @@ cudaError_t launch_tma_one(const QuantArgs& a) {
   int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kNT, smem);
+  e = resident_ctas(kernel, kNT, smem, 32, &per_sm);
   if (e != cudaSuccess) return e;
-  if (per_sm < 1) per_sm = 1;
   const int64_t n_ct = ROWWISE ? (a.cols + kRowTileCols - 1) / kRowTileCols : (a.cols + kColTileCols - 1) / kColTileCols;
   const int64_t n_tiles = ROWWISE ? ((a.rows + kRowBoxRows - 1) / kRowBoxRows) * n_ct
                                   : ((a.rows + kColTileRows - 1) / kColTileRows) * n_ct;

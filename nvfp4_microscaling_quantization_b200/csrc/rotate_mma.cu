@@ -25,6 +25,7 @@
 #include <cudaTypedefs.h>
 
 #include "kernels.h"
+#include "launch_config.h"
 #include "nvfp4_device.cuh"
 #include "quant_core.cuh"
 #include "tcgen05.cuh"
@@ -34,16 +35,45 @@ namespace nvfp4 {
 
 namespace {
 
-constexpr int kEpiWarps = 8;
+#ifndef NVFP4_MMA_GROUPS
+#define NVFP4_MMA_GROUPS 4
+#endif
+#ifndef NVFP4_MMA_ACCUM
+#define NVFP4_MMA_ACCUM 4
+#endif
+#ifndef NVFP4_MMA_STAGES
+#define NVFP4_MMA_STAGES 3
+#endif
+#ifndef NVFP4_MMA_CTAS
+#define NVFP4_MMA_CTAS 1
+#endif
+
+#ifndef NVFP4_MMA_GROUP_WARPS
+#define NVFP4_MMA_GROUP_WARPS 4
+#endif
+#ifndef NVFP4_MMA_QUAD
+#define NVFP4_MMA_QUAD 0
+#endif
+
+constexpr int kGroups = NVFP4_MMA_GROUPS;           // epilogue groups, each on its own tiles
+constexpr int kGroupWarps = NVFP4_MMA_GROUP_WARPS;  // 4 (a thread owns 128 columns) or 8 (64)
+constexpr int kHalves = 8 / kGroupWarps;            // 64-column halves of a row per thread
+constexpr bool kQuad = NVFP4_MMA_QUAD != 0;         // four blocks in flight instead of two
+constexpr int kEpiWarps = kGroupWarps * kGroups;
+static_assert(kGroupWarps == 4 || kGroupWarps == 8, "a group covers the four lane quarters once or twice");
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
-constexpr int kStagesA = 2;                 // A tiles in flight
-constexpr int kAccum = 2;                   // accumulators in tensor memory
-constexpr int kTile = 128;                  // tile rows and columns of X
+constexpr int kStagesA = NVFP4_MMA_STAGES;   // A tiles in flight
+constexpr int kAccum = NVFP4_MMA_ACCUM;      // accumulators in tensor memory
+constexpr int kCtasPerSm = NVFP4_MMA_CTAS;   // resident CTAs per SM
+constexpr int kTile = 128;                   // tile rows and columns of X
 constexpr uint32_t kTileBytes = kTile * kTile * 2;
 constexpr uint32_t kBoxBytes = kTile * 128;  // 128 rows x 64 bf16
-constexpr uint32_t kTmemCols = kAccum * kTile;
+// tensor-memory allocations are powers of two columns
+constexpr uint32_t kTmemCols = kAccum <= 1 ? 128u : (kAccum <= 2 ? 256u : 512u);
 constexpr size_t kDynSmem = (kStagesA + 1) * kTileBytes + 1024;
+static_assert(kAccum >= 1 && kAccum <= 4, "up to four 128-column accumulators");
+static_assert(kCtasPerSm * kTmemCols <= 512, "the resident CTAs' accumulators must fit in tensor memory");
 
 enum Kind { kQuantize = 0, kAmax = 1, kStoreZ = 2 };
 
@@ -63,14 +93,24 @@ __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
   return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
 }
 
+// Accumulator column of output column n: inside each 32-column group the two
+// 16-element blocks are interleaved (block a element i at 2i, block b element
+// i at 2i + 1), so a 32-column load from tensor memory yields the (a_i, b_i)
+// register pairs that the packed f32x2 arithmetic works on.
+__device__ __forceinline__ uint32_t output_col_of(uint32_t acc_col) {
+  return (acc_col & ~31u) | ((acc_col & 1u) << 4) | ((acc_col & 31u) >> 1);
+}
+
 // B operand, K-major with the 128-byte swizzle: two 64-wide K halves of 128
-// rows (n) x 128 bytes; element (n, k) = sigma_(k mod G) * H_G[n mod G][k mod G]
-// inside the diagonal G x G blocks, 0 elsewhere.  bf16 +1 = 0x3F80, -1 = 0xBF80.
+// rows x 128 bytes; row r holds output column n = output_col_of(r), element
+// (n, k) = sigma_(k mod G) * H_G[n mod G][k mod G] inside the diagonal G x G
+// blocks, 0 elsewhere.  bf16 +1 = 0x3F80, -1 = 0xBF80.
 template <int G>
 __device__ __forceinline__ void build_hadamard_b(uint8_t* bmat, PhiloxKey key, uint32_t tid) {
   const uint4 w = philox_call(key, 0, kTagSigns);
   for (uint32_t c = tid; c < 2048; c += kThreads) {
-    const uint32_t half = c >> 10, n = (c >> 3) & 127u, kc = c & 7u;
+    const uint32_t half = c >> 10, r = (c >> 3) & 127u, kc = c & 7u;
+    const uint32_t n = output_col_of(r);
     uint32_t packed[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -88,13 +128,13 @@ __device__ __forceinline__ void build_hadamard_b(uint8_t* bmat, PhiloxKey key, u
       }
       packed[i] = two;
     }
-    *reinterpret_cast<uint4*>(bmat + half * kBoxBytes + n * 128 + ((kc ^ (n & 7u)) << 4)) =
+    *reinterpret_cast<uint4*>(bmat + half * kBoxBytes + r * 128 + ((kc ^ (r & 7u)) << 4)) =
         make_uint4(packed[0], packed[1], packed[2], packed[3]);
   }
 }
 
 template <int MODE, int G, int KIND, bool ROWWISE>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed,
                   const float* __restrict__ amax, unsigned int* __restrict__ amax_accum, uint8_t* __restrict__ codes,
                   uint8_t* __restrict__ scales, float* __restrict__ gscale, float* __restrict__ zout) {
@@ -115,7 +155,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     }
     for (int a = 0; a < kAccum; ++a) {
       mbar_init(&sh.tfull[a], 1);
-      mbar_init(&sh.tfree[a], kEpiWarps);
+      mbar_init(&sh.tfree[a], kGroupWarps);  // the warps of one epilogue group
     }
     sh.issued_a = 0;
     sh.issued_mma = 0;
@@ -189,7 +229,12 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const uint32_t q = warp & 3u, j = warp >> 2;
+    // group `grp` takes the CTA's tiles k = grp, grp + kGroups, ...; within it
+    // a warp reads lane quarter q (= warp % 4, as tensor memory requires) and
+    // either all 128 columns (groups of 4 warps) or the half 64j .. 64j+63
+    // (groups of 8 warps)
+    const uint32_t q = warp & 3u, grp = warp / kGroupWarps;
+    const uint32_t j0 = kGroupWarps == 8 ? (warp >> 2) & 1u : 0u;
     ScaleCtx sc{1.0f, 0.0f, 0.0f};
     if constexpr (KIND == kQuantize) {
       sc.s_g = global_scale_of<MODE>(*amax);
@@ -198,79 +243,97 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
       if (blockIdx.x == 0 && tid == 0) *gscale = sc.s_g;
     }
     const int64_t vcols = ROWWISE ? cols : rows;
+    const int64_t vrows = ROWWISE ? rows : cols;
     const bool codes_aligned16 = ((vcols / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes) % 16) == 0;
     const bool scales_aligned4 = ((vcols / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales) % 4) == 0;
     const float2 c2 = f2(RhtConst<G>::c, RhtConst<G>::c);
     float local_max = 0.0f;
-    int k = 0;
-    for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++k) {
+    int k = static_cast<int>(grp);
+    for (int64_t t = blockIdx.x + grp * step; t < n_tiles; t += kGroups * step, k += kGroups) {
       const int a = k % kAccum;
       if (!mbar_wait(&sh.tfull[a], (k / kAccum) & 1u)) {
         atomicExch(&sh.abort_flag, 1);
         break;
       }
       tc_fence_after_sync();
-      const uint32_t taddr = tmem_base + ((32u * q) << 16) + a * kTile + j * 64;
       const int64_t rt = t / n_ct, ct = t - rt * n_ct;
-      // view row of this thread and view column of its first element
+      // view row of this thread
       const int64_t vrow = (ROWWISE ? rt : ct) * kTile + 32 * q + lane;
-      const int64_t vcol0 = (ROWWISE ? ct : rt) * kTile + 64 * j;
-      const int64_t vrows = ROWWISE ? rows : cols;
+#pragma unroll 1
+      for (int h = 0; h < kHalves; ++h) {
+        const uint32_t j = j0 + h;
+        const uint32_t taddr = tmem_base + ((32u * q) << 16) + a * kTile + j * 64;
+        const int64_t vcol0 = (ROWWISE ? ct : rt) * kTile + 64 * j;  // view column of the first element
+        const bool last = h == kHalves - 1;
 
-      if constexpr (KIND == kQuantize) {
-        // one pair of blocks at a time: load 32 columns, quantize, then the next 32
-        const bool valid = vrow < vrows && vcol0 < vcols;
-        const uint64_t e0 = static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols) + static_cast<uint64_t>(vcol0);
-        float u[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        if constexpr (MODE == kMSEDEN) block_uniforms4(key, e0 >> 4, u);
-        BlockOut o[4];
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          float v[32];
-          tmem_ld32_wait(taddr + 32 * p, v);
-          if (p == 1) {
+        if constexpr (KIND == kQuantize && kQuad) {
+          float v[64];
+          tmem_ld64_wait(taddr, v);
+          if (last) {
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.tfree[a]);
           }
-          float2 zp[16];
+          float2 z[2][16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) zp[i] = __fmul2_rn(f2(v[i], v[16 + i]), c2);
-          const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, u[2 * p], u[2 * p + 1]};
-          quantize_pair<MODE>(zp, sc.s_g, sc.q6, sc.q4, rng, o[2 * p], o[2 * p + 1]);
-        }
-        if (valid) store64(o, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);
-        continue;
-      }
-
-      float v[64];
-      tmem_ld64_wait(taddr, v);
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.tfree[a]);
-
-      float2 z[2][16];
+          for (int p = 0; p < 2; ++p)
 #pragma unroll
-      for (int p = 0; p < 2; ++p)
+            for (int i = 0; i < 16; ++i) z[p][i] = __fmul2_rn(f2(v[32 * p + 2 * i], v[32 * p + 2 * i + 1]), c2);
+          if (vrow < vrows && vcol0 < vcols)
+            quantize_store64<MODE>(z, sc, key, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);
+        } else if constexpr (KIND == kQuantize) {
+          // one pair of blocks at a time: load 32 columns, quantize, then the next 32
+          const bool valid = vrow < vrows && vcol0 < vcols;
+          const uint64_t e0 = static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols) + static_cast<uint64_t>(vcol0);
+          float u[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          if constexpr (MODE == kMSEDEN) block_uniforms4(key, e0 >> 4, u);
+          BlockOut o[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) z[p][i] = __fmul2_rn(f2(v[32 * p + i], v[32 * p + 16 + i]), c2);
-
-      if constexpr (KIND == kAmax) {
-        local_max = fmaxf(local_max, absmax64(z));
-      } else if constexpr (KIND == kStoreZ) {
-        if (vrow < vrows && vcol0 < vcols) {
-          float4* dst = reinterpret_cast<float4*>(zout + vrow * vcols + vcol0);
-          const int64_t left = (vcols - vcol0) / 16;
-          const int nvalid = left < 4 ? static_cast<int>(left) : 4;
+          for (int p = 0; p < 2; ++p) {
+            float v[32];
+            tmem_ld32_wait(taddr + 32 * p, v);
+            if (last && p == 1) {
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sh.tfree[a]);
+            }
+            float2 zp[16];
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            if (b >= nvalid) continue;
-            const int p = b >> 1;
+            for (int i = 0; i < 16; ++i) zp[i] = __fmul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
+            const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, u[2 * p], u[2 * p + 1]};
+            quantize_pair<MODE>(zp, sc.s_g, sc.q6, sc.q4, rng, o[2 * p], o[2 * p + 1]);
+          }
+          if (valid) store64(o, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);
+        } else {
+          // max |z| or z itself, one pair of blocks (32 columns) at a time
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int i = 4 * e;
-              dst[4 * b + e] = (b & 1) ? make_float4(z[p][i].y, z[p][i + 1].y, z[p][i + 2].y, z[p][i + 3].y)
-                                       : make_float4(z[p][i].x, z[p][i + 1].x, z[p][i + 2].x, z[p][i + 3].x);
+          for (int p = 0; p < 2; ++p) {
+            float v[32];
+            tmem_ld32_wait(taddr + 32 * p, v);
+            if (last && p == 1) {
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sh.tfree[a]);
+            }
+            float2 zp[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) zp[i] = __fmul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
+            if constexpr (KIND == kAmax) {
+              float ma, mb;
+              absmax_pair(zp, ma, mb);
+              local_max = fmaxf(local_max, fmaxf(ma, mb));
+            } else {
+              const int64_t c0 = vcol0 + 32 * p;  // view column of block 2p
+              if (vrow < vrows && c0 < vcols) {
+                float4* dst = reinterpret_cast<float4*>(zout + vrow * vcols + c0);
+                const bool second = c0 + 16 < vcols;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int i = 4 * e;
+                  dst[e] = make_float4(zp[i].x, zp[i + 1].x, zp[i + 2].x, zp[i + 3].x);
+                  if (second) dst[4 + e] = make_float4(zp[i].y, zp[i + 1].y, zp[i + 2].y, zp[i + 3].y);
+                }
+              }
             }
           }
         }
@@ -346,15 +409,12 @@ cudaError_t launch_one(const QuantArgs& a, float* zout) {
   auto kernel = rotate_mma_kernel<MODE, G, KIND, ROWWISE>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDynSmem));
   if (e != cudaSuccess) return e;
-  // two CTAs per SM need the largest shared-memory carveout
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-  if (e != cudaSuccess) return e;
+  // at most kCtasPerSm CTAs per SM: tensor memory holds that many CTAs' accumulators
   int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, kDynSmem);
+  e = resident_ctas(kernel, kThreads, kDynSmem, kCtasPerSm, &per_sm);
   if (e != cudaSuccess) return e;
-  per_sm = per_sm < 1 ? 1 : (per_sm > 2 ? 2 : per_sm);  // tensor memory holds two CTAs' accumulators
   const int64_t n_tiles = ((a.rows + kTile - 1) / kTile) * ((a.cols + kTile - 1) / kTile);
   int64_t grid = n_tiles < int64_t(sms) * per_sm ? n_tiles : int64_t(sms) * per_sm;
   if (grid == 0) {
