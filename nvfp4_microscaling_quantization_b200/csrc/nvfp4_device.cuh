@@ -46,7 +46,7 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, PhiloxKey key) {
 
 // Stream tags carried in counter word 2.
 constexpr uint32_t kTagElement = 0;  // element stochastic rounding: 8 x 16-bit uniforms per call
-constexpr uint32_t kTagBlock = 1;    // scale stochastic rounding: 4 x 24-bit uniforms per call
+constexpr uint32_t kTagBlock = 1;    // scale stochastic rounding: 8 x 16-bit uniforms per call
 constexpr uint32_t kTagSigns = 2;    // RHT signs: 128 sign bits from call 0
 
 __device__ __forceinline__ uint4 philox_call(PhiloxKey key, uint64_t call, uint32_t tag) {
@@ -56,6 +56,16 @@ __device__ __forceinline__ uint4 philox_call(PhiloxKey key, uint64_t call, uint3
 
 __device__ __forceinline__ uint32_t word_of(const uint4& w, uint32_t i) {
   return i == 0 ? w.x : (i == 1 ? w.y : (i == 2 ? w.z : w.w));
+}
+
+// 16-bit draw i (0..7) of a call: word i/2, low half for even i, high for odd.
+__device__ __forceinline__ uint32_t half_word(const uint4& w, uint32_t i) {
+  return (word_of(w, i >> 1) >> ((i & 1u) * 16u)) & 0xFFFFu;
+}
+
+// k * 2^-16 for k < 2^16, exactly: k placed in the fraction of 1.0 minus 1.
+__device__ __forceinline__ float uniform16(uint32_t k) {
+  return __fsub_rn(__uint_as_float(0x3F800000u | (k << 7)), 1.0f);
 }
 
 // ---------------------------------------------------------------------------
@@ -262,7 +272,7 @@ __device__ __forceinline__ uint32_t sr_code(float y, uint32_t k16) {
   const float fl = floorf(t);
   const float frac = __fsub_rn(t, fl);     // exact: position inside the interval
   uint32_t mag = static_cast<uint32_t>(fl) + base;
-  const float U = __fmul_rn(static_cast<float>(k16), 0x1p-16f);
+  const float U = uniform16(k16);
   if (U < frac) ++mag;
   if (mag == 0u) return 0u;
   return mag | (y < 0.0f ? 8u : 0u);
@@ -351,8 +361,8 @@ __device__ __forceinline__ BlockOut quantize_block(const float* z, float s_g, co
       }
       const float c = (num > 0.0f && den > 0.0f) ? __fdiv_rn(num, den) : 1.0f;
       const float t = __fmul_rn(e4m3_decode(S), c);
-      const uint4 w = philox_call(rng.key, rng.block >> 2, kTagBlock);
-      const float U = __fmul_rn(static_cast<float>(word_of(w, rng.block & 3u) >> 8), 0x1p-24f);
+      const uint4 w = philox_call(rng.key, rng.block >> 3, kTagBlock);
+      const float U = uniform16(half_word(w, static_cast<uint32_t>(rng.block & 7u)));
       out.scale = e4m3_sr(t, U);
     } else {  // kIF4
       uint32_t f_lo, f_hi;
@@ -402,6 +412,46 @@ struct PairRng {
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
+// Per-launch constants of the block-scale step: the tensor scale s_g, the
+// divisors q6 = RN(6 s_g) and q4 = RN(4 s_g) of s_f = RN(absmax / q), and
+// their round-to-nearest reciprocals for the division below.
+struct ScaleCtx {
+  float s_g, q6, q4, r6, r4;
+  bool markstein;  // the reciprocal-based division is exact for every block
+};
+
+template <int MODE>
+__device__ __forceinline__ ScaleCtx make_scale_ctx(float amax) {
+  ScaleCtx c;
+  c.s_g = global_scale_of<MODE>(amax);
+  c.q6 = __fmul_rn(6.0f, c.s_g);
+  c.q4 = __fmul_rn(4.0f, c.s_g);
+  c.r6 = __frcp_rn(c.q6);
+  c.r4 = __frcp_rn(c.q4);
+  // With q in [2^-90, 2^100] the remainder below cannot underflow unless
+  // a / q < 2^-12, where any value within an ulp gives the same (zero) E4M3
+  // scale; outside that range the kernels divide with __fdiv_rn.
+  c.markstein = c.q4 >= 0x1p-90f && c.q6 <= 0x1p100f;
+  return c;
+}
+
+// RN(a / q) for the two lanes, with r = RN(1/q): Markstein's correction
+// (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Dev. 34(1), 1990): t = RN(a r) is within
+// an ulp of a/q, the remainder a - t q is exact in one fused multiply-add, and
+// RN(t + (a - t q) r) is the correctly rounded quotient.
+__device__ __forceinline__ float2 div2_by(float2 a, float q, float r, bool markstein) {
+  if (!markstein) return f2(__fdiv_rn(a.x, q), __fdiv_rn(a.y, q));
+  const float2 q2 = f2(q, q), r2 = f2(r, r);
+  const float2 t = __fmul2_rn(a, r2);
+  const float2 rem = __ffma2_rn(f2(-t.x, -t.y), q2, a);
+  const float2 d = __ffma2_rn(rem, r2, t);
+  // a quotient that overflows (an absmax far above the tensor amax given)
+  // comes out NaN here and infinite from the division; both saturate the
+  // E4M3 scale, and so does 1024
+  return f2(fminf(d.x, 1024.0f), fminf(d.y, 1024.0f));
+}
+
 // a - b per lane: the negation is exact, so each lane is the one RN subtraction.
 __device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) { return __fadd2_rn(a, f2(-b.x, -b.y)); }
 
@@ -419,6 +469,22 @@ __device__ __forceinline__ float2 e4m3x2_decode(uint32_t codes) {
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
   const __half2 p = *reinterpret_cast<const __half2*>(&h2);
   return f2(__low2float(p), __high2float(p));
+}
+
+// Stochastic rounding of two t >= 0 onto E4M3, the two-lane form of e4m3_sr:
+// bits 0..7 for t.x with the uniform ua, bits 8..15 for t.y with ub.  Each
+// byte stays in 0..0x7F: the RNE code is lowered only when it decodes above
+// t (so it is nonzero), and 0x7E + 1 = 0x7F decodes to NaN, which never
+// rounds up.
+__device__ __forceinline__ uint32_t e4m3x2_sr(float2 t, float ua, float ub) {
+  uint32_t lo = e4m3x2_rne_sat(t.x, t.y);
+  const float2 d = e4m3x2_decode(lo);
+  lo -= (d.x > t.x ? 1u : 0u) + (d.y > t.y ? 0x100u : 0u);
+  const float2 l = e4m3x2_decode(lo);
+  const float2 h = e4m3x2_decode(lo + 0x0101u);
+  const float2 below = __fmul2_rn(f2(ua, ub), sub2_rn(h, l));  // exact: the gap is a power of two
+  const float2 above = sub2_rn(t, l);                          // exact
+  return lo + (below.x < above.x ? 1u : 0u) + (below.y < above.y ? 0x100u : 0u);
 }
 
 // Stochastic rounding of one block of 16 scaled values; elem = view index of element 0.
@@ -465,19 +531,20 @@ __device__ __forceinline__ float2 rcp_or_zero(float2 d) {
 }
 
 template <int MODE>
-__device__ __forceinline__ void quantize_pair(const float2 (&z)[16], float s_g, float q6, float q4,
-                                              const PairRng& rng, BlockOut& oa, BlockOut& ob) {
+__device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const ScaleCtx& sc, const PairRng& rng,
+                                              BlockOut& oa, BlockOut& ob) {
   float aa, ab;
   absmax_pair(z, aa, ab);
-  const float2 sg2 = f2(s_g, s_g);
+  const float2 sg2 = f2(sc.s_g, sc.s_g);
 
   if constexpr (MODE == k4over6) {
     uint32_t S[2], ca_lo[2], ca_hi[2], cb_lo[2], cb_hi[2];
     float2 err[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const float q = k == 0 ? q6 : q4;
-      S[k] = e4m3x2_rne_sat(__fdiv_rn(aa, q), __fdiv_rn(ab, q));
+      const float2 sf = k == 0 ? div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein)
+                               : div2_by(f2(aa, ab), sc.q4, sc.r4, sc.markstein);
+      S[k] = e4m3x2_rne_sat(sf.x, sf.y);
       const float2 d = __fmul2_rn(e4m3x2_decode(S[k]), sg2);
       const float2 r = rcp_or_zero(d);
       float ya[16], yb[16];
@@ -511,13 +578,13 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], float s_g, 
     ob.scale = ((pb ? S[1] : S[0]) >> 8) & 0xFFu;
     return;
   } else {
-    uint32_t S2 = e4m3x2_rne_sat(__fdiv_rn(aa, q6), __fdiv_rn(ab, q6));
+    const float2 sf = div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein);
+    uint32_t S2 = e4m3x2_rne_sat(sf.x, sf.y);
     uint32_t Sa = S2 & 0xFFu, Sb = S2 >> 8;
     float2 dS = e4m3x2_decode(S2);
     if constexpr (MODE == kSR) {
-      const float sfa = __fdiv_rn(aa, q6), sfb = __fdiv_rn(ab, q6);
-      if (Sa < 0x7Eu && dS.x < sfa) ++Sa;
-      if (Sb < 0x7Eu && dS.y < sfb) ++Sb;
+      if (Sa < 0x7Eu && dS.x < sf.x) ++Sa;
+      if (Sb < 0x7Eu && dS.y < sf.y) ++Sb;
       S2 = Sa | (Sb << 8);
       dS = e4m3x2_decode(S2);
     }
@@ -556,9 +623,9 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], float s_g, 
       const float qa = __fdiv_rn(num.x, den.x), qb = __fdiv_rn(num.y, den.y);
       const float ca = (num.x > 0.0f && den.x > 0.0f) ? qa : 1.0f;
       const float cb = (num.y > 0.0f && den.y > 0.0f) ? qb : 1.0f;
-      const float2 t = __fmul2_rn(dS, f2(ca, cb));
-      oa.scale = e4m3_sr(t.x, rng.u_a);
-      ob.scale = e4m3_sr(t.y, rng.u_b);
+      const uint32_t S = e4m3x2_sr(__fmul2_rn(dS, f2(ca, cb)), rng.u_a, rng.u_b);
+      oa.scale = S & 0xFFu;
+      ob.scale = S >> 8;
     } else {  // kIF4
       uint32_t fa_lo, fa_hi, fb_lo, fb_hi;
       rtn_codes(ya, fa_lo, fa_hi);
@@ -602,22 +669,21 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], float s_g, 
   }
 }
 
-// Scale uniforms of four consecutive view blocks b0..b0+3 (MS-EDEN): one
-// Philox call when b0 is a multiple of 4, two otherwise.
-__device__ __forceinline__ void block_uniforms4(PhiloxKey key, uint64_t b0, float (&u)[4]) {
-  const uint4 w0 = philox_call(key, b0 >> 2, kTagBlock);
-  if ((b0 & 3u) == 0) {
-    u[0] = __fmul_rn(static_cast<float>(w0.x >> 8), 0x1p-24f);
-    u[1] = __fmul_rn(static_cast<float>(w0.y >> 8), 0x1p-24f);
-    u[2] = __fmul_rn(static_cast<float>(w0.z >> 8), 0x1p-24f);
-    u[3] = __fmul_rn(static_cast<float>(w0.w >> 8), 0x1p-24f);
-  } else {
-    const uint4 w1 = philox_call(key, (b0 >> 2) + 1, kTagBlock);
+// Scale uniforms of N consecutive view blocks b0 .. b0+N-1 (MS-EDEN): one
+// Philox call when they lie in one group of eight, two otherwise.
+template <int N>
+__device__ __forceinline__ void block_uniforms(PhiloxKey key, uint64_t b0, float (&u)[N]) {
+  const uint32_t first = static_cast<uint32_t>(b0 & 7u);
+  const uint4 w0 = philox_call(key, b0 >> 3, kTagBlock);
+  if (first + N <= 8) {
 #pragma unroll
-    for (uint32_t k = 0; k < 4; ++k) {
-      const uint64_t b = b0 + k;
-      const uint32_t word = (b >> 2) == (b0 >> 2) ? word_of(w0, b & 3u) : word_of(w1, b & 3u);
-      u[k] = __fmul_rn(static_cast<float>(word >> 8), 0x1p-24f);
+    for (int k = 0; k < N; ++k) u[k] = uniform16(half_word(w0, first + k));
+  } else {
+    const uint4 w1 = philox_call(key, (b0 >> 3) + 1, kTagBlock);
+#pragma unroll
+    for (int k = 0; k < N; ++k) {
+      const uint32_t i = first + k;
+      u[k] = uniform16(i < 8 ? half_word(w0, i) : half_word(w1, i - 8));
     }
   }
 }

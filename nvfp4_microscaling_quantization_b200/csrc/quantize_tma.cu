@@ -214,11 +214,9 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
     for (int k = 0; k < kStages; ++k) load(k);
   }
 
-  ScaleCtx sc{1.0f, 0.0f, 0.0f};
+  ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false};
   if constexpr (!AMAX_ONLY) {
-    sc.s_g = global_scale_of<MODE>(*amax);
-    sc.q6 = __fmul_rn(6.0f, sc.s_g);
-    sc.q4 = __fmul_rn(4.0f, sc.s_g);
+    sc = make_scale_ctx<MODE>(*amax);
     if (blockIdx.x == 0 && tid == 0) *gscale = sc.s_g;
   }
   // thread roles

@@ -235,17 +235,16 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     // (groups of 8 warps)
     const uint32_t q = warp & 3u, grp = warp / kGroupWarps;
     const uint32_t j0 = kGroupWarps == 8 ? (warp >> 2) & 1u : 0u;
-    ScaleCtx sc{1.0f, 0.0f, 0.0f};
+    ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false};
     if constexpr (KIND == kQuantize) {
-      sc.s_g = global_scale_of<MODE>(*amax);
-      sc.q6 = __fmul_rn(6.0f, sc.s_g);
-      sc.q4 = __fmul_rn(4.0f, sc.s_g);
+      sc = make_scale_ctx<MODE>(*amax);
       if (blockIdx.x == 0 && tid == 0) *gscale = sc.s_g;
     }
     const int64_t vcols = ROWWISE ? cols : rows;
     const int64_t vrows = ROWWISE ? rows : cols;
     const bool codes_aligned16 = ((vcols / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes) % 16) == 0;
     const bool scales_aligned4 = ((vcols / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales) % 4) == 0;
+    const bool row_blocks8 = ((vcols / 16) % 8) == 0;
     const float2 c2 = f2(RhtConst<G>::c, RhtConst<G>::c);
     float local_max = 0.0f;
     int k = static_cast<int>(grp);
@@ -259,6 +258,16 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
       const int64_t rt = t / n_ct, ct = t - rt * n_ct;
       // view row of this thread
       const int64_t vrow = (ROWWISE ? rt : ct) * kTile + 32 * q + lane;
+      // MS-EDEN scale uniforms: when a thread owns a whole 128-column row of
+      // the tile and view rows hold whole groups of eight blocks, its eight
+      // blocks take the eight draws of one Philox call
+      uint4 wu = make_uint4(0u, 0u, 0u, 0u);
+      if constexpr (KIND == kQuantize && MODE == kMSEDEN && kHalves == 2) {
+        if (row_blocks8)
+          wu = philox_call(key, (static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols / 16) +
+                                 static_cast<uint64_t>((ROWWISE ? ct : rt) * (kTile / 16))) >> 3,
+                           kTagBlock);
+      }
 #pragma unroll 1
       for (int h = 0; h < kHalves; ++h) {
         const uint32_t j = j0 + h;
@@ -286,7 +295,14 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
           const bool valid = vrow < vrows && vcol0 < vcols;
           const uint64_t e0 = static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols) + static_cast<uint64_t>(vcol0);
           float u[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-          if constexpr (MODE == kMSEDEN) block_uniforms4(key, e0 >> 4, u);
+          if constexpr (MODE == kMSEDEN) {
+            if (kHalves == 2 && row_blocks8) {
+#pragma unroll
+              for (int b = 0; b < 4; ++b) u[b] = uniform16(half_word(wu, 4 * j + b));
+            } else {
+              block_uniforms<4>(key, e0 >> 4, u);
+            }
+          }
           BlockOut o[4];
 #pragma unroll
           for (int p = 0; p < 2; ++p) {
@@ -301,7 +317,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
 #pragma unroll
             for (int i = 0; i < 16; ++i) zp[i] = __fmul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
             const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, u[2 * p], u[2 * p + 1]};
-            quantize_pair<MODE>(zp, sc.s_g, sc.q6, sc.q4, rng, o[2 * p], o[2 * p + 1]);
+            quantize_pair<MODE>(zp, sc, rng, o[2 * p], o[2 * p + 1]);
           }
           if (valid) store64(o, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);
         } else {

@@ -107,13 +107,15 @@ float oracle_uniform_element(uint64_t seed, uint64_t e) {
 }
 
 /* Scale stochastic-rounding uniform (tag 1): block b of the quantized view
- * (row-major linear block index).  Call b/4 yields 4 uniforms of 24 bits:
- * U = (word[b mod 4] >> 8) * 2^-24. */
+ * (row-major linear block index).  Call b/8 yields 8 uniforms of 16 bits, laid
+ * out like the element uniforms: word (b mod 8)/2, low half for even b, high
+ * half for odd b.  U = k * 2^-16. */
 float oracle_uniform_block(uint64_t seed, uint64_t b) {
   uint32_t w[4];
-  philox_call(seed, b >> 2, 1u, w);
-  uint32_t k = w[b & 3u] >> 8;
-  return (float)k * 0x1p-24f; /* exact: k < 2^24 */
+  philox_call(seed, b >> 3, 1u, w);
+  uint32_t word = w[(b & 7u) >> 1];
+  uint32_t k = (word >> (16u * (uint32_t)(b & 1u))) & 0xFFFFu;
+  return (float)k * 0x1p-16f; /* exact */
 }
 
 /* Random Hadamard signs (tag 2): sigma_j for j < g (g <= 128) is -1 when bit

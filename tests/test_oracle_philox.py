@@ -69,10 +69,12 @@ def test_streams_follow_their_counters(orc):
         word = int(w[(e & 7) >> 1])
         k = (word >> (16 * (e & 1))) & 0xFFFF
         assert orc.uniform_element(seed, e) == k / 65536.0
-    # block b -> call b>>2, tag 1
-    for b in [0, 1, 2, 3, 4, 999, 77777]:
-        w = curand_block(lib, seed, (b >> 2) * 65536 + 1)
-        assert orc.uniform_block(seed, b) == (int(w[b & 3]) >> 8) / 16777216.0
+    # block b -> call b>>3, tag 1, 16-bit halves like the element draws
+    for b in [0, 1, 2, 3, 4, 7, 8, 999, 77777]:
+        w = curand_block(lib, seed, (b >> 3) * 65536 + 1)
+        word = int(w[(b & 7) >> 1])
+        k = (word >> (16 * (b & 1))) & 0xFFFF
+        assert orc.uniform_block(seed, b) == k / 65536.0
     # sign j -> call 0, tag 2
     w = curand_block(lib, seed, 2)
     signs = orc.rht_signs(seed, 128)
