@@ -44,7 +44,11 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes per launch measured by ncu for the dominant kernel, keyed by the
 # hash of the kernel sources they were taken with (see profiles/).  A changed
 # kernel reports traffic = null until it is captured again.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/rotate_mma_eden_dy.md: dram__bytes_read.sum + dram__bytes_write.sum, one launch
+    ("bea7130ec89ddce6", "dy.transposed.ms_eden.g128"): 470032384 + 108876544,
+    ("bea7130ec89ddce6", "dy.rowwise.ms_eden.g128"): 469903104 + 109543680,
+}
 
 
 def parse_args(argv=None):

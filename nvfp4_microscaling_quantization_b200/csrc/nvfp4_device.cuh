@@ -90,9 +90,10 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
 
 // For each nibble: keep the sign bit only if the magnitude bits are nonzero.
 __device__ __forceinline__ uint32_t clear_negative_zero(uint32_t w) {
-  const uint32_t mag = w & 0x77777777u;
-  const uint32_t nonzero = (mag + 0x77777777u) & 0x88888888u;  // bit 3 of a nibble set iff mag != 0
-  return mag | (w & nonzero);
+  // mag + 7 carries into bit 3 of a nibble iff its magnitude is nonzero (and
+  // never into the next nibble); the magnitude bits of w always pass
+  const uint32_t carry = (w & 0x77777777u) + 0x77777777u;
+  return w & (carry | 0x77777777u);
 }
 
 // 8 packed E2M1 codes -> 8 floats (exact: every grid value is an f16).

@@ -77,6 +77,30 @@ static_assert(kCtasPerSm * kTmemCols <= 512, "the resident CTAs' accumulators mu
 
 enum Kind { kQuantize = 0, kAmax = 1, kStoreZ = 2 };
 
+#ifndef NVFP4_MMA_BAND_ROWS
+#define NVFP4_MMA_BAND_ROWS 1
+#endif
+#ifndef NVFP4_MMA_BAND_ROWS_T
+#define NVFP4_MMA_BAND_ROWS_T 16
+#endif
+
+// Tile order: tiles are taken in bands of `band` tile rows, column by column
+// inside a band (tile t -> (rt, ct)), so the tiles in flight at once read
+// long runs of each input row and, for the transposed layout, write long
+// runs of each output row.  32-bit arithmetic: the routing admits fewer than
+// 2^31 tiles.
+struct TileGrid {
+  uint32_t n_rt, n_ct, band;
+  __device__ __forceinline__ void coords(uint32_t t, uint32_t& rt, uint32_t& ct) const {
+    const uint32_t per_band = band * n_ct;
+    const uint32_t bg = t / per_band, r = t - bg * per_band;
+    const uint32_t left = n_rt - bg * band;
+    const uint32_t h = left < band ? left : band;  // tile rows in this band
+    ct = r / h;
+    rt = bg * band + (r - ct * h);
+  }
+};
+
 struct MmaShared {
   uint64_t full[kStagesA];   // A tile landed (TMA transaction bytes)
   uint64_t sfree[kStagesA];  // MMAs reading the A tile are done (tcgen05.commit)
@@ -145,8 +169,9 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
 
   const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
   const PhiloxKey key = philox_key(seed);
-  const int64_t n_ct = (cols + kTile - 1) / kTile;
-  const int64_t n_tiles = ((rows + kTile - 1) / kTile) * n_ct;
+  const TileGrid tg{static_cast<uint32_t>((rows + kTile - 1) / kTile), static_cast<uint32_t>((cols + kTile - 1) / kTile),
+                    static_cast<uint32_t>(ROWWISE ? NVFP4_MMA_BAND_ROWS : NVFP4_MMA_BAND_ROWS_T)};
+  const int64_t n_tiles = static_cast<int64_t>(tg.n_rt) * tg.n_ct;
 
   if (tid == kProducerWarp * 32) {
     for (int s = 0; s < kStagesA; ++s) {
@@ -186,7 +211,8 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
           break;
         }
         if (*reinterpret_cast<volatile int*>(&sh.abort_flag)) break;
-        const int64_t rt = t / n_ct, ct = t - rt * n_ct;
+        uint32_t rt, ct;
+        tg.coords(static_cast<uint32_t>(t), rt, ct);
         const int32_t x = static_cast<int32_t>(ct * kTile), y = static_cast<int32_t>(rt * kTile);
         mbar_arrive_expect_tx(&sh.full[s], kTileBytes);
         uint8_t* dst = a_tiles + s * kTileBytes;
@@ -255,7 +281,8 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
         break;
       }
       tc_fence_after_sync();
-      const int64_t rt = t / n_ct, ct = t - rt * n_ct;
+      uint32_t rt, ct;
+      tg.coords(static_cast<uint32_t>(t), rt, ct);
       // view row of this thread
       const int64_t vrow = (ROWWISE ? rt : ct) * kTile + 32 * q + lane;
       // MS-EDEN scale uniforms: when a thread owns a whole 128-column row of
@@ -461,6 +488,7 @@ bool mma_path_applies(const QuantArgs& a) {
   if (a.rht_group == 0) return false;
   if (a.rows < kTile || a.cols < kTile) return false;
   if (a.rows >= (int64_t(1) << 31) || a.cols >= (int64_t(1) << 31)) return false;
+  if (((a.rows + kTile - 1) / kTile) * ((a.cols + kTile - 1) / kTile) >= (int64_t(1) << 31)) return false;
   // the tensor map needs a 16-byte aligned base and row pitch
   if (reinterpret_cast<uintptr_t>(a.x) % 16 != 0 || a.ld % 8 != 0) return false;
   return encode_fn() != nullptr;
