@@ -62,6 +62,8 @@ def parse_args(argv=None):
                    help="fraction of each call's view rows the CPU baseline quantizes")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-per-mode", action="store_true",
+                   help="skip the per-mode table (every mode on dY, quantize kernel alone)")
     return p.parse_args(argv)
 
 
@@ -212,6 +214,39 @@ class Call:
         return self.codes.numel() + self.scales.numel() + 4
 
 
+def per_mode_table(N, W, x, seed, stream, device, flush, peak, reps=5):
+    """Every mode on one tensor (the headline gradient dY), both layouts, with
+    and without the 128-point rotation: the quantize kernel alone with the
+    tensor amax supplied (from its own pre-pass), CUDA events, L2 flushed
+    before each launch.  MS-EDEN is defined with the rotation only."""
+    from nvfp4_microscaling_quantization_b200.workloads import Call as WCall
+    out = []
+    for layout in (W.ROWWISE, W.TRANSPOSED):
+        for mode in (W.RTN, W.SR, W.MS_EDEN, W.IF4, W.FOUR_OVER_SIX):
+            for g in (0, 128):
+                if mode == W.MS_EDEN and g == 0:
+                    continue
+                c = Call(N, WCall("dy", layout, mode, g), x, seed, stream)
+                c.amax_pass()
+                c.quantize()
+                ts = []
+                for _ in range(reps):
+                    flush.zero_()
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    c.quantize()
+                    b.record()
+                    b.synchronize()
+                    ts.append(a.elapsed_time(b) / 1e3)
+                t = statistics.median(ts)
+                gbs = BYTES_PER_ELEMENT * c.elements / t / 1e9
+                out.append({"call": c.call.name, "us": round(t * 1e6, 1), "gbs": round(gbs, 1),
+                            "frac_of_hbm_peak": round(gbs / peak, 4), "gelem_s": round(c.elements / t / 1e9, 1)})
+                del c
+    torch.cuda.synchronize(device)
+    return out
+
+
 def run_ours(args, world, rank, local):
     import ctypes
     from nvfp4_microscaling_quantization_b200 import binding as N
@@ -290,6 +325,10 @@ def run_ours(args, world, rank, local):
             "quantize_gelem_s": round(c.elements / (quant_ms[i] / 1e3) / 1e9, 1),
         })
 
+    per_mode = None
+    if not args.no_per_mode:
+        per_mode = per_mode_table(N, W, tensors["dy"], wl.seed, sh, device, flush, peak)
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, calls, tensors, stream, device, world, bytes_per_step)
@@ -324,6 +363,8 @@ def run_ours(args, world, rank, local):
         "clocks": clock,
         "kernel_source": src_hash,
     }
+    if per_mode is not None:
+        result["per_mode_dy"] = per_mode
     if e2e is not None:
         result["e2e"] = e2e
     if cpu is not None:

@@ -1,9 +1,11 @@
 // nvfp4_device.cuh -- device building blocks of the NVFP4 quantizer (sm_100a).
 //
 // Every floating-point step that decides a code or a scale is one IEEE
-// binary32 operation with round-to-nearest-even, written with the explicit
-// __f*_rn intrinsics (and the library is built with -fmad=false, so nothing is
-// contracted).  The step order is the method's: rotate, block absmax, block
+// binary32 operation with round-to-nearest-even: scalar steps through the
+// __f*_rn intrinsics, two-lane steps through add/mul/fma .rn.f32x2 written in
+// PTX with the rounding stated (an instruction with an explicit rounding
+// modifier is never fused with another), and the library is built with
+// -fmad=false.  The step order is the method's: rotate, block absmax, block
 // scale, scale to the grid, round, pack.
 #pragma once
 
@@ -14,6 +16,45 @@
 namespace nvfp4 {
 
 enum Mode { kRTN = 0, kSR = 1, kMSEDEN = 2, kIF4 = 3, k4over6 = 4 };
+
+// ---------------------------------------------------------------------------
+// Two-lane binary32 arithmetic (sm_100a f32x2): each lane is one IEEE RN
+// operation.  The explicit .rn keeps a product from being fused into a
+// following add, which would skip the product's rounding.
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+__device__ __forceinline__ unsigned long long pack2(float2 a) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
+  return r;
+}
+__device__ __forceinline__ float2 unpack2(unsigned long long r) {
+  float2 a;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(r));
+  return a;
+}
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pack2(a)), "l"(pack2(b)));
+  return unpack2(d);
+}
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pack2(a)), "l"(pack2(b)));
+  return unpack2(d);
+}
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pack2(a)), "l"(pack2(b)), "l"(pack2(c)));
+  return unpack2(d);
+}
+// a - b per lane: the negation is exact, so each lane is the one RN subtraction.
+__device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) { return add2_rn(a, f2(-b.x, -b.y)); }
+// a + b and a - b lane by lane through the scalar intrinsics, which are never
+// merged with the multiplication that produced b: for a sum whose operand is
+// a rounded product.
+__device__ __forceinline__ float2 add2_after_mul(float2 a, float2 b) { return f2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y)); }
+__device__ __forceinline__ float2 sub2_after_mul(float2 a, float2 b) { return f2(__fsub_rn(a.x, b.x), __fsub_rn(a.y, b.y)); }
 
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy
@@ -237,6 +278,7 @@ __device__ __forceinline__ float global_scale_of(float amax) {
 // INT4 option of IF4: levels k in [-7, 7] standing for k * 6/7.
 constexpr float kIF4K1 = 0x1.2aaaaap+0f;  // RN(7/6)
 constexpr float kIF4K2 = 0x1.b6db6ep-1f;  // RN(6/7)
+constexpr float kRoundMagic = 12582912.0f; // 1.5 * 2^23: RN(t + it) - it = RNE(t) for |t| < 2^22
 
 // Where the random draws of one 16-element block come from.
 struct BlockRng {
@@ -263,18 +305,23 @@ __device__ __forceinline__ void rtn_codes(const float* y, uint32_t& lo, uint32_t
   hi = clear_negative_zero(cvt_e2m1x8(y + 8));
 }
 
-// Stochastic rounding of one scaled value with the uniform k * 2^-16.
+// Stochastic rounding of one scaled value with the uniform U = k * 2^-16:
+// a = min(|y|, 6) between grid neighbours l <= a < u goes up iff
+// U < (a - l) / (u - l), done on the bits of a with no conversion
+// instruction.  For a in [1, 6] the grid keeps one mantissa bit, so
+// (a - l) / (u - l) = low22 / 2^22 (low22 = the 22 mantissa bits below it)
+// and U < that iff 64k < low22 iff low22 + (2^22 - 1 - 64k) carries into
+// the kept bit; the code index is then (bits >> 22) - 252.  For a in
+// [0.5, 1) the same with all 23 mantissa bits (index (bits >> 23) - 125).
+// For a in [0, 0.5) the neighbours are 0 and 0.5 and the fraction is 2a.
 __device__ __forceinline__ uint32_t sr_code(float y, uint32_t k16) {
   const float a = fminf(fabsf(y), 6.0f);
-  // grid interval: [0,2) step 1/2, [2,4) step 1, [4,6] step 2
-  const float inv_step = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
-  const uint32_t base = a < 2.0f ? 0u : (a < 4.0f ? 2u : 4u);
-  const float t = __fmul_rn(a, inv_step);  // exact
-  const float fl = floorf(t);
-  const float frac = __fsub_rn(t, fl);     // exact: position inside the interval
-  uint32_t mag = static_cast<uint32_t>(fl) + base;
-  const float U = uniform16(k16);
-  if (U < frac) ++mag;
+  const uint32_t b = __float_as_uint(a);
+  const uint32_t x22 = 0x3FFFFFu - 64u * k16;        // 2^22 - 1 - 64k >= 63
+  const uint32_t i1 = (b + x22 - (252u << 22)) >> 22;  // a >= 1
+  const uint32_t i2 = (b + 2u * x22 + 1u - (125u << 23)) >> 23;  // a in [0.5, 1): 2^23 - 1 - 128k
+  const uint32_t i3 = uniform16(k16) < __fadd_rn(a, a) ? 1u : 0u;  // a < 0.5
+  const uint32_t mag = a >= 1.0f ? i1 : (a >= 0.5f ? i2 : i3);
   if (mag == 0u) return 0u;
   return mag | (y < 0.0f ? 8u : 0u);
 }
@@ -411,8 +458,6 @@ struct PairRng {
   float u_a, u_b;           // scale uniforms of block a / b (MS-EDEN)
 };
 
-__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
-
 // Per-launch constants of the block-scale step: the tensor scale s_g, the
 // divisors q6 = RN(6 s_g) and q4 = RN(4 s_g) of s_f = RN(absmax / q), and
 // their round-to-nearest reciprocals for the division below.
@@ -444,17 +489,15 @@ __device__ __forceinline__ ScaleCtx make_scale_ctx(float amax) {
 __device__ __forceinline__ float2 div2_by(float2 a, float q, float r, bool markstein) {
   if (!markstein) return f2(__fdiv_rn(a.x, q), __fdiv_rn(a.y, q));
   const float2 q2 = f2(q, q), r2 = f2(r, r);
-  const float2 t = __fmul2_rn(a, r2);
-  const float2 rem = __ffma2_rn(f2(-t.x, -t.y), q2, a);
-  const float2 d = __ffma2_rn(rem, r2, t);
+  const float2 t = mul2_rn(a, r2);
+  const float2 rem = fma2_rn(f2(-t.x, -t.y), q2, a);
+  const float2 d = fma2_rn(rem, r2, t);
   // a quotient that overflows (an absmax far above the tensor amax given)
   // comes out NaN here and infinite from the division; both saturate the
   // E4M3 scale, and so does 1024
   return f2(fminf(d.x, 1024.0f), fminf(d.y, 1024.0f));
 }
 
-// a - b per lane: the negation is exact, so each lane is the one RN subtraction.
-__device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) { return __fadd2_rn(a, f2(-b.x, -b.y)); }
 
 // E4M3 RNE of two non-negative floats in one conversion: .x -> bits 0..7, .y -> bits 8..15.
 __device__ __forceinline__ uint32_t e4m3x2_rne_sat(float a, float b) {
@@ -483,8 +526,8 @@ __device__ __forceinline__ uint32_t e4m3x2_sr(float2 t, float ua, float ub) {
   lo -= (d.x > t.x ? 1u : 0u) + (d.y > t.y ? 0x100u : 0u);
   const float2 l = e4m3x2_decode(lo);
   const float2 h = e4m3x2_decode(lo + 0x0101u);
-  const float2 below = __fmul2_rn(f2(ua, ub), sub2_rn(h, l));  // exact: the gap is a power of two
-  const float2 above = sub2_rn(t, l);                          // exact
+  const float2 below = mul2_rn(f2(ua, ub), sub2_rn(h, l));  // exact: the gap is a power of two
+  const float2 above = sub2_after_mul(t, l);                   // exact (t is a rounded product)
   return lo + (below.x < above.x ? 1u : 0u) + (below.y < above.y ? 0x100u : 0u);
 }
 
@@ -546,12 +589,12 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
       const float2 sf = k == 0 ? div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein)
                                : div2_by(f2(aa, ab), sc.q4, sc.r4, sc.markstein);
       S[k] = e4m3x2_rne_sat(sf.x, sf.y);
-      const float2 d = __fmul2_rn(e4m3x2_decode(S[k]), sg2);
+      const float2 d = mul2_rn(e4m3x2_decode(S[k]), sg2);
       const float2 r = rcp_or_zero(d);
       float ya[16], yb[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float2 y = __fmul2_rn(z[i], r);
+        const float2 y = mul2_rn(z[i], r);
         ya[i] = y.x;
         yb[i] = y.y;
       }
@@ -565,8 +608,8 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
       float2 e = f2(0.0f, 0.0f);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float2 diff = sub2_rn(z[i], __fmul2_rn(f2(va[i], vb[i]), d));
-        e = __ffma2_rn(diff, diff, e);
+        const float2 diff = sub2_after_mul(z[i], mul2_rn(f2(va[i], vb[i]), d));
+        e = fma2_rn(diff, diff, e);
       }
       err[k] = e;
     }
@@ -591,12 +634,12 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
     }
     oa.scale = Sa;
     ob.scale = Sb;
-    const float2 d = __fmul2_rn(dS, sg2);
+    const float2 d = mul2_rn(dS, sg2);
     const float2 r = rcp_or_zero(d);
     float ya[16], yb[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const float2 y = __fmul2_rn(z[i], r);
+      const float2 y = mul2_rn(z[i], r);
       ya[i] = y.x;
       yb[i] = y.y;
     }
@@ -618,13 +661,13 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float2 y = f2(ya[i], yb[i]);
-        num = __ffma2_rn(y, y, num);
-        den = __ffma2_rn(y, f2(va[i], vb[i]), den);
+        num = fma2_rn(y, y, num);
+        den = fma2_rn(y, f2(va[i], vb[i]), den);
       }
       const float qa = __fdiv_rn(num.x, den.x), qb = __fdiv_rn(num.y, den.y);
       const float ca = (num.x > 0.0f && den.x > 0.0f) ? qa : 1.0f;
       const float cb = (num.y > 0.0f && den.y > 0.0f) ? qb : 1.0f;
-      const uint32_t S = e4m3x2_sr(__fmul2_rn(dS, f2(ca, cb)), rng.u_a, rng.u_b);
+      const uint32_t S = e4m3x2_sr(mul2_rn(dS, f2(ca, cb)), rng.u_a, rng.u_b);
       oa.scale = S & 0xFFu;
       ob.scale = S >> 8;
     } else {  // kIF4
@@ -641,16 +684,23 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float2 y = f2(ya[i], yb[i]);
-        const float2 dF = sub2_rn(y, f2(va[i], vb[i]));
-        eF = __ffma2_rn(dF, dF, eF);
-        const float2 t = __fmul2_rn(y, f2(kIF4K1, kIF4K1));
-        const int ka = max(-7, min(7, __float2int_rn(t.x)));
-        const int kb = max(-7, min(7, __float2int_rn(t.y)));
-        const float2 vi = __fmul2_rn(f2(static_cast<float>(ka), static_cast<float>(kb)), f2(kIF4K2, kIF4K2));
-        const float2 dI = sub2_rn(y, vi);
-        eI = __ffma2_rn(dI, dI, eI);
-        const uint32_t codea = ka == 0 ? 0u : (static_cast<uint32_t>(ka < 0 ? -ka : ka) | (ka < 0 ? 8u : 0u));
-        const uint32_t codeb = kb == 0 ? 0u : (static_cast<uint32_t>(kb < 0 ? -kb : kb) | (kb < 0 ? 8u : 0u));
+        const float2 dF = sub2_after_mul(y, f2(va[i], vb[i]));
+        eF = fma2_rn(dF, dF, eF);
+        const float2 t = mul2_rn(y, f2(kIF4K1, kIF4K1));
+        // k = clamp(RNE(t), -7, 7) with no conversion instruction: |t| < 2^22,
+        // so s = RN(t + 1.5 * 2^23) rounds t at the units bit (ties to even),
+        // s - 1.5 * 2^23 = RNE(t) exactly, and the bits of s are 0x4B400000 + RNE(t)
+        const float2 s2 = add2_after_mul(t, f2(kRoundMagic, kRoundMagic));
+        const float2 r2 = sub2_rn(s2, f2(kRoundMagic, kRoundMagic));
+        const float2 kf = f2(fminf(fmaxf(r2.x, -7.0f), 7.0f), fminf(fmaxf(r2.y, -7.0f), 7.0f));
+        const int ka = max(-7, min(7, static_cast<int>(__float_as_uint(s2.x) - 0x4B400000u)));
+        const int kb = max(-7, min(7, static_cast<int>(__float_as_uint(s2.y) - 0x4B400000u)));
+        const float2 vi = mul2_rn(kf, f2(kIF4K2, kIF4K2));
+        const float2 dI = sub2_after_mul(y, vi);
+        eI = fma2_rn(dI, dI, eI);
+        // sign-magnitude nibble; k = 0 gives 0
+        const uint32_t codea = static_cast<uint32_t>(abs(ka)) | ((static_cast<uint32_t>(ka) >> 28) & 8u);
+        const uint32_t codeb = static_cast<uint32_t>(abs(kb)) | ((static_cast<uint32_t>(kb) >> 28) & 8u);
         if (i < 8) {
           ia_lo |= codea << (4 * i);
           ib_lo |= codeb << (4 * i);

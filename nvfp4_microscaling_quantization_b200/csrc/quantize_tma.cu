@@ -117,7 +117,7 @@ __device__ __forceinline__ void rotate64(float2 (&z)[2][16], bool upper_half) {
       for (int i = 0; i < 16; ++i) {
         if (i & h) continue;
         const float2 a = z[p][i], b = z[p][i + h];
-        z[p][i] = __fadd2_rn(a, b);
+        z[p][i] = add2_rn(a, b);
         z[p][i + h] = sub2_rn(a, b);
       }
   }
@@ -134,7 +134,7 @@ __device__ __forceinline__ void rotate64(float2 (&z)[2][16], bool upper_half) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float2 a = z[0][i], b = z[1][i];
-      z[0][i] = __fadd2_rn(a, b);
+      z[0][i] = add2_rn(a, b);
       z[1][i] = sub2_rn(a, b);
     }
   }
@@ -147,14 +147,14 @@ __device__ __forceinline__ void rotate64(float2 (&z)[2][16], bool upper_half) {
       for (int i = 0; i < 16; ++i) {
         const float2 other =
             f2(__shfl_xor_sync(0xFFFFFFFFu, z[p][i].x, 16), __shfl_xor_sync(0xFFFFFFFFu, z[p][i].y, 16));
-        z[p][i] = __ffma2_rn(sgn, z[p][i], other);
+        z[p][i] = fma2_rn(sgn, z[p][i], other);
       }
   }
   const float2 c2 = f2(RhtConst<G>::c, RhtConst<G>::c);
 #pragma unroll
   for (int p = 0; p < 2; ++p)
 #pragma unroll
-    for (int i = 0; i < 16; ++i) z[p][i] = __fmul2_rn(z[p][i], c2);
+    for (int i = 0; i < 16; ++i) z[p][i] = mul2_rn(z[p][i], c2);
 }
 
 // -------------------------------------------------------------- the kernel

@@ -314,7 +314,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
 #pragma unroll
           for (int p = 0; p < 2; ++p)
 #pragma unroll
-            for (int i = 0; i < 16; ++i) z[p][i] = __fmul2_rn(f2(v[32 * p + 2 * i], v[32 * p + 2 * i + 1]), c2);
+            for (int i = 0; i < 16; ++i) z[p][i] = mul2_rn(f2(v[32 * p + 2 * i], v[32 * p + 2 * i + 1]), c2);
           if (vrow < vrows && vcol0 < vcols)
             quantize_store64<MODE>(z, sc, key, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);
         } else if constexpr (KIND == kQuantize) {
@@ -342,7 +342,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
             }
             float2 zp[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) zp[i] = __fmul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
+            for (int i = 0; i < 16; ++i) zp[i] = mul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
             const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, u[2 * p], u[2 * p + 1]};
             quantize_pair<MODE>(zp, sc, rng, o[2 * p], o[2 * p + 1]);
           }
@@ -360,7 +360,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
             }
             float2 zp[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) zp[i] = __fmul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
+            for (int i = 0; i < 16; ++i) zp[i] = mul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
             if constexpr (KIND == kAmax) {
               float ma, mb;
               absmax_pair(zp, ma, mb);

@@ -297,3 +297,24 @@ def test_outputs_at_8_byte_offsets(layout, mode, g):
     assert_same((got_c, got_s, float(gs.item())), gpu_quantize(xd, layout, mode, g, 21))
     if g == 0:
         assert_same((got_c, got_s, float(gs.item())), oracle.quantize(bits(x), layout, mode, g, 21))
+
+
+def test_if4_int4_rounding_ties():
+    """IF4 blocks that take the scaled-INT4 option and hold y = 3.0, whose
+    RN(y * RN(7/6)) is exactly 3.5: the level is RNE(3.5) = 4 only if the
+    product is rounded before the level is (a fused multiply-add would give 3).
+
+    amax_in = 10.5 gives s_g = 2^-8; with a 6.0 in every block the block scale
+    is 256 and d = 1, so y = x.  The other values sit near the INT4 levels
+    k * 6/7 so that the INT4 option wins."""
+    levels = np.array([k * 6.0 / 7.0 for k in range(-7, 8)], dtype=np.float32)
+    rng = np.random.default_rng(17)
+    rows, cols = 64, 256
+    blocks = rng.choice(levels, size=(rows * cols // 16, 16)).astype(np.float32)
+    blocks[:, 0] = 6.0
+    pos = 1 + rng.integers(0, 15, len(blocks))
+    blocks[np.arange(len(blocks)), pos] = np.where(rng.random(len(blocks)) < 0.5, 3.0, -3.0)
+    x = torch.from_numpy(blocks.reshape(rows, cols)).to(torch.bfloat16)
+    gpu = compare_call(x, W.ROWWISE, W.IF4, 0, 5, amax=10.5)
+    flagged = int(np.sum(gpu[1] >= 0x80))
+    assert flagged > len(blocks) // 2, f"only {flagged} of {len(blocks)} blocks took the INT4 option"
