@@ -5,8 +5,9 @@ One step quantizes the tensors of one Llama-style MLP up-projection training
 step (X 16384x4096, W 14336x4096, dY 16384x14336, bf16) the way a fully-NVFP4
 linear layer needs them: RTN on X and W along d_model (forward), MS-EDEN with
 a 128-point random Hadamard rotation on dY row-wise and transposed, and on X
-and W transposed (backward) -- six calls, each the tensor-amax pre-pass then
-the quantization kernel, through the library's C ABI.
+and W transposed (backward) -- six quantize calls through the library's C
+ABI, each tensor's two tensor amaxes first, from one read of the tensor
+(nvfp4_amax_dual).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -214,6 +215,34 @@ class Call:
         return self.codes.numel() + self.scales.numel() + 4
 
 
+class TensorCalls:
+    """The calls on one tensor.  A tensor quantized in both layouts gets its
+    two tensor amaxes from one nvfp4_amax_dual pre-pass (one read of the
+    tensor); any other set of calls runs one pre-pass per call."""
+
+    def __init__(self, N, calls):
+        self.N, self.calls = N, calls
+        layouts = sorted(c.call.layout for c in calls)
+        self.dual = len(calls) == 2 and layouts == [0, 1]
+        if self.dual:
+            self.row = next(c for c in calls if c.call.layout == 0)
+            self.col = next(c for c in calls if c.call.layout == 1)
+
+    def amax_passes(self):
+        if not self.dual:
+            for c in self.calls:
+                c.amax_pass()
+            return
+        r, c = self.row, self.col
+        st = self.N.nvfp4_amax_dual(r.p["x"], r.rows, r.cols, r.ld, r.call.rht_group, c.call.rht_group, r.seed,
+                                    r.p["amax"], c.p["amax"], r.stream)
+        if st:
+            raise self.N.Nvfp4Error(st, "nvfp4_amax_dual")
+
+    def launches(self):
+        return (1 if self.dual else len(self.calls)) + len(self.calls)
+
+
 def per_mode_table(N, W, x, seed, stream, device, flush, peak, reps=5):
     """Every mode on one tensor (the headline gradient dY), both layouts, with
     and without the 128-point rotation: the quantize kernel alone with the
@@ -261,20 +290,28 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(device)
     sh = ctypes.c_void_p(stream.cuda_stream)
     calls = [Call(N, c, tensors[c.tensor], wl.seed, sh) for c in wl.calls]
+    groups = [TensorCalls(N, [c for c in calls if c.call.tensor == name])
+              for name in dict.fromkeys(c.tensor for c in wl.calls)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     bytes_per_step = sum(BYTES_PER_ELEMENT * c.elements for c in calls)
     elems_per_step = sum(c.elements for c in calls)
 
+    # per step: for each tensor its pre-pass(es), then its quantize calls;
+    # events: [pre-pass start, pre-pass end] per tensor, [start, end] per call
     def step(evs=None):
-        for i, c in enumerate(calls):
+        for gi, grp in enumerate(groups):
             if evs is not None:
-                evs[i][0].record(stream)
-            c.amax_pass()
+                evs["amax"][gi][0].record(stream)
+            grp.amax_passes()
             if evs is not None:
-                evs[i][1].record(stream)
-            c.quantize()
-            if evs is not None:
-                evs[i][2].record(stream)
+                evs["amax"][gi][1].record(stream)
+            for c in grp.calls:
+                i = calls.index(c)
+                if evs is not None:
+                    evs["quant"][i][0].record(stream)
+                c.quantize()
+                if evs is not None:
+                    evs["quant"][i][1].record(stream)
 
     for _ in range(max(args.warmup, 0)):
         flush.zero_()
@@ -284,7 +321,8 @@ def run_ours(args, world, rank, local):
     K = args.steps
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     starts, ends = [ev() for _ in range(K)], [ev() for _ in range(K)]
-    call_evs = [[[ev(), ev(), ev()] for _ in calls] for _ in range(K)]
+    call_evs = [{"amax": [[ev(), ev()] for _ in groups], "quant": [[ev(), ev()] for _ in calls]}
+                for _ in range(K)]
     with ClockSampler(local) as clocks:
         barrier(world, local)
         torch.cuda.synchronize(device)
@@ -299,10 +337,10 @@ def run_ours(args, world, rank, local):
 
     step_ms = [starts[k].elapsed_time(ends[k]) for k in range(K)]
     total_s = max_over_ranks(sum(step_ms) / 1e3, world, device)
-    amax_ms = [statistics.mean(call_evs[k][i][0].elapsed_time(call_evs[k][i][1]) for k in range(K))
-               for i in range(len(calls))]
-    quant_ms = [statistics.mean(call_evs[k][i][1].elapsed_time(call_evs[k][i][2]) for k in range(K))
-                for i in range(len(calls))]
+    amax_ms = [statistics.mean(call_evs[k]["amax"][g][0].elapsed_time(call_evs[k]["amax"][g][1]) for k in range(K))
+               for g in range(len(groups))]
+    quant_ms = [statistics.mean(call_evs[k]["quant"][i][0].elapsed_time(call_evs[k]["quant"][i][1])
+                                for k in range(K)) for i in range(len(calls))]
     quant_total_s = max_over_ranks(sum(quant_ms) * K / 1e3, world, device)
     value = weak_scaling_value(bytes_per_step, K, world, total_s)
     value_supplied = weak_scaling_value(bytes_per_step, K, world, quant_total_s)
@@ -319,10 +357,17 @@ def run_ours(args, world, rank, local):
     for i, c in enumerate(calls):
         per_call.append({
             "call": c.call.name, "elements": c.elements,
-            "quantize_us": round(quant_ms[i] * 1e3, 2), "amax_us": round(amax_ms[i] * 1e3, 2),
+            "quantize_us": round(quant_ms[i] * 1e3, 2),
             "quantize_gbs": round(BYTES_PER_ELEMENT * c.elements / (quant_ms[i] / 1e3) / 1e9, 1),
-            "amax_gbs": round(PREPASS_BYTES_PER_ELEMENT * c.elements / (amax_ms[i] / 1e3) / 1e9, 1),
             "quantize_gelem_s": round(c.elements / (quant_ms[i] / 1e3) / 1e9, 1),
+        })
+    pre_passes = []
+    for g, grp in enumerate(groups):
+        read = PREPASS_BYTES_PER_ELEMENT * grp.calls[0].elements
+        pre_passes.append({
+            "tensor": grp.calls[0].call.tensor, "kind": "dual" if grp.dual else "single",
+            "for_calls": [c.call.name for c in grp.calls], "us": round(amax_ms[g] * 1e3, 2),
+            "read_gbs": round(read / (amax_ms[g] / 1e3) / 1e9, 1),
         })
 
     per_mode = None
@@ -346,7 +391,8 @@ def run_ours(args, world, rank, local):
             "workload": "mlp_up: one Llama-style MLP up-projection training step's tensors, "
                         "X 16384x4096 N(0,1), W 14336x4096 N(0,0.02^2), dY 16384x14336 Student-t3 std 1e-4",
             "calls": [c.call.name for c in calls],
-            "path": "per call: tensor-amax pre-pass kernel + quantize kernel (C ABI), one stream",
+            "path": "per tensor: one tensor-amax pre-pass for both layouts (nvfp4_amax_dual), then its "
+                    "quantize kernels (C ABI), one stream",
             "input_dtype": "bf16", "l2": "flushed before every timed step (256 MiB write, untimed)",
             "parallelism": f"replicas x{world} (independent tensors per rank)",
         },
@@ -359,7 +405,8 @@ def run_ours(args, world, rank, local):
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_bytes": int(dom_bytes), "avg_launch_us": round(quant_ms[dom] * 1e3, 2)},
         "per_call": per_call,
-        "gpu_launches": 2 * len(calls) * K,
+        "amax_pre_passes": pre_passes,
+        "gpu_launches": sum(g.launches() for g in groups) * K,
         "clocks": clock,
         "kernel_source": src_hash,
     }
@@ -385,12 +432,16 @@ def run_e2e(args, calls, tensors, stream, device, world, bytes_per_step):
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(c.output_bytes() for c in calls)
 
+    groups = [TensorCalls(calls[0].N, [c for c in calls if c.call.tensor == name])
+              for name in dict.fromkeys(c.call.tensor for c in calls)]
+
     def e2e_step():
         for k, t in tensors.items():
             t.copy_(host_in[k], non_blocking=True)
-        for c in calls:
-            c.amax_pass()
-            c.quantize()
+        for grp in groups:
+            grp.amax_passes()
+            for c in grp.calls:
+                c.quantize()
         for c, (hc, hs, hg) in zip(calls, host_out):
             hc.copy_(c.codes, non_blocking=True)
             hs.copy_(c.scales, non_blocking=True)

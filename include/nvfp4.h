@@ -103,6 +103,22 @@ NVFP4_API size_t nvfp4_workspace_bytes(int64_t rows, int64_t cols, int layout, i
 NVFP4_API int nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int layout,
                int rht_group, uint64_t seed, float* amax_out, void* stream);
 
+/* Both layouts' tensor amax from one read of x: *amax_row = nvfp4_amax of the
+ * row-wise view with rotation group rht_group_row, *amax_col = nvfp4_amax of
+ * the transposed view with rht_group_col (either may be 0), same seed; the
+ * two values equal those of the two single calls bit for bit.  A fully-NVFP4
+ * linear layer quantizes each of W, X and dY in both orientations (forward
+ * along one dimension, backward along the other: Quartet II article, section
+ * "Quantisierung im Vorwaertsdurchlauf", W and X re-quantized for the
+ * backward pass), so reading the tensor once for both pre-passes halves
+ * their HBM traffic.  Shape rules: those of nvfp4_amax for each layout
+ * (cols a multiple of 16 and of rht_group_row, rows a multiple of 16 and of
+ * rht_group_col, cols a multiple of 8).  amax_row, amax_col: device floats,
+ * overwritten.  Tensors too small for the fused kernel run as two pre-passes. */
+NVFP4_API int nvfp4_amax_dual(const void* x, int64_t rows, int64_t cols, int64_t ld, int rht_group_row,
+                              int rht_group_col, uint64_t seed, float* amax_row, float* amax_col,
+                              void* stream);
+
 /* Quantize x to packed E2M1/INT4 codes, E4M3 block scales and the FP32
  * tensor scale, in the given layout and mode (see the conventions above).
  *  amax_in:   device float holding the tensor amax of the (rotated) view, or

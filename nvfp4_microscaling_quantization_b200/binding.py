@@ -43,6 +43,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_workspace_bytes.restype = sz
         L.nvfp4_amax.argtypes = [P, i64, i64, i64, i32, i32, u64, P, P]
         L.nvfp4_amax.restype = i32
+        L.nvfp4_amax_dual.argtypes = [P, i64, i64, i64, i32, i32, u64, P, P, P]
+        L.nvfp4_amax_dual.restype = i32
         L.nvfp4_quantize.argtypes = [P, i64, i64, i64, i32, i32, i32, u64, P, P, P, P, P, sz, P]
         L.nvfp4_quantize.restype = i32
         L.nvfp4_dequantize.argtypes = [P, P, P, i64, i64, i32, i32, u64, i32, P, P]
@@ -72,6 +74,11 @@ def nvfp4_workspace_bytes(rows, cols, layout, mode, rht_group) -> int:
 
 def nvfp4_amax(x, rows, cols, ld, layout, rht_group, seed, amax_out, stream) -> int:
     return lib().nvfp4_amax(x, rows, cols, ld, layout, rht_group, seed, amax_out, stream)
+
+
+def nvfp4_amax_dual(x, rows, cols, ld, rht_group_row, rht_group_col, seed, amax_row, amax_col, stream) -> int:
+    return lib().nvfp4_amax_dual(x, rows, cols, ld, rht_group_row, rht_group_col, seed, amax_row, amax_col,
+                                 stream)
 
 
 def nvfp4_quantize(x, rows, cols, ld, layout, mode, rht_group, seed, amax_in, codes, scales,
@@ -141,6 +148,16 @@ def amax(x: torch.Tensor, layout: int = ROWWISE, rht_group: int = 0, seed: int =
     _check(nvfp4_amax(_p(x), rows, cols, ld, layout, rht_group, seed, _p(out), _stream_handle(stream)),
            "nvfp4_amax")
     return out
+
+
+def amax_dual(x: torch.Tensor, rht_group_row: int = 0, rht_group_col: int = 0, seed: int = 0,
+              stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(amax of the row-wise view, amax of the transposed view) from one read of x."""
+    rows, cols, ld = _matrix(x, torch.bfloat16)
+    out = torch.empty(2, dtype=torch.float32, device=x.device)
+    _check(nvfp4_amax_dual(_p(x), rows, cols, ld, rht_group_row, rht_group_col, seed, _p(out[0:1]),
+                           _p(out[1:2]), _stream_handle(stream)), "nvfp4_amax_dual")
+    return out[0:1], out[1:2]
 
 
 def alloc_outputs(rows: int, cols: int, layout: int, device) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:

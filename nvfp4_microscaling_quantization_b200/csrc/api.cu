@@ -60,6 +60,29 @@ int nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int layout
   return from_cuda(nvfp4::launch_amax(a));
 }
 
+int nvfp4_amax_dual(const void* x, int64_t rows, int64_t cols, int64_t ld, int rht_group_row,
+                    int rht_group_col, uint64_t seed, float* amax_row, float* amax_col, void* stream) {
+  int64_t vr, vc;
+  int st = check_tensor(x, rows, cols, ld, NVFP4_ROWWISE, rht_group_row, &vr, &vc);
+  if (st) return st;
+  if ((st = check_tensor(x, rows, cols, ld, NVFP4_TRANSPOSED, rht_group_col, &vr, &vc))) return st;
+  if (!amax_row || !amax_col) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(amax_row, 4) || !aligned(amax_col, 4)) return NVFP4_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = from_cuda(cudaMemsetAsync(amax_row, 0, sizeof(float), s)))) return st;
+  if ((st = from_cuda(cudaMemsetAsync(amax_col, 0, sizeof(float), s)))) return st;
+  if (rows > 0 && cols > 0 && nvfp4::dual_mma_path_applies(x, rows, cols, ld))
+    return from_cuda(nvfp4::launch_amax_dual_mma(x, rows, cols, ld, rht_group_row, rht_group_col, seed, amax_row,
+                                                 amax_col, s));
+  nvfp4::QuantArgs a{x, rows, cols, ld, NVFP4_ROWWISE, NVFP4_RTN, rht_group_row, seed, nullptr, amax_row,
+                     nullptr, nullptr, nullptr, s};
+  if ((st = from_cuda(nvfp4::launch_amax(a)))) return st;
+  a.layout = NVFP4_TRANSPOSED;
+  a.rht_group = rht_group_col;
+  a.amax_accum = amax_col;
+  return from_cuda(nvfp4::launch_amax(a));
+}
+
 int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int layout, int mode,
                    int rht_group, uint64_t seed, const float* amax_in, uint8_t* codes,
                    uint8_t* scales, float* global_scale, void* workspace, size_t workspace_bytes,

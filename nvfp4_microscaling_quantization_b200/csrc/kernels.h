@@ -63,6 +63,14 @@ bool mma_path_applies(const QuantArgs& a);
 cudaError_t launch_amax_mma(const QuantArgs& a);
 cudaError_t launch_quantize_mma(const QuantArgs& a);
 cudaError_t launch_rotate_mma(const QuantArgs& a, float* zout);
+
+// Both layouts' tensor amax from one read (rotate_mma.cu): row-wise view with
+// rotation group g_r, transposed view with g_c (0 = no rotation).  amax_r and
+// amax_c are zeroed 32-bit accumulators.  Applies where the single-layout
+// tensor-core path does (both dimensions >= 128, 16-byte aligned rows).
+bool dual_mma_path_applies(const void* x, int64_t rows, int64_t cols, int64_t ld);
+cudaError_t launch_amax_dual_mma(const void* x, int64_t rows, int64_t cols, int64_t ld, int g_r, int g_c,
+                                 uint64_t seed, float* amax_r, float* amax_c, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantArgs& a);
 cudaError_t launch_rht(const RhtArgs& a);
 cudaError_t launch_encode_e2m1(const float* in, int64_t n, uint8_t* out, cudaStream_t stream);

@@ -417,6 +417,245 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
   }
 }
 
+// ------------------------------------------------------- both layouts at once
+// The tensor amax of the row-wise view (rotated along rows with group g_r)
+// and of the transposed view (rotated along columns with group g_c) from one
+// read of X: every tile goes through two MMAs, the K-major one against B_r
+// and the MN-major one against B_c (g = 0: the identity, z = x exactly), into
+// the two accumulators of the epilogue group that takes the tile.  The
+// results are those of two single-layout pre-passes bit for bit (the same
+// MMAs, the same scaling).  Two epilogue groups, each owning two 128-column
+// accumulators (all 512 columns); in a group of eight warps, warp (q, j)
+// reads lane quarter q of the row-view (j = 0) or column-view (j = 1)
+// accumulator, 64 columns per load.
+
+#ifndef NVFP4_DUAL_STAGES
+#define NVFP4_DUAL_STAGES 3
+#endif
+constexpr int kDualStages = NVFP4_DUAL_STAGES;  // A tiles in flight (each held until both MMAs are done)
+constexpr int kDualGroups = 2;
+constexpr int kDualEpiWarps = 8 * kDualGroups;
+constexpr int kDualThreads = (kDualEpiWarps + 2) * 32;
+constexpr int kDualProducerWarp = kDualEpiWarps, kDualMmaWarp = kDualEpiWarps + 1;
+constexpr size_t kDualDynSmem = (kDualStages + 2) * kTileBytes + 1024;
+
+struct DualShared {
+  uint64_t full[kDualStages];
+  uint64_t sfree[kDualStages];
+  uint64_t tfull[kDualGroups];   // both accumulators of the group ready
+  uint64_t tfree[kDualGroups];   // both loaded by the group
+  uint32_t tmem_base;
+  uint32_t issued_a;
+  uint32_t issued_mma;
+  int abort_flag;
+  unsigned int warp_max[2][kDualEpiWarps];
+};
+
+__device__ __forceinline__ float rht_scale_of(int g) {
+  return g == 16 ? RhtConst<16>::c : g == 32 ? RhtConst<32>::c : g == 64 ? RhtConst<64>::c
+                                                                         : g == 128 ? RhtConst<128>::c : 1.0f;
+}
+
+// B for a rotation group g chosen at run time, laid out like build_hadamard_b;
+// g = 0 gives the identity (row r holds output column output_col_of(r)).
+__device__ __forceinline__ void build_rotation_b(uint8_t* bmat, PhiloxKey key, uint32_t tid, uint32_t nthreads,
+                                                 int g) {
+  const uint4 w = philox_call(key, 0, kTagSigns);
+  const uint32_t gg = g > 0 ? static_cast<uint32_t>(g) : 1u;
+  for (uint32_t c = tid; c < 2048; c += nthreads) {
+    const uint32_t half = c >> 10, r = (c >> 3) & 127u, kc = c & 7u;
+    const uint32_t n = output_col_of(r);
+    uint32_t packed[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t two = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t k = half * 64 + kc * 8 + 2 * i + h;
+        uint32_t v = 0;
+        if (g == 0) {
+          v = n == k ? 0x3F80u : 0u;
+        } else if (n / gg == k / gg) {
+          const uint32_t kg = k % gg, ng = n % gg;
+          const uint32_t neg = ((word_of(w, kg >> 5) >> (kg & 31)) ^ __popc(ng & kg)) & 1u;
+          v = neg ? 0xBF80u : 0x3F80u;
+        }
+        two |= v << (16 * h);
+      }
+      packed[i] = two;
+    }
+    *reinterpret_cast<uint4*>(bmat + half * kBoxBytes + r * 128 + ((kc ^ (r & 7u)) << 4)) =
+        make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  }
+}
+
+__global__ void __launch_bounds__(kDualThreads, 1)
+dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed, int g_r,
+                 int g_c, unsigned int* __restrict__ amax_r, unsigned int* __restrict__ amax_c) {
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ __align__(8) DualShared sh;
+  uint8_t* a_tiles = align_1024(dyn_smem);
+  uint8_t* b_r = a_tiles + kDualStages * kTileBytes;
+  uint8_t* b_c = b_r + kTileBytes;
+
+  const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+  const PhiloxKey key = philox_key(seed);
+  const TileGrid tg{static_cast<uint32_t>((rows + kTile - 1) / kTile), static_cast<uint32_t>((cols + kTile - 1) / kTile),
+                    static_cast<uint32_t>(NVFP4_MMA_BAND_ROWS)};
+  const int64_t n_tiles = static_cast<int64_t>(tg.n_rt) * tg.n_ct;
+
+  if (tid == kDualProducerWarp * 32) {
+    for (int s = 0; s < kDualStages; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.sfree[s], 1);
+    }
+    for (int a = 0; a < kDualGroups; ++a) {
+      mbar_init(&sh.tfull[a], 1);
+      mbar_init(&sh.tfree[a], 8);
+    }
+    sh.issued_a = 0;
+    sh.issued_mma = 0;
+    sh.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kDualMmaWarp) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  build_rotation_b(b_r, key, tid, kDualThreads, g_r);
+  build_rotation_b(b_c, key, tid, kDualThreads, g_c);
+  fence_proxy_async_smem();
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = sh.tmem_base;
+  const int64_t step = gridDim.x;
+
+  if (warp == kDualProducerWarp) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmap);
+      int k = 0;
+      for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++k) {
+        const int s = k % kDualStages;
+        const uint32_t u = k / kDualStages;
+        if (k >= kDualStages && !mbar_wait(&sh.sfree[s], (u - 1) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        if (*reinterpret_cast<volatile int*>(&sh.abort_flag)) break;
+        uint32_t rt, ct;
+        tg.coords(static_cast<uint32_t>(t), rt, ct);
+        const int32_t x = static_cast<int32_t>(ct * kTile), y = static_cast<int32_t>(rt * kTile);
+        mbar_arrive_expect_tx(&sh.full[s], kTileBytes);
+        uint8_t* dst = a_tiles + s * kTileBytes;
+        tma_load_2d(dst, &tmap, x, y, &sh.full[s]);
+        tma_load_2d(dst + kBoxBytes, &tmap, x + 64, y, &sh.full[s]);
+        sh.issued_a = (sh.issued_a & ~(0x101u << s)) | (1u << s) | ((u & 1u) << (8 + s));
+      }
+    }
+  } else if (warp == kDualMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_r = idesc_bf16_f32(kTile, kTile, 0u);
+      constexpr uint32_t idesc_c = idesc_bf16_f32(kTile, kTile, 1u);
+      const uint32_t br_addr = smem_u32(b_r), bc_addr = smem_u32(b_c);
+      int k = 0;
+      for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++k) {
+        const int s = k % kDualStages, a = k % kDualGroups;
+        const uint32_t use = k / kDualGroups;
+        if (!mbar_wait(&sh.full[s], (k / kDualStages) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        if (use > 0 && !mbar_wait(&sh.tfree[a], (use - 1) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t a_addr = smem_u32(a_tiles + s * kTileBytes);
+        const uint32_t d_r = tmem_base + a * 256, d_c = d_r + 128;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          const uint64_t adesc = smem_desc_sw128(a_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(br_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+          umma_bf16(d_r, adesc, bdesc, idesc_r, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          const uint64_t adesc = smem_desc_sw128(a_addr + kk * 2048, kBoxBytes, 1024);
+          const uint64_t bdesc = smem_desc_sw128(bc_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+          umma_bf16(d_c, adesc, bdesc, idesc_c, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&sh.sfree[s]);
+        umma_commit(&sh.tfull[a]);
+        sh.issued_mma = (sh.issued_mma & ~(0x101u << a)) | (1u << a) | ((use & 1u) << (8 + a));
+      }
+    }
+  } else {
+    const uint32_t q = warp & 3u, j = (warp >> 2) & 1u, grp = warp >> 3;
+    const float c = rht_scale_of(j == 0 ? g_r : g_c);
+    const float2 c2 = f2(c, c);
+    float m = 0.0f;
+    int k = static_cast<int>(grp);
+    for (int64_t t = blockIdx.x + grp * step; t < n_tiles; t += kDualGroups * step, k += kDualGroups) {
+      if (!mbar_wait(&sh.tfull[grp], (k / kDualGroups) & 1u)) {
+        atomicExch(&sh.abort_flag, 1);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t base = tmem_base + ((32u * q) << 16) + grp * 256 + j * 128;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float v[64];
+        tmem_ld64_wait(base + 64 * h, v);
+        if (h == 1) {
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.tfree[grp]);
+        }
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          float2 zp[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) zp[i] = mul2_rn(f2(v[32 * p + 2 * i], v[32 * p + 2 * i + 1]), c2);
+          float ma, mb;
+          absmax_pair(zp, ma, mb);
+          m = fmaxf(m, fmaxf(ma, mb));
+        }
+      }
+    }
+    const unsigned int bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
+    if (lane == 0) sh.warp_max[j][warp] = bits;
+  }
+
+  __syncthreads();
+  const bool failed = *reinterpret_cast<volatile int*>(&sh.abort_flag) != 0;
+  if (failed) {
+    if (tid == kDualProducerWarp * 32)
+      for (int s = 0; s < kDualStages; ++s)
+        if ((sh.issued_a >> s) & 1u) mbar_wait(&sh.full[s], (sh.issued_a >> (8 + s)) & 1u);
+    if (tid == kDualMmaWarp * 32)
+      for (int a = 0; a < kDualGroups; ++a)
+        if ((sh.issued_mma >> a) & 1u) mbar_wait(&sh.tfull[a], (sh.issued_mma >> (8 + a)) & 1u);
+  }
+  if (tid == 0) {
+    unsigned int mr = 0, mc = 0;
+#pragma unroll
+    for (int w = 0; w < kDualEpiWarps; ++w) {
+      // warps with (w >> 2) odd read the column view
+      if (((w >> 2) & 1) == 0) mr = max(mr, sh.warp_max[0][w]);
+      else mc = max(mc, sh.warp_max[1][w]);
+    }
+    atomicMax(amax_r, failed ? 0x7FC00000u : mr);
+    atomicMax(amax_c, failed ? 0x7FC00000u : mc);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kDualMmaWarp) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
 // --------------------------------------------------------------------- host
 using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
 
@@ -507,6 +746,32 @@ cudaError_t launch_quantize_mma(const QuantArgs& a) {
     case k4over6: return dispatch<k4over6, kQuantize>(a, nullptr);
     default: return cudaErrorInvalidValue;
   }
+}
+
+bool dual_mma_path_applies(const void* x, int64_t rows, int64_t cols, int64_t ld) {
+  QuantArgs a{x, rows, cols, ld, 0, kRTN, 128, 0, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  return mma_path_applies(a);
+}
+
+cudaError_t launch_amax_dual_mma(const void* x, int64_t rows, int64_t cols, int64_t ld, int g_r, int g_c,
+                                 uint64_t seed, float* amax_r, float* amax_c, cudaStream_t stream) {
+  CUtensorMap map;
+  if (!make_map(&map, x, rows, cols, ld)) return cudaErrorInvalidValue;
+  cudaError_t e =
+      cudaFuncSetAttribute(dual_amax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDualDynSmem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148, per_sm = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  e = resident_ctas(dual_amax_kernel, kDualThreads, kDualDynSmem, 1, &per_sm);
+  if (e != cudaSuccess) return e;
+  const int64_t n_tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
+  const int64_t grid = n_tiles < int64_t(sms) ? n_tiles : int64_t(sms);
+  if (grid == 0) return cudaSuccess;
+  dual_amax_kernel<<<static_cast<unsigned>(grid), kDualThreads, kDualDynSmem, stream>>>(
+      map, rows, cols, seed, g_r, g_c, reinterpret_cast<unsigned int*>(amax_r),
+      reinterpret_cast<unsigned int*>(amax_c));
+  return cudaGetLastError();
 }
 
 }  // namespace nvfp4

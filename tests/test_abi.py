@@ -33,7 +33,8 @@ def declared_symbols():
 def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ["nvfp4_quantize", "nvfp4_dequantize", "nvfp4_rht", "nvfp4_amax", "nvfp4_workspace_bytes",
-              "nvfp4_status_string", "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_quantize_noalloc"]:
+              "nvfp4_status_string", "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_quantize_noalloc",
+              "nvfp4_amax_dual"]:
         assert n in names
 
 
@@ -107,6 +108,14 @@ def test_other_entry_points_reject(N):
     assert N.nvfp4_amax(None, 64, 64, 64, 0, 0, 0, FAKE, None) == INVALID
     assert N.nvfp4_amax(FAKE, 64, 64, 64, 0, 0, 0, None, None) == INVALID
     assert N.nvfp4_amax(FAKE, 64, 40, 40, 0, 0, 0, FAKE, None) == SHAPE
+    ad = N.nvfp4_amax_dual
+    assert ad(None, 64, 64, 64, 0, 0, 0, FAKE, FAKE, None) == INVALID
+    assert ad(FAKE, 64, 64, 64, 0, 0, 0, FAKE, None, None) == INVALID
+    assert ad(FAKE, 64, 64, 64, 48, 0, 0, FAKE, FAKE, None) == INVALID   # group
+    assert ad(FAKE, 64, 40, 40, 0, 0, 0, FAKE, FAKE, None) == SHAPE      # row view: cols % 16
+    assert ad(FAKE, 40, 64, 64, 0, 0, 0, FAKE, FAKE, None) == SHAPE      # column view: rows % 16
+    assert ad(FAKE, 64, 64, 64, 0, 128, 0, FAKE, FAKE, None) == SHAPE    # column view: rows % g
+    assert ad(FAKE, 64, 64, 64, 0, 0, 0, FAKE + 2, FAKE, None) == ALIGN
     d = N.nvfp4_dequantize
     assert d(None, FAKE, FAKE, 4, 64, 0, 0, 0, 0, FAKE, None) == INVALID
     assert d(FAKE, FAKE, FAKE, 4, 64, 0, 0, 0, 1, FAKE, None) == INVALID  # inverse without rotation

@@ -318,3 +318,27 @@ def test_if4_int4_rounding_ties():
     gpu = compare_call(x, W.ROWWISE, W.IF4, 0, 5, amax=10.5)
     flagged = int(np.sum(gpu[1] >= 0x80))
     assert flagged > len(blocks) // 2, f"only {flagged} of {len(blocks)} blocks took the INT4 option"
+
+
+@pytest.mark.parametrize("shape,g_row,g_col", [
+    ((256, 384), 128, 128), ((640, 384), 0, 128), ((384, 1280), 128, 0), ((512, 512), 16, 64),
+    ((256, 256), 0, 0), ((1280, 896), 32, 128),
+    ((96, 256), 32, 32),      # below one tensor-core tile: two single pre-passes
+])
+def test_amax_dual_equals_two_single_passes(shape, g_row, g_col):
+    """nvfp4_amax_dual (both layouts from one read) gives the two single-layout
+    pre-passes' values bit for bit, and the oracle's within the rotation tolerance."""
+    rows, cols = shape
+    x = W.gradient(rows=rows, cols=cols).tensors()["g"]
+    xd = x.cuda()
+    a_row, a_col = N.amax_dual(xd, g_row, g_col, 41)
+    s_row = N.amax(xd, W.ROWWISE, g_row, 41)
+    s_col = N.amax(xd, W.TRANSPOSED, g_col, 41)
+    torch.cuda.synchronize()
+    assert a_row.item() == s_row.item() and a_col.item() == s_col.item()
+    for layout, g, got in ((W.ROWWISE, g_row, a_row.item()), (W.TRANSPOSED, g_col, a_col.item())):
+        exp = oracle.amax(bits(x), layout, g, 41)
+        if g == 0:
+            assert got == exp
+        else:
+            assert abs(got - exp) <= ROT_TOL * exp
