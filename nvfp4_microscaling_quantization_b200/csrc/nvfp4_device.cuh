@@ -463,12 +463,14 @@ struct PairRng {
 // their round-to-nearest reciprocals for the division below.
 struct ScaleCtx {
   float s_g, q6, q4, r6, r4;
-  bool markstein;  // the reciprocal-based division is exact for every block
+  bool markstein;       // the reciprocal-based division is exact for every block
+  const float4* tbl;    // per E4M3 code S: {dec(S), d = RN(dec(S) s_g), RN(1/d) or 0, 0}
 };
 
 template <int MODE>
 __device__ __forceinline__ ScaleCtx make_scale_ctx(float amax) {
   ScaleCtx c;
+  c.tbl = nullptr;
   c.s_g = global_scale_of<MODE>(amax);
   c.q6 = __fmul_rn(6.0f, c.s_g);
   c.q4 = __fmul_rn(4.0f, c.s_g);
@@ -567,6 +569,18 @@ __device__ __forceinline__ void absmax_pair(const float2 (&z)[16], float& aa, fl
   ab = mb[0];
 }
 
+// The scale table of one launch: for every E4M3 code S (0x7F, never produced,
+// decodes to NaN) dec(S), d = RN(dec(S) s_g) and RN(1/d) (0 when d = 0), the
+// same values quantize_pair would compute per block.  Built by `n` threads
+// of the CTA into shared memory; the caller synchronises before use.
+__device__ __forceinline__ void build_scale_table(float4* tbl, float s_g, uint32_t tid, uint32_t n) {
+  for (uint32_t S = tid; S < 128; S += n) {
+    const float dS = e4m3_decode(S);
+    const float d = __fmul_rn(dS, s_g);
+    tbl[S] = make_float4(dS, d, d != 0.0f ? __frcp_rn(d) : 0.0f, 0.0f);
+  }
+}
+
 // RN(1/d) per lane, 0 for a zero scale (a zero block): computed unconditionally
 // and selected, so the reciprocal sits on no branch.
 __device__ __forceinline__ float2 rcp_or_zero(float2 d) {
@@ -579,7 +593,6 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
                                               BlockOut& oa, BlockOut& ob) {
   float aa, ab;
   absmax_pair(z, aa, ab);
-  const float2 sg2 = f2(sc.s_g, sc.s_g);
 
   if constexpr (MODE == k4over6) {
     uint32_t S[2], ca_lo[2], ca_hi[2], cb_lo[2], cb_hi[2];
@@ -589,8 +602,9 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
       const float2 sf = k == 0 ? div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein)
                                : div2_by(f2(aa, ab), sc.q4, sc.r4, sc.markstein);
       S[k] = e4m3x2_rne_sat(sf.x, sf.y);
-      const float2 d = mul2_rn(e4m3x2_decode(S[k]), sg2);
-      const float2 r = rcp_or_zero(d);
+      const float4 ta = sc.tbl[S[k] & 0xFFu], tb = sc.tbl[(S[k] >> 8) & 0xFFu];
+      const float2 d = f2(ta.y, tb.y);
+      const float2 r = f2(ta.z, tb.z);
       float ya[16], yb[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -625,17 +639,16 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
     const float2 sf = div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein);
     uint32_t S2 = e4m3x2_rne_sat(sf.x, sf.y);
     uint32_t Sa = S2 & 0xFFu, Sb = S2 >> 8;
-    float2 dS = e4m3x2_decode(S2);
+    float4 ta = sc.tbl[Sa], tb = sc.tbl[Sb];
     if constexpr (MODE == kSR) {
-      if (Sa < 0x7Eu && dS.x < sf.x) ++Sa;
-      if (Sb < 0x7Eu && dS.y < sf.y) ++Sb;
-      S2 = Sa | (Sb << 8);
-      dS = e4m3x2_decode(S2);
+      if (Sa < 0x7Eu && ta.x < sf.x) ta = sc.tbl[++Sa];
+      if (Sb < 0x7Eu && tb.x < sf.y) tb = sc.tbl[++Sb];
     }
+    const float2 dS = f2(ta.x, tb.x);
     oa.scale = Sa;
     ob.scale = Sb;
-    const float2 d = mul2_rn(dS, sg2);
-    const float2 r = rcp_or_zero(d);
+    const float2 d = f2(ta.y, tb.y);
+    const float2 r = f2(ta.z, tb.z);
     float ya[16], yb[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {

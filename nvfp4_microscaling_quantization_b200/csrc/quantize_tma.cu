@@ -167,6 +167,7 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
   __shared__ __align__(8) Ring ring;
   __shared__ __align__(16) uint32_t sign_tab[128];
   __shared__ unsigned int warp_max[kNT / 32];
+  __shared__ __align__(16) float4 scale_tbl[128];  // block-scale constants per E4M3 code
   uint8_t* stages = align_1024(dyn_smem);
 
   const uint32_t tid = threadIdx.x;
@@ -196,6 +197,7 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
       sign_tab[tid] = sgn(tid) << 31;
     }
   }
+  if constexpr (!AMAX_ONLY) build_scale_table(scale_tbl, global_scale_of<MODE>(*amax), tid, kNT);
   __syncthreads();
   const int64_t step = gridDim.x, drt = step / n_ct, dct = step - drt * n_ct;
   // load the CTA's k-th tile (sequence index) into stage k mod kStages
@@ -214,9 +216,10 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
     for (int k = 0; k < kStages; ++k) load(k);
   }
 
-  ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false};
+  ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false, nullptr};
   if constexpr (!AMAX_ONLY) {
     sc = make_scale_ctx<MODE>(*amax);
+    sc.tbl = scale_tbl;
     if (blockIdx.x == 0 && tid == 0) *gscale = sc.s_g;
   }
   // thread roles

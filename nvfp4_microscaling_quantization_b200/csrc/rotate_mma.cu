@@ -111,6 +111,7 @@ struct MmaShared {
   uint32_t issued_mma;       // bit a: MMAs went into accumulator a; bit 8+a: parity
   int abort_flag;
   unsigned int warp_max[kEpiWarps];
+  float4 scale_tbl[128];     // the launch's block-scale constants per E4M3 code
 };
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
@@ -192,6 +193,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     tmem_relinquish();
   }
   build_hadamard_b<G>(bmat, key, tid);
+  if constexpr (KIND == kQuantize) build_scale_table(sh.scale_tbl, global_scale_of<MODE>(*amax), tid, kThreads);
   fence_proxy_async_smem();
   tc_fence_before_sync();
   __syncthreads();
@@ -261,9 +263,10 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     // (groups of 8 warps)
     const uint32_t q = warp & 3u, grp = warp / kGroupWarps;
     const uint32_t j0 = kGroupWarps == 8 ? (warp >> 2) & 1u : 0u;
-    ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false};
+    ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false, nullptr};
     if constexpr (KIND == kQuantize) {
       sc = make_scale_ctx<MODE>(*amax);
+      sc.tbl = sh.scale_tbl;
       if (blockIdx.x == 0 && tid == 0) *gscale = sc.s_g;
     }
     const int64_t vcols = ROWWISE ? cols : rows;
