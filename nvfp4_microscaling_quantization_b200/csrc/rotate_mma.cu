@@ -8,17 +8,21 @@
 // columns), transposed tiles are the same TMA boxes read MN-major (K = the
 // tile's rows), so both layouts share one kernel and one load pattern.
 //
-// Warp roles in a CTA of 10 warps (two CTAs per SM):
-//   warps 0-7  epilogue: thread (lane quarter q = warp % 4, half j = warp / 4)
-//              owns view row 32q + lane of the tile and its 64 columns
-//              64j .. 64j+63 (four 16-element blocks); it loads them from
-//              tensor memory, scales by c_g and quantizes (or takes max|z|, or
-//              stores z).
-//   warp 8     TMA producer: two 64-column boxes of 128 rows per tile into a
-//              2-stage shared-memory ring.
-//   warp 9     allocates tensor memory (2 accumulators x 128 columns), and one
-//              lane issues the 8 MMAs (K = 16 each) of a tile, committing
-//              "stage free" and "accumulator full" mbarriers.
+// One CTA per SM (it allocates all 512 tensor-memory columns).  Warp roles:
+//   epilogue   groups of four warps (Shape: four groups, three for SR), each
+//              owning one 128-column fp32 accumulator and taking every
+//              groups-th tile of the CTA; warp w reads lane quarter w % 4 (as
+//              tensor memory requires), so its thread owns one tile row, all
+//              128 columns (eight 16-element blocks), loaded 32 columns at a
+//              time, scaled by c_g and quantized two blocks at a time (or
+//              reduced to max|z|, or stored).  The accumulator columns are
+//              permuted so a load yields (block a, block b) register pairs.
+//   producer   one lane issues the TMA loads: two 64-column boxes of 128 rows
+//              per tile into a kStagesA-stage shared-memory ring.
+//   MMA        allocates the tensor memory, and one lane issues the 8 MMAs
+//              (K = 16 each) of a tile into the accumulator of the group that
+//              takes it, committing "stage free" and "accumulator full"
+//              mbarriers.
 // Every wait is bounded (tma_pipeline.cuh); on a failed wait the CTA drains
 // what it issued, frees tensor memory and reports NaN in its scalar output.
 #include <cuda.h>
@@ -35,47 +39,31 @@ namespace nvfp4 {
 
 namespace {
 
-#ifndef NVFP4_MMA_GROUPS
-#define NVFP4_MMA_GROUPS 4
-#endif
-#ifndef NVFP4_MMA_ACCUM
-#define NVFP4_MMA_ACCUM 4
-#endif
 #ifndef NVFP4_MMA_STAGES
 #define NVFP4_MMA_STAGES 3
 #endif
-#ifndef NVFP4_MMA_CTAS
-#define NVFP4_MMA_CTAS 1
-#endif
 
-#ifndef NVFP4_MMA_GROUP_WARPS
-#define NVFP4_MMA_GROUP_WARPS 4
-#endif
-#ifndef NVFP4_MMA_QUAD
-#define NVFP4_MMA_QUAD 0
-#endif
+enum Kind { kQuantize = 0, kAmax = 1, kStoreZ = 2 };
 
-constexpr int kGroups = NVFP4_MMA_GROUPS;           // epilogue groups, each on its own tiles
-constexpr int kGroupWarps = NVFP4_MMA_GROUP_WARPS;  // 4 (a thread owns 128 columns) or 8 (64)
-constexpr int kHalves = 8 / kGroupWarps;            // 64-column halves of a row per thread
-constexpr bool kQuad = NVFP4_MMA_QUAD != 0;         // four blocks in flight instead of two
-constexpr int kEpiWarps = kGroupWarps * kGroups;
-static_assert(kGroupWarps == 4 || kGroupWarps == 8, "a group covers the four lane quarters once or twice");
-constexpr int kThreads = (kEpiWarps + 2) * 32;
-constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
+// Launch shape of one instantiation: epilogue groups of four warps, each
+// owning one 128-column accumulator and taking every groups-th tile of the
+// CTA; one TMA producer warp and one MMA warp.  SR runs three groups (14
+// warps, 128 registers a thread: its Philox-heavy epilogue spills at 96),
+// everything else four (18 warps, 96 registers).
+template <int MODE, int KIND>
+struct Shape {
+  static constexpr int groups = (KIND == kQuantize && MODE == kSR) ? 3 : 4;
+  static constexpr int epi_warps = 4 * groups;
+  static constexpr int producer_warp = epi_warps, mma_warp = epi_warps + 1;
+  static constexpr int threads = (epi_warps + 2) * 32;
+};
+constexpr int kMaxGroups = 4;
 constexpr int kStagesA = NVFP4_MMA_STAGES;   // A tiles in flight
-constexpr int kAccum = NVFP4_MMA_ACCUM;      // accumulators in tensor memory
-constexpr int kCtasPerSm = NVFP4_MMA_CTAS;   // resident CTAs per SM
 constexpr int kTile = 128;                   // tile rows and columns of X
 constexpr uint32_t kTileBytes = kTile * kTile * 2;
 constexpr uint32_t kBoxBytes = kTile * 128;  // 128 rows x 64 bf16
-// tensor-memory allocations are powers of two columns
-constexpr uint32_t kTmemCols = kAccum <= 1 ? 128u : (kAccum <= 2 ? 256u : 512u);
+constexpr uint32_t kTmemCols = 512;          // up to four 128-column accumulators (a power of two)
 constexpr size_t kDynSmem = (kStagesA + 1) * kTileBytes + 1024;
-static_assert(kAccum >= 1 && kAccum <= 4, "up to four 128-column accumulators");
-static_assert(kCtasPerSm * kTmemCols <= 512, "the resident CTAs' accumulators must fit in tensor memory");
-
-enum Kind { kQuantize = 0, kAmax = 1, kStoreZ = 2 };
 
 #ifndef NVFP4_MMA_BAND_ROWS
 #define NVFP4_MMA_BAND_ROWS 1
@@ -104,13 +92,13 @@ struct TileGrid {
 struct MmaShared {
   uint64_t full[kStagesA];   // A tile landed (TMA transaction bytes)
   uint64_t sfree[kStagesA];  // MMAs reading the A tile are done (tcgen05.commit)
-  uint64_t tfull[kAccum];    // accumulator ready (tcgen05.commit)
-  uint64_t tfree[kAccum];    // accumulator read by the epilogue warps
+  uint64_t tfull[kMaxGroups];  // the group's accumulator ready (tcgen05.commit)
+  uint64_t tfree[kMaxGroups];  // the group's accumulator read by its warps
   uint32_t tmem_base;
   uint32_t issued_a;         // bit s: a load went into stage s; bit 8+s: its phase parity
   uint32_t issued_mma;       // bit a: MMAs went into accumulator a; bit 8+a: parity
   int abort_flag;
-  unsigned int warp_max[kEpiWarps];
+  unsigned int warp_max[4 * kMaxGroups];
   float4 scale_tbl[128];     // the launch's block-scale constants per E4M3 code
 };
 
@@ -131,9 +119,9 @@ __device__ __forceinline__ uint32_t output_col_of(uint32_t acc_col) {
 // (n, k) = sigma_(k mod G) * H_G[n mod G][k mod G] inside the diagonal G x G
 // blocks, 0 elsewhere.  bf16 +1 = 0x3F80, -1 = 0xBF80.
 template <int G>
-__device__ __forceinline__ void build_hadamard_b(uint8_t* bmat, PhiloxKey key, uint32_t tid) {
+__device__ __forceinline__ void build_hadamard_b(uint8_t* bmat, PhiloxKey key, uint32_t tid, uint32_t nthreads) {
   const uint4 w = philox_call(key, 0, kTagSigns);
-  for (uint32_t c = tid; c < 2048; c += kThreads) {
+  for (uint32_t c = tid; c < 2048; c += nthreads) {
     const uint32_t half = c >> 10, r = (c >> 3) & 127u, kc = c & 7u;
     const uint32_t n = output_col_of(r);
     uint32_t packed[4];
@@ -159,10 +147,12 @@ __device__ __forceinline__ void build_hadamard_b(uint8_t* bmat, PhiloxKey key, u
 }
 
 template <int MODE, int G, int KIND, bool ROWWISE>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(Shape<MODE, KIND>::threads, 1)
 rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed,
                   const float* __restrict__ amax, unsigned int* __restrict__ amax_accum, uint8_t* __restrict__ codes,
                   uint8_t* __restrict__ scales, float* __restrict__ gscale, float* __restrict__ zout) {
+  using S = Shape<MODE, KIND>;
+  constexpr int kGroups = S::groups, kAccum = S::groups;
   extern __shared__ uint8_t dyn_smem[];
   __shared__ __align__(8) MmaShared sh;
   uint8_t* a_tiles = align_1024(dyn_smem);
@@ -174,26 +164,26 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
                     static_cast<uint32_t>(ROWWISE ? NVFP4_MMA_BAND_ROWS : NVFP4_MMA_BAND_ROWS_T)};
   const int64_t n_tiles = static_cast<int64_t>(tg.n_rt) * tg.n_ct;
 
-  if (tid == kProducerWarp * 32) {
+  if (tid == S::producer_warp * 32) {
     for (int s = 0; s < kStagesA; ++s) {
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.sfree[s], 1);
     }
     for (int a = 0; a < kAccum; ++a) {
       mbar_init(&sh.tfull[a], 1);
-      mbar_init(&sh.tfree[a], kGroupWarps);  // the warps of one epilogue group
+      mbar_init(&sh.tfree[a], 4);  // the four warps of one epilogue group
     }
     sh.issued_a = 0;
     sh.issued_mma = 0;
     sh.abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == S::mma_warp) {
     tmem_alloc(&sh.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  build_hadamard_b<G>(bmat, key, tid);
-  if constexpr (KIND == kQuantize) build_scale_table(sh.scale_tbl, global_scale_of<MODE>(*amax), tid, kThreads);
+  build_hadamard_b<G>(bmat, key, tid, S::threads);
+  if constexpr (KIND == kQuantize) build_scale_table(sh.scale_tbl, global_scale_of<MODE>(*amax), tid, S::threads);
   fence_proxy_async_smem();
   tc_fence_before_sync();
   __syncthreads();
@@ -201,7 +191,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
   const uint32_t tmem_base = sh.tmem_base;
   const int64_t step = gridDim.x;
 
-  if (warp == kProducerWarp) {
+  if (warp == S::producer_warp) {
     if (lane == 0) {
       prefetch_tensormap(&tmap);
       int k = 0;
@@ -223,7 +213,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
         sh.issued_a = (sh.issued_a & ~(0x101u << s)) | (1u << s) | ((u & 1u) << (8 + s));
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == S::mma_warp) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kTile, kTile, ROWWISE ? 0u : 1u);
       const uint32_t b_addr = smem_u32(bmat);
@@ -257,12 +247,10 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // group `grp` takes the CTA's tiles k = grp, grp + kGroups, ...; within it
-    // a warp reads lane quarter q (= warp % 4, as tensor memory requires) and
-    // either all 128 columns (groups of 4 warps) or the half 64j .. 64j+63
-    // (groups of 8 warps)
-    const uint32_t q = warp & 3u, grp = warp / kGroupWarps;
-    const uint32_t j0 = kGroupWarps == 8 ? (warp >> 2) & 1u : 0u;
+    // group `grp` takes the CTA's tiles k = grp, grp + groups, ... into its
+    // accumulator grp; a warp reads lane quarter q (= warp % 4, as tensor
+    // memory requires): its thread owns one tile row, all 128 columns
+    const uint32_t q = warp & 3u, grp = warp >> 2;
     ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false, nullptr};
     if constexpr (KIND == kQuantize) {
       sc = make_scale_ctx<MODE>(*amax);
@@ -292,41 +280,26 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
       // the tile and view rows hold whole groups of eight blocks, its eight
       // blocks take the eight draws of one Philox call
       uint4 wu = make_uint4(0u, 0u, 0u, 0u);
-      if constexpr (KIND == kQuantize && MODE == kMSEDEN && kHalves == 2) {
+      if constexpr (KIND == kQuantize && MODE == kMSEDEN) {
         if (row_blocks8)
           wu = philox_call(key, (static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols / 16) +
                                  static_cast<uint64_t>((ROWWISE ? ct : rt) * (kTile / 16))) >> 3,
                            kTagBlock);
       }
 #pragma unroll 1
-      for (int h = 0; h < kHalves; ++h) {
-        const uint32_t j = j0 + h;
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t j = h;
         const uint32_t taddr = tmem_base + ((32u * q) << 16) + a * kTile + j * 64;
         const int64_t vcol0 = (ROWWISE ? ct : rt) * kTile + 64 * j;  // view column of the first element
-        const bool last = h == kHalves - 1;
+        const bool last = h == 1;
 
-        if constexpr (KIND == kQuantize && kQuad) {
-          float v[64];
-          tmem_ld64_wait(taddr, v);
-          if (last) {
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.tfree[a]);
-          }
-          float2 z[2][16];
-#pragma unroll
-          for (int p = 0; p < 2; ++p)
-#pragma unroll
-            for (int i = 0; i < 16; ++i) z[p][i] = mul2_rn(f2(v[32 * p + 2 * i], v[32 * p + 2 * i + 1]), c2);
-          if (vrow < vrows && vcol0 < vcols)
-            quantize_store64<MODE>(z, sc, key, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);
-        } else if constexpr (KIND == kQuantize) {
+        if constexpr (KIND == kQuantize) {
           // one pair of blocks at a time: load 32 columns, quantize, then the next 32
           const bool valid = vrow < vrows && vcol0 < vcols;
           const uint64_t e0 = static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols) + static_cast<uint64_t>(vcol0);
           float u[4] = {0.0f, 0.0f, 0.0f, 0.0f};
           if constexpr (MODE == kMSEDEN) {
-            if (kHalves == 2 && row_blocks8) {
+            if (row_blocks8) {
 #pragma unroll
               for (int b = 0; b < 4; ++b) u[b] = uniform16(half_word(wu, 4 * j + b));
             } else {
@@ -395,10 +368,10 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
   const bool failed = *reinterpret_cast<volatile int*>(&sh.abort_flag) != 0;
   if (failed) {
     // let every load and MMA still in flight finish before the CTA lets go
-    if (tid == kProducerWarp * 32)
+    if (tid == S::producer_warp * 32)
       for (int s = 0; s < kStagesA; ++s)
         if ((sh.issued_a >> s) & 1u) mbar_wait(&sh.full[s], (sh.issued_a >> (8 + s)) & 1u);
-    if (tid == kMmaWarp * 32)
+    if (tid == S::mma_warp * 32)
       for (int a = 0; a < kAccum; ++a)
         if ((sh.issued_mma >> a) & 1u) mbar_wait(&sh.tfull[a], (sh.issued_mma >> (8 + a)) & 1u);
   }
@@ -406,7 +379,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     if constexpr (KIND == kAmax) {
       unsigned int m = 0;
 #pragma unroll
-      for (int w = 0; w < kEpiWarps; ++w) m = max(m, sh.warp_max[w]);
+      for (int w = 0; w < S::epi_warps; ++w) m = max(m, sh.warp_max[w]);
       atomicMax(amax_accum, failed ? 0x7FC00000u : m);
     } else if constexpr (KIND == kQuantize) {
       if (failed) *gscale = __uint_as_float(0x7FC00000u);
@@ -414,7 +387,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
   }
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == S::mma_warp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, kTmemCols);
   }
@@ -694,11 +667,12 @@ cudaError_t launch_one(const QuantArgs& a, float* zout) {
   auto kernel = rotate_mma_kernel<MODE, G, KIND, ROWWISE>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDynSmem));
   if (e != cudaSuccess) return e;
-  // at most kCtasPerSm CTAs per SM: tensor memory holds that many CTAs' accumulators
+  // one CTA per SM: it allocates all of tensor memory
+  constexpr int threads = Shape<MODE, KIND>::threads;
   int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  e = resident_ctas(kernel, kThreads, kDynSmem, kCtasPerSm, &per_sm);
+  e = resident_ctas(kernel, threads, kDynSmem, 1, &per_sm);
   if (e != cudaSuccess) return e;
   const int64_t n_tiles = ((a.rows + kTile - 1) / kTile) * ((a.cols + kTile - 1) / kTile);
   int64_t grid = n_tiles < int64_t(sms) * per_sm ? n_tiles : int64_t(sms) * per_sm;
@@ -706,7 +680,7 @@ cudaError_t launch_one(const QuantArgs& a, float* zout) {
     if (KIND == kAmax) return cudaSuccess;
     grid = 1;
   }
-  kernel<<<static_cast<unsigned>(grid), kThreads, kDynSmem, a.stream>>>(
+  kernel<<<static_cast<unsigned>(grid), threads, kDynSmem, a.stream>>>(
       map, a.rows, a.cols, a.seed, a.amax, reinterpret_cast<unsigned int*>(a.amax_accum), a.codes, a.scales,
       a.gscale, zout);
   return cudaGetLastError();
