@@ -197,7 +197,6 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
       sign_tab[tid] = sgn(tid) << 31;
     }
   }
-  if constexpr (!AMAX_ONLY) build_scale_table(scale_tbl, global_scale_of<MODE>(*amax), tid, kNT);
   __syncthreads();
   const int64_t step = gridDim.x, drt = step / n_ct, dct = step - drt * n_ct;
   // load the CTA's k-th tile (sequence index) into stage k mod kStages
@@ -218,6 +217,9 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
 
   ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false, nullptr};
   if constexpr (!AMAX_ONLY) {
+    // the first loads are in flight: build the scale table meanwhile
+    build_scale_table(scale_tbl, global_scale_of<MODE>(*amax), tid, kNT);
+    __syncthreads();
     sc = make_scale_ctx<MODE>(*amax);
     sc.tbl = scale_tbl;
     if (blockIdx.x == 0 && tid == 0) *gscale = sc.s_g;

@@ -183,7 +183,6 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     tmem_relinquish();
   }
   build_hadamard_b<G>(bmat, key, tid, S::threads);
-  if constexpr (KIND == kQuantize) build_scale_table(sh.scale_tbl, global_scale_of<MODE>(*amax), tid, S::threads);
   fence_proxy_async_smem();
   tc_fence_before_sync();
   __syncthreads();
@@ -254,6 +253,9 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false, nullptr};
     if constexpr (KIND == kQuantize) {
       sc = make_scale_ctx<MODE>(*amax);
+      // the scale table, built by the epilogue warps while the first tiles load
+      build_scale_table(sh.scale_tbl, sc.s_g, tid, S::epi_warps * 32);
+      asm volatile("bar.sync 1, %0;" ::"r"(S::epi_warps * 32) : "memory");
       sc.tbl = sh.scale_tbl;
       if (blockIdx.x == 0 && tid == 0) *gscale = sc.s_g;
     }
@@ -481,13 +483,15 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
   const int64_t n_tiles = static_cast<int64_t>(tg.n_rt) * tg.n_ct;
 
   if (tid == kDualProducerWarp * 32) {
+    // with g_r = 0 the row view needs no MMA: the group's four row-view
+    // warps take max|x| from the staged tile and release the stage themselves
     for (int s = 0; s < kDualStages; ++s) {
       mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.sfree[s], 1);
+      mbar_init(&sh.sfree[s], g_r == 0 ? 5 : 1);
     }
     for (int a = 0; a < kDualGroups; ++a) {
       mbar_init(&sh.tfull[a], 1);
-      mbar_init(&sh.tfree[a], 8);
+      mbar_init(&sh.tfree[a], g_r == 0 ? 4 : 8);
     }
     sh.issued_a = 0;
     sh.issued_mma = 0;
@@ -498,7 +502,7 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
     tmem_alloc(&sh.tmem_base, 512);
     tmem_relinquish();
   }
-  build_rotation_b(b_r, key, tid, kDualThreads, g_r);
+  if (g_r != 0) build_rotation_b(b_r, key, tid, kDualThreads, g_r);
   build_rotation_b(b_c, key, tid, kDualThreads, g_c);
   fence_proxy_async_smem();
   tc_fence_before_sync();
@@ -549,11 +553,13 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
         tc_fence_after_sync();
         const uint32_t a_addr = smem_u32(a_tiles + s * kTileBytes);
         const uint32_t d_r = tmem_base + a * 256, d_c = d_r + 128;
+        if (g_r != 0) {
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint64_t adesc = smem_desc_sw128(a_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(br_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
-          umma_bf16(d_r, adesc, bdesc, idesc_r, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(a_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(br_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+            umma_bf16(d_r, adesc, bdesc, idesc_r, kk > 0 ? 1u : 0u);
+          }
         }
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
@@ -572,6 +578,30 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
     const float2 c2 = f2(c, c);
     float m = 0.0f;
     int k = static_cast<int>(grp);
+    if (j == 0 && g_r == 0) {
+      // max|x| of the staged tile: 128 threads, 256 bytes each (the order of
+      // the swizzled bytes does not matter to a maximum); bf16 -> f32 is exact
+      const uint32_t part = (warp & 3u) * 32u + lane;
+      for (int64_t t = blockIdx.x + grp * step; t < n_tiles; t += kDualGroups * step, k += kDualGroups) {
+        const int s = k % kDualStages;
+        if (!mbar_wait(&sh.full[s], (k / kDualStages) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(a_tiles + s * kTileBytes) + part;
+        uint32_t bmax = 0;  // max of |x| as bf16 bit patterns (monotone for non-negative values)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint4 w4 = src[i * 128];
+          const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) bmax = max(bmax, max(w[e] & 0x7FFFu, (w[e] >> 16) & 0x7FFFu));
+        }
+        m = fmaxf(m, __uint_as_float(bmax << 16));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.sfree[s]);
+      }
+    } else {
     for (int64_t t = blockIdx.x + grp * step; t < n_tiles; t += kDualGroups * step, k += kDualGroups) {
       if (!mbar_wait(&sh.tfull[grp], (k / kDualGroups) & 1u)) {
         atomicExch(&sh.abort_flag, 1);
@@ -598,6 +628,7 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
           m = fmaxf(m, fmaxf(ma, mb));
         }
       }
+    }
     }
     const unsigned int bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
     if (lane == 0) sh.warp_max[j][warp] = bits;
