@@ -182,13 +182,19 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     tmem_alloc(&sh.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  build_hadamard_b<G>(bmat, key, tid, S::threads);
-  fence_proxy_async_smem();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = sh.tmem_base;
   const int64_t step = gridDim.x;
+  if (warp != S::producer_warp) {
+    // B is built by every warp but the producer, which starts loading tiles
+    // meanwhile; the builders meet at barrier 2 before the first MMA
+    const uint32_t bt = warp < S::producer_warp ? tid : tid - 32, nb = S::threads - 32;
+    build_hadamard_b<G>(bmat, key, bt, nb);
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 2, %0;" ::"r"(nb) : "memory");
+  }
 
   if (warp == S::producer_warp) {
     if (lane == 0) {
@@ -502,14 +508,19 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
     tmem_alloc(&sh.tmem_base, 512);
     tmem_relinquish();
   }
-  if (g_r != 0) build_rotation_b(b_r, key, tid, kDualThreads, g_r);
-  build_rotation_b(b_c, key, tid, kDualThreads, g_c);
-  fence_proxy_async_smem();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = sh.tmem_base;
   const int64_t step = gridDim.x;
+  if (warp != kDualProducerWarp) {
+    // the B matrices, built while the producer starts loading (barrier 2)
+    const uint32_t bt = warp < kDualProducerWarp ? tid : tid - 32, nb = kDualThreads - 32;
+    if (g_r != 0) build_rotation_b(b_r, key, bt, nb, g_r);
+    build_rotation_b(b_c, key, bt, nb, g_c);
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 2, %0;" ::"r"(nb) : "memory");
+  }
 
   if (warp == kDualProducerWarp) {
     if (lane == 0) {
