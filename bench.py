@@ -47,8 +47,8 @@ L2_FLUSH_BYTES = 256 << 20
 # kernel reports traffic = null until it is captured again.
 NCU_TRAFFIC = {
     # profiles/rotate_mma_eden_dy.md: dram__bytes_read.sum + dram__bytes_write.sum, one launch
-    ("bea7130ec89ddce6", "dy.transposed.ms_eden.g128"): 470032384 + 108876544,
-    ("bea7130ec89ddce6", "dy.rowwise.ms_eden.g128"): 469903104 + 109543680,
+    ("c16e804ffa2c44f6", "dy.transposed.ms_eden.g128"): 470047488 + 108913920,
+    ("c16e804ffa2c44f6", "dy.rowwise.ms_eden.g128"): 469990912 + 108828672,
 }
 
 
