@@ -98,3 +98,21 @@ def _check_workload(wl):
 @pytest.mark.parametrize("name", ["weight", "gradient", "activation", "mlp_up"])
 def test_full_size_sampled(name):
     _check_workload(W.ALL[name]())
+
+
+def test_full_size_dual_pre_pass():
+    """The dual pre-pass bench.py runs (one read per tensor) gives, at the MLP
+    workload's full sizes, the two single-layout tensor amaxes bit for bit."""
+    wl = W.mlp_up()
+    tensors = wl.tensors("cuda")
+    for name in ("x", "w", "dy"):
+        calls = [c for c in wl.calls if c.tensor == name]
+        row = next(c for c in calls if c.layout == W.ROWWISE)
+        col = next(c for c in calls if c.layout == W.TRANSPOSED)
+        x = tensors[name]
+        a_row, a_col = N.amax_dual(x, row.rht_group, col.rht_group, wl.seed)
+        s_row = N.amax(x, W.ROWWISE, row.rht_group, wl.seed)
+        s_col = N.amax(x, W.TRANSPOSED, col.rht_group, wl.seed)
+        torch.cuda.synchronize()
+        assert a_row.item() == s_row.item(), name
+        assert a_col.item() == s_col.item(), name
