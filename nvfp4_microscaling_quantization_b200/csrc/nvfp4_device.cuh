@@ -706,14 +706,13 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
         const float2 s2 = add2_after_mul(t, f2(kRoundMagic, kRoundMagic));
         const float2 r2 = sub2_rn(s2, f2(kRoundMagic, kRoundMagic));
         const float2 kf = f2(fminf(fmaxf(r2.x, -7.0f), 7.0f), fminf(fmaxf(r2.y, -7.0f), 7.0f));
-        const int ka = max(-7, min(7, static_cast<int>(__float_as_uint(s2.x) - 0x4B400000u)));
-        const int kb = max(-7, min(7, static_cast<int>(__float_as_uint(s2.y) - 0x4B400000u)));
         const float2 vi = mul2_rn(kf, f2(kIF4K2, kIF4K2));
         const float2 dI = sub2_after_mul(y, vi);
         eI = fma2_rn(dI, dI, eI);
-        // sign-magnitude nibble; k = 0 gives 0
-        const uint32_t codea = static_cast<uint32_t>(abs(ka)) | ((static_cast<uint32_t>(ka) >> 28) & 8u);
-        const uint32_t codeb = static_cast<uint32_t>(abs(kb)) | ((static_cast<uint32_t>(kb) >> 28) & 8u);
+        // sign-magnitude nibble of the integer kf (never -0): |k| is the low
+        // mantissa bits of 2^23 + |kf| (exact), the sign is bit 31 of kf
+        const uint32_t codea = (__float_as_uint(fabsf(kf.x) + 8388608.0f) & 7u) | ((__float_as_uint(kf.x) >> 28) & 8u);
+        const uint32_t codeb = (__float_as_uint(fabsf(kf.y) + 8388608.0f) & 7u) | ((__float_as_uint(kf.y) >> 28) & 8u);
         if (i < 8) {
           ia_lo |= codea << (4 * i);
           ib_lo |= codeb << (4 * i);
