@@ -581,13 +581,9 @@ __device__ __forceinline__ void build_scale_table(float4* tbl, float s_g, uint32
   }
 }
 
-// RN(1/d) per lane, 0 for a zero scale (a zero block): computed unconditionally
-// and selected, so the reciprocal sits on no branch.
-__device__ __forceinline__ float2 rcp_or_zero(float2 d) {
-  const float ra = __frcp_rn(d.x), rb = __frcp_rn(d.y);
-  return f2(d.x != 0.0f ? ra : 0.0f, d.y != 0.0f ? rb : 0.0f);
-}
-
+// Quantize blocks a (z[i].x) and b (z[i].y) of one pair under the launch's
+// ScaleCtx (its scale table must be built: sc.tbl), writing their codes and
+// scales; the same results as quantize_block on each block.
 template <int MODE>
 __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const ScaleCtx& sc, const PairRng& rng,
                                               BlockOut& oa, BlockOut& ob) {
