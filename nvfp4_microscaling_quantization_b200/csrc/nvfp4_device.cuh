@@ -581,10 +581,23 @@ __device__ __forceinline__ void build_scale_table(float4* tbl, float s_g, uint32
   }
 }
 
+// The scale constants of E4M3 code S: from the launch's table (TBL), or
+// computed (the same values).
+template <bool TBL>
+__device__ __forceinline__ float4 scale_entry(const ScaleCtx& sc, uint32_t S) {
+  if constexpr (TBL) {
+    return sc.tbl[S];
+  } else {
+    const float dS = e4m3_decode(S);
+    const float d = __fmul_rn(dS, sc.s_g);
+    return make_float4(dS, d, d != 0.0f ? __frcp_rn(d) : 0.0f, 0.0f);
+  }
+}
+
 // Quantize blocks a (z[i].x) and b (z[i].y) of one pair under the launch's
-// ScaleCtx (its scale table must be built: sc.tbl), writing their codes and
-// scales; the same results as quantize_block on each block.
-template <int MODE>
+// ScaleCtx (with TBL its scale table must be built: sc.tbl), writing their
+// codes and scales; the same results as quantize_block on each block.
+template <int MODE, bool TBL = true>
 __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const ScaleCtx& sc, const PairRng& rng,
                                               BlockOut& oa, BlockOut& ob) {
   float aa, ab;
@@ -598,7 +611,7 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
       const float2 sf = k == 0 ? div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein)
                                : div2_by(f2(aa, ab), sc.q4, sc.r4, sc.markstein);
       S[k] = e4m3x2_rne_sat(sf.x, sf.y);
-      const float4 ta = sc.tbl[S[k] & 0xFFu], tb = sc.tbl[(S[k] >> 8) & 0xFFu];
+      const float4 ta = scale_entry<TBL>(sc, S[k] & 0xFFu), tb = scale_entry<TBL>(sc, (S[k] >> 8) & 0xFFu);
       const float2 d = f2(ta.y, tb.y);
       const float2 r = f2(ta.z, tb.z);
       float ya[16], yb[16];
@@ -635,10 +648,10 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
     const float2 sf = div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein);
     uint32_t S2 = e4m3x2_rne_sat(sf.x, sf.y);
     uint32_t Sa = S2 & 0xFFu, Sb = S2 >> 8;
-    float4 ta = sc.tbl[Sa], tb = sc.tbl[Sb];
+    float4 ta = scale_entry<TBL>(sc, Sa), tb = scale_entry<TBL>(sc, Sb);
     if constexpr (MODE == kSR) {
-      if (Sa < 0x7Eu && ta.x < sf.x) ta = sc.tbl[++Sa];
-      if (Sb < 0x7Eu && tb.x < sf.y) tb = sc.tbl[++Sb];
+      if (Sa < 0x7Eu && ta.x < sf.x) ta = scale_entry<TBL>(sc, ++Sa);
+      if (Sb < 0x7Eu && tb.x < sf.y) tb = scale_entry<TBL>(sc, ++Sb);
     }
     const float2 dS = f2(ta.x, tb.x);
     oa.scale = Sa;

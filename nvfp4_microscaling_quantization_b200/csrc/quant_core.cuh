@@ -49,7 +49,7 @@ __device__ __forceinline__ void store64(const BlockOut (&o)[4], int64_t vrow, in
 
 // Quantize the four blocks of view row `vrow` starting at view column `vcol0`
 // and store their codes and scales (blocks at or beyond vcols are skipped).
-template <int MODE>
+template <int MODE, bool TBL = true>
 __device__ __forceinline__ void quantize_store64(const float2 (&z)[2][16], const ScaleCtx& sc, PhiloxKey key,
                                                  int64_t vrow, int64_t vcol0, int64_t vcols, uint8_t* codes,
                                                  uint8_t* scales, bool codes_aligned16, bool scales_aligned4) {
@@ -60,7 +60,7 @@ __device__ __forceinline__ void quantize_store64(const float2 (&z)[2][16], const
 #pragma unroll
   for (int p = 0; p < 2; ++p) {
     const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, u[2 * p], u[2 * p + 1]};
-    quantize_pair<MODE>(z[p], sc, rng, o[2 * p], o[2 * p + 1]);
+    quantize_pair<MODE, TBL>(z[p], sc, rng, o[2 * p], o[2 * p + 1]);
   }
   store64(o, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);
 }
