@@ -41,11 +41,6 @@ namespace {
 #endif
 
 constexpr int kNT = 128;                   // threads per CTA
-// Block-scale constants from a per-CTA table for the modes that form two or
-// more scales per block pair; RTN computes them (its per-block work is light
-// enough that the table's build and lookups cost more than they save).
-template <int MODE>
-__host__ __device__ constexpr bool tma_table() { return MODE != kRTN; }
 constexpr int kStages = NVFP4_TMA_STAGES;  // ring depth
 constexpr int kMinBlocks = NVFP4_TMA_MIN_BLOCKS;
 constexpr uint32_t kStageBytes = 16384;
@@ -222,11 +217,9 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
 
   ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false, nullptr};
   if constexpr (!AMAX_ONLY) {
-    if constexpr (tma_table<MODE>()) {
-      // the first loads are in flight: build the scale table meanwhile
-      build_scale_table(scale_tbl, global_scale_of<MODE>(*amax), tid, kNT);
-      __syncthreads();
-    }
+    // the first loads are in flight: build the scale table meanwhile
+    build_scale_table(scale_tbl, global_scale_of<MODE>(*amax), tid, kNT);
+    __syncthreads();
     sc = make_scale_ctx<MODE>(*amax);
     sc.tbl = scale_tbl;
     if (blockIdx.x == 0 && tid == 0) *gscale = sc.s_g;
@@ -323,11 +316,11 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
     } else if constexpr (ROWWISE) {
       const int64_t row = rt * kRowBoxRows + j, col0 = ct * kRowTileCols + 64 * piece;
       if (row < rows && col0 < cols)
-        quantize_store64<MODE, tma_table<MODE>()>(z, sc, key, row, col0, cols, codes, scales, codes_aligned16, scales_aligned4);
+        quantize_store64<MODE>(z, sc, key, row, col0, cols, codes, scales, codes_aligned16, scales_aligned4);
     } else {
       const int64_t vrow = ct * kColTileCols + col, vcol0 = rt * kColTileRows + 64 * half;
       if (vrow < cols && vcol0 < rows)
-        quantize_store64<MODE, tma_table<MODE>()>(z, sc, key, vrow, vcol0, rows, codes, scales, codes_aligned16, scales_aligned4);
+        quantize_store64<MODE>(z, sc, key, vrow, vcol0, rows, codes, scales, codes_aligned16, scales_aligned4);
     }
   }
 
