@@ -305,25 +305,33 @@ __device__ __forceinline__ void rtn_codes(const float* y, uint32_t& lo, uint32_t
   hi = clear_negative_zero(cvt_e2m1x8(y + 8));
 }
 
-// Stochastic rounding of one scaled value with the uniform U = k * 2^-16:
-// a = min(|y|, 6) between grid neighbours l <= a < u goes up iff
-// U < (a - l) / (u - l), done on the bits of a with no conversion
-// instruction.  For a in [1, 6] the grid keeps one mantissa bit, so
-// (a - l) / (u - l) = low22 / 2^22 (low22 = the 22 mantissa bits below it)
-// and U < that iff 64k < low22 iff low22 + (2^22 - 1 - 64k) carries into
-// the kept bit; the code index is then (bits >> 22) - 252.  For a in
-// [0.5, 1) the same with all 23 mantissa bits (index (bits >> 23) - 125).
-// For a in [0, 0.5) the neighbours are 0 and 0.5 and the fraction is 2a.
-__device__ __forceinline__ uint32_t sr_code(float y, uint32_t k16) {
-  const float a = fminf(fabsf(y), 6.0f);
-  const uint32_t b = __float_as_uint(a);
-  const uint32_t x22 = 0x3FFFFFu - 64u * k16;        // 2^22 - 1 - 64k >= 63
-  const uint32_t i1 = (b + x22 - (252u << 22)) >> 22;  // a >= 1
-  const uint32_t i2 = (b + 2u * x22 + 1u - (125u << 23)) >> 23;  // a in [0.5, 1): 2^23 - 1 - 128k
-  const uint32_t i3 = uniform16(k16) < __fadd_rn(a, a) ? 1u : 0u;  // a < 0.5
-  const uint32_t mag = a >= 1.0f ? i1 : (a >= 0.5f ? i2 : i3);
-  if (mag == 0u) return 0u;
-  return mag | (y < 0.0f ? 8u : 0u);
+// Stochastic rounding of eight scaled values y[0..7] with the eight 16-bit
+// uniforms U_i = k_i * 2^-16 of one Philox call w (draw i = half i&1 of word
+// i/2), done on the bits of the floats with no conversion instruction.
+// a = min(|y|, 6) lies between grid neighbours l <= a < u and goes up iff
+// U < (a - l) / (u - l).  For a in [1, 6] the grid keeps one mantissa bit, so
+// the fraction is low22 / 2^22 (low22 = the 22 mantissa bits below it) and
+// U < low22 / 2^22 iff 64k < low22 iff low22 + (2^22 - 1 - 64k) carries into
+// the kept bit; the code index is then (bits >> 22) - 252.  For a in [0, 1)
+// the grid {0, 0.5, 1} is that of 0.5 + a/2 on [0.5, 1] (one kept bit below
+// 0.5), and 0.5 + a/2 rounded upward is exact for the decision: 64k * 2^-23
+// lies on the 2^-23 grid that the upward rounding lands on, so a - l exceeds
+// it iff the rounded value does.  max(a, RU(0.5 + a/2)) picks the right one
+// of the two (0.5 + a/2 <= a iff a >= 1).  2^22 - 1 - 64k = (64k) ^ (2^22 - 1).
+// Signs go in afterwards, and a code of magnitude 0 drops its sign.
+__device__ __forceinline__ uint32_t sr_codes8(const float* y, const uint4& w) {
+  uint32_t mag = 0u, sgn = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t word = word_of(w, static_cast<uint32_t>(i >> 1));
+    const uint32_t k64 = ((i & 1) ? (word >> 10) : (word << 6)) & 0x3FFFC0u;
+    const float a = fminf(fabsf(y[i]), 6.0f);
+    const float a1 = fmaxf(a, __fmaf_ru(a, 0.5f, 0.5f));
+    const uint32_t v = __float_as_uint(a1) + (k64 ^ 0x3FFFFFu) - (252u << 22);  // index in bits 22..24
+    mag |= (4 * i <= 22 ? v >> (22 - 4 * i) : v << (4 * i - 22)) & (7u << (4 * i));
+    sgn |= (__float_as_uint(y[i]) >> (28 - 4 * i)) & (8u << (4 * i));
+  }
+  return clear_negative_zero(mag | sgn);
 }
 
 // Quantize one block of 16 (already rotated) values z under tensor scale s_g.
@@ -383,19 +391,8 @@ __device__ __forceinline__ BlockOut quantize_block(const float* z, float s_g, co
       rtn_codes(y, out.lo, out.hi);
     } else if constexpr (MODE == kSR) {
       const uint64_t call0 = rng.first_element >> 3;
-      const uint4 w0 = philox_call(rng.key, call0, kTagElement);
-      const uint4 w1 = philox_call(rng.key, call0 + 1, kTagElement);
-      uint32_t lo = 0u, hi = 0u;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t word0 = word_of(w0, i >> 1), word1 = word_of(w1, i >> 1);
-        const uint32_t k0 = (word0 >> ((i & 1) * 16)) & 0xFFFFu;
-        const uint32_t k1 = (word1 >> ((i & 1) * 16)) & 0xFFFFu;
-        lo |= sr_code(y[i], k0) << (4 * i);
-        hi |= sr_code(y[8 + i], k1) << (4 * i);
-      }
-      out.lo = lo;
-      out.hi = hi;
+      out.lo = sr_codes8(y, philox_call(rng.key, call0, kTagElement));
+      out.hi = sr_codes8(y + 8, philox_call(rng.key, call0 + 1, kTagElement));
     } else if constexpr (MODE == kMSEDEN) {
       rtn_codes(y, out.lo, out.hi);
       float v[16];
@@ -537,17 +534,8 @@ __device__ __forceinline__ uint32_t e4m3x2_sr(float2 t, float ua, float ub) {
 __device__ __forceinline__ void sr_block(const float (&y)[16], PhiloxKey key, uint64_t elem, uint32_t& lo,
                                          uint32_t& hi) {
   const uint64_t call0 = elem >> 3;
-  const uint4 w0 = philox_call(key, call0, kTagElement);
-  const uint4 w1 = philox_call(key, call0 + 1, kTagElement);
-  lo = 0u;
-  hi = 0u;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t k0 = (word_of(w0, i >> 1) >> ((i & 1) * 16)) & 0xFFFFu;
-    const uint32_t k1 = (word_of(w1, i >> 1) >> ((i & 1) * 16)) & 0xFFFFu;
-    lo |= sr_code(y[i], k0) << (4 * i);
-    hi |= sr_code(y[8 + i], k1) << (4 * i);
-  }
+  lo = sr_codes8(y, philox_call(key, call0, kTagElement));
+  hi = sr_codes8(y + 8, philox_call(key, call0 + 1, kTagElement));
 }
 
 // max |z| of each of the two blocks of a pair, as a tree (exact in any order).
