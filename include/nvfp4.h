@@ -147,6 +147,41 @@ NVFP4_API int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, cons
                      int64_t vrows, int64_t vcols, int mode, int rht_group, uint64_t seed,
                      int inverse_rht, float* out, void* stream);
 
+typedef enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 } nvfp4_out_dtype;
+
+/* NVFP4 GEMM on the block-scaled tensor cores, consuming two quantizer
+ * outputs as they are:
+ *   D[i][j] = RN(gA * gB) * sum_k qA[i][k] SA[i][k/16] qB[j][k] SB[j][k/16]
+ * with q the E2M1 values and S the E4M3 block scales; the sum is accumulated
+ * in fp32 by the tensor cores, the product with RN(gA * gB) is one fp32
+ * multiply, then the store rounds to out_dtype (RN).  A is the m x k view
+ * quantized along k (nvfp4_quantize row-wise on an m x k tensor, or
+ * transposed on a k x m one), B likewise n x k; so Y = X W^T, dX = dY W and
+ * dW = dY^T X of a fully-NVFP4 linear layer are each one call (Quartet II
+ * record, abstract: NVFP4 is supported in hardware by Blackwell GPUs, the
+ * authors' kernels run linear layers up to 4.2x faster than BF16; the
+ * article's sections "Quantisierung im Vorwaertsdurchlauf" and "...
+ * Rueckwaertsdurchlauf" for which operand is quantized along which
+ * dimension).  The scales must be plain E4M3 (modes RTN, SR, MS-EDEN, 4/6):
+ * an IF4 scale carries the INT4 flag in bit 7, which the tensor cores do not
+ * interpret, so IF4 outputs are not valid operands.  Two operands rotated along k with
+ * the same seed and group give the product of the unrotated ones up to the
+ * quantization error (the rotation is orthogonal up to the rounding of its
+ * constant).
+ *  a_codes: m x k/2 bytes, a_scales: m x k/16 bytes, a_gscale: device float;
+ *  b_codes, b_scales, b_gscale: the same for n x k.  All device memory, owned
+ *  by the caller, read only.
+ *  d: m rows of n values (fp32 or bf16 per out_dtype), row stride ldd
+ *  elements, overwritten.
+ * Shapes: m and n multiples of 128, k a positive multiple of 256, ldd >= n
+ * (NVFP4_ERR_SHAPE); m or n zero is a no-op.  Alignment: codes and scales
+ * 16-byte aligned, d 16-byte aligned with ldd a multiple of 4 (fp32) or 8
+ * (bf16) (NVFP4_ERR_ALIGNMENT).  Asynchronous on `stream`; a kernel whose
+ * internal waits time out (a broken device) writes NaN to D[0][0]. */
+NVFP4_API int nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_gscale,
+                         const uint8_t* b_codes, const uint8_t* b_scales, const float* b_gscale, int64_t m,
+                         int64_t n, int64_t k, int out_dtype, void* d, int64_t ldd, void* stream);
+
 /* The random Hadamard rotation of the view, as fp32: out (vrows x vcols,
  * dense, 16-byte aligned) = the view of `in` with every rht_group-long piece
  * of a row rotated (inverse == 0) or un-rotated (inverse != 0).  in_dtype 0 =

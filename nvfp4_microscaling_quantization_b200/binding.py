@@ -1,9 +1,9 @@
 """Thin Python binding of libnvfp4.so (argument marshalling only).
 
 The functions named like the C ABI (nvfp4_quantize, nvfp4_dequantize, nvfp4_rht,
-nvfp4_amax, nvfp4_workspace_bytes, nvfp4_status_string) take raw device
+nvfp4_amax, nvfp4_gemm, nvfp4_workspace_bytes, nvfp4_status_string) take raw device
 pointers and sizes exactly as include/nvfp4.h declares them.  The tensor-level
-helpers (quantize, dequantize, rht, amax) take torch CUDA tensors, allocate the
+helpers (quantize, dequantize, rht, amax, gemm) take torch CUDA tensors, allocate the
 outputs with torch (device memory is the only thing torch provides here) and
 call the same entry points on the current CUDA stream.  Every step of the
 computation runs in the library's kernels; there is no CPU path.  If the
@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_encode_e4m3.restype = i32
         L.nvfp4_quantize_noalloc.argtypes = [P, i64, i64, i64, i32, i32, i32, u64, P, P, P, P, P]
         L.nvfp4_quantize_noalloc.restype = i32
+        L.nvfp4_gemm.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, P, i64, P]
+        L.nvfp4_gemm.restype = i32
         L.nvfp4_status_string.argtypes = [i32]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -101,6 +103,12 @@ def nvfp4_quantize_noalloc(x, rows, cols, ld, layout, mode, rht_group, seed, ama
                            global_scale, stream) -> int:
     return lib().nvfp4_quantize_noalloc(x, rows, cols, ld, layout, mode, rht_group, seed, amax_in, codes,
                                         scales, global_scale, stream)
+
+
+def nvfp4_gemm(a_codes, a_scales, a_gscale, b_codes, b_scales, b_gscale, m, n, k, out_dtype, d, ldd,
+               stream) -> int:
+    return lib().nvfp4_gemm(a_codes, a_scales, a_gscale, b_codes, b_scales, b_gscale, m, n, k, out_dtype, d,
+                            ldd, stream)
 
 
 def nvfp4_encode_e2m1(x, n, out, stream) -> int:
@@ -231,4 +239,36 @@ def encode_e4m3(x: torch.Tensor, round_up: bool = False, stream=None) -> torch.T
     out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     _check(nvfp4_encode_e4m3(_p(x), x.numel(), int(round_up), _p(out), _stream_handle(stream)),
            "nvfp4_encode_e4m3")
+    return out
+
+
+OUT_F32, OUT_BF16 = 0, 1
+
+
+def gemm(a, b, out_dtype=torch.float32, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """D = gA gB A B^T on the block-scaled tensor cores.
+
+    a, b: (codes, scales, global_scale) device tensors as quantize returns them,
+    for an m x k and an n x k view quantized along k (RTN, SR, MS-EDEN or 4/6).
+    Returns D [m, n] in out_dtype (torch.float32 or torch.bfloat16), or writes
+    `out` (m rows, row stride out.stride(0)).
+    """
+    (ac, asc, ag), (bc, bsc, bg) = a, b
+    m, k = ac.shape[0], 2 * ac.shape[1]
+    n = bc.shape[0]
+    if 2 * bc.shape[1] != k:
+        raise ValueError(f"operands disagree on k: {k} and {2 * bc.shape[1]}")
+    for t in (ac, asc, ag, bc, bsc, bg):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("gemm operands must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty(m, n, dtype=out_dtype, device=ac.device)
+    if out.dtype not in (torch.float32, torch.bfloat16) or out.stride(1) != 1 or tuple(out.shape) != (m, n):
+        raise ValueError("out must be an m x n float32 or bfloat16 tensor with unit column stride")
+    st = nvfp4_gemm(ctypes.c_void_p(ac.data_ptr()), ctypes.c_void_p(asc.data_ptr()), ctypes.c_void_p(ag.data_ptr()),
+                    ctypes.c_void_p(bc.data_ptr()), ctypes.c_void_p(bsc.data_ptr()), ctypes.c_void_p(bg.data_ptr()),
+                    m, n, k, OUT_BF16 if out.dtype == torch.bfloat16 else OUT_F32,
+                    ctypes.c_void_p(out.data_ptr()), out.stride(0), _stream_handle(stream))
+    if st:
+        raise Nvfp4Error(st, "nvfp4_gemm")
     return out

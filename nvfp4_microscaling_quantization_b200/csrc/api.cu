@@ -125,6 +125,25 @@ int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g
   return from_cuda(nvfp4::launch_dequantize(a));
 }
 
+int nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_gscale, const uint8_t* b_codes,
+               const uint8_t* b_scales, const float* b_gscale, int64_t m, int64_t n, int64_t k, int out_dtype,
+               void* d, int64_t ldd, void* stream) {
+  if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
+  if (m < 0 || n < 0 || k < 0 || m % 128 || n % 128 || k % 256 || ldd < n) return NVFP4_ERR_SHAPE;
+  if (m == 0 || n == 0) return NVFP4_OK;
+  if (!d || !a_gscale || !b_gscale) return NVFP4_ERR_INVALID_ARG;
+  if (k == 0) return NVFP4_ERR_SHAPE;
+  if (!a_codes || !a_scales || !b_codes || !b_scales) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_scales, 16) || !aligned(b_scales, 16) ||
+      !aligned(a_gscale, 4) || !aligned(b_gscale, 4) || !aligned(d, 16) ||
+      ldd % (out_dtype == NVFP4_OUT_F32 ? 4 : 8))
+    return NVFP4_ERR_ALIGNMENT;
+  if (!nvfp4::gemm_available()) return NVFP4_ERR_CUDA;
+  nvfp4::GemmArgs g{a_codes, a_scales, a_gscale, b_codes, b_scales, b_gscale, m, n, k,
+                    out_dtype == NVFP4_OUT_BF16 ? 1 : 0, d, ldd, static_cast<cudaStream_t>(stream)};
+  return from_cuda(nvfp4::launch_gemm(g));
+}
+
 int nvfp4_rht(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld, int layout,
               int rht_group, uint64_t seed, int inverse, float* out, void* stream) {
   if (!in || !out) return NVFP4_ERR_INVALID_ARG;

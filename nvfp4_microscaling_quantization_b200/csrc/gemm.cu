@@ -1,0 +1,359 @@
+// gemm.cu -- the NVFP4 GEMM that consumes the quantizer's output on the
+// sm_100a block-scaled tensor cores.
+//
+//   D[m][n] = gA * gB * sum_k (qA[m][k] * SA[m][k/16]) * (qB[n][k] * SB[n][k/16])
+//
+// qA, qB are E2M1 codes packed two per byte (element 2j in the low nibble),
+// SA, SB their E4M3 block scales stored row-major ([rows][K/16] bytes), and
+// gA, gB the FP32 tensor scales: exactly what nvfp4_quantize writes for an
+// M x K (row-wise, or the transposed view of a K x M tensor) and an N x K
+// operand.  Every GEMM of a fully-NVFP4 linear layer's training step takes
+// this form (Quartet II article, sections "Quantisierung im
+// Vorwaertsdurchlauf" and "... Rueckwaertsdurchlauf": Y = X W^T, dX = dY W,
+// dW = dY^T X, each operand quantized along the reduction dimension; the
+// Quartet II record's abstract: NVFP4 GEMMs in Blackwell hardware).
+//
+// Design (one persistent CTA per SM, 10 warps):
+//   warp 0      TMA producer: 128 x 256 E2M1 tiles of A and B (128 bytes a
+//               row, 128-byte swizzle) into a 6-stage shared-memory ring;
+//   warp 1      allocates all 512 tensor-memory columns; one thread issues
+//               tcgen05.mma kind::mxf4nvf4 (M = N = 128, K = 64, UE4M3 scale
+//               vector of 4 per row) -- four per K tile -- into one of two
+//               128-column fp32 accumulators;
+//   warps 2..5  scale-factor writers: read the row-major E4M3 scales of the
+//               stage's 128 rows of A and of B straight from global memory
+//               and store them into the stage's tensor-memory scale columns
+//               in the layout the MMA reads (row 32h + l of a K step in byte
+//               f of column 4 * step + h, lane l of every lane quarter);
+//   warps 6..9  epilogue: drain an accumulator (tcgen05.ld), multiply by
+//               gA * gB, store fp32 or bf16 rows of D, release the
+//               accumulator, so the next tile's MMAs overlap the stores.
+// Scale factors go to tensor memory from registers, so the GEMM reads the
+// quantizer's row-major scale layout as it is: no reordered copy of the
+// scales is needed in HBM.
+//
+// Every wait is bounded (tma_pipeline.cuh); a CTA whose wait runs out stops,
+// lets its loads and MMAs in flight finish, and writes NaN to D[0][0].
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "tcgen05.cuh"
+#include "tma_pipeline.cuh"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int kGBM = 128, kGBN = 128;           // output tile
+constexpr int kGBK = 256;                        // K elements per stage = 128 bytes of E2M1 a row
+constexpr int kGStages = 6;
+constexpr int kGAccum = 2;
+constexpr uint32_t kGOpBytes = kGBM * kGBK / 2;  // 16 KB per operand per stage
+constexpr uint32_t kGStageBytes = 2 * kGOpBytes;
+constexpr uint32_t kGSfCols = 32;                // per stage: 4 K steps x 4 columns for A, the same for B
+constexpr uint32_t kGSfBase = kGAccum * kGBN;    // scale columns follow the accumulators
+constexpr uint32_t kGTmemCols = 512;
+static_assert(kGSfBase + kGStages * kGSfCols <= kGTmemCols, "tensor memory");
+constexpr int kGProducerWarp = 0, kGMmaWarp = 1, kGEpiWarp0 = 6;  // scale writers: warps 2..5
+constexpr int kGThreads = 320;
+constexpr size_t kGDynSmem = kGStages * kGStageBytes + 1024;
+
+struct GemmShared {
+  uint64_t full[kGStages];     // A and B bytes of the stage landed
+  uint64_t sf_full[kGStages];  // the stage's scale factors are in tensor memory (4 writer warps)
+  uint64_t empty[kGStages];    // the MMAs that read the stage completed
+  uint64_t tfull[kGAccum];     // accumulator holds a finished tile
+  uint64_t tfree[kGAccum];     // epilogue drained the accumulator (4 warps)
+  uint32_t tmem_base;
+  uint32_t issued_ab;          // per stage: a load in flight (bit s) and its phase (bit 8 + s)
+  uint32_t issued_mma;         // per accumulator: a commit pending (bit a) and its phase (bit 8 + a)
+  int abort_flag;
+};
+
+__device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ bool aborted(GemmShared& sh) {
+  return *reinterpret_cast<volatile int*>(&sh.abort_flag) != 0;
+}
+
+template <int OUT_BF16>
+__global__ void __launch_bounds__(kGThreads, 1)
+nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                  const uint8_t* __restrict__ a_scales, const uint8_t* __restrict__ b_scales,
+                  const float* __restrict__ a_gscale, const float* __restrict__ b_gscale, int64_t m, int64_t n,
+                  int64_t k, void* __restrict__ d, int64_t ldd) {
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ __align__(8) GemmShared sh;
+  uint8_t* tiles = align_1024(dyn_smem);
+
+  const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+  const int64_t n_tn = n / kGBN;
+  const int64_t n_tiles = (m / kGBM) * n_tn;
+  const int kt_count = static_cast<int>(k / kGBK);
+  const int64_t step = gridDim.x;
+
+  if (tid == 0) {
+    for (int s = 0; s < kGStages; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.sf_full[s], 4);
+      mbar_init(&sh.empty[s], 1);
+    }
+    for (int a = 0; a < kGAccum; ++a) {
+      mbar_init(&sh.tfull[a], 1);
+      mbar_init(&sh.tfree[a], 4);
+    }
+    sh.issued_ab = 0;
+    sh.issued_mma = 0;
+    sh.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kGMmaWarp) {
+    tmem_alloc(&sh.tmem_base, kGTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = sh.tmem_base;
+
+  if (warp == kGProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_a);
+      prefetch_tensormap(&tmap_b);
+      uint32_t it = 0;
+      for (int64_t t = blockIdx.x; t < n_tiles && !aborted(sh); t += step) {
+        const int32_t ya = static_cast<int32_t>((t / n_tn) * kGBM), yb = static_cast<int32_t>((t % n_tn) * kGBN);
+        for (int kt = 0; kt < kt_count; ++kt, ++it) {
+          const uint32_t s = it % kGStages, u = it / kGStages;
+          if (it >= kGStages && !mbar_wait(&sh.empty[s], (u - 1) & 1u)) {
+            atomicExch(&sh.abort_flag, 1);
+            break;
+          }
+          if (aborted(sh)) break;
+          uint8_t* dst = tiles + s * kGStageBytes;
+          mbar_arrive_expect_tx(&sh.full[s], kGStageBytes);
+          // x in bytes: 128 per K tile, a multiple of 16
+          tma_load_2d(dst, &tmap_a, kt * (kGBK / 2), ya, &sh.full[s]);
+          tma_load_2d(dst + kGOpBytes, &tmap_b, kt * (kGBK / 2), yb, &sh.full[s]);
+          sh.issued_ab = (sh.issued_ab & ~(0x101u << s)) | (1u << s) | ((u & 1u) << (8 + s));
+        }
+      }
+    }
+  } else if (warp == kGMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_nvfp4_f32(kGBM, kGBN);
+      uint32_t it = 0, tile = 0;
+      for (int64_t t = blockIdx.x; t < n_tiles && !aborted(sh); t += step, ++tile) {
+        const uint32_t a = tile % kGAccum, ua = tile / kGAccum;
+        if (tile >= kGAccum && !mbar_wait(&sh.tfree[a], (ua - 1) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        tc_fence_after_sync();
+        bool ok = true;
+        for (int kt = 0; kt < kt_count; ++kt, ++it) {
+          const uint32_t s = it % kGStages, u = it / kGStages;
+          if (!mbar_wait(&sh.full[s], u & 1u) || !mbar_wait(&sh.sf_full[s], u & 1u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem_u32(tiles + s * kGStageBytes), b_addr = a_addr + kGOpBytes;
+          const uint32_t sf = tmem_base + kGSfBase + s * kGSfCols;
+#pragma unroll
+          for (int j = 0; j < kGBK / 64; ++j) {
+            // K step j: 32 bytes further along each 128-byte swizzled row
+            const uint64_t adesc = smem_desc_sw128(a_addr + j * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(b_addr + j * 32, 16, 1024);
+            umma_nvfp4(tmem_base + a * kGBN, adesc, bdesc, idesc, sf + 4 * j, sf + 16 + 4 * j,
+                       (kt | j) != 0 ? 1u : 0u);
+          }
+          umma_commit(&sh.empty[s]);
+        }
+        // committed even after a failed wait, so the accumulator's phase is
+        // tracked for the drain below
+        umma_commit(&sh.tfull[a]);
+        sh.issued_mma = (sh.issued_mma & ~(0x101u << a)) | (1u << a) | ((ua & 1u) << (8 + a));
+        if (!ok) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+      }
+    }
+  } else if (warp < kGEpiWarp0) {
+    // ------------------------------------------------- scale-factor writers
+    // warp q = warp % 4 fills lane quarter q; its thread l carries rows l,
+    // 32 + l, 64 + l, 96 + l of the tile, 16 scale bytes (one K tile) each
+    const uint32_t q = warp & 3u;
+    const int64_t srow = k / 16;  // scale bytes per row
+    uint32_t it = 0;
+    for (int64_t t = blockIdx.x; t < n_tiles && !aborted(sh); t += step) {
+      const int64_t ra = (t / n_tn) * kGBM + lane, rb = (t % n_tn) * kGBN + lane;
+      bool ok = true;
+      for (int kt = 0; kt < kt_count; ++kt, ++it) {
+        const uint32_t s = it % kGStages, u = it / kGStages;
+        uint4 va[4], vb[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          va[h] = __ldg(reinterpret_cast<const uint4*>(a_scales + (ra + 32 * h) * srow + kt * 16));
+          vb[h] = __ldg(reinterpret_cast<const uint4*>(b_scales + (rb + 32 * h) * srow + kt * 16));
+        }
+        if (it >= kGStages && !mbar_wait(&sh.empty[s], (u - 1) & 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        // column 4j + h: the four factors of K step j of row 32h + l
+        uint32_t ca[16], cb[16];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          ca[h] = va[h].x, ca[4 + h] = va[h].y, ca[8 + h] = va[h].z, ca[12 + h] = va[h].w;
+          cb[h] = vb[h].x, cb[4 + h] = vb[h].y, cb[8 + h] = vb[h].z, cb[12 + h] = vb[h].w;
+        }
+        const uint32_t sf = tmem_base + ((32u * q) << 16) + kGSfBase + s * kGSfCols;
+        tmem_st16_wait(sf, ca);
+        tmem_st16_wait(sf + 16, cb);
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.sf_full[s]);
+      }
+      if (!ok) {
+        atomicExch(&sh.abort_flag, 1);
+        break;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t q = warp & 3u;
+    const float gab = __fmul_rn(*a_gscale, *b_gscale);
+    uint32_t tile = 0;
+    for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++tile) {
+      const uint32_t a = tile % kGAccum;
+      if (!mbar_wait(&sh.tfull[a], (tile / kGAccum) & 1u)) {
+        atomicExch(&sh.abort_flag, 1);
+        break;
+      }
+      if (aborted(sh)) break;
+      tc_fence_after_sync();
+      const int64_t row = (t / n_tn) * kGBM + 32 * q + lane, col0 = (t % n_tn) * kGBN;
+#pragma unroll 1
+      for (int c = 0; c < kGBN; c += 32) {
+        float v[32];
+        tmem_ld32_wait(tmem_base + ((32u * q) << 16) + a * kGBN + c, v);
+        if constexpr (OUT_BF16) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(d) + row * ldd + col0 + c);
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 p =
+                  __floats2bfloat162_rn(__fmul_rn(v[i + 2 * e], gab), __fmul_rn(v[i + 2 * e + 1], gab));
+              w[e] = *reinterpret_cast<const uint32_t*>(&p);
+            }
+            dst[i / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(d) + row * ldd + col0 + c);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            dst[i / 4] = make_float4(__fmul_rn(v[i], gab), __fmul_rn(v[i + 1], gab), __fmul_rn(v[i + 2], gab),
+                                     __fmul_rn(v[i + 3], gab));
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.tfree[a]);
+    }
+  }
+
+  __syncthreads();
+  const bool failed = aborted(sh);
+  if (failed) {
+    // let every load and MMA still in flight finish before the CTA lets go
+    if (tid == kGProducerWarp * 32)
+      for (int s = 0; s < kGStages; ++s)
+        if ((sh.issued_ab >> s) & 1u) mbar_wait(&sh.full[s], (sh.issued_ab >> (8 + s)) & 1u);
+    if (tid == kGMmaWarp * 32)
+      for (int a = 0; a < kGAccum; ++a)
+        if ((sh.issued_mma >> a) & 1u) mbar_wait(&sh.tfull[a], (sh.issued_mma >> (8 + a)) & 1u);
+    if (tid == 0) {
+      if (OUT_BF16)
+        *static_cast<uint16_t*>(d) = 0x7FC0u;
+      else
+        *static_cast<uint32_t*>(d) = 0x7FC00000u;
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kGMmaWarp) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, kGTmemCols);
+  }
+}
+
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeTiledFn gemm_encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// rows x (k / 2) bytes of packed E2M1, boxes of 128 bytes x 128 rows.
+bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k) {
+  EncodeTiledFn fn = gemm_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 2)};
+  cuuint32_t box[2] = {kGBK / 2, kGBM};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int OUT_BF16>
+cudaError_t launch_gemm_t(const GemmArgs& g) {
+  CUtensorMap ma, mb;
+  if (!make_codes_map(&ma, g.a_codes, g.m, g.k) || !make_codes_map(&mb, g.b_codes, g.n, g.k))
+    return cudaErrorInvalidValue;
+  auto kernel = nvfp4_gemm_kernel<OUT_BF16>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kGDynSmem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t n_tiles = (g.m / kGBM) * (g.n / kGBN);
+  const int64_t grid = n_tiles < sms ? n_tiles : sms;
+  if (grid == 0) return cudaSuccess;
+  kernel<<<static_cast<unsigned>(grid), kGThreads, kGDynSmem, g.stream>>>(
+      ma, mb, g.a_scales, g.b_scales, g.a_gscale, g.b_gscale, g.m, g.n, g.k, g.d, g.ldd);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_available() { return gemm_encode_fn() != nullptr; }
+
+cudaError_t launch_gemm(const GemmArgs& g) {
+  return g.out_bf16 ? launch_gemm_t<1>(g) : launch_gemm_t<0>(g);
+}
+
+}  // namespace nvfp4

@@ -72,6 +72,24 @@ bool dual_mma_path_applies(const void* x, int64_t rows, int64_t cols, int64_t ld
 cudaError_t launch_amax_dual_mma(const void* x, int64_t rows, int64_t cols, int64_t ld, int g_r, int g_c,
                                  uint64_t seed, float* amax_r, float* amax_c, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantArgs& a);
+
+// D = gA gB A B^T from two quantizer outputs (gemm.cu); shapes checked by the
+// caller: m, n multiples of 128, k of 256, 16-byte aligned codes, scales, D rows.
+struct GemmArgs {
+  const uint8_t* a_codes;   // m x k/2
+  const uint8_t* a_scales;  // m x k/16
+  const float* a_gscale;
+  const uint8_t* b_codes;   // n x k/2
+  const uint8_t* b_scales;  // n x k/16
+  const float* b_gscale;
+  int64_t m, n, k;
+  int out_bf16;
+  void* d;                  // m rows, leading dimension ldd (elements)
+  int64_t ldd;
+  cudaStream_t stream;
+};
+bool gemm_available();
+cudaError_t launch_gemm(const GemmArgs& g);
 cudaError_t launch_rht(const RhtArgs& a);
 cudaError_t launch_encode_e2m1(const float* in, int64_t n, uint8_t* out, cudaStream_t stream);
 cudaError_t launch_encode_e4m3(const float* in, int64_t n, int round_up, uint8_t* out, cudaStream_t stream);

@@ -1,7 +1,7 @@
 // tcgen05.cuh -- the 5th-generation tensor core (sm_100a) pieces the rotation
-// kernel uses: tensor-memory allocation, single-thread MMA issue with shared-
-// memory matrix descriptors, completion tracking on mbarriers, and loads of
-// the fp32 accumulator from tensor memory into registers.
+// and GEMM kernels use: tensor-memory allocation, single-thread MMA issue with
+// shared-memory matrix descriptors (bf16, and block-scaled E2M1), completion
+// tracking on mbarriers, register <-> tensor-memory moves.
 #pragma once
 
 #include <cstdint>
@@ -59,6 +59,39 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u)
+      : "memory");
+}
+
+// Instruction descriptor of a dense block-scaled kind::mxf4nvf4 MMA: packed
+// E2M1 A and B (format 1), both K-major, UE4M3 scale factors (scale format
+// 0), one factor per 16 elements of K, fp32 D, M x N, K = 64 per instruction.
+__host__ __device__ constexpr uint32_t idesc_nvfp4_f32(int m, int n) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// D[tmem] (+)= (A . SFA) x (B . SFB)^T over K = 64: A, B packed E2M1 in shared
+// memory, their UE4M3 scale factors in tensor memory at sfa / sfb (four
+// factors per row in the four bytes of a column, one column per 32 rows,
+// copied into every lane quarter); issued by one thread.
+__device__ __forceinline__ void umma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns from registers: thread i of the
+// warp writes lane (the warp's lane quarter base + i), columns taddr.col ..
+// +15; the wait makes the writes complete before the thread goes on.
+__device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 

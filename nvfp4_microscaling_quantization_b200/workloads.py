@@ -181,6 +181,21 @@ def mlp_up(tokens=16384, d_model=4096, d_ff=14336, seed=4) -> Workload:
                     calls, "MLP up-projection step: X 16384x4096, W 14336x4096, dY 16384x14336")
 
 
+def gemm_operand(rows: int, k: int, seed: int, scale_codes=None, device="cpu"):
+    """Random bytes standing for one quantized GEMM operand (rows x k view):
+    packed E2M1 codes (rows x k/2, every byte value equally likely) and E4M3
+    scale bytes (rows x k/16) drawn uniformly from `scale_codes` (default:
+    every finite positive code, 0x00..0x7E).  Plain integers, no quantization:
+    for checking the GEMM on operands of known structure."""
+    g = _gen(seed, device)
+    codes = torch.randint(0, 256, (rows, k // 2), generator=g, dtype=torch.int32, device=device).to(torch.uint8)
+    if scale_codes is None:
+        scale_codes = list(range(0x7F))
+    table = torch.tensor(list(scale_codes), dtype=torch.uint8, device=device)
+    idx = torch.randint(0, len(table), (rows, k // 16), generator=g, dtype=torch.int64, device=device)
+    return codes, table[idx]
+
+
 ALL = {"small": small, "weight": weight, "gradient": gradient, "activation": activation, "mlp_up": mlp_up}
 
 

@@ -263,3 +263,46 @@ def unpack_codes(codes):
     out[..., 0::2] = codes & 15
     out[..., 1::2] = codes >> 4
     return out
+
+
+def _gemm_operand_ints(codes, scales, rows=None):
+    """Dequantized operand times 2^10, as exact int64: every E2M1 value is a
+    multiple of 1/2 and every E4M3 value a multiple of 2^-9, so q * dec(S) is a
+    multiple of 2^-10 below 6 * 448 < 2^12."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    scales = np.asarray(scales, dtype=np.uint8)
+    if rows is not None:
+        codes, scales = codes[rows], scales[rows]
+    if np.any(scales >= 0x7F):
+        raise ValueError("GEMM operands take finite plain E4M3 scales (bit 7 clear, not 0x7F)")
+    q2 = np.array([round(2.0 * e2m1_decode(c)) for c in range(16)], dtype=np.int64)       # 2 * value
+    s9 = np.array([round(512.0 * e4m3_decode(s)) if s != 0x7F else 0 for s in range(128)], dtype=np.int64)
+    q = q2[unpack_codes(codes)]
+    s = np.repeat(s9[scales], 16, axis=-1)
+    return q * s
+
+
+def gemm(a_codes, a_scales, a_gscale, b_codes, b_scales, b_gscale, a_rows=None, b_rows=None):
+    """The NVFP4 GEMM on two quantized operands (A: m x k view, B: n x k view,
+    both quantized along k), as float64:
+
+        D[i][j] = RN32(gA * gB) * sum_k qA[i][k] SA[i][k/16] qB[j][k] SB[j][k/16]
+
+    (Quartet II record, abstract: NVFP4 GEMMs run in Blackwell hardware;
+    Quartet II article, sections "Quantisierung im Vorwaertsdurchlauf" and
+    "... Rueckwaertsdurchlauf": every GEMM operand is quantized along the
+    reduction dimension).  The sum is exact: each operand element times 2^10
+    is an integer below 2^22, so a product is below 2^44 and a sum of up to
+    2^19 products stays below 2^63 in int64.  The one product with the tensor
+    scales is rounded to float64.  a_rows / b_rows select rows of A / B (then
+    D is len(a_rows) x len(b_rows)).
+    """
+    ai = _gemm_operand_ints(a_codes, a_scales, a_rows)
+    bi = _gemm_operand_ints(b_codes, b_scales, b_rows)
+    if ai.shape[1] != bi.shape[1]:
+        raise ValueError("operands disagree on k")
+    if ai.shape[1] > (1 << 19):
+        raise ValueError("k above 2^19: the int64 sum could overflow")
+    s = ai @ bi.T
+    gab = float(np.float32(np.float32(a_gscale) * np.float32(b_gscale)))
+    return s.astype(np.float64) * (2.0 ** -20) * gab

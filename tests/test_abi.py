@@ -34,7 +34,7 @@ def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ["nvfp4_quantize", "nvfp4_dequantize", "nvfp4_rht", "nvfp4_amax", "nvfp4_workspace_bytes",
               "nvfp4_status_string", "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_quantize_noalloc",
-              "nvfp4_amax_dual"]:
+              "nvfp4_amax_dual", "nvfp4_gemm"]:
         assert n in names
 
 
@@ -130,6 +130,20 @@ def test_other_entry_points_reject(N):
     assert N.nvfp4_encode_e2m1(None, 4, FAKE, None) == INVALID
     assert N.nvfp4_encode_e2m1(FAKE, -1, FAKE, None) == SHAPE
     assert N.nvfp4_encode_e4m3(FAKE + 2, 4, 0, FAKE, None) == ALIGN
+    g = N.nvfp4_gemm
+    ok = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert g(*ok, 128, 128, 256, 2, FAKE, 128, None) == INVALID        # output dtype
+    assert g(*ok, 100, 128, 256, 0, FAKE, 128, None) == SHAPE          # m % 128
+    assert g(*ok, 128, 130, 256, 0, FAKE, 130, None) == SHAPE          # n % 128
+    assert g(*ok, 128, 128, 320, 0, FAKE, 128, None) == SHAPE          # k % 256
+    assert g(*ok, 128, 128, 0, 0, FAKE, 128, None) == SHAPE            # k = 0
+    assert g(*ok, 128, 128, 256, 0, FAKE, 64, None) == SHAPE           # ldd < n
+    assert g(*ok, 0, 128, 256, 0, None, 128, None) == OK               # empty: nothing touched
+    assert g(None, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 128, 256, 0, FAKE, 128, None) == INVALID
+    assert g(*ok, 128, 128, 256, 0, None, 128, None) == INVALID
+    assert g(FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 128, 256, 0, FAKE, 128, None) == ALIGN
+    assert g(*ok, 128, 128, 256, 0, FAKE, 130, None) == ALIGN          # fp32 rows: ldd % 4
+    assert g(*ok, 128, 128, 256, 1, FAKE, 132, None) == ALIGN          # bf16 rows: ldd % 8
 
 
 def test_binding_refuses_cpu_tensors(N):
