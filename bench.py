@@ -40,6 +40,7 @@ UNIT = "GB/s"
 BYTES_PER_ELEMENT = 2.0 + 0.5 + 0.0625   # bf16 in, E2M1 codes out, E4M3 scales out
 PREPASS_BYTES_PER_ELEMENT = 2.0          # the amax pre-pass reads the tensor once more
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
 
 # DRAM bytes per launch measured by ncu for the dominant kernel, keyed by the
@@ -47,8 +48,8 @@ L2_FLUSH_BYTES = 256 << 20
 # kernel reports traffic = null until it is captured again.
 NCU_TRAFFIC = {
     # profiles/rotate_mma_eden_dy.md: dram__bytes_read.sum + dram__bytes_write.sum, one launch
-    ("676723f05e9d54eb", "dy.transposed.ms_eden.g128"): 470099712 + 109061376,
-    ("676723f05e9d54eb", "dy.rowwise.ms_eden.g128"): 469893120 + 109283072,
+    ("c7f0c0e2cc2dbd5d", "dy.transposed.ms_eden.g128"): 470117888 + 108601344,
+    ("c7f0c0e2cc2dbd5d", "dy.rowwise.ms_eden.g128"): 469887232 + 108546048,
 }
 
 
@@ -63,6 +64,8 @@ def parse_args(argv=None):
                    help="fraction of each call's view rows the CPU baseline quantizes")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-gemm", action="store_true",
+                   help="skip the NVFP4 GEMMs of the step (measured after the quantization step)")
     p.add_argument("--no-per-mode", action="store_true",
                    help="skip the per-mode table (every mode on dY, quantize kernel alone)")
     return p.parse_args(argv)
@@ -170,6 +173,16 @@ def hbm_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak_bf16():
+    """Measured dense bf16 tensor throughput (TFLOP/s, burst), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def kernel_source_hash():
@@ -280,6 +293,46 @@ def per_mode_table(N, W, x, seed, stream, device, flush, peak, reps=5):
     return out
 
 
+def gemm_table(N, calls, stream, device, reps=10):
+    """The three GEMMs of the linear layer's training step on the step's own
+    quantized outputs (nvfp4_gemm, bf16 D): Y = X W^T (RTN X and W row-wise),
+    dX = dY W (MS-EDEN dY row-wise, W transposed), dW = dY^T X (MS-EDEN dY and
+    X transposed).  CUDA events over each launch after warm-up; the fp4 dense
+    tensor peak is the measured bf16 peak x 4 (nominal 9 / 2.25 PF)."""
+    by = {c.call.name: c for c in calls}
+    q = lambda name: (by[name].codes, by[name].scales, by[name].gscale)  # noqa: E731
+    cases = [("Y = X W^T", "x.rowwise.rtn.norht", "w.rowwise.rtn.norht"),
+             ("dX = dY W", "dy.rowwise.ms_eden.g128", "w.transposed.ms_eden.g128"),
+             ("dW = dY^T X", "dy.transposed.ms_eden.g128", "x.transposed.ms_eden.g128")]
+    peak_bf16, kind = tensor_peak_bf16()
+    peak = 4.0 * peak_bf16
+    out = []
+    for name, an, bn in cases:
+        a, b = q(an), q(bn)
+        m, k, n = a[0].shape[0], 2 * a[0].shape[1], b[0].shape[0]
+        d = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+        for _ in range(3):
+            N.gemm(a, b, out=d)
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            N.gemm(a, b, out=d)
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) / 1e3)
+        t = statistics.median(ts)
+        tf = 2.0 * m * n * k / t / 1e12
+        out.append({"gemm": name, "a": an, "b": bn, "m": m, "n": n, "k": k, "out": "bf16",
+                    "us": round(t * 1e6, 1), "tflops": round(tf, 1),
+                    "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(peak, 1),
+                                 "peak_kind": f"fp4 dense = 4 x {kind} bf16", "unit": "TFLOP/s",
+                                 "frac": round(tf / peak, 4)}})
+        del d
+    torch.cuda.synchronize(device)
+    return out
+
+
 def run_ours(args, world, rank, local):
     import ctypes
     from nvfp4_microscaling_quantization_b200 import binding as N
@@ -374,6 +427,10 @@ def run_ours(args, world, rank, local):
             "read_gbs": round(read / (amax_ms[g] / 1e3) / 1e9, 1),
         })
 
+    gemms = None
+    if not args.no_gemm:
+        gemms = gemm_table(N, calls, stream, device)
+
     per_mode = None
     if not args.no_per_mode:
         per_mode = per_mode_table(N, W, tensors["dy"], wl.seed, sh, device, flush, peak)
@@ -414,6 +471,8 @@ def run_ours(args, world, rank, local):
         "clocks": clock,
         "kernel_source": src_hash,
     }
+    if gemms is not None:
+        result["nvfp4_gemm"] = gemms
     if per_mode is not None:
         result["per_mode_dy"] = per_mode
     if e2e is not None:

@@ -15,20 +15,20 @@
 //
 // Design (one persistent CTA per SM, 10 warps):
 //   warp 0      TMA producer: 128 x 256 E2M1 tiles of A and B (128 bytes a
-//               row, 128-byte swizzle) into a 6-stage shared-memory ring;
+//               row, 128-byte swizzle) and their 128 x 16 scale bytes into
+//               a 6-stage shared-memory ring;
 //   warp 1      allocates all 512 tensor-memory columns; one thread issues
 //               tcgen05.mma kind::mxf4nvf4 (M = N = 128, K = 64, UE4M3 scale
 //               vector of 4 per row) -- four per K tile -- into one of two
 //               128-column fp32 accumulators;
-//   warps 2..5  scale-factor writers: read the row-major E4M3 scales of the
-//               stage's 128 rows of A and of B straight from global memory
-//               and store them into the stage's tensor-memory scale columns
-//               in the layout the MMA reads (row 32h + l of a K step in byte
-//               f of column 4 * step + h, lane l of every lane quarter);
+//   warps 2..5  scale-factor writers: move the stage's scale bytes from
+//               shared memory into the stage's tensor-memory scale columns in
+//               the layout the MMA reads (row 32h + l of a K step in byte f of
+//               column 4 * step + h, lane l of every lane quarter);
 //   warps 6..9  epilogue: drain an accumulator (tcgen05.ld), multiply by
 //               gA * gB, store fp32 or bf16 rows of D, release the
 //               accumulator, so the next tile's MMAs overlap the stores.
-// Scale factors go to tensor memory from registers, so the GEMM reads the
+// Scale factors go to tensor memory through registers, so the GEMM reads the
 // quantizer's row-major scale layout as it is: no reordered copy of the
 // scales is needed in HBM.
 //
@@ -54,7 +54,8 @@ constexpr int kGBK = 256;                        // K elements per stage = 128 b
 constexpr int kGStages = 6;
 constexpr int kGAccum = 2;
 constexpr uint32_t kGOpBytes = kGBM * kGBK / 2;  // 16 KB per operand per stage
-constexpr uint32_t kGStageBytes = 2 * kGOpBytes;
+constexpr uint32_t kGSfBytes = kGBM * (kGBK / 16);  // 2 KB of scale bytes per operand per stage
+constexpr uint32_t kGStageBytes = 2 * kGOpBytes + 2 * kGSfBytes;  // a multiple of 1024
 constexpr uint32_t kGSfCols = 32;                // per stage: 4 K steps x 4 columns for A, the same for B
 constexpr uint32_t kGSfBase = kGAccum * kGBN;    // scale columns follow the accumulators
 constexpr uint32_t kGTmemCols = 512;
@@ -64,7 +65,7 @@ constexpr int kGThreads = 320;
 constexpr size_t kGDynSmem = kGStages * kGStageBytes + 1024;
 
 struct GemmShared {
-  uint64_t full[kGStages];     // A and B bytes of the stage landed
+  uint64_t full[kGStages];     // A and B codes and scale bytes of the stage landed
   uint64_t sf_full[kGStages];  // the stage's scale factors are in tensor memory (4 writer warps)
   uint64_t empty[kGStages];    // the MMAs that read the stage completed
   uint64_t tfull[kGAccum];     // accumulator holds a finished tile
@@ -86,7 +87,7 @@ __device__ __forceinline__ bool aborted(GemmShared& sh) {
 template <int OUT_BF16>
 __global__ void __launch_bounds__(kGThreads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                  const uint8_t* __restrict__ a_scales, const uint8_t* __restrict__ b_scales,
+                  const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ CUtensorMap tmap_sb,
                   const float* __restrict__ a_gscale, const float* __restrict__ b_gscale, int64_t m, int64_t n,
                   int64_t k, void* __restrict__ d, int64_t ldd) {
   extern __shared__ uint8_t dyn_smem[];
@@ -128,6 +129,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     if (lane == 0) {
       prefetch_tensormap(&tmap_a);
       prefetch_tensormap(&tmap_b);
+      prefetch_tensormap(&tmap_sa);
+      prefetch_tensormap(&tmap_sb);
       uint32_t it = 0;
       for (int64_t t = blockIdx.x; t < n_tiles && !aborted(sh); t += step) {
         const int32_t ya = static_cast<int32_t>((t / n_tn) * kGBM), yb = static_cast<int32_t>((t % n_tn) * kGBN);
@@ -139,10 +142,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           }
           if (aborted(sh)) break;
           uint8_t* dst = tiles + s * kGStageBytes;
+          // codes (x in bytes, 128 per K tile), then the scale bytes (x = 16
+          // per K tile): both multiples of 16.  Issuing the 16-byte scale rows
+          // ahead of the codes measured slower.
           mbar_arrive_expect_tx(&sh.full[s], kGStageBytes);
-          // x in bytes: 128 per K tile, a multiple of 16
           tma_load_2d(dst, &tmap_a, kt * (kGBK / 2), ya, &sh.full[s]);
           tma_load_2d(dst + kGOpBytes, &tmap_b, kt * (kGBK / 2), yb, &sh.full[s]);
+          tma_load_2d(dst + 2 * kGOpBytes, &tmap_sa, kt * (kGBK / 16), ya, &sh.full[s]);
+          tma_load_2d(dst + 2 * kGOpBytes + kGSfBytes, &tmap_sb, kt * (kGBK / 16), yb, &sh.full[s]);
           sh.issued_ab = (sh.issued_ab & ~(0x101u << s)) | (1u << s) | ((u & 1u) << (8 + s));
         }
       }
@@ -192,45 +199,42 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
   } else if (warp < kGEpiWarp0) {
     // ------------------------------------------------- scale-factor writers
     // warp q = warp % 4 fills lane quarter q; its thread l carries rows l,
-    // 32 + l, 64 + l, 96 + l of the tile, 16 scale bytes (one K tile) each
+    // 32 + l, 64 + l, 96 + l of the tile, 16 scale bytes (one K tile) each.
+    // The stage landing (full) also means the MMAs of the stage's previous
+    // use have completed (the producer waited for them before loading), so
+    // its scale columns are free.
     const uint32_t q = warp & 3u;
-    const int64_t srow = k / 16;  // scale bytes per row
     uint32_t it = 0;
-    for (int64_t t = blockIdx.x; t < n_tiles && !aborted(sh); t += step) {
-      const int64_t ra = (t / n_tn) * kGBM + lane, rb = (t % n_tn) * kGBN + lane;
-      bool ok = true;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < n_tiles && ok && !aborted(sh); t += step) {
       for (int kt = 0; kt < kt_count; ++kt, ++it) {
         const uint32_t s = it % kGStages, u = it / kGStages;
-        uint4 va[4], vb[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          va[h] = __ldg(reinterpret_cast<const uint4*>(a_scales + (ra + 32 * h) * srow + kt * 16));
-          vb[h] = __ldg(reinterpret_cast<const uint4*>(b_scales + (rb + 32 * h) * srow + kt * 16));
-        }
-        if (it >= kGStages && !mbar_wait(&sh.empty[s], (u - 1) & 1u)) {
+        if (!mbar_wait(&sh.full[s], u & 1u)) {
           ok = false;
           break;
         }
-        tc_fence_after_sync();
-        // column 4j + h: the four factors of K step j of row 32h + l
+        const uint4* sa = reinterpret_cast<const uint4*>(tiles + s * kGStageBytes + 2 * kGOpBytes);
+        const uint4* sb = sa + kGBM;
         uint32_t ca[16], cb[16];
+        // column 4j + h: the four factors of K step j of row 32h + l
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          ca[h] = va[h].x, ca[4 + h] = va[h].y, ca[8 + h] = va[h].z, ca[12 + h] = va[h].w;
-          cb[h] = vb[h].x, cb[4 + h] = vb[h].y, cb[8 + h] = vb[h].z, cb[12 + h] = vb[h].w;
+          const uint4 va = sa[32 * h + lane], vb = sb[32 * h + lane];
+          ca[h] = va.x, ca[4 + h] = va.y, ca[8 + h] = va.z, ca[12 + h] = va.w;
+          cb[h] = vb.x, cb[4 + h] = vb.y, cb[8 + h] = vb.z, cb[12 + h] = vb.w;
         }
+        tc_fence_after_sync();
         const uint32_t sf = tmem_base + ((32u * q) << 16) + kGSfBase + s * kGSfCols;
-        tmem_st16_wait(sf, ca);
-        tmem_st16_wait(sf + 16, cb);
+        tmem_st16(sf, ca);
+        tmem_st_wait();
+        tmem_st16(sf + 16, cb);
+        tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.sf_full[s]);
       }
-      if (!ok) {
-        atomicExch(&sh.abort_flag, 1);
-        break;
-      }
     }
+    if (!ok) atomicExch(&sh.abort_flag, 1);
   } else {
     // ------------------------------------------------------------ epilogue
     const uint32_t q = warp & 3u;
@@ -329,10 +333,24 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// rows x (k / 16) scale bytes, boxes of 16 bytes x 128 rows (no swizzle).
+bool make_scales_map(CUtensorMap* map, const uint8_t* scales, int64_t rows, int64_t k) {
+  EncodeTiledFn fn = gemm_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 16), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 16)};
+  cuuint32_t box[2] = {kGBK / 16, kGBM};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(scales), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int OUT_BF16>
 cudaError_t launch_gemm_t(const GemmArgs& g) {
-  CUtensorMap ma, mb;
-  if (!make_codes_map(&ma, g.a_codes, g.m, g.k) || !make_codes_map(&mb, g.b_codes, g.n, g.k))
+  CUtensorMap ma, mb, msa, msb;
+  if (!make_codes_map(&ma, g.a_codes, g.m, g.k) || !make_codes_map(&mb, g.b_codes, g.n, g.k) ||
+      !make_scales_map(&msa, g.a_scales, g.m, g.k) || !make_scales_map(&msb, g.b_scales, g.n, g.k))
     return cudaErrorInvalidValue;
   auto kernel = nvfp4_gemm_kernel<OUT_BF16>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kGDynSmem));
@@ -344,7 +362,7 @@ cudaError_t launch_gemm_t(const GemmArgs& g) {
   const int64_t grid = n_tiles < sms ? n_tiles : sms;
   if (grid == 0) return cudaSuccess;
   kernel<<<static_cast<unsigned>(grid), kGThreads, kGDynSmem, g.stream>>>(
-      ma, mb, g.a_scales, g.b_scales, g.a_gscale, g.b_gscale, g.m, g.n, g.k, g.d, g.ldd);
+      ma, mb, msa, msb, g.a_gscale, g.b_gscale, g.m, g.n, g.k, g.d, g.ldd);
   return cudaGetLastError();
 }
 

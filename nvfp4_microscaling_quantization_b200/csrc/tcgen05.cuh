@@ -85,15 +85,15 @@ __device__ __forceinline__ void umma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uin
 
 // 32 lanes x 16 consecutive 32-bit columns from registers: thread i of the
 // warp writes lane (the warp's lane quarter base + i), columns taddr.col ..
-// +15; the wait makes the writes complete before the thread goes on.
-__device__ __forceinline__ void tmem_st16_wait(uint32_t taddr, const uint32_t (&v)[16]) {
+// +15.  Asynchronous: tmem_st_wait() completes this thread's stores.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Arrive (once) on an mbarrier when every tcgen05 operation this thread issued
 // before has completed.
