@@ -98,8 +98,8 @@ NVFP4_API size_t nvfp4_workspace_bytes(int64_t rows, int64_t cols, int layout, i
  * z the view rotated by the RHT when rht_group > 0.  This is the pre-pass of
  * nvfp4_quantize, exposed so a caller can compute the amax once (or take it
  * from a producer) and pass it as amax_in.  amax_out: one device float,
- * overwritten.  Source: "FP32 scale per tensor", Quartet II article, section
- * "Quantisierung im Vorwaertsdurchlauf". */
+ * overwritten.  Source: the FP32 per-tensor scale of the Quartet II article,
+ * section "Quantisierung im Vorwaertsdurchlauf". */
 NVFP4_API int nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int layout,
                int rht_group, uint64_t seed, float* amax_out, void* stream);
 

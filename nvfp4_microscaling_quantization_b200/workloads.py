@@ -33,8 +33,9 @@ from typing import Dict, List, Tuple
 import torch
 
 ROWWISE, TRANSPOSED = 0, 1
-RTN, SR, MS_EDEN, IF4, FOUR_OVER_SIX = 0, 1, 2, 3, 4
-MODE_NAMES = {RTN: "rtn", SR: "sr", MS_EDEN: "ms_eden", IF4: "if4", FOUR_OVER_SIX: "4over6"}
+RTN, SR, MS_EDEN, IF4, FOUR_OVER_SIX, SCALE_SEARCH = 0, 1, 2, 3, 4, 5
+MODE_NAMES = {RTN: "rtn", SR: "sr", MS_EDEN: "ms_eden", IF4: "if4", FOUR_OVER_SIX: "4over6",
+              SCALE_SEARCH: "scale_search"}
 LAYOUT_NAMES = {ROWWISE: "rowwise", TRANSPOSED: "transposed"}
 
 

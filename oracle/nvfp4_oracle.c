@@ -14,8 +14,8 @@
  * and no fast-math, so the compiler never fuses or reorders it.  The only
  * fused operation is the explicit C99 fmaf() used for the per-block dot
  * products, which is itself a single correctly rounded operation.  binary32
- * is the precision the pages fix for the per-tensor scale ("FP32 scale per
- * tensor"), and every integer decision (a 4-bit code, an 8-bit scale, the IF4
+ * is the precision the pages fix for the per-tensor scale (an FP32 scale per
+ * tensor), and every integer decision (a 4-bit code, an 8-bit scale, the IF4
  * flag, the 4/6 choice) is taken in that precision on both sides.
  *
  * Sources (page title, then section / table / figure):
@@ -34,6 +34,9 @@
  *  [IF4-abs]  IF4 paper page (arXiv 2603.28765, "Adaptive Block-Scaled Data
  *             Types"), abstract; [IF4-F1] its Figure 1; [IF4-T1] its Table 1;
  *             [IF4-F3] its Figure 3.
+ *  [SS-abs]   the same IF4 paper page, its related-paper entry on ScaleSearch
+ *             (abstract): block scales chosen by searching the scale's
+ *             mantissa values for the lowest quantization error.
  *  [PHILOX]   Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy
  *             as 1, 2, 3", SC'11 -- the Philox4x32 bijection with 10 rounds.
  *
@@ -53,7 +56,7 @@
 
 /* modes and layouts: same numbering as the public C ABI (an interface, not
  * shared code). */
-enum { ORC_RTN = 0, ORC_SR = 1, ORC_MS_EDEN = 2, ORC_IF4 = 3, ORC_4OVER6 = 4 };
+enum { ORC_RTN = 0, ORC_SR = 1, ORC_MS_EDEN = 2, ORC_IF4 = 3, ORC_4OVER6 = 4, ORC_SCALE_SEARCH = 5 };
 enum { ORC_ROWWISE = 0, ORC_TRANSPOSED = 1 };
 
 /* ------------------------------------------------------------------------ */
@@ -327,7 +330,7 @@ static void load_view_row(const uint16_t* x, int64_t ld, int layout, int64_t vr,
 static int check_quant_args(int64_t rows, int64_t cols, int64_t ld, int layout,
                             int mode, int g, int64_t* vr, int64_t* vc) {
   if (layout != ORC_ROWWISE && layout != ORC_TRANSPOSED) return ORC_ERR_ARG;
-  if (mode < ORC_RTN || mode > ORC_4OVER6) return ORC_ERR_ARG;
+  if (mode < ORC_RTN || mode > ORC_SCALE_SEARCH) return ORC_ERR_ARG;
   if (g != 0 && !valid_group(g)) return ORC_ERR_ARG;
   if (mode == ORC_MS_EDEN && g == 0) return ORC_ERR_UNSUPPORTED;
   if (rows < 0 || cols < 0 || ld < cols) return ORC_ERR_SHAPE;
@@ -361,10 +364,13 @@ int oracle_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int l
   return ORC_OK;
 }
 
-/* FP32 per-tensor scale s_g.  Reading ([QII-fwd] gives only "FP32 scale per
- * tensor"; [IF4-T1] gives the maxima 6 x 448 and, for 4/6, 6 x 256): the
+/* FP32 per-tensor scale s_g.  Reading ([QII-fwd] only says that each tensor
+ * has an FP32 scale; [IF4-T1] gives the maxima 6 x 448 and, for 4/6, 6 x 256): the
  * tensor amax is mapped to the format maximum, s_g = RN(A / (6 M)) with
- * M = 448, or M = 256 for 4/6 and for MS-EDEN.  A zero tensor gets s_g = 1.
+ * M = 448, or M = 256 for 4/6, MS-EDEN and scale search.  A zero tensor
+ * gets s_g = 1.  Scale search takes 256 like 4/6, whose larger-scale option
+ * it contains: its upper candidates then reach above the absmax scale before
+ * the E4M3 maximum.
  * MS-EDEN takes the 4/6 cap for the same reason 4/6 does: its block scale is
  * later multiplied by a correction factor c, and the scale's stochastic
  * rounding must never saturate at 448 or it loses unbiasedness.  c stays
@@ -372,7 +378,8 @@ int oracle_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int l
  * elements rounded to zero add at most 15 * 0.25^2 to <y, y>, and the block
  * maximum contributes at least 3 * 3 to <y, v>; so 256 * 1.61 < 448. */
 float oracle_global_scale(float A, int mode) {
-  float sixM = (mode == ORC_4OVER6 || mode == ORC_MS_EDEN) ? 1536.0f : 2688.0f; /* exact */
+  float sixM = (mode == ORC_4OVER6 || mode == ORC_MS_EDEN || mode == ORC_SCALE_SEARCH) ? 1536.0f
+                                                                                      : 2688.0f; /* exact */
   if (!(A > 0.0f)) return 1.0f;
   return A / sixM;
 }
@@ -400,7 +407,7 @@ static float int4_value(int k) { return (float)k * IF4_K2; }
  * Writes 16 codes (one per element, low nibble) and returns the scale byte. */
 static uint8_t quantize_block(const float* z, int mode, float s_g, uint64_t seed,
                               int64_t vr, int64_t vc, int64_t bc, uint8_t* code) {
-  float a_b = 0.0f; /* block absmax [PAL-corners] "scales each block by its absmax" */
+  float a_b = 0.0f; /* block absmax [PAL-corners]: the absmax sets each block's scale */
   for (int i = 0; i < 16; ++i)
     if (fabsf(z[i]) > a_b) a_b = fabsf(z[i]);
 
@@ -435,6 +442,49 @@ static uint8_t quantize_block(const float* z, int mode, float s_g, uint64_t seed
     int pick = err[1] < err[0] ? 1 : 0;
     memcpy(code, cc[pick], 16);
     return Sc[pick];
+  }
+
+  if (mode == ORC_SCALE_SEARCH) {
+    /* Scale search [PAL-corners]: the low-error corner tries 19 candidate
+     * scales per block with round-to-nearest and keeps the one with the
+     * least error; [SS-abs]: a search over the microscale's mantissa values
+     * for the lowest quantization error.
+     * Reading: the candidates are the 19 E4M3 codes S0 - 9 .. S0 + 9 around
+     * the absmax scale S0 = E4M3_RNE(RN(a_b / RN(6 s_g))) (E4M3 codes are
+     * ordered like their values, so a code step is one mantissa step),
+     * clamped to 0 .. 0x7E and visited in the order S0, S0 - 1, S0 + 1,
+     * S0 - 2, ...; each is scored as 4/6 scores its two (RTN codes, squared
+     * error in the original domain, fmaf in element order); only a strictly
+     * lower error replaces the best so far, so ties keep the candidate
+     * nearest S0, and S0 first. */
+    float q0 = 6.0f * s_g;
+    int S0 = oracle_e4m3_rne_sat(a_b / q0);
+    uint8_t best_S = 0, cc[16];
+    float best_e = INFINITY;
+    for (int t = 0; t < 19; ++t) {
+      int delta = ((t + 1) / 2) * ((t & 1) ? -1 : 1);
+      int Sc = S0 + delta;
+      if (Sc < 0) Sc = 0;
+      if (Sc > 0x7E) Sc = 0x7E;
+      float d = oracle_e4m3_decode((uint8_t)Sc) * s_g;
+      float e = 0.0f;
+      if (d == 0.0f) {
+        for (int i = 0; i < 16; ++i) { cc[i] = 0; e = fmaf(z[i], z[i], e); }
+      } else {
+        float r = 1.0f / d;
+        for (int i = 0; i < 16; ++i) {
+          cc[i] = oracle_e2m1_rtn(z[i] * r);
+          float diff = z[i] - oracle_e2m1_decode(cc[i]) * d;
+          e = fmaf(diff, diff, e);
+        }
+      }
+      if (e < best_e) {
+        best_e = e;
+        best_S = (uint8_t)Sc;
+        memcpy(code, cc, 16);
+      }
+    }
+    return best_S;
   }
 
   float q = 6.0f * s_g;
@@ -560,7 +610,7 @@ int oracle_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, i
 int oracle_dequantize(const uint8_t* codes, const uint8_t* scales, float s_g,
                       int64_t vr, int64_t vc, int mode, int g, uint64_t seed,
                       int inverse_rht, float* out) {
-  if (mode < ORC_RTN || mode > ORC_4OVER6) return ORC_ERR_ARG;
+  if (mode < ORC_RTN || mode > ORC_SCALE_SEARCH) return ORC_ERR_ARG;
   if (g != 0 && !valid_group(g)) return ORC_ERR_ARG;
   if (vr < 0 || vc < 0 || vc % 16 || (g && vc % g)) return ORC_ERR_SHAPE;
   if (inverse_rht && g == 0) return ORC_ERR_ARG;
@@ -618,7 +668,7 @@ void oracle_e4m3_array(const float* in, int64_t n, int round_up, uint8_t* out) {
 int oracle_quantize_rotated(const float* z, int64_t row0, int64_t vr, int64_t vc, int mode,
                             uint64_t seed, float amax, uint8_t* codes, uint8_t* scales,
                             float* global_scale) {
-  if (mode < ORC_RTN || mode > ORC_4OVER6) return ORC_ERR_ARG;
+  if (mode < ORC_RTN || mode > ORC_SCALE_SEARCH) return ORC_ERR_ARG;
   if (row0 < 0 || vr < 0 || vc < 0 || vc % 16) return ORC_ERR_SHAPE;
   float s_g = oracle_global_scale(amax, mode);
   *global_scale = s_g;

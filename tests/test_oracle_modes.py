@@ -12,6 +12,11 @@
   the scale's sign bit (IF4 paper page, abstract, Figure 1 and Figure 3).
 * 4/6 keeps the lower-error of the two block scales (Quartet II article,
   "Quantisierung im Vorwaertsdurchlauf"; IF4 page Table 1, scale max 256).
+* Scale search keeps the lowest-error of the 19 E4M3 codes around the absmax
+  scale (palettes post, "The two corners, and what the palette does to
+  them"; the ScaleSearch entry of the IF4 page): checked against a search
+  recomputed with torch's E4M3 decoder and a brute-force E2M1 rounding, and
+  per block no worse than 4/6, whose two scales are among its candidates.
 * Structural properties: transposed view = row-wise quantization of X^T,
   leading dimension, amax_in, zero tensor and zero blocks, nibble order.
 """
@@ -22,7 +27,7 @@ import torch
 from nvfp4_microscaling_quantization_b200 import workloads as W
 
 ROW, TR = 0, 1
-RTN, SR, EDEN, IF4, FO6 = 0, 1, 2, 3, 4
+RTN, SR, EDEN, IF4, FO6, SS = 0, 1, 2, 3, 4, 5
 GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
 
 
@@ -265,8 +270,76 @@ def test_four_over_six_not_worse_than_rtn(orc):
     assert m_46 <= m_rtn
 
 
+# ------------------------------------------------------------------ scale search
+def _e4m3_value(code):
+    return np.float32(torch.tensor([code], dtype=torch.uint8).view(torch.float8_e4m3fn).float().item())
+
+
+def _e2m1_rtn_value(y):
+    """Nearest E2M1 grid value to y (float32), ties to the even code index (brute force)."""
+    a = min(abs(float(y)), 6.0)
+    dist = np.abs(GRID - a)
+    best = np.flatnonzero(dist == dist.min())
+    i = best[0] if len(best) == 1 else best[best % 2 == 0][0]
+    return np.float32(-GRID[i] if y < 0 else GRID[i])
+
+
+def test_scale_search_picks_lowest_of_19(orc):
+    wl = W.weight(rows=8, cols=256)
+    bits = bits_of(wl.tensors()["w"])
+    codes, scales, gs, z = _block_views(orc, bits, ROW, SS, 0, 1)
+    assert gs == orc.global_scale(np.abs(z).max(), FO6)  # tensor scale M = 256, as 4/6
+    cu = orc.unpack_codes(codes)
+    moved = 0
+    for r in range(z.shape[0]):
+        for b in range(z.shape[1] // 16):
+            zb = z[r, 16 * b:16 * b + 16]
+            ab = f32(np.abs(zb).max())
+            S0 = orc.e4m3_rne_sat(f32(ab / f32(f32(6.0) * f32(gs))))
+            errs = {}
+            for delta in range(-9, 10):
+                Sc = min(max(S0 + delta, 0), 0x7E)
+                d = f32(_e4m3_value(Sc) * f32(gs))
+                if d == 0:
+                    errs[Sc] = float(np.sum(zb.astype(np.float64) ** 2))
+                    continue
+                y = (zb * f32(f32(1.0) / d)).astype(np.float32)
+                v = np.array([_e2m1_rtn_value(t) for t in y], dtype=np.float32)
+                errs[Sc] = float(np.sum((zb.astype(np.float64) - (v * d).astype(np.float32)) ** 2))
+            S = int(scales[r, b])
+            assert S in errs, (r, b)
+            assert errs[S] <= min(errs.values()) * (1 + 1e-5) + 1e-30, (r, b)
+            d = f32(_e4m3_value(S) * f32(gs))
+            if d > 0:  # codes are the RTN codes under the chosen scale
+                y = (zb * f32(f32(1.0) / d)).astype(np.float32)
+                vals = np.array([orc.e2m1_decode(int(c)) for c in cu[r, 16 * b:16 * b + 16]], dtype=np.float32)
+                assert np.array_equal(vals, np.array([_e2m1_rtn_value(t) for t in y], dtype=np.float32))
+            moved += S != S0
+    print(f"\nscale search: scale moved off the absmax scale in {moved} of {len(scales.flat)} blocks")
+    assert moved > 0
+
+
+def test_scale_search_no_worse_than_four_over_six_per_block(orc):
+    wl = W.weight(rows=64, cols=512)
+    bits = bits_of(wl.tensors()["w"])
+    z = bits_of(wl.tensors()["w"])
+    z = torch.from_numpy(z.view(np.int16)).view(torch.bfloat16).double().numpy()
+    errs = {}
+    for mode in (FO6, SS):
+        c, s, gs = orc.quantize(bits, ROW, mode, 0, 1)
+        dq = deq(orc, c, s, gs, mode, 0, 1)
+        errs[mode] = ((z - dq) ** 2).reshape(z.shape[0], -1, 16).sum(-1)
+    assert np.all(errs[SS] <= errs[FO6] * (1 + 1e-6) + 1e-30)
+    m_rtn = _mse(orc, wl.tensors()["w"], RTN, 0, [0])
+    m_46, m_ss = errs[FO6].sum() / z.size, errs[SS].sum() / z.size
+    print(f"\nweight-like MSE: RTN {m_rtn:.3e}  4/6 {m_46:.3e}  scale search {m_ss:.3e} "
+          f"({100 * (1 - m_ss / m_rtn):.1f}% below RTN)")
+    assert m_ss <= m_46 <= m_rtn
+
+
 # ------------------------------------------------------------------- structural
-@pytest.mark.parametrize("mode,g", [(RTN, 0), (SR, 0), (EDEN, 128), (IF4, 0), (FO6, 0), (SR, 32)])
+@pytest.mark.parametrize("mode,g", [(RTN, 0), (SR, 0), (EDEN, 128), (IF4, 0), (FO6, 0), (SR, 32), (SS, 0),
+                                    (SS, 64)])
 def test_transposed_is_rowwise_of_transpose(orc, mode, g):
     rng = np.random.default_rng(6)
     x = bf16(rng.standard_normal((256, 64)))
