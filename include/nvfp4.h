@@ -86,7 +86,11 @@ typedef enum {
   NVFP4_SR = 1,      /* stochastic rounding, block scale rounded up, amax -> 6 x 448 */
   NVFP4_MS_EDEN = 2, /* RTN codes + EDEN-corrected, stochastically rounded scale; needs g > 0; amax -> 6 x 256 */
   NVFP4_IF4 = 3,     /* per block FP4 or scaled INT4 (flag in scale bit 7), amax -> 6 x 448 */
-  NVFP4_4OVER6 = 4   /* per block scale mapping the absmax to 6 or to 4, amax -> 6 x 256 */
+  NVFP4_4OVER6 = 4,  /* per block scale mapping the absmax to 6 or to 4, amax -> 6 x 256 */
+  NVFP4_SCALE_SEARCH = 5 /* per block the best of 19 E4M3 scales around the absmax scale (lowest
+                            squared error, RTN codes; palettes post, "The two corners, and what
+                            the palette does to them"; the ScaleSearch entry of the IF4 paper
+                            page), amax -> 6 x 256 */
 } nvfp4_mode;
 
 /* Bytes of device workspace nvfp4_quantize needs when amax_in is NULL (the
@@ -124,7 +128,7 @@ NVFP4_API int nvfp4_amax_dual(const void* x, int64_t rows, int64_t cols, int64_t
  *  amax_in:   device float holding the tensor amax of the (rotated) view, or
  *             NULL to compute it in a pre-pass (needs the workspace).  The
  *             tensor scale is s_g = RN(amax / (6 M)), M = 448 (RTN, SR, IF4)
- *             or 256 (MS-EDEN, 4/6); s_g = 1 for a zero amax.
+ *             or 256 (MS-EDEN, 4/6, scale search); s_g = 1 for a zero amax.
  *  codes, scales, global_scale: outputs (sizes above); global_scale is one
  *             device float.
  *  workspace: device memory of at least nvfp4_workspace_bytes(...) bytes when
@@ -162,7 +166,8 @@ typedef enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 } nvfp4_out_dtype;
  * authors' kernels run linear layers up to 4.2x faster than BF16; the
  * article's sections "Quantisierung im Vorwaertsdurchlauf" and "...
  * Rueckwaertsdurchlauf" for which operand is quantized along which
- * dimension).  The scales must be plain E4M3 (modes RTN, SR, MS-EDEN, 4/6):
+ * dimension).  The scales must be plain E4M3 (modes RTN, SR, MS-EDEN, 4/6,
+ * scale search):
  * an IF4 scale carries the INT4 flag in bit 7, which the tensor cores do not
  * interpret, so IF4 outputs are not valid operands.  Two operands rotated along k with
  * the same seed and group give the product of the unrotated ones up to the

@@ -15,7 +15,17 @@
 
 namespace nvfp4 {
 
-enum Mode { kRTN = 0, kSR = 1, kMSEDEN = 2, kIF4 = 3, k4over6 = 4 };
+enum Mode { kRTN = 0, kSR = 1, kMSEDEN = 2, kIF4 = 3, k4over6 = 4, kScaleSearch = 5 };
+
+// Scale search: the candidates are the E4M3 codes S0 + delta(t), t = 0 ..
+// 18, around the absmax scale S0, visited nearest first (0, -1, +1, -2, ...),
+// clamped to 0 .. 0x7E; a strictly lower error replaces the best so far.
+constexpr int kSearchCandidates = 19;
+__host__ __device__ constexpr int search_delta(int t) { return ((t + 1) / 2) * ((t & 1) ? -1 : 1); }
+__device__ __forceinline__ uint32_t search_code(uint32_t s0, int t) {
+  const int s = static_cast<int>(s0) + search_delta(t);
+  return static_cast<uint32_t>(s < 0 ? 0 : (s > 0x7E ? 0x7E : s));
+}
 
 // ---------------------------------------------------------------------------
 // Two-lane binary32 arithmetic (sm_100a f32x2): each lane is one IEEE RN
@@ -268,10 +278,11 @@ __device__ __forceinline__ void rht_inverse(float* v, uint32_t sign_bits, uint32
 }
 
 // ---------------------------------------------------------------------------
-// Tensor scale: s_g = RN(A / (6 M)), M = 256 for MS-EDEN and 4/6, else 448.
+// Tensor scale: s_g = RN(A / (6 M)), M = 256 for MS-EDEN, 4/6 and scale
+// search, else 448.
 template <int MODE>
 __device__ __forceinline__ float global_scale_of(float amax) {
-  constexpr float six_m = (MODE == kMSEDEN || MODE == k4over6) ? 1536.0f : 2688.0f;
+  constexpr float six_m = (MODE == kMSEDEN || MODE == k4over6 || MODE == kScaleSearch) ? 1536.0f : 2688.0f;
   return amax > 0.0f ? __fdiv_rn(amax, six_m) : 1.0f;
 }
 
@@ -375,6 +386,41 @@ __device__ __forceinline__ BlockOut quantize_block(const float* z, float s_g, co
     out.lo = c_lo[pick];
     out.hi = c_hi[pick];
     out.scale = S[pick];
+    return out;
+  } else if constexpr (MODE == kScaleSearch) {
+    const uint32_t s0 = e4m3_rne_sat(__fdiv_rn(a_b, __fmul_rn(6.0f, s_g)));
+    float best = __int_as_float(0x7F800000);  // +inf
+#pragma unroll 1
+    for (int t = 0; t < kSearchCandidates; ++t) {
+      const uint32_t S = search_code(s0, t);
+      const float d = __fmul_rn(e4m3_decode(S), s_g);
+      uint32_t lo = 0u, hi = 0u;
+      float e = 0.0f;
+      if (d == 0.0f) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) e = __fmaf_rn(z[i], z[i], e);
+      } else {
+        const float r = __frcp_rn(d);
+        float y[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(z[i], r);
+        rtn_codes(y, lo, hi);
+        float v[16];
+        e2m1x8_to_f32(lo, v);
+        e2m1x8_to_f32(hi, v + 8);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float diff = __fsub_rn(z[i], __fmul_rn(v[i], d));
+          e = __fmaf_rn(diff, diff, e);
+        }
+      }
+      if (e < best) {
+        best = e;
+        out.lo = lo;
+        out.hi = hi;
+        out.scale = S;
+      }
+    }
     return out;
   } else {
     const float s_f = __fdiv_rn(a_b, __fmul_rn(6.0f, s_g));
@@ -631,6 +677,51 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
     ob.lo = pb ? cb_lo[1] : cb_lo[0];
     ob.hi = pb ? cb_hi[1] : cb_hi[0];
     ob.scale = ((pb ? S[1] : S[0]) >> 8) & 0xFFu;
+    return;
+  } else if constexpr (MODE == kScaleSearch) {
+    const float2 sf = div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein);
+    const uint32_t s02 = e4m3x2_rne_sat(sf.x, sf.y);
+    const uint32_t s0a = s02 & 0xFFu, s0b = s02 >> 8;
+    float2 best = f2(__int_as_float(0x7F800000), __int_as_float(0x7F800000));
+    oa = BlockOut{0u, 0u, 0u};
+    ob = BlockOut{0u, 0u, 0u};
+#pragma unroll 1
+    for (int t = 0; t < kSearchCandidates; ++t) {
+      const uint32_t Sa = search_code(s0a, t), Sb = search_code(s0b, t);
+      const float4 ta = scale_entry<TBL>(sc, Sa), tb = scale_entry<TBL>(sc, Sb);
+      const float2 d = f2(ta.y, tb.y), r = f2(ta.z, tb.z);
+      // a zero scale (d = 0, RN(1/d) tabulated as 0) gives y = 0, codes 0 and
+      // the error sum of z^2, as the block with no scale
+      float ya[16], yb[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 y = mul2_rn(z[i], r);
+        ya[i] = y.x;
+        yb[i] = y.y;
+      }
+      uint32_t ca_lo, ca_hi, cb_lo, cb_hi;
+      rtn_codes(ya, ca_lo, ca_hi);
+      rtn_codes(yb, cb_lo, cb_hi);
+      float va[16], vb[16];
+      e2m1x8_to_f32(ca_lo, va);
+      e2m1x8_to_f32(ca_hi, va + 8);
+      e2m1x8_to_f32(cb_lo, vb);
+      e2m1x8_to_f32(cb_hi, vb + 8);
+      float2 e = f2(0.0f, 0.0f);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 diff = sub2_after_mul(z[i], mul2_rn(f2(va[i], vb[i]), d));
+        e = fma2_rn(diff, diff, e);
+      }
+      if (e.x < best.x) {
+        best.x = e.x;
+        oa = BlockOut{ca_lo, ca_hi, Sa};
+      }
+      if (e.y < best.y) {
+        best.y = e.y;
+        ob = BlockOut{cb_lo, cb_hi, Sb};
+      }
+    }
     return;
   } else {
     const float2 sf = div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein);

@@ -253,6 +253,7 @@ cudaError_t launch_quantize(const QuantArgs& a) {
     case kMSEDEN: return dispatch_group<kMSEDEN, false>(a);
     case kIF4: return dispatch_group<kIF4, false>(a);
     case k4over6: return dispatch_group<k4over6, false>(a);
+    case kScaleSearch: return dispatch_group<kScaleSearch, false>(a);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -52,7 +52,8 @@ enum Kind { kQuantize = 0, kAmax = 1, kStoreZ = 2 };
 // everything else four (18 warps, 96 registers).
 template <int MODE, int KIND>
 struct Shape {
-  static constexpr int groups = (KIND == kQuantize && MODE == kSR) ? 3 : 4;
+  // SR (Philox) and scale search (19 candidates) get 128 registers a thread
+  static constexpr int groups = (KIND == kQuantize && (MODE == kSR || MODE == kScaleSearch)) ? 3 : 4;
   static constexpr int epi_warps = 4 * groups;
   static constexpr int producer_warp = epi_warps, mma_warp = epi_warps + 1;
   static constexpr int threads = (epi_warps + 2) * 32;
@@ -763,6 +764,7 @@ cudaError_t launch_quantize_mma(const QuantArgs& a) {
     case kMSEDEN: return dispatch<kMSEDEN, kQuantize>(a, nullptr);
     case kIF4: return dispatch<kIF4, kQuantize>(a, nullptr);
     case k4over6: return dispatch<k4over6, kQuantize>(a, nullptr);
+    case kScaleSearch: return dispatch<kScaleSearch, kQuantize>(a, nullptr);
     default: return cudaErrorInvalidValue;
   }
 }

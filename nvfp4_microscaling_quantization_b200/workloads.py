@@ -150,8 +150,8 @@ def small(rows=256, cols=256) -> Workload:
 
 
 def weight(rows=4096, cols=4096) -> Workload:
-    """Weight-like 4096x4096 N(0, 0.02^2) with 1% outliers x10, seed 1: RTN and 4/6 row-wise."""
-    calls = [Call("w", ROWWISE, RTN, 0), Call("w", ROWWISE, FOUR_OVER_SIX, 0)]
+    """Weight-like 4096x4096 N(0, 0.02^2) with 1% outliers x10, seed 1: RTN, 4/6 and scale search row-wise."""
+    calls = [Call("w", ROWWISE, RTN, 0), Call("w", ROWWISE, FOUR_OVER_SIX, 0), Call("w", ROWWISE, SCALE_SEARCH, 0)]
     return Workload("weight", 1, {"w": (rows, cols)}, calls, "4096x4096 N(0,0.02) + 1% x10 outliers")
 
 

@@ -22,7 +22,8 @@ from nvfp4_microscaling_quantization_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 CASES = [(W.ROWWISE, W.RTN, 0), (W.ROWWISE, W.MS_EDEN, 128), (W.TRANSPOSED, W.MS_EDEN, 128),
-         (W.TRANSPOSED, W.SR, 32), (W.ROWWISE, W.IF4, 0), (W.ROWWISE, W.FOUR_OVER_SIX, 16)]
+         (W.TRANSPOSED, W.SR, 32), (W.ROWWISE, W.IF4, 0), (W.ROWWISE, W.FOUR_OVER_SIX, 16),
+         (W.TRANSPOSED, W.SCALE_SEARCH, 0)]
 
 
 def _noalloc(x, layout, mode, g, seed, stream):
