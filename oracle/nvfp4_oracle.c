@@ -56,7 +56,7 @@
 
 /* modes and layouts: same numbering as the public C ABI (an interface, not
  * shared code). */
-enum { ORC_RTN = 0, ORC_SR = 1, ORC_MS_EDEN = 2, ORC_IF4 = 3, ORC_4OVER6 = 4, ORC_SCALE_SEARCH = 5 };
+enum { ORC_RTN = 0, ORC_SR = 1, ORC_MS_EDEN = 2, ORC_IF4 = 3, ORC_4OVER6 = 4, ORC_SCALE_SEARCH = 5, ORC_MXFP4 = 6 };
 enum { ORC_ROWWISE = 0, ORC_TRANSPOSED = 1 };
 
 /* ------------------------------------------------------------------------ */
@@ -330,13 +330,14 @@ static void load_view_row(const uint16_t* x, int64_t ld, int layout, int64_t vr,
 static int check_quant_args(int64_t rows, int64_t cols, int64_t ld, int layout,
                             int mode, int g, int64_t* vr, int64_t* vc) {
   if (layout != ORC_ROWWISE && layout != ORC_TRANSPOSED) return ORC_ERR_ARG;
-  if (mode < ORC_RTN || mode > ORC_SCALE_SEARCH) return ORC_ERR_ARG;
+  if (mode < ORC_RTN || mode > ORC_MXFP4) return ORC_ERR_ARG;
   if (g != 0 && !valid_group(g)) return ORC_ERR_ARG;
   if (mode == ORC_MS_EDEN && g == 0) return ORC_ERR_UNSUPPORTED;
   if (rows < 0 || cols < 0 || ld < cols) return ORC_ERR_SHAPE;
   *vr = layout == ORC_ROWWISE ? rows : cols;
   *vc = layout == ORC_ROWWISE ? cols : rows;
   if (*vc % 16) return ORC_ERR_SHAPE;
+  if (mode == ORC_MXFP4 && *vc % 32) return ORC_ERR_SHAPE;
   if (g > 0 && *vc % g) return ORC_ERR_SHAPE;
   return ORC_OK;
 }
@@ -378,6 +379,7 @@ int oracle_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int l
  * elements rounded to zero add at most 15 * 0.25^2 to <y, y>, and the block
  * maximum contributes at least 3 * 3 to <y, v>; so 256 * 1.61 < 448. */
 float oracle_global_scale(float A, int mode) {
+  if (mode == ORC_MXFP4) return 1.0f; /* MXFP4 has no tensor scale [IF4-T1] */
   float sixM = (mode == ORC_4OVER6 || mode == ORC_MS_EDEN || mode == ORC_SCALE_SEARCH) ? 1536.0f
                                                                                       : 2688.0f; /* exact */
   if (!(A > 0.0f)) return 1.0f;
@@ -410,6 +412,34 @@ static uint8_t quantize_block(const float* z, int mode, float s_g, uint64_t seed
   float a_b = 0.0f; /* block absmax [PAL-corners]: the absmax sets each block's scale */
   for (int i = 0; i < 16; ++i)
     if (fabsf(z[i]) > a_b) a_b = fabsf(z[i]);
+
+  if (mode == ORC_MXFP4) {
+    /* MXFP4 [IF4-T1]: 32-element groups, one UE8M0 (power of two) scale, E2M1
+     * values, no tensor scale; maximum 6 x 2^127, minimum 0.5 x 2^-127.
+     * Reading (the pages give only that row; the scale rule is that of the
+     * OCP Microscaling specification, whose format the row names): the
+     * shared exponent is E = floor(log2(max |x| over the group)) - 2 (2 = the
+     * exponent of E2M1's largest value), clamped to [-127, 127] (-127 for an
+     * all-zero group); the elements are x / 2^E rounded to nearest E2M1, ties
+     * to even, saturating at 6.  The scale byte is E + 127, stored for both
+     * 16-element halves of the group, so every mode has one scale per 16
+     * elements.  This block is the half (bc & 1) of its group. */
+    const float* grp = (bc & 1) ? z - 16 : z;
+    float a = 0.0f;
+    for (int i = 0; i < 32; ++i)
+      if (fabsf(grp[i]) > a) a = fabsf(grp[i]);
+    int E = -127;
+    if (a > 0.0f) {
+      int e2;
+      frexpf(a, &e2); /* a = m 2^e2, m in [0.5, 1): floor(log2 a) = e2 - 1 */
+      E = e2 - 1 - 2;
+      if (E < -127) E = -127;
+      if (E > 127) E = 127;
+    }
+    float X = ldexpf(1.0f, E);
+    for (int i = 0; i < 16; ++i) code[i] = oracle_e2m1_rtn(z[i] / X);
+    return (uint8_t)(E + 127);
+  }
 
   if (mode == ORC_4OVER6) {
     /* 4/6 [QII-fwd] "Four Over Six", [IF4-T1] scale maximum 256.  Reading:
@@ -610,9 +640,10 @@ int oracle_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, i
 int oracle_dequantize(const uint8_t* codes, const uint8_t* scales, float s_g,
                       int64_t vr, int64_t vc, int mode, int g, uint64_t seed,
                       int inverse_rht, float* out) {
-  if (mode < ORC_RTN || mode > ORC_SCALE_SEARCH) return ORC_ERR_ARG;
+  if (mode < ORC_RTN || mode > ORC_MXFP4) return ORC_ERR_ARG;
   if (g != 0 && !valid_group(g)) return ORC_ERR_ARG;
   if (vr < 0 || vc < 0 || vc % 16 || (g && vc % g)) return ORC_ERR_SHAPE;
+  if (mode == ORC_MXFP4 && vc % 32) return ORC_ERR_SHAPE;
   if (inverse_rht && g == 0) return ORC_ERR_ARG;
   for (int64_t r = 0; r < vr; ++r) {
     for (int64_t j = 0; j < vc; ++j) {
@@ -620,7 +651,8 @@ int oracle_dequantize(const uint8_t* codes, const uint8_t* scales, float s_g,
       uint8_t byte = codes[r * (vc / 2) + j / 2];
       uint8_t code = (j & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15u);
       int int4 = mode == ORC_IF4 && (S & 0x80u);
-      float d = oracle_e4m3_decode((uint8_t)(S & 0x7Fu)) * s_g;
+      float d = mode == ORC_MXFP4 ? ldexpf(1.0f, (int)S - 127)  /* UE8M0: 2^(S - 127) */
+                                  : oracle_e4m3_decode((uint8_t)(S & 0x7Fu)) * s_g;
       float v;
       if (int4) {
         int k = (int)(code & 7u);
@@ -668,8 +700,8 @@ void oracle_e4m3_array(const float* in, int64_t n, int round_up, uint8_t* out) {
 int oracle_quantize_rotated(const float* z, int64_t row0, int64_t vr, int64_t vc, int mode,
                             uint64_t seed, float amax, uint8_t* codes, uint8_t* scales,
                             float* global_scale) {
-  if (mode < ORC_RTN || mode > ORC_SCALE_SEARCH) return ORC_ERR_ARG;
-  if (row0 < 0 || vr < 0 || vc < 0 || vc % 16) return ORC_ERR_SHAPE;
+  if (mode < ORC_RTN || mode > ORC_MXFP4) return ORC_ERR_ARG;
+  if (row0 < 0 || vr < 0 || vc < 0 || vc % 16 || (mode == ORC_MXFP4 && vc % 32)) return ORC_ERR_SHAPE;
   float s_g = oracle_global_scale(amax, mode);
   *global_scale = s_g;
   for (int64_t r = 0; r < vr; ++r) {

@@ -17,6 +17,11 @@
   them"; the ScaleSearch entry of the IF4 page): checked against a search
   recomputed with torch's E4M3 decoder and a brute-force E2M1 rounding, and
   per block no worse than 4/6, whose two scales are among its candidates.
+* MXFP4 (IF4 page, Table 1: groups of 32, UE8M0 scale, max 6 x 2^127, min
+  0.5 x 2^-127): shared exponent floor(log2 amax) - 2 recomputed with numpy's
+  frexp, codes by brute-force nearest E2M1 of x / 2^E, a lossless round trip.
+* Table 1's MSE column (NVFP4 9.0, 4/6 7.5, IF4 6.2, MXFP4 13.2, x1e-3) on
+  standard normal data, within 2% (tests/golden/if4_table1_mse.txt).
 * Structural properties: transposed view = row-wise quantization of X^T,
   leading dimension, amax_in, zero tensor and zero blocks, nibble order.
 """
@@ -27,7 +32,7 @@ import torch
 from nvfp4_microscaling_quantization_b200 import workloads as W
 
 ROW, TR = 0, 1
-RTN, SR, EDEN, IF4, FO6, SS = 0, 1, 2, 3, 4, 5
+RTN, SR, EDEN, IF4, FO6, SS, MX = 0, 1, 2, 3, 4, 5, 6
 GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
 
 
@@ -337,9 +342,91 @@ def test_scale_search_no_worse_than_four_over_six_per_block(orc):
     assert m_ss <= m_46 <= m_rtn
 
 
+# ------------------------------------------------------------------------ MXFP4
+def _rtn_grid_index(a):
+    """Brute-force nearest E2M1 magnitude index of |a| <= 6 (ties to the even index)."""
+    dist = np.abs(GRID - min(abs(float(a)), 6.0))
+    best = np.flatnonzero(dist == dist.min())
+    return int(best[0] if len(best) == 1 else best[best % 2 == 0][0])
+
+
+def test_mxfp4_shared_exponent_and_codes(orc):
+    rng = np.random.default_rng(12)
+    rows, cols = 6, 256
+    x = rng.standard_normal((rows, cols)) * 2.0 ** rng.integers(-30, 30, (rows, cols // 32)).repeat(32, 1)
+    x[0, :32] = 0.0                       # an all-zero group
+    x[1, 32:64] = 1e-39                   # subnormal-only group in binary32 (bf16 keeps it)
+    xb = bf16(x)
+    codes, scales, gs = orc.quantize(bits_of(xb), ROW, MX, 0, 0)
+    assert gs == 1.0
+    xv = xb.float().numpy()
+    cu = orc.unpack_codes(codes)
+    for r in range(rows):
+        for gi in range(cols // 32):
+            grp = xv[r, 32 * gi:32 * gi + 32].astype(np.float64)
+            a = np.abs(grp).max()
+            E = -127 if a == 0 else int(np.clip(np.frexp(a)[1] - 1 - 2, -127, 127))
+            assert scales[r, 2 * gi] == scales[r, 2 * gi + 1] == E + 127, (r, gi)
+            y = grp / 2.0 ** E
+            for i in range(32):
+                k = _rtn_grid_index(y[i])
+                exp = 0 if k == 0 else (k | (8 if y[i] < 0 else 0))
+                assert cu[r, 32 * gi + i] == exp, (r, gi, i)
+
+
+def test_mxfp4_lossless_round_trip(orc):
+    rng = np.random.default_rng(13)
+    rows, cols = 8, 512
+    v = GRID[rng.integers(0, 8, (rows, cols))] * np.where(rng.random((rows, cols)) < 0.5, -1.0, 1.0)
+    v = v.reshape(rows, cols // 32, 32)
+    v[:, :, 0] = np.where(rng.random((rows, cols // 32)) < 0.5, 4.0, 6.0)  # group max in [4, 6]
+    e = rng.integers(-40, 40, (rows, cols // 32))
+    x = (v * 2.0 ** e[:, :, None]).reshape(rows, cols)
+    xb = bf16(x)
+    assert np.array_equal(xb.double().numpy(), x)
+    codes, scales, gs = orc.quantize(bits_of(xb), ROW, MX, 0, 0)
+    assert np.array_equal(scales[:, ::2].astype(int), e + 127)
+    assert np.array_equal(deq(orc, codes, scales, gs, MX, 0, 0), x)
+
+
+def test_mxfp4_mse_above_nvfp4_on_gaussian(orc):
+    """Table 1 (IF4 page) orders MXFP4's MSE above NVFP4's (13.2 vs 9.0, x1e-3); reported."""
+    rng = np.random.default_rng(14)
+    x = bf16(rng.standard_normal((128, 1024)))
+    m_mx = _mse(orc, x, MX, 0, [0])
+    m_nv = _mse(orc, x, RTN, 0, [0])
+    print(f"\nN(0,1) MSE: NVFP4 {m_nv * 1e3:.2f}e-3  MXFP4 {m_mx * 1e3:.2f}e-3  ratio {m_mx / m_nv:.2f} "
+          f"(Table 1: 9.0, 13.2, ratio 1.47)")
+    assert m_mx > m_nv
+
+
+def test_table1_mse_on_gaussian(orc):
+    """The MSE column of the IF4 page's Table 1 (tests/golden/if4_table1_mse.txt):
+    NVFP4, 4/6, IF4 and MXFP4 on 2^20 standard normal values, each within 2% of
+    the printed value (the table prints two digits; measured: 9.03, 7.57,
+    6.15, 13.20).  This pins the readings behind 4/6 (two candidate scales,
+    original-domain error, M = 256) and IF4 (INT4 levels k * 6/7, y-domain
+    error, flag) against numbers the pages print."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "if4_table1_mse.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    rng = np.random.default_rng(16)
+    x = bf16(rng.standard_normal((1024, 1024)))
+    for name, mode, want in rows:
+        got = _mse(orc, x, int(mode), 0, [0]) * 1e3
+        print(f"\n{name}: MSE {got:.3f}e-3 (Table 1: {want})", end="")
+        assert abs(got - float(want)) <= 0.02 * float(want), (name, got, want)
+
+
+def test_mxfp4_needs_whole_groups(orc):
+    x = bf16(np.ones((4, 48)))
+    with pytest.raises(Exception):
+        orc.quantize(bits_of(x), ROW, MX, 0, 0)
+
+
 # ------------------------------------------------------------------- structural
 @pytest.mark.parametrize("mode,g", [(RTN, 0), (SR, 0), (EDEN, 128), (IF4, 0), (FO6, 0), (SR, 32), (SS, 0),
-                                    (SS, 64)])
+                                    (SS, 64), (MX, 0), (MX, 128)])
 def test_transposed_is_rowwise_of_transpose(orc, mode, g):
     rng = np.random.default_rng(6)
     x = bf16(rng.standard_normal((256, 64)))
