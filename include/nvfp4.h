@@ -87,10 +87,16 @@ typedef enum {
   NVFP4_MS_EDEN = 2, /* RTN codes + EDEN-corrected, stochastically rounded scale; needs g > 0; amax -> 6 x 256 */
   NVFP4_IF4 = 3,     /* per block FP4 or scaled INT4 (flag in scale bit 7), amax -> 6 x 448 */
   NVFP4_4OVER6 = 4,  /* per block scale mapping the absmax to 6 or to 4, amax -> 6 x 256 */
-  NVFP4_SCALE_SEARCH = 5 /* per block the best of 19 E4M3 scales around the absmax scale (lowest
-                            squared error, RTN codes; palettes post, "The two corners, and what
-                            the palette does to them"; the ScaleSearch entry of the IF4 paper
-                            page), amax -> 6 x 256 */
+  NVFP4_SCALE_SEARCH = 5, /* per block the best of 19 E4M3 scales around the absmax scale (lowest
+                             squared error, RTN codes; palettes post, "The two corners, and what
+                             the palette does to them"; the ScaleSearch entry of the IF4 paper
+                             page), amax -> 6 x 256 */
+  NVFP4_MXFP4 = 6    /* MXFP4 (IF4 paper page, Table 1): groups of 32 view elements with one
+                        UE8M0 scale 2^E, E = floor(log2 max|z|) - 2 clamped to [-127, 127], RTN
+                        E2M1 values of z / 2^E; no tensor scale (global_scale = 1, amax_in and
+                        the workspace unused); the scale byte E + 127 is stored for each
+                        16-element half of a group; needs vcols % 32 == 0 and a view of at least
+                        one tile of the tiled kernels (else NVFP4_ERR_UNSUPPORTED) */
 } nvfp4_mode;
 
 /* Bytes of device workspace nvfp4_quantize needs when amax_in is NULL (the

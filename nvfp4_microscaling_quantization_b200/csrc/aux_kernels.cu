@@ -37,7 +37,10 @@ dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
     if (valid) {
       const uint2 c = *reinterpret_cast<const uint2*>(codes + b * 8);
       const uint32_t S = scales[b];
-      const float d = __fmul_rn(e4m3_decode(S & 0x7Fu), s_g);
+      // MXFP4: UE8M0 scale 2^(S - 127) (S = 0: the subnormal 2^-127); else
+      // RN(E4M3(S) * s_g)
+      const float d = mode == kMXFP4 ? __uint_as_float(S ? (S << 23) : 0x00400000u)
+                                     : __fmul_rn(e4m3_decode(S & 0x7Fu), s_g);
       if (mode == kIF4 && (S & 0x80u)) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {

@@ -15,7 +15,7 @@
 
 namespace nvfp4 {
 
-enum Mode { kRTN = 0, kSR = 1, kMSEDEN = 2, kIF4 = 3, k4over6 = 4, kScaleSearch = 5 };
+enum Mode { kRTN = 0, kSR = 1, kMSEDEN = 2, kIF4 = 3, k4over6 = 4, kScaleSearch = 5, kMXFP4 = 6 };
 
 // Scale search: the candidates are the E4M3 codes S0 + delta(t), t = 0 ..
 // 18, around the absmax scale S0, visited nearest first (0, -1, +1, -2, ...),
@@ -282,6 +282,7 @@ __device__ __forceinline__ void rht_inverse(float* v, uint32_t sign_bits, uint32
 // search, else 448.
 template <int MODE>
 __device__ __forceinline__ float global_scale_of(float amax) {
+  if constexpr (MODE == kMXFP4) return 1.0f;  // MXFP4 has no tensor scale
   constexpr float six_m = (MODE == kMSEDEN || MODE == k4over6 || MODE == kScaleSearch) ? 1536.0f : 2688.0f;
   return amax > 0.0f ? __fdiv_rn(amax, six_m) : 1.0f;
 }
@@ -677,6 +678,29 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
     ob.lo = pb ? cb_lo[1] : cb_lo[0];
     ob.hi = pb ? cb_hi[1] : cb_hi[0];
     ob.scale = ((pb ? S[1] : S[0]) >> 8) & 0xFFu;
+    return;
+  } else if constexpr (MODE == kMXFP4) {
+    // The pair is one 32-element MXFP4 group (block a its first half, b its
+    // second).  Shared exponent E = floor(log2 max|z|) - 2 clamped to
+    // [-127, 127]: from the exponent field f of the group maximum, the scale
+    // byte E + 127 = max(f - 2, 0) (f = 0 for zero and subnormal maxima, whose
+    // E clamps to -127).  y = z * 2^-E is z / 2^E rounded once (2^-E is a
+    // normal float for every E here); RTN codes saturate at 6.
+    const uint32_t f = __float_as_uint(fmaxf(aa, ab)) >> 23;
+    const uint32_t byte = f > 2u ? f - 2u : 0u;
+    const float inv = __uint_as_float((254u - byte) << 23);
+    const float2 inv2 = f2(inv, inv);
+    float ya[16], yb[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 y = mul2_rn(z[i], inv2);
+      ya[i] = y.x;
+      yb[i] = y.y;
+    }
+    rtn_codes(ya, oa.lo, oa.hi);
+    rtn_codes(yb, ob.lo, ob.hi);
+    oa.scale = byte;
+    ob.scale = byte;
     return;
   } else if constexpr (MODE == kScaleSearch) {
     const float2 sf = div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein);

@@ -244,9 +244,19 @@ cudaError_t launch_amax(const QuantArgs& a) {
   return dispatch_group<kRTN, true>(a);
 }
 
+// The tensor scale of an empty MXFP4 call (MXFP4 has none: 1).
+__global__ void set_one_kernel(float* p) { *p = 1.0f; }
+
 cudaError_t launch_quantize(const QuantArgs& a) {
   if (mma_path_applies(a)) return launch_quantize_mma(a);
   if (tma_path_applies(a)) return launch_quantize_tma(a);
+  if (a.mode == kMXFP4) {
+    // MXFP4 groups are the block pairs of the tiled kernels; the one-block
+    // kernels do not form them (the C ABI rejects such shapes up front)
+    if (a.rows != 0 && a.cols != 0) return cudaErrorNotSupported;
+    set_one_kernel<<<1, 1, 0, a.stream>>>(a.gscale);
+    return cudaGetLastError();
+  }
   switch (a.mode) {
     case kRTN: return dispatch_group<kRTN, false>(a);
     case kSR: return dispatch_group<kSR, false>(a);

@@ -78,7 +78,9 @@ def test_quantize_rejects(N):
     assert q(N, x=None, rows=0, gs=None) == INVALID
     assert q(N, layout=2) == INVALID
     assert q(N, g=48) == INVALID
-    assert q(N, mode=6) == INVALID
+    assert q(N, mode=7) == INVALID
+    assert q(N, mode=6, cols=48, ld=48) == SHAPE          # MXFP4: whole 32-element groups
+    assert q(N, mode=6, rows=8, cols=64) == UNSUPPORTED   # MXFP4: below one tile of the tiled kernels
     assert q(N, cols=40, ld=40) == SHAPE            # row-wise blocks need cols % 16 == 0
     assert q(N, rows=40, layout=1) == SHAPE         # transposed blocks need rows % 16 == 0
     assert q(N, cols=64, g=128) == SHAPE            # rotation group must divide the block dimension
