@@ -15,7 +15,7 @@ import numpy as np
 from . import build as _build
 
 ROWWISE, TRANSPOSED = 0, 1
-RTN, SR, MS_EDEN, IF4, FOUR_OVER_SIX, SCALE_SEARCH, MXFP4 = 0, 1, 2, 3, 4, 5, 6
+RTN, SR, MS_EDEN, IF4, FOUR_OVER_SIX, SCALE_SEARCH, MXFP4, NVINT4 = 0, 1, 2, 3, 4, 5, 6, 7
 
 _lib = None
 

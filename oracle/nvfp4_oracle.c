@@ -56,7 +56,8 @@
 
 /* modes and layouts: same numbering as the public C ABI (an interface, not
  * shared code). */
-enum { ORC_RTN = 0, ORC_SR = 1, ORC_MS_EDEN = 2, ORC_IF4 = 3, ORC_4OVER6 = 4, ORC_SCALE_SEARCH = 5, ORC_MXFP4 = 6 };
+enum { ORC_RTN = 0, ORC_SR = 1, ORC_MS_EDEN = 2, ORC_IF4 = 3, ORC_4OVER6 = 4, ORC_SCALE_SEARCH = 5, ORC_MXFP4 = 6,
+       ORC_NVINT4 = 7 };
 enum { ORC_ROWWISE = 0, ORC_TRANSPOSED = 1 };
 
 /* ------------------------------------------------------------------------ */
@@ -330,7 +331,7 @@ static void load_view_row(const uint16_t* x, int64_t ld, int layout, int64_t vr,
 static int check_quant_args(int64_t rows, int64_t cols, int64_t ld, int layout,
                             int mode, int g, int64_t* vr, int64_t* vc) {
   if (layout != ORC_ROWWISE && layout != ORC_TRANSPOSED) return ORC_ERR_ARG;
-  if (mode < ORC_RTN || mode > ORC_MXFP4) return ORC_ERR_ARG;
+  if (mode < ORC_RTN || mode > ORC_NVINT4) return ORC_ERR_ARG;
   if (g != 0 && !valid_group(g)) return ORC_ERR_ARG;
   if (mode == ORC_MS_EDEN && g == 0) return ORC_ERR_UNSUPPORTED;
   if (rows < 0 || cols < 0 || ld < cols) return ORC_ERR_SHAPE;
@@ -380,6 +381,7 @@ int oracle_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int l
  * maximum contributes at least 3 * 3 to <y, v>; so 256 * 1.61 < 448. */
 float oracle_global_scale(float A, int mode) {
   if (mode == ORC_MXFP4) return 1.0f; /* MXFP4 has no tensor scale [IF4-T1] */
+  if (mode == ORC_NVINT4) return A > 0.0f ? A / 3136.0f : 1.0f; /* NVINT4: 7 x 448 [IF4-T1] */
   float sixM = (mode == ORC_4OVER6 || mode == ORC_MS_EDEN || mode == ORC_SCALE_SEARCH) ? 1536.0f
                                                                                       : 2688.0f; /* exact */
   if (!(A > 0.0f)) return 1.0f;
@@ -412,6 +414,30 @@ static uint8_t quantize_block(const float* z, int mode, float s_g, uint64_t seed
   float a_b = 0.0f; /* block absmax [PAL-corners]: the absmax sets each block's scale */
   for (int i = 0; i < 16; ++i)
     if (fabsf(z[i]) > a_b) a_b = fabsf(z[i]);
+
+  if (mode == ORC_NVINT4) {
+    /* NVINT4 [IF4-T1]: 16-element blocks, E4M3 scale, INT4 values, maximum
+     * 7 x 448, minimum 1 x 2^-9.  Reading: as NVFP4 with the integer grid
+     * k in [-7, 7] in place of E2M1: s_g = RN(A / (7 448)) (set above),
+     * S = E4M3_RNE(RN(a_b / RN(7 s_g))), d = RN(dec(S) s_g),
+     * k = clamp(RNE(RN(z RN(1/d))), -7, 7), stored as IF4's INT4 nibble
+     * (sign bit 3, |k| in bits 0..2), value RN(k d). */
+    float q7 = 7.0f * s_g;
+    uint8_t S7 = oracle_e4m3_rne_sat(a_b / q7);
+    float d7 = oracle_e4m3_decode(S7) * s_g;
+    if (d7 == 0.0f) {
+      memset(code, 0, 16);
+      return S7;
+    }
+    float r7 = 1.0f / d7;
+    for (int i = 0; i < 16; ++i) {
+      float k = nearbyintf(z[i] * r7); /* ties to even (default rounding mode) */
+      if (k > 7.0f) k = 7.0f;
+      if (k < -7.0f) k = -7.0f;
+      code[i] = int4_code((int)k);
+    }
+    return S7;
+  }
 
   if (mode == ORC_MXFP4) {
     /* MXFP4 [IF4-T1]: 32-element groups, one UE8M0 (power of two) scale, E2M1
@@ -640,7 +666,7 @@ int oracle_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, i
 int oracle_dequantize(const uint8_t* codes, const uint8_t* scales, float s_g,
                       int64_t vr, int64_t vc, int mode, int g, uint64_t seed,
                       int inverse_rht, float* out) {
-  if (mode < ORC_RTN || mode > ORC_MXFP4) return ORC_ERR_ARG;
+  if (mode < ORC_RTN || mode > ORC_NVINT4) return ORC_ERR_ARG;
   if (g != 0 && !valid_group(g)) return ORC_ERR_ARG;
   if (vr < 0 || vc < 0 || vc % 16 || (g && vc % g)) return ORC_ERR_SHAPE;
   if (mode == ORC_MXFP4 && vc % 32) return ORC_ERR_SHAPE;
@@ -650,13 +676,14 @@ int oracle_dequantize(const uint8_t* codes, const uint8_t* scales, float s_g,
       uint8_t S = scales[r * (vc / 16) + j / 16];
       uint8_t byte = codes[r * (vc / 2) + j / 2];
       uint8_t code = (j & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15u);
-      int int4 = mode == ORC_IF4 && (S & 0x80u);
+      int int4 = (mode == ORC_IF4 && (S & 0x80u)) || mode == ORC_NVINT4;
       float d = mode == ORC_MXFP4 ? ldexpf(1.0f, (int)S - 127)  /* UE8M0: 2^(S - 127) */
                                   : oracle_e4m3_decode((uint8_t)(S & 0x7Fu)) * s_g;
       float v;
       if (int4) {
         int k = (int)(code & 7u);
-        v = int4_value((code & 8u) ? -k : k);
+        k = (code & 8u) ? -k : k;
+        v = mode == ORC_NVINT4 ? (float)k : int4_value(k);
       } else {
         v = oracle_e2m1_decode(code);
       }
@@ -700,7 +727,7 @@ void oracle_e4m3_array(const float* in, int64_t n, int round_up, uint8_t* out) {
 int oracle_quantize_rotated(const float* z, int64_t row0, int64_t vr, int64_t vc, int mode,
                             uint64_t seed, float amax, uint8_t* codes, uint8_t* scales,
                             float* global_scale) {
-  if (mode < ORC_RTN || mode > ORC_MXFP4) return ORC_ERR_ARG;
+  if (mode < ORC_RTN || mode > ORC_NVINT4) return ORC_ERR_ARG;
   if (row0 < 0 || vr < 0 || vc < 0 || vc % 16 || (mode == ORC_MXFP4 && vc % 32)) return ORC_ERR_SHAPE;
   float s_g = oracle_global_scale(amax, mode);
   *global_scale = s_g;

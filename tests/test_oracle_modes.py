@@ -20,8 +20,11 @@
 * MXFP4 (IF4 page, Table 1: groups of 32, UE8M0 scale, max 6 x 2^127, min
   0.5 x 2^-127): shared exponent floor(log2 amax) - 2 recomputed with numpy's
   frexp, codes by brute-force nearest E2M1 of x / 2^E, a lossless round trip.
-* Table 1's MSE column (NVFP4 9.0, 4/6 7.5, IF4 6.2, MXFP4 13.2, x1e-3) on
-  standard normal data, within 2% (tests/golden/if4_table1_mse.txt).
+* NVINT4 (IF4 page, Table 1: E4M3 scale, INT4 values, max 7 x 448): integer
+  levels by brute-force nearest integer (ties to even) of the scaled value,
+  and a lossless round trip.
+* Table 1's MSE column (NVFP4 9.0, NVINT4 7.4, 4/6 7.5, IF4 6.2, MXFP4 13.2,
+  x1e-3) on standard normal data, within 2% (tests/golden/if4_table1_mse.txt).
 * Structural properties: transposed view = row-wise quantization of X^T,
   leading dimension, amax_in, zero tensor and zero blocks, nibble order.
 """
@@ -32,7 +35,7 @@ import torch
 from nvfp4_microscaling_quantization_b200 import workloads as W
 
 ROW, TR = 0, 1
-RTN, SR, EDEN, IF4, FO6, SS, MX = 0, 1, 2, 3, 4, 5, 6
+RTN, SR, EDEN, IF4, FO6, SS, MX, NI4 = 0, 1, 2, 3, 4, 5, 6, 7
 GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
 
 
@@ -400,11 +403,46 @@ def test_mxfp4_mse_above_nvfp4_on_gaussian(orc):
     assert m_mx > m_nv
 
 
+def test_nvint4_levels_and_round_trip(orc):
+    rng = np.random.default_rng(21)
+    x = bf16(rng.standard_normal((16, 256)) * 3.0)
+    codes, scales, gs = orc.quantize(bits_of(x), ROW, NI4, 0, 0)
+    xv = x.float().numpy()
+    assert gs == np.float32(np.float32(np.abs(xv).max()) / np.float32(3136.0))
+    cu = orc.unpack_codes(codes)
+    for r in range(xv.shape[0]):
+        for b in range(xv.shape[1] // 16):
+            zb = xv[r, 16 * b:16 * b + 16]
+            S = orc.e4m3_rne_sat(f32(f32(np.abs(zb).max()) / f32(f32(7.0) * f32(gs))))
+            assert scales[r, b] == S
+            d = f32(_e4m3_value(S) * f32(gs))
+            y = (zb * f32(f32(1.0) / d)).astype(np.float64)
+            k = np.clip(np.round(y), -7, 7)          # numpy rounds half to even
+            c = cu[r, 16 * b:16 * b + 16]
+            kk = np.where(c & 8, -(c & 7).astype(int), (c & 7).astype(int))
+            assert np.array_equal(kk, k.astype(int)), (r, b)
+            assert np.all(c != 8)                     # zero is code 0
+    # integers under a power-of-two scale quantize exactly: blocks holding +-7,
+    # tensor max 7 * 448 * 2^-10 so that s_g = 2^-10 and every block scale is
+    # an exact power of two
+    k = rng.integers(-7, 8, (8, 256)).astype(np.float64).reshape(8, 16, 16)
+    k[:, :, 0] = 7.0
+    e = rng.integers(-6, 8, (8, 16)).astype(np.float64)
+    e[0, 0] = 0
+    blk = 2.0 ** e
+    blk[0, 0] = 448.0
+    xx = (k * blk[:, :, None] * 2.0 ** -10).reshape(8, 256)
+    xb = bf16(xx)
+    c2, s2, g2 = orc.quantize(bits_of(xb), ROW, NI4, 0, 0)
+    assert g2 == 2.0 ** -10
+    assert np.array_equal(deq(orc, c2, s2, g2, NI4, 0, 0), xx)
+
+
 def test_table1_mse_on_gaussian(orc):
     """The MSE column of the IF4 page's Table 1 (tests/golden/if4_table1_mse.txt):
     NVFP4, 4/6, IF4 and MXFP4 on 2^20 standard normal values, each within 2% of
     the printed value (the table prints two digits; measured: 9.03, 7.57,
-    6.15, 13.20).  This pins the readings behind 4/6 (two candidate scales,
+    6.15, 13.20, and NVINT4 7.43).  This pins the readings behind 4/6 (two candidate scales,
     original-domain error, M = 256) and IF4 (INT4 levels k * 6/7, y-domain
     error, flag) against numbers the pages print."""
     import os
@@ -426,7 +464,7 @@ def test_mxfp4_needs_whole_groups(orc):
 
 # ------------------------------------------------------------------- structural
 @pytest.mark.parametrize("mode,g", [(RTN, 0), (SR, 0), (EDEN, 128), (IF4, 0), (FO6, 0), (SR, 32), (SS, 0),
-                                    (SS, 64), (MX, 0), (MX, 128)])
+                                    (SS, 64), (MX, 0), (MX, 128), (NI4, 0), (NI4, 32)])
 def test_transposed_is_rowwise_of_transpose(orc, mode, g):
     rng = np.random.default_rng(6)
     x = bf16(rng.standard_normal((256, 64)))
