@@ -91,12 +91,15 @@ typedef enum {
                              squared error, RTN codes; palettes post, "The two corners, and what
                              the palette does to them"; the ScaleSearch entry of the IF4 paper
                              page), amax -> 6 x 256 */
-  NVFP4_MXFP4 = 6    /* MXFP4 (IF4 paper page, Table 1): groups of 32 view elements with one
+  NVFP4_MXFP4 = 6,   /* MXFP4 (IF4 paper page, Table 1): groups of 32 view elements with one
                         UE8M0 scale 2^E, E = floor(log2 max|z|) - 2 clamped to [-127, 127], RTN
                         E2M1 values of z / 2^E; no tensor scale (global_scale = 1, amax_in and
                         the workspace unused); the scale byte E + 127 is stored for each
                         16-element half of a group; needs vcols % 32 == 0 and a view of at least
                         one tile of the tiled kernels (else NVFP4_ERR_UNSUPPORTED) */
+  NVFP4_NVINT4 = 7   /* NVINT4 (IF4 paper page, Table 1): E4M3 block scale mapping the absmax to
+                        7, INT4 levels k = clamp(RNE(z / d), -7, 7) stored as sign-magnitude
+                        nibbles (as IF4's INT4 option, value k d), amax -> 7 x 448 */
 } nvfp4_mode;
 
 /* Bytes of device workspace nvfp4_quantize needs when amax_in is NULL (the
@@ -134,7 +137,8 @@ NVFP4_API int nvfp4_amax_dual(const void* x, int64_t rows, int64_t cols, int64_t
  *  amax_in:   device float holding the tensor amax of the (rotated) view, or
  *             NULL to compute it in a pre-pass (needs the workspace).  The
  *             tensor scale is s_g = RN(amax / (6 M)), M = 448 (RTN, SR, IF4)
- *             or 256 (MS-EDEN, 4/6, scale search); s_g = 1 for a zero amax.
+ *             or 256 (MS-EDEN, 4/6, scale search); RN(amax / (7 x 448)) for
+ *             NVINT4; 1 for MXFP4; s_g = 1 for a zero amax.
  *  codes, scales, global_scale: outputs (sizes above); global_scale is one
  *             device float.
  *  workspace: device memory of at least nvfp4_workspace_bytes(...) bytes when

@@ -41,12 +41,14 @@ dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
       // RN(E4M3(S) * s_g)
       const float d = mode == kMXFP4 ? __uint_as_float(S ? (S << 23) : 0x00400000u)
                                      : __fmul_rn(e4m3_decode(S & 0x7Fu), s_g);
-      if (mode == kIF4 && (S & 0x80u)) {
+      if ((mode == kIF4 && (S & 0x80u)) || mode == kNVINT4) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const uint32_t code = ((i < 8 ? c.x : c.y) >> (4 * (i & 7))) & 0xFu;
           const int k = (code & 8u) ? -static_cast<int>(code & 7u) : static_cast<int>(code & 7u);
-          v[i] = __fmul_rn(__fmul_rn(static_cast<float>(k), kIF4K2), d);
+          // IF4: RN(RN(k RN(6/7)) d); NVINT4: RN(k d)
+          const float lv = mode == kNVINT4 ? static_cast<float>(k) : __fmul_rn(static_cast<float>(k), kIF4K2);
+          v[i] = __fmul_rn(lv, d);
         }
       } else {
         e2m1x8_to_f32(c.x, v);

@@ -15,7 +15,7 @@
 
 namespace nvfp4 {
 
-enum Mode { kRTN = 0, kSR = 1, kMSEDEN = 2, kIF4 = 3, k4over6 = 4, kScaleSearch = 5, kMXFP4 = 6 };
+enum Mode { kRTN = 0, kSR = 1, kMSEDEN = 2, kIF4 = 3, k4over6 = 4, kScaleSearch = 5, kMXFP4 = 6, kNVINT4 = 7 };
 
 // Scale search: the candidates are the E4M3 codes S0 + delta(t), t = 0 ..
 // 18, around the absmax scale S0, visited nearest first (0, -1, +1, -2, ...),
@@ -283,6 +283,7 @@ __device__ __forceinline__ void rht_inverse(float* v, uint32_t sign_bits, uint32
 template <int MODE>
 __device__ __forceinline__ float global_scale_of(float amax) {
   if constexpr (MODE == kMXFP4) return 1.0f;  // MXFP4 has no tensor scale
+  if constexpr (MODE == kNVINT4) return amax > 0.0f ? __fdiv_rn(amax, 3136.0f) : 1.0f;  // 7 x 448
   constexpr float six_m = (MODE == kMSEDEN || MODE == k4over6 || MODE == kScaleSearch) ? 1536.0f : 2688.0f;
   return amax > 0.0f ? __fdiv_rn(amax, six_m) : 1.0f;
 }
@@ -291,6 +292,17 @@ __device__ __forceinline__ float global_scale_of(float amax) {
 constexpr float kIF4K1 = 0x1.2aaaaap+0f;  // RN(7/6)
 constexpr float kIF4K2 = 0x1.b6db6ep-1f;  // RN(6/7)
 constexpr float kRoundMagic = 12582912.0f; // 1.5 * 2^23: RN(t + it) - it = RNE(t) for |t| < 2^22
+
+// NVINT4 code of one scaled value y: k = clamp(RNE(y), -7, 7) as a
+// sign-magnitude nibble (sign bit 3, |k| in bits 0..2, never -0), with no
+// conversion instruction: s = RN(y + 1.5 2^23) rounds y at the units bit
+// (ties to even, |y| < 2^22), s - 1.5 2^23 = RNE(y) exactly; |k| is the low
+// mantissa bits of 2^23 + |k| and the sign is the sign of k.
+__device__ __forceinline__ uint32_t int4_nibble(float y) {
+  const float s = __fadd_rn(y, kRoundMagic);
+  const float k = fminf(fmaxf(__fsub_rn(s, kRoundMagic), -7.0f), 7.0f);
+  return (__float_as_uint(__fadd_rn(fabsf(k), 8388608.0f)) & 7u) | ((__float_as_uint(k) >> 28) & 8u);
+}
 
 // Where the random draws of one 16-element block come from.
 struct BlockRng {
@@ -387,6 +399,19 @@ __device__ __forceinline__ BlockOut quantize_block(const float* z, float s_g, co
     out.lo = c_lo[pick];
     out.hi = c_hi[pick];
     out.scale = S[pick];
+    return out;
+  } else if constexpr (MODE == kNVINT4) {
+    const uint32_t S = e4m3_rne_sat(__fdiv_rn(a_b, __fmul_rn(7.0f, s_g)));
+    const float d = __fmul_rn(e4m3_decode(S), s_g);
+    out.scale = S;
+    if (d == 0.0f) return out;
+    const float r = __frcp_rn(d);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t c = int4_nibble(__fmul_rn(z[i], r));
+      if (i < 8) out.lo |= c << (4 * i);
+      else out.hi |= c << (4 * (i - 8));
+    }
     return out;
   } else if constexpr (MODE == kScaleSearch) {
     const uint32_t s0 = e4m3_rne_sat(__fdiv_rn(a_b, __fmul_rn(6.0f, s_g)));
@@ -516,7 +541,8 @@ __device__ __forceinline__ ScaleCtx make_scale_ctx(float amax) {
   ScaleCtx c;
   c.tbl = nullptr;
   c.s_g = global_scale_of<MODE>(amax);
-  c.q6 = __fmul_rn(6.0f, c.s_g);
+  // the absmax divisor: RN(6 s_g), or RN(7 s_g) for NVINT4 (INT4's maximum 7)
+  c.q6 = __fmul_rn(MODE == kNVINT4 ? 7.0f : 6.0f, c.s_g);
   c.q4 = __fmul_rn(4.0f, c.s_g);
   c.r6 = __frcp_rn(c.q6);
   c.r4 = __frcp_rn(c.q4);
@@ -678,6 +704,28 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
     ob.lo = pb ? cb_lo[1] : cb_lo[0];
     ob.hi = pb ? cb_hi[1] : cb_hi[0];
     ob.scale = ((pb ? S[1] : S[0]) >> 8) & 0xFFu;
+    return;
+  } else if constexpr (MODE == kNVINT4) {
+    // q6 holds RN(7 s_g) for this mode (make_scale_ctx)
+    const float2 sf = div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein);
+    const uint32_t S2 = e4m3x2_rne_sat(sf.x, sf.y);
+    const uint32_t Sa = S2 & 0xFFu, Sb = S2 >> 8;
+    const float4 ta = scale_entry<TBL>(sc, Sa), tb = scale_entry<TBL>(sc, Sb);
+    const float2 r = f2(ta.z, tb.z);  // RN(1/d), 0 for a zero scale: y = 0, codes 0
+    oa = BlockOut{0u, 0u, Sa};
+    ob = BlockOut{0u, 0u, Sb};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 y = mul2_rn(z[i], r);
+      const uint32_t ca = int4_nibble(y.x), cb = int4_nibble(y.y);
+      if (i < 8) {
+        oa.lo |= ca << (4 * i);
+        ob.lo |= cb << (4 * i);
+      } else {
+        oa.hi |= ca << (4 * (i - 8));
+        ob.hi |= cb << (4 * (i - 8));
+      }
+    }
     return;
   } else if constexpr (MODE == kMXFP4) {
     // The pair is one 32-element MXFP4 group (block a its first half, b its

@@ -264,6 +264,7 @@ cudaError_t launch_quantize(const QuantArgs& a) {
     case kIF4: return dispatch_group<kIF4, false>(a);
     case k4over6: return dispatch_group<k4over6, false>(a);
     case kScaleSearch: return dispatch_group<kScaleSearch, false>(a);
+    case kNVINT4: return dispatch_group<kNVINT4, false>(a);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -441,6 +441,7 @@ cudaError_t launch_quantize_tma(const QuantArgs& a) {
     case k4over6: return dispatch_tma<k4over6, false>(a);
     case kScaleSearch: return dispatch_tma<kScaleSearch, false>(a);
     case kMXFP4: return dispatch_tma<kMXFP4, false>(a);
+    case kNVINT4: return dispatch_tma<kNVINT4, false>(a);
     default: return cudaErrorInvalidValue;
   }
 }

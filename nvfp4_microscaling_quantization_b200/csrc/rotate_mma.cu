@@ -766,6 +766,7 @@ cudaError_t launch_quantize_mma(const QuantArgs& a) {
     case k4over6: return dispatch<k4over6, kQuantize>(a, nullptr);
     case kScaleSearch: return dispatch<kScaleSearch, kQuantize>(a, nullptr);
     case kMXFP4: return dispatch<kMXFP4, kQuantize>(a, nullptr);
+    case kNVINT4: return dispatch<kNVINT4, kQuantize>(a, nullptr);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -27,7 +27,8 @@ def digest_lines():
     lines = []
     calls = list(wl.calls) + [workloads.Call("x", 1, m, 128) for m in (0, 1, 2, 3, 4)] + \
         [workloads.Call("x", 0, 3, 0), workloads.Call("x", 0, 4, 0), workloads.Call("x", 0, 5, 0),
-         workloads.Call("x", 1, 5, 128), workloads.Call("x", 0, 6, 0), workloads.Call("x", 1, 6, 128)]
+         workloads.Call("x", 1, 5, 128), workloads.Call("x", 0, 6, 0), workloads.Call("x", 1, 6, 128),
+         workloads.Call("x", 0, 7, 0), workloads.Call("x", 1, 7, 128)]
     for c in calls:
         codes, scales, gs = oracle.quantize(x, c.layout, c.mode, c.rht_group, wl.seed)
         h = hashlib.sha256(codes.tobytes() + scales.tobytes()).hexdigest()

@@ -78,7 +78,7 @@ def test_quantize_rejects(N):
     assert q(N, x=None, rows=0, gs=None) == INVALID
     assert q(N, layout=2) == INVALID
     assert q(N, g=48) == INVALID
-    assert q(N, mode=7) == INVALID
+    assert q(N, mode=8) == INVALID
     assert q(N, mode=6, cols=48, ld=48) == SHAPE          # MXFP4: whole 32-element groups
     assert q(N, mode=6, rows=8, cols=64) == UNSUPPORTED   # MXFP4: below one tile of the tiled kernels
     assert q(N, cols=40, ld=40) == SHAPE            # row-wise blocks need cols % 16 == 0
@@ -122,7 +122,7 @@ def test_other_entry_points_reject(N):
     assert d(None, FAKE, FAKE, 4, 64, 0, 0, 0, 0, FAKE, None) == INVALID
     assert d(FAKE, FAKE, FAKE, 4, 64, 0, 0, 0, 1, FAKE, None) == INVALID  # inverse without rotation
     assert d(FAKE, FAKE, FAKE, 4, 40, 0, 0, 0, 0, FAKE, None) == SHAPE
-    assert d(FAKE, FAKE, FAKE, 4, 64, 7, 0, 0, 0, FAKE, None) == INVALID
+    assert d(FAKE, FAKE, FAKE, 4, 64, 8, 0, 0, 0, FAKE, None) == INVALID
     assert d(FAKE, FAKE, FAKE, 4, 64, 0, 0, 0, 0, FAKE + 4, None) == ALIGN
     r = N.nvfp4_rht
     assert r(FAKE, 0, 64, 64, 64, 0, 0, 0, 0, FAKE, None) == INVALID      # group 0
