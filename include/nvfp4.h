@@ -155,7 +155,8 @@ NVFP4_API int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t 
  * out[r][j] = value(code, flag) * RN(E4M3(scale & 0x7F) * s_g), and, when
  * inverse_rht != 0 (needs rht_group > 0 and the seed used to quantize), the
  * inverse rotation along each row.  value is the E2M1 value, or for an IF4
- * block with bit 7 of its scale set, RN(k * RN(6/7)).  out: vrows x vcols
+ * block with bit 7 of its scale set, RN(k * RN(6/7)); for NVINT4 the integer
+ * k itself; for MXFP4 the scale factor is 2^(scale - 127) instead (no s_g).  out: vrows x vcols
  * dense fp32, 16-byte aligned.  global_scale: device float. */
 NVFP4_API int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
                      int64_t vrows, int64_t vcols, int mode, int rht_group, uint64_t seed,
