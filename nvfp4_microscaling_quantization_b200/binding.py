@@ -17,6 +17,7 @@ import torch
 
 ROWWISE, TRANSPOSED = 0, 1
 RTN, SR, MS_EDEN, IF4, FOUR_OVER_SIX, SCALE_SEARCH, MXFP4, NVINT4 = 0, 1, 2, 3, 4, 5, 6, 7
+NVFP3, NVINT3, IF3, MXFP3 = 8, 9, 10, 11
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
 

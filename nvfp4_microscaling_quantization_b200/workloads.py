@@ -34,8 +34,10 @@ import torch
 
 ROWWISE, TRANSPOSED = 0, 1
 RTN, SR, MS_EDEN, IF4, FOUR_OVER_SIX, SCALE_SEARCH, MXFP4, NVINT4 = 0, 1, 2, 3, 4, 5, 6, 7
+NVFP3, NVINT3, IF3, MXFP3 = 8, 9, 10, 11
 MODE_NAMES = {RTN: "rtn", SR: "sr", MS_EDEN: "ms_eden", IF4: "if4", FOUR_OVER_SIX: "4over6",
-              SCALE_SEARCH: "scale_search", MXFP4: "mxfp4", NVINT4: "nvint4"}
+              SCALE_SEARCH: "scale_search", MXFP4: "mxfp4", NVINT4: "nvint4", NVFP3: "nvfp3",
+              NVINT3: "nvint3", IF3: "if3", MXFP3: "mxfp3"}
 LAYOUT_NAMES = {ROWWISE: "rowwise", TRANSPOSED: "transposed"}
 
 

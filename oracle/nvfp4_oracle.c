@@ -34,6 +34,8 @@
  *  [IF4-abs]  IF4 paper page (arXiv 2603.28765, "Adaptive Block-Scaled Data
  *             Types"), abstract; [IF4-F1] its Figure 1; [IF4-T1] its Table 1;
  *             [IF4-F3] its Figure 3.
+ *  [IF4-T6]  the same page's 3-bit formats table (MXFP3, NVINT3, NVFP3, IF3:
+ *             scale type, element type, group size, bits per value).
  *  [SS-abs]   the same IF4 paper page, its related-paper entry on ScaleSearch
  *             (abstract): block scales chosen by searching the scale's
  *             mantissa values for the lowest quantization error.
@@ -57,7 +59,7 @@
 /* modes and layouts: same numbering as the public C ABI (an interface, not
  * shared code). */
 enum { ORC_RTN = 0, ORC_SR = 1, ORC_MS_EDEN = 2, ORC_IF4 = 3, ORC_4OVER6 = 4, ORC_SCALE_SEARCH = 5, ORC_MXFP4 = 6,
-       ORC_NVINT4 = 7 };
+       ORC_NVINT4 = 7, ORC_NVFP3 = 8, ORC_NVINT3 = 9, ORC_IF3 = 10, ORC_MXFP3 = 11 };
 enum { ORC_ROWWISE = 0, ORC_TRANSPOSED = 1 };
 
 /* ------------------------------------------------------------------------ */
@@ -331,14 +333,14 @@ static void load_view_row(const uint16_t* x, int64_t ld, int layout, int64_t vr,
 static int check_quant_args(int64_t rows, int64_t cols, int64_t ld, int layout,
                             int mode, int g, int64_t* vr, int64_t* vc) {
   if (layout != ORC_ROWWISE && layout != ORC_TRANSPOSED) return ORC_ERR_ARG;
-  if (mode < ORC_RTN || mode > ORC_NVINT4) return ORC_ERR_ARG;
+  if (mode < ORC_RTN || mode > ORC_MXFP3) return ORC_ERR_ARG;
   if (g != 0 && !valid_group(g)) return ORC_ERR_ARG;
   if (mode == ORC_MS_EDEN && g == 0) return ORC_ERR_UNSUPPORTED;
   if (rows < 0 || cols < 0 || ld < cols) return ORC_ERR_SHAPE;
   *vr = layout == ORC_ROWWISE ? rows : cols;
   *vc = layout == ORC_ROWWISE ? cols : rows;
   if (*vc % 16) return ORC_ERR_SHAPE;
-  if (mode == ORC_MXFP4 && *vc % 32) return ORC_ERR_SHAPE;
+  if ((mode == ORC_MXFP4 || mode == ORC_MXFP3) && *vc % 32) return ORC_ERR_SHAPE;
   if (g > 0 && *vc % g) return ORC_ERR_SHAPE;
   return ORC_OK;
 }
@@ -382,6 +384,10 @@ int oracle_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int l
 float oracle_global_scale(float A, int mode) {
   if (mode == ORC_MXFP4) return 1.0f; /* MXFP4 has no tensor scale [IF4-T1] */
   if (mode == ORC_NVINT4) return A > 0.0f ? A / 3136.0f : 1.0f; /* NVINT4: 7 x 448 [IF4-T1] */
+  if (mode == ORC_MXFP3) return 1.0f;
+  /* 3-bit formats [IF4-T6]: the element maximum x 448 (E2M0: 4, INT3: 3) */
+  if (mode == ORC_NVFP3 || mode == ORC_IF3) return A > 0.0f ? A / 1792.0f : 1.0f;
+  if (mode == ORC_NVINT3) return A > 0.0f ? A / 1344.0f : 1.0f;
   float sixM = (mode == ORC_4OVER6 || mode == ORC_MS_EDEN || mode == ORC_SCALE_SEARCH) ? 1536.0f
                                                                                       : 2688.0f; /* exact */
   if (!(A > 0.0f)) return 1.0f;
@@ -407,6 +413,34 @@ static int int4_level(float y) {
 static uint8_t int4_code(int k) { return k == 0 ? 0 : (uint8_t)((k < 0 ? 8 : 0) | (k < 0 ? -k : k)); }
 static float int4_value(int k) { return (float)k * IF4_K2; }
 
+/* 3-bit elements [IF4-T6] (the page lists MXFP3 and NVFP3 with E2M0
+ * elements, NVINT3 with INT3, IF3 with INT3 / E2M0).  Readings: E2M0 is the
+ * E2M1 layout without the mantissa bit (bias 1, the zero exponent holding
+ * only 0): magnitudes {0, 1, 2, 4}, round to nearest with ties to the even
+ * code; INT3 is sign-magnitude, |k| <= 3.  A 3-bit code is stored in a
+ * nibble: sign bit 3, magnitude code in bits 0..1 (bit 2 clear); zero is code
+ * 0.  IF3's INT3 levels k stand for k * 4/3 under the shared scale, so both
+ * options span +-4 (as IF4's k * 6/7 spans E2M1's +-6). */
+static const float E2M0_MAG[4] = {0.0f, 1.0f, 2.0f, 4.0f};
+static const float IF3_K1 = (float)(3.0 / 4.0); /* RN(3/4), exact */
+static const float IF3_K2 = (float)(4.0 / 3.0); /* RN(4/3) */
+
+static uint8_t e2m0_rtn(float y) {
+  float a = fabsf(y);
+  uint8_t m = (uint8_t)((a > 0.5f) + (a >= 1.5f) + (a > 3.0f)); /* ties 0.5, 1.5, 3 to codes 0, 2, 2 */
+  return m == 0 ? 0 : (uint8_t)(m | (y < 0.0f ? 8u : 0u));
+}
+static float e2m0_decode(uint8_t c) {
+  float v = E2M0_MAG[c & 3u];
+  return (c & 8u) ? -v : v;
+}
+static int int3_level(float t) {
+  float k = nearbyintf(t);
+  if (k > 3.0f) k = 3.0f;
+  if (k < -3.0f) k = -3.0f;
+  return (int)k;
+}
+
 /* Quantize one 16-element block z[0..15] of view row vr, block column bc.
  * Writes 16 codes (one per element, low nibble) and returns the scale byte. */
 static uint8_t quantize_block(const float* z, int mode, float s_g, uint64_t seed,
@@ -415,6 +449,72 @@ static uint8_t quantize_block(const float* z, int mode, float s_g, uint64_t seed
   for (int i = 0; i < 16; ++i)
     if (fabsf(z[i]) > a_b) a_b = fabsf(z[i]);
 
+  if (mode == ORC_MXFP3) {
+    /* MXFP3 [IF4-T6]: as MXFP4 (32-element groups, UE8M0 shared exponent)
+     * with E2M0 elements: E = floor(log2 max |x|) - 2 (2 = the exponent of
+     * E2M0's largest value, 4), clamped to [-127, 127]; codes E2M0 RTN of
+     * x / 2^E, saturating at 4. */
+    const float* grp = (bc & 1) ? z - 16 : z;
+    float a = 0.0f;
+    for (int i = 0; i < 32; ++i)
+      if (fabsf(grp[i]) > a) a = fabsf(grp[i]);
+    int E = -127;
+    if (a > 0.0f) {
+      int e2;
+      frexpf(a, &e2);
+      E = e2 - 1 - 2;
+      if (E < -127) E = -127;
+      if (E > 127) E = 127;
+    }
+    float X = ldexpf(1.0f, E);
+    for (int i = 0; i < 16; ++i) code[i] = e2m0_rtn(z[i] / X);
+    return (uint8_t)(E + 127);
+  }
+  if (mode == ORC_NVFP3 || mode == ORC_NVINT3 || mode == ORC_IF3) {
+    /* NVFP3 / NVINT3 / IF3 [IF4-T6]: NVFP4's steps with the 3-bit grids, the
+     * block absmax mapped to the element maximum m (4 for E2M0 and IF3, 3
+     * for INT3): S = E4M3_RNE(RN(a_b / RN(m s_g))), d = RN(dec(S) s_g),
+     * y = RN(z RN(1/d)).  IF3 keeps the option with the lower squared error
+     * in the y domain (fmaf in element order; ties keep E2M0) and sets bit 7
+     * of the scale for INT3, as IF4 does. */
+    float m = mode == ORC_NVINT3 ? 3.0f : 4.0f;
+    float q = m * s_g;
+    uint8_t S3 = oracle_e4m3_rne_sat(a_b / q);
+    float d3 = oracle_e4m3_decode(S3) * s_g;
+    if (d3 == 0.0f) {
+      memset(code, 0, 16);
+      return S3;
+    }
+    float r3 = 1.0f / d3;
+    uint8_t cf[16], ci[16];
+    float eF = 0.0f, eI = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+      float y = z[i] * r3;
+      if (mode == ORC_NVINT3) {
+        code[i] = int4_code(int3_level(y));
+        continue;
+      }
+      cf[i] = e2m0_rtn(y);
+      if (mode == ORC_NVFP3) {
+        code[i] = cf[i];
+        continue;
+      }
+      float dF = y - e2m0_decode(cf[i]);
+      eF = fmaf(dF, dF, eF);
+      int k = int3_level(y * IF3_K1);
+      ci[i] = int4_code(k);
+      float dI = y - (float)k * IF3_K2;
+      eI = fmaf(dI, dI, eI);
+    }
+    if (mode == ORC_IF3) {
+      if (eI < eF) {
+        memcpy(code, ci, 16);
+        return (uint8_t)(S3 | 0x80u);
+      }
+      memcpy(code, cf, 16);
+    }
+    return S3;
+  }
   if (mode == ORC_NVINT4) {
     /* NVINT4 [IF4-T1]: 16-element blocks, E4M3 scale, INT4 values, maximum
      * 7 x 448, minimum 1 x 2^-9.  Reading: as NVFP4 with the integer grid
@@ -666,24 +766,29 @@ int oracle_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, i
 int oracle_dequantize(const uint8_t* codes, const uint8_t* scales, float s_g,
                       int64_t vr, int64_t vc, int mode, int g, uint64_t seed,
                       int inverse_rht, float* out) {
-  if (mode < ORC_RTN || mode > ORC_NVINT4) return ORC_ERR_ARG;
+  if (mode < ORC_RTN || mode > ORC_MXFP3) return ORC_ERR_ARG;
   if (g != 0 && !valid_group(g)) return ORC_ERR_ARG;
   if (vr < 0 || vc < 0 || vc % 16 || (g && vc % g)) return ORC_ERR_SHAPE;
-  if (mode == ORC_MXFP4 && vc % 32) return ORC_ERR_SHAPE;
+  if ((mode == ORC_MXFP4 || mode == ORC_MXFP3) && vc % 32) return ORC_ERR_SHAPE;
   if (inverse_rht && g == 0) return ORC_ERR_ARG;
   for (int64_t r = 0; r < vr; ++r) {
     for (int64_t j = 0; j < vc; ++j) {
       uint8_t S = scales[r * (vc / 16) + j / 16];
       uint8_t byte = codes[r * (vc / 2) + j / 2];
       uint8_t code = (j & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15u);
-      int int4 = (mode == ORC_IF4 && (S & 0x80u)) || mode == ORC_NVINT4;
-      float d = mode == ORC_MXFP4 ? ldexpf(1.0f, (int)S - 127)  /* UE8M0: 2^(S - 127) */
-                                  : oracle_e4m3_decode((uint8_t)(S & 0x7Fu)) * s_g;
+      int flagged = (mode == ORC_IF4 || mode == ORC_IF3) && (S & 0x80u);
+      int integer = flagged || mode == ORC_NVINT4 || mode == ORC_NVINT3;
+      int e2m0 = mode == ORC_NVFP3 || mode == ORC_MXFP3 || (mode == ORC_IF3 && !flagged);
+      float d = (mode == ORC_MXFP4 || mode == ORC_MXFP3)
+                    ? ldexpf(1.0f, (int)S - 127) /* UE8M0: 2^(S - 127) */
+                    : oracle_e4m3_decode((uint8_t)(S & 0x7Fu)) * s_g;
       float v;
-      if (int4) {
+      if (integer) {
         int k = (int)(code & 7u);
         k = (code & 8u) ? -k : k;
-        v = mode == ORC_NVINT4 ? (float)k : int4_value(k);
+        v = mode == ORC_IF4 ? int4_value(k) : (mode == ORC_IF3 ? (float)k * IF3_K2 : (float)k);
+      } else if (e2m0) {
+        v = e2m0_decode(code);
       } else {
         v = oracle_e2m1_decode(code);
       }
@@ -727,8 +832,8 @@ void oracle_e4m3_array(const float* in, int64_t n, int round_up, uint8_t* out) {
 int oracle_quantize_rotated(const float* z, int64_t row0, int64_t vr, int64_t vc, int mode,
                             uint64_t seed, float amax, uint8_t* codes, uint8_t* scales,
                             float* global_scale) {
-  if (mode < ORC_RTN || mode > ORC_NVINT4) return ORC_ERR_ARG;
-  if (row0 < 0 || vr < 0 || vc < 0 || vc % 16 || (mode == ORC_MXFP4 && vc % 32)) return ORC_ERR_SHAPE;
+  if (mode < ORC_RTN || mode > ORC_MXFP3) return ORC_ERR_ARG;
+  if (row0 < 0 || vr < 0 || vc < 0 || vc % 16 || ((mode == ORC_MXFP4 || mode == ORC_MXFP3) && vc % 32)) return ORC_ERR_SHAPE;
   float s_g = oracle_global_scale(amax, mode);
   *global_scale = s_g;
   for (int64_t r = 0; r < vr; ++r) {

@@ -23,6 +23,9 @@
 * NVINT4 (IF4 page, Table 1: E4M3 scale, INT4 values, max 7 x 448): integer
   levels by brute-force nearest integer (ties to even) of the scaled value,
   and a lossless round trip.
+* 3-bit formats (IF4 page, 3-bit table: MXFP3, NVINT3, NVFP3, IF3): E2M0 and
+  INT3 rounding by brute force over every bf16 value in range, IF3 keeping
+  the lower-error option, MXFP3's shared exponent.
 * Table 1's MSE column (NVFP4 9.0, NVINT4 7.4, 4/6 7.5, IF4 6.2, MXFP4 13.2,
   x1e-3) on standard normal data, within 2% (tests/golden/if4_table1_mse.txt).
 * Structural properties: transposed view = row-wise quantization of X^T,
@@ -36,6 +39,8 @@ from nvfp4_microscaling_quantization_b200 import workloads as W
 
 ROW, TR = 0, 1
 RTN, SR, EDEN, IF4, FO6, SS, MX, NI4 = 0, 1, 2, 3, 4, 5, 6, 7
+NF3, NI3, IF3M, MX3 = 8, 9, 10, 11
+E2M0 = np.array([0.0, 1.0, 2.0, 4.0])
 GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
 
 
@@ -438,6 +443,101 @@ def test_nvint4_levels_and_round_trip(orc):
     assert np.array_equal(deq(orc, c2, s2, g2, NI4, 0, 0), xx)
 
 
+def _nearest_even(levels, t):
+    """Nearest of the magnitudes `levels` to |t| (ties to the even index), with t's sign."""
+    dist = np.abs(levels - min(abs(t), levels[-1]))
+    best = np.flatnonzero(dist == dist.min())
+    idx = int(best[0] if len(best) == 1 else best[best % 2 == 0][0])
+    return -levels[idx] if t < 0 else levels[idx]
+
+
+def _all_bf16_up_to(limit):
+    b = np.arange(1 << 16, dtype=np.uint32)
+    f = (b << 16).view(np.float32)
+    return f[np.isfinite(f) & (np.abs(f) <= limit)]
+
+
+def _unit_scale_blocks(vals, head):
+    """Blocks [head, v1..v15] (the head sets every block scale), 8 blocks a row."""
+    n = (len(vals) + 14) // 15
+    v = np.concatenate([vals, np.zeros(n * 15 - len(vals), dtype=np.float32)]).reshape(n, 15)
+    blocks = np.concatenate([np.full((n, 1), head, dtype=np.float32), v], axis=1)
+    rows = (n + 7) // 8
+    blocks = np.concatenate([blocks, np.zeros((rows * 8 - n, 16), dtype=np.float32)])
+    return blocks.reshape(rows, 128), v
+
+
+@pytest.mark.parametrize("mode,head,amax,levels,even", [
+    (NF3, 4.0, 7.0, E2M0, True),          # s_g = 7 / 1792 = 2^-8, block scale 256, d = 1
+    (NI3, 3.0, 5.25, np.array([0.0, 1.0, 2.0, 3.0]), True),  # s_g = 5.25 / 1344 = 2^-8
+])
+def test_3bit_grids_brute_force(orc, mode, head, amax, levels, even):
+    """Every bf16 value up to the grid maximum under a block scale of exactly 1:
+    the code is the nearest grid level (ties to the even level index, the
+    E2M0 code / the integer), sign in bit 3, zero as code 0."""
+    vals = _all_bf16_up_to(levels[-1])
+    mat, v = _unit_scale_blocks(vals, head)
+    codes, scales, gs = orc.quantize(bits_of(bf16(mat)), ROW, mode, 0, 0, amax_in=amax)
+    assert gs == 2.0 ** -8 and np.all(scales[:len(v) // 8] == 0x78)   # E4M3 256
+    cu = orc.unpack_codes(codes).reshape(-1, 16)[:len(v), 1:]
+    for i in range(len(v)):
+        for j in range(15):
+            a = abs(float(v[i, j]))
+            dist = np.abs(levels - a)
+            best = np.flatnonzero(dist == dist.min())
+            idx = int(best[0] if len(best) == 1 else best[best % 2 == 0][0])
+            exp = 0 if idx == 0 else (idx | (8 if v[i, j] < 0 else 0))
+            assert cu[i, j] == exp, (v[i, j], cu[i, j], exp)
+
+
+def test_if3_picks_lower_error_option(orc):
+    wl = W.activation(rows=32, cols=512)
+    bits = bits_of(wl.tensors()["a"])
+    codes, scales, gs, z = _block_views(orc, bits, ROW, IF3M, 0, 3)
+    cu = orc.unpack_codes(codes)
+    n_int = 0
+    for r in range(z.shape[0]):
+        for b in range(z.shape[1] // 16):
+            S = int(scales[r, b])
+            d = f32(f32(orc.e4m3_decode(S & 0x7F)) * f32(gs))
+            if d == 0:
+                continue
+            y = (z[r, 16 * b:16 * b + 16] * f32(f32(1.0) / d)).astype(np.float32)
+            fp = np.array([_nearest_even(E2M0, float(t)) for t in y])
+            k = np.clip(np.round((y * f32(0.75)).astype(np.float32)), -3, 3)
+            it = (k * f32(4.0 / 3.0)).astype(np.float32).astype(np.float64)
+            e_fp, e_int = np.sum((y - fp) ** 2), np.sum((y - it) ** 2)
+            flag = bool(S & 0x80)
+            n_int += flag
+            chosen, other = (e_int, e_fp) if flag else (e_fp, e_int)
+            assert chosen <= other * (1 + 1e-5) + 1e-12, (r, b)
+            if flag:
+                c = cu[r, 16 * b:16 * b + 16]
+                kk = np.where(c & 8, -(c & 7).astype(int), (c & 7).astype(int))
+                assert np.array_equal(kk, k.astype(int))
+    assert 0 < n_int < scales.size
+
+
+def test_mxfp3_shared_exponent(orc):
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((4, 256)) * 2.0 ** rng.integers(-20, 20, (4, 8)).repeat(32, 1)
+    xb = bf16(x)
+    codes, scales, gs = orc.quantize(bits_of(xb), ROW, MX3, 0, 0)
+    assert gs == 1.0
+    xv = xb.float().numpy()
+    cu = orc.unpack_codes(codes)
+    for r in range(4):
+        for gi in range(8):
+            grp = xv[r, 32 * gi:32 * gi + 32].astype(np.float64)
+            E = int(np.clip(np.frexp(np.abs(grp).max())[1] - 1 - 2, -127, 127))
+            assert scales[r, 2 * gi] == scales[r, 2 * gi + 1] == E + 127
+            vals = np.array([E2M0[c & 3] * (-1 if c & 8 else 1) for c in cu[r, 32 * gi:32 * gi + 32]])
+            # every code is a nearest E2M0 level of x / 2^E (saturating at 4)
+            y = np.minimum(np.abs(grp / 2.0 ** E), 4.0)
+            nearest = np.min(np.abs(E2M0[None, :] - y[:, None]), axis=1)
+            assert np.allclose(np.abs(np.abs(vals) - y), nearest)
+
+
 def test_table1_mse_on_gaussian(orc):
     """The MSE column of the IF4 page's Table 1 (tests/golden/if4_table1_mse.txt):
     NVFP4, 4/6, IF4 and MXFP4 on 2^20 standard normal values, each within 2% of
@@ -464,7 +564,8 @@ def test_mxfp4_needs_whole_groups(orc):
 
 # ------------------------------------------------------------------- structural
 @pytest.mark.parametrize("mode,g", [(RTN, 0), (SR, 0), (EDEN, 128), (IF4, 0), (FO6, 0), (SR, 32), (SS, 0),
-                                    (SS, 64), (MX, 0), (MX, 128), (NI4, 0), (NI4, 32)])
+                                    (SS, 64), (MX, 0), (MX, 128), (NI4, 0), (NI4, 32),
+                                    (NF3, 0), (NI3, 16), (IF3M, 0), (IF3M, 128), (MX3, 0)])
 def test_transposed_is_rowwise_of_transpose(orc, mode, g):
     rng = np.random.default_rng(6)
     x = bf16(rng.standard_normal((256, 64)))
