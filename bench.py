@@ -48,8 +48,8 @@ L2_FLUSH_BYTES = 256 << 20
 # kernel reports traffic = null until it is captured again.
 NCU_TRAFFIC = {
     # profiles/rotate_mma_eden_dy.md: dram__bytes_read.sum + dram__bytes_write.sum, one launch
-    ("91ca2cb3659b8b2c", "dy.transposed.ms_eden.g128"): 470039296 + 108451584,
-    ("91ca2cb3659b8b2c", "dy.rowwise.ms_eden.g128"): 469872128 + 108522240,
+    ("99074ee665c907e2", "dy.transposed.ms_eden.g128"): 470025472 + 108604928,
+    ("99074ee665c907e2", "dy.rowwise.ms_eden.g128"): 469999616 + 110624256,
 }
 
 
@@ -268,7 +268,8 @@ def per_mode_table(N, W, x, seed, stream, device, flush, peak, reps=5):
     from nvfp4_microscaling_quantization_b200.workloads import Call as WCall
     out = []
     for layout in (W.ROWWISE, W.TRANSPOSED):
-        for mode in (W.RTN, W.SR, W.MS_EDEN, W.IF4, W.FOUR_OVER_SIX, W.SCALE_SEARCH, W.MXFP4, W.NVINT4):
+        for mode in (W.RTN, W.SR, W.MS_EDEN, W.IF4, W.FOUR_OVER_SIX, W.SCALE_SEARCH, W.MXFP4, W.NVINT4,
+                     W.NVFP3, W.NVINT3, W.IF3, W.MXFP3):
             for g in (0, 128):
                 if mode == W.MS_EDEN and g == 0:
                     continue

@@ -97,9 +97,17 @@ typedef enum {
                         the workspace unused); the scale byte E + 127 is stored for each
                         16-element half of a group; needs vcols % 32 == 0 and a view of at least
                         one tile of the tiled kernels (else NVFP4_ERR_UNSUPPORTED) */
-  NVFP4_NVINT4 = 7   /* NVINT4 (IF4 paper page, Table 1): E4M3 block scale mapping the absmax to
+  NVFP4_NVINT4 = 7,  /* NVINT4 (IF4 paper page, Table 1): E4M3 block scale mapping the absmax to
                         7, INT4 levels k = clamp(RNE(z / d), -7, 7) stored as sign-magnitude
                         nibbles (as IF4's INT4 option, value k d), amax -> 7 x 448 */
+  /* 3-bit formats (IF4 paper page, the 3-bit table), codes held in nibbles
+   * (sign bit 3, magnitude code bits 0..1): E2M0 magnitudes {0, 1, 2, 4}
+   * (nearest, ties to the even code), INT3 levels |k| <= 3. */
+  NVFP4_NVFP3 = 8,   /* E4M3 block scale mapping the absmax to 4, E2M0 values, amax -> 4 x 448 */
+  NVFP4_NVINT3 = 9,  /* E4M3 block scale mapping the absmax to 3, INT3 levels, amax -> 3 x 448 */
+  NVFP4_IF3 = 10,    /* per block E2M0 or INT3 levels k standing for k 4/3 under one E4M3 scale
+                        (lower squared error, bit 7 of the scale = INT3), amax -> 4 x 448 */
+  NVFP4_MXFP3 = 11   /* as NVFP4_MXFP4 with E2M0 values (same shape rules) */
 } nvfp4_mode;
 
 /* Bytes of device workspace nvfp4_quantize needs when amax_in is NULL (the

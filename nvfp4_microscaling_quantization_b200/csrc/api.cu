@@ -40,7 +40,7 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CU
 extern "C" {
 
 size_t nvfp4_workspace_bytes(int64_t rows, int64_t cols, int layout, int mode, int rht_group) {
-  if (rows < 0 || cols < 0 || (layout != 0 && layout != 1) || mode < 0 || mode > NVFP4_NVINT4 ||
+  if (rows < 0 || cols < 0 || (layout != 0 && layout != 1) || mode < 0 || mode > NVFP4_MXFP3 ||
       !valid_group(rht_group))
     return 0;
   return kWorkspaceBytes;
@@ -90,15 +90,16 @@ int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int la
   int64_t vr, vc;
   int st = check_tensor(x, rows, cols, ld, layout, rht_group, &vr, &vc);
   if (st) return st;
-  if (mode < NVFP4_RTN || mode > NVFP4_NVINT4) return NVFP4_ERR_INVALID_ARG;
+  if (mode < NVFP4_RTN || mode > NVFP4_MXFP3) return NVFP4_ERR_INVALID_ARG;
   if (mode == NVFP4_MS_EDEN && rht_group == 0) return NVFP4_ERR_UNSUPPORTED;
-  if (mode == NVFP4_MXFP4 && vc % 32) return NVFP4_ERR_SHAPE;
+  const bool mx = mode == NVFP4_MXFP4 || mode == NVFP4_MXFP3;
+  if (mx && vc % 32) return NVFP4_ERR_SHAPE;
   const bool empty = vr == 0 || vc == 0;
   if (!global_scale || (!empty && (!codes || !scales))) return NVFP4_ERR_INVALID_ARG;
   if (!aligned(codes, 8) || !aligned(global_scale, 4)) return NVFP4_ERR_ALIGNMENT;
   if (amax_in && !aligned(amax_in, 4)) return NVFP4_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (mode == NVFP4_MXFP4) {
+  if (mx) {
     // no tensor amax: amax_in and the workspace are not used; the kernels
     // read one float from amax (ignored), so they get the output scalar
     nvfp4::QuantArgs m{x, rows, cols, ld, layout, mode, rht_group, seed, global_scale, nullptr,
@@ -125,8 +126,8 @@ int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g
                      int64_t vrows, int64_t vcols, int mode, int rht_group, uint64_t seed,
                      int inverse_rht, float* out, void* stream) {
   if (!codes || !scales || !global_scale || !out) return NVFP4_ERR_INVALID_ARG;
-  if (mode < NVFP4_RTN || mode > NVFP4_NVINT4 || !valid_group(rht_group)) return NVFP4_ERR_INVALID_ARG;
-  if (mode == NVFP4_MXFP4 && vcols % 32) return NVFP4_ERR_SHAPE;
+  if (mode < NVFP4_RTN || mode > NVFP4_MXFP3 || !valid_group(rht_group)) return NVFP4_ERR_INVALID_ARG;
+  if ((mode == NVFP4_MXFP4 || mode == NVFP4_MXFP3) && vcols % 32) return NVFP4_ERR_SHAPE;
   if (inverse_rht && rht_group == 0) return NVFP4_ERR_INVALID_ARG;
   if (vrows < 0 || vcols < 0 || vcols % 16 || (rht_group && vcols % rht_group)) return NVFP4_ERR_SHAPE;
   if (!aligned(codes, 8) || !aligned(out, 16) || !aligned(global_scale, 4)) return NVFP4_ERR_ALIGNMENT;

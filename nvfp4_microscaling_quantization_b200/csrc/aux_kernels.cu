@@ -37,19 +37,25 @@ dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
     if (valid) {
       const uint2 c = *reinterpret_cast<const uint2*>(codes + b * 8);
       const uint32_t S = scales[b];
-      // MXFP4: UE8M0 scale 2^(S - 127) (S = 0: the subnormal 2^-127); else
-      // RN(E4M3(S) * s_g)
-      const float d = mode == kMXFP4 ? __uint_as_float(S ? (S << 23) : 0x00400000u)
-                                     : __fmul_rn(e4m3_decode(S & 0x7Fu), s_g);
-      if ((mode == kIF4 && (S & 0x80u)) || mode == kNVINT4) {
+      // MXFP4 / MXFP3: UE8M0 scale 2^(S - 127) (S = 0: the subnormal
+      // 2^-127); else RN(E4M3(S) * s_g)
+      const bool mx = mode == kMXFP4 || mode == kMXFP3;
+      const float d = mx ? __uint_as_float(S ? (S << 23) : 0x00400000u) : __fmul_rn(e4m3_decode(S & 0x7Fu), s_g);
+      const bool flagged = (mode == kIF4 || mode == kIF3) && (S & 0x80u);
+      if (flagged || mode == kNVINT4 || mode == kNVINT3) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const uint32_t code = ((i < 8 ? c.x : c.y) >> (4 * (i & 7))) & 0xFu;
           const int k = (code & 8u) ? -static_cast<int>(code & 7u) : static_cast<int>(code & 7u);
-          // IF4: RN(RN(k RN(6/7)) d); NVINT4: RN(k d)
-          const float lv = mode == kNVINT4 ? static_cast<float>(k) : __fmul_rn(static_cast<float>(k), kIF4K2);
+          // IF4: RN(RN(k RN(6/7)) d); IF3: RN(RN(k RN(4/3)) d); NVINT4/3: RN(k d)
+          const float lv = mode == kIF4 ? __fmul_rn(static_cast<float>(k), kIF4K2)
+                           : (mode == kIF3 ? __fmul_rn(static_cast<float>(k), kIF3K2) : static_cast<float>(k));
           v[i] = __fmul_rn(lv, d);
         }
+      } else if (mode == kNVFP3 || mode == kMXFP3 || mode == kIF3) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          v[i] = __fmul_rn(e2m0_value(((i < 8 ? c.x : c.y) >> (4 * (i & 7))) & 0xFu), d);
       } else {
         e2m1x8_to_f32(c.x, v);
         e2m1x8_to_f32(c.y, v + 8);

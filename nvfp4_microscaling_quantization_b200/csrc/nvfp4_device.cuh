@@ -15,7 +15,14 @@
 
 namespace nvfp4 {
 
-enum Mode { kRTN = 0, kSR = 1, kMSEDEN = 2, kIF4 = 3, k4over6 = 4, kScaleSearch = 5, kMXFP4 = 6, kNVINT4 = 7 };
+enum Mode {
+  kRTN = 0, kSR = 1, kMSEDEN = 2, kIF4 = 3, k4over6 = 4, kScaleSearch = 5, kMXFP4 = 6, kNVINT4 = 7,
+  kNVFP3 = 8, kNVINT3 = 9, kIF3 = 10, kMXFP3 = 11
+};
+template <int MODE>
+__host__ __device__ constexpr bool is_mx() { return MODE == kMXFP4 || MODE == kMXFP3; }
+template <int MODE>
+__host__ __device__ constexpr bool is_3bit_e4m3() { return MODE == kNVFP3 || MODE == kNVINT3 || MODE == kIF3; }
 
 // Scale search: the candidates are the E4M3 codes S0 + delta(t), t = 0 ..
 // 18, around the absmax scale S0, visited nearest first (0, -1, +1, -2, ...),
@@ -282,8 +289,10 @@ __device__ __forceinline__ void rht_inverse(float* v, uint32_t sign_bits, uint32
 // search, else 448.
 template <int MODE>
 __device__ __forceinline__ float global_scale_of(float amax) {
-  if constexpr (MODE == kMXFP4) return 1.0f;  // MXFP4 has no tensor scale
+  if constexpr (is_mx<MODE>()) return 1.0f;  // MXFP4 / MXFP3 have no tensor scale
   if constexpr (MODE == kNVINT4) return amax > 0.0f ? __fdiv_rn(amax, 3136.0f) : 1.0f;  // 7 x 448
+  if constexpr (MODE == kNVFP3 || MODE == kIF3) return amax > 0.0f ? __fdiv_rn(amax, 1792.0f) : 1.0f;  // 4 x 448
+  if constexpr (MODE == kNVINT3) return amax > 0.0f ? __fdiv_rn(amax, 1344.0f) : 1.0f;  // 3 x 448
   constexpr float six_m = (MODE == kMSEDEN || MODE == k4over6 || MODE == kScaleSearch) ? 1536.0f : 2688.0f;
   return amax > 0.0f ? __fdiv_rn(amax, six_m) : 1.0f;
 }
@@ -304,6 +313,29 @@ __device__ __forceinline__ uint32_t int4_nibble(float y) {
   return (__float_as_uint(__fadd_rn(fabsf(k), 8388608.0f)) & 7u) | ((__float_as_uint(k) >> 28) & 8u);
 }
 
+// 3-bit elements, stored in nibbles (sign bit 3, magnitude code bits 0..1).
+// E2M0: magnitudes {0, 1, 2, 4}, nearest with ties to the even code (0.5 ->
+// 0, 1.5 -> 2, 3 -> 2), saturating at 4; zero is code 0.
+__device__ __forceinline__ uint32_t e2m0_nibble(float y) {
+  const float a = fabsf(y);
+  const uint32_t m = (a > 0.5f ? 1u : 0u) + (a >= 1.5f ? 1u : 0u) + (a > 3.0f ? 1u : 0u);
+  return m == 0u ? 0u : (m | ((__float_as_uint(y) >> 28) & 8u));
+}
+// signed E2M0 value of a nibble: 2^(m - 1) for m = 1..3
+__device__ __forceinline__ float e2m0_value(uint32_t c) {
+  const uint32_t m = c & 3u;
+  return m == 0u ? 0.0f : __uint_as_float(((126u + m) << 23) | ((c & 8u) << 28));
+}
+// INT3: k = clamp(RNE(t), -3, 3) as a sign-magnitude nibble (as int4_nibble)
+__device__ __forceinline__ float int3_level(float t) {
+  return fminf(fmaxf(__fsub_rn(__fadd_rn(t, kRoundMagic), kRoundMagic), -3.0f), 3.0f);
+}
+__device__ __forceinline__ uint32_t level_nibble(float k) {
+  return (__float_as_uint(__fadd_rn(fabsf(k), 8388608.0f)) & 7u) | ((__float_as_uint(k) >> 28) & 8u);
+}
+constexpr float kIF3K1 = 0.75f;            // RN(3/4)
+constexpr float kIF3K2 = 0x1.555556p+0f;   // RN(4/3)
+
 // Where the random draws of one 16-element block come from.
 struct BlockRng {
   PhiloxKey key;
@@ -313,8 +345,52 @@ struct BlockRng {
 
 struct BlockOut {
   uint32_t lo, hi;  // 16 packed codes: lo = elements 0..7, hi = elements 8..15
-  uint32_t scale;   // scale byte (bit 7 = IF4 INT4 flag)
+  uint32_t scale;   // scale byte (bit 7 = the IF4 / IF3 integer flag)
 };
+
+// NVFP3 / NVINT3 / IF3 codes of one block of scaled values y under scale
+// byte S: E2M0, INT3, or (IF3) the option with the lower squared error in the
+// y domain (fmaf in element order, ties keep E2M0) with bit 7 set for INT3.
+template <int MODE>
+__device__ __forceinline__ BlockOut block3_codes(const float* y, uint32_t S) {
+  BlockOut o{0u, 0u, S};
+  uint32_t f_lo = 0u, f_hi = 0u, i_lo = 0u, i_hi = 0u;
+  float eF = 0.0f, eI = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    uint32_t cf = 0u, ci = 0u;
+    if constexpr (MODE == kNVINT3) {
+      cf = level_nibble(int3_level(y[i]));
+    } else {
+      cf = e2m0_nibble(y[i]);
+      if constexpr (MODE == kIF3) {
+        const float dF = __fsub_rn(y[i], e2m0_value(cf));
+        eF = __fmaf_rn(dF, dF, eF);
+        const float k = int3_level(__fmul_rn(y[i], kIF3K1));
+        const float dI = __fsub_rn(y[i], __fmul_rn(k, kIF3K2));
+        eI = __fmaf_rn(dI, dI, eI);
+        ci = level_nibble(k);
+      }
+    }
+    if (i < 8) {
+      f_lo |= cf << (4 * i);
+      i_lo |= ci << (4 * i);
+    } else {
+      f_hi |= cf << (4 * (i - 8));
+      i_hi |= ci << (4 * (i - 8));
+    }
+  }
+  if (MODE == kIF3 && eI < eF) {
+    o.lo = i_lo;
+    o.hi = i_hi;
+    o.scale = S | 0x80u;
+  } else {
+    o.lo = f_lo;
+    o.hi = f_hi;
+  }
+  return o;
+}
+
 
 __device__ __forceinline__ float block_absmax(const float* z) {
   float a = 0.0f;
@@ -400,6 +476,17 @@ __device__ __forceinline__ BlockOut quantize_block(const float* z, float s_g, co
     out.hi = c_hi[pick];
     out.scale = S[pick];
     return out;
+  } else if constexpr (is_3bit_e4m3<MODE>()) {
+    const float m = MODE == kNVINT3 ? 3.0f : 4.0f;
+    const uint32_t S = e4m3_rne_sat(__fdiv_rn(a_b, __fmul_rn(m, s_g)));
+    const float d = __fmul_rn(e4m3_decode(S), s_g);
+    out.scale = S;
+    if (d == 0.0f) return out;
+    const float r = __frcp_rn(d);
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(z[i], r);
+    return block3_codes<MODE>(y, S);
   } else if constexpr (MODE == kNVINT4) {
     const uint32_t S = e4m3_rne_sat(__fdiv_rn(a_b, __fmul_rn(7.0f, s_g)));
     const float d = __fmul_rn(e4m3_decode(S), s_g);
@@ -541,8 +628,12 @@ __device__ __forceinline__ ScaleCtx make_scale_ctx(float amax) {
   ScaleCtx c;
   c.tbl = nullptr;
   c.s_g = global_scale_of<MODE>(amax);
-  // the absmax divisor: RN(6 s_g), or RN(7 s_g) for NVINT4 (INT4's maximum 7)
-  c.q6 = __fmul_rn(MODE == kNVINT4 ? 7.0f : 6.0f, c.s_g);
+  // the absmax divisor RN(m s_g), m = the element maximum: 6 (E2M1), 7
+  // (NVINT4), 4 (E2M0: NVFP3, IF3), 3 (NVINT3)
+  constexpr float m = MODE == kNVINT4 ? 7.0f
+                      : (MODE == kNVFP3 || MODE == kIF3) ? 4.0f
+                      : MODE == kNVINT3 ? 3.0f : 6.0f;
+  c.q6 = __fmul_rn(m, c.s_g);
   c.q4 = __fmul_rn(4.0f, c.s_g);
   c.r6 = __frcp_rn(c.q6);
   c.r4 = __frcp_rn(c.q4);
@@ -704,6 +795,44 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
     ob.lo = pb ? cb_lo[1] : cb_lo[0];
     ob.hi = pb ? cb_hi[1] : cb_hi[0];
     ob.scale = ((pb ? S[1] : S[0]) >> 8) & 0xFFu;
+    return;
+  } else if constexpr (is_3bit_e4m3<MODE>()) {
+    // q6 holds RN(m s_g) for the mode's element maximum m (make_scale_ctx)
+    const float2 sf = div2_by(f2(aa, ab), sc.q6, sc.r6, sc.markstein);
+    const uint32_t S2 = e4m3x2_rne_sat(sf.x, sf.y);
+    const uint32_t Sa = S2 & 0xFFu, Sb = S2 >> 8;
+    const float4 ta = scale_entry<TBL>(sc, Sa), tb = scale_entry<TBL>(sc, Sb);
+    const float2 r = f2(ta.z, tb.z);  // 0 for a zero scale: y = 0, codes 0, no flag
+    float ya[16], yb[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 y = mul2_rn(z[i], r);
+      ya[i] = y.x;
+      yb[i] = y.y;
+    }
+    oa = block3_codes<MODE>(ya, Sa);
+    ob = block3_codes<MODE>(yb, Sb);
+    return;
+  } else if constexpr (MODE == kMXFP3) {
+    // one 32-element group, as MXFP4 with E2M0 elements (E2M0's largest
+    // value, 4, has exponent 2 as E2M1's 6 does: the same scale byte)
+    const uint32_t f = __float_as_uint(fmaxf(aa, ab)) >> 23;
+    const uint32_t byte = f > 2u ? f - 2u : 0u;
+    const float inv = __uint_as_float((254u - byte) << 23);
+    oa = BlockOut{0u, 0u, byte};
+    ob = BlockOut{0u, 0u, byte};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 y = mul2_rn(z[i], f2(inv, inv));
+      const uint32_t ca = e2m0_nibble(y.x), cb = e2m0_nibble(y.y);
+      if (i < 8) {
+        oa.lo |= ca << (4 * i);
+        ob.lo |= cb << (4 * i);
+      } else {
+        oa.hi |= ca << (4 * (i - 8));
+        ob.hi |= cb << (4 * (i - 8));
+      }
+    }
     return;
   } else if constexpr (MODE == kNVINT4) {
     // q6 holds RN(7 s_g) for this mode (make_scale_ctx)

@@ -244,13 +244,13 @@ cudaError_t launch_amax(const QuantArgs& a) {
   return dispatch_group<kRTN, true>(a);
 }
 
-// The tensor scale of an empty MXFP4 call (MXFP4 has none: 1).
+// The tensor scale of an empty MXFP4 / MXFP3 call (they have none: 1).
 __global__ void set_one_kernel(float* p) { *p = 1.0f; }
 
 cudaError_t launch_quantize(const QuantArgs& a) {
   if (mma_path_applies(a)) return launch_quantize_mma(a);
   if (tma_path_applies(a)) return launch_quantize_tma(a);
-  if (a.mode == kMXFP4) {
+  if (a.mode == kMXFP4 || a.mode == kMXFP3) {
     // MXFP4 groups are the block pairs of the tiled kernels; the one-block
     // kernels do not form them (the C ABI rejects such shapes up front)
     if (a.rows != 0 && a.cols != 0) return cudaErrorNotSupported;
@@ -265,6 +265,9 @@ cudaError_t launch_quantize(const QuantArgs& a) {
     case k4over6: return dispatch_group<k4over6, false>(a);
     case kScaleSearch: return dispatch_group<kScaleSearch, false>(a);
     case kNVINT4: return dispatch_group<kNVINT4, false>(a);
+    case kNVFP3: return dispatch_group<kNVFP3, false>(a);
+    case kNVINT3: return dispatch_group<kNVINT3, false>(a);
+    case kIF3: return dispatch_group<kIF3, false>(a);
     default: return cudaErrorInvalidValue;
   }
 }

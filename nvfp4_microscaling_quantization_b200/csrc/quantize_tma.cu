@@ -442,6 +442,10 @@ cudaError_t launch_quantize_tma(const QuantArgs& a) {
     case kScaleSearch: return dispatch_tma<kScaleSearch, false>(a);
     case kMXFP4: return dispatch_tma<kMXFP4, false>(a);
     case kNVINT4: return dispatch_tma<kNVINT4, false>(a);
+    case kNVFP3: return dispatch_tma<kNVFP3, false>(a);
+    case kNVINT3: return dispatch_tma<kNVINT3, false>(a);
+    case kIF3: return dispatch_tma<kIF3, false>(a);
+    case kMXFP3: return dispatch_tma<kMXFP3, false>(a);
     default: return cudaErrorInvalidValue;
   }
 }

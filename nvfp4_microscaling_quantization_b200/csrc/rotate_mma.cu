@@ -767,6 +767,10 @@ cudaError_t launch_quantize_mma(const QuantArgs& a) {
     case kScaleSearch: return dispatch<kScaleSearch, kQuantize>(a, nullptr);
     case kMXFP4: return dispatch<kMXFP4, kQuantize>(a, nullptr);
     case kNVINT4: return dispatch<kNVINT4, kQuantize>(a, nullptr);
+    case kNVFP3: return dispatch<kNVFP3, kQuantize>(a, nullptr);
+    case kNVINT3: return dispatch<kNVINT3, kQuantize>(a, nullptr);
+    case kIF3: return dispatch<kIF3, kQuantize>(a, nullptr);
+    case kMXFP3: return dispatch<kMXFP3, kQuantize>(a, nullptr);
     default: return cudaErrorInvalidValue;
   }
 }

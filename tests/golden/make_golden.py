@@ -28,7 +28,8 @@ def digest_lines():
     calls = list(wl.calls) + [workloads.Call("x", 1, m, 128) for m in (0, 1, 2, 3, 4)] + \
         [workloads.Call("x", 0, 3, 0), workloads.Call("x", 0, 4, 0), workloads.Call("x", 0, 5, 0),
          workloads.Call("x", 1, 5, 128), workloads.Call("x", 0, 6, 0), workloads.Call("x", 1, 6, 128),
-         workloads.Call("x", 0, 7, 0), workloads.Call("x", 1, 7, 128)]
+         workloads.Call("x", 0, 7, 0), workloads.Call("x", 1, 7, 128)] + \
+        [workloads.Call("x", lay, m, g) for m in (8, 9, 10, 11) for lay, g in ((0, 0), (1, 128))]
     for c in calls:
         codes, scales, gs = oracle.quantize(x, c.layout, c.mode, c.rht_group, wl.seed)
         h = hashlib.sha256(codes.tobytes() + scales.tobytes()).hexdigest()

@@ -63,7 +63,7 @@ def test_status_strings(N):
 def test_workspace_bytes(N):
     assert N.nvfp4_workspace_bytes(4096, 4096, 0, 2, 128) == 256
     assert N.nvfp4_workspace_bytes(4096, 4096, 2, 2, 128) == 0
-    assert N.nvfp4_workspace_bytes(4096, 4096, 0, 9, 128) == 0
+    assert N.nvfp4_workspace_bytes(4096, 4096, 0, 12, 128) == 0
     assert N.nvfp4_workspace_bytes(4096, 4096, 0, 0, 48) == 0
 
 
@@ -78,9 +78,11 @@ def test_quantize_rejects(N):
     assert q(N, x=None, rows=0, gs=None) == INVALID
     assert q(N, layout=2) == INVALID
     assert q(N, g=48) == INVALID
-    assert q(N, mode=8) == INVALID
+    assert q(N, mode=12) == INVALID
     assert q(N, mode=6, cols=48, ld=48) == SHAPE          # MXFP4: whole 32-element groups
     assert q(N, mode=6, rows=8, cols=64) == UNSUPPORTED   # MXFP4: below one tile of the tiled kernels
+    assert q(N, mode=11, cols=48, ld=48) == SHAPE         # MXFP3 likewise
+    assert q(N, mode=11, rows=8, cols=64) == UNSUPPORTED
     assert q(N, cols=40, ld=40) == SHAPE            # row-wise blocks need cols % 16 == 0
     assert q(N, rows=40, layout=1) == SHAPE         # transposed blocks need rows % 16 == 0
     assert q(N, cols=64, g=128) == SHAPE            # rotation group must divide the block dimension
@@ -103,7 +105,7 @@ def test_noalloc_rejects_like_quantize(N):
     nq = N.nvfp4_quantize_noalloc
     assert nq(FAKE, 64, 64, 64, 2, 0, 0, 0, None, FAKE, FAKE, FAKE, None) == INVALID   # layout
     assert nq(FAKE, 64, 64, 64, 0, 0, 48, 0, None, FAKE, FAKE, FAKE, None) == INVALID  # group
-    assert nq(FAKE, 64, 64, 64, 0, 9, 0, 0, None, FAKE, FAKE, FAKE, None) == INVALID   # mode
+    assert nq(FAKE, 64, 64, 64, 0, 12, 0, 0, None, FAKE, FAKE, FAKE, None) == INVALID  # mode
 
 
 def test_other_entry_points_reject(N):
@@ -122,7 +124,7 @@ def test_other_entry_points_reject(N):
     assert d(None, FAKE, FAKE, 4, 64, 0, 0, 0, 0, FAKE, None) == INVALID
     assert d(FAKE, FAKE, FAKE, 4, 64, 0, 0, 0, 1, FAKE, None) == INVALID  # inverse without rotation
     assert d(FAKE, FAKE, FAKE, 4, 40, 0, 0, 0, 0, FAKE, None) == SHAPE
-    assert d(FAKE, FAKE, FAKE, 4, 64, 8, 0, 0, 0, FAKE, None) == INVALID
+    assert d(FAKE, FAKE, FAKE, 4, 64, 12, 0, 0, 0, FAKE, None) == INVALID
     assert d(FAKE, FAKE, FAKE, 4, 64, 0, 0, 0, 0, FAKE + 4, None) == ALIGN
     r = N.nvfp4_rht
     assert r(FAKE, 0, 64, 64, 64, 0, 0, 0, 0, FAKE, None) == INVALID      # group 0

@@ -21,7 +21,8 @@ from gpu_helpers import (ROT_TOL, assert_same, bits, check_rotation, compare_cal
 
 pytestmark = pytest.mark.gpu
 
-MODES = [W.RTN, W.SR, W.MS_EDEN, W.IF4, W.FOUR_OVER_SIX, W.SCALE_SEARCH, W.MXFP4, W.NVINT4]
+MODES = [W.RTN, W.SR, W.MS_EDEN, W.IF4, W.FOUR_OVER_SIX, W.SCALE_SEARCH, W.MXFP4, W.NVINT4, W.NVFP3, W.NVINT3, W.IF3,
+         W.MXFP3]
 GROUPS = [0, 16, 32, 64, 128]
 
 
@@ -94,6 +95,16 @@ RAGGED = [
     (40, 176, 8, W.ROWWISE, W.NVINT4, 16),
     (208, 72, 8, W.TRANSPOSED, W.NVINT4, 0),
     (640, 384, 0, W.TRANSPOSED, W.NVINT4, 128),
+    # 3-bit formats on each path
+    (37, 48, 8, W.ROWWISE, W.NVFP3, 16),
+    (48, 72, 0, W.TRANSPOSED, W.IF3, 0),
+    (5, 16, 0, W.ROWWISE, W.NVINT3, 0),
+    (40, 176, 8, W.ROWWISE, W.IF3, 16),
+    (208, 72, 8, W.TRANSPOSED, W.NVINT3, 0),
+    (19, 1056, 0, W.ROWWISE, W.MXFP3, 0),
+    (640, 384, 0, W.TRANSPOSED, W.IF3, 128),
+    (384, 1152, 0, W.ROWWISE, W.MXFP3, 128),
+    (256, 64, 0, W.TRANSPOSED, W.NVFP3, 128),
 ]
 
 
@@ -176,7 +187,8 @@ def test_rotation_parity(layout, g, shape):
 
 
 EDGE_MODES = [(W.RTN, 0), (W.SR, 0), (W.MS_EDEN, 16), (W.IF4, 0), (W.FOUR_OVER_SIX, 0), (W.IF4, 128),
-              (W.SR, 128), (W.SCALE_SEARCH, 0), (W.MXFP4, 0), (W.NVINT4, 0)]
+              (W.SR, 128), (W.SCALE_SEARCH, 0), (W.MXFP4, 0), (W.NVINT4, 0), (W.NVFP3, 0), (W.NVINT3, 0),
+              (W.IF3, 0), (W.MXFP3, 0)]
 
 
 def _edge_tensors():
@@ -226,7 +238,8 @@ def test_exhaustive_bf16_rtn_path():
     pad = np.zeros((rows * 8 - n, 16), dtype=np.float32)
     mat = np.concatenate([blocks, pad]).reshape(rows, 128)
     x = torch.from_numpy(mat).to(torch.bfloat16)
-    for mode in (W.RTN, W.SR, W.IF4, W.FOUR_OVER_SIX, W.SCALE_SEARCH, W.MXFP4, W.NVINT4):
+    for mode in (W.RTN, W.SR, W.IF4, W.FOUR_OVER_SIX, W.SCALE_SEARCH, W.MXFP4, W.NVINT4, W.NVFP3, W.NVINT3, W.IF3,
+                 W.MXFP3):
         gpu = compare_call(x, W.ROWWISE, mode, 0, 7, amax=10.5)
         if mode == W.RTN:
             assert gpu[2] == 2.0 ** -8
