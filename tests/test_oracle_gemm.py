@@ -8,7 +8,9 @@
   quantize (RTN) without error, so the GEMM of their quantizations is X W^T
   exactly, computed here by numpy from X and W themselves;
 - operand-order invariants: swapping A and B transposes D, scaling one tensor
-  scale by 2 scales D by 2.
+  scale by 2 scales D by 2;
+- operands rotated with the same seed multiply to X W^T within the
+  quantization error; with different seeds they do not.
 """
 from fractions import Fraction
 
@@ -101,3 +103,34 @@ def test_gemm_rejects_if4_scales():
     asc[0, 0] |= 0x80
     with pytest.raises(ValueError):
         oracle.gemm(ac, asc, 1.0, ac, asc, 1.0)
+
+
+def test_gemm_of_rotated_operands_cancels_the_rotation():
+    """Two operands rotated along k with the same seed (one sign vector shared
+    by every group and both operands) multiply to X W^T up to the quantization
+    error, because c_g H_g diag(sigma) is orthogonal up to the rounding of c_g
+    (Quartet II article, "Quantisierung im Vorwaertsdurchlauf": rotations
+    along the microscaling groups; the shared sign vector is the reading that
+    makes them cancel).  With different seeds the rotations do not cancel and
+    the product is unrelated to X W^T."""
+    gen = torch.Generator().manual_seed(3)
+    x = torch.randn(128, 1024, generator=gen).to(torch.bfloat16)
+    w = (torch.randn(96, 1024, generator=gen) * 0.02).to(torch.bfloat16)
+    exact = x.double().numpy() @ w.double().numpy().T
+    xb, wb = W.bf16_bits(x), W.bf16_bits(w)
+
+    def rel(seed_x, seed_w, mode, g):
+        qa = oracle.quantize(xb, oracle.ROWWISE, mode, g, seed_x)
+        qb = oracle.quantize(wb, oracle.ROWWISE, mode, g, seed_w)
+        d = oracle.gemm(*qa, *qb)
+        return np.linalg.norm(d - exact) / np.linalg.norm(exact)
+
+    plain = rel(5, 5, oracle.RTN, 0)
+    same = rel(5, 5, oracle.MS_EDEN, 128)
+    other = rel(5, 6, oracle.MS_EDEN, 128)
+    print(f"\nrelative Frobenius error of the GEMM: RTN {plain:.4f}, MS-EDEN same seed {same:.4f}, "
+          f"different seeds {other:.3f}")
+    # each operand carries ~9.5% relative RMS quantization error (NVFP4 MSE
+    # 9e-3 per unit variance), so a dot product of two carries ~sqrt(2) x 9.5%
+    assert plain < 0.2 and same < 1.2 * plain
+    assert other > 0.9
