@@ -538,6 +538,20 @@ def test_mxfp3_shared_exponent(orc):
             assert np.allclose(np.abs(np.abs(vals) - y), nearest)
 
 
+def test_3bit_error_ordering_follows_the_3bit_table(orc):
+    """The IF4 page's 3-bit table ranks the formats by perplexity (IF3 10.67 <
+    NVFP3 11.12 < NVINT3 12.78 < MXFP3 70.04).  The quantization MSE under
+    the readings ranks them the same way on Gaussian and on Laplace
+    per-channel data (reported; gated on the order)."""
+    rng = np.random.default_rng(16)
+    data = {"N(0,1)": bf16(rng.standard_normal((256, 1024))),
+            "laplace channels": W.activation(rows=128, cols=1024).tensors()["a"]}
+    for name, x in data.items():
+        m = [_mse(orc, x, mode, 0, [0]) for mode in (IF3M, NF3, NI3, MX3)]
+        print(f"\n{name}: MSE IF3 {m[0]:.4g}  NVFP3 {m[1]:.4g}  NVINT3 {m[2]:.4g}  MXFP3 {m[3]:.4g}", end="")
+        assert m[0] < m[1] < m[2] < m[3]
+
+
 def test_table1_mse_on_gaussian(orc):
     """The MSE column of the IF4 page's Table 1 (tests/golden/if4_table1_mse.txt):
     NVFP4, 4/6, IF4 and MXFP4 on 2^20 standard normal values, each within 2% of
