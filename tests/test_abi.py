@@ -154,3 +154,19 @@ def test_binding_refuses_cpu_tensors(N):
     import torch
     with pytest.raises(ValueError):
         N.quantize(torch.zeros(16, 16, dtype=torch.bfloat16))
+
+
+def test_mode_numbers_agree_everywhere(N):
+    """The nvfp4_mode values of include/nvfp4.h are the binding's, the
+    workloads module's and the oracle's (each side defines them itself)."""
+    import oracle
+    from nvfp4_microscaling_quantization_b200 import workloads as W
+    text = open(HEADER).read()
+    enum = dict((name, int(v)) for name, v in re.findall(r"NVFP4_([A-Z0-9_]+) = (\d+)", text))
+    names = {"RTN": "RTN", "SR": "SR", "MS_EDEN": "MS_EDEN", "IF4": "IF4", "4OVER6": "FOUR_OVER_SIX",
+             "SCALE_SEARCH": "SCALE_SEARCH", "MXFP4": "MXFP4", "NVINT4": "NVINT4", "NVFP3": "NVFP3",
+             "NVINT3": "NVINT3", "IF3": "IF3", "MXFP3": "MXFP3"}
+    for c_name, py_name in names.items():
+        v = enum[c_name]
+        assert getattr(N, py_name) == v and getattr(W, py_name) == v and getattr(oracle, py_name) == v, c_name
+    assert set(W.MODE_NAMES) == set(enum[c] for c in names)
