@@ -19,6 +19,12 @@
  *  - IF4: per 16-element block, the lower-error of FP4 and scaled INT4 under
  *    the same E4M3 scale, flagged in the scale's sign bit.  IF4 paper page
  *    (arXiv 2603.28765), abstract, Figure 1, Table 1, Figure 3.
+ *  - The other block-scaled formats of that page (Table 1: MXFP4, NVINT4;
+ *    the 3-bit table: NVFP3, NVINT3, IF3, MXFP3) and scale search (the
+ *    palettes post's low-error corner, the page's ScaleSearch entry): see
+ *    nvfp4_mode.
+ *  - nvfp4_gemm multiplies two quantized operands on the block-scaled tensor
+ *    cores (Quartet II abstract: NVFP4 in Blackwell hardware).
  *
  * Conventions shared by every entry point:
  *  - Pointers are DEVICE pointers unless stated otherwise.  The library
@@ -38,10 +44,12 @@
  *  - codes: vrows x vcols/2 bytes; byte k of a row holds element 2k in its
  *    low nibble and element 2k+1 in its high nibble.  An E2M1 code is sign
  *    (bit 3) and a magnitude index (bits 0..2) into {0,.5,1,1.5,2,3,4,6}; an
- *    INT4 code (IF4 blocks flagged INT4) is sign (bit 3) and |k| (bits 0..2),
- *    value k * 6/7.  Zero is always code 0.
- *  - scales: vrows x vcols/16 bytes, E4M3 (bias 7, max 448, min 2^-9); for
- *    IF4, bit 7 set means the block holds INT4 codes.
+ *    INT4 code (IF4 blocks flagged INT4, NVINT4) is sign (bit 3) and |k|
+ *    (bits 0..2), value k * 6/7 (IF4) or k (NVINT4); the 3-bit codes use
+ *    bits 0..1 for the magnitude.  Zero is always code 0.
+ *  - scales: vrows x vcols/16 bytes, E4M3 (bias 7, max 448, min 2^-9), or
+ *    UE8M0 for MXFP4 / MXFP3 (the 32-element group's byte in both halves);
+ *    for IF4 and IF3, bit 7 set means the block holds integer codes.
  *  - global_scale: one float s_g; an element decodes to
  *    value(code) * RN(E4M3(scale & 0x7F) * s_g).
  *  - rht_group g in {0 (no rotation), 16, 32, 64, 128}: the random Hadamard
