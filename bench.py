@@ -14,9 +14,12 @@ ABI, each tensor's two tensor amaxes first, from one read of the tensor
 Prints one JSON line (rank 0).  value = algorithmic bytes (2 B read + 0.5 B
 codes + 0.0625 B scales per element of every call) / device time, all ranks
 summed (weak scaling: each rank quantizes its own step's tensors, no data-path
-collective).  L2 is flushed (a 256 MiB write) before every timed step, outside
-the timed region.  --impl reference times the CPU oracle on a bounded sample
-of the same workload.
+collective).  The K timed steps are captured once as a CUDA graph of the
+C-ABI launches and replayed once, with CUDA events between the launches, so
+host enqueue time stays out of the device timeline; L2 is flushed (a 256 MiB
+write) before every timed step, outside the marks.  --impl reference times the
+CPU oracle, run over ranges of view rows on every host core, on a bounded
+sample of the same workload.
 """
 import argparse
 import datetime
@@ -28,6 +31,8 @@ import subprocess
 import sys
 import tempfile
 import time
+
+import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -44,10 +49,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
 
 # DRAM bytes per launch measured by ncu for the dominant kernel, keyed by the
-# hash of the kernel sources they were taken with (see profiles/).  A changed
-# kernel reports traffic = null until it is captured again.
+# hash of the kernel sources they were taken with.  A changed kernel reports
+# traffic = null until it is captured again.
 NCU_TRAFFIC = {
-    # profiles/rotate_mma_eden_dy.md: dram__bytes_read.sum + dram__bytes_write.sum, one launch
+    # the ncu capture of the dominant kernel: dram__bytes_read.sum + dram__bytes_write.sum, one launch
     ("99074ee665c907e2", "dy.transposed.ms_eden.g128"): 470025472 + 108604928,
     ("99074ee665c907e2", "dy.rowwise.ms_eden.g128"): 469999616 + 110624256,
 }
@@ -68,6 +73,10 @@ def parse_args(argv=None):
                    help="skip the NVFP4 GEMMs of the step (measured after the quantization step)")
     p.add_argument("--no-per-mode", action="store_true",
                    help="skip the per-mode table (every mode on dY, quantize kernel alone)")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the other workloads' calls (256x256, weight, gradient, activation)")
+    p.add_argument("--no-eager", action="store_true",
+                   help="skip the eager (host-launched) run reported beside the graph-timed value")
     return p.parse_args(argv)
 
 
@@ -260,11 +269,77 @@ class TensorCalls:
         return (1 if self.dual else len(self.calls)) + len(self.calls)
 
 
-def per_mode_table(N, W, x, seed, stream, device, flush, peak, reps=5):
+def dist_us(seconds):
+    """mean, median, p10 and p90 of a list of durations, in microseconds."""
+    a = np.asarray(seconds, dtype=np.float64) * 1e6
+    return {"mean": round(float(a.mean()), 2), "median": round(float(np.median(a)), 2),
+            "p10": round(float(np.percentile(a, 10)), 2), "p90": round(float(np.percentile(a, 90)), 2)}
+
+
+class GraphTimer:
+    """Times launch sequences inside one CUDA graph.
+
+    Each of `reps` repetitions is: an L2 flush (a write of L2_FLUSH_BYTES,
+    outside the marks), then the callables of `body` with a CUDA event
+    recorded before the first, between each two and after the last.  The
+    repetitions are captured once on `stream` (the callables launch on it
+    through the C ABI) and the graph is replayed once, so the host takes no
+    part while the marks are being recorded: the device runs every launch
+    back to back.  durations()[r][i] is callable i of repetition r, seconds."""
+
+    def __init__(self, stream, body, reps, flush):
+        self.stream, self.body, self.reps, self.flush = stream, body, reps, flush
+        mk = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
+        self.ev = [[mk() for _ in range(len(body) + 1)] for _ in range(reps)]
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=stream, capture_error_mode="thread_local"):
+            for r in range(reps):
+                if flush is not None:
+                    flush.zero_()
+                self.ev[r][0].record()
+                for i, fn in enumerate(body):
+                    fn()
+                    self.ev[r][i + 1].record()
+
+    def replay(self):
+        self.graph.replay()
+
+    def durations(self):
+        return [[self.ev[r][i].elapsed_time(self.ev[r][i + 1]) / 1e3 for i in range(len(self.body))]
+                for r in range(self.reps)]
+
+    def totals(self):
+        return [self.ev[r][0].elapsed_time(self.ev[r][-1]) / 1e3 for r in range(self.reps)]
+
+    def release(self):
+        self.graph.reset()
+        self.graph = None
+
+
+def timed_in_graph(stream, body, reps, flush, device):
+    """Capture, replay once, and return (per-callable durations, per-rep totals)."""
+    t = GraphTimer(stream, body, reps, flush)
+    torch.cuda.synchronize(device)
+    t.replay()
+    torch.cuda.synchronize(device)
+    out = t.durations(), t.totals()
+    t.release()
+    return out
+
+
+def call_line(name, elements, secs, peak):
+    d = dist_us(secs)
+    t = d["mean"] / 1e6
+    gbs = BYTES_PER_ELEMENT * elements / t / 1e9
+    return {"call": name, "elements": elements, "us": d, "gbs": round(gbs, 1), "gelem_s": round(elements / t / 1e9, 1),
+            "frac_of_hbm_peak": round(gbs / peak, 4)}
+
+
+def per_mode_table(N, W, x, seed, stream, sh, device, flush, peak, reps=5):
     """Every mode on one tensor (the headline gradient dY), both layouts, with
     and without the 128-point rotation: the quantize kernel alone with the
-    tensor amax supplied (from its own pre-pass), CUDA events, L2 flushed
-    before each launch.  MS-EDEN is defined with the rotation only."""
+    tensor amax supplied (from its own pre-pass), L2 flushed before each
+    launch, timed inside a CUDA graph.  MS-EDEN is defined with the rotation only."""
     from nvfp4_microscaling_quantization_b200.workloads import Call as WCall
     out = []
     for layout in (W.ROWWISE, W.TRANSPOSED):
@@ -273,24 +348,43 @@ def per_mode_table(N, W, x, seed, stream, device, flush, peak, reps=5):
             for g in (0, 128):
                 if mode == W.MS_EDEN and g == 0:
                     continue
-                c = Call(N, WCall("dy", layout, mode, g), x, seed, stream)
-                c.amax_pass()
-                c.quantize()
-                ts = []
-                for _ in range(reps):
-                    flush.zero_()
-                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    a.record()
+                c = Call(N, WCall("dy", layout, mode, g), x, seed, sh)
+                with torch.cuda.stream(stream):
+                    c.amax_pass()
                     c.quantize()
-                    b.record()
-                    b.synchronize()
-                    ts.append(a.elapsed_time(b) / 1e3)
-                t = statistics.median(ts)
-                gbs = BYTES_PER_ELEMENT * c.elements / t / 1e9
-                out.append({"call": c.call.name, "us": round(t * 1e6, 1), "gbs": round(gbs, 1),
-                            "frac_of_hbm_peak": round(gbs / peak, 4), "gelem_s": round(c.elements / t / 1e9, 1)})
+                durs, _ = timed_in_graph(stream, [c.quantize], reps, flush, device)
+                out.append(call_line(c.call.name, c.elements, [d[0] for d in durs], peak))
                 del c
     torch.cuda.synchronize(device)
+    return out
+
+
+def workload_table(N, W, stream, sh, device, flush, peak, reps=10):
+    """The other configurations' calls, each on its own tensor: the quantize
+    kernel with the tensor amax supplied (`quantize`), and the two-pass path
+    that computes the amax first (`two_pass`: pre-pass + quantize).  L2 is
+    flushed before each repetition; CUDA graph timing."""
+    out = []
+    for make in (W.small, W.weight, W.gradient, W.activation):
+        wl = make()
+        tensors = wl.tensors(device)
+        lines = []
+        for wc in wl.calls:
+            c = Call(N, wc, tensors[wc.tensor], wl.seed, sh)
+            with torch.cuda.stream(stream):
+                c.amax_pass()
+                c.quantize()
+            durs, _ = timed_in_graph(stream, [c.amax_pass, c.quantize], reps, flush, device)
+            q = call_line(wc.name, c.elements, [d[1] for d in durs], peak)
+            two = call_line(wc.name, c.elements, [d[0] + d[1] for d in durs], peak)
+            lines.append({"call": wc.name, "elements": c.elements,
+                          "quantize": {k: q[k] for k in ("us", "gbs", "gelem_s", "frac_of_hbm_peak")},
+                          "two_pass": {k: two[k] for k in ("us", "gbs", "gelem_s", "frac_of_hbm_peak")}})
+            del c
+        out.append({"workload": wl.name, "description": wl.description,
+                    "shapes": {k: list(v) for k, v in wl.shapes.items()}, "seed": wl.seed, "calls": lines})
+        del tensors
+        torch.cuda.synchronize(device)
     return out
 
 
@@ -298,8 +392,9 @@ def gemm_table(N, calls, stream, device, reps=10):
     """The three GEMMs of the linear layer's training step on the step's own
     quantized outputs (nvfp4_gemm, bf16 D): Y = X W^T (RTN X and W row-wise),
     dX = dY W (MS-EDEN dY row-wise, W transposed), dW = dY^T X (MS-EDEN dY and
-    X transposed).  CUDA events over each launch after warm-up; the fp4 dense
-    tensor peak is the measured bf16 peak x 4 (nominal 9 / 2.25 PF)."""
+    X transposed).  Timed inside a CUDA graph (no L2 flush: the operands are
+    re-read from L2 within a launch anyway); the fp4 dense tensor peak is the
+    measured bf16 peak x 4 (nominal 9 / 2.25 PF)."""
     by = {c.call.name: c for c in calls}
     q = lambda name: (by[name].codes, by[name].scales, by[name].gscale)  # noqa: E731
     cases = [("Y = X W^T", "x.rowwise.rtn.norht", "w.rowwise.rtn.norht"),
@@ -312,20 +407,14 @@ def gemm_table(N, calls, stream, device, reps=10):
         a, b = q(an), q(bn)
         m, k, n = a[0].shape[0], 2 * a[0].shape[1], b[0].shape[0]
         d = torch.empty(m, n, dtype=torch.bfloat16, device=device)
-        for _ in range(3):
-            N.gemm(a, b, out=d)
-        ts = []
-        for _ in range(reps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            N.gemm(a, b, out=d)
-            e1.record(stream)
-            e1.synchronize()
-            ts.append(e0.elapsed_time(e1) / 1e3)
-        t = statistics.median(ts)
-        tf = 2.0 * m * n * k / t / 1e12
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                N.gemm(a, b, out=d)
+        durs, _ = timed_in_graph(stream, [lambda: N.gemm(a, b, out=d)], reps, None, device)
+        ts = dist_us([x[0] for x in durs])
+        tf = 2.0 * m * n * k / (ts["mean"] / 1e6) / 1e12
         out.append({"gemm": name, "a": an, "b": bn, "m": m, "n": n, "k": k, "out": "bf16",
-                    "us": round(t * 1e6, 1), "tflops": round(tf, 1),
+                    "us": ts, "tflops": round(tf, 1),
                     "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(peak, 1),
                                  "peak_kind": f"fp4 dense = 4 x {kind} bf16", "unit": "TFLOP/s",
                                  "frac": round(tf / peak, 4)}})
@@ -345,7 +434,7 @@ def run_ours(args, world, rank, local):
     N.lib()
     wl = W.mlp_up(seed=4 + 1000 * rank)
     tensors = wl.tensors(device)
-    stream = torch.cuda.current_stream(device)
+    stream = torch.cuda.Stream(device)
     sh = ctypes.c_void_p(stream.cuda_stream)
     calls = [Call(N, c, tensors[c.tensor], wl.seed, sh) for c in wl.calls]
     groups = [TensorCalls(N, [c for c in calls if c.call.tensor == name])
@@ -353,80 +442,90 @@ def run_ours(args, world, rank, local):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     bytes_per_step = sum(BYTES_PER_ELEMENT * c.elements for c in calls)
     elems_per_step = sum(c.elements for c in calls)
+    # one step = per tensor its pre-pass, then its quantize calls: 9 launches
+    body, body_names = [], []
+    for grp in groups:
+        body.append(grp.amax_passes)
+        body_names.append(("amax", grp))
+        for c in grp.calls:
+            body.append(c.quantize)
+            body_names.append(("quant", c))
 
-    # per step: for each tensor its pre-pass(es), then its quantize calls;
-    # events: [pre-pass start, pre-pass end] per tensor, [start, end] per call
-    def step(evs=None):
-        for gi, grp in enumerate(groups):
-            if evs is not None:
-                evs["amax"][gi][0].record(stream)
-            grp.amax_passes()
-            if evs is not None:
-                evs["amax"][gi][1].record(stream)
-            for c in grp.calls:
-                i = calls.index(c)
-                if evs is not None:
-                    evs["quant"][i][0].record(stream)
-                c.quantize()
-                if evs is not None:
-                    evs["quant"][i][1].record(stream)
+    def step():
+        for fn in body:
+            fn()
 
-    for _ in range(max(args.warmup, 0)):
-        flush.zero_()
-        step()
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 0)):
+            flush.zero_()
+            step()
     torch.cuda.synchronize(device)
-
     K = args.steps
-    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    starts, ends = [ev() for _ in range(K)], [ev() for _ in range(K)]
-    call_evs = [{"amax": [[ev(), ev()] for _ in groups], "quant": [[ev(), ev()] for _ in calls]}
-                for _ in range(K)]
+
+    # eager reference run (host enqueues every launch; reported, not the value)
+    eager = None
+    if not args.no_eager:
+        ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        marks = [[ev() for _ in range(len(body) + 1)] for _ in range(K)]
+        with torch.cuda.stream(stream):
+            for k in range(K):
+                flush.zero_()
+                marks[k][0].record()
+                for i, fn in enumerate(body):
+                    fn()
+                    marks[k][i + 1].record()
+        torch.cuda.synchronize(device)
+        e_steps = [marks[k][0].elapsed_time(marks[k][-1]) / 1e3 for k in range(K)]
+        e_calls = [[marks[k][i].elapsed_time(marks[k][i + 1]) / 1e3 for k in range(K)] for i in range(len(body))]
+
+    # the timed region: the K steps as one CUDA graph of the same C-ABI launches
+    timer = GraphTimer(stream, body, K, flush)
     with ClockSampler(local) as clocks:
         barrier(world, local)
         torch.cuda.synchronize(device)
-        for k in range(K):
-            flush.zero_()                    # L2 flush, outside the timed region
-            starts[k].record(stream)
-            step(call_evs[k])
-            ends[k].record(stream)
+        timer.replay()
         torch.cuda.synchronize(device)
         barrier(world, local)
     clock = clocks.summary()
+    durs, totals = timer.durations(), timer.totals()
+    timer.release()
 
-    step_ms = [starts[k].elapsed_time(ends[k]) for k in range(K)]
-    total_s = max_over_ranks(sum(step_ms) / 1e3, world, device)
-    amax_ms = [statistics.mean(call_evs[k]["amax"][g][0].elapsed_time(call_evs[k]["amax"][g][1]) for k in range(K))
-               for g in range(len(groups))]
-    quant_ms = [statistics.mean(call_evs[k]["quant"][i][0].elapsed_time(call_evs[k]["quant"][i][1])
-                                for k in range(K)) for i in range(len(calls))]
-    quant_total_s = max_over_ranks(sum(quant_ms) * K / 1e3, world, device)
+    total_s = max_over_ranks(sum(totals), world, device)
+    per_fn = [[durs[k][i] for k in range(K)] for i in range(len(body))]
+    quant_idx = [i for i, (kind, _) in enumerate(body_names) if kind == "quant"]
+    quant_total_s = max_over_ranks(sum(sum(per_fn[i]) for i in quant_idx), world, device)
     value = weak_scaling_value(bytes_per_step, K, world, total_s)
     value_supplied = weak_scaling_value(bytes_per_step, K, world, quant_total_s)
     peak, peak_kind = hbm_peak()
 
-    # dominant kernel: the quantize kernel with the largest share of the step
-    dom = max(range(len(calls)), key=lambda i: quant_ms[i])
-    dom_bytes = BYTES_PER_ELEMENT * calls[dom].elements
-    achieved = dom_bytes / (quant_ms[dom] / 1e3) / 1e9
+    # dominant kernel: the quantize launch with the largest mean duration in the step
+    dom_i = max(quant_idx, key=lambda i: statistics.mean(per_fn[i]))
+    dom = body_names[dom_i][1]
+    dom_stats = dist_us(per_fn[dom_i])
+    dom_bytes = BYTES_PER_ELEMENT * dom.elements
+    achieved = dom_bytes / (dom_stats["mean"] / 1e6) / 1e9
     src_hash = kernel_source_hash()
-    traffic = NCU_TRAFFIC.get((src_hash, calls[dom].call.name))
+    traffic = NCU_TRAFFIC.get((src_hash, dom.call.name))
 
-    per_call = []
-    for i, c in enumerate(calls):
-        per_call.append({
-            "call": c.call.name, "elements": c.elements,
-            "quantize_us": round(quant_ms[i] * 1e3, 2),
-            "quantize_gbs": round(BYTES_PER_ELEMENT * c.elements / (quant_ms[i] / 1e3) / 1e9, 1),
-            "quantize_gelem_s": round(c.elements / (quant_ms[i] / 1e3) / 1e9, 1),
-        })
-    pre_passes = []
-    for g, grp in enumerate(groups):
-        read = PREPASS_BYTES_PER_ELEMENT * grp.calls[0].elements
-        pre_passes.append({
-            "tensor": grp.calls[0].call.tensor, "kind": "dual" if grp.dual else "single",
-            "for_calls": [c.call.name for c in grp.calls], "us": round(amax_ms[g] * 1e3, 2),
-            "read_gbs": round(read / (amax_ms[g] / 1e3) / 1e9, 1),
-        })
+    per_call, pre_passes = [], []
+    for i, (kind, obj) in enumerate(body_names):
+        d = dist_us(per_fn[i])
+        t = d["mean"] / 1e6
+        if kind == "quant":
+            per_call.append({"call": obj.call.name, "elements": obj.elements, "us": d,
+                             "gbs": round(BYTES_PER_ELEMENT * obj.elements / t / 1e9, 1),
+                             "gelem_s": round(obj.elements / t / 1e9, 1),
+                             "frac_of_hbm_peak": round(BYTES_PER_ELEMENT * obj.elements / t / 1e9 / peak, 4)})
+        else:
+            read = PREPASS_BYTES_PER_ELEMENT * obj.calls[0].elements
+            pre_passes.append({"tensor": obj.calls[0].call.tensor, "kind": "dual" if obj.dual else "single",
+                               "for_calls": [c.call.name for c in obj.calls], "us": d,
+                               "read_gbs": round(read / t / 1e9, 1)})
+    if not args.no_eager:
+        eager = {"note": "the same K steps launched eagerly from Python (host enqueue in the device timeline); "
+                         "not the value",
+                 "ms_per_step": dist_us(e_steps), "dominant_launch_us": dist_us(e_calls[dom_i])}
+        eager["ms_per_step"] = {k: round(v / 1e3, 4) for k, v in eager["ms_per_step"].items()}
 
     gemms = None
     if not args.no_gemm:
@@ -434,7 +533,11 @@ def run_ours(args, world, rank, local):
 
     per_mode = None
     if not args.no_per_mode:
-        per_mode = per_mode_table(N, W, tensors["dy"], wl.seed, sh, device, flush, peak)
+        per_mode = per_mode_table(N, W, tensors["dy"], wl.seed, stream, sh, device, flush, peak)
+
+    configs = None
+    if not args.no_configs:
+        configs = workload_table(N, W, stream, sh, device, flush, peak)
 
     e2e = None
     if not args.no_e2e:
@@ -445,6 +548,7 @@ def run_ours(args, world, rank, local):
         host = {k: v.cpu() for k, v in tensors.items()}
         cpu = cpu_baseline(wl, host, args.cpu_sample_fraction)
 
+    step_stats = {k: round(v / 1e3, 4) for k, v in dist_us(totals).items()}
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(total_s * 1e3 / K, 4), "higher_is_better": True,
@@ -455,27 +559,35 @@ def run_ours(args, world, rank, local):
             "calls": [c.call.name for c in calls],
             "path": "per tensor: one tensor-amax pre-pass for both layouts (nvfp4_amax_dual), then its "
                     "quantize kernels (C ABI), one stream",
-            "input_dtype": "bf16", "l2": "flushed before every timed step (256 MiB write, untimed)",
+            "timing": "the K steps captured once as one CUDA graph of the C-ABI launches and replayed once; "
+                      "CUDA events (graph event nodes) before, between and after the launches of each step",
+            "input_dtype": "bf16", "l2": "flushed before every timed step (256 MiB write, outside the marks)",
             "parallelism": f"replicas x{world} (independent tensors per rank)",
         },
         "gelem_per_s": round(elems_per_step * K * world / total_s / 1e9, 1),
         "frac_of_hbm_peak": round(value / world / peak, 4),
+        "step_ms": step_stats,
         "value_amax_supplied": round(value_supplied, 1),
         "frac_of_hbm_peak_amax_supplied": round(value_supplied / world / peak, 4),
-        "roofline": {"bound": "hbm", "kernel": f"quantize {calls[dom].call.name}",
+        "roofline": {"bound": "hbm", "kernel": f"quantize {dom.call.name}",
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "algorithmic_bytes": int(dom_bytes), "avg_launch_us": round(quant_ms[dom] * 1e3, 2)},
+                     "algorithmic_bytes": int(dom_bytes), "avg_launch_us": dom_stats["mean"],
+                     "launch_us": dom_stats},
         "per_call": per_call,
         "amax_pre_passes": pre_passes,
         "gpu_launches": sum(g.launches() for g in groups) * K,
         "clocks": clock,
         "kernel_source": src_hash,
     }
+    if eager is not None:
+        result["eager"] = eager
     if gemms is not None:
         result["nvfp4_gemm"] = gemms
     if per_mode is not None:
         result["per_mode_dy"] = per_mode
+    if configs is not None:
+        result["configs"] = configs
     if e2e is not None:
         result["e2e"] = e2e
     if cpu is not None:
@@ -571,53 +683,63 @@ def _sample_calls(wl, host, fraction):
     return out
 
 
-def time_oracle_sample(wl, samples):
-    import oracle
+def time_oracle_sample(wl, samples, pool):
+    """The oracle on every sampled call: its amax pre-pass, then the quantization,
+    each split over the pool's worker processes by view rows."""
     elements = 0
     t0 = time.perf_counter()
     for c, xb in samples:
-        a = oracle.amax(xb, c.layout, c.rht_group, wl.seed)
-        oracle.quantize(xb, c.layout, c.mode, c.rht_group, wl.seed, amax_in=a)
+        a = pool.amax(xb, c.layout, c.rht_group, wl.seed)
+        pool.quantize(xb, c.layout, c.mode, c.rht_group, wl.seed, a)
         elements += xb.size
     return elements, time.perf_counter() - t0
 
 
 def cpu_baseline(wl, host, fraction):
+    from oracle.pool import OraclePool
     samples = _sample_calls(wl, host, fraction)
-    elements, secs = time_oracle_sample(wl, samples)
-    return {"value": round(BYTES_PER_ELEMENT * elements / secs / 1e9, 4), "unit": UNIT, "cores": 1,
+    with OraclePool() as pool:
+        elements, secs = time_oracle_sample(wl, samples, pool)
+        cores = pool.workers
+    return {"value": round(BYTES_PER_ELEMENT * elements / secs / 1e9, 4), "unit": UNIT, "cores": cores,
             "kind": "oracle",
-            "sample": f"first {fraction:.4g} of the view rows of each of the 6 calls "
-                      f"({elements} elements, amax pre-pass + quantize, single-threaded C), {secs:.1f} s"}
+            "sample": f"first {fraction:.4g} of the view rows of each of the {len(samples)} calls "
+                      f"({elements} elements, amax pre-pass + quantize), the single-threaded C oracle run on "
+                      f"ranges of view rows in {cores} processes (one per host core), {secs:.1f} s"}
 
 
-def run_reference(args, world, rank, wl=None, fraction=1.0 / 128):
+def run_reference(args, world, rank, wl=None, fraction=1.0 / 64):
     """The CPU oracle as the reference arm, on rank 0 only (the other ranks return at once)."""
     if rank != 0:
         return None
+    from oracle.pool import OraclePool
     from nvfp4_microscaling_quantization_b200 import workloads as W
     wl = W.mlp_up(seed=4) if wl is None else wl
-    device = "cuda" if torch.cuda.is_available() else "cpu"
-    full = wl.tensors(device)
-    host = {k: v.cpu() for k, v in full.items()}
-    del full
-    samples = _sample_calls(wl, host, fraction)
-    for _ in range(max(args.warmup, 0)):
-        time_oracle_sample(wl, samples)
-    total_e, total_s = 0, 0.0
-    for _ in range(args.steps):
-        e, s = time_oracle_sample(wl, samples)
-        total_e += e
-        total_s += s
+    # the worker processes start (spawn) before this process touches a GPU
+    with OraclePool() as pool:
+        device = "cuda" if torch.cuda.is_available() else "cpu"
+        full = wl.tensors(device)
+        host = {k: v.cpu() for k, v in full.items()}
+        del full
+        samples = _sample_calls(wl, host, fraction)
+        for _ in range(max(args.warmup, 0)):
+            time_oracle_sample(wl, samples, pool)
+        total_e, total_s = 0, 0.0
+        for _ in range(args.steps):
+            e, s = time_oracle_sample(wl, samples, pool)
+            total_e += e
+            total_s += s
+        cores = pool.workers
     value = BYTES_PER_ELEMENT * total_e / total_s / 1e9
     sample = (f"each step: first {fraction:.4g} of the view rows of each of the {wl.name} calls "
-              f"({total_e // max(args.steps, 1)} elements, amax pre-pass + quantize)")
+              f"({total_e // max(args.steps, 1)} elements, amax pre-pass + quantize), the single-threaded C "
+              f"oracle on ranges of view rows in {cores} processes")
     line = json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_s * 1e3 / max(args.steps, 1), 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": f"{wl.name} (bounded sample per step)", "input_dtype": "bf16"},
-        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     })
     print(line, flush=True)

@@ -236,8 +236,11 @@ NVFP4_API int nvfp4_rht(const void* in, int in_dtype, int64_t rows, int64_t cols
  * fixed 256-byte array of device memory compiled into the library (every GPU
  * that loads the library keeps those bytes until the process exits).  It
  * allocates nothing and calls no allocating routine.
- *  - The first call on a device looks up that array's device address (with
- *    the device current); make that first call before any stream capture.
+ *  - The first call in a CUDA context looks up that array's device address
+ *    (with the device current) and keeps it for that context; make that
+ *    first call before any stream capture.  A context created again on the
+ *    same device (after cudaDeviceReset) gets a fresh lookup, never the old
+ *    address.
  *  - All calls on a device share the one array.  Each call clears the part
  *    that must start at zero on its own stream, but two calls that overlap
  *    on the GPU (different streams, or different host threads) race on it

@@ -43,6 +43,7 @@
 #include <cstdint>
 
 #include "kernels.h"
+#include "launch_config.h"
 #include "tcgen05.cuh"
 #include "tma_pipeline.cuh"
 
@@ -353,11 +354,10 @@ cudaError_t launch_gemm_t(const GemmArgs& g) {
       !make_scales_map(&msa, g.a_scales, g.m, g.k) || !make_scales_map(&msb, g.b_scales, g.n, g.k))
     return cudaErrorInvalidValue;
   auto kernel = nvfp4_gemm_kernel<OUT_BF16>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kGDynSmem));
+  LaunchGeom geom;
+  const cudaError_t e = launch_geometry(kernel, kGThreads, kGDynSmem, 1, &geom);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = geom.sms;
   const int64_t n_tiles = (g.m / kGBM) * (g.n / kGBN);
   const int64_t grid = n_tiles < sms ? n_tiles : sms;
   if (grid == 0) return cudaSuccess;

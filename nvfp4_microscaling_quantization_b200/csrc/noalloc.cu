@@ -10,10 +10,12 @@
 // fixed-size array of device memory that is part of the library image itself,
 // so nothing is allocated at call time.
 #include <cstdint>
+#include <map>
 #include <mutex>
 
 #include <cuda_runtime.h>
 
+#include "launch_config.h"
 #include "nvfp4.h"
 
 namespace {
@@ -23,24 +25,35 @@ namespace {
 constexpr size_t kScratchBytes = 256;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::once_flag g_setup_once[kMaxDevices];
-void* g_scratch_address[kMaxDevices];
-cudaError_t g_setup_status[kMaxDevices];
-
 // In host code g_noalloc_scratch names a host-side stand-in, not device
-// memory; the device address is looked up once per device, with that device
-// current.
+// memory.  The device address is looked up with the device current, once per
+// CUDA context (the first call in a context does it) and kept for later calls
+// in that context.  The key is the context's process-unique id, so a context
+// created again on the same device (after cudaDeviceReset) looks the address
+// up again instead of reusing a stale one; a failed lookup is not kept.
 int scratch_for_current_device(void** out) {
+  static std::mutex mu;
+  static std::map<uint64_t, void*> by_context;
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
-  std::call_once(g_setup_once[dev], [dev] {
-    void* p = nullptr;
-    g_setup_status[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    g_scratch_address[dev] = p;
-  });
-  if (g_setup_status[dev] != cudaSuccess || g_scratch_address[dev] == nullptr) return NVFP4_ERR_CUDA;
-  *out = g_scratch_address[dev];
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return NVFP4_ERR_CUDA;
+  uint64_t ctx = nvfp4::current_context_id();
+  if (ctx != 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = by_context.find(ctx);
+    if (it != by_context.end()) {
+      *out = it->second;
+      return NVFP4_OK;
+    }
+  }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return NVFP4_ERR_CUDA;
+  // the lookup made the device's context current if it was not yet
+  if (ctx == 0) ctx = nvfp4::current_context_id();
+  if (ctx != 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    by_context[ctx] = p;
+  }
+  *out = p;
   return NVFP4_OK;
 }
 

@@ -383,13 +383,10 @@ cudaError_t launch_tma_one(const QuantArgs& a) {
     return cudaErrorInvalidValue;
   auto kernel = quantize_tma_kernel<MODE, G, AMAX_ONLY, ROWWISE>;
   const size_t smem = kStages * kStageBytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  LaunchGeom geom;
+  const cudaError_t e = launch_geometry(kernel, kNT, smem, 32, &geom);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148, per_sm = 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  e = resident_ctas(kernel, kNT, smem, 32, &per_sm);
-  if (e != cudaSuccess) return e;
+  const int sms = geom.sms, per_sm = geom.per_sm;
   const int64_t n_ct = ROWWISE ? (a.cols + kRowTileCols - 1) / kRowTileCols : (a.cols + kColTileCols - 1) / kColTileCols;
   const int64_t n_tiles = ROWWISE ? ((a.rows + kRowBoxRows - 1) / kRowBoxRows) * n_ct
                                   : ((a.rows + kColTileRows - 1) / kColTileRows) * n_ct;

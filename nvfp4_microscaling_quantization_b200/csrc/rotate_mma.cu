@@ -708,15 +708,12 @@ cudaError_t launch_one(const QuantArgs& a, float* zout) {
   CUtensorMap map;
   if (!make_map(&map, a.x, a.rows, a.cols, a.ld)) return cudaErrorInvalidValue;
   auto kernel = rotate_mma_kernel<MODE, G, KIND, ROWWISE>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDynSmem));
-  if (e != cudaSuccess) return e;
   // one CTA per SM: it allocates all of tensor memory
   constexpr int threads = Shape<MODE, KIND>::threads;
-  int dev = 0, sms = 148, per_sm = 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  e = resident_ctas(kernel, threads, kDynSmem, 1, &per_sm);
+  LaunchGeom geom;
+  cudaError_t e = launch_geometry(kernel, threads, kDynSmem, 1, &geom);
   if (e != cudaSuccess) return e;
+  const int sms = geom.sms, per_sm = geom.per_sm;
   const int64_t n_tiles = ((a.rows + kTile - 1) / kTile) * ((a.cols + kTile - 1) / kTile);
   int64_t grid = n_tiles < int64_t(sms) * per_sm ? n_tiles : int64_t(sms) * per_sm;
   if (grid == 0) {
@@ -784,14 +781,10 @@ cudaError_t launch_amax_dual_mma(const void* x, int64_t rows, int64_t cols, int6
                                  uint64_t seed, float* amax_r, float* amax_c, cudaStream_t stream) {
   CUtensorMap map;
   if (!make_map(&map, x, rows, cols, ld)) return cudaErrorInvalidValue;
-  cudaError_t e =
-      cudaFuncSetAttribute(dual_amax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDualDynSmem));
+  LaunchGeom geom;
+  cudaError_t e = launch_geometry(dual_amax_kernel, kDualThreads, kDualDynSmem, 1, &geom);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148, per_sm = 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  e = resident_ctas(dual_amax_kernel, kDualThreads, kDualDynSmem, 1, &per_sm);
-  if (e != cudaSuccess) return e;
+  const int sms = geom.sms;
   const int64_t n_tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
   const int64_t grid = n_tiles < int64_t(sms) ? n_tiles : int64_t(sms);
   if (grid == 0) return cudaSuccess;
