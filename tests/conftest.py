@@ -23,7 +23,13 @@ def orc():
 def pytest_terminal_summary(terminalreporter):
     """Report the end-to-end differences of the rotated modes against the oracle."""
     helpers = sys.modules.get("gpu_helpers")
-    if helpers is None or not helpers.ROTATED_MISMATCH[1]:
+    if helpers is None:
+        return
+    if helpers.ROTATION_WORST[0]:
+        terminalreporter.write_line(
+            f"rotated values against the oracle: largest difference {helpers.ROTATION_WORST[0]:.1f} fp32 ulps of "
+            f"the group maximum; above the floor, {helpers.ROTATION_WORST[1]:.2e} of the value")
+    if not helpers.ROTATED_MISMATCH[1]:
         return
     cb, c, sb, s = helpers.ROTATED_MISMATCH
     terminalreporter.write_line(

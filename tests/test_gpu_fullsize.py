@@ -1,103 +1,119 @@
-"""GPU parity at the workloads' full sizes, in the launch configuration bench.py
-times (the same C-ABI call on the same shapes), on sampled output rows.  The
-tensors are drawn on the GPU and copied to the host for the oracle.
+"""GPU parity at the workloads' full sizes, whole tensors, in the launch
+configuration bench.py times (the same C-ABI calls on the same shapes).
 
-For each call the oracle computes the tensor amax over the whole tensor, then
-only the sampled view rows (the first, the last and randomly drawn ones).
+The tensors are drawn on the GPU and copied to the host; the oracle runs over
+ranges of view rows in worker processes (oracle/pool.py), which assembles
+exactly its single-process result.  For every call of the weight (4096x4096),
+gradient (8192x4096), activation (16384x8192) and MLP up-projection
+(X 16384x4096, W 14336x4096, dY 16384x14336) workloads, every output is
+compared:
 
-Without the rotation the GPU's rows must equal the oracle's bit for bit, and
-so must the FP32 tensor scale.  With the rotation the four-part comparison of
-gpu_helpers is applied to the sampled rows: the rotated values within the
-tolerance, the GPU pre-pass amax equal to max |z| of the GPU's own rotation
-(over the whole tensor) and within the tolerance of the oracle's, the sampled
-rows of the GPU's quantization bit-exact against the oracle quantizing the
-GPU's own rotated rows, and the end-to-end difference (both sides given the
-oracle's amax) confined to blocks with differing rotated values and at most
-1e-5 of the sampled outputs.
+without the rotation, the GPU's codes, scales and FP32 tensor scale equal the
+oracle's bit for bit (the GPU computes the tensor amax itself; it must equal
+the oracle's exactly);
+
+with the rotation, the four-part comparison of gpu_helpers over the whole
+view: every rotated value within the tolerance; the GPU pre-pass amax equal
+to max |z| of the GPU's own rotation and within the tolerance of the
+oracle's; the GPU's codes, scales and tensor scale bit-exact against the
+oracle quantizing the GPU's own rotated view; and end to end (both sides
+given the oracle's amax) every differing scale group explained by the
+rotation's rounding, at most 1e-5 of the codes and of the scales differing.
 """
-import zlib
-
 import numpy as np
 import pytest
 import torch
 
 import oracle
+from oracle.pool import OraclePool
 from nvfp4_microscaling_quantization_b200 import binding as N
 from nvfp4_microscaling_quantization_b200 import workloads as W
 
-from gpu_helpers import ROT_TOL, assert_same, bits, check_rotation, end_to_end_mismatch, record_mismatch
+from gpu_helpers import (MISMATCH_MAX, ROT_TOL, assert_same, bits, check_rotation, end_to_end_mismatch,
+                         record_mismatch)
 
 pytestmark = pytest.mark.gpu
 
-N_SAMPLED_ROWS = 12
+CHUNK_ROWS = 2048
 
 
-def _view_row_bits(xb, layout, r):
-    """bf16 patterns whose (single-row) view is view row r of the full tensor."""
-    return xb[r:r + 1] if layout == W.ROWWISE else np.ascontiguousarray(xb[:, r:r + 1])
+@pytest.fixture(scope="module")
+def pool():
+    with OraclePool() as p:
+        yield p
 
 
-def _check_call(wl, call, x, xb):
+def _host(t):
+    return t.cpu().numpy()
+
+
+def _check_call(pool, wl, call, x, xb):
     rows, cols = x.shape
     vr, vc = N.view_shape(rows, cols, call.layout)
     g, seed, mode, layout = call.rht_group, wl.seed, call.mode, call.layout
-    rng = np.random.default_rng(zlib.crc32(call.name.encode()))
-    sample = sorted(set([0, vr - 1] + list(rng.integers(0, vr, N_SAMPLED_ROWS - 2))))
-    a_orc = oracle.amax(xb, layout, g, seed)
+    name = call.name
+    mx = mode in (W.MXFP4, W.MXFP3)
+    a_orc = 0.0 if mx else pool.amax(xb, layout, g, seed)
 
     codes, scales, gs = N.quantize(x, layout, mode, g, seed)
     torch.cuda.synchronize()
-    codes_h, scales_h, gs_h = codes.cpu().numpy(), scales.cpu().numpy(), float(gs.item())
+    got = (_host(codes), _host(scales), float(gs.item()))
     del codes, scales, gs
 
     if g == 0:
-        assert gs_h == oracle.global_scale(a_orc, mode), call.name
-        for r in sample:
-            oc, osc, _ = oracle.quantize(xb, layout, mode, g, seed, amax_in=a_orc, row_range=(r, r + 1))
-            assert np.array_equal(codes_h[r], oc[r]), (call.name, r, int(np.sum(codes_h[r] != oc[r])))
-            assert np.array_equal(scales_h[r], osc[r]), (call.name, r, int(np.sum(scales_h[r] != osc[r])))
+        exp = pool.quantize(xb, layout, mode, g, seed, a_orc)
+        assert_same(got, exp, name)
         return
 
-    z = N.rht(x, layout, g, seed)
-    a_gpu = N.amax(x, layout, g, seed).item()
-    a_own = z.abs().max().item()
-    z_rows = z[sample].cpu().numpy()
-    del z
-    assert a_gpu == a_own, (call.name, a_gpu, a_own)
-    assert abs(a_gpu - a_orc) <= ROT_TOL * a_orc, (call.name, a_gpu, a_orc)
-    assert gs_h == oracle.global_scale(a_gpu, mode), call.name
+    z_dev = N.rht(x, layout, g, seed)
+    a_gpu = 0.0 if mx else N.amax(x, layout, g, seed).item()
+    a_own = z_dev.abs().max().item()
+    z_gpu = _host(z_dev)
+    del z_dev
+    if not mx:
+        assert a_gpu == a_own, (name, a_gpu, a_own)
+        assert abs(a_gpu - a_orc) <= ROT_TOL * a_orc, (name, a_gpu, a_orc)
+    z_orc = pool.rht_view(xb, layout, g, seed)
+    for r0 in range(0, vr, CHUNK_ROWS):
+        check_rotation(z_gpu[r0:r0 + CHUNK_ROWS], z_orc[r0:r0 + CHUNK_ROWS], g, f"{name} rows {r0}..")
 
+    # every step after the rotation, exactly, on the GPU's own rotated view
+    assert_same(got, pool.quantize_rotated(z_gpu, mode, seed, a_gpu), name + " (on the GPU's rotation)")
+
+    # end to end against the oracle from x, both sides given the oracle's amax
     amax_t = torch.tensor([a_orc], dtype=torch.float32, device="cuda")
-    codes_e, scales_e, gs_e = N.quantize(x, layout, mode, g, seed, amax_in=amax_t)
+    codes_e, scales_e, gs_e = N.quantize(x, layout, mode, g, seed, amax_in=None if mx else amax_t)
     torch.cuda.synchronize()
-    codes_e, scales_e, gs_e = codes_e.cpu().numpy(), scales_e.cpu().numpy(), float(gs_e.item())
+    gpu_e = (_host(codes_e), _host(scales_e), float(gs_e.item()))
+    del codes_e, scales_e, gs_e
+    orc_e = pool.quantize(xb, layout, mode, g, seed, a_orc)
+    n_codes, n_scales = vr * vc, vr * vc // 16
+    diff_codes = int((oracle.unpack_codes(gpu_e[0]) != oracle.unpack_codes(orc_e[0])).sum())
+    diff_scales = int((gpu_e[1] != orc_e[1]).sum())
+    assert diff_codes <= MISMATCH_MAX * n_codes and diff_scales <= MISMATCH_MAX * n_scales, \
+        (name, diff_codes, diff_scales)
+    nc = ns = 0
+    for r0 in range(0, vr, CHUNK_ROWS):
+        r1 = min(vr, r0 + CHUNK_ROWS)
+        c, s = end_to_end_mismatch((gpu_e[0][r0:r1], gpu_e[1][r0:r1], gpu_e[2]),
+                                   (orc_e[0][r0:r1], orc_e[1][r0:r1], orc_e[2]),
+                                   z_gpu[r0:r1], z_orc[r0:r1], f"{name} rows {r0}..", mode=mode, seed=seed, row0=r0)
+        nc += c
+        ns += s
+    record_mismatch(nc, n_codes, ns, n_scales, name)
+    print(f"{name}: whole view {vr}x{vc}: {nc} of {n_codes} codes and {ns} of {n_scales} scales differ end to end")
 
-    n_codes_bad = n_scales_bad = 0
-    for i, r in enumerate(sample):
-        what = f"{call.name} view row {r}"
-        zg = z_rows[i:i + 1]
-        zo = oracle.rht_view(_view_row_bits(xb, layout, r), layout, g, seed)
-        check_rotation(zg, zo, g, what)
-        oc, osc, og = oracle.quantize_rotated(zg, mode, seed, a_gpu, row0=r)
-        assert_same((codes_h[r:r + 1], scales_h[r:r + 1], gs_h), (oc, osc, og), what + " (on the GPU's rotation)")
-        oc, osc, og = oracle.quantize(xb, layout, mode, g, seed, amax_in=a_orc, row_range=(r, r + 1))
-        nc, ns = end_to_end_mismatch((codes_e[r:r + 1], scales_e[r:r + 1], gs_e),
-                                     (oc[r:r + 1], osc[r:r + 1], og), zg, zo, what)
-        n_codes_bad += nc
-        n_scales_bad += ns
-    record_mismatch(n_codes_bad, len(sample) * vc, n_scales_bad, len(sample) * vc // 16, call.name)
 
-
-def _check_workload(wl):
+def _check_workload(pool, wl):
     tensors = wl.tensors("cuda")
     host = {k: bits(v) for k, v in tensors.items()}
     for call in wl.calls:
-        _check_call(wl, call, tensors[call.tensor], host[call.tensor])
+        _check_call(pool, wl, call, tensors[call.tensor], host[call.tensor])
 
 
 @pytest.mark.parametrize("name", ["weight", "gradient", "activation", "mlp_up"])
-def test_full_size_sampled(name):
-    _check_workload(W.ALL[name]())
+def test_full_size_whole_tensors(pool, name):
+    _check_workload(pool, W.ALL[name]())
 
 
 def test_full_size_dual_pre_pass():
