@@ -75,6 +75,8 @@ def parse_args(argv=None):
                    help="skip the per-mode table (every mode on dY, quantize kernel alone)")
     p.add_argument("--no-configs", action="store_true",
                    help="skip the other workloads' calls (256x256, weight, gradient, activation)")
+    p.add_argument("--no-unfused", action="store_true",
+                   help="skip the comparison step with one quantize launch per call")
     p.add_argument("--no-eager", action="store_true",
                    help="skip the eager (host-launched) run reported beside the graph-timed value")
     return p.parse_args(argv)
@@ -265,8 +267,29 @@ class TensorCalls:
         if st:
             raise self.N.Nvfp4Error(st, "nvfp4_amax_dual")
 
-    def launches(self):
-        return (1 if self.dual else len(self.calls)) + len(self.calls)
+    def quantize_dual(self):
+        """Both layouts' codes and scales from one read (nvfp4_quantize_dual)."""
+        r, c = self.row, self.col
+        st = self.N.nvfp4_quantize_dual(r.p["x"], r.rows, r.cols, r.ld, r.call.mode, r.call.rht_group, c.call.mode,
+                                        c.call.rht_group, r.seed, r.p["amax"], c.p["amax"], r.p["codes"],
+                                        r.p["scales"], r.p["gscale"], c.p["codes"], c.p["scales"], c.p["gscale"],
+                                        r.stream)
+        if st:
+            raise self.N.Nvfp4Error(st, "nvfp4_quantize_dual")
+
+    def body(self, fused):
+        """The launches of this tensor's part of a step: its pre-pass(es), then
+        one dual quantize (fused) or one quantize per call."""
+        out = [(self.amax_passes, "amax", self)]
+        if fused and self.dual:
+            out.append((self.quantize_dual, "dual", self))
+        else:
+            out += [(c.quantize, "quant", c) for c in self.calls]
+        return out
+
+    def launches(self, fused=True):
+        pre = 1 if self.dual else len(self.calls)
+        return pre + (1 if fused and self.dual else len(self.calls))
 
 
 def dist_us(seconds):
@@ -423,6 +446,63 @@ def gemm_table(N, calls, stream, device, reps=10):
     return out
 
 
+def linear_layer_table(N, groups, stream, device, flush, tensors, reps=10):
+    """The Quartet II linear layer of the MLP up-projection, fully NVFP4, as
+    one forward and one backward pass:
+      forward : per operand (X, W) the dual pre-pass and the dual quantize
+                (row-wise RTN for Y, transposed MS-EDEN kept for the backward
+                pass), then Y = X W^T (nvfp4_gemm, bf16 out);
+      backward: dY's dual pre-pass and dual quantize (MS-EDEN both ways),
+                then dX = dY W and dW = dY^T X (nvfp4_gemm, bf16 out).
+    Timed inside CUDA graphs (L2 flushed before each repetition), beside the
+    same three GEMMs in bf16 through torch.matmul (cuBLAS) on the unquantized
+    tensors -- the comparison behind the pages' "up to 4.2x faster than BF16"
+    for their Blackwell kernels (context, not a target)."""
+    by = {g.calls[0].call.tensor: g for g in groups}
+    gx, gw, gdy = by["x"], by["w"], by["dy"]
+    q = lambda c: (c.codes, c.scales, c.gscale)  # noqa: E731
+    x, w, dy = tensors["x"], tensors["w"], tensors["dy"]
+    y = torch.empty(x.shape[0], w.shape[0], dtype=torch.bfloat16, device=device)
+    dx = torch.empty(dy.shape[0], w.shape[1], dtype=torch.bfloat16, device=device)
+    dw = torch.empty(dy.shape[1], x.shape[1], dtype=torch.bfloat16, device=device)
+    fwd = [gx.amax_passes, gw.amax_passes, gx.quantize_dual, gw.quantize_dual,
+           lambda: N.gemm(q(gx.row), q(gw.row), out=y)]
+    bwd = [gdy.amax_passes, gdy.quantize_dual,
+           lambda: N.gemm(q(gdy.row), q(gw.col), out=dx),
+           lambda: N.gemm(q(gdy.col), q(gx.col), out=dw)]
+    with torch.cuda.stream(stream):
+        for fn in fwd + bwd:
+            fn()
+    d_fwd, t_fwd = timed_in_graph(stream, fwd, reps, flush, device)
+    d_bwd, t_bwd = timed_in_graph(stream, bwd, reps, flush, device)
+    bf = [lambda: torch.matmul(x, w.t(), out=y), lambda: torch.matmul(dy, w, out=dx),
+          lambda: torch.matmul(dy.t(), x, out=dw)]
+    with torch.cuda.stream(stream):
+        for fn in bf:
+            fn()
+    d_bf, t_bf = timed_in_graph(stream, bf, reps, flush, device)
+    torch.cuda.synchronize(device)
+    f, b, r = dist_us(t_fwd), dist_us(t_bwd), dist_us(t_bf)
+    m, k, n = x.shape[0], x.shape[1], w.shape[0]
+    flops = 3 * 2.0 * m * n * k
+    names_f = ["amax_dual x", "amax_dual w", "quantize_dual x", "quantize_dual w", "gemm Y = X W^T"]
+    names_b = ["amax_dual dy", "quantize_dual dy", "gemm dX = dY W", "gemm dW = dY^T X"]
+    step_us = f["median"] + b["median"]
+    return {
+        "shapes": {"x": list(x.shape), "w": list(w.shape), "dy": list(dy.shape)},
+        "forward_us": f, "backward_us": b, "step_us": round(step_us, 2),
+        "forward_launches": {nm: dist_us([d[i] for d in d_fwd]) for i, nm in enumerate(names_f)},
+        "backward_launches": {nm: dist_us([d[i] for d in d_bwd]) for i, nm in enumerate(names_b)},
+        "gemm_tflops_effective": round(flops / (step_us / 1e6) / 1e12, 1),
+        "bf16_cublas_step_us": r,
+        "bf16_gemms_us": {nm: dist_us([d[i] for d in d_bf]) for i, nm in
+                          enumerate(["Y = X W^T", "dX = dY W", "dW = dY^T X"])},
+        "speedup_over_bf16": round(r["median"] / step_us, 3),
+        "note": "quantization of all three operands in both layouts included in the NVFP4 step; the bf16 step "
+                "is the three GEMMs alone",
+    }
+
+
 def run_ours(args, world, rank, local):
     import ctypes
     from nvfp4_microscaling_quantization_b200 import binding as N
@@ -442,14 +522,15 @@ def run_ours(args, world, rank, local):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     bytes_per_step = sum(BYTES_PER_ELEMENT * c.elements for c in calls)
     elems_per_step = sum(c.elements for c in calls)
-    # one step = per tensor its pre-pass, then its quantize calls: 9 launches
+    # one step = per tensor its dual pre-pass, then its dual quantize (both
+    # layouts from one read): 6 launches; the unfused step (one quantize per
+    # call, 9 launches) is timed too, for comparison
     body, body_names = [], []
     for grp in groups:
-        body.append(grp.amax_passes)
-        body_names.append(("amax", grp))
-        for c in grp.calls:
-            body.append(c.quantize)
-            body_names.append(("quant", c))
+        for fn, kind, obj in grp.body(fused=True):
+            body.append(fn)
+            body_names.append((kind, obj))
+    body_unfused = [fn for grp in groups for fn, _, _ in grp.body(fused=False)]
 
     def step():
         for fn in body:
@@ -492,35 +573,61 @@ def run_ours(args, world, rank, local):
 
     total_s = max_over_ranks(sum(totals), world, device)
     per_fn = [[durs[k][i] for k in range(K)] for i in range(len(body))]
-    quant_idx = [i for i, (kind, _) in enumerate(body_names) if kind == "quant"]
+    quant_idx = [i for i, (kind, _) in enumerate(body_names) if kind in ("quant", "dual")]
     quant_total_s = max_over_ranks(sum(sum(per_fn[i]) for i in quant_idx), world, device)
     value = weak_scaling_value(bytes_per_step, K, world, total_s)
     value_supplied = weak_scaling_value(bytes_per_step, K, world, quant_total_s)
     peak, peak_kind = hbm_peak()
 
+    def moved_bytes(kind, obj):
+        """Bytes a launch must move: a quantize reads 2 B and writes 0.5625 B
+        per element; a dual quantize reads once and writes both views."""
+        if kind == "quant":
+            return BYTES_PER_ELEMENT * obj.elements
+        if kind == "dual":
+            return (PREPASS_BYTES_PER_ELEMENT + 2 * (BYTES_PER_ELEMENT - 2.0)) * obj.row.elements
+        return PREPASS_BYTES_PER_ELEMENT * obj.calls[0].elements
+
+    def launch_name(kind, obj):
+        if kind == "quant":
+            return f"quantize {obj.call.name}"
+        t = obj.calls[0].call.tensor
+        return (f"quantize_dual {t} ({obj.row.call.name} + {obj.col.call.name})" if kind == "dual"
+                else f"amax_{'dual' if obj.dual else 'single'} {t}")
+
     # dominant kernel: the quantize launch with the largest mean duration in the step
     dom_i = max(quant_idx, key=lambda i: statistics.mean(per_fn[i]))
-    dom = body_names[dom_i][1]
+    dom_kind, dom = body_names[dom_i]
     dom_stats = dist_us(per_fn[dom_i])
-    dom_bytes = BYTES_PER_ELEMENT * dom.elements
+    dom_bytes = moved_bytes(dom_kind, dom)
     achieved = dom_bytes / (dom_stats["mean"] / 1e6) / 1e9
     src_hash = kernel_source_hash()
-    traffic = NCU_TRAFFIC.get((src_hash, dom.call.name))
+    traffic = NCU_TRAFFIC.get((src_hash, launch_name(dom_kind, dom)))
 
-    per_call, pre_passes = [], []
+    per_launch = []
     for i, (kind, obj) in enumerate(body_names):
         d = dist_us(per_fn[i])
         t = d["mean"] / 1e6
-        if kind == "quant":
-            per_call.append({"call": obj.call.name, "elements": obj.elements, "us": d,
-                             "gbs": round(BYTES_PER_ELEMENT * obj.elements / t / 1e9, 1),
-                             "gelem_s": round(obj.elements / t / 1e9, 1),
-                             "frac_of_hbm_peak": round(BYTES_PER_ELEMENT * obj.elements / t / 1e9 / peak, 4)})
+        line = {"launch": launch_name(kind, obj), "us": d}
+        if kind == "amax":
+            line["read_gbs"] = round(moved_bytes(kind, obj) / t / 1e9, 1)
         else:
-            read = PREPASS_BYTES_PER_ELEMENT * obj.calls[0].elements
-            pre_passes.append({"tensor": obj.calls[0].call.tensor, "kind": "dual" if obj.dual else "single",
-                               "for_calls": [c.call.name for c in obj.calls], "us": d,
-                               "read_gbs": round(read / t / 1e9, 1)})
+            calls_of = [obj] if kind == "quant" else [obj.row, obj.col]
+            metric_bytes = sum(BYTES_PER_ELEMENT * c.elements for c in calls_of)
+            line.update({"for_calls": [c.call.name for c in calls_of],
+                         "gbs": round(metric_bytes / t / 1e9, 1),
+                         "gelem_s": round(sum(c.elements for c in calls_of) / t / 1e9, 1),
+                         "moved_gbs": round(moved_bytes(kind, obj) / t / 1e9, 1),
+                         "frac_of_hbm_peak": round(moved_bytes(kind, obj) / t / 1e9 / peak, 4)})
+        per_launch.append(line)
+
+    unfused = None
+    if not args.no_unfused:
+        _, u_tot = timed_in_graph(stream, body_unfused, K, flush, device)
+        u_s = sum(u_tot)
+        unfused = {"note": "the same step with one quantize launch per call (9 launches), CUDA graph timing",
+                   "ms_per_step": {k: round(v / 1e3, 4) for k, v in dist_us(u_tot).items()},
+                   "value": round(weak_scaling_value(bytes_per_step, K, 1, u_s), 1)}
     if not args.no_eager:
         eager = {"note": "the same K steps launched eagerly from Python (host enqueue in the device timeline); "
                          "not the value",
@@ -530,6 +637,10 @@ def run_ours(args, world, rank, local):
     gemms = None
     if not args.no_gemm:
         gemms = gemm_table(N, calls, stream, device)
+
+    layer = None
+    if not args.no_gemm:
+        layer = linear_layer_table(N, groups, stream, device, flush, tensors)
 
     per_mode = None
     if not args.no_per_mode:
@@ -557,8 +668,8 @@ def run_ours(args, world, rank, local):
             "workload": "mlp_up: one Llama-style MLP up-projection training step's tensors, "
                         "X 16384x4096 N(0,1), W 14336x4096 N(0,0.02^2), dY 16384x14336 Student-t3 std 1e-4",
             "calls": [c.call.name for c in calls],
-            "path": "per tensor: one tensor-amax pre-pass for both layouts (nvfp4_amax_dual), then its "
-                    "quantize kernels (C ABI), one stream",
+            "path": "per tensor: one tensor-amax pre-pass for both layouts (nvfp4_amax_dual), then both "
+                    "layouts' codes and scales from one read (nvfp4_quantize_dual), C ABI, one stream",
             "timing": "the K steps captured once as one CUDA graph of the C-ABI launches and replayed once; "
                       "CUDA events (graph event nodes) before, between and after the launches of each step",
             "input_dtype": "bf16", "l2": "flushed before every timed step (256 MiB write, outside the marks)",
@@ -569,21 +680,26 @@ def run_ours(args, world, rank, local):
         "step_ms": step_stats,
         "value_amax_supplied": round(value_supplied, 1),
         "frac_of_hbm_peak_amax_supplied": round(value_supplied / world / peak, 4),
-        "roofline": {"bound": "hbm", "kernel": f"quantize {dom.call.name}",
+        "roofline": {"bound": "hbm", "kernel": launch_name(dom_kind, dom),
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "algorithmic_bytes": int(dom_bytes), "avg_launch_us": dom_stats["mean"],
-                     "launch_us": dom_stats},
-        "per_call": per_call,
-        "amax_pre_passes": pre_passes,
-        "gpu_launches": sum(g.launches() for g in groups) * K,
+                     "algorithmic_bytes": int(dom_bytes),
+                     "algorithmic_bytes_per_element": round(dom_bytes / (dom.elements if dom_kind == "quant"
+                                                                         else dom.row.elements), 4),
+                     "avg_launch_us": dom_stats["mean"], "launch_us": dom_stats},
+        "per_launch": per_launch,
+        "gpu_launches": sum(g.launches(fused=True) for g in groups) * K,
         "clocks": clock,
         "kernel_source": src_hash,
     }
     if eager is not None:
         result["eager"] = eager
+    if unfused is not None:
+        result["unfused"] = unfused
     if gemms is not None:
         result["nvfp4_gemm"] = gemms
+    if layer is not None:
+        result["linear_layer"] = layer
     if per_mode is not None:
         result["per_mode_dy"] = per_mode
     if configs is not None:
@@ -635,9 +751,8 @@ def run_e2e(args, calls, tensors, stream, device, world, bytes_per_step):
             if i >= 2:
                 s_comp.wait_event(ev["out"][i - 2])  # output set b copied out
             for grp in group_sets[b]:
-                grp.amax_passes()
-                for c in grp.calls:
-                    c.quantize()
+                for fn, _, _ in grp.body(fused=True):
+                    fn()
             ev["comp"][i].record(s_comp)
             s_out.wait_event(ev["comp"][i])
             with torch.cuda.stream(s_out):

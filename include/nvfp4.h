@@ -167,6 +167,35 @@ NVFP4_API int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t 
                    uint8_t* codes, uint8_t* scales, float* global_scale, void* workspace,
                    size_t workspace_bytes, void* stream);
 
+/* Both layouts' quantization of x from one read of it: the outputs of
+ *   nvfp4_quantize(x, ..., NVFP4_ROWWISE, mode_row, rht_group_row, seed, amax_row, codes_row, scales_row, gscale_row)
+ *   nvfp4_quantize(x, ..., NVFP4_TRANSPOSED, mode_col, rht_group_col, seed, amax_col, codes_col, scales_col, gscale_col)
+ * bit for bit.  A fully-NVFP4 linear layer needs W, X and dY quantized along
+ * both dimensions (Quartet II article, section "Quantisierung im
+ * Vorwaertsdurchlauf": W and X are re-quantized for the backward pass; section
+ * "Quantisierung im Rueckwaertsdurchlauf": dY enters both backward GEMMs), so
+ * one kernel that reads each tile once and writes both views saves a full
+ * read of the tensor.  The fused kernel takes the pairs such a layer uses --
+ * row-wise RTN without rotation with transposed MS-EDEN (group g), and MS-EDEN
+ * with the same group g in both layouts, g in {16, 32, 64, 128} -- on tensors
+ * of at least 128 x 128; any other pair (and smaller tensors) runs as the two
+ * single-layout calls, with the same results.
+ *  amax_row, amax_col: device floats holding the two views' tensor amaxes
+ *             (nvfp4_amax_dual gives both from one read); required, except
+ *             for the MX modes, which have no tensor scale.
+ *  codes_row, scales_row, gscale_row: the row-wise view's outputs (rows x
+ *             cols/2, rows x cols/16 bytes, one float); codes_col, scales_col,
+ *             gscale_col: the transposed view's (cols x rows/2, cols x rows/16,
+ *             one float).  Caller-owned device memory; the two sets must not
+ *             overlap.
+ * Shape and alignment rules: those of nvfp4_quantize for each layout.
+ * Errors as nvfp4_quantize; nothing is launched when a check fails. */
+NVFP4_API int nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int64_t ld, int mode_row,
+                                  int rht_group_row, int mode_col, int rht_group_col, uint64_t seed,
+                                  const float* amax_row, const float* amax_col, uint8_t* codes_row,
+                                  uint8_t* scales_row, float* gscale_row, uint8_t* codes_col,
+                                  uint8_t* scales_col, float* gscale_col, void* stream);
+
 /* Decode a quantized view (vrows x vcols) back to fp32:
  * out[r][j] = value(code, flag) * RN(E4M3(scale & 0x7F) * s_g), and, when
  * inverse_rht != 0 (needs rht_group > 0 and the seed used to quantize), the

@@ -48,6 +48,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_amax_dual.restype = i32
         L.nvfp4_quantize.argtypes = [P, i64, i64, i64, i32, i32, i32, u64, P, P, P, P, P, sz, P]
         L.nvfp4_quantize.restype = i32
+        L.nvfp4_quantize_dual.argtypes = [P, i64, i64, i64, i32, i32, i32, i32, u64, P, P, P, P, P, P, P, P, P]
+        L.nvfp4_quantize_dual.restype = i32
         L.nvfp4_dequantize.argtypes = [P, P, P, i64, i64, i32, i32, u64, i32, P, P]
         L.nvfp4_dequantize.restype = i32
         L.nvfp4_rht.argtypes = [P, i32, i64, i64, i64, i32, i32, u64, i32, P, P]
@@ -88,6 +90,14 @@ def nvfp4_quantize(x, rows, cols, ld, layout, mode, rht_group, seed, amax_in, co
                    global_scale, workspace, workspace_bytes, stream) -> int:
     return lib().nvfp4_quantize(x, rows, cols, ld, layout, mode, rht_group, seed, amax_in, codes,
                                 scales, global_scale, workspace, workspace_bytes, stream)
+
+
+def nvfp4_quantize_dual(x, rows, cols, ld, mode_row, rht_group_row, mode_col, rht_group_col, seed, amax_row,
+                        amax_col, codes_row, scales_row, gscale_row, codes_col, scales_col, gscale_col,
+                        stream) -> int:
+    return lib().nvfp4_quantize_dual(x, rows, cols, ld, mode_row, rht_group_row, mode_col, rht_group_col, seed,
+                                     amax_row, amax_col, codes_row, scales_row, gscale_row, codes_col, scales_col,
+                                     gscale_col, stream)
 
 
 def nvfp4_dequantize(codes, scales, global_scale, vrows, vcols, mode, rht_group, seed, inverse_rht,
@@ -194,6 +204,24 @@ def quantize(x: torch.Tensor, layout: int = ROWWISE, mode: int = RTN, rht_group:
                         _stream_handle(stream))
     _check(st, "nvfp4_quantize")
     return codes, scales, gscale
+
+
+def quantize_dual(x: torch.Tensor, mode_row: int, rht_group_row: int, mode_col: int, rht_group_col: int,
+                  seed: int = 0, amax_row: Optional[torch.Tensor] = None, amax_col: Optional[torch.Tensor] = None,
+                  out_row=None, out_col=None, stream=None):
+    """Both layouts of a bf16 CUDA matrix from one read (nvfp4_quantize_dual);
+    returns ((codes, scales, gscale) row-wise, (codes, scales, gscale)
+    transposed).  Without amax_row / amax_col both tensor amaxes come from one
+    nvfp4_amax_dual pre-pass on the same stream."""
+    rows, cols, ld = _matrix(x, torch.bfloat16)
+    if amax_row is None or amax_col is None:
+        amax_row, amax_col = amax_dual(x, rht_group_row, rht_group_col, seed, stream=stream)
+    r = alloc_outputs(rows, cols, ROWWISE, x.device) if out_row is None else out_row
+    c = alloc_outputs(rows, cols, TRANSPOSED, x.device) if out_col is None else out_col
+    _check(nvfp4_quantize_dual(_p(x), rows, cols, ld, mode_row, rht_group_row, mode_col, rht_group_col, seed,
+                               _p(amax_row), _p(amax_col), _p(r[0]), _p(r[1]), _p(r[2]), _p(c[0]), _p(c[1]),
+                               _p(c[2]), _stream_handle(stream)), "nvfp4_quantize_dual")
+    return r, c
 
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, gscale: torch.Tensor, mode: int = RTN,

@@ -122,6 +122,45 @@ int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int la
   return from_cuda(nvfp4::launch_quantize(a));
 }
 
+int nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int64_t ld, int mode_row, int rht_group_row,
+                        int mode_col, int rht_group_col, uint64_t seed, const float* amax_row, const float* amax_col,
+                        uint8_t* codes_row, uint8_t* scales_row, float* gscale_row, uint8_t* codes_col,
+                        uint8_t* scales_col, float* gscale_col, void* stream) {
+  int64_t vr, vc;
+  int st = check_tensor(x, rows, cols, ld, NVFP4_ROWWISE, rht_group_row, &vr, &vc);
+  if (st) return st;
+  if ((st = check_tensor(x, rows, cols, ld, NVFP4_TRANSPOSED, rht_group_col, &vr, &vc))) return st;
+  for (int m : {mode_row, mode_col})
+    if (m < NVFP4_RTN || m > NVFP4_MXFP3) return NVFP4_ERR_INVALID_ARG;
+  if ((mode_row == NVFP4_MS_EDEN && rht_group_row == 0) || (mode_col == NVFP4_MS_EDEN && rht_group_col == 0))
+    return NVFP4_ERR_UNSUPPORTED;
+  const bool mx_r = mode_row == NVFP4_MXFP4 || mode_row == NVFP4_MXFP3;
+  const bool mx_c = mode_col == NVFP4_MXFP4 || mode_col == NVFP4_MXFP3;
+  if ((mx_r && cols % 32) || (mx_c && rows % 32)) return NVFP4_ERR_SHAPE;
+  const bool empty = rows == 0 || cols == 0;
+  if (!gscale_row || !gscale_col) return NVFP4_ERR_INVALID_ARG;
+  if (!empty && (!codes_row || !scales_row || !codes_col || !scales_col)) return NVFP4_ERR_INVALID_ARG;
+  if ((!mx_r && !amax_row) || (!mx_c && !amax_col)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes_row, 8) || !aligned(codes_col, 8) || !aligned(gscale_row, 4) || !aligned(gscale_col, 4))
+    return NVFP4_ERR_ALIGNMENT;
+  if ((amax_row && !aligned(amax_row, 4)) || (amax_col && !aligned(amax_col, 4))) return NVFP4_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  nvfp4::DualQuantArgs d{x, rows, cols, ld, mode_row, rht_group_row, mode_col, rht_group_col, seed,
+                         amax_row, amax_col, codes_row, scales_row, gscale_row, codes_col, scales_col, gscale_col,
+                         1, s};
+  if (!empty && nvfp4::dual_quantize_fused(d)) return from_cuda(nvfp4::launch_quantize_dual_mma(d));
+  // any other pair: the two single-layout launches (MX modes read no amax:
+  // their kernels are given the output scalar, as nvfp4_quantize does)
+  nvfp4::QuantArgs a{x, rows, cols, ld, NVFP4_ROWWISE, mode_row, rht_group_row, seed,
+                     mx_r ? gscale_row : amax_row, nullptr, codes_row, scales_row, gscale_row, s};
+  if (!empty && mx_r && !nvfp4::mma_path_applies(a) && !nvfp4::tma_path_applies(a)) return NVFP4_ERR_UNSUPPORTED;
+  if ((st = from_cuda(nvfp4::launch_quantize(a)))) return st;
+  nvfp4::QuantArgs b{x, rows, cols, ld, NVFP4_TRANSPOSED, mode_col, rht_group_col, seed,
+                     mx_c ? gscale_col : amax_col, nullptr, codes_col, scales_col, gscale_col, s};
+  if (!empty && mx_c && !nvfp4::mma_path_applies(b) && !nvfp4::tma_path_applies(b)) return NVFP4_ERR_UNSUPPORTED;
+  return from_cuda(nvfp4::launch_quantize(b));
+}
+
 int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
                      int64_t vrows, int64_t vcols, int mode, int rht_group, uint64_t seed,
                      int inverse_rht, float* out, void* stream) {

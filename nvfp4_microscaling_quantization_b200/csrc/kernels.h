@@ -73,6 +73,31 @@ cudaError_t launch_amax_dual_mma(const void* x, int64_t rows, int64_t cols, int6
                                  uint64_t seed, float* amax_r, float* amax_c, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantArgs& a);
 
+// Both layouts' codes and scales from one read of X (rotate_mma.cu), given
+// both tensor amaxes.  The fused kernel takes the mode pairs of a fully-NVFP4
+// linear layer's operands: row view RTN without rotation + column view
+// MS-EDEN with group g (the forward operands X, W re-quantized for the
+// backward pass), and MS-EDEN with group g in both views (the output
+// gradient dY); dual_quantize_fused says whether it applies.
+struct DualQuantArgs {
+  const void* x;
+  int64_t rows, cols, ld;
+  int mode_row, rht_group_row, mode_col, rht_group_col;
+  uint64_t seed;
+  const float* amax_row;
+  const float* amax_col;
+  uint8_t* codes_row;
+  uint8_t* scales_row;
+  float* gscale_row;
+  uint8_t* codes_col;
+  uint8_t* scales_col;
+  float* gscale_col;
+  int reverse;            // walk the tiles from the last one back
+  cudaStream_t stream;
+};
+bool dual_quantize_fused(const DualQuantArgs& a);
+cudaError_t launch_quantize_dual_mma(const DualQuantArgs& a);
+
 // D = gA gB A B^T from two quantizer outputs (gemm.cu); shapes checked by the
 // caller: m, n multiples of 128, k of 256, 16-byte aligned codes, scales, D rows.
 struct GemmArgs {

@@ -147,6 +147,66 @@ __device__ __forceinline__ void build_hadamard_b(uint8_t* bmat, PhiloxKey key, u
   }
 }
 
+// Quantize one thread's row of a 128 x 128 tile of a view from tensor memory:
+// the accumulator columns at taddr (this thread's lane; columns permuted by
+// output_col_of) hold the unscaled rotation sums of view row vrow, view
+// columns vcol_base .. vcol_base + 127.  Each 32-column load is scaled by
+// c_G and quantized two blocks at a time; lane 0 of the warp arrives on
+// free_bar once the warp's last columns are loaded.  Blocks outside the view
+// are not stored.
+template <int MODE, int G>
+__device__ __forceinline__ void quantize_tmem_row(uint32_t taddr, uint64_t* free_bar, const ScaleCtx& sc,
+                                                  PhiloxKey key, int64_t vrow, int64_t vcol_base, int64_t vrows,
+                                                  int64_t vcols, bool row_blocks8, bool codes_aligned16,
+                                                  bool scales_aligned4, uint8_t* codes, uint8_t* scales) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const float2 c2 = f2(RhtConst<G>::c, RhtConst<G>::c);
+  // MS-EDEN scale uniforms: when a thread owns a whole 128-column row of the
+  // tile and view rows hold whole groups of eight blocks, its eight blocks
+  // take the eight draws of one Philox call
+  uint4 wu = make_uint4(0u, 0u, 0u, 0u);
+  if constexpr (MODE == kMSEDEN) {
+    if (row_blocks8)
+      wu = philox_call(key, (static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols / 16) +
+                             static_cast<uint64_t>(vcol_base / 16)) >> 3,
+                       kTagBlock);
+  }
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    const int64_t vcol0 = vcol_base + 64 * h;  // view column of the first element
+    const bool last = h == 1;
+    // one pair of blocks at a time: load 32 columns, quantize, then the next 32
+    const bool valid = vrow < vrows && vcol0 < vcols;
+    const uint64_t e0 = static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols) + static_cast<uint64_t>(vcol0);
+    float u[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if constexpr (MODE == kMSEDEN) {
+      if (row_blocks8) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) u[b] = uniform16(half_word(wu, 4 * h + b));
+      } else {
+        block_uniforms<4>(key, e0 >> 4, u);
+      }
+    }
+    BlockOut o[4];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      float v[32];
+      tmem_ld32_wait(taddr + 64 * h + 32 * p, v);
+      if (last && p == 1) {
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(free_bar);
+      }
+      float2 zp[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) zp[i] = mul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
+      const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, u[2 * p], u[2 * p + 1]};
+      quantize_pair<MODE>(zp, sc, rng, o[2 * p], o[2 * p + 1]);
+    }
+    if (valid) store64(o, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);
+  }
+}
+
 template <int MODE, int G, int KIND, bool ROWWISE>
 __global__ void __launch_bounds__(Shape<MODE, KIND>::threads, 1)
 rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed,
@@ -285,54 +345,16 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
       tg.coords(static_cast<uint32_t>(t), rt, ct);
       // view row of this thread
       const int64_t vrow = (ROWWISE ? rt : ct) * kTile + 32 * q + lane;
-      // MS-EDEN scale uniforms: when a thread owns a whole 128-column row of
-      // the tile and view rows hold whole groups of eight blocks, its eight
-      // blocks take the eight draws of one Philox call
-      uint4 wu = make_uint4(0u, 0u, 0u, 0u);
-      if constexpr (KIND == kQuantize && MODE == kMSEDEN) {
-        if (row_blocks8)
-          wu = philox_call(key, (static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols / 16) +
-                                 static_cast<uint64_t>((ROWWISE ? ct : rt) * (kTile / 16))) >> 3,
-                           kTagBlock);
-      }
+      if constexpr (KIND == kQuantize) {
+        quantize_tmem_row<MODE, G>(tmem_base + ((32u * q) << 16) + a * kTile, &sh.tfree[a], sc, key, vrow,
+                                   static_cast<int64_t>(ROWWISE ? ct : rt) * kTile, vrows, vcols, row_blocks8,
+                                   codes_aligned16, scales_aligned4, codes, scales);
+      } else {
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t j = h;
-        const uint32_t taddr = tmem_base + ((32u * q) << 16) + a * kTile + j * 64;
-        const int64_t vcol0 = (ROWWISE ? ct : rt) * kTile + 64 * j;  // view column of the first element
-        const bool last = h == 1;
-
-        if constexpr (KIND == kQuantize) {
-          // one pair of blocks at a time: load 32 columns, quantize, then the next 32
-          const bool valid = vrow < vrows && vcol0 < vcols;
-          const uint64_t e0 = static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols) + static_cast<uint64_t>(vcol0);
-          float u[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-          if constexpr (MODE == kMSEDEN) {
-            if (row_blocks8) {
-#pragma unroll
-              for (int b = 0; b < 4; ++b) u[b] = uniform16(half_word(wu, 4 * j + b));
-            } else {
-              block_uniforms<4>(key, e0 >> 4, u);
-            }
-          }
-          BlockOut o[4];
-#pragma unroll
-          for (int p = 0; p < 2; ++p) {
-            float v[32];
-            tmem_ld32_wait(taddr + 32 * p, v);
-            if (last && p == 1) {
-              tc_fence_before_sync();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&sh.tfree[a]);
-            }
-            float2 zp[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) zp[i] = mul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
-            const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, u[2 * p], u[2 * p + 1]};
-            quantize_pair<MODE>(zp, sc, rng, o[2 * p], o[2 * p + 1]);
-          }
-          if (valid) store64(o, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);
-        } else {
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t taddr = tmem_base + ((32u * q) << 16) + a * kTile + h * 64;
+          const int64_t vcol0 = (ROWWISE ? ct : rt) * kTile + 64 * h;  // view column of the first element
+          const bool last = h == 1;
           // max |z| or z itself, one pair of blocks (32 columns) at a time
 #pragma unroll
           for (int p = 0; p < 2; ++p) {
@@ -405,21 +427,26 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
 // ------------------------------------------------------- both layouts at once
 // The tensor amax of the row-wise view (rotated along rows with group g_r)
 // and of the transposed view (rotated along columns with group g_c) from one
-// read of X: every tile goes through two MMAs, the K-major one against B_r
-// and the MN-major one against B_c (g = 0: the identity, z = x exactly), into
-// the two accumulators of the epilogue group that takes the tile.  The
-// results are those of two single-layout pre-passes bit for bit (the same
-// MMAs, the same scaling).  Two epilogue groups, each owning two 128-column
-// accumulators (all 512 columns); in a group of eight warps, warp (q, j)
-// reads lane quarter q of the row-view (j = 0) or column-view (j = 1)
-// accumulator, 64 columns per load.
+// read of X.  Every tile goes through the MMAs its views need -- the K-major
+// one against B_r (when g_r > 0) and the MN-major one against B_c (g_c = 0:
+// the identity, z = x exactly) -- each into the next of four 128-column
+// accumulator slots (all 512 tensor-memory columns), each slot with its own
+// "full" and "free" barriers, so a view's epilogue starts as soon as its own
+// MMAs land and the MMA warp refills a slot as soon as it is read.  Slot s is
+// read by epilogue warps 4s .. 4s+3 (warp 4s + q reads lane quarter q).
+// With g_r = 0 (the forward RTN operands X and W) the row view needs no MMA:
+// the slot's warps also take max|x| straight from the staged tile before its
+// stage is released, and four tiles are in flight in tensor memory.
+// Because RN(c t) is monotone in t >= 0, the epilogue keeps max |acc| and
+// scales once at the end: max RN(c |acc|) = RN(c max |acc|), so the results
+// are those of the single-layout pre-passes bit for bit.
 
 #ifndef NVFP4_DUAL_STAGES
-#define NVFP4_DUAL_STAGES 3
+#define NVFP4_DUAL_STAGES 4
 #endif
-constexpr int kDualStages = NVFP4_DUAL_STAGES;  // A tiles in flight (each held until both MMAs are done)
-constexpr int kDualGroups = 2;
-constexpr int kDualEpiWarps = 8 * kDualGroups;
+constexpr int kDualStages = NVFP4_DUAL_STAGES;  // A tiles in flight (each held until its MMAs are done)
+constexpr int kDualSlots = 4;                   // 128-column accumulator slots
+constexpr int kDualEpiWarps = 4 * kDualSlots;
 constexpr int kDualThreads = (kDualEpiWarps + 2) * 32;
 constexpr int kDualProducerWarp = kDualEpiWarps, kDualMmaWarp = kDualEpiWarps + 1;
 constexpr size_t kDualDynSmem = (kDualStages + 2) * kTileBytes + 1024;
@@ -427,8 +454,8 @@ constexpr size_t kDualDynSmem = (kDualStages + 2) * kTileBytes + 1024;
 struct DualShared {
   uint64_t full[kDualStages];
   uint64_t sfree[kDualStages];
-  uint64_t tfull[kDualGroups];   // both accumulators of the group ready
-  uint64_t tfree[kDualGroups];   // both loaded by the group
+  uint64_t tfull[kDualSlots];   // the slot's accumulator is ready
+  uint64_t tfree[kDualSlots];   // the slot's accumulator has been read by its four warps
   uint32_t tmem_base;
   uint32_t issued_a;
   uint32_t issued_mma;
@@ -474,6 +501,17 @@ __device__ __forceinline__ void build_rotation_b(uint8_t* bmat, PhiloxKey key, u
   }
 }
 
+// max |v| over 64 accumulator values, kept in two chains.
+__device__ __forceinline__ float absmax64(const float (&v)[64], float m) {
+  float m0 = m, m1 = m;
+#pragma unroll
+  for (int i = 0; i < 64; i += 2) {
+    m0 = fmaxf(m0, fabsf(v[i]));
+    m1 = fmaxf(m1, fabsf(v[i + 1]));
+  }
+  return fmaxf(m0, m1);
+}
+
 __global__ void __launch_bounds__(kDualThreads, 1)
 dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed, int g_r,
                  int g_c, unsigned int* __restrict__ amax_r, unsigned int* __restrict__ amax_c) {
@@ -488,17 +526,23 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
   const TileGrid tg{static_cast<uint32_t>((rows + kTile - 1) / kTile), static_cast<uint32_t>((cols + kTile - 1) / kTile),
                     static_cast<uint32_t>(NVFP4_MMA_BAND_ROWS)};
   const int64_t n_tiles = static_cast<int64_t>(tg.n_rt) * tg.n_ct;
+  const int64_t step = gridDim.x;
+  // this CTA's tiles: blockIdx.x, blockIdx.x + step, ...
+  const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - blockIdx.x + step - 1) / step : 0;
+  // accumulators per tile: the row view's (if rotated) then the column view's
+  const int views = g_r != 0 ? 2 : 1;
+  const bool row_from_smem = g_r == 0;
 
   if (tid == kDualProducerWarp * 32) {
-    // with g_r = 0 the row view needs no MMA: the group's four row-view
-    // warps take max|x| from the staged tile and release the stage themselves
     for (int s = 0; s < kDualStages; ++s) {
       mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.sfree[s], g_r == 0 ? 5 : 1);
+      // released by the MMA commit, and with the row view taken from shared
+      // memory also by the four warps of the slot that reads the tile
+      mbar_init(&sh.sfree[s], row_from_smem ? 5 : 1);
     }
-    for (int a = 0; a < kDualGroups; ++a) {
+    for (int a = 0; a < kDualSlots; ++a) {
       mbar_init(&sh.tfull[a], 1);
-      mbar_init(&sh.tfree[a], g_r == 0 ? 4 : 8);
+      mbar_init(&sh.tfree[a], 4);
     }
     sh.issued_a = 0;
     sh.issued_mma = 0;
@@ -513,7 +557,6 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = sh.tmem_base;
-  const int64_t step = gridDim.x;
   if (warp != kDualProducerWarp) {
     // the B matrices, built while the producer starts loading (barrier 2)
     const uint32_t bt = warp < kDualProducerWarp ? tid : tid - 32, nb = kDualThreads - 32;
@@ -526,17 +569,16 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
   if (warp == kDualProducerWarp) {
     if (lane == 0) {
       prefetch_tensormap(&tmap);
-      int k = 0;
-      for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++k) {
-        const int s = k % kDualStages;
-        const uint32_t u = k / kDualStages;
+      for (int64_t k = 0; k < my_tiles; ++k) {
+        const int s = static_cast<int>(k % kDualStages);
+        const uint32_t u = static_cast<uint32_t>(k / kDualStages);
         if (k >= kDualStages && !mbar_wait(&sh.sfree[s], (u - 1) & 1u)) {
           atomicExch(&sh.abort_flag, 1);
           break;
         }
         if (*reinterpret_cast<volatile int*>(&sh.abort_flag)) break;
         uint32_t rt, ct;
-        tg.coords(static_cast<uint32_t>(t), rt, ct);
+        tg.coords(static_cast<uint32_t>(blockIdx.x + k * step), rt, ct);
         const int32_t x = static_cast<int32_t>(ct * kTile), y = static_cast<int32_t>(rt * kTile);
         mbar_arrive_expect_tx(&sh.full[s], kTileBytes);
         uint8_t* dst = a_tiles + s * kTileBytes;
@@ -550,100 +592,107 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
       constexpr uint32_t idesc_r = idesc_bf16_f32(kTile, kTile, 0u);
       constexpr uint32_t idesc_c = idesc_bf16_f32(kTile, kTile, 1u);
       const uint32_t br_addr = smem_u32(b_r), bc_addr = smem_u32(b_c);
-      int k = 0;
-      for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++k) {
-        const int s = k % kDualStages, a = k % kDualGroups;
-        const uint32_t use = k / kDualGroups;
-        if (!mbar_wait(&sh.full[s], (k / kDualStages) & 1u)) {
-          atomicExch(&sh.abort_flag, 1);
-          break;
-        }
-        if (use > 0 && !mbar_wait(&sh.tfree[a], (use - 1) & 1u)) {
+      int64_t j = 0;  // running accumulator index: slot j % 4, use j / 4
+      for (int64_t k = 0; k < my_tiles && !*reinterpret_cast<volatile int*>(&sh.abort_flag); ++k) {
+        const int s = static_cast<int>(k % kDualStages);
+        if (!mbar_wait(&sh.full[s], static_cast<uint32_t>(k / kDualStages) & 1u)) {
           atomicExch(&sh.abort_flag, 1);
           break;
         }
         tc_fence_after_sync();
         const uint32_t a_addr = smem_u32(a_tiles + s * kTileBytes);
-        const uint32_t d_r = tmem_base + a * 256, d_c = d_r + 128;
-        if (g_r != 0) {
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(a_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(br_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
-            umma_bf16(d_r, adesc, bdesc, idesc_r, kk > 0 ? 1u : 0u);
+        bool ok = true;
+        for (int v = 0; v < views; ++v, ++j) {
+          const int a = static_cast<int>(j % kDualSlots);
+          const uint32_t use = static_cast<uint32_t>(j / kDualSlots);
+          if (use > 0 && !mbar_wait(&sh.tfree[a], (use - 1) & 1u)) {
+            atomicExch(&sh.abort_flag, 1);
+            ok = false;
+            break;
           }
-        }
+          tc_fence_after_sync();
+          const uint32_t d = tmem_base + a * kTile;
+          if (v == 0 && views == 2) {
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint64_t adesc = smem_desc_sw128(a_addr + kk * 2048, kBoxBytes, 1024);
-          const uint64_t bdesc = smem_desc_sw128(bc_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
-          umma_bf16(d_c, adesc, bdesc, idesc_c, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t adesc = smem_desc_sw128(a_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+              const uint64_t bdesc = smem_desc_sw128(br_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+              umma_bf16(d, adesc, bdesc, idesc_r, kk > 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t adesc = smem_desc_sw128(a_addr + kk * 2048, kBoxBytes, 1024);
+              const uint64_t bdesc = smem_desc_sw128(bc_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+              umma_bf16(d, adesc, bdesc, idesc_c, kk > 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&sh.tfull[a]);
+          sh.issued_mma = (sh.issued_mma & ~(0x101u << a)) | (1u << a) | ((use & 1u) << (8 + a));
         }
+        if (!ok) break;
         umma_commit(&sh.sfree[s]);
-        umma_commit(&sh.tfull[a]);
-        sh.issued_mma = (sh.issued_mma & ~(0x101u << a)) | (1u << a) | ((use & 1u) << (8 + a));
       }
     }
   } else {
-    const uint32_t q = warp & 3u, j = (warp >> 2) & 1u, grp = warp >> 3;
-    const float c = rht_scale_of(j == 0 ? g_r : g_c);
-    const float2 c2 = f2(c, c);
-    float m = 0.0f;
-    int k = static_cast<int>(grp);
-    if (j == 0 && g_r == 0) {
-      // max|x| of the staged tile: 128 threads, 256 bytes each (the order of
-      // the swizzled bytes does not matter to a maximum); bf16 -> f32 is exact
-      const uint32_t part = (warp & 3u) * 32u + lane;
-      for (int64_t t = blockIdx.x + grp * step; t < n_tiles; t += kDualGroups * step, k += kDualGroups) {
-        const int s = k % kDualStages;
-        if (!mbar_wait(&sh.full[s], (k / kDualStages) & 1u)) {
+    // epilogue: slot `slot`, lane quarter q
+    const uint32_t q = warp & 3u, slot = warp >> 2;
+    float m_r = 0.0f, m_c = 0.0f;  // max |acc| (unscaled) of the row and column views; max |x| from smem
+    const int64_t n_acc = my_tiles * views;
+    const uint32_t part = q * 32u + lane;
+    for (int64_t j = slot; j < n_acc; j += kDualSlots) {
+      const int64_t k = j / views;
+      const int v = static_cast<int>(j % views);
+      if (row_from_smem) {
+        // max|x| of the staged tile for the row view: 128 threads, 256 bytes
+        // each (the order of the swizzled bytes does not matter to a
+        // maximum); bf16 -> f32 is exact
+        const int s = static_cast<int>(k % kDualStages);
+        if (!mbar_wait(&sh.full[s], static_cast<uint32_t>(k / kDualStages) & 1u)) {
           atomicExch(&sh.abort_flag, 1);
           break;
         }
         const uint4* src = reinterpret_cast<const uint4*>(a_tiles + s * kTileBytes) + part;
-        uint32_t bmax = 0;  // max of |x| as bf16 bit patterns (monotone for non-negative values)
+        uint32_t bmax = 0;  // max of |x| as bf16 bit-pattern pairs (monotone for non-negative values)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const uint4 w4 = src[i * 128];
-          const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) bmax = max(bmax, max(w[e] & 0x7FFFu, (w[e] >> 16) & 0x7FFFu));
+          bmax = __vmaxu2(bmax, __vmaxu2(__vmaxu2(w4.x & 0x7FFF7FFFu, w4.y & 0x7FFF7FFFu),
+                                         __vmaxu2(w4.z & 0x7FFF7FFFu, w4.w & 0x7FFF7FFFu)));
         }
-        m = fmaxf(m, __uint_as_float(bmax << 16));
+        m_r = fmaxf(m_r, __uint_as_float(max(bmax & 0xFFFFu, bmax >> 16) << 16));
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.sfree[s]);
       }
-    } else {
-    for (int64_t t = blockIdx.x + grp * step; t < n_tiles; t += kDualGroups * step, k += kDualGroups) {
-      if (!mbar_wait(&sh.tfull[grp], (k / kDualGroups) & 1u)) {
+      if (!mbar_wait(&sh.tfull[slot], static_cast<uint32_t>(j / kDualSlots) & 1u)) {
         atomicExch(&sh.abort_flag, 1);
         break;
       }
       tc_fence_after_sync();
-      const uint32_t base = tmem_base + ((32u * q) << 16) + grp * 256 + j * 128;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float v[64];
-        tmem_ld64_wait(base + 64 * h, v);
-        if (h == 1) {
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.tfree[grp]);
-        }
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          float2 zp[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) zp[i] = mul2_rn(f2(v[32 * p + 2 * i], v[32 * p + 2 * i + 1]), c2);
-          float ma, mb;
-          absmax_pair(zp, ma, mb);
-          m = fmaxf(m, fmaxf(ma, mb));
-        }
+      const uint32_t base = tmem_base + ((32u * q) << 16) + slot * kTile;
+      float m = 0.0f;
+      {
+        float v0[64];
+        tmem_ld64_wait(base, v0);
+        m = absmax64(v0, m);
       }
+      {
+        float v1[64];
+        tmem_ld64_wait(base + 64, v1);
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.tfree[slot]);
+        m = absmax64(v1, m);
+      }
+      if (v == 0 && views == 2) m_r = fmaxf(m_r, m);
+      else m_c = fmaxf(m_c, m);
     }
+    const unsigned int br = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m_r));
+    const unsigned int bc = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m_c));
+    if (lane == 0) {
+      sh.warp_max[0][warp] = br;
+      sh.warp_max[1][warp] = bc;
     }
-    const unsigned int bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
-    if (lane == 0) sh.warp_max[j][warp] = bits;
   }
 
   __syncthreads();
@@ -653,19 +702,303 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
       for (int s = 0; s < kDualStages; ++s)
         if ((sh.issued_a >> s) & 1u) mbar_wait(&sh.full[s], (sh.issued_a >> (8 + s)) & 1u);
     if (tid == kDualMmaWarp * 32)
-      for (int a = 0; a < kDualGroups; ++a)
+      for (int a = 0; a < kDualSlots; ++a)
         if ((sh.issued_mma >> a) & 1u) mbar_wait(&sh.tfull[a], (sh.issued_mma >> (8 + a)) & 1u);
   }
   if (tid == 0) {
     unsigned int mr = 0, mc = 0;
 #pragma unroll
     for (int w = 0; w < kDualEpiWarps; ++w) {
-      // warps with (w >> 2) odd read the column view
-      if (((w >> 2) & 1) == 0) mr = max(mr, sh.warp_max[0][w]);
-      else mc = max(mc, sh.warp_max[1][w]);
+      mr = max(mr, sh.warp_max[0][w]);
+      mc = max(mc, sh.warp_max[1][w]);
     }
-    atomicMax(amax_r, failed ? 0x7FC00000u : mr);
-    atomicMax(amax_c, failed ? 0x7FC00000u : mc);
+    // one rounding of the largest magnitude by the rotation constant (the
+    // row view read from shared memory is x itself)
+    const float cr = row_from_smem ? 1.0f : rht_scale_of(g_r), cc = rht_scale_of(g_c);
+    const unsigned int sr = __float_as_uint(__fmul_rn(__uint_as_float(mr), cr));
+    const unsigned int sc = __float_as_uint(__fmul_rn(__uint_as_float(mc), cc));
+    atomicMax(amax_r, failed ? 0x7FC00000u : sr);
+    atomicMax(amax_c, failed ? 0x7FC00000u : sc);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kDualMmaWarp) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ------------------------------------------------ both layouts' quantization
+// One read of X for both views' codes and scales (given both tensor amaxes):
+// the pre-pass structure above -- four accumulator slots, per-slot barriers,
+// the row view's MMA against B_r when it is rotated (G_R > 0) and the column
+// view's MN-major MMA against B_c -- with quantizing epilogues.  A slot's four
+// warps quantize the view held in it (quantize_tmem_row, the code path of the
+// single-layout kernel); with G_R = 0 they also quantize the row view straight
+// from the staged tile (quantize_smem_row) before releasing its stage.  The
+// outputs equal those of two single-layout calls bit for bit: the same MMAs
+// give the same rotated values and the same per-pair arithmetic follows.
+// `reverse` walks the tiles from the last one back, so that a launch right
+// after the pre-pass starts on the tiles the pre-pass read last (still in L2).
+
+// Quantize row r of the staged 128 x 128 tile (two 64-column boxes, 128-byte
+// swizzle): view row vrow, view columns vcol_base .. +127, no rotation.
+template <int MODE>
+__device__ __forceinline__ void quantize_smem_row(const uint8_t* tile, uint32_t r, const ScaleCtx& sc, PhiloxKey key,
+                                                  int64_t vrow, int64_t vcol_base, int64_t vrows, int64_t vcols,
+                                                  bool codes_aligned16, bool scales_aligned4, uint8_t* codes,
+                                                  uint8_t* scales) {
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    const int64_t vcol0 = vcol_base + 64 * h;
+    const bool valid = vrow < vrows && vcol0 < vcols;
+    const uint64_t e0 = static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols) + static_cast<uint64_t>(vcol0);
+    const uint8_t* rowp = tile + h * kBoxBytes + r * 128u;
+    BlockOut o[4];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      // block a = columns 32p .. 32p+15 (16-byte chunks 4p, 4p+1), block b =
+      // columns 32p+16 .. 32p+31 (chunks 4p+2, 4p+3)
+      uint32_t wa[8], wb[8];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const uint4 ua = *reinterpret_cast<const uint4*>(rowp + (((4u * p + c) ^ (r & 7u)) << 4));
+        const uint4 ub = *reinterpret_cast<const uint4*>(rowp + (((4u * p + 2u + c) ^ (r & 7u)) << 4));
+        wa[4 * c] = ua.x; wa[4 * c + 1] = ua.y; wa[4 * c + 2] = ua.z; wa[4 * c + 3] = ua.w;
+        wb[4 * c] = ub.x; wb[4 * c + 1] = ub.y; wb[4 * c + 2] = ub.z; wb[4 * c + 3] = ub.w;
+      }
+      float2 z[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float a0, a1, b0, b1;
+        bf16x2_to_f32(wa[i], a0, a1);
+        bf16x2_to_f32(wb[i], b0, b1);
+        z[2 * i] = f2(a0, b0);
+        z[2 * i + 1] = f2(a1, b1);
+      }
+      const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, 0.0f, 0.0f};
+      quantize_pair<MODE>(z, sc, rng, o[2 * p], o[2 * p + 1]);
+    }
+    if (valid) store64(o, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);
+  }
+}
+
+struct DualQuantShared {
+  uint64_t full[kDualStages];
+  uint64_t sfree[kDualStages];
+  uint64_t tfull[kDualSlots];
+  uint64_t tfree[kDualSlots];
+  uint32_t tmem_base;
+  uint32_t issued_a;
+  uint32_t issued_mma;
+  int abort_flag;
+  float4 scale_tbl[2][128];   // the launch's block-scale constants per E4M3 code, row and column view
+};
+
+#ifndef NVFP4_DUALQ_BAND_ROWS
+#define NVFP4_DUALQ_BAND_ROWS 1
+#endif
+
+template <int MODE_R, int G_R, int MODE_C, int G_C>
+__global__ void __launch_bounds__(kDualThreads, 1)
+dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed,
+                     const float* __restrict__ amax_r, const float* __restrict__ amax_c,
+                     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ scales_r, float* __restrict__ gscale_r,
+                     uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c, float* __restrict__ gscale_c,
+                     int reverse) {
+  static_assert(G_C > 0, "the column view is rotated on the tensor cores");
+  constexpr int kViews = G_R != 0 ? 2 : 1;
+  constexpr bool kRowFromSmem = G_R == 0;
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ __align__(16) DualQuantShared sh;
+  uint8_t* a_tiles = align_1024(dyn_smem);
+  uint8_t* b_r = a_tiles + kDualStages * kTileBytes;
+  uint8_t* b_c = b_r + kTileBytes;
+
+  const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+  const PhiloxKey key = philox_key(seed);
+  const TileGrid tg{static_cast<uint32_t>((rows + kTile - 1) / kTile), static_cast<uint32_t>((cols + kTile - 1) / kTile),
+                    static_cast<uint32_t>(NVFP4_DUALQ_BAND_ROWS)};
+  const int64_t n_tiles = static_cast<int64_t>(tg.n_rt) * tg.n_ct;
+  const int64_t step = gridDim.x;
+  const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - blockIdx.x + step - 1) / step : 0;
+  // tile k of this CTA
+  auto tile_of = [&](int64_t k) -> uint32_t {
+    const int64_t t = blockIdx.x + k * step;
+    return static_cast<uint32_t>(reverse ? n_tiles - 1 - t : t);
+  };
+
+  if (tid == kDualProducerWarp * 32) {
+    for (int s = 0; s < kDualStages; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.sfree[s], kRowFromSmem ? 5 : 1);
+    }
+    for (int a = 0; a < kDualSlots; ++a) {
+      mbar_init(&sh.tfull[a], 1);
+      mbar_init(&sh.tfree[a], 4);
+    }
+    sh.issued_a = 0;
+    sh.issued_mma = 0;
+    sh.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kDualMmaWarp) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = sh.tmem_base;
+  if (warp != kDualProducerWarp) {
+    const uint32_t bt = warp < kDualProducerWarp ? tid : tid - 32, nb = kDualThreads - 32;
+    if constexpr (G_R != 0) build_hadamard_b<G_R>(b_r, key, bt, nb);
+    build_hadamard_b<G_C>(b_c, key, bt, nb);
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 2, %0;" ::"r"(nb) : "memory");
+  }
+
+  if (warp == kDualProducerWarp) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmap);
+      for (int64_t k = 0; k < my_tiles; ++k) {
+        const int s = static_cast<int>(k % kDualStages);
+        const uint32_t u = static_cast<uint32_t>(k / kDualStages);
+        if (k >= kDualStages && !mbar_wait(&sh.sfree[s], (u - 1) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        if (*reinterpret_cast<volatile int*>(&sh.abort_flag)) break;
+        uint32_t rt, ct;
+        tg.coords(tile_of(k), rt, ct);
+        const int32_t x = static_cast<int32_t>(ct * kTile), y = static_cast<int32_t>(rt * kTile);
+        mbar_arrive_expect_tx(&sh.full[s], kTileBytes);
+        uint8_t* dst = a_tiles + s * kTileBytes;
+        tma_load_2d(dst, &tmap, x, y, &sh.full[s]);
+        tma_load_2d(dst + kBoxBytes, &tmap, x + 64, y, &sh.full[s]);
+        sh.issued_a = (sh.issued_a & ~(0x101u << s)) | (1u << s) | ((u & 1u) << (8 + s));
+      }
+    }
+  } else if (warp == kDualMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_r = idesc_bf16_f32(kTile, kTile, 0u);
+      constexpr uint32_t idesc_c = idesc_bf16_f32(kTile, kTile, 1u);
+      const uint32_t br_addr = smem_u32(b_r), bc_addr = smem_u32(b_c);
+      int64_t j = 0;
+      for (int64_t k = 0; k < my_tiles && !*reinterpret_cast<volatile int*>(&sh.abort_flag); ++k) {
+        const int s = static_cast<int>(k % kDualStages);
+        if (!mbar_wait(&sh.full[s], static_cast<uint32_t>(k / kDualStages) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t a_addr = smem_u32(a_tiles + s * kTileBytes);
+        bool ok = true;
+#pragma unroll
+        for (int v = 0; v < kViews; ++v) {
+          const int a = static_cast<int>(j % kDualSlots);
+          const uint32_t use = static_cast<uint32_t>(j / kDualSlots);
+          ++j;
+          if (use > 0 && !mbar_wait(&sh.tfree[a], (use - 1) & 1u)) {
+            atomicExch(&sh.abort_flag, 1);
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t d = tmem_base + a * kTile;
+          if (kViews == 2 && v == 0) {
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t adesc = smem_desc_sw128(a_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+              const uint64_t bdesc = smem_desc_sw128(br_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+              umma_bf16(d, adesc, bdesc, idesc_r, kk > 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t adesc = smem_desc_sw128(a_addr + kk * 2048, kBoxBytes, 1024);
+              const uint64_t bdesc = smem_desc_sw128(bc_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+              umma_bf16(d, adesc, bdesc, idesc_c, kk > 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&sh.tfull[a]);
+          sh.issued_mma = (sh.issued_mma & ~(0x101u << a)) | (1u << a) | ((use & 1u) << (8 + a));
+        }
+        if (!ok) break;
+        umma_commit(&sh.sfree[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t q = warp & 3u, slot = warp >> 2;
+    ScaleCtx sc_r = make_scale_ctx<MODE_R>(*amax_r);
+    ScaleCtx sc_c = make_scale_ctx<MODE_C>(*amax_c);
+    build_scale_table(sh.scale_tbl[0], sc_r.s_g, tid, kDualEpiWarps * 32);
+    build_scale_table(sh.scale_tbl[1], sc_c.s_g, tid, kDualEpiWarps * 32);
+    asm volatile("bar.sync 1, %0;" ::"r"(kDualEpiWarps * 32) : "memory");
+    sc_r.tbl = sh.scale_tbl[0];
+    sc_c.tbl = sh.scale_tbl[1];
+    if (blockIdx.x == 0 && tid == 0) {
+      *gscale_r = sc_r.s_g;
+      *gscale_c = sc_c.s_g;
+    }
+    // row view: rows x cols; column view: cols x rows
+    const bool r_codes16 = ((cols / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes_r) % 16) == 0;
+    const bool r_scales4 = ((cols / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales_r) % 4) == 0;
+    const bool c_codes16 = ((rows / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes_c) % 16) == 0;
+    const bool c_scales4 = ((rows / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales_c) % 4) == 0;
+    const bool r_blocks8 = ((cols / 16) % 8) == 0, c_blocks8 = ((rows / 16) % 8) == 0;
+    const int64_t n_acc = my_tiles * kViews;
+    const uint32_t r_in_tile = 32u * q + lane;
+    for (int64_t j = slot; j < n_acc; j += kDualSlots) {
+      const int64_t k = j / kViews;
+      const int v = static_cast<int>(j % kViews);
+      uint32_t rt, ct;
+      tg.coords(tile_of(k), rt, ct);
+      if constexpr (kRowFromSmem) {
+        const int s = static_cast<int>(k % kDualStages);
+        if (!mbar_wait(&sh.full[s], static_cast<uint32_t>(k / kDualStages) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        quantize_smem_row<MODE_R>(a_tiles + s * kTileBytes, r_in_tile, sc_r, key,
+                                  static_cast<int64_t>(rt) * kTile + r_in_tile, static_cast<int64_t>(ct) * kTile, rows,
+                                  cols, r_codes16, r_scales4, codes_r, scales_r);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.sfree[s]);
+      }
+      if (!mbar_wait(&sh.tfull[slot], static_cast<uint32_t>(j / kDualSlots) & 1u)) {
+        atomicExch(&sh.abort_flag, 1);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t base = tmem_base + ((32u * q) << 16) + slot * kTile;
+      if (kViews == 2 && v == 0) {
+        if constexpr (G_R != 0)
+          quantize_tmem_row<MODE_R, (G_R != 0 ? G_R : 16)>(
+              base, &sh.tfree[slot], sc_r, key, static_cast<int64_t>(rt) * kTile + r_in_tile,
+              static_cast<int64_t>(ct) * kTile, rows, cols, r_blocks8, r_codes16, r_scales4, codes_r, scales_r);
+      } else {
+        quantize_tmem_row<MODE_C, G_C>(base, &sh.tfree[slot], sc_c, key, static_cast<int64_t>(ct) * kTile + r_in_tile,
+                                       static_cast<int64_t>(rt) * kTile, cols, rows, c_blocks8, c_codes16, c_scales4,
+                                       codes_c, scales_c);
+      }
+    }
+  }
+
+  __syncthreads();
+  const bool failed = *reinterpret_cast<volatile int*>(&sh.abort_flag) != 0;
+  if (failed) {
+    if (tid == kDualProducerWarp * 32)
+      for (int s = 0; s < kDualStages; ++s)
+        if ((sh.issued_a >> s) & 1u) mbar_wait(&sh.full[s], (sh.issued_a >> (8 + s)) & 1u);
+    if (tid == kDualMmaWarp * 32)
+      for (int a = 0; a < kDualSlots; ++a)
+        if ((sh.issued_mma >> a) & 1u) mbar_wait(&sh.tfull[a], (sh.issued_mma >> (8 + a)) & 1u);
+    if (tid == 0) {
+      *gscale_r = __uint_as_float(0x7FC00000u);
+      *gscale_c = __uint_as_float(0x7FC00000u);
+    }
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -792,6 +1125,51 @@ cudaError_t launch_amax_dual_mma(const void* x, int64_t rows, int64_t cols, int6
       map, rows, cols, seed, g_r, g_c, reinterpret_cast<unsigned int*>(amax_r),
       reinterpret_cast<unsigned int*>(amax_c));
   return cudaGetLastError();
+}
+
+namespace {
+
+template <int MODE_R, int G_R, int MODE_C, int G_C>
+cudaError_t launch_dual_quantize_t(const DualQuantArgs& a) {
+  CUtensorMap map;
+  if (!make_map(&map, a.x, a.rows, a.cols, a.ld)) return cudaErrorInvalidValue;
+  auto kernel = dual_quantize_kernel<MODE_R, G_R, MODE_C, G_C>;
+  LaunchGeom geom;
+  cudaError_t e = launch_geometry(kernel, kDualThreads, kDualDynSmem, 1, &geom);
+  if (e != cudaSuccess) return e;
+  const int64_t n_tiles = ((a.rows + kTile - 1) / kTile) * ((a.cols + kTile - 1) / kTile);
+  const int64_t grid = n_tiles < int64_t(geom.sms) ? n_tiles : int64_t(geom.sms);
+  if (grid == 0) return cudaSuccess;
+  kernel<<<static_cast<unsigned>(grid), kDualThreads, kDualDynSmem, a.stream>>>(
+      map, a.rows, a.cols, a.seed, a.amax_row, a.amax_col, a.codes_row, a.scales_row, a.gscale_row, a.codes_col,
+      a.scales_col, a.gscale_col, a.reverse);
+  return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t dispatch_dual_quantize(const DualQuantArgs& a) {
+  if (a.mode_row == kRTN && a.rht_group_row == 0) return launch_dual_quantize_t<kRTN, 0, kMSEDEN, G>(a);
+  return launch_dual_quantize_t<kMSEDEN, G, kMSEDEN, G>(a);
+}
+
+}  // namespace
+
+bool dual_quantize_fused(const DualQuantArgs& a) {
+  if (!dual_mma_path_applies(a.x, a.rows, a.cols, a.ld)) return false;
+  const int g = a.rht_group_col;
+  if (a.mode_col != kMSEDEN || (g != 16 && g != 32 && g != 64 && g != 128)) return false;
+  if (a.mode_row == kRTN && a.rht_group_row == 0) return true;
+  return a.mode_row == kMSEDEN && a.rht_group_row == g;
+}
+
+cudaError_t launch_quantize_dual_mma(const DualQuantArgs& a) {
+  switch (a.rht_group_col) {
+    case 16: return dispatch_dual_quantize<16>(a);
+    case 32: return dispatch_dual_quantize<32>(a);
+    case 64: return dispatch_dual_quantize<64>(a);
+    case 128: return dispatch_dual_quantize<128>(a);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace nvfp4

@@ -18,9 +18,11 @@ CFLAGS = ["-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast
 def build(force: bool = False) -> str:
     if not force and os.path.exists(OUT) and os.path.getmtime(OUT) >= os.path.getmtime(SRC):
         return OUT
-    cmd = ["gcc", *CFLAGS, SRC, "-o", OUT + ".tmp", "-lm"]
+    # a private temporary name: several processes may build at once
+    tmp = f"{OUT}.{os.getpid()}.tmp"
+    cmd = ["gcc", *CFLAGS, SRC, "-o", tmp, "-lm"]
     subprocess.run(cmd, check=True)
-    os.replace(OUT + ".tmp", OUT)
+    os.replace(tmp, OUT)
     return OUT
 
 

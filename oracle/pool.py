@@ -147,6 +147,19 @@ class OraclePool:
         self._n += 1
         return os.path.join(self._dir, f"{tag}_{self._n}.bin")
 
+    def put(self, a):
+        """Share an input array with the workers once; the handle can be
+        passed to the methods below in place of the array (saves writing
+        the same tensor again for every call on it)."""
+        return SharedArray(self._share(a, "in"), np.ascontiguousarray(a).dtype, np.shape(a))
+
+    def _input(self, a, dtype, tag):
+        """(path, shape, owned) of an input given as an array or a SharedArray."""
+        if isinstance(a, SharedArray):
+            return a.path, a.shape, False
+        a = np.ascontiguousarray(a, dtype=dtype)
+        return self._share(a, tag), a.shape, True
+
     def _share(self, a, tag):
         a = np.ascontiguousarray(a)
         path = self._path(tag)
@@ -179,49 +192,48 @@ class OraclePool:
     # the oracle, in pieces ---------------------------------------------------
     def amax(self, x_bits, layout, g, seed):
         """oracle.amax of the whole view: the largest of the pieces' amaxes."""
-        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
-        rows, cols = x.shape
-        if x.size == 0:
+        xpath, (rows, cols), owned = self._input(x_bits, np.uint16, "x")
+        if rows * cols == 0:
+            if owned:
+                os.unlink(xpath)
             return 0.0
-        xpath = self._share(x, "x")
         # row-wise: pieces of x rows; transposed: pieces of x columns (whole
         # view rows), 8-aligned as the transposed layout requires
         n = rows if layout == 0 else cols
         futs = [self._ex.submit(_w_amax, xpath, (rows, cols), layout, g, seed, b, e)
                 for b, e in self._ranges(n, 1 if layout == 0 else 8)]
         a = max(f.result() for f in futs)
-        os.unlink(xpath)
+        if owned:
+            os.unlink(xpath)
         return a
 
     def quantize(self, x_bits, layout, mode, g, seed, amax_in, row_range=None):
         """oracle.quantize(x_bits, layout, mode, g, seed, amax_in, row_range) in pieces."""
-        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
-        rows, cols = x.shape
+        xpath, (rows, cols), owned = self._input(x_bits, np.uint16, "x")
         vr, vc = (rows, cols) if layout == 0 else (cols, rows)
         b0, e0 = (0, vr) if row_range is None else row_range
-        xpath = self._share(x, "x")
         cpath = self._zeros(np.uint8, (vr, vc // 2), "codes")
         spath = self._zeros(np.uint8, (vr, vc // 16), "scales")
         futs = [self._ex.submit(_w_quantize, xpath, (rows, cols), layout, mode, g, seed, float(amax_in),
                                 b0 + b, b0 + e, cpath, spath, vr, vc) for b, e in self._ranges(e0 - b0)]
         gs = [f.result() for f in futs]
-        os.unlink(xpath)
+        if owned:
+            os.unlink(xpath)
         codes = self._collect(cpath, np.uint8, (vr, vc // 2))
         scales = self._collect(spath, np.uint8, (vr, vc // 16))
         return codes, scales, gs[0] if gs else _global_scale(amax_in, mode)
 
     def rht_view(self, x_bits, layout, g, seed):
         """oracle.rht_view in pieces of view rows."""
-        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
-        rows, cols = x.shape
+        xpath, (rows, cols), owned = self._input(x_bits, np.uint16, "x")
         vr, vc = (rows, cols) if layout == 0 else (cols, rows)
-        xpath = self._share(x, "x")
         zpath = self._zeros(np.float32, (vr, vc), "z")
         futs = [self._ex.submit(_w_rht_view, xpath, (rows, cols), layout, g, seed, b, e, zpath, vr, vc)
                 for b, e in self._ranges(vr, 1 if layout == 0 else 8)]
         for f in futs:
             f.result()
-        os.unlink(xpath)
+        if owned:
+            os.unlink(xpath)
         return self._collect(zpath, np.float32, (vr, vc))
 
     def quantize_rotated(self, z, mode, seed, amax):
@@ -238,6 +250,13 @@ class OraclePool:
         codes = self._collect(cpath, np.uint8, (vr, vc // 2))
         scales = self._collect(spath, np.uint8, (vr, vc // 16))
         return codes, scales, gs[0] if gs else _global_scale(amax, mode)
+
+
+class SharedArray:
+    """An input array already written for the workers (OraclePool.put)."""
+
+    def __init__(self, path, dtype, shape):
+        self.path, self.dtype, self.shape = path, dtype, tuple(shape)
 
 
 def _w_ready_n(_):

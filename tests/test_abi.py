@@ -34,7 +34,7 @@ def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ["nvfp4_quantize", "nvfp4_dequantize", "nvfp4_rht", "nvfp4_amax", "nvfp4_workspace_bytes",
               "nvfp4_status_string", "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_quantize_noalloc",
-              "nvfp4_amax_dual", "nvfp4_gemm"]:
+              "nvfp4_amax_dual", "nvfp4_gemm", "nvfp4_quantize_dual"]:
         assert n in names
 
 
@@ -106,6 +106,31 @@ def test_noalloc_rejects_like_quantize(N):
     assert nq(FAKE, 64, 64, 64, 2, 0, 0, 0, None, FAKE, FAKE, FAKE, None) == INVALID   # layout
     assert nq(FAKE, 64, 64, 64, 0, 0, 48, 0, None, FAKE, FAKE, FAKE, None) == INVALID  # group
     assert nq(FAKE, 64, 64, 64, 0, 12, 0, 0, None, FAKE, FAKE, FAKE, None) == INVALID  # mode
+
+
+def qd(N, x=FAKE, rows=256, cols=256, ld=256, mr=0, gr=0, mc=2, gc=128, ar=FAKE, ac=FAKE, outs=None):
+    o = outs if outs is not None else (FAKE + 0x1000, FAKE + 0x2000, FAKE + 0x3000, FAKE + 0x4000, FAKE + 0x5000,
+                                       FAKE + 0x6000)
+    return N.nvfp4_quantize_dual(x, rows, cols, ld, mr, gr, mc, gc, 0, ar, ac, *o, None)
+
+
+def test_quantize_dual_rejects(N):
+    assert qd(N, x=None) == INVALID
+    assert qd(N, mr=12) == INVALID
+    assert qd(N, gr=48) == INVALID
+    assert qd(N, mr=2, gr=0) == UNSUPPORTED          # MS-EDEN needs the rotation, in either view
+    assert qd(N, mc=2, gc=0) == UNSUPPORTED
+    assert qd(N, cols=40, ld=40) == SHAPE            # row view: cols % 16
+    assert qd(N, rows=40) == SHAPE                   # column view: rows % 16
+    assert qd(N, rows=64, gc=128) == SHAPE           # column view: rows % g
+    assert qd(N, mc=6, gc=0, rows=48) == SHAPE       # MXFP4 column view: whole 32-element groups
+    assert qd(N, ar=None) == INVALID                 # the row view's amax is required (not an MX mode)
+    assert qd(N, ac=None) == INVALID
+    assert qd(N, outs=(None, FAKE, FAKE, FAKE, FAKE, FAKE)) == INVALID
+    assert qd(N, outs=(FAKE, FAKE, FAKE, FAKE, FAKE, None)) == INVALID
+    assert qd(N, outs=(FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE)) == ALIGN
+    assert qd(N, x=FAKE + 8) == ALIGN
+    assert qd(N, ar=FAKE + 2) == ALIGN
 
 
 def test_other_entry_points_reject(N):

@@ -106,7 +106,7 @@ def _check_call(pool, wl, call, x, xb):
 
 def _check_workload(pool, wl):
     tensors = wl.tensors("cuda")
-    host = {k: bits(v) for k, v in tensors.items()}
+    host = {k: pool.put(bits(v)) for k, v in tensors.items()}   # each tensor written once for the workers
     for call in wl.calls:
         _check_call(pool, wl, call, tensors[call.tensor], host[call.tensor])
 

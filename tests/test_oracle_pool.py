@@ -41,6 +41,17 @@ def test_pool_matches_oracle(pool, layout, mode, g):
         assert np.array_equal(got_r[0], exp_r[0]) and np.array_equal(got_r[1], exp_r[1])
 
 
+def test_pool_shared_input(pool):
+    xb = _x(128, 256, 4)
+    h = pool.put(xb)
+    a = oracle.amax(xb, W.TRANSPOSED, 64, 2)
+    assert pool.amax(h, W.TRANSPOSED, 64, 2) == a
+    exp = oracle.quantize(xb, W.TRANSPOSED, W.MS_EDEN, 64, 2, amax_in=a)
+    got = pool.quantize(h, W.TRANSPOSED, W.MS_EDEN, 64, 2, a)
+    assert np.array_equal(got[0], exp[0]) and np.array_equal(got[1], exp[1])
+    assert np.array_equal(pool.rht_view(h, W.TRANSPOSED, 64, 2), oracle.rht_view(xb, W.TRANSPOSED, 64, 2))
+
+
 def test_pool_row_range(pool):
     xb = _x(96, 256, 3)
     a = oracle.amax(xb, W.ROWWISE, 0, 5)
