@@ -295,6 +295,29 @@ NVFP4_API int nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, 
 NVFP4_API int nvfp4_encode_e2m1(const float* in, int64_t n, uint8_t* out, void* stream);
 NVFP4_API int nvfp4_encode_e4m3(const float* in, int64_t n, int round_up, uint8_t* out, void* stream);
 
+/* Packed storage of the 3-bit formats (IF4 paper page, the 3-bit formats
+ * table: 3.5 bits per value for NVFP3, NVINT3 and IF3 -- 3-bit elements and
+ * an 8-bit scale per 16 -- and 3.25 for MXFP3 -- one 8-bit scale per 32).
+ * nvfp4_quantize holds a 3-bit code in a nibble (sign bit 3, magnitude code
+ * bits 0..1, bit 2 clear); nvfp4_pack3 keeps 3 bits of it: the 16 codes of a
+ * block in 6 bytes, element i in bits 3i .. 3i+2 of the block's 48-bit
+ * little-endian field (bit 3i+2 the sign, bits 3i .. 3i+1 the magnitude code).
+ *  codes, scales:   a quantized view as nvfp4_quantize writes it for `mode`
+ *                   (vrows x vcols/2 and vrows x vcols/16 bytes);
+ *  packed_codes:    vrows x (vcols/16) x 6 bytes, 2-byte aligned;
+ *  packed_scales:   vrows x vcols/16 bytes (E4M3 modes), or vrows x vcols/32
+ *                   (NVFP4_MXFP3: the group's byte once).
+ * nvfp4_unpack3 restores codes and scales exactly (the MXFP3 byte in both
+ * halves of its group).  mode: NVFP4_NVFP3, NVFP4_NVINT3, NVFP4_IF3 or
+ * NVFP4_MXFP3 (others: NVFP4_ERR_UNSUPPORTED).  vcols: a multiple of 16 (32
+ * for MXFP3).  Nibbles with bit 2 set (never produced by the 3-bit modes) do
+ * not survive the packing.  The layout is this library's reading: the pages
+ * give the bits per value, not a bit order. */
+NVFP4_API int nvfp4_pack3(const uint8_t* codes, const uint8_t* scales, int64_t vrows, int64_t vcols, int mode,
+                          uint8_t* packed_codes, uint8_t* packed_scales, void* stream);
+NVFP4_API int nvfp4_unpack3(const uint8_t* packed_codes, const uint8_t* packed_scales, int64_t vrows,
+                            int64_t vcols, int mode, uint8_t* codes, uint8_t* scales, void* stream);
+
 /* Static string naming a status code (never NULL). */
 NVFP4_API const char* nvfp4_status_string(int status);
 

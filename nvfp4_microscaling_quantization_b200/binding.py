@@ -62,6 +62,10 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_quantize_noalloc.restype = i32
         L.nvfp4_gemm.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, P, i64, P]
         L.nvfp4_gemm.restype = i32
+        L.nvfp4_pack3.argtypes = [P, P, i64, i64, i32, P, P, P]
+        L.nvfp4_pack3.restype = i32
+        L.nvfp4_unpack3.argtypes = [P, P, i64, i64, i32, P, P, P]
+        L.nvfp4_unpack3.restype = i32
         L.nvfp4_status_string.argtypes = [i32]
         L.nvfp4_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -120,6 +124,14 @@ def nvfp4_gemm(a_codes, a_scales, a_gscale, b_codes, b_scales, b_gscale, m, n, k
                stream) -> int:
     return lib().nvfp4_gemm(a_codes, a_scales, a_gscale, b_codes, b_scales, b_gscale, m, n, k, out_dtype, d,
                             ldd, stream)
+
+
+def nvfp4_pack3(codes, scales, vrows, vcols, mode, packed_codes, packed_scales, stream) -> int:
+    return lib().nvfp4_pack3(codes, scales, vrows, vcols, mode, packed_codes, packed_scales, stream)
+
+
+def nvfp4_unpack3(packed_codes, packed_scales, vrows, vcols, mode, codes, scales, stream) -> int:
+    return lib().nvfp4_unpack3(packed_codes, packed_scales, vrows, vcols, mode, codes, scales, stream)
 
 
 def nvfp4_encode_e2m1(x, n, out, stream) -> int:
@@ -248,6 +260,27 @@ def rht(x: torch.Tensor, layout: int = ROWWISE, rht_group: int = 128, seed: int 
     _check(nvfp4_rht(_p(x), dt, rows, cols, ld, layout, rht_group, seed, int(inverse), _p(out),
                      _stream_handle(stream)), "nvfp4_rht")
     return out
+
+
+def pack3(codes: torch.Tensor, scales: torch.Tensor, mode: int, stream=None):
+    """Packed 3-bit storage of a quantized view (NVFP3, NVINT3, IF3, MXFP3):
+    returns (packed codes [vrows, vcols/16 * 6], packed scales [vrows, vcols/16],
+    or [vrows, vcols/32] for MXFP3)."""
+    vr, vc = codes.shape[0], 2 * codes.shape[1]
+    pc = torch.empty((vr, vc // 16 * 6), dtype=torch.uint8, device=codes.device)
+    ps = torch.empty((vr, vc // (32 if mode == MXFP3 else 16)), dtype=torch.uint8, device=codes.device)
+    _check(nvfp4_pack3(_p(codes), _p(scales), vr, vc, mode, _p(pc), _p(ps), _stream_handle(stream)), "nvfp4_pack3")
+    return pc, ps
+
+
+def unpack3(packed_codes: torch.Tensor, packed_scales: torch.Tensor, vcols: int, mode: int, stream=None):
+    """Inverse of pack3: (codes [vrows, vcols/2], scales [vrows, vcols/16])."""
+    vr = packed_codes.shape[0]
+    codes = torch.empty((vr, vcols // 2), dtype=torch.uint8, device=packed_codes.device)
+    scales = torch.empty((vr, vcols // 16), dtype=torch.uint8, device=packed_codes.device)
+    _check(nvfp4_unpack3(_p(packed_codes), _p(packed_scales), vr, vcols, mode, _p(codes), _p(scales),
+                         _stream_handle(stream)), "nvfp4_unpack3")
+    return codes, scales
 
 
 def encode_e2m1(x: torch.Tensor, stream=None) -> torch.Tensor:

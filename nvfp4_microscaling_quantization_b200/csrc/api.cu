@@ -223,6 +223,35 @@ int nvfp4_encode_e4m3(const float* in, int64_t n, int round_up, uint8_t* out, vo
   return from_cuda(nvfp4::launch_encode_e4m3(in, n, round_up, out, static_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+int check_pack3(const void* a, const void* b, const void* c, const void* d, int64_t vrows, int64_t vcols, int mode) {
+  if (mode != NVFP4_NVFP3 && mode != NVFP4_NVINT3 && mode != NVFP4_IF3 && mode != NVFP4_MXFP3)
+    return NVFP4_ERR_UNSUPPORTED;
+  if (vrows < 0 || vcols < 0 || vcols % (mode == NVFP4_MXFP3 ? 32 : 16)) return NVFP4_ERR_SHAPE;
+  if (vrows == 0 || vcols == 0) return NVFP4_OK;
+  if (!a || !b || !c || !d) return NVFP4_ERR_INVALID_ARG;
+  return NVFP4_OK;
+}
+}  // namespace
+
+int nvfp4_pack3(const uint8_t* codes, const uint8_t* scales, int64_t vrows, int64_t vcols, int mode,
+                uint8_t* packed_codes, uint8_t* packed_scales, void* stream) {
+  int st = check_pack3(codes, scales, packed_codes, packed_scales, vrows, vcols, mode);
+  if (st || vrows == 0 || vcols == 0) return st;
+  if (!aligned(codes, 8) || !aligned(packed_codes, 2)) return NVFP4_ERR_ALIGNMENT;
+  return from_cuda(nvfp4::launch_pack3(codes, scales, vrows * (vcols / 16), mode == NVFP4_MXFP3, packed_codes,
+                                       packed_scales, static_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_unpack3(const uint8_t* packed_codes, const uint8_t* packed_scales, int64_t vrows, int64_t vcols, int mode,
+                  uint8_t* codes, uint8_t* scales, void* stream) {
+  int st = check_pack3(packed_codes, packed_scales, codes, scales, vrows, vcols, mode);
+  if (st || vrows == 0 || vcols == 0) return st;
+  if (!aligned(codes, 8) || !aligned(packed_codes, 2)) return NVFP4_ERR_ALIGNMENT;
+  return from_cuda(nvfp4::launch_unpack3(packed_codes, packed_scales, vrows * (vcols / 16), mode == NVFP4_MXFP3,
+                                         codes, scales, static_cast<cudaStream_t>(stream)));
+}
+
 const char* nvfp4_status_string(int status) {
   switch (status) {
     case NVFP4_OK: return "NVFP4_OK";

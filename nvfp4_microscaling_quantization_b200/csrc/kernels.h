@@ -116,6 +116,13 @@ struct GemmArgs {
 bool gemm_available();
 cudaError_t launch_gemm(const GemmArgs& g);
 cudaError_t launch_rht(const RhtArgs& a);
+// Packed 3-bit storage (pack3.cu): `blocks` 16-element blocks of nibble codes
+// (8 bytes each) <-> 6 bytes each; scales copied, or for MX (mx != 0) one
+// byte per block pair.
+cudaError_t launch_pack3(const uint8_t* codes, const uint8_t* scales, int64_t blocks, int mx, uint8_t* pcodes,
+                         uint8_t* pscales, cudaStream_t stream);
+cudaError_t launch_unpack3(const uint8_t* pcodes, const uint8_t* pscales, int64_t blocks, int mx, uint8_t* codes,
+                           uint8_t* scales, cudaStream_t stream);
 cudaError_t launch_encode_e2m1(const float* in, int64_t n, uint8_t* out, cudaStream_t stream);
 cudaError_t launch_encode_e4m3(const float* in, int64_t n, int round_up, uint8_t* out, cudaStream_t stream);
 

@@ -79,6 +79,10 @@ def _declare(L):
     L.oracle_e2m1_rtn_array.restype = None
     L.oracle_e4m3_array.argtypes = [P, i64, i32, P]
     L.oracle_e4m3_array.restype = None
+    L.oracle_pack3.argtypes = [P, P, i64, i64, i32, P, P]
+    L.oracle_pack3.restype = None
+    L.oracle_unpack3.argtypes = [P, P, i64, i64, i32, P, P]
+    L.oracle_unpack3.restype = None
 
 
 class OracleError(RuntimeError):
@@ -255,6 +259,29 @@ def dequantize(codes, scales, gscale, mode, g, seed, inverse_rht=False):
     _check(lib().oracle_dequantize(_ptr(codes), _ptr(scales), float(gscale), vr, vc, mode, g,
                                    seed, int(inverse_rht), _ptr(out)))
     return out
+
+
+def pack3(codes, scales, mode):
+    """Packed 3-bit storage of a quantized view (NVFP3, NVINT3, IF3, MXFP3):
+    (packed codes [vr, vc/16 * 6], packed scales [vr, vc/16] or [vr, vc/32] for MXFP3)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    vr, vc = codes.shape[0], codes.shape[1] * 2
+    mx = int(mode == MXFP3)
+    pc = np.zeros((vr, vc // 16 * 6), dtype=np.uint8)
+    ps = np.zeros((vr, vc // (32 if mx else 16)), dtype=np.uint8)
+    lib().oracle_pack3(_ptr(codes), _ptr(scales), vr, vc, mx, _ptr(pc), _ptr(ps))
+    return pc, ps
+
+
+def unpack3(packed, packed_scales, vcols, mode):
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    packed_scales = np.ascontiguousarray(packed_scales, dtype=np.uint8)
+    vr = packed.shape[0]
+    codes = np.zeros((vr, vcols // 2), dtype=np.uint8)
+    scales = np.zeros((vr, vcols // 16), dtype=np.uint8)
+    lib().oracle_unpack3(_ptr(packed), _ptr(packed_scales), vr, vcols, int(mode == MXFP3), _ptr(codes), _ptr(scales))
+    return codes, scales
 
 
 def unpack_codes(codes):

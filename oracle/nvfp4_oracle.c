@@ -824,6 +824,58 @@ void oracle_e4m3_array(const float* in, int64_t n, int round_up, uint8_t* out) {
     out[i] = round_up ? oracle_e4m3_ru_sat(in[i]) : oracle_e4m3_rne_sat(in[i]);
 }
 
+/* Packed storage of the 3-bit formats (a storage layout, this library's
+ * reading; [IF4-T6] fixes only the bits per value: 3 bits per element plus
+ * the scale, 3.5 for NVFP3 / NVINT3 / IF3 and 3.25 for MXFP3).  Element j of
+ * block b of a view row: its nibble code (sign bit 3, magnitude bits 0..1) is
+ * written as the 3-bit value sign * 4 + magnitude at bit 3 (j mod 16) of the
+ * block's 6 bytes, least significant bit first, one bit at a time.  Scales:
+ * copied, or for MXFP3 (mx != 0) the byte of every even block only. */
+void oracle_pack3(const uint8_t* codes, const uint8_t* scales, int64_t vr, int64_t vc, int mx,
+                  uint8_t* packed, uint8_t* packed_scales) {
+  const int64_t nb = vc / 16;
+  for (int64_t r = 0; r < vr; ++r) {
+    for (int64_t b = 0; b < nb; ++b) {
+      uint8_t* dst = packed + (r * nb + b) * 6;
+      for (int k = 0; k < 6; ++k) dst[k] = 0;
+      for (int j = 0; j < 16; ++j) {
+        const int64_t e = b * 16 + j;
+        const uint8_t byte = codes[r * (vc / 2) + e / 2];
+        const uint8_t nib = (e % 2) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15u);
+        const unsigned v3 = (unsigned)(nib & 3u) + ((nib & 8u) ? 4u : 0u);
+        for (int t = 0; t < 3; ++t) {
+          const int bit = 3 * j + t;
+          if ((v3 >> t) & 1u) dst[bit / 8] = (uint8_t)(dst[bit / 8] | (1u << (bit % 8)));
+        }
+      }
+      if (!mx) packed_scales[r * nb + b] = scales[r * nb + b];
+      else if (b % 2 == 0) packed_scales[r * (nb / 2) + b / 2] = scales[r * nb + b];
+    }
+  }
+}
+
+void oracle_unpack3(const uint8_t* packed, const uint8_t* packed_scales, int64_t vr, int64_t vc, int mx,
+                    uint8_t* codes, uint8_t* scales) {
+  const int64_t nb = vc / 16;
+  for (int64_t r = 0; r < vr; ++r) {
+    for (int64_t b = 0; b < nb; ++b) {
+      const uint8_t* src = packed + (r * nb + b) * 6;
+      for (int j = 0; j < 16; ++j) {
+        unsigned v3 = 0;
+        for (int t = 0; t < 3; ++t) {
+          const int bit = 3 * j + t;
+          v3 |= (unsigned)((src[bit / 8] >> (bit % 8)) & 1u) << t;
+        }
+        const uint8_t nib = (uint8_t)((v3 & 3u) | ((v3 & 4u) ? 8u : 0u));
+        const int64_t e = b * 16 + j;
+        uint8_t* byte = &codes[r * (vc / 2) + e / 2];
+        *byte = (e % 2) ? (uint8_t)((*byte & 15u) | (nib << 4)) : (uint8_t)((*byte & 0xF0u) | nib);
+      }
+      scales[r * nb + b] = mx ? packed_scales[r * (nb / 2) + b / 2] : packed_scales[r * nb + b];
+    }
+  }
+}
+
 /* Quantize an already rotated view z with a given tensor amax: steps 2 onward
  * of oracle_quantize_rows, for checking a quantizer on rotated values it
  * computed itself.  z holds the vr view rows row0 .. row0+vr-1 (vc fp32 each,

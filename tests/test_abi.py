@@ -34,7 +34,7 @@ def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ["nvfp4_quantize", "nvfp4_dequantize", "nvfp4_rht", "nvfp4_amax", "nvfp4_workspace_bytes",
               "nvfp4_status_string", "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_quantize_noalloc",
-              "nvfp4_amax_dual", "nvfp4_gemm", "nvfp4_quantize_dual"]:
+              "nvfp4_amax_dual", "nvfp4_gemm", "nvfp4_quantize_dual", "nvfp4_pack3", "nvfp4_unpack3"]:
         assert n in names
 
 
@@ -131,6 +131,19 @@ def test_quantize_dual_rejects(N):
     assert qd(N, outs=(FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE)) == ALIGN
     assert qd(N, x=FAKE + 8) == ALIGN
     assert qd(N, ar=FAKE + 2) == ALIGN
+
+
+def test_pack3_rejects(N):
+    p, u = N.nvfp4_pack3, N.nvfp4_unpack3
+    assert p(FAKE, FAKE, 4, 64, 0, FAKE, FAKE, None) == UNSUPPORTED      # RTN is not a 3-bit mode
+    assert p(FAKE, FAKE, 4, 40, 8, FAKE, FAKE, None) == SHAPE            # vcols % 16
+    assert p(FAKE, FAKE, 4, 48, 11, FAKE, FAKE, None) == SHAPE           # MXFP3: vcols % 32
+    assert p(None, FAKE, 4, 64, 8, FAKE, FAKE, None) == INVALID
+    assert p(FAKE, FAKE, 0, 64, 8, None, None, None) == OK               # empty: nothing touched
+    assert p(FAKE + 4, FAKE, 4, 64, 8, FAKE, FAKE, None) == ALIGN        # codes 8-byte aligned
+    assert p(FAKE, FAKE, 4, 64, 8, FAKE + 1, FAKE, None) == ALIGN        # packed codes 2-byte aligned
+    assert u(FAKE, FAKE, 4, 64, 9, None, FAKE, None) == INVALID
+    assert u(FAKE, FAKE, 4, 64, 3, FAKE, FAKE, None) == UNSUPPORTED
 
 
 def test_other_entry_points_reject(N):
