@@ -75,6 +75,10 @@ def parse_args(argv=None):
                    help="skip the per-mode table (every mode on dY, quantize kernel alone)")
     p.add_argument("--no-configs", action="store_true",
                    help="skip the other workloads' calls (256x256, weight, gradient, activation)")
+    p.add_argument("--profile-case", default=None, metavar="ROWSxCOLS",
+                   help="profiling run: only one gradient-like tensor of this shape through the step's launches "
+                        "(dual pre-pass, dual quantize, single-layout MS-EDEN and RTN quantizes), --steps times; "
+                        "prints the per-launch times, not the benchmark line")
     p.add_argument("--no-unfused", action="store_true",
                    help="skip the comparison step with one quantize launch per call")
     p.add_argument("--no-eager", action="store_true",
@@ -861,9 +865,54 @@ def run_reference(args, world, rank, wl=None, fraction=1.0 / 64):
     return line
 
 
+def run_profile_case(args):
+    """A small, self-contained run of the step's kernels on one tensor, for ncu
+    captures that must stay within a few GB: a Student-t3 (std 1e-4) tensor of
+    the given shape, and per iteration its dual pre-pass, its dual quantize
+    (MS-EDEN both ways, and RTN rows + MS-EDEN columns), and the single-layout
+    quantizes (MS-EDEN g = 128 both layouts, RTN row-wise)."""
+    import ctypes
+    from nvfp4_microscaling_quantization_b200 import binding as N
+    from nvfp4_microscaling_quantization_b200 import workloads as W
+    rows, cols = (int(v) for v in args.profile_case.lower().split("x"))
+    device = torch.device("cuda", 0)
+    g = torch.Generator(device=device)
+    g.manual_seed(11)
+    x = W.student_t3((rows, cols), 1e-4, g)
+    stream = torch.cuda.Stream(device)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    calls = {(lay, mode, grp): Call(N, W.Call("p", lay, mode, grp), x, 11, sh)
+             for lay, mode, grp in [(W.ROWWISE, W.MS_EDEN, 128), (W.TRANSPOSED, W.MS_EDEN, 128),
+                                    (W.ROWWISE, W.RTN, 0)]}
+    eden = TensorCalls(N, [calls[(W.ROWWISE, W.MS_EDEN, 128)], calls[(W.TRANSPOSED, W.MS_EDEN, 128)]])
+    mixed = TensorCalls(N, [calls[(W.ROWWISE, W.RTN, 0)], calls[(W.TRANSPOSED, W.MS_EDEN, 128)]])
+    body = [("amax_dual eden", eden.amax_passes), ("quantize_dual eden", eden.quantize_dual),
+            ("amax_dual mixed", mixed.amax_passes), ("quantize_dual mixed", mixed.quantize_dual)]
+    body += [(f"quantize {c.call.name}", c.quantize) for c in calls.values()]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    times = {name: [] for name, _ in body}
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.steps, 1)):
+            for name, fn in body:
+                flush.zero_()
+                a, b = ev(), ev()
+                a.record()
+                fn()
+                b.record()
+                b.synchronize()
+                times[name].append(a.elapsed_time(b) * 1e3)
+    torch.cuda.synchronize(device)
+    print(json.dumps({"profile_case": [rows, cols], "launch_us_median": {k: round(statistics.median(v), 2)
+                                                                         for k, v in times.items()}}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     world, rank, local = dist_env()
+    if args.profile_case:
+        run_profile_case(args)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)
         return

@@ -50,27 +50,45 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int kGBM = 128, kGBN = 128;           // output tile
+constexpr int kGBM = 128;                        // output tile rows
 constexpr int kGBK = 256;                        // K elements per stage = 128 bytes of E2M1 a row
-constexpr int kGStages = 6;
-constexpr int kGAccum = 2;
-constexpr uint32_t kGOpBytes = kGBM * kGBK / 2;  // 16 KB per operand per stage
-constexpr uint32_t kGSfBytes = kGBM * (kGBK / 16);  // 2 KB of scale bytes per operand per stage
-constexpr uint32_t kGStageBytes = 2 * kGOpBytes + 2 * kGSfBytes;  // a multiple of 1024
-constexpr uint32_t kGSfCols = 32;                // per stage: 4 K steps x 4 columns for A, the same for B
-constexpr uint32_t kGSfBase = kGAccum * kGBN;    // scale columns follow the accumulators
+constexpr uint32_t kGOpBytes = kGBM * kGBK / 2;  // 16 KB of A codes per stage
+constexpr uint32_t kGSfBytes = kGBM * (kGBK / 16);  // 2 KB of A scale bytes per stage
 constexpr uint32_t kGTmemCols = 512;
-static_assert(kGSfBase + kGStages * kGSfCols <= kGTmemCols, "tensor memory");
 constexpr int kGProducerWarp = 0, kGMmaWarp = 1, kGEpiWarp0 = 6;  // scale writers: warps 2..5
-constexpr int kGThreads = 320;
-constexpr size_t kGDynSmem = kGStages * kGStageBytes + 1024;
+
+// The shape of one instance: output tiles of 128 x BN.
+//   BN = 128: two 128-column accumulators (the next tile's MMAs overlap the
+//             epilogue), six stages of 36 KB, four epilogue warps;
+//   BN = 256: one 256-column accumulator (A is read once for twice the
+//             columns: 25% fewer operand bytes per FLOP from L2), four
+//             stages of 54 KB, eight epilogue warps (two per lane quarter,
+//             128 columns each) to drain it quickly.
+// Scale columns per stage: A 4 K steps x 4 columns, B 4 K steps x BN/32.
+template <int BN>
+struct GemmShape {
+  static constexpr int accum = BN == 128 ? 2 : 1;
+  static constexpr int stages = BN == 128 ? 6 : 4;
+  static constexpr uint32_t b_bytes = BN * kGBK / 2;
+  static constexpr uint32_t sfb_bytes = BN * (kGBK / 16);
+  static constexpr uint32_t stage_bytes = kGOpBytes + b_bytes + kGSfBytes + sfb_bytes;  // a multiple of 1024
+  static constexpr uint32_t sfb_cols_per_step = BN / 32;
+  static constexpr uint32_t sf_cols = 16 + 4 * sfb_cols_per_step;
+  static constexpr uint32_t sf_base = accum * BN;  // scale columns follow the accumulators
+  static constexpr int epi_warps = 4 * (BN / 128);
+  static constexpr int threads = (kGEpiWarp0 + epi_warps) * 32;
+  static constexpr size_t dyn_smem = stages * stage_bytes + 1024;
+  static_assert(sf_base + stages * sf_cols <= kGTmemCols, "tensor memory");
+  static_assert(stage_bytes % 1024 == 0, "stage alignment");
+};
+constexpr int kGMaxStages = 6, kGMaxAccum = 2;
 
 struct GemmShared {
-  uint64_t full[kGStages];     // A and B codes and scale bytes of the stage landed
-  uint64_t sf_full[kGStages];  // the stage's scale factors are in tensor memory (4 writer warps)
-  uint64_t empty[kGStages];    // the MMAs that read the stage completed
-  uint64_t tfull[kGAccum];     // accumulator holds a finished tile
-  uint64_t tfree[kGAccum];     // epilogue drained the accumulator (4 warps)
+  uint64_t full[kGMaxStages];     // A and B codes and scale bytes of the stage landed
+  uint64_t sf_full[kGMaxStages];  // the stage's scale factors are in tensor memory (4 writer warps)
+  uint64_t empty[kGMaxStages];    // the MMAs that read the stage completed
+  uint64_t tfull[kGMaxAccum];     // accumulator holds a finished tile
+  uint64_t tfree[kGMaxAccum];     // epilogue drained the accumulator (all epilogue warps)
   uint32_t tmem_base;
   uint32_t issued_ab;          // per stage: a load in flight (bit s) and its phase (bit 8 + s)
   uint32_t issued_mma;         // per accumulator: a commit pending (bit a) and its phase (bit 8 + a)
@@ -85,18 +103,21 @@ __device__ __forceinline__ bool aborted(GemmShared& sh) {
   return *reinterpret_cast<volatile int*>(&sh.abort_flag) != 0;
 }
 
-template <int OUT_BF16>
-__global__ void __launch_bounds__(kGThreads, 1)
+template <int OUT_BF16, int BN>
+__global__ void __launch_bounds__(GemmShape<BN>::threads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                   const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ CUtensorMap tmap_sb,
                   const float* __restrict__ a_gscale, const float* __restrict__ b_gscale, int64_t m, int64_t n,
                   int64_t k, void* __restrict__ d, int64_t ldd) {
+  using GS = GemmShape<BN>;
+  constexpr int kGStages = GS::stages, kGAccum = GS::accum;
+  constexpr uint32_t kGStageBytes = GS::stage_bytes, kGSfCols = GS::sf_cols, kGSfBase = GS::sf_base;
   extern __shared__ uint8_t dyn_smem[];
   __shared__ __align__(8) GemmShared sh;
   uint8_t* tiles = align_1024(dyn_smem);
 
   const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
-  const int64_t n_tn = n / kGBN;
+  const int64_t n_tn = n / BN;
   const int64_t n_tiles = (m / kGBM) * n_tn;
   const int kt_count = static_cast<int>(k / kGBK);
   const int64_t step = gridDim.x;
@@ -109,7 +130,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     }
     for (int a = 0; a < kGAccum; ++a) {
       mbar_init(&sh.tfull[a], 1);
-      mbar_init(&sh.tfree[a], 4);
+      mbar_init(&sh.tfree[a], GS::epi_warps);
     }
     sh.issued_ab = 0;
     sh.issued_mma = 0;
@@ -134,7 +155,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       prefetch_tensormap(&tmap_sb);
       uint32_t it = 0;
       for (int64_t t = blockIdx.x; t < n_tiles && !aborted(sh); t += step) {
-        const int32_t ya = static_cast<int32_t>((t / n_tn) * kGBM), yb = static_cast<int32_t>((t % n_tn) * kGBN);
+        const int32_t ya = static_cast<int32_t>((t / n_tn) * kGBM), yb = static_cast<int32_t>((t % n_tn) * BN);
         for (int kt = 0; kt < kt_count; ++kt, ++it) {
           const uint32_t s = it % kGStages, u = it / kGStages;
           if (it >= kGStages && !mbar_wait(&sh.empty[s], (u - 1) & 1u)) {
@@ -149,8 +170,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           mbar_arrive_expect_tx(&sh.full[s], kGStageBytes);
           tma_load_2d(dst, &tmap_a, kt * (kGBK / 2), ya, &sh.full[s]);
           tma_load_2d(dst + kGOpBytes, &tmap_b, kt * (kGBK / 2), yb, &sh.full[s]);
-          tma_load_2d(dst + 2 * kGOpBytes, &tmap_sa, kt * (kGBK / 16), ya, &sh.full[s]);
-          tma_load_2d(dst + 2 * kGOpBytes + kGSfBytes, &tmap_sb, kt * (kGBK / 16), yb, &sh.full[s]);
+          tma_load_2d(dst + kGOpBytes + GS::b_bytes, &tmap_sa, kt * (kGBK / 16), ya, &sh.full[s]);
+          tma_load_2d(dst + kGOpBytes + GS::b_bytes + kGSfBytes, &tmap_sb, kt * (kGBK / 16), yb, &sh.full[s]);
           sh.issued_ab = (sh.issued_ab & ~(0x101u << s)) | (1u << s) | ((u & 1u) << (8 + s));
         }
       }
@@ -158,7 +179,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
   } else if (warp == kGMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_nvfp4_f32(kGBM, kGBN);
+      constexpr uint32_t idesc = idesc_nvfp4_f32(kGBM, BN);
       uint32_t it = 0, tile = 0;
       for (int64_t t = blockIdx.x; t < n_tiles && !aborted(sh); t += step, ++tile) {
         const uint32_t a = tile % kGAccum, ua = tile / kGAccum;
@@ -182,7 +203,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
             // K step j: 32 bytes further along each 128-byte swizzled row
             const uint64_t adesc = smem_desc_sw128(a_addr + j * 32, 16, 1024);
             const uint64_t bdesc = smem_desc_sw128(b_addr + j * 32, 16, 1024);
-            umma_nvfp4(tmem_base + a * kGBN, adesc, bdesc, idesc, sf + 4 * j, sf + 16 + 4 * j,
+            umma_nvfp4(tmem_base + a * BN, adesc, bdesc, idesc, sf + 4 * j, sf + 16 + GS::sfb_cols_per_step * j,
                        (kt | j) != 0 ? 1u : 0u);
           }
           umma_commit(&sh.empty[s]);
@@ -214,22 +235,34 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           ok = false;
           break;
         }
-        const uint4* sa = reinterpret_cast<const uint4*>(tiles + s * kGStageBytes + 2 * kGOpBytes);
+        const uint4* sa = reinterpret_cast<const uint4*>(tiles + s * kGStageBytes + kGOpBytes + GS::b_bytes);
         const uint4* sb = sa + kGBM;
-        uint32_t ca[16], cb[16];
-        // column 4j + h: the four factors of K step j of row 32h + l
+        // A: column 4j + h holds the four factors of K step j of row 32h + l;
+        // B: column (BN/32) j + h likewise for its BN rows
+        constexpr int kHb = BN / 32;
+        uint32_t ca[16], cb[4 * kHb];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          const uint4 va = sa[32 * h + lane], vb = sb[32 * h + lane];
+          const uint4 va = sa[32 * h + lane];
           ca[h] = va.x, ca[4 + h] = va.y, ca[8 + h] = va.z, ca[12 + h] = va.w;
-          cb[h] = vb.x, cb[4 + h] = vb.y, cb[8 + h] = vb.z, cb[12 + h] = vb.w;
+        }
+#pragma unroll
+        for (int h = 0; h < kHb; ++h) {
+          const uint4 vb = sb[32 * h + lane];
+          cb[h] = vb.x, cb[kHb + h] = vb.y, cb[2 * kHb + h] = vb.z, cb[3 * kHb + h] = vb.w;
         }
         tc_fence_after_sync();
         const uint32_t sf = tmem_base + ((32u * q) << 16) + kGSfBase + s * kGSfCols;
         tmem_st16(sf, ca);
         tmem_st_wait();
-        tmem_st16(sf + 16, cb);
-        tmem_st_wait();
+#pragma unroll
+        for (int c = 0; c < 4 * kHb; c += 16) {
+          uint32_t part[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) part[i] = cb[c + i];
+          tmem_st16(sf + 16 + c, part);
+          tmem_st_wait();
+        }
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.sf_full[s]);
@@ -238,7 +271,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     if (!ok) atomicExch(&sh.abort_flag, 1);
   } else {
     // ------------------------------------------------------------ epilogue
-    const uint32_t q = warp & 3u;
+    // warp e (0 .. epi_warps-1): lane quarter e % 4, columns 128 (e / 4) .. +127
+    const uint32_t e = warp - kGEpiWarp0, q = e & 3u, c_begin = 128u * (e >> 2);
     const float gab = __fmul_rn(*a_gscale, *b_gscale);
     uint32_t tile = 0;
     for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++tile) {
@@ -249,21 +283,21 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       }
       if (aborted(sh)) break;
       tc_fence_after_sync();
-      const int64_t row = (t / n_tn) * kGBM + 32 * q + lane, col0 = (t % n_tn) * kGBN;
+      const int64_t row = (t / n_tn) * kGBM + 32 * q + lane, col0 = (t % n_tn) * BN;
 #pragma unroll 1
-      for (int c = 0; c < kGBN; c += 32) {
+      for (uint32_t c = c_begin; c < c_begin + 128u; c += 32) {
         float v[32];
-        tmem_ld32_wait(tmem_base + ((32u * q) << 16) + a * kGBN + c, v);
+        tmem_ld32_wait(tmem_base + ((32u * q) << 16) + a * BN + c, v);
         if constexpr (OUT_BF16) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(d) + row * ldd + col0 + c);
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
             uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int k2 = 0; k2 < 4; ++k2) {
               const __nv_bfloat162 p =
-                  __floats2bfloat162_rn(__fmul_rn(v[i + 2 * e], gab), __fmul_rn(v[i + 2 * e + 1], gab));
-              w[e] = *reinterpret_cast<const uint32_t*>(&p);
+                  __floats2bfloat162_rn(__fmul_rn(v[i + 2 * k2], gab), __fmul_rn(v[i + 2 * k2 + 1], gab));
+              w[k2] = *reinterpret_cast<const uint32_t*>(&p);
             }
             dst[i / 8] = make_uint4(w[0], w[1], w[2], w[3]);
           }
@@ -321,47 +355,48 @@ EncodeTiledFn gemm_encode_fn() {
   return fn;
 }
 
-// rows x (k / 2) bytes of packed E2M1, boxes of 128 bytes x 128 rows.
-bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k) {
+// rows x (k / 2) bytes of packed E2M1, boxes of 128 bytes x box_rows rows.
+bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k, uint32_t box_rows) {
   EncodeTiledFn fn = gemm_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 2), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 2)};
-  cuuint32_t box[2] = {kGBK / 2, kGBM};
+  cuuint32_t box[2] = {kGBK / 2, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// rows x (k / 16) scale bytes, boxes of 16 bytes x 128 rows (no swizzle).
-bool make_scales_map(CUtensorMap* map, const uint8_t* scales, int64_t rows, int64_t k) {
+// rows x (k / 16) scale bytes, boxes of 16 bytes x box_rows rows (no swizzle).
+bool make_scales_map(CUtensorMap* map, const uint8_t* scales, int64_t rows, int64_t k, uint32_t box_rows) {
   EncodeTiledFn fn = gemm_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 16), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 16)};
-  cuuint32_t box[2] = {kGBK / 16, kGBM};
+  cuuint32_t box[2] = {kGBK / 16, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(scales), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int OUT_BF16>
+template <int OUT_BF16, int BN>
 cudaError_t launch_gemm_t(const GemmArgs& g) {
+  using GS = GemmShape<BN>;
   CUtensorMap ma, mb, msa, msb;
-  if (!make_codes_map(&ma, g.a_codes, g.m, g.k) || !make_codes_map(&mb, g.b_codes, g.n, g.k) ||
-      !make_scales_map(&msa, g.a_scales, g.m, g.k) || !make_scales_map(&msb, g.b_scales, g.n, g.k))
+  if (!make_codes_map(&ma, g.a_codes, g.m, g.k, kGBM) || !make_codes_map(&mb, g.b_codes, g.n, g.k, BN) ||
+      !make_scales_map(&msa, g.a_scales, g.m, g.k, kGBM) || !make_scales_map(&msb, g.b_scales, g.n, g.k, BN))
     return cudaErrorInvalidValue;
-  auto kernel = nvfp4_gemm_kernel<OUT_BF16>;
+  auto kernel = nvfp4_gemm_kernel<OUT_BF16, BN>;
   LaunchGeom geom;
-  const cudaError_t e = launch_geometry(kernel, kGThreads, kGDynSmem, 1, &geom);
+  const cudaError_t e = launch_geometry(kernel, GS::threads, GS::dyn_smem, 1, &geom);
   if (e != cudaSuccess) return e;
   const int sms = geom.sms;
-  const int64_t n_tiles = (g.m / kGBM) * (g.n / kGBN);
+  const int64_t n_tiles = (g.m / kGBM) * (g.n / BN);
   const int64_t grid = n_tiles < sms ? n_tiles : sms;
   if (grid == 0) return cudaSuccess;
-  kernel<<<static_cast<unsigned>(grid), kGThreads, kGDynSmem, g.stream>>>(
+  kernel<<<static_cast<unsigned>(grid), GS::threads, GS::dyn_smem, g.stream>>>(
       ma, mb, msa, msb, g.a_gscale, g.b_gscale, g.m, g.n, g.k, g.d, g.ldd);
   return cudaGetLastError();
 }
@@ -370,8 +405,12 @@ cudaError_t launch_gemm_t(const GemmArgs& g) {
 
 bool gemm_available() { return gemm_encode_fn() != nullptr; }
 
+// 128 x 256 tiles where n allows (the default), else 128 x 128; g.tile_n
+// forces one (128 or 256) for tests.
 cudaError_t launch_gemm(const GemmArgs& g) {
-  return g.out_bf16 ? launch_gemm_t<1>(g) : launch_gemm_t<0>(g);
+  const bool wide = g.tile_n == 256 || (g.tile_n == 0 && g.n % 256 == 0);
+  if (wide) return g.out_bf16 ? launch_gemm_t<1, 256>(g) : launch_gemm_t<0, 256>(g);
+  return g.out_bf16 ? launch_gemm_t<1, 128>(g) : launch_gemm_t<0, 128>(g);
 }
 
 }  // namespace nvfp4

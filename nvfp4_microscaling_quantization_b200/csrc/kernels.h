@@ -112,6 +112,7 @@ struct GemmArgs {
   void* d;                  // m rows, leading dimension ldd (elements)
   int64_t ldd;
   cudaStream_t stream;
+  int tile_n;               // 0: 256-column tiles when n % 256 == 0, else 128; 128 or 256 forces one
 };
 bool gemm_available();
 cudaError_t launch_gemm(const GemmArgs& g);

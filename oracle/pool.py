@@ -111,6 +111,19 @@ def _w_quantize_rotated(zpath, vr, vc, mode, seed, amax, b, e, cpath, spath):
 
 
 # ------------------------------------------------------------------ caller side
+def _scratch_dir(min_free=16 << 30):
+    """A RAM-backed directory for the shared files when one has room, else the
+    default temporary directory."""
+    try:
+        st = os.statvfs("/dev/shm")
+        if st.f_bavail * st.f_frsize >= min_free:
+            return "/dev/shm"
+    except OSError:
+        pass
+    return None
+
+
+
 class OraclePool:
     """A pool of spawn-started worker processes running the oracle on row ranges.
 
@@ -121,7 +134,7 @@ class OraclePool:
 
     def __init__(self, workers: int = 0):
         self.workers = workers if workers > 0 else host_cores()
-        self._dir = tempfile.mkdtemp(prefix="oracle_pool_")
+        self._dir = tempfile.mkdtemp(prefix="oracle_pool_", dir=_scratch_dir())
         self._n = 0
         ctx = multiprocessing.get_context("spawn")
         self._ex = concurrent.futures.ProcessPoolExecutor(max_workers=self.workers, mp_context=ctx)
