@@ -56,6 +56,7 @@ constexpr uint32_t kGOpBytes = kGBM * kGBK / 2;  // 16 KB of A codes per stage
 constexpr uint32_t kGSfBytes = kGBM * (kGBK / 16);  // 2 KB of A scale bytes per stage
 constexpr uint32_t kGTmemCols = 512;
 constexpr int kGProducerWarp = 0, kGMmaWarp = 1, kGEpiWarp0 = 6;  // scale writers: warps 2..5
+static_assert(kGEpiWarp0 % 2 == 0, "each run of four epilogue warps covers the four lane quarters");
 
 // The shape of one instance: output tiles of 128 x BN.
 //   BN = 128: two 128-column accumulators (the next tile's MMAs overlap the
@@ -271,8 +272,11 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     if (!ok) atomicExch(&sh.abort_flag, 1);
   } else {
     // ------------------------------------------------------------ epilogue
-    // warp e (0 .. epi_warps-1): lane quarter e % 4, columns 128 (e / 4) .. +127
-    const uint32_t e = warp - kGEpiWarp0, q = e & 3u, c_begin = 128u * (e >> 2);
+    // epilogue warp e = warp - kGEpiWarp0 reads the lane quarter tensor memory
+    // allows it (warp % 4) and columns 128 (e / 4) .. +127: the epilogue warps
+    // start at a multiple of four minus two, so each group of four consecutive
+    // warps covers every lane quarter once
+    const uint32_t e = warp - kGEpiWarp0, q = warp & 3u, c_begin = 128u * (e >> 2);
     const float gab = __fmul_rn(*a_gscale, *b_gscale);
     uint32_t tile = 0;
     for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++tile) {

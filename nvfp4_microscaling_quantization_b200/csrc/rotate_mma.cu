@@ -783,6 +783,13 @@ __device__ __forceinline__ void quantize_smem_row(const uint8_t* tile, uint32_t 
   }
 }
 
+// Tile k of this CTA (tiles blockIdx.x, blockIdx.x + gridDim.x, ...), or
+// counted from the last tile back when `reverse` is set.
+__device__ __forceinline__ uint32_t dual_tile_index(int64_t k, int64_t n_tiles, int reverse) {
+  const int64_t t = blockIdx.x + k * static_cast<int64_t>(gridDim.x);
+  return static_cast<uint32_t>(reverse ? n_tiles - 1 - t : t);
+}
+
 struct DualQuantShared {
   uint64_t full[kDualStages];
   uint64_t sfree[kDualStages];
@@ -822,11 +829,6 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
   const int64_t n_tiles = static_cast<int64_t>(tg.n_rt) * tg.n_ct;
   const int64_t step = gridDim.x;
   const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - blockIdx.x + step - 1) / step : 0;
-  // tile k of this CTA
-  auto tile_of = [&](int64_t k) -> uint32_t {
-    const int64_t t = blockIdx.x + k * step;
-    return static_cast<uint32_t>(reverse ? n_tiles - 1 - t : t);
-  };
 
   if (tid == kDualProducerWarp * 32) {
     for (int s = 0; s < kDualStages; ++s) {
@@ -870,7 +872,7 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
         }
         if (*reinterpret_cast<volatile int*>(&sh.abort_flag)) break;
         uint32_t rt, ct;
-        tg.coords(tile_of(k), rt, ct);
+        tg.coords(dual_tile_index(k, n_tiles, reverse), rt, ct);
         const int32_t x = static_cast<int32_t>(ct * kTile), y = static_cast<int32_t>(rt * kTile);
         mbar_arrive_expect_tx(&sh.full[s], kTileBytes);
         uint8_t* dst = a_tiles + s * kTileBytes;
@@ -954,7 +956,7 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
       const int64_t k = j / kViews;
       const int v = static_cast<int>(j % kViews);
       uint32_t rt, ct;
-      tg.coords(tile_of(k), rt, ct);
+      tg.coords(dual_tile_index(k, n_tiles, reverse), rt, ct);
       if constexpr (kRowFromSmem) {
         const int s = static_cast<int>(k % kDualStages);
         if (!mbar_wait(&sh.full[s], static_cast<uint32_t>(k / kDualStages) & 1u)) {
