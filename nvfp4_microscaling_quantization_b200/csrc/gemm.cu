@@ -145,11 +145,13 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  allow_dependent_launch();
   const uint32_t tmem_base = sh.tmem_base;
 
   if (warp == kGProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      grid_dependency_wait();
       prefetch_tensormap(&tmap_a);
       prefetch_tensormap(&tmap_b);
       prefetch_tensormap(&tmap_sa);
@@ -277,6 +279,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     // start at a multiple of four minus two, so each group of four consecutive
     // warps covers every lane quarter once
     const uint32_t e = warp - kGEpiWarp0, q = warp & 3u, c_begin = 128u * (e >> 2);
+    grid_dependency_wait();
     const float gab = __fmul_rn(*a_gscale, *b_gscale);
     uint32_t tile = 0;
     for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++tile) {
@@ -288,10 +291,24 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       if (aborted(sh)) break;
       tc_fence_after_sync();
       const int64_t row = (t / n_tn) * kGBM + 32 * q + lane, col0 = (t % n_tn) * BN;
-#pragma unroll 1
-      for (uint32_t c = c_begin; c < c_begin + 128u; c += 32) {
+      // all 128 columns of this warp's part in flight at once, one wait, then
+      // the accumulator is released before the conversion and the stores, so
+      // the next tile's MMAs overlap them
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32_nowait(tmem_base + ((32u * q) << 16) + a * BN + c_begin + 32 * c4, r[c4]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) tmem_regs_after_wait(r[c4]);
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.tfree[a]);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const uint32_t c = c_begin + 32u * c4;
         float v[32];
-        tmem_ld32_wait(tmem_base + ((32u * q) << 16) + a * BN + c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[c4][i]);
         if constexpr (OUT_BF16) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(d) + row * ldd + col0 + c);
 #pragma unroll
@@ -313,9 +330,6 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
                                      __fmul_rn(v[i + 3], gab));
         }
       }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.tfree[a]);
     }
   }
 
@@ -400,9 +414,8 @@ cudaError_t launch_gemm_t(const GemmArgs& g) {
   const int64_t n_tiles = (g.m / kGBM) * (g.n / BN);
   const int64_t grid = n_tiles < sms ? n_tiles : sms;
   if (grid == 0) return cudaSuccess;
-  kernel<<<static_cast<unsigned>(grid), GS::threads, GS::dyn_smem, g.stream>>>(
-      ma, mb, msa, msb, g.a_gscale, g.b_gscale, g.m, g.n, g.k, g.d, g.ldd);
-  return cudaGetLastError();
+  return launch_overlapped(kernel, static_cast<unsigned>(grid), GS::threads, GS::dyn_smem, g.stream, ma, mb, msa,
+                           msb, g.a_gscale, g.b_gscale, g.m, g.n, g.k, g.d, g.ldd);
 }
 
 }  // namespace

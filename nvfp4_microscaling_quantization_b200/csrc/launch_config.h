@@ -116,4 +116,27 @@ cudaError_t launch_geometry(Kernel kernel, int threads, size_t dyn_smem, int cap
   return cudaSuccess;
 }
 
+// Launch `kernel` with programmatic stream serialization: it may begin (its
+// CTAs scheduled, its prologue run) while the previous kernel on the stream
+// finishes; the kernel itself calls grid_dependency_wait() before touching
+// global memory.  For the persistent kernels, whose one CTA per SM cannot
+// share an SM with the previous kernel's, the overlap is the next kernel's
+// prologue (barrier set-up, tensor-memory allocation, the rotation matrix)
+// with the previous kernel's last tiles.
+template <typename... ExpTypes, typename... ActTypes>
+cudaError_t launch_overlapped(void (*kernel)(ExpTypes...), unsigned grid, unsigned threads, size_t smem,
+                              cudaStream_t stream, ActTypes&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<ActTypes&&>(args)...);
+}
+
 }  // namespace nvfp4

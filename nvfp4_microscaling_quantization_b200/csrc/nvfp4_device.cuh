@@ -67,9 +67,11 @@ __device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
 }
 // a - b per lane: the negation is exact, so each lane is the one RN subtraction.
 __device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) { return add2_rn(a, f2(-b.x, -b.y)); }
-// a + b and a - b lane by lane through the scalar intrinsics, which are never
-// merged with the multiplication that produced b: for a sum whose operand is
-// a rounded product.
+// a + b and a - b lane by lane through the scalar intrinsics, for a sum
+// whose operand b is a rounded product: the scalar adds are never merged with
+// the multiplication that produced b.  (The packed add.rn.f32x2 is not safe
+// here: a GPU parity test of IF4 found a packed product and sum contracted
+// into one fused operation, skipping the product's rounding.)
 __device__ __forceinline__ float2 add2_after_mul(float2 a, float2 b) { return f2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y)); }
 __device__ __forceinline__ float2 sub2_after_mul(float2 a, float2 b) { return f2(__fsub_rn(a.x, b.x), __fsub_rn(a.y, b.y)); }
 

@@ -246,6 +246,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  allow_dependent_launch();
   const uint32_t tmem_base = sh.tmem_base;
   const int64_t step = gridDim.x;
   if (warp != S::producer_warp) {
@@ -259,6 +260,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
 
   if (warp == S::producer_warp) {
     if (lane == 0) {
+      grid_dependency_wait();
       prefetch_tensormap(&tmap);
       int k = 0;
       for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++k) {
@@ -317,6 +319,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     // accumulator grp; a warp reads lane quarter q (= warp % 4, as tensor
     // memory requires): its thread owns one tile row, all 128 columns
     const uint32_t q = warp & 3u, grp = warp >> 2;
+    grid_dependency_wait();
     ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false, nullptr};
     if constexpr (KIND == kQuantize) {
       sc = make_scale_ctx<MODE>(*amax);
@@ -501,15 +504,17 @@ __device__ __forceinline__ void build_rotation_b(uint8_t* bmat, PhiloxKey key, u
   }
 }
 
-// max |v| over 64 accumulator values, kept in two chains.
+// max |v| over 64 accumulator values (and m), as a tree: short dependency
+// chains, so a warp's reduction does not wait on its own previous result.
 __device__ __forceinline__ float absmax64(const float (&v)[64], float m) {
-  float m0 = m, m1 = m;
+  float t[32];
 #pragma unroll
-  for (int i = 0; i < 64; i += 2) {
-    m0 = fmaxf(m0, fabsf(v[i]));
-    m1 = fmaxf(m1, fabsf(v[i + 1]));
-  }
-  return fmaxf(m0, m1);
+  for (int i = 0; i < 32; ++i) t[i] = fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1]));
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
+  return fmaxf(m, t[0]);
 }
 
 __global__ void __launch_bounds__(kDualThreads, 1)
@@ -556,6 +561,7 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  allow_dependent_launch();
   const uint32_t tmem_base = sh.tmem_base;
   if (warp != kDualProducerWarp) {
     // the B matrices, built while the producer starts loading (barrier 2)
@@ -568,6 +574,7 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
 
   if (warp == kDualProducerWarp) {
     if (lane == 0) {
+      grid_dependency_wait();
       prefetch_tensormap(&tmap);
       for (int64_t k = 0; k < my_tiles; ++k) {
         const int s = static_cast<int>(k % kDualStages);
@@ -637,6 +644,7 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
   } else {
     // epilogue: slot `slot`, lane quarter q
     const uint32_t q = warp & 3u, slot = warp >> 2;
+    grid_dependency_wait();
     float m_r = 0.0f, m_c = 0.0f;  // max |acc| (unscaled) of the row and column views; max |x| from smem
     const int64_t n_acc = my_tiles * views;
     const uint32_t part = q * 32u + lane;
@@ -851,6 +859,7 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  allow_dependent_launch();
   const uint32_t tmem_base = sh.tmem_base;
   if (warp != kDualProducerWarp) {
     const uint32_t bt = warp < kDualProducerWarp ? tid : tid - 32, nb = kDualThreads - 32;
@@ -862,6 +871,7 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
 
   if (warp == kDualProducerWarp) {
     if (lane == 0) {
+      grid_dependency_wait();
       prefetch_tensormap(&tmap);
       for (int64_t k = 0; k < my_tiles; ++k) {
         const int s = static_cast<int>(k % kDualStages);
@@ -933,6 +943,7 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
   } else {
     // ------------------------------------------------------------ epilogue
     const uint32_t q = warp & 3u, slot = warp >> 2;
+    grid_dependency_wait();
     ScaleCtx sc_r = make_scale_ctx<MODE_R>(*amax_r);
     ScaleCtx sc_c = make_scale_ctx<MODE_C>(*amax_c);
     build_scale_table(sh.scale_tbl[0], sc_r.s_g, tid, kDualEpiWarps * 32);
@@ -975,7 +986,17 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
       }
       tc_fence_after_sync();
       const uint32_t base = tmem_base + ((32u * q) << 16) + slot * kTile;
-      if (kViews == 2 && v == 0) {
+      if constexpr (kViews == 2 && MODE_R == MODE_C && G_R == G_C) {
+        // both views run the same code: one call site with the view's
+        // parameters selected, so the epilogue is one copy of the code in
+        // the instruction cache whichever view a warp holds
+        const bool row = v == 0;
+        quantize_tmem_row<MODE_C, G_C>(
+            base, &sh.tfree[slot], row ? sc_r : sc_c, key,
+            static_cast<int64_t>(row ? rt : ct) * kTile + r_in_tile, static_cast<int64_t>(row ? ct : rt) * kTile,
+            row ? rows : cols, row ? cols : rows, row ? r_blocks8 : c_blocks8, row ? r_codes16 : c_codes16,
+            row ? r_scales4 : c_scales4, row ? codes_r : codes_c, row ? scales_r : scales_c);
+      } else if (kViews == 2 && v == 0) {
         if constexpr (G_R != 0)
           quantize_tmem_row<MODE_R, (G_R != 0 ? G_R : 16)>(
               base, &sh.tfree[slot], sc_r, key, static_cast<int64_t>(rt) * kTile + r_in_tile,
@@ -1055,10 +1076,9 @@ cudaError_t launch_one(const QuantArgs& a, float* zout) {
     if (KIND == kAmax) return cudaSuccess;
     grid = 1;
   }
-  kernel<<<static_cast<unsigned>(grid), threads, kDynSmem, a.stream>>>(
-      map, a.rows, a.cols, a.seed, a.amax, reinterpret_cast<unsigned int*>(a.amax_accum), a.codes, a.scales,
-      a.gscale, zout);
-  return cudaGetLastError();
+  return launch_overlapped(kernel, static_cast<unsigned>(grid), threads, kDynSmem, a.stream, map, a.rows, a.cols,
+                           a.seed, a.amax, reinterpret_cast<unsigned int*>(a.amax_accum), a.codes, a.scales, a.gscale,
+                           zout);
 }
 
 template <int MODE, int KIND>
@@ -1123,10 +1143,9 @@ cudaError_t launch_amax_dual_mma(const void* x, int64_t rows, int64_t cols, int6
   const int64_t n_tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
   const int64_t grid = n_tiles < int64_t(sms) ? n_tiles : int64_t(sms);
   if (grid == 0) return cudaSuccess;
-  dual_amax_kernel<<<static_cast<unsigned>(grid), kDualThreads, kDualDynSmem, stream>>>(
-      map, rows, cols, seed, g_r, g_c, reinterpret_cast<unsigned int*>(amax_r),
-      reinterpret_cast<unsigned int*>(amax_c));
-  return cudaGetLastError();
+  return launch_overlapped(dual_amax_kernel, static_cast<unsigned>(grid), kDualThreads, kDualDynSmem, stream, map,
+                           rows, cols, seed, g_r, g_c, reinterpret_cast<unsigned int*>(amax_r),
+                           reinterpret_cast<unsigned int*>(amax_c));
 }
 
 namespace {
@@ -1142,10 +1161,9 @@ cudaError_t launch_dual_quantize_t(const DualQuantArgs& a) {
   const int64_t n_tiles = ((a.rows + kTile - 1) / kTile) * ((a.cols + kTile - 1) / kTile);
   const int64_t grid = n_tiles < int64_t(geom.sms) ? n_tiles : int64_t(geom.sms);
   if (grid == 0) return cudaSuccess;
-  kernel<<<static_cast<unsigned>(grid), kDualThreads, kDualDynSmem, a.stream>>>(
-      map, a.rows, a.cols, a.seed, a.amax_row, a.amax_col, a.codes_row, a.scales_row, a.gscale_row, a.codes_col,
-      a.scales_col, a.gscale_col, a.reverse);
-  return cudaGetLastError();
+  return launch_overlapped(kernel, static_cast<unsigned>(grid), kDualThreads, kDualDynSmem, a.stream, map, a.rows,
+                           a.cols, a.seed, a.amax_row, a.amax_col, a.codes_row, a.scales_row, a.gscale_row,
+                           a.codes_col, a.scales_col, a.gscale_col, a.reverse);
 }
 
 template <int G>

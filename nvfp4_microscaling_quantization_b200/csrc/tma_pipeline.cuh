@@ -99,6 +99,18 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Programmatic dependent launch.  grid_dependency_wait(): wait until the
+// grids this one depends on (the previous kernel on the stream) have
+// completed and their memory operations are visible -- called by every thread
+// before its first global-memory access, so a kernel launched early never
+// reads an input its predecessor is still writing or overwrites an output it
+// is still reading; it returns at once for a launch without that dependency.
+// allow_dependent_launch(): this CTA lets the next kernel on the stream begin
+// launching (its CTAs then take SMs as this grid's CTAs exit and run their
+// prologue, before their own grid_dependency_wait).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependent_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
