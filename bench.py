@@ -312,12 +312,18 @@ class GraphTimer:
     repetitions are captured once on `stream` (the callables launch on it
     through the C ABI) and the graph is replayed once, so the host takes no
     part while the marks are being recorded: the device runs every launch
-    back to back.  durations()[r][i] is callable i of repetition r, seconds."""
+    back to back.  durations()[r][i] is callable i of repetition r, seconds.
+    With per_launch=False only the repetition's first and last marks are
+    recorded, so consecutive launches are adjacent graph nodes (a kernel
+    launched with programmatic stream serialization can then start its
+    prologue during its predecessor's tail); totals() only."""
 
-    def __init__(self, stream, body, reps, flush):
+    def __init__(self, stream, body, reps, flush, per_launch=True):
         self.stream, self.body, self.reps, self.flush = stream, body, reps, flush
+        self.per_launch = per_launch
         mk = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
-        self.ev = [[mk() for _ in range(len(body) + 1)] for _ in range(reps)]
+        n_marks = len(body) + 1 if per_launch else 2
+        self.ev = [[mk() for _ in range(n_marks)] for _ in range(reps)]
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph, stream=stream, capture_error_mode="thread_local"):
             for r in range(reps):
@@ -326,7 +332,10 @@ class GraphTimer:
                 self.ev[r][0].record()
                 for i, fn in enumerate(body):
                     fn()
-                    self.ev[r][i + 1].record()
+                    if per_launch:
+                        self.ev[r][i + 1].record()
+                if not per_launch:
+                    self.ev[r][1].record()
 
     def replay(self):
         self.graph.replay()
@@ -343,13 +352,13 @@ class GraphTimer:
         self.graph = None
 
 
-def timed_in_graph(stream, body, reps, flush, device):
-    """Capture, replay once, and return (per-callable durations, per-rep totals)."""
-    t = GraphTimer(stream, body, reps, flush)
+def timed_in_graph(stream, body, reps, flush, device, per_launch=True):
+    """Capture, replay once, and return (per-callable durations or None, per-rep totals)."""
+    t = GraphTimer(stream, body, reps, flush, per_launch=per_launch)
     torch.cuda.synchronize(device)
     t.replay()
     torch.cuda.synchronize(device)
-    out = t.durations(), t.totals()
+    out = (t.durations() if per_launch else None), t.totals()
     t.release()
     return out
 
@@ -477,14 +486,19 @@ def linear_layer_table(N, groups, stream, device, flush, tensors, reps=10):
     with torch.cuda.stream(stream):
         for fn in fwd + bwd:
             fn()
-    d_fwd, t_fwd = timed_in_graph(stream, fwd, reps, flush, device)
-    d_bwd, t_bwd = timed_in_graph(stream, bwd, reps, flush, device)
+    # pass times with marks at the pass boundaries only; the per-launch split
+    # from a second, instrumented replay
+    _, t_fwd = timed_in_graph(stream, fwd, reps, flush, device, per_launch=False)
+    _, t_bwd = timed_in_graph(stream, bwd, reps, flush, device, per_launch=False)
+    d_fwd, _ = timed_in_graph(stream, fwd, reps, flush, device)
+    d_bwd, _ = timed_in_graph(stream, bwd, reps, flush, device)
     bf = [lambda: torch.matmul(x, w.t(), out=y), lambda: torch.matmul(dy, w, out=dx),
           lambda: torch.matmul(dy.t(), x, out=dw)]
     with torch.cuda.stream(stream):
         for fn in bf:
             fn()
-    d_bf, t_bf = timed_in_graph(stream, bf, reps, flush, device)
+    _, t_bf = timed_in_graph(stream, bf, reps, flush, device, per_launch=False)
+    d_bf, _ = timed_in_graph(stream, bf, reps, flush, device)
     torch.cuda.synchronize(device)
     f, b, r = dist_us(t_fwd), dist_us(t_bwd), dist_us(t_bf)
     m, k, n = x.shape[0], x.shape[1], w.shape[0]
@@ -563,17 +577,25 @@ def run_ours(args, world, rank, local):
         e_steps = [marks[k][0].elapsed_time(marks[k][-1]) / 1e3 for k in range(K)]
         e_calls = [[marks[k][i].elapsed_time(marks[k][i + 1]) / 1e3 for k in range(K)] for i in range(len(body))]
 
-    # the timed region: the K steps as one CUDA graph of the same C-ABI launches
-    timer = GraphTimer(stream, body, K, flush)
+    # the timed region: the K steps as one CUDA graph of the same C-ABI
+    # launches, marks at the step boundaries only (value); then the same K
+    # steps with a mark between every two launches (per-launch times, roofline)
+    timer = GraphTimer(stream, body, K, flush, per_launch=False)
+    inst = GraphTimer(stream, body, K, flush, per_launch=True)
     with ClockSampler(local) as clocks:
         barrier(world, local)
         torch.cuda.synchronize(device)
         timer.replay()
         torch.cuda.synchronize(device)
         barrier(world, local)
+        inst.replay()
+        torch.cuda.synchronize(device)
+        barrier(world, local)
     clock = clocks.summary()
-    durs, totals = timer.durations(), timer.totals()
+    totals = timer.totals()
+    durs, inst_totals = inst.durations(), inst.totals()
     timer.release()
+    inst.release()
 
     total_s = max_over_ranks(sum(totals), world, device)
     per_fn = [[durs[k][i] for k in range(K)] for i in range(len(body))]
@@ -627,7 +649,7 @@ def run_ours(args, world, rank, local):
 
     unfused = None
     if not args.no_unfused:
-        _, u_tot = timed_in_graph(stream, body_unfused, K, flush, device)
+        _, u_tot = timed_in_graph(stream, body_unfused, K, flush, device, per_launch=False)
         u_s = sum(u_tot)
         unfused = {"note": "the same step with one quantize launch per call (9 launches), CUDA graph timing",
                    "ms_per_step": {k: round(v / 1e3, 4) for k, v in dist_us(u_tot).items()},
@@ -674,14 +696,16 @@ def run_ours(args, world, rank, local):
             "calls": [c.call.name for c in calls],
             "path": "per tensor: one tensor-amax pre-pass for both layouts (nvfp4_amax_dual), then both "
                     "layouts' codes and scales from one read (nvfp4_quantize_dual), C ABI, one stream",
-            "timing": "the K steps captured once as one CUDA graph of the C-ABI launches and replayed once; "
-                      "CUDA events (graph event nodes) before, between and after the launches of each step",
+            "timing": "the K steps captured once as one CUDA graph of the C-ABI launches (consecutive launches "
+                      "adjacent, CUDA events at the step boundaries) and replayed once; per-launch times from a "
+                      "second replay with an event between every two launches",
             "input_dtype": "bf16", "l2": "flushed before every timed step (256 MiB write, outside the marks)",
             "parallelism": f"replicas x{world} (independent tensors per rank)",
         },
         "gelem_per_s": round(elems_per_step * K * world / total_s / 1e9, 1),
         "frac_of_hbm_peak": round(value / world / peak, 4),
         "step_ms": step_stats,
+        "step_ms_with_launch_marks": {k: round(v / 1e3, 4) for k, v in dist_us(inst_totals).items()},
         "value_amax_supplied": round(value_supplied, 1),
         "frac_of_hbm_peak_amax_supplied": round(value_supplied / world / peak, 4),
         "roofline": {"bound": "hbm", "kernel": launch_name(dom_kind, dom),
@@ -869,8 +893,9 @@ def run_profile_case(args):
     """A small, self-contained run of the step's kernels on one tensor, for ncu
     captures that must stay within a few GB: a Student-t3 (std 1e-4) tensor of
     the given shape, and per iteration its dual pre-pass, its dual quantize
-    (MS-EDEN both ways, and RTN rows + MS-EDEN columns), and the single-layout
-    quantizes (MS-EDEN g = 128 both layouts, RTN row-wise)."""
+    (MS-EDEN both ways, and RTN rows + MS-EDEN columns), the single-layout
+    quantizes (MS-EDEN g = 128 both layouts, RTN row-wise), and the NVFP4 GEMM
+    of the RTN row-wise quantization with itself."""
     import ctypes
     from nvfp4_microscaling_quantization_b200 import binding as N
     from nvfp4_microscaling_quantization_b200 import workloads as W
@@ -889,10 +914,18 @@ def run_profile_case(args):
     body = [("amax_dual eden", eden.amax_passes), ("quantize_dual eden", eden.quantize_dual),
             ("amax_dual mixed", mixed.amax_passes), ("quantize_dual mixed", mixed.quantize_dual)]
     body += [(f"quantize {c.call.name}", c.quantize) for c in calls.values()]
+    # one NVFP4 GEMM of the RTN row-wise quantization with itself (P P^T)
+    rq = calls[(W.ROWWISE, W.RTN, 0)]
+    d = torch.empty(rows, rows, dtype=torch.bfloat16, device=device)
+    body.append(("gemm P P^T", lambda: N.gemm((rq.codes, rq.scales, rq.gscale), (rq.codes, rq.scales, rq.gscale),
+                                               out=d, stream=stream)))
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     times = {name: [] for name, _ in body}
     with torch.cuda.stream(stream):
+        for _, fn in body:        # first launches (module loading) outside the timing
+            fn()
+        torch.cuda.synchronize(device)
         for _ in range(max(args.steps, 1)):
             for name, fn in body:
                 flush.zero_()

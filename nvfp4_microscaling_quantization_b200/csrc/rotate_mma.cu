@@ -736,6 +736,236 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
   }
 }
 
+// The same pre-pass when both views are rotated (dY of the backward pass),
+// in groups: two epilogue groups of eight warps, each owning two 128-column
+// accumulators (row view and column view of one tile, one commit for both);
+// warp (q, j) of a group reads lane quarter q of view j, 64 columns per load,
+// scales by c_g and reduces with a tree.  Measured faster than the slot ring
+// when every tile carries two MMAs; the results are identical.
+constexpr int kGrpStages = 3;     // A tiles in flight (each held until both MMAs are done)
+constexpr int kGrpGroups = 2;
+constexpr int kGrpEpiWarps = 8 * kGrpGroups;
+constexpr int kGrpThreads = (kGrpEpiWarps + 2) * 32;
+constexpr int kGrpProducerWarp = kGrpEpiWarps, kGrpMmaWarp = kGrpEpiWarps + 1;
+constexpr size_t kGrpDynSmem = (kGrpStages + 2) * kTileBytes + 1024;
+
+struct GroupDualShared {
+  uint64_t full[kGrpStages];
+  uint64_t sfree[kGrpStages];
+  uint64_t tfull[kGrpGroups];   // both accumulators of the group ready
+  uint64_t tfree[kGrpGroups];   // both loaded by the group
+  uint32_t tmem_base;
+  uint32_t issued_a;
+  uint32_t issued_mma;
+  int abort_flag;
+  unsigned int warp_max[2][kGrpEpiWarps];
+};
+
+__global__ void __launch_bounds__(kGrpThreads, 1)
+dual_amax_group_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed, int g_r,
+                 int g_c, unsigned int* __restrict__ amax_r, unsigned int* __restrict__ amax_c) {
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ __align__(8) GroupDualShared sh;
+  uint8_t* a_tiles = align_1024(dyn_smem);
+  uint8_t* b_r = a_tiles + kGrpStages * kTileBytes;
+  uint8_t* b_c = b_r + kTileBytes;
+
+  const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+  const PhiloxKey key = philox_key(seed);
+  const TileGrid tg{static_cast<uint32_t>((rows + kTile - 1) / kTile), static_cast<uint32_t>((cols + kTile - 1) / kTile),
+                    static_cast<uint32_t>(NVFP4_MMA_BAND_ROWS)};
+  const int64_t n_tiles = static_cast<int64_t>(tg.n_rt) * tg.n_ct;
+
+  if (tid == kGrpProducerWarp * 32) {
+    // with g_r = 0 the row view needs no MMA: the group's four row-view
+    // warps take max|x| from the staged tile and release the stage themselves
+    for (int s = 0; s < kGrpStages; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.sfree[s], g_r == 0 ? 5 : 1);
+    }
+    for (int a = 0; a < kGrpGroups; ++a) {
+      mbar_init(&sh.tfull[a], 1);
+      mbar_init(&sh.tfree[a], g_r == 0 ? 4 : 8);
+    }
+    sh.issued_a = 0;
+    sh.issued_mma = 0;
+    sh.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kGrpMmaWarp) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  allow_dependent_launch();
+  const uint32_t tmem_base = sh.tmem_base;
+  const int64_t step = gridDim.x;
+  if (warp != kGrpProducerWarp) {
+    // the B matrices, built while the producer starts loading (barrier 2)
+    const uint32_t bt = warp < kGrpProducerWarp ? tid : tid - 32, nb = kGrpThreads - 32;
+    if (g_r != 0) build_rotation_b(b_r, key, bt, nb, g_r);
+    build_rotation_b(b_c, key, bt, nb, g_c);
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 2, %0;" ::"r"(nb) : "memory");
+  }
+
+  if (warp == kGrpProducerWarp) {
+    if (lane == 0) {
+      grid_dependency_wait();
+      prefetch_tensormap(&tmap);
+      int k = 0;
+      for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++k) {
+        const int s = k % kGrpStages;
+        const uint32_t u = k / kGrpStages;
+        if (k >= kGrpStages && !mbar_wait(&sh.sfree[s], (u - 1) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        if (*reinterpret_cast<volatile int*>(&sh.abort_flag)) break;
+        uint32_t rt, ct;
+        tg.coords(static_cast<uint32_t>(t), rt, ct);
+        const int32_t x = static_cast<int32_t>(ct * kTile), y = static_cast<int32_t>(rt * kTile);
+        mbar_arrive_expect_tx(&sh.full[s], kTileBytes);
+        uint8_t* dst = a_tiles + s * kTileBytes;
+        tma_load_2d(dst, &tmap, x, y, &sh.full[s]);
+        tma_load_2d(dst + kBoxBytes, &tmap, x + 64, y, &sh.full[s]);
+        sh.issued_a = (sh.issued_a & ~(0x101u << s)) | (1u << s) | ((u & 1u) << (8 + s));
+      }
+    }
+  } else if (warp == kGrpMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_r = idesc_bf16_f32(kTile, kTile, 0u);
+      constexpr uint32_t idesc_c = idesc_bf16_f32(kTile, kTile, 1u);
+      const uint32_t br_addr = smem_u32(b_r), bc_addr = smem_u32(b_c);
+      int k = 0;
+      for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++k) {
+        const int s = k % kGrpStages, a = k % kGrpGroups;
+        const uint32_t use = k / kGrpGroups;
+        if (!mbar_wait(&sh.full[s], (k / kGrpStages) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        if (use > 0 && !mbar_wait(&sh.tfree[a], (use - 1) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t a_addr = smem_u32(a_tiles + s * kTileBytes);
+        const uint32_t d_r = tmem_base + a * 256, d_c = d_r + 128;
+        if (g_r != 0) {
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(a_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(br_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+            umma_bf16(d_r, adesc, bdesc, idesc_r, kk > 0 ? 1u : 0u);
+          }
+        }
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          const uint64_t adesc = smem_desc_sw128(a_addr + kk * 2048, kBoxBytes, 1024);
+          const uint64_t bdesc = smem_desc_sw128(bc_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+          umma_bf16(d_c, adesc, bdesc, idesc_c, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&sh.sfree[s]);
+        umma_commit(&sh.tfull[a]);
+        sh.issued_mma = (sh.issued_mma & ~(0x101u << a)) | (1u << a) | ((use & 1u) << (8 + a));
+      }
+    }
+  } else {
+    const uint32_t q = warp & 3u, j = (warp >> 2) & 1u, grp = warp >> 3;
+    grid_dependency_wait();
+    const float c = rht_scale_of(j == 0 ? g_r : g_c);
+    const float2 c2 = f2(c, c);
+    float m = 0.0f;
+    int k = static_cast<int>(grp);
+    if (j == 0 && g_r == 0) {
+      // max|x| of the staged tile: 128 threads, 256 bytes each (the order of
+      // the swizzled bytes does not matter to a maximum); bf16 -> f32 is exact
+      const uint32_t part = (warp & 3u) * 32u + lane;
+      for (int64_t t = blockIdx.x + grp * step; t < n_tiles; t += kGrpGroups * step, k += kGrpGroups) {
+        const int s = k % kGrpStages;
+        if (!mbar_wait(&sh.full[s], (k / kGrpStages) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(a_tiles + s * kTileBytes) + part;
+        uint32_t bmax = 0;  // max of |x| as bf16 bit patterns (monotone for non-negative values)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint4 w4 = src[i * 128];
+          const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) bmax = max(bmax, max(w[e] & 0x7FFFu, (w[e] >> 16) & 0x7FFFu));
+        }
+        m = fmaxf(m, __uint_as_float(bmax << 16));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.sfree[s]);
+      }
+    } else {
+    for (int64_t t = blockIdx.x + grp * step; t < n_tiles; t += kGrpGroups * step, k += kGrpGroups) {
+      if (!mbar_wait(&sh.tfull[grp], (k / kGrpGroups) & 1u)) {
+        atomicExch(&sh.abort_flag, 1);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t base = tmem_base + ((32u * q) << 16) + grp * 256 + j * 128;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float v[64];
+        tmem_ld64_wait(base + 64 * h, v);
+        if (h == 1) {
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.tfree[grp]);
+        }
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          float2 zp[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) zp[i] = mul2_rn(f2(v[32 * p + 2 * i], v[32 * p + 2 * i + 1]), c2);
+          float ma, mb;
+          absmax_pair(zp, ma, mb);
+          m = fmaxf(m, fmaxf(ma, mb));
+        }
+      }
+    }
+    }
+    const unsigned int bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
+    if (lane == 0) sh.warp_max[j][warp] = bits;
+  }
+
+  __syncthreads();
+  const bool failed = *reinterpret_cast<volatile int*>(&sh.abort_flag) != 0;
+  if (failed) {
+    if (tid == kGrpProducerWarp * 32)
+      for (int s = 0; s < kGrpStages; ++s)
+        if ((sh.issued_a >> s) & 1u) mbar_wait(&sh.full[s], (sh.issued_a >> (8 + s)) & 1u);
+    if (tid == kGrpMmaWarp * 32)
+      for (int a = 0; a < kGrpGroups; ++a)
+        if ((sh.issued_mma >> a) & 1u) mbar_wait(&sh.tfull[a], (sh.issued_mma >> (8 + a)) & 1u);
+  }
+  if (tid == 0) {
+    unsigned int mr = 0, mc = 0;
+#pragma unroll
+    for (int w = 0; w < kGrpEpiWarps; ++w) {
+      // warps with (w >> 2) odd read the column view
+      if (((w >> 2) & 1) == 0) mr = max(mr, sh.warp_max[0][w]);
+      else mc = max(mc, sh.warp_max[1][w]);
+    }
+    atomicMax(amax_r, failed ? 0x7FC00000u : mr);
+    atomicMax(amax_c, failed ? 0x7FC00000u : mc);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kGrpMmaWarp) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+
 // ------------------------------------------------ both layouts' quantization
 // One read of X for both views' codes and scales (given both tensor amaxes):
 // the pre-pass structure above -- four accumulator slots, per-slot barriers,
@@ -1136,16 +1366,20 @@ cudaError_t launch_amax_dual_mma(const void* x, int64_t rows, int64_t cols, int6
                                  uint64_t seed, float* amax_r, float* amax_c, cudaStream_t stream) {
   CUtensorMap map;
   if (!make_map(&map, x, rows, cols, ld)) return cudaErrorInvalidValue;
+  // both views rotated: the group kernel; the row view straight from the tile: the slot ring
+  const bool groups = g_r != 0;
+  auto kernel = groups ? dual_amax_group_kernel : dual_amax_kernel;
+  const int threads = groups ? kGrpThreads : kDualThreads;
+  const size_t smem = groups ? kGrpDynSmem : kDualDynSmem;
   LaunchGeom geom;
-  cudaError_t e = launch_geometry(dual_amax_kernel, kDualThreads, kDualDynSmem, 1, &geom);
+  cudaError_t e = launch_geometry(kernel, threads, smem, 1, &geom);
   if (e != cudaSuccess) return e;
   const int sms = geom.sms;
   const int64_t n_tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
   const int64_t grid = n_tiles < int64_t(sms) ? n_tiles : int64_t(sms);
   if (grid == 0) return cudaSuccess;
-  return launch_overlapped(dual_amax_kernel, static_cast<unsigned>(grid), kDualThreads, kDualDynSmem, stream, map,
-                           rows, cols, seed, g_r, g_c, reinterpret_cast<unsigned int*>(amax_r),
-                           reinterpret_cast<unsigned int*>(amax_c));
+  return launch_overlapped(kernel, static_cast<unsigned>(grid), threads, smem, stream, map, rows, cols, seed, g_r, g_c,
+                           reinterpret_cast<unsigned int*>(amax_r), reinterpret_cast<unsigned int*>(amax_c));
 }
 
 namespace {
