@@ -625,8 +625,13 @@ def run_ours(args, world, rank, local):
     dom_i = max(quant_idx, key=lambda i: statistics.mean(per_fn[i]))
     dom_kind, dom = body_names[dom_i]
     dom_stats = dist_us(per_fn[dom_i])
-    dom_bytes = moved_bytes(dom_kind, dom)
+    # algorithmic bytes: 2.5625 B per element of every call the launch serves
+    # (two calls for a both-layout launch); moved bytes: what it must transfer
+    dom_calls = [dom] if dom_kind == "quant" else [dom.row, dom.col]
+    dom_bytes = sum(BYTES_PER_ELEMENT * c.elements for c in dom_calls)
+    dom_moved = moved_bytes(dom_kind, dom)
     achieved = dom_bytes / (dom_stats["mean"] / 1e6) / 1e9
+    achieved_moved = dom_moved / (dom_stats["mean"] / 1e6) / 1e9
     src_hash = kernel_source_hash()
     traffic = NCU_TRAFFIC.get((src_hash, launch_name(dom_kind, dom)))
 
@@ -712,8 +717,10 @@ def run_ours(args, world, rank, local):
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_bytes": int(dom_bytes),
-                     "algorithmic_bytes_per_element": round(dom_bytes / (dom.elements if dom_kind == "quant"
-                                                                         else dom.row.elements), 4),
+                     "algorithmic_bytes_note": "2.5625 B per element of each call the launch serves",
+                     "calls": [c.call.name for c in dom_calls],
+                     "moved_bytes": int(dom_moved),
+                     "moved_gbs": round(achieved_moved, 1), "frac_of_moved": round(achieved_moved / peak, 4),
                      "avg_launch_us": dom_stats["mean"], "launch_us": dom_stats},
         "per_launch": per_launch,
         "gpu_launches": sum(g.launches(fused=True) for g in groups) * K,
