@@ -665,21 +665,27 @@ def run_ours(args, world, rank, local):
                  "ms_per_step": dist_us(e_steps), "dominant_launch_us": dist_us(e_calls[dom_i])}
         eager["ms_per_step"] = {k: round(v / 1e3, 4) for k, v in eager["ms_per_step"].items()}
 
-    gemms = None
-    if not args.no_gemm:
-        gemms = gemm_table(N, calls, stream, device)
-
-    layer = None
-    if not args.no_gemm:
-        layer = linear_layer_table(N, groups, stream, device, flush, tensors)
-
+    # the quantization tables first, the GEMM tables (about 1 kW) after them,
+    # each with the clocks sampled while it runs
+    table_clocks = {}
     per_mode = None
     if not args.no_per_mode:
-        per_mode = per_mode_table(N, W, tensors["dy"], wl.seed, stream, sh, device, flush, peak)
+        with ClockSampler(local) as ck:
+            per_mode = per_mode_table(N, W, tensors["dy"], wl.seed, stream, sh, device, flush, peak)
+        table_clocks["per_mode_dy"] = ck.summary()
 
     configs = None
     if not args.no_configs:
-        configs = workload_table(N, W, stream, sh, device, flush, peak)
+        with ClockSampler(local) as ck:
+            configs = workload_table(N, W, stream, sh, device, flush, peak)
+        table_clocks["configs"] = ck.summary()
+
+    gemms = layer = None
+    if not args.no_gemm:
+        with ClockSampler(local) as ck:
+            gemms = gemm_table(N, calls, stream, device)
+            layer = linear_layer_table(N, groups, stream, device, flush, tensors)
+        table_clocks["nvfp4_gemm+linear_layer"] = ck.summary()
 
     e2e = None
     if not args.no_e2e:
@@ -735,6 +741,8 @@ def run_ours(args, world, rank, local):
         result["nvfp4_gemm"] = gemms
     if layer is not None:
         result["linear_layer"] = layer
+    if table_clocks:
+        result["table_clocks"] = table_clocks
     if per_mode is not None:
         result["per_mode_dy"] = per_mode
     if configs is not None:
