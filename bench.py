@@ -52,9 +52,10 @@ L2_FLUSH_BYTES = 256 << 20
 # hash of the kernel sources they were taken with.  A changed kernel reports
 # traffic = null until it is captured again.
 NCU_TRAFFIC = {
-    # the ncu capture of the dominant kernel: dram__bytes_read.sum + dram__bytes_write.sum, one launch
-    ("99074ee665c907e2", "dy.transposed.ms_eden.g128"): 470025472 + 108604928,
-    ("99074ee665c907e2", "dy.rowwise.ms_eden.g128"): 469999616 + 110624256,
+    # the ncu capture of the dominant launch at full size (one pass):
+    # dram__bytes_read.sum + dram__bytes_write.sum, one launch
+    ("fa43c9f0070e72b0", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
+        472454400 + 224126976,
 }
 
 
