@@ -75,6 +75,48 @@ __device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) { return add2_rn(a
 __device__ __forceinline__ float2 add2_after_mul(float2 a, float2 b) { return f2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y)); }
 __device__ __forceinline__ float2 sub2_after_mul(float2 a, float2 b) { return f2(__fsub_rn(a.x, b.x), __fsub_rn(a.y, b.y)); }
 
+// max(|a|, |b|, |c|) in one three-input sm_100 max (exact; a NaN operand is
+// ignored as by fmaxf).
+__device__ __forceinline__ float absmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// max of N non-negative values, as a tree of three-input maxima (short
+// dependency chains for latency-bound reductions).
+template <int N>
+__device__ __forceinline__ float max_tree(const float (&m)[N]) {
+  if constexpr (N == 1) {
+    return m[0];
+  } else if constexpr (N == 2) {
+    return fmaxf(m[0], m[1]);
+  } else {
+    constexpr int M = (N + 2) / 3;
+    float r[M];
+#pragma unroll
+    for (int i = 0; i < N / 3; ++i) r[i] = max3(m[3 * i], m[3 * i + 1], m[3 * i + 2]);
+    if constexpr (N % 3 == 1) r[M - 1] = m[N - 1];
+    if constexpr (N % 3 == 2) r[M - 1] = fmaxf(m[N - 2], m[N - 1]);
+    return max_tree<M>(r);
+  }
+}
+// max |v[i]| of N values as a tree.
+template <int N>
+__device__ __forceinline__ float absmax_tree(const float (&v)[N]) {
+  constexpr int M = (N + 2) / 3;
+  float r[M];
+#pragma unroll
+  for (int i = 0; i < N / 3; ++i) r[i] = absmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  if constexpr (N % 3 == 1) r[M - 1] = fabsf(v[N - 1]);
+  if constexpr (N % 3 == 2) r[M - 1] = fmaxf(fabsf(v[N - 2]), fabsf(v[N - 1]));
+  return max_tree<M>(r);
+}
+
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy
 // as 1, 2, 3", SC'11): ten rounds of two 32x32->64 multiplications by the
@@ -315,6 +357,29 @@ __device__ __forceinline__ uint32_t int4_nibble(float y) {
   return (__float_as_uint(__fadd_rn(fabsf(k), 8388608.0f)) & 7u) | ((__float_as_uint(k) >> 28) & 8u);
 }
 
+// INT4 codes of eight values from the bits s_i of s = min(RN(|t_i| + 1.5
+// 2^23), 1.5 2^23 + 7) (|t_i| < 2^22), whose low byte is |k_i| =
+// min(RNE(|t_i|), 7), and a word whose bit 3 of nibble i holds the sign of
+// element i wherever |k_i| > 0: the low bytes gathered into nibbles with byte
+// permutes, the signs added, and a zero code cleared of its sign.
+__device__ __forceinline__ uint32_t int_nibbles8(const uint32_t* s, uint32_t signs) {
+  const uint32_t even = __byte_perm(__byte_perm(s[0], s[2], 0x0040u), __byte_perm(s[4], s[6], 0x4000u), 0x7610u);
+  const uint32_t odd = __byte_perm(__byte_perm(s[1], s[3], 0x0040u), __byte_perm(s[5], s[7], 0x4000u), 0x7610u);
+  return clear_negative_zero(even | (odd << 4) | (signs & 0x88888888u));
+}
+// The signs of eight floats in bit 3 of nibbles 0..7 (top bytes gathered).
+__device__ __forceinline__ uint32_t sign_nibbles8(const float* y) {
+  const uint32_t even = __byte_perm(__byte_perm(__float_as_uint(y[0]), __float_as_uint(y[2]), 0x0073u),
+                                    __byte_perm(__float_as_uint(y[4]), __float_as_uint(y[6]), 0x7300u), 0x7610u);
+  const uint32_t odd = __byte_perm(__byte_perm(__float_as_uint(y[1]), __float_as_uint(y[3]), 0x0073u),
+                                   __byte_perm(__float_as_uint(y[5]), __float_as_uint(y[7]), 0x7300u), 0x7610u);
+  return ((even >> 4) & 0x08080808u) | (odd & 0x80808080u);
+}
+// s = min(RN(|t| + 1.5 2^23), 1.5 2^23 + 7): RNE(|t|) clamped to 7 in its low bits.
+__device__ __forceinline__ float int_magnitude_sum(float t) {
+  return fminf(__fadd_rn(fabsf(t), kRoundMagic), kRoundMagic + 7.0f);
+}
+
 // 3-bit elements, stored in nibbles (sign bit 3, magnitude code bits 0..1).
 // E2M0: magnitudes {0, 1, 2, 4}, nearest with ties to the even code (0.5 ->
 // 0, 1.5 -> 2, 3 -> 2), saturating at 4; zero is code 0.
@@ -418,22 +483,31 @@ __device__ __forceinline__ void rtn_codes(const float* y, uint32_t& lo, uint32_t
 // the grid {0, 0.5, 1} is that of 0.5 + a/2 on [0.5, 1] (one kept bit below
 // 0.5), and 0.5 + a/2 rounded upward is exact for the decision: 64k * 2^-23
 // lies on the 2^-23 grid that the upward rounding lands on, so a - l exceeds
-// it iff the rounded value does.  max(a, RU(0.5 + a/2)) picks the right one
-// of the two (0.5 + a/2 <= a iff a >= 1).  2^22 - 1 - 64k = (64k) ^ (2^22 - 1).
-// Signs go in afterwards, and a code of magnitude 0 drops its sign.
+// it iff the rounded value does.  a1 = max(a, RU(0.5 + a/2)) picks the right
+// one of the two (0.5 + a/2 <= a iff a >= 1); taking the minimum with 6 last
+// gives the same a1 (a NaN or a value above 6 ends at 6 either way).
+// The sum is formed 64 times larger, modulo 2^32, so that the index lands in
+// bits 28..30 with bit 31 clear: v = 64 bits(a1) + 64 (2^22 - 1 - 64k - 252
+// 2^22), whose second term is ~k in bits 12..27, ones in bits 6..11 and 2^30.
+// The sign of y goes into bit 31, and the top nibbles of the eight v are
+// gathered into one word with byte permutes; a code of magnitude 0 drops its
+// sign.
 __device__ __forceinline__ uint32_t sr_codes8(const float* y, const uint4& w) {
-  uint32_t mag = 0u, sgn = 0u;
+  uint32_t v[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t word = word_of(w, static_cast<uint32_t>(i >> 1));
-    const uint32_t k64 = ((i & 1) ? (word >> 10) : (word << 6)) & 0x3FFFC0u;
-    const float a = fminf(fabsf(y[i]), 6.0f);
-    const float a1 = fmaxf(a, __fmaf_ru(a, 0.5f, 0.5f));
-    const uint32_t v = __float_as_uint(a1) + (k64 ^ 0x3FFFFFu) - (252u << 22);  // index in bits 22..24
-    mag |= (4 * i <= 22 ? v >> (22 - 4 * i) : v << (4 * i - 22)) & (7u << (4 * i));
-    sgn |= (__float_as_uint(y[i]) >> (28 - 4 * i)) & (8u << (4 * i));
+    const uint32_t k_at12 = (i & 1) ? (word >> 4) : (word << 12);  // k_i in bits 12..27
+    const uint32_t n = (~k_at12 & 0x0FFFF000u) | 0x40000FC0u;
+    const float a = fabsf(y[i]);
+    const float a1 = fminf(fmaxf(a, __fmaf_ru(a, 0.5f, 0.5f)), 6.0f);
+    const uint32_t t = __float_as_uint(a1) * 64u + n;
+    v[i] = (t & 0x7FFFFFFFu) | (__float_as_uint(y[i]) & 0x80000000u);
   }
-  return clear_negative_zero(mag | sgn);
+  // byte m of `even` / `odd` = top byte of v[2m] / v[2m+1]
+  const uint32_t even = __byte_perm(__byte_perm(v[0], v[2], 0x0073u), __byte_perm(v[4], v[6], 0x7300u), 0x7610u);
+  const uint32_t odd = __byte_perm(__byte_perm(v[1], v[3], 0x0073u), __byte_perm(v[5], v[7], 0x7300u), 0x7610u);
+  return clear_negative_zero(((even >> 4) & 0x0F0F0F0Fu) | (odd & 0xF0F0F0F0u));
 }
 
 // Quantize one block of 16 (already rotated) values z under tensor scale s_g.
@@ -704,23 +778,17 @@ __device__ __forceinline__ void sr_block(const float (&y)[16], PhiloxKey key, ui
   hi = sr_codes8(y + 8, philox_call(key, call0 + 1, kTagElement));
 }
 
-// max |z| of each of the two blocks of a pair, as a tree (exact in any order).
+// max |z| of each of the two blocks of a pair: one chain of three-input
+// maxima per block (exact in any order; two live values).
 __device__ __forceinline__ void absmax_pair(const float2 (&z)[16], float& aa, float& ab) {
-  float ma[8], mb[8];
+  float a = absmax3(z[0].x, z[1].x, z[2].x), b = absmax3(z[0].y, z[1].y, z[2].y);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    ma[i] = fmaxf(fabsf(z[2 * i].x), fabsf(z[2 * i + 1].x));
-    mb[i] = fmaxf(fabsf(z[2 * i].y), fabsf(z[2 * i + 1].y));
+  for (int i = 3; i < 15; i += 2) {
+    a = max3(a, fabsf(z[i].x), fabsf(z[i + 1].x));
+    b = max3(b, fabsf(z[i].y), fabsf(z[i + 1].y));
   }
-#pragma unroll
-  for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) {
-      ma[i] = fmaxf(ma[i], ma[i + w]);
-      mb[i] = fmaxf(mb[i], mb[i + w]);
-    }
-  aa = ma[0];
-  ab = mb[0];
+  aa = fmaxf(a, fabsf(z[15].x));
+  ab = fmaxf(b, fabsf(z[15].y));
 }
 
 // The scale table of one launch: for every E4M3 code S (0x7F, never produced,
@@ -843,20 +911,19 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
     const uint32_t Sa = S2 & 0xFFu, Sb = S2 >> 8;
     const float4 ta = scale_entry<TBL>(sc, Sa), tb = scale_entry<TBL>(sc, Sb);
     const float2 r = f2(ta.z, tb.z);  // RN(1/d), 0 for a zero scale: y = 0, codes 0
-    oa = BlockOut{0u, 0u, Sa};
-    ob = BlockOut{0u, 0u, Sb};
+    // k = clamp(RNE(y), -7, 7): |k| from int_magnitude_sum, the sign that of y
+    float ya[16], yb[16];
+    uint32_t sa[16], sb[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float2 y = mul2_rn(z[i], r);
-      const uint32_t ca = int4_nibble(y.x), cb = int4_nibble(y.y);
-      if (i < 8) {
-        oa.lo |= ca << (4 * i);
-        ob.lo |= cb << (4 * i);
-      } else {
-        oa.hi |= ca << (4 * (i - 8));
-        ob.hi |= cb << (4 * (i - 8));
-      }
+      ya[i] = y.x;
+      yb[i] = y.y;
+      sa[i] = __float_as_uint(int_magnitude_sum(y.x));
+      sb[i] = __float_as_uint(int_magnitude_sum(y.y));
     }
+    oa = BlockOut{int_nibbles8(sa, sign_nibbles8(ya)), int_nibbles8(sa + 8, sign_nibbles8(ya + 8)), Sa};
+    ob = BlockOut{int_nibbles8(sb, sign_nibbles8(yb)), int_nibbles8(sb + 8, sign_nibbles8(yb + 8)), Sb};
     return;
   } else if constexpr (MODE == kMXFP4) {
     // The pair is one 32-element MXFP4 group (block a its first half, b its
@@ -984,34 +1051,27 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
       e2m1x8_to_f32(fb_lo, vb);
       e2m1x8_to_f32(fb_hi, vb + 8);
       float2 eF = f2(0.0f, 0.0f), eI = f2(0.0f, 0.0f);
-      uint32_t ia_lo = 0u, ia_hi = 0u, ib_lo = 0u, ib_hi = 0u;
+      uint32_t sa[16], sb[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float2 y = f2(ya[i], yb[i]);
         const float2 dF = sub2_after_mul(y, f2(va[i], vb[i]));
         eF = fma2_rn(dF, dF, eF);
+        // the INT4 level k = clamp(RNE(y K1), -7, 7) through its magnitude:
+        // |k| = s - 1.5 2^23 exactly, and |y| - |k| K2 = +-(y - k K2), the
+        // same square (k is 0 or has the sign of y)
         const float2 t = mul2_rn(y, f2(kIF4K1, kIF4K1));
-        // k = clamp(RNE(t), -7, 7) with no conversion instruction: |t| < 2^22,
-        // so s = RN(t + 1.5 * 2^23) rounds t at the units bit (ties to even),
-        // s - 1.5 * 2^23 = RNE(t) exactly, and the bits of s are 0x4B400000 + RNE(t)
-        const float2 s2 = add2_after_mul(t, f2(kRoundMagic, kRoundMagic));
-        const float2 r2 = sub2_rn(s2, f2(kRoundMagic, kRoundMagic));
-        const float2 kf = f2(fminf(fmaxf(r2.x, -7.0f), 7.0f), fminf(fmaxf(r2.y, -7.0f), 7.0f));
-        const float2 vi = mul2_rn(kf, f2(kIF4K2, kIF4K2));
-        const float2 dI = sub2_after_mul(y, vi);
+        const float2 s2 = f2(int_magnitude_sum(t.x), int_magnitude_sum(t.y));
+        sa[i] = __float_as_uint(s2.x);
+        sb[i] = __float_as_uint(s2.y);
+        const float2 vi = mul2_rn(sub2_rn(s2, f2(kRoundMagic, kRoundMagic)), f2(kIF4K2, kIF4K2));
+        const float2 dI = f2(__fsub_rn(fabsf(y.x), vi.x), __fsub_rn(fabsf(y.y), vi.y));
         eI = fma2_rn(dI, dI, eI);
-        // sign-magnitude nibble of the integer kf (never -0): |k| is the low
-        // mantissa bits of 2^23 + |kf| (exact), the sign is bit 31 of kf
-        const uint32_t codea = (__float_as_uint(fabsf(kf.x) + 8388608.0f) & 7u) | ((__float_as_uint(kf.x) >> 28) & 8u);
-        const uint32_t codeb = (__float_as_uint(fabsf(kf.y) + 8388608.0f) & 7u) | ((__float_as_uint(kf.y) >> 28) & 8u);
-        if (i < 8) {
-          ia_lo |= codea << (4 * i);
-          ib_lo |= codeb << (4 * i);
-        } else {
-          ia_hi |= codea << (4 * (i - 8));
-          ib_hi |= codeb << (4 * (i - 8));
-        }
       }
+      // signs: a nonzero level needs RN(|y| K1) > 1/2, so |y| > 3/8, where
+      // the E2M1 code of y is nonzero and carries its sign
+      const uint32_t ia_lo = int_nibbles8(sa, fa_lo), ia_hi = int_nibbles8(sa + 8, fa_hi);
+      const uint32_t ib_lo = int_nibbles8(sb, fb_lo), ib_hi = int_nibbles8(sb + 8, fb_hi);
       const bool inta = eI.x < eF.x, intb = eI.y < eF.y;
       oa.lo = inta ? ia_lo : fa_lo;
       oa.hi = inta ? ia_hi : fa_hi;

@@ -10,15 +10,10 @@
 namespace nvfp4 {
 
 __device__ __forceinline__ float absmax64(const float2 (&z)[2][16]) {
-  float m[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-    m[i] = fmaxf(fmaxf(fabsf(z[0][i].x), fabsf(z[0][i].y)), fmaxf(fabsf(z[1][i].x), fabsf(z[1][i].y)));
-#pragma unroll
-  for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
-  return m[0];
+  float aa, ab, ac, ad;
+  absmax_pair(z[0], aa, ab);
+  absmax_pair(z[1], ac, ad);
+  return fmaxf(max3(aa, ab, ac), ad);
 }
 
 // Store the codes and scales of the four blocks of view row `vrow` starting at

@@ -368,14 +368,12 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
               __syncwarp();
               if (lane == 0) mbar_arrive(&sh.tfree[a]);
             }
-            float2 zp[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) zp[i] = mul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
             if constexpr (KIND == kAmax) {
-              float ma, mb;
-              absmax_pair(zp, ma, mb);
-              local_max = fmaxf(local_max, fmaxf(ma, mb));
+              local_max = fmaxf(local_max, absmax_tree<32>(v));  // of |acc|: scaled by c_g at the end
             } else {
+              float2 zp[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) zp[i] = mul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
               const int64_t c0 = vcol0 + 32 * p;  // view column of block 2p
               if (vrow < vrows && c0 < vcols) {
                 float4* dst = reinterpret_cast<float4*>(zout + vrow * vcols + c0);
@@ -393,6 +391,8 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
       }
     }
     if constexpr (KIND == kAmax) {
+      // RN(c t) is monotone in t >= 0: max RN(c |acc|) = RN(c max |acc|)
+      local_max = __fmul_rn(RhtConst<G>::c, local_max);
       const unsigned int bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(local_max));
       if (lane == 0) sh.warp_max[warp] = bits;
     }
@@ -506,16 +506,7 @@ __device__ __forceinline__ void build_rotation_b(uint8_t* bmat, PhiloxKey key, u
 
 // max |v| over 64 accumulator values (and m), as a tree: short dependency
 // chains, so a warp's reduction does not wait on its own previous result.
-__device__ __forceinline__ float absmax64(const float (&v)[64], float m) {
-  float t[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) t[i] = fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1]));
-#pragma unroll
-  for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
-  return fmaxf(m, t[0]);
-}
+__device__ __forceinline__ float absmax64(const float (&v)[64], float m) { return fmaxf(m, absmax_tree<64>(v)); }
 
 __global__ void __launch_bounds__(kDualThreads, 1)
 dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed, int g_r,
@@ -877,7 +868,6 @@ dual_amax_group_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, i
     const uint32_t q = warp & 3u, j = (warp >> 2) & 1u, grp = warp >> 3;
     grid_dependency_wait();
     const float c = rht_scale_of(j == 0 ? g_r : g_c);
-    const float2 c2 = f2(c, c);
     float m = 0.0f;
     int k = static_cast<int>(grp);
     if (j == 0 && g_r == 0) {
@@ -920,17 +910,11 @@ dual_amax_group_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, i
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.tfree[grp]);
         }
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          float2 zp[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) zp[i] = mul2_rn(f2(v[32 * p + 2 * i], v[32 * p + 2 * i + 1]), c2);
-          float ma, mb;
-          absmax_pair(zp, ma, mb);
-          m = fmaxf(m, fmaxf(ma, mb));
-        }
+        m = absmax64(v, m);
       }
     }
+    // max |acc| so far: RN(c t) is monotone in t >= 0, so max RN(c |acc|) = RN(c max |acc|)
+    m = __fmul_rn(c, m);
     }
     const unsigned int bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
     if (lane == 0) sh.warp_max[j][warp] = bits;
