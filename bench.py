@@ -80,6 +80,9 @@ def parse_args(argv=None):
                    help="profiling run: only one gradient-like tensor of this shape through the step's launches "
                         "(dual pre-pass, dual quantize, single-layout MS-EDEN and RTN quantizes), --steps times; "
                         "prints the per-launch times, not the benchmark line")
+    p.add_argument("--profile-modes", default="", metavar="MODES",
+                   help="with --profile-case: also quantize row-wise in these modes (comma-separated names, "
+                        "e.g. sr,if4,4over6), without rotation and with g = 128")
     p.add_argument("--no-unfused", action="store_true",
                    help="skip the comparison step with one quantize launch per call")
     p.add_argument("--no-eager", action="store_true",
@@ -910,8 +913,9 @@ def run_profile_case(args):
     captures that must stay within a few GB: a Student-t3 (std 1e-4) tensor of
     the given shape, and per iteration its dual pre-pass, its dual quantize
     (MS-EDEN both ways, and RTN rows + MS-EDEN columns), the single-layout
-    quantizes (MS-EDEN g = 128 both layouts, RTN row-wise), and the NVFP4 GEMM
-    of the RTN row-wise quantization with itself."""
+    quantizes (MS-EDEN g = 128 both layouts, RTN row-wise, and row-wise in the
+    modes of --profile-modes without rotation and with g = 128), and the NVFP4
+    GEMM of the RTN row-wise quantization with itself."""
     import ctypes
     from nvfp4_microscaling_quantization_b200 import binding as N
     from nvfp4_microscaling_quantization_b200 import workloads as W
@@ -925,6 +929,10 @@ def run_profile_case(args):
     calls = {(lay, mode, grp): Call(N, W.Call("p", lay, mode, grp), x, 11, sh)
              for lay, mode, grp in [(W.ROWWISE, W.MS_EDEN, 128), (W.TRANSPOSED, W.MS_EDEN, 128),
                                     (W.ROWWISE, W.RTN, 0)]}
+    by_name = {name: mode for mode, name in W.MODE_NAMES.items()}
+    for name in filter(None, args.profile_modes.split(",")):
+        for grp in (0, 128):
+            calls[(W.ROWWISE, by_name[name], grp)] = Call(N, W.Call("p", W.ROWWISE, by_name[name], grp), x, 11, sh)
     eden = TensorCalls(N, [calls[(W.ROWWISE, W.MS_EDEN, 128)], calls[(W.TRANSPOSED, W.MS_EDEN, 128)]])
     mixed = TensorCalls(N, [calls[(W.ROWWISE, W.RTN, 0)], calls[(W.TRANSPOSED, W.MS_EDEN, 128)]])
     body = [("amax_dual eden", eden.amax_passes), ("quantize_dual eden", eden.quantize_dual),
@@ -939,6 +947,8 @@ def run_profile_case(args):
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     times = {name: [] for name, _ in body}
     with torch.cuda.stream(stream):
+        for c in calls.values():  # every call's own tensor amax (the extra modes have no dual pre-pass)
+            c.amax_pass()
         for _, fn in body:        # first launches (module loading) outside the timing
             fn()
         torch.cuda.synchronize(device)

@@ -733,7 +733,7 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
 // warp (q, j) of a group reads lane quarter q of view j, 64 columns per load,
 // scales by c_g and reduces with a tree.  Measured faster than the slot ring
 // when every tile carries two MMAs; the results are identical.
-constexpr int kGrpStages = 3;     // A tiles in flight (each held until both MMAs are done)
+constexpr int kGrpStages = 5;     // A tiles in flight (each held until both MMAs are done)
 constexpr int kGrpGroups = 2;
 constexpr int kGrpEpiWarps = 8 * kGrpGroups;
 constexpr int kGrpThreads = (kGrpEpiWarps + 2) * 32;
@@ -751,6 +751,8 @@ struct GroupDualShared {
   int abort_flag;
   unsigned int warp_max[2][kGrpEpiWarps];
 };
+// 227 KB of shared memory per CTA on sm_100
+static_assert(kGrpDynSmem + sizeof(GroupDualShared) <= 227u * 1024u, "group pre-pass shared memory");
 
 __global__ void __launch_bounds__(kGrpThreads, 1)
 dual_amax_group_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed, int g_r,
