@@ -100,6 +100,13 @@ __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// One 32-byte global store (sm_100 st.global.v8.b32); dst 32-byte aligned.
+__device__ __forceinline__ void st_global_32B(void* dst, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 __device__ __forceinline__ bool aborted(GemmShared& sh) {
   return *reinterpret_cast<volatile int*>(&sh.abort_flag) != 0;
 }
@@ -281,6 +288,9 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     const uint32_t e = warp - kGEpiWarp0, q = warp & 3u, c_begin = 128u * (e >> 2);
     grid_dependency_wait();
     const float gab = __fmul_rn(*a_gscale, *b_gscale);
+    // 32-byte stores need D and its row pitch 32-byte aligned (one test for the launch)
+    const bool wide_stores =
+        ((reinterpret_cast<uintptr_t>(d) | static_cast<uintptr_t>(ldd * (OUT_BF16 ? 2 : 4))) & 31u) == 0;
     uint32_t tile = 0;
     for (int64_t t = blockIdx.x; t < n_tiles; t += step, ++tile) {
       const uint32_t a = tile % kGAccum;
@@ -309,25 +319,38 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[c4][i]);
+        // each thread writes its own row: 32-byte stores fill whole L2 sectors
+        // (half the store instructions and sector writes of 16-byte ones)
         if constexpr (OUT_BF16) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(d) + row * ldd + col0 + c);
+          uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint32_t w[4];
+          for (int k2 = 0; k2 < 16; ++k2) {
+            const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(v[2 * k2], gab), __fmul_rn(v[2 * k2 + 1], gab));
+            w[k2] = *reinterpret_cast<const uint32_t*>(&p);
+          }
+          uint8_t* dst = reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(d) + row * ldd + col0 + c);
+          if (wide_stores) {
+            st_global_32B(dst, w);
+            st_global_32B(dst + 32, w + 8);
+          } else {
 #pragma unroll
-            for (int k2 = 0; k2 < 4; ++k2) {
-              const __nv_bfloat162 p =
-                  __floats2bfloat162_rn(__fmul_rn(v[i + 2 * k2], gab), __fmul_rn(v[i + 2 * k2 + 1], gab));
-              w[k2] = *reinterpret_cast<const uint32_t*>(&p);
-            }
-            dst[i / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int i = 0; i < 4; ++i)
+              reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
           }
         } else {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(d) + row * ldd + col0 + c);
+          uint8_t* dst = reinterpret_cast<uint8_t*>(static_cast<float*>(d) + row * ldd + col0 + c);
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            dst[i / 4] = make_float4(__fmul_rn(v[i], gab), __fmul_rn(v[i + 1], gab), __fmul_rn(v[i + 2], gab),
-                                     __fmul_rn(v[i + 3], gab));
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) w[j] = __float_as_uint(__fmul_rn(v[8 * i + j], gab));
+            if (wide_stores) {
+              st_global_32B(dst + 32 * i, w);
+            } else {
+              reinterpret_cast<uint4*>(dst)[2 * i] = make_uint4(w[0], w[1], w[2], w[3]);
+              reinterpret_cast<uint4*>(dst)[2 * i + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+          }
         }
       }
     }

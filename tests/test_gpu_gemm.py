@@ -106,16 +106,21 @@ def test_gemm_bf16_output():
     assert np.all(np.abs(got - ref) <= GEMM_TOL * l1 + 2.0 ** -8 * np.abs(ref) + 1e-30)
 
 
-def test_gemm_output_row_stride():
+# Output row pitches: 32-byte aligned rows take the 32-byte store path, rows
+# aligned to 16 bytes only take the 16-byte one.
+@pytest.mark.parametrize("dtype,extra", [(torch.float32, 64), (torch.float32, 4), (torch.bfloat16, 8)])
+def test_gemm_output_row_stride(dtype, extra):
     m, n, k = 128, 256, 512
     a = tuple(t.to("cuda") for t in _operand(m, k, 601, POW2_SCALES))
     b = tuple(t.to("cuda") for t in _operand(n, k, 602, POW2_SCALES))
     one = torch.ones(1, dtype=torch.float32, device="cuda")
-    big = torch.full((m, n + 64), 7.0, dtype=torch.float32, device="cuda")
+    big = torch.full((m, n + extra), 7.0, dtype=dtype, device="cuda")
     N.gemm((a[0], a[1], one), (b[0], b[1], one), out=big[:, :n])
     torch.cuda.synchronize()
     ref = oracle.gemm(a[0].cpu().numpy(), a[1].cpu().numpy(), 1.0, b[0].cpu().numpy(), b[1].cpu().numpy(), 1.0)
-    assert np.array_equal(big[:, :n].cpu().numpy().astype(np.float64), ref)
+    # exact in fp32 (power-of-two scales); bf16 D is that value rounded to nearest even
+    want = torch.from_numpy(ref.astype(np.float32)).to(dtype).float().numpy().astype(np.float64)
+    assert np.array_equal(big[:, :n].float().cpu().numpy().astype(np.float64), want)
     assert torch.all(big[:, n:] == 7.0)  # columns past n untouched
 
 
