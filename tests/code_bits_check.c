@@ -1,0 +1,233 @@
+/* CPU check of the bit-level code formation the quantization kernels use,
+ * against the rules written from their definitions.
+ *
+ * (1) Stochastic rounding onto E2M1 (eight elements per 16-bit-uniform call).
+ *     Rule: a = min(|y|, 6); l = the largest grid value <= a, u the next one
+ *     (grid 0, 0.5, 1, 1.5, 2, 3, 4, 6); with U = k 2^-16 the magnitude goes
+ *     up iff U < (a - l) / (u - l); code = sign(y) << 3 | index, and a code of
+ *     magnitude 0 is 0.  Evaluated in binary64, where a - l and the quotient
+ *     by the power-of-two gap are exact.
+ *     Kernel form (restated): a1 = min(max(a, RU(0.5 a + 0.5)), 6);
+ *     t = 64 bits(a1) + ((~k << 12 & 0x0FFFF000) | 0x40000FC0) (mod 2^32);
+ *     v = (t & 0x7FFFFFFF) | (bits(y) & 0x80000000); the top nibbles of the
+ *     eight v gathered into one word with byte permutes, then the sign of a
+ *     zero magnitude cleared.
+ * (2) INT4 levels (NVINT4, and IF4's integer option).
+ *     Rule: k = clamp(RNE(t), -7, 7) as a sign-magnitude nibble, never -0.
+ *     Kernel form (restated): s = min(RN(|t| + 1.5 2^23), 1.5 2^23 + 7); the
+ *     low bytes of eight s gathered into nibbles with byte permutes, the
+ *     signs of the eight t added from their top bytes, then the sign of a
+ *     zero magnitude cleared.
+ * Byte permute: byte n of perm(x, y, s) is byte (nibble n of s) of the
+ * eight bytes y:x (x bytes 0..3, y bytes 4..7).
+ * Build: cc -O2 -ffp-contract=off -fno-fast-math -frounding-math, linked with
+ * -lm (the upward-rounded fused multiply-add runs under FE_UPWARD). */
+#include <fenv.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+static float from_bits(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t to_bits(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+static uint32_t perm(uint32_t x, uint32_t y, uint32_t s) {
+  const uint64_t b = ((uint64_t)y << 32) | x;
+  uint32_t r = 0;
+  for (int n = 0; n < 4; ++n) r |= (uint32_t)((b >> (8 * ((s >> (4 * n)) & 7u))) & 0xFFu) << (8 * n);
+  return r;
+}
+static uint32_t clear_negative_zero(uint32_t w) {
+  uint32_t out = 0;
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t c = (w >> (4 * i)) & 0xFu;
+    out |= ((c & 7u) ? c : 0u) << (4 * i);
+  }
+  return out;
+}
+static float fma_up(float a, float b, float c) {
+  const int old = fegetround();
+  fesetround(FE_UPWARD);
+  volatile float r = fmaf(a, b, c);
+  fesetround(old);
+  return r;
+}
+
+/* ------------------------------------------------------------------ SR */
+static const double kGrid[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+static uint32_t sr_rule(float y, uint32_t k) {
+  double a = fabs((double)y);
+  if (!(a <= 6.0)) a = 6.0;
+  int i = 0;
+  while (i < 7 && kGrid[i + 1] <= a) ++i;
+  uint32_t idx = (uint32_t)i;
+  if (i < 7 && (double)k * 0x1p-16 < (a - kGrid[i]) / (kGrid[i + 1] - kGrid[i])) idx = (uint32_t)i + 1u;
+  return idx == 0 ? 0u : (idx | (signbit(y) ? 8u : 0u));
+}
+
+/* the eight-element kernel form; k[i] = draw of element i, held as the
+ * generator delivers it: word i/2, low half for even i, high for odd */
+static uint32_t sr_kernel8(const float* y, const uint32_t* k) {
+  uint32_t word[4], v[8];
+  for (int m = 0; m < 4; ++m) word[m] = k[2 * m] | (k[2 * m + 1] << 16);
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t k_at12 = (i & 1) ? (word[i >> 1] >> 4) : (word[i >> 1] << 12);
+    const uint32_t n = (~k_at12 & 0x0FFFF000u) | 0x40000FC0u;
+    const float a = fabsf(y[i]);
+    const float a1 = fminf(fmaxf(a, fma_up(a, 0.5f, 0.5f)), 6.0f);
+    const uint32_t t = to_bits(a1) * 64u + n;
+    v[i] = (t & 0x7FFFFFFFu) | (to_bits(y[i]) & 0x80000000u);
+  }
+  const uint32_t even = perm(perm(v[0], v[2], 0x0073u), perm(v[4], v[6], 0x7300u), 0x7610u);
+  const uint32_t odd = perm(perm(v[1], v[3], 0x0073u), perm(v[5], v[7], 0x7300u), 0x7610u);
+  return clear_negative_zero(((even >> 4) & 0x0F0F0F0Fu) | (odd & 0xF0F0F0F0u));
+}
+
+/* The draws next to the decision point of y: k with k 2^-16 just below and
+ * above (a - l)/(u - l), and the extremes. */
+static int decision_draws(float y, uint32_t* out) {
+  double a = fabs((double)y);
+  if (!(a <= 6.0)) a = 6.0;
+  int i = 0;
+  while (i < 7 && kGrid[i + 1] <= a) ++i;
+  const double f = i < 7 ? (a - kGrid[i]) / (kGrid[i + 1] - kGrid[i]) : 0.0;
+  const int64_t c = (int64_t)floor(f * 65536.0);
+  int n = 0;
+  for (int64_t d = -2; d <= 2; ++d)
+    if (c + d >= 0 && c + d <= 65535) out[n++] = (uint32_t)(c + d);
+  out[n++] = 0;
+  out[n++] = 65535;
+  return n;
+}
+
+static uint64_t rng_state;
+static uint64_t next64(void) {
+  rng_state ^= rng_state << 13;
+  rng_state ^= rng_state >> 7;
+  rng_state ^= rng_state << 17;
+  return rng_state;
+}
+
+/* Every finite bf16 value (both signs) at the draws next to its decision
+ * point, each as element `slot` of an eight-element word whose other
+ * elements are random; then `n_random` words of random binary32 values in
+ * (-8, 8) with random draws.  Returns the number of elements whose code
+ * differs from the rule; *checked receives the number compared. */
+int64_t sr_check(int64_t n_random, int variant, int64_t* checked) {
+  int64_t bad = 0, n = 0;
+  rng_state = 0x9E3779B97F4A7C15ull;
+  for (uint32_t h = 0; h < 65536u; ++h) {
+    const float y0 = from_bits(h << 16);
+    if (!isfinite(y0)) continue;
+    uint32_t ks[8];
+    const int nk = decision_draws(y0, ks);
+    for (int j = 0; j < nk; ++j) {
+      float y[8];
+      uint32_t k[8];
+      const int slot = (int)(next64() & 7u);
+      for (int e = 0; e < 8; ++e) {
+        y[e] = from_bits((uint32_t)next64() & 0xC0FFFFFFu);  /* |y| < 8 */
+        k[e] = (uint32_t)next64() & 0xFFFFu;
+      }
+      y[slot] = y0;
+      k[slot] = ks[j];
+      uint32_t w = sr_kernel8(y, k);
+      if (variant == 1) w ^= 1u << (4 * slot);  /* a planted mistake: one index bit flipped */
+      for (int e = 0; e < 8; ++e) {
+        ++n;
+        bad += ((w >> (4 * e)) & 0xFu) != sr_rule(y[e], k[e]);
+      }
+    }
+  }
+  for (int64_t r = 0; r < n_random; ++r) {
+    float y[8];
+    uint32_t k[8];
+    for (int e = 0; e < 8; ++e) {
+      y[e] = from_bits((uint32_t)next64() & 0xC0FFFFFFu);
+      k[e] = (uint32_t)next64() & 0xFFFFu;
+    }
+    /* below 1, where 0.5 + a/2 is inexact and its upward rounding decides:
+     * one element of each word at a draw next to its decision point */
+    if (r & 1) {
+      uint32_t ks[8];
+      const int slot = (int)(next64() & 7u);
+      y[slot] = from_bits(((uint32_t)next64() & 0x807FFFFFu) | 0x3F000000u) * (float)((next64() & 1u) + 1u) * 0.5f;
+      const int nk = decision_draws(y[slot], ks);
+      k[slot] = ks[next64() % (uint64_t)nk];
+    }
+    const uint32_t w = sr_kernel8(y, k);
+    for (int e = 0; e < 8; ++e) {
+      ++n;
+      bad += ((w >> (4 * e)) & 0xFu) != sr_rule(y[e], k[e]);
+    }
+  }
+  *checked = n;
+  return bad;
+}
+
+/* ------------------------------------------------------------------ INT4 */
+static uint32_t int4_rule(float t) {
+  double k = nearbyint((double)t);  /* ties to even (default rounding mode) */
+  if (k > 7.0) k = 7.0;
+  if (k < -7.0) k = -7.0;
+  const int ki = (int)k;
+  return ki == 0 ? 0u : ((uint32_t)(ki < 0 ? -ki : ki) | (ki < 0 ? 8u : 0u));
+}
+
+static uint32_t int4_kernel8(const float* t) {
+  const float magic = 12582912.0f;  /* 1.5 2^23 */
+  uint32_t s[8];
+  for (int i = 0; i < 8; ++i) s[i] = to_bits(fminf(fabsf(t[i]) + magic, magic + 7.0f));
+  const uint32_t even = perm(perm(s[0], s[2], 0x0040u), perm(s[4], s[6], 0x4000u), 0x7610u);
+  const uint32_t odd = perm(perm(s[1], s[3], 0x0040u), perm(s[5], s[7], 0x4000u), 0x7610u);
+  const uint32_t se = perm(perm(to_bits(t[0]), to_bits(t[2]), 0x0073u), perm(to_bits(t[4]), to_bits(t[6]), 0x7300u), 0x7610u);
+  const uint32_t so = perm(perm(to_bits(t[1]), to_bits(t[3]), 0x0073u), perm(to_bits(t[5]), to_bits(t[7]), 0x7300u), 0x7610u);
+  const uint32_t signs = ((se >> 4) & 0x08080808u) | (so & 0x80808080u);
+  return clear_negative_zero(even | (odd << 4) | (signs & 0x88888888u));
+}
+
+/* Values t: every multiple of 1/4 in [-10, 10] (the ties x.5 among them, and
+ * values past the clamp), their binary32 neighbours, every finite bf16 value
+ * (at 2^22 and above RN(|t| + 1.5 2^23) is past the clamp as well), and
+ * random binary32 values in (-16, 16); eight per word in order.  Returns the
+ * number of elements whose nibble differs from the rule. */
+int64_t int4_check(int64_t n_random, int variant, int64_t* checked) {
+  int64_t bad = 0, n = 0;
+  rng_state = 0xD1B54A32D192ED03ull;
+  float vals[8];
+  int nv = 0;
+#define FLUSH()                                                              \
+  do {                                                                       \
+    uint32_t w = int4_kernel8(vals);                                         \
+    if (variant == 1) w ^= 4u;                                               \
+    for (int e = 0; e < nv; ++e) {                                           \
+      ++n;                                                                   \
+      bad += ((w >> (4 * e)) & 0xFu) != int4_rule(vals[e]);                  \
+    }                                                                        \
+    nv = 0;                                                                  \
+  } while (0)
+#define PUSH(x)                                                              \
+  do {                                                                       \
+    vals[nv++] = (x);                                                        \
+    if (nv == 8) FLUSH();                                                    \
+  } while (0)
+  for (int q = -40; q <= 40; ++q) {
+    const float t = (float)q * 0.25f;
+    PUSH(t);
+    PUSH(nextafterf(t, INFINITY));
+    PUSH(nextafterf(t, -INFINITY));
+  }
+  for (uint32_t h = 0; h < 65536u; ++h) {
+    const float t = from_bits(h << 16);
+    if (isfinite(t)) PUSH(t);
+  }
+  for (int64_t r = 0; r < n_random; ++r) PUSH(from_bits((uint32_t)next64() & 0xC1FFFFFFu));
+  if (nv) {
+    while (nv < 8) vals[nv++] = 0.0f;
+    FLUSH();
+  }
+#undef PUSH
+#undef FLUSH
+  *checked = n;
+  return bad;
+}

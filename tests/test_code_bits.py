@@ -1,0 +1,62 @@
+"""The kernels' bit-level formation of codes, pinned on the CPU.
+
+Stochastic rounding onto E2M1 and the INT4 levels of NVINT4 and IF4 are
+formed in the kernels without conversion instructions: integer sums on the
+bits of the floats, and byte permutes that gather eight elements' nibbles
+into one code word.  tests/code_bits_check.c restates those sequences in C
+and compares every element, bit for bit, with the rules written from their
+definitions: stochastic rounding goes up iff U < (a - l)/(u - l) (the
+palettes post, "The two corners, and what the palette does to them"), the
+INT4 level is clamp(RNE(t), -7, 7) as a sign-magnitude nibble (IF4 paper
+page, Table 1 and Figure 3).  Inputs: every finite bf16 value at the draws
+next to its decision point and at the extremes, in random word slots, plus
+random binary32 values; the ties, clamp edges and signed zeros of the INT4
+levels.  No difference is allowed.
+"""
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+@pytest.fixture(scope="module")
+def checker():
+    d = tempfile.mkdtemp(prefix="code_bits_")
+    so = os.path.join(d, "code_bits_check.so")
+    subprocess.run(["cc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-frounding-math", "-fPIC", "-shared",
+                    os.path.join(HERE, "code_bits_check.c"), "-o", so, "-lm"], check=True)
+    L = ctypes.CDLL(so)
+    for fn in (L.sr_check, L.int4_check):
+        fn.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
+        fn.restype = ctypes.c_int64
+    return L
+
+
+def _run(fn, n_random, variant=0):
+    n = ctypes.c_int64(0)
+    bad = fn(n_random, variant, ctypes.byref(n))
+    return bad, n.value
+
+
+def test_planted_mistakes_are_caught(checker):
+    """The comparisons have teeth: one flipped code bit per word is found."""
+    bad, n = _run(checker.sr_check, 0, variant=1)
+    assert bad > 100000 and n > 0
+    bad, n = _run(checker.int4_check, 0, variant=1)
+    assert bad > 1000 and n > 0
+
+
+def test_stochastic_rounding_codes(checker):
+    bad, n = _run(checker.sr_check, 1 << 18)
+    assert n > 3_000_000
+    assert bad == 0, f"{bad} of {n} stochastic-rounding codes differ from the rule"
+
+
+def test_int4_level_codes(checker):
+    bad, n = _run(checker.int4_check, 1 << 20)
+    assert n > 1_000_000
+    assert bad == 0, f"{bad} of {n} INT4 nibbles differ from the rule"
