@@ -22,6 +22,7 @@ CPU oracle, run over ranges of view rows on every host core, on a bounded
 sample of the same workload.
 """
 import argparse
+import ctypes
 import datetime
 import hashlib
 import json
@@ -224,7 +225,6 @@ class Call:
     """One quantization call bound to device buffers, issued through the raw C ABI."""
 
     def __init__(self, N, call, x, seed, stream_handle):
-        import ctypes
         self.N, self.call, self.x, self.seed = N, call, x, seed
         rows, cols = x.shape
         self.rows, self.cols, self.ld = rows, cols, x.stride(0)
@@ -300,6 +300,90 @@ class TensorCalls:
     def launches(self, fused=True):
         pre = 1 if self.dual else len(self.calls)
         return pre + (1 if fused and self.dual else len(self.calls))
+
+    def label(self):
+        return self.calls[0].call.tensor
+
+    def prepass_elements(self):
+        """Elements the pre-pass launch(es) read."""
+        return self.calls[0].elements if self.dual else sum(c.elements for c in self.calls)
+
+    def dual_calls(self):
+        return [self.row, self.col]
+
+
+class DualGroupCalls:
+    """Several tensors quantized in both layouts with the same modes and
+    rotation groups (the linear layer's forward operands X and W): one
+    both-layout pre-pass launch and one both-layout quantize launch for all
+    of them (nvfp4_amax_dual_group, nvfp4_quantize_dual_group), each walking
+    all their tiles with one persistent grid."""
+
+    def __init__(self, N, members):
+        self.N, self.members, self.dual = N, members, True
+        self.calls = [c for m in members for c in m.calls]
+        rows, cols = [m.row for m in members], [m.col for m in members]
+        self.n = len(members)
+        r0, c0 = rows[0], cols[0]
+        self.modes = (r0.call.mode, r0.call.rht_group, c0.call.mode, c0.call.rht_group)
+        self.seed, self.stream = r0.seed, r0.stream
+        ptrs = lambda vals: (ctypes.c_void_p * self.n)(*vals)  # noqa: E731
+        i64s = lambda vals: (ctypes.c_int64 * self.n)(*vals)  # noqa: E731
+        self.a = dict(x=ptrs([r.p["x"] for r in rows]), rows=i64s([r.rows for r in rows]),
+                      cols=i64s([r.cols for r in rows]), ld=i64s([r.ld for r in rows]),
+                      amax_r=ptrs([r.p["amax"] for r in rows]), amax_c=ptrs([c.p["amax"] for c in cols]),
+                      codes_r=ptrs([r.p["codes"] for r in rows]), scales_r=ptrs([r.p["scales"] for r in rows]),
+                      gscale_r=ptrs([r.p["gscale"] for r in rows]), codes_c=ptrs([c.p["codes"] for c in cols]),
+                      scales_c=ptrs([c.p["scales"] for c in cols]), gscale_c=ptrs([c.p["gscale"] for c in cols]))
+
+    def amax_passes(self):
+        a, (_, g_r, _, g_c) = self.a, self.modes
+        st = self.N.nvfp4_amax_dual_group(self.n, a["x"], a["rows"], a["cols"], a["ld"], g_r, g_c, self.seed,
+                                          a["amax_r"], a["amax_c"], self.stream)
+        if st:
+            raise self.N.Nvfp4Error(st, "nvfp4_amax_dual_group")
+
+    def quantize_dual(self):
+        a, (m_r, g_r, m_c, g_c) = self.a, self.modes
+        st = self.N.nvfp4_quantize_dual_group(self.n, a["x"], a["rows"], a["cols"], a["ld"], m_r, g_r, m_c, g_c,
+                                              self.seed, a["amax_r"], a["amax_c"], a["codes_r"], a["scales_r"],
+                                              a["gscale_r"], a["codes_c"], a["scales_c"], a["gscale_c"],
+                                              self.stream)
+        if st:
+            raise self.N.Nvfp4Error(st, "nvfp4_quantize_dual_group")
+
+    def body(self, fused=True):
+        return [(self.amax_passes, "amax", self), (self.quantize_dual, "dual", self)]
+
+    def launches(self, fused=True):
+        return 2
+
+    def label(self):
+        return "+".join(m.label() for m in self.members)
+
+    def prepass_elements(self):
+        return sum(m.row.elements for m in self.members)
+
+    def dual_calls(self):
+        return [c for m in self.members for c in (m.row, m.col)]
+
+
+def group_step_parts(parts):
+    """The step's launch groups: tensors quantized in both layouts with the
+    same modes and rotation groups share a DualGroupCalls (in order of first
+    appearance); the others keep their own."""
+    out, by_modes = [], {}
+    for p in parts:
+        if not p.dual:
+            out.append([p])
+            continue
+        key = (p.row.call.mode, p.row.call.rht_group, p.col.call.mode, p.col.call.rht_group)
+        if key in by_modes:
+            by_modes[key].append(p)
+        else:
+            by_modes[key] = [p]
+            out.append(by_modes[key])
+    return [ms[0] if len(ms) == 1 else DualGroupCalls(ms[0].N, ms) for ms in out]
 
 
 def dist_us(seconds):
@@ -468,9 +552,10 @@ def gemm_table(N, calls, stream, device, reps=10):
 def linear_layer_table(N, groups, stream, device, flush, tensors, reps=10):
     """The Quartet II linear layer of the MLP up-projection, fully NVFP4, as
     one forward and one backward pass:
-      forward : per operand (X, W) the dual pre-pass and the dual quantize
-                (row-wise RTN for Y, transposed MS-EDEN kept for the backward
-                pass), then Y = X W^T (nvfp4_gemm, bf16 out);
+      forward : X and W's both-layout pre-pass and both-layout quantize, one
+                launch each for the two operands (row-wise RTN for Y,
+                transposed MS-EDEN kept for the backward pass), then
+                Y = X W^T (nvfp4_gemm, bf16 out);
       backward: dY's dual pre-pass and dual quantize (MS-EDEN both ways),
                 then dX = dY W and dW = dY^T X (nvfp4_gemm, bf16 out).
     Timed inside CUDA graphs (L2 flushed before each repetition), beside the
@@ -484,8 +569,8 @@ def linear_layer_table(N, groups, stream, device, flush, tensors, reps=10):
     y = torch.empty(x.shape[0], w.shape[0], dtype=torch.bfloat16, device=device)
     dx = torch.empty(dy.shape[0], w.shape[1], dtype=torch.bfloat16, device=device)
     dw = torch.empty(dy.shape[1], x.shape[1], dtype=torch.bfloat16, device=device)
-    fwd = [gx.amax_passes, gw.amax_passes, gx.quantize_dual, gw.quantize_dual,
-           lambda: N.gemm(q(gx.row), q(gw.row), out=y)]
+    gxw = DualGroupCalls(N, [gx, gw])
+    fwd = [gxw.amax_passes, gxw.quantize_dual, lambda: N.gemm(q(gx.row), q(gw.row), out=y)]
     bwd = [gdy.amax_passes, gdy.quantize_dual,
            lambda: N.gemm(q(gdy.row), q(gw.col), out=dx),
            lambda: N.gemm(q(gdy.col), q(gx.col), out=dw)]
@@ -509,7 +594,7 @@ def linear_layer_table(N, groups, stream, device, flush, tensors, reps=10):
     f, b, r = dist_us(t_fwd), dist_us(t_bwd), dist_us(t_bf)
     m, k, n = x.shape[0], x.shape[1], w.shape[0]
     flops = 3 * 2.0 * m * n * k
-    names_f = ["amax_dual x", "amax_dual w", "quantize_dual x", "quantize_dual w", "gemm Y = X W^T"]
+    names_f = ["amax_dual x+w", "quantize_dual x+w", "gemm Y = X W^T"]
     names_b = ["amax_dual dy", "quantize_dual dy", "gemm dX = dY W", "gemm dW = dY^T X"]
     step_us = f["median"] + b["median"]
     return {
@@ -528,7 +613,6 @@ def linear_layer_table(N, groups, stream, device, flush, tensors, reps=10):
 
 
 def run_ours(args, world, rank, local):
-    import ctypes
     from nvfp4_microscaling_quantization_b200 import binding as N
     from nvfp4_microscaling_quantization_b200 import workloads as W
 
@@ -541,20 +625,22 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.Stream(device)
     sh = ctypes.c_void_p(stream.cuda_stream)
     calls = [Call(N, c, tensors[c.tensor], wl.seed, sh) for c in wl.calls]
-    groups = [TensorCalls(N, [c for c in calls if c.call.tensor == name])
-              for name in dict.fromkeys(c.tensor for c in wl.calls)]
+    per_tensor = [TensorCalls(N, [c for c in calls if c.call.tensor == name])
+                  for name in dict.fromkeys(c.tensor for c in wl.calls)]
+    groups = group_step_parts(per_tensor)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     bytes_per_step = sum(BYTES_PER_ELEMENT * c.elements for c in calls)
     elems_per_step = sum(c.elements for c in calls)
-    # one step = per tensor its dual pre-pass, then its dual quantize (both
-    # layouts from one read): 6 launches; the unfused step (one quantize per
-    # call, 9 launches) is timed too, for comparison
+    # one step = per launch group (X and W together, dY alone) its both-layout
+    # pre-pass, then its both-layout quantize (both layouts from one read): 4
+    # launches; the unfused step (per tensor a pre-pass, one quantize per call,
+    # 9 launches) is timed too, for comparison
     body, body_names = [], []
     for grp in groups:
         for fn, kind, obj in grp.body(fused=True):
             body.append(fn)
             body_names.append((kind, obj))
-    body_unfused = [fn for grp in groups for fn, _, _ in grp.body(fused=False)]
+    body_unfused = [fn for grp in per_tensor for fn, _, _ in grp.body(fused=False)]
 
     def step():
         for fn in body:
@@ -617,14 +703,14 @@ def run_ours(args, world, rank, local):
         if kind == "quant":
             return BYTES_PER_ELEMENT * obj.elements
         if kind == "dual":
-            return (PREPASS_BYTES_PER_ELEMENT + 2 * (BYTES_PER_ELEMENT - 2.0)) * obj.row.elements
-        return PREPASS_BYTES_PER_ELEMENT * obj.calls[0].elements
+            return (PREPASS_BYTES_PER_ELEMENT + 2 * (BYTES_PER_ELEMENT - 2.0)) * obj.prepass_elements()
+        return PREPASS_BYTES_PER_ELEMENT * obj.prepass_elements()
 
     def launch_name(kind, obj):
         if kind == "quant":
             return f"quantize {obj.call.name}"
-        t = obj.calls[0].call.tensor
-        return (f"quantize_dual {t} ({obj.row.call.name} + {obj.col.call.name})" if kind == "dual"
+        t = obj.label()
+        return (f"quantize_dual {t} ({' + '.join(c.call.name for c in obj.dual_calls())})" if kind == "dual"
                 else f"amax_{'dual' if obj.dual else 'single'} {t}")
 
     # dominant kernel: the quantize launch with the largest mean duration in the step
@@ -633,7 +719,7 @@ def run_ours(args, world, rank, local):
     dom_stats = dist_us(per_fn[dom_i])
     # algorithmic bytes: 2.5625 B per element of every call the launch serves
     # (two calls for a both-layout launch); moved bytes: what it must transfer
-    dom_calls = [dom] if dom_kind == "quant" else [dom.row, dom.col]
+    dom_calls = [dom] if dom_kind == "quant" else dom.dual_calls()
     dom_bytes = sum(BYTES_PER_ELEMENT * c.elements for c in dom_calls)
     dom_moved = moved_bytes(dom_kind, dom)
     achieved = dom_bytes / (dom_stats["mean"] / 1e6) / 1e9
@@ -649,7 +735,7 @@ def run_ours(args, world, rank, local):
         if kind == "amax":
             line["read_gbs"] = round(moved_bytes(kind, obj) / t / 1e9, 1)
         else:
-            calls_of = [obj] if kind == "quant" else [obj.row, obj.col]
+            calls_of = [obj] if kind == "quant" else obj.dual_calls()
             metric_bytes = sum(BYTES_PER_ELEMENT * c.elements for c in calls_of)
             line.update({"for_calls": [c.call.name for c in calls_of],
                          "gbs": round(metric_bytes / t / 1e9, 1),
@@ -690,7 +776,7 @@ def run_ours(args, world, rank, local):
     if not args.no_gemm:
         with ClockSampler(local) as ck:
             gemms = gemm_table(N, calls, stream, device)
-            layer = linear_layer_table(N, groups, stream, device, flush, tensors)
+            layer = linear_layer_table(N, per_tensor, stream, device, flush, tensors)
         table_clocks["nvfp4_gemm+linear_layer"] = ck.summary()
 
     e2e = None
@@ -772,13 +858,12 @@ def run_e2e(args, calls, tensors, stream, device, world, bytes_per_step):
     copies (another stream) of step i-1, the kernels run on a third, and the
     outputs are double-buffered so step i's kernels never overwrite what step
     i-1 is still copying out."""
-    import ctypes
     N = calls[0].N
     s_in, s_comp, s_out = (torch.cuda.Stream(device) for _ in range(3))
     sh = ctypes.c_void_p(s_comp.cuda_stream)
     sets = [[Call(N, c.call, tensors[c.call.tensor], c.seed, sh) for c in calls] for _ in range(2)]
-    group_sets = [[TensorCalls(N, [c for c in cs if c.call.tensor == name])
-                   for name in dict.fromkeys(c.call.tensor for c in cs)] for cs in sets]
+    group_sets = [group_step_parts([TensorCalls(N, [c for c in cs if c.call.tensor == name])
+                                    for name in dict.fromkeys(c.call.tensor for c in cs)]) for cs in sets]
     host_in = {k: v.cpu().pin_memory() for k, v in tensors.items()}
     host_out = [(torch.empty(c.codes.shape, dtype=torch.uint8).pin_memory(),
                  torch.empty(c.scales.shape, dtype=torch.uint8).pin_memory(),
@@ -918,7 +1003,6 @@ def run_profile_case(args):
     quantizes (MS-EDEN g = 128 both layouts, RTN row-wise, and row-wise in the
     modes of --profile-modes without rotation and with g = 128), and the NVFP4
     GEMM of the RTN row-wise quantization with itself."""
-    import ctypes
     from nvfp4_microscaling_quantization_b200 import binding as N
     from nvfp4_microscaling_quantization_b200 import workloads as W
     rows, cols = (int(v) for v in args.profile_case.lower().split("x"))

@@ -148,6 +148,24 @@ NVFP4_API int nvfp4_amax_dual(const void* x, int64_t rows, int64_t cols, int64_t
                               int rht_group_col, uint64_t seed, float* amax_row, float* amax_col,
                               void* stream);
 
+/* The largest n the group calls below take. */
+#define NVFP4_MAX_GROUP 64
+
+/* nvfp4_amax_dual for n tensors at once (1 <= n <= NVFP4_MAX_GROUP): member i
+ * is (x[i], rows[i], cols[i], ld[i]) with outputs amax_row[i], amax_col[i];
+ * the rotation groups and the seed are common to all.  The results are those
+ * of n nvfp4_amax_dual calls bit for bit.  A linear layer's forward operands
+ * X and W are both measured before their quantization (Quartet II article,
+ * section "Quantisierung im Vorwaertsdurchlauf"); with an unrotated row view
+ * (rht_group_row = 0) up to four members share one launch, which walks all
+ * their tiles with one persistent grid (one ramp and one tail instead of
+ * one per tensor).  x, rows, cols, ld, amax_row, amax_col: host arrays of n
+ * entries (the tensors and outputs they point to are device memory).
+ * Checks: every member as nvfp4_amax_dual, all before any launch. */
+NVFP4_API int nvfp4_amax_dual_group(int n, const void* const* x, const int64_t* rows, const int64_t* cols,
+                                    const int64_t* ld, int rht_group_row, int rht_group_col, uint64_t seed,
+                                    float* const* amax_row, float* const* amax_col, void* stream);
+
 /* Quantize x to packed E2M1/INT4 codes, E4M3 block scales and the FP32
  * tensor scale, in the given layout and mode (see the conventions above).
  *  amax_in:   device float holding the tensor amax of the (rotated) view, or
@@ -195,6 +213,27 @@ NVFP4_API int nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int
                                   const float* amax_row, const float* amax_col, uint8_t* codes_row,
                                   uint8_t* scales_row, float* gscale_row, uint8_t* codes_col,
                                   uint8_t* scales_col, float* gscale_col, void* stream);
+
+/* nvfp4_quantize_dual for n tensors at once (1 <= n <= NVFP4_MAX_GROUP):
+ * member i is (x[i], rows[i], cols[i], ld[i]) with amaxes amax_row[i],
+ * amax_col[i] and outputs codes_row[i], scales_row[i], gscale_row[i],
+ * codes_col[i], scales_col[i], gscale_col[i]; the modes, rotation groups and
+ * seed are common to all.  The results are those of n nvfp4_quantize_dual
+ * calls bit for bit.  Members on the fused path (see nvfp4_quantize_dual)
+ * share one launch, up to four at a time -- a linear layer's forward operands
+ * X and W, both quantized in both layouts (Quartet II article, section
+ * "Quantisierung im Vorwaertsdurchlauf"), in one pass with one ramp and one
+ * tail; the others run as their single calls.  All pointer arguments are
+ * host arrays of n entries (pointing to device memory); entries of the MX
+ * modes' amax arrays may be NULL.  Checks: every member as
+ * nvfp4_quantize_dual, all before any launch. */
+NVFP4_API int nvfp4_quantize_dual_group(int n, const void* const* x, const int64_t* rows, const int64_t* cols,
+                                        const int64_t* ld, int mode_row, int rht_group_row, int mode_col,
+                                        int rht_group_col, uint64_t seed, const float* const* amax_row,
+                                        const float* const* amax_col, uint8_t* const* codes_row,
+                                        uint8_t* const* scales_row, float* const* gscale_row,
+                                        uint8_t* const* codes_col, uint8_t* const* scales_col,
+                                        float* const* gscale_col, void* stream);
 
 /* Decode a quantized view (vrows x vcols) back to fp32:
  * out[r][j] = value(code, flag) * RN(E4M3(scale & 0x7F) * s_g), and, when

@@ -50,6 +50,12 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_quantize.restype = i32
         L.nvfp4_quantize_dual.argtypes = [P, i64, i64, i64, i32, i32, i32, i32, u64, P, P, P, P, P, P, P, P, P]
         L.nvfp4_quantize_dual.restype = i32
+        PP, I64P = ctypes.POINTER(P), ctypes.POINTER(i64)
+        L.nvfp4_amax_dual_group.argtypes = [i32, PP, I64P, I64P, I64P, i32, i32, u64, PP, PP, P]
+        L.nvfp4_amax_dual_group.restype = i32
+        L.nvfp4_quantize_dual_group.argtypes = [i32, PP, I64P, I64P, I64P, i32, i32, i32, i32, u64,
+                                                PP, PP, PP, PP, PP, PP, PP, PP, P]
+        L.nvfp4_quantize_dual_group.restype = i32
         L.nvfp4_dequantize.argtypes = [P, P, P, i64, i64, i32, i32, u64, i32, P, P]
         L.nvfp4_dequantize.restype = i32
         L.nvfp4_rht.argtypes = [P, i32, i64, i64, i64, i32, i32, u64, i32, P, P]
@@ -88,6 +94,22 @@ def nvfp4_amax(x, rows, cols, ld, layout, rht_group, seed, amax_out, stream) -> 
 def nvfp4_amax_dual(x, rows, cols, ld, rht_group_row, rht_group_col, seed, amax_row, amax_col, stream) -> int:
     return lib().nvfp4_amax_dual(x, rows, cols, ld, rht_group_row, rht_group_col, seed, amax_row, amax_col,
                                  stream)
+
+
+def nvfp4_amax_dual_group(n, x, rows, cols, ld, rht_group_row, rht_group_col, seed, amax_row, amax_col,
+                          stream) -> int:
+    """x, amax_row, amax_col: ctypes arrays of n pointers; rows, cols, ld: of n int64."""
+    return lib().nvfp4_amax_dual_group(n, x, rows, cols, ld, rht_group_row, rht_group_col, seed, amax_row,
+                                       amax_col, stream)
+
+
+def nvfp4_quantize_dual_group(n, x, rows, cols, ld, mode_row, rht_group_row, mode_col, rht_group_col, seed,
+                              amax_row, amax_col, codes_row, scales_row, gscale_row, codes_col, scales_col,
+                              gscale_col, stream) -> int:
+    """Pointer arguments: ctypes arrays of n pointers; rows, cols, ld: of n int64."""
+    return lib().nvfp4_quantize_dual_group(n, x, rows, cols, ld, mode_row, rht_group_row, mode_col, rht_group_col,
+                                           seed, amax_row, amax_col, codes_row, scales_row, gscale_row, codes_col,
+                                           scales_col, gscale_col, stream)
 
 
 def nvfp4_quantize(x, rows, cols, ld, layout, mode, rht_group, seed, amax_in, codes, scales,
@@ -234,6 +256,48 @@ def quantize_dual(x: torch.Tensor, mode_row: int, rht_group_row: int, mode_col: 
                                _p(amax_row), _p(amax_col), _p(r[0]), _p(r[1]), _p(r[2]), _p(c[0]), _p(c[1]),
                                _p(c[2]), _stream_handle(stream)), "nvfp4_quantize_dual")
     return r, c
+
+
+def _ptrs(ts):
+    return (ctypes.c_void_p * len(ts))(*[(t.data_ptr() if t is not None else None) for t in ts])
+
+
+def _i64s(vals):
+    return (ctypes.c_int64 * len(vals))(*vals)
+
+
+def amax_dual_group(xs, rht_group_row: int = 0, rht_group_col: int = 0, seed: int = 0, stream=None):
+    """amax_dual of every tensor of xs (nvfp4_amax_dual_group): a list of
+    (amax of the row-wise view, amax of the transposed view) pairs."""
+    shapes = [_matrix(x, torch.bfloat16) for x in xs]
+    outs = [torch.empty(2, dtype=torch.float32, device=x.device) for x in xs]
+    n = len(xs)
+    _check(nvfp4_amax_dual_group(n, _ptrs(xs), _i64s([s[0] for s in shapes]), _i64s([s[1] for s in shapes]),
+                                 _i64s([s[2] for s in shapes]), rht_group_row, rht_group_col, seed,
+                                 _ptrs([o[0:1] for o in outs]), _ptrs([o[1:2] for o in outs]),
+                                 _stream_handle(stream)), "nvfp4_amax_dual_group")
+    return [(o[0:1], o[1:2]) for o in outs]
+
+
+def quantize_dual_group(xs, mode_row: int, rht_group_row: int, mode_col: int, rht_group_col: int, seed: int = 0,
+                        amaxes=None, outs=None, stream=None):
+    """quantize_dual of every tensor of xs (nvfp4_quantize_dual_group);
+    amaxes: a list of (amax_row, amax_col) pairs (from amax_dual_group when
+    None); returns a list of (row-wise outputs, transposed outputs)."""
+    shapes = [_matrix(x, torch.bfloat16) for x in xs]
+    if amaxes is None:
+        amaxes = amax_dual_group(xs, rht_group_row, rht_group_col, seed, stream=stream)
+    if outs is None:
+        outs = [(alloc_outputs(r, c, ROWWISE, x.device), alloc_outputs(r, c, TRANSPOSED, x.device))
+                for x, (r, c, _) in zip(xs, shapes)]
+    n = len(xs)
+    _check(nvfp4_quantize_dual_group(
+        n, _ptrs(xs), _i64s([s[0] for s in shapes]), _i64s([s[1] for s in shapes]), _i64s([s[2] for s in shapes]),
+        mode_row, rht_group_row, mode_col, rht_group_col, seed, _ptrs([a[0] for a in amaxes]),
+        _ptrs([a[1] for a in amaxes]), _ptrs([o[0][0] for o in outs]), _ptrs([o[0][1] for o in outs]),
+        _ptrs([o[0][2] for o in outs]), _ptrs([o[1][0] for o in outs]), _ptrs([o[1][1] for o in outs]),
+        _ptrs([o[1][2] for o in outs]), _stream_handle(stream)), "nvfp4_quantize_dual_group")
+    return outs
 
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, gscale: torch.Tensor, mode: int = RTN,

@@ -62,25 +62,65 @@ int nvfp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int layout
 
 int nvfp4_amax_dual(const void* x, int64_t rows, int64_t cols, int64_t ld, int rht_group_row,
                     int rht_group_col, uint64_t seed, float* amax_row, float* amax_col, void* stream) {
-  int64_t vr, vc;
-  int st = check_tensor(x, rows, cols, ld, NVFP4_ROWWISE, rht_group_row, &vr, &vc);
-  if (st) return st;
-  if ((st = check_tensor(x, rows, cols, ld, NVFP4_TRANSPOSED, rht_group_col, &vr, &vc))) return st;
-  if (!amax_row || !amax_col) return NVFP4_ERR_INVALID_ARG;
-  if (!aligned(amax_row, 4) || !aligned(amax_col, 4)) return NVFP4_ERR_ALIGNMENT;
+  return nvfp4_amax_dual_group(1, &x, &rows, &cols, &ld, rht_group_row, rht_group_col, seed, &amax_row, &amax_col,
+                               stream);
+}
+
+int nvfp4_amax_dual_group(int n, const void* const* x, const int64_t* rows, const int64_t* cols, const int64_t* ld,
+                          int rht_group_row, int rht_group_col, uint64_t seed, float* const* amax_row,
+                          float* const* amax_col, void* stream) {
+  if (n < 1 || n > NVFP4_MAX_GROUP || !x || !rows || !cols || !ld || !amax_row || !amax_col)
+    return NVFP4_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    int64_t vr, vc;
+    int st = check_tensor(x[i], rows[i], cols[i], ld[i], NVFP4_ROWWISE, rht_group_row, &vr, &vc);
+    if (st) return st;
+    if ((st = check_tensor(x[i], rows[i], cols[i], ld[i], NVFP4_TRANSPOSED, rht_group_col, &vr, &vc))) return st;
+    if (!amax_row[i] || !amax_col[i]) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(amax_row[i], 4) || !aligned(amax_col[i], 4)) return NVFP4_ERR_ALIGNMENT;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = from_cuda(cudaMemsetAsync(amax_row, 0, sizeof(float), s)))) return st;
-  if ((st = from_cuda(cudaMemsetAsync(amax_col, 0, sizeof(float), s)))) return st;
-  if (rows > 0 && cols > 0 && nvfp4::dual_mma_path_applies(x, rows, cols, ld))
-    return from_cuda(nvfp4::launch_amax_dual_mma(x, rows, cols, ld, rht_group_row, rht_group_col, seed, amax_row,
-                                                 amax_col, s));
-  nvfp4::QuantArgs a{x, rows, cols, ld, NVFP4_ROWWISE, NVFP4_RTN, rht_group_row, seed, nullptr, amax_row,
-                     nullptr, nullptr, nullptr, s};
-  if ((st = from_cuda(nvfp4::launch_amax(a)))) return st;
-  a.layout = NVFP4_TRANSPOSED;
-  a.rht_group = rht_group_col;
-  a.amax_accum = amax_col;
-  return from_cuda(nvfp4::launch_amax(a));
+  int st;
+  for (int i = 0; i < n; ++i) {
+    if ((st = from_cuda(cudaMemsetAsync(amax_row[i], 0, sizeof(float), s)))) return st;
+    if ((st = from_cuda(cudaMemsetAsync(amax_col[i], 0, sizeof(float), s)))) return st;
+  }
+  // members with an unrotated row view go through the slot-ring kernel, up to
+  // kMaxDualMembers of them in one launch; the rest one by one
+  const void* gx[nvfp4::kMaxDualMembers];
+  int64_t gr[nvfp4::kMaxDualMembers], gc[nvfp4::kMaxDualMembers], gl[nvfp4::kMaxDualMembers];
+  float *ga[nvfp4::kMaxDualMembers], *gb[nvfp4::kMaxDualMembers];
+  int m = 0;
+  for (int i = 0; i < n; ++i) {
+    const bool empty = rows[i] == 0 || cols[i] == 0;
+    if (empty) continue;
+    if (nvfp4::dual_mma_path_applies(x[i], rows[i], cols[i], ld[i])) {
+      if (rht_group_row == 0) {
+        gx[m] = x[i], gr[m] = rows[i], gc[m] = cols[i], gl[m] = ld[i], ga[m] = amax_row[i], gb[m] = amax_col[i];
+        if (++m == nvfp4::kMaxDualMembers) {
+          if ((st = from_cuda(nvfp4::launch_amax_dual_ring(m, gx, gr, gc, gl, rht_group_row, rht_group_col, seed,
+                                                           ga, gb, s))))
+            return st;
+          m = 0;
+        }
+        continue;
+      }
+      if ((st = from_cuda(nvfp4::launch_amax_dual_mma(x[i], rows[i], cols[i], ld[i], rht_group_row, rht_group_col,
+                                                      seed, amax_row[i], amax_col[i], s))))
+        return st;
+      continue;
+    }
+    nvfp4::QuantArgs a{x[i], rows[i], cols[i], ld[i], NVFP4_ROWWISE, NVFP4_RTN, rht_group_row, seed, nullptr,
+                       amax_row[i], nullptr, nullptr, nullptr, s};
+    if ((st = from_cuda(nvfp4::launch_amax(a)))) return st;
+    a.layout = NVFP4_TRANSPOSED;
+    a.rht_group = rht_group_col;
+    a.amax_accum = amax_col[i];
+    if ((st = from_cuda(nvfp4::launch_amax(a)))) return st;
+  }
+  if (m > 0)
+    return from_cuda(nvfp4::launch_amax_dual_ring(m, gx, gr, gc, gl, rht_group_row, rht_group_col, seed, ga, gb, s));
+  return NVFP4_OK;
 }
 
 int nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int layout, int mode,
@@ -126,39 +166,73 @@ int nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int64_t ld, i
                         int mode_col, int rht_group_col, uint64_t seed, const float* amax_row, const float* amax_col,
                         uint8_t* codes_row, uint8_t* scales_row, float* gscale_row, uint8_t* codes_col,
                         uint8_t* scales_col, float* gscale_col, void* stream) {
-  int64_t vr, vc;
-  int st = check_tensor(x, rows, cols, ld, NVFP4_ROWWISE, rht_group_row, &vr, &vc);
-  if (st) return st;
-  if ((st = check_tensor(x, rows, cols, ld, NVFP4_TRANSPOSED, rht_group_col, &vr, &vc))) return st;
+  return nvfp4_quantize_dual_group(1, &x, &rows, &cols, &ld, mode_row, rht_group_row, mode_col, rht_group_col, seed,
+                                   &amax_row, &amax_col, &codes_row, &scales_row, &gscale_row, &codes_col,
+                                   &scales_col, &gscale_col, stream);
+}
+
+int nvfp4_quantize_dual_group(int n, const void* const* x, const int64_t* rows, const int64_t* cols,
+                              const int64_t* ld, int mode_row, int rht_group_row, int mode_col, int rht_group_col,
+                              uint64_t seed, const float* const* amax_row, const float* const* amax_col,
+                              uint8_t* const* codes_row, uint8_t* const* scales_row, float* const* gscale_row,
+                              uint8_t* const* codes_col, uint8_t* const* scales_col, float* const* gscale_col,
+                              void* stream) {
+  if (n < 1 || n > NVFP4_MAX_GROUP || !x || !rows || !cols || !ld || !amax_row || !amax_col || !codes_row ||
+      !scales_row || !gscale_row || !codes_col || !scales_col || !gscale_col)
+    return NVFP4_ERR_INVALID_ARG;
   for (int m : {mode_row, mode_col})
     if (m < NVFP4_RTN || m > NVFP4_MXFP3) return NVFP4_ERR_INVALID_ARG;
   if ((mode_row == NVFP4_MS_EDEN && rht_group_row == 0) || (mode_col == NVFP4_MS_EDEN && rht_group_col == 0))
     return NVFP4_ERR_UNSUPPORTED;
   const bool mx_r = mode_row == NVFP4_MXFP4 || mode_row == NVFP4_MXFP3;
   const bool mx_c = mode_col == NVFP4_MXFP4 || mode_col == NVFP4_MXFP3;
-  if ((mx_r && cols % 32) || (mx_c && rows % 32)) return NVFP4_ERR_SHAPE;
-  const bool empty = rows == 0 || cols == 0;
-  if (!gscale_row || !gscale_col) return NVFP4_ERR_INVALID_ARG;
-  if (!empty && (!codes_row || !scales_row || !codes_col || !scales_col)) return NVFP4_ERR_INVALID_ARG;
-  if ((!mx_r && !amax_row) || (!mx_c && !amax_col)) return NVFP4_ERR_INVALID_ARG;
-  if (!aligned(codes_row, 8) || !aligned(codes_col, 8) || !aligned(gscale_row, 4) || !aligned(gscale_col, 4))
-    return NVFP4_ERR_ALIGNMENT;
-  if ((amax_row && !aligned(amax_row, 4)) || (amax_col && !aligned(amax_col, 4))) return NVFP4_ERR_ALIGNMENT;
+  for (int i = 0; i < n; ++i) {
+    int64_t vr, vc;
+    int st = check_tensor(x[i], rows[i], cols[i], ld[i], NVFP4_ROWWISE, rht_group_row, &vr, &vc);
+    if (st) return st;
+    if ((st = check_tensor(x[i], rows[i], cols[i], ld[i], NVFP4_TRANSPOSED, rht_group_col, &vr, &vc))) return st;
+    if ((mx_r && cols[i] % 32) || (mx_c && rows[i] % 32)) return NVFP4_ERR_SHAPE;
+    const bool empty = rows[i] == 0 || cols[i] == 0;
+    if (!gscale_row[i] || !gscale_col[i]) return NVFP4_ERR_INVALID_ARG;
+    if (!empty && (!codes_row[i] || !scales_row[i] || !codes_col[i] || !scales_col[i])) return NVFP4_ERR_INVALID_ARG;
+    if ((!mx_r && !amax_row[i]) || (!mx_c && !amax_col[i])) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(codes_row[i], 8) || !aligned(codes_col[i], 8) || !aligned(gscale_row[i], 4) ||
+        !aligned(gscale_col[i], 4))
+      return NVFP4_ERR_ALIGNMENT;
+    if ((amax_row[i] && !aligned(amax_row[i], 4)) || (amax_col[i] && !aligned(amax_col[i], 4)))
+      return NVFP4_ERR_ALIGNMENT;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  nvfp4::DualQuantArgs d{x, rows, cols, ld, mode_row, rht_group_row, mode_col, rht_group_col, seed,
-                         amax_row, amax_col, codes_row, scales_row, gscale_row, codes_col, scales_col, gscale_col,
-                         1, s};
-  if (!empty && nvfp4::dual_quantize_fused(d)) return from_cuda(nvfp4::launch_quantize_dual_mma(d));
-  // any other pair: the two single-layout launches (MX modes read no amax:
-  // their kernels are given the output scalar, as nvfp4_quantize does)
-  nvfp4::QuantArgs a{x, rows, cols, ld, NVFP4_ROWWISE, mode_row, rht_group_row, seed,
-                     mx_r ? gscale_row : amax_row, nullptr, codes_row, scales_row, gscale_row, s};
-  if (!empty && mx_r && !nvfp4::mma_path_applies(a) && !nvfp4::tma_path_applies(a)) return NVFP4_ERR_UNSUPPORTED;
-  if ((st = from_cuda(nvfp4::launch_quantize(a)))) return st;
-  nvfp4::QuantArgs b{x, rows, cols, ld, NVFP4_TRANSPOSED, mode_col, rht_group_col, seed,
-                     mx_c ? gscale_col : amax_col, nullptr, codes_col, scales_col, gscale_col, s};
-  if (!empty && mx_c && !nvfp4::mma_path_applies(b) && !nvfp4::tma_path_applies(b)) return NVFP4_ERR_UNSUPPORTED;
-  return from_cuda(nvfp4::launch_quantize(b));
+  int st;
+  // members on the fused path: up to kMaxDualMembers of them in one launch
+  nvfp4::DualQuantArgs grp[nvfp4::kMaxDualMembers];
+  int m = 0;
+  for (int i = 0; i < n; ++i) {
+    const bool empty = rows[i] == 0 || cols[i] == 0;
+    nvfp4::DualQuantArgs d{x[i], rows[i], cols[i], ld[i], mode_row, rht_group_row, mode_col, rht_group_col, seed,
+                           amax_row[i], amax_col[i], codes_row[i], scales_row[i], gscale_row[i], codes_col[i],
+                           scales_col[i], gscale_col[i], 1, s};
+    if (!empty && nvfp4::dual_quantize_fused(d)) {
+      grp[m] = d;
+      if (++m == nvfp4::kMaxDualMembers) {
+        if ((st = from_cuda(nvfp4::launch_quantize_dual_group(grp, m)))) return st;
+        m = 0;
+      }
+      continue;
+    }
+    // any other pair: the two single-layout launches (MX modes read no amax:
+    // their kernels are given the output scalar, as nvfp4_quantize does)
+    nvfp4::QuantArgs a{x[i], rows[i], cols[i], ld[i], NVFP4_ROWWISE, mode_row, rht_group_row, seed,
+                       mx_r ? gscale_row[i] : amax_row[i], nullptr, codes_row[i], scales_row[i], gscale_row[i], s};
+    if (!empty && mx_r && !nvfp4::mma_path_applies(a) && !nvfp4::tma_path_applies(a)) return NVFP4_ERR_UNSUPPORTED;
+    if ((st = from_cuda(nvfp4::launch_quantize(a)))) return st;
+    nvfp4::QuantArgs b{x[i], rows[i], cols[i], ld[i], NVFP4_TRANSPOSED, mode_col, rht_group_col, seed,
+                       mx_c ? gscale_col[i] : amax_col[i], nullptr, codes_col[i], scales_col[i], gscale_col[i], s};
+    if (!empty && mx_c && !nvfp4::mma_path_applies(b) && !nvfp4::tma_path_applies(b)) return NVFP4_ERR_UNSUPPORTED;
+    if ((st = from_cuda(nvfp4::launch_quantize(b)))) return st;
+  }
+  if (m > 0) return from_cuda(nvfp4::launch_quantize_dual_group(grp, m));
+  return NVFP4_OK;
 }
 
 int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale,

@@ -68,7 +68,16 @@ cudaError_t launch_rotate_mma(const QuantArgs& a, float* zout);
 // rotation group g_r, transposed view with g_c (0 = no rotation).  amax_r and
 // amax_c are zeroed 32-bit accumulators.  Applies where the single-layout
 // tensor-core path does (both dimensions >= 128, 16-byte aligned rows).
+// Tensors one both-layout launch can take at once (a group: the same rotation
+// groups, modes and seed for every member).
+constexpr int kMaxDualMembers = 4;
+
 bool dual_mma_path_applies(const void* x, int64_t rows, int64_t cols, int64_t ld);
+// Both-layout pre-pass of n (1 .. kMaxDualMembers) non-empty tensors whose row
+// view is not rotated (g_r = 0), in one launch of the slot-ring kernel.
+cudaError_t launch_amax_dual_ring(int n, const void* const* x, const int64_t* rows, const int64_t* cols,
+                                  const int64_t* ld, int g_r, int g_c, uint64_t seed, float* const* amax_r,
+                                  float* const* amax_c, cudaStream_t stream);
 cudaError_t launch_amax_dual_mma(const void* x, int64_t rows, int64_t cols, int64_t ld, int g_r, int g_c,
                                  uint64_t seed, float* amax_r, float* amax_c, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantArgs& a);
@@ -97,6 +106,9 @@ struct DualQuantArgs {
 };
 bool dual_quantize_fused(const DualQuantArgs& a);
 cudaError_t launch_quantize_dual_mma(const DualQuantArgs& a);
+// One launch for a[0 .. n-1] (n <= kMaxDualMembers, each non-empty and fused,
+// all with a[0]'s modes, groups, seed, tile order and stream).
+cudaError_t launch_quantize_dual_group(const DualQuantArgs* a, int n);
 
 // D = gA gB A B^T from two quantizer outputs (gemm.cu); shapes checked by the
 // caller: m, n multiples of 128, k of 256, 16-byte aligned codes, scales, D rows.

@@ -25,6 +25,7 @@
 //              mbarriers.
 // Every wait is bounded (tma_pipeline.cuh); on a failed wait the CTA drains
 // what it issued, frees tensor memory and reports NaN in its scalar output.
+#include <cstring>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -463,7 +464,7 @@ struct DualShared {
   uint32_t issued_a;
   uint32_t issued_mma;
   int abort_flag;
-  unsigned int warp_max[2][kDualEpiWarps];
+  unsigned int warp_max[2][kMaxDualMembers][kDualEpiWarps];
 };
 
 __device__ __forceinline__ float rht_scale_of(int g) {
@@ -508,9 +509,50 @@ __device__ __forceinline__ void build_rotation_b(uint8_t* bmat, PhiloxKey key, u
 // chains, so a warp's reduction does not wait on its own previous result.
 __device__ __forceinline__ float absmax64(const float (&v)[64], float m) { return fmaxf(m, absmax_tree<64>(v)); }
 
+// A group of tensors measured or quantized by one launch: the same rotation
+// groups, modes and seed for every member; the members' tiles are numbered
+// one member after the other (member i owns tiles tile0 .. tile0 + its count
+// - 1), so one persistent grid walks them all and pays one ramp and one tail.
+struct DualMember {
+  int64_t rows, cols;   // the tensor (row view rows x cols, column view cols x rows)
+  int64_t tile0;        // its first tile in the group's numbering
+  uint32_t n_rt, n_ct;  // its grid of 128 x 128 tiles
+  const float* amax_r;  // quantize: the tensor amax of each view
+  const float* amax_c;
+  uint8_t* codes_r;
+  uint8_t* scales_r;
+  float* gscale_r;
+  uint8_t* codes_c;
+  uint8_t* scales_c;
+  float* gscale_c;
+  unsigned int* max_r;  // pre-pass: the amax of each view (binary32 patterns, atomicMax)
+  unsigned int* max_c;
+};
+struct DualGroup {
+  CUtensorMap map[kMaxDualMembers];
+  DualMember m[kMaxDualMembers];
+  int64_t n_tiles;      // all members' tiles
+  int n;                // members
+};
+
+// The member that owns tile t of the group (members without tiles own none).
+__device__ __forceinline__ int group_member(const DualGroup& g, int64_t t) {
+  int i = 0;
+#pragma unroll
+  for (int j = 1; j < kMaxDualMembers; ++j)
+    if (j < g.n && t >= g.m[j].tile0) i = j;
+  return i;
+}
+// Tile t of the group as (member, tile row, tile column) of the member.
+__device__ __forceinline__ int group_tile(const DualGroup& g, int64_t t, uint32_t band, uint32_t& rt, uint32_t& ct) {
+  const int i = group_member(g, t);
+  const TileGrid tg{g.m[i].n_rt, g.m[i].n_ct, band};
+  tg.coords(static_cast<uint32_t>(t - g.m[i].tile0), rt, ct);
+  return i;
+}
+
 __global__ void __launch_bounds__(kDualThreads, 1)
-dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed, int g_r,
-                 int g_c, unsigned int* __restrict__ amax_r, unsigned int* __restrict__ amax_c) {
+dual_amax_kernel(const __grid_constant__ DualGroup grp, uint64_t seed, int g_r, int g_c) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ __align__(8) DualShared sh;
   uint8_t* a_tiles = align_1024(dyn_smem);
@@ -519,9 +561,8 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
 
   const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
   const PhiloxKey key = philox_key(seed);
-  const TileGrid tg{static_cast<uint32_t>((rows + kTile - 1) / kTile), static_cast<uint32_t>((cols + kTile - 1) / kTile),
-                    static_cast<uint32_t>(NVFP4_MMA_BAND_ROWS)};
-  const int64_t n_tiles = static_cast<int64_t>(tg.n_rt) * tg.n_ct;
+  const uint32_t band = static_cast<uint32_t>(NVFP4_MMA_BAND_ROWS);
+  const int64_t n_tiles = grp.n_tiles;
   const int64_t step = gridDim.x;
   // this CTA's tiles: blockIdx.x, blockIdx.x + step, ...
   const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - blockIdx.x + step - 1) / step : 0;
@@ -566,7 +607,7 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
   if (warp == kDualProducerWarp) {
     if (lane == 0) {
       grid_dependency_wait();
-      prefetch_tensormap(&tmap);
+      for (int i = 0; i < grp.n; ++i) prefetch_tensormap(&grp.map[i]);
       for (int64_t k = 0; k < my_tiles; ++k) {
         const int s = static_cast<int>(k % kDualStages);
         const uint32_t u = static_cast<uint32_t>(k / kDualStages);
@@ -576,12 +617,12 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
         }
         if (*reinterpret_cast<volatile int*>(&sh.abort_flag)) break;
         uint32_t rt, ct;
-        tg.coords(static_cast<uint32_t>(blockIdx.x + k * step), rt, ct);
+        const int mi = group_tile(grp, blockIdx.x + k * step, band, rt, ct);
         const int32_t x = static_cast<int32_t>(ct * kTile), y = static_cast<int32_t>(rt * kTile);
         mbar_arrive_expect_tx(&sh.full[s], kTileBytes);
         uint8_t* dst = a_tiles + s * kTileBytes;
-        tma_load_2d(dst, &tmap, x, y, &sh.full[s]);
-        tma_load_2d(dst + kBoxBytes, &tmap, x + 64, y, &sh.full[s]);
+        tma_load_2d(dst, &grp.map[mi], x, y, &sh.full[s]);
+        tma_load_2d(dst + kBoxBytes, &grp.map[mi], x + 64, y, &sh.full[s]);
         sh.issued_a = (sh.issued_a & ~(0x101u << s)) | (1u << s) | ((u & 1u) << (8 + s));
       }
     }
@@ -636,12 +677,16 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
     // epilogue: slot `slot`, lane quarter q
     const uint32_t q = warp & 3u, slot = warp >> 2;
     grid_dependency_wait();
-    float m_r = 0.0f, m_c = 0.0f;  // max |acc| (unscaled) of the row and column views; max |x| from smem
+    // per member: max |acc| (unscaled) of the row and column views; max |x| from smem
+    float m_r[kMaxDualMembers], m_c[kMaxDualMembers];
+#pragma unroll
+    for (int i = 0; i < kMaxDualMembers; ++i) m_r[i] = m_c[i] = 0.0f;
     const int64_t n_acc = my_tiles * views;
     const uint32_t part = q * 32u + lane;
     for (int64_t j = slot; j < n_acc; j += kDualSlots) {
       const int64_t k = j / views;
       const int v = static_cast<int>(j % views);
+      const int mi = group_member(grp, blockIdx.x + k * step);
       if (row_from_smem) {
         // max|x| of the staged tile for the row view: 128 threads, 256 bytes
         // each (the order of the swizzled bytes does not matter to a
@@ -659,7 +704,10 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
           bmax = __vmaxu2(bmax, __vmaxu2(__vmaxu2(w4.x & 0x7FFF7FFFu, w4.y & 0x7FFF7FFFu),
                                          __vmaxu2(w4.z & 0x7FFF7FFFu, w4.w & 0x7FFF7FFFu)));
         }
-        m_r = fmaxf(m_r, __uint_as_float(max(bmax & 0xFFFFu, bmax >> 16) << 16));
+        const float mx = __uint_as_float(max(bmax & 0xFFFFu, bmax >> 16) << 16);
+#pragma unroll
+        for (int i = 0; i < kMaxDualMembers; ++i)
+          if (i == mi) m_r[i] = fmaxf(m_r[i], mx);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.sfree[s]);
       }
@@ -683,14 +731,22 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
         if (lane == 0) mbar_arrive(&sh.tfree[slot]);
         m = absmax64(v1, m);
       }
-      if (v == 0 && views == 2) m_r = fmaxf(m_r, m);
-      else m_c = fmaxf(m_c, m);
+      const bool row = v == 0 && views == 2;
+#pragma unroll
+      for (int i = 0; i < kMaxDualMembers; ++i)
+        if (i == mi) {
+          if (row) m_r[i] = fmaxf(m_r[i], m);
+          else m_c[i] = fmaxf(m_c[i], m);
+        }
     }
-    const unsigned int br = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m_r));
-    const unsigned int bc = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m_c));
-    if (lane == 0) {
-      sh.warp_max[0][warp] = br;
-      sh.warp_max[1][warp] = bc;
+#pragma unroll
+    for (int i = 0; i < kMaxDualMembers; ++i) {
+      const unsigned int br = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m_r[i]));
+      const unsigned int bc = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m_c[i]));
+      if (lane == 0) {
+        sh.warp_max[0][i][warp] = br;
+        sh.warp_max[1][i][warp] = bc;
+      }
     }
   }
 
@@ -704,20 +760,22 @@ dual_amax_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t
       for (int a = 0; a < kDualSlots; ++a)
         if ((sh.issued_mma >> a) & 1u) mbar_wait(&sh.tfull[a], (sh.issued_mma >> (8 + a)) & 1u);
   }
-  if (tid == 0) {
+  if (tid < static_cast<uint32_t>(grp.n)) {
+    // thread i finishes member i
+    const int i = static_cast<int>(tid);
     unsigned int mr = 0, mc = 0;
 #pragma unroll
     for (int w = 0; w < kDualEpiWarps; ++w) {
-      mr = max(mr, sh.warp_max[0][w]);
-      mc = max(mc, sh.warp_max[1][w]);
+      mr = max(mr, sh.warp_max[0][i][w]);
+      mc = max(mc, sh.warp_max[1][i][w]);
     }
     // one rounding of the largest magnitude by the rotation constant (the
     // row view read from shared memory is x itself)
     const float cr = row_from_smem ? 1.0f : rht_scale_of(g_r), cc = rht_scale_of(g_c);
     const unsigned int sr = __float_as_uint(__fmul_rn(__uint_as_float(mr), cr));
     const unsigned int sc = __float_as_uint(__fmul_rn(__uint_as_float(mc), cc));
-    atomicMax(amax_r, failed ? 0x7FC00000u : sr);
-    atomicMax(amax_c, failed ? 0x7FC00000u : sc);
+    atomicMax(grp.m[i].max_r, failed ? 0x7FC00000u : sr);
+    atomicMax(grp.m[i].max_c, failed ? 0x7FC00000u : sc);
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -1023,8 +1081,11 @@ struct DualQuantShared {
   uint32_t issued_a;
   uint32_t issued_mma;
   int abort_flag;
-  float4 scale_tbl[2][128];   // the launch's block-scale constants per E4M3 code, row and column view
+  float4 scale_tbl[kMaxDualMembers][2][128];  // block-scale constants per E4M3 code: member, view
+  ScaleCtx sc[kMaxDualMembers][2];             // each member's scale constants: row and column view
 };
+// 227 KB of shared memory per CTA on sm_100
+static_assert(kDualDynSmem + sizeof(DualQuantShared) <= 227u * 1024u, "both-layout quantize shared memory");
 
 #ifndef NVFP4_DUALQ_BAND_ROWS
 #define NVFP4_DUALQ_BAND_ROWS 1
@@ -1032,11 +1093,7 @@ struct DualQuantShared {
 
 template <int MODE_R, int G_R, int MODE_C, int G_C>
 __global__ void __launch_bounds__(kDualThreads, 1)
-dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed,
-                     const float* __restrict__ amax_r, const float* __restrict__ amax_c,
-                     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ scales_r, float* __restrict__ gscale_r,
-                     uint8_t* __restrict__ codes_c, uint8_t* __restrict__ scales_c, float* __restrict__ gscale_c,
-                     int reverse) {
+dual_quantize_kernel(const __grid_constant__ DualGroup grp, uint64_t seed, int reverse) {
   static_assert(G_C > 0, "the column view is rotated on the tensor cores");
   constexpr int kViews = G_R != 0 ? 2 : 1;
   constexpr bool kRowFromSmem = G_R == 0;
@@ -1048,9 +1105,8 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
 
   const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
   const PhiloxKey key = philox_key(seed);
-  const TileGrid tg{static_cast<uint32_t>((rows + kTile - 1) / kTile), static_cast<uint32_t>((cols + kTile - 1) / kTile),
-                    static_cast<uint32_t>(NVFP4_DUALQ_BAND_ROWS)};
-  const int64_t n_tiles = static_cast<int64_t>(tg.n_rt) * tg.n_ct;
+  const uint32_t band = static_cast<uint32_t>(NVFP4_DUALQ_BAND_ROWS);
+  const int64_t n_tiles = grp.n_tiles;
   const int64_t step = gridDim.x;
   const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - blockIdx.x + step - 1) / step : 0;
 
@@ -1088,7 +1144,7 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
   if (warp == kDualProducerWarp) {
     if (lane == 0) {
       grid_dependency_wait();
-      prefetch_tensormap(&tmap);
+      for (int i = 0; i < grp.n; ++i) prefetch_tensormap(&grp.map[i]);
       for (int64_t k = 0; k < my_tiles; ++k) {
         const int s = static_cast<int>(k % kDualStages);
         const uint32_t u = static_cast<uint32_t>(k / kDualStages);
@@ -1098,12 +1154,12 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
         }
         if (*reinterpret_cast<volatile int*>(&sh.abort_flag)) break;
         uint32_t rt, ct;
-        tg.coords(dual_tile_index(k, n_tiles, reverse), rt, ct);
+        const int mi = group_tile(grp, dual_tile_index(k, n_tiles, reverse), band, rt, ct);
         const int32_t x = static_cast<int32_t>(ct * kTile), y = static_cast<int32_t>(rt * kTile);
         mbar_arrive_expect_tx(&sh.full[s], kTileBytes);
         uint8_t* dst = a_tiles + s * kTileBytes;
-        tma_load_2d(dst, &tmap, x, y, &sh.full[s]);
-        tma_load_2d(dst + kBoxBytes, &tmap, x + 64, y, &sh.full[s]);
+        tma_load_2d(dst, &grp.map[mi], x, y, &sh.full[s]);
+        tma_load_2d(dst + kBoxBytes, &grp.map[mi], x + 64, y, &sh.full[s]);
         sh.issued_a = (sh.issued_a & ~(0x101u << s)) | (1u << s) | ((u & 1u) << (8 + s));
       }
     }
@@ -1160,30 +1216,43 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
     // ------------------------------------------------------------ epilogue
     const uint32_t q = warp & 3u, slot = warp >> 2;
     grid_dependency_wait();
-    ScaleCtx sc_r = make_scale_ctx<MODE_R>(*amax_r);
-    ScaleCtx sc_c = make_scale_ctx<MODE_C>(*amax_c);
-    build_scale_table(sh.scale_tbl[0], sc_r.s_g, tid, kDualEpiWarps * 32);
-    build_scale_table(sh.scale_tbl[1], sc_c.s_g, tid, kDualEpiWarps * 32);
-    asm volatile("bar.sync 1, %0;" ::"r"(kDualEpiWarps * 32) : "memory");
-    sc_r.tbl = sh.scale_tbl[0];
-    sc_c.tbl = sh.scale_tbl[1];
-    if (blockIdx.x == 0 && tid == 0) {
-      *gscale_r = sc_r.s_g;
-      *gscale_c = sc_c.s_g;
+    // every member's scale constants and tables, once per CTA
+    for (int i = 0; i < grp.n; ++i) {
+      const float s_r = global_scale_of<MODE_R>(*grp.m[i].amax_r), s_c = global_scale_of<MODE_C>(*grp.m[i].amax_c);
+      build_scale_table(sh.scale_tbl[i][0], s_r, tid, kDualEpiWarps * 32);
+      build_scale_table(sh.scale_tbl[i][1], s_c, tid, kDualEpiWarps * 32);
+      if (tid == 0) {
+        sh.sc[i][0] = make_scale_ctx<MODE_R>(*grp.m[i].amax_r);
+        sh.sc[i][1] = make_scale_ctx<MODE_C>(*grp.m[i].amax_c);
+        sh.sc[i][0].tbl = sh.scale_tbl[i][0];
+        sh.sc[i][1].tbl = sh.scale_tbl[i][1];
+        if (blockIdx.x == 0) {
+          *grp.m[i].gscale_r = sh.sc[i][0].s_g;
+          *grp.m[i].gscale_c = sh.sc[i][1].s_g;
+        }
+      }
     }
-    // row view: rows x cols; column view: cols x rows
-    const bool r_codes16 = ((cols / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes_r) % 16) == 0;
-    const bool r_scales4 = ((cols / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales_r) % 4) == 0;
-    const bool c_codes16 = ((rows / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes_c) % 16) == 0;
-    const bool c_scales4 = ((rows / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales_c) % 4) == 0;
-    const bool r_blocks8 = ((cols / 16) % 8) == 0, c_blocks8 = ((rows / 16) % 8) == 0;
+    asm volatile("bar.sync 1, %0;" ::"r"(kDualEpiWarps * 32) : "memory");
     const int64_t n_acc = my_tiles * kViews;
     const uint32_t r_in_tile = 32u * q + lane;
     for (int64_t j = slot; j < n_acc; j += kDualSlots) {
       const int64_t k = j / kViews;
       const int v = static_cast<int>(j % kViews);
       uint32_t rt, ct;
-      tg.coords(dual_tile_index(k, n_tiles, reverse), rt, ct);
+      const int mi = group_tile(grp, dual_tile_index(k, n_tiles, reverse), band, rt, ct);
+      const DualMember& mb = grp.m[mi];
+      const int64_t rows = mb.rows, cols = mb.cols;
+      const ScaleCtx sc_r = sh.sc[mi][0], sc_c = sh.sc[mi][1];
+      uint8_t* const codes_r = mb.codes_r;
+      uint8_t* const scales_r = mb.scales_r;
+      uint8_t* const codes_c = mb.codes_c;
+      uint8_t* const scales_c = mb.scales_c;
+      // row view: rows x cols; column view: cols x rows
+      const bool r_codes16 = ((cols / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes_r) % 16) == 0;
+      const bool r_scales4 = ((cols / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales_r) % 4) == 0;
+      const bool c_codes16 = ((rows / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes_c) % 16) == 0;
+      const bool c_scales4 = ((rows / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales_c) % 4) == 0;
+      const bool r_blocks8 = ((cols / 16) % 8) == 0, c_blocks8 = ((rows / 16) % 8) == 0;
       if constexpr (kRowFromSmem) {
         const int s = static_cast<int>(k % kDualStages);
         if (!mbar_wait(&sh.full[s], static_cast<uint32_t>(k / kDualStages) & 1u)) {
@@ -1234,9 +1303,9 @@ dual_quantize_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int
     if (tid == kDualMmaWarp * 32)
       for (int a = 0; a < kDualSlots; ++a)
         if ((sh.issued_mma >> a) & 1u) mbar_wait(&sh.tfull[a], (sh.issued_mma >> (8 + a)) & 1u);
-    if (tid == 0) {
-      *gscale_r = __uint_as_float(0x7FC00000u);
-      *gscale_c = __uint_as_float(0x7FC00000u);
+    if (tid < static_cast<uint32_t>(grp.n)) {
+      *grp.m[tid].gscale_r = __uint_as_float(0x7FC00000u);
+      *grp.m[tid].gscale_c = __uint_as_float(0x7FC00000u);
     }
   }
   tc_fence_before_sync();
@@ -1348,48 +1417,109 @@ bool dual_mma_path_applies(const void* x, int64_t rows, int64_t cols, int64_t ld
   return mma_path_applies(a);
 }
 
+namespace {
+
+// A group's kernel parameter from up to kMaxDualMembers non-empty tensors;
+// false if a tensor map cannot be encoded.
+bool make_group(DualGroup& g, int n, const void* const* x, const int64_t* rows, const int64_t* cols,
+                const int64_t* ld) {
+  std::memset(&g, 0, sizeof(g));
+  g.n = n;
+  int64_t t0 = 0;
+  for (int i = 0; i < n; ++i) {
+    if (!make_map(&g.map[i], x[i], rows[i], cols[i], ld[i])) return false;
+    DualMember& m = g.m[i];
+    m.rows = rows[i];
+    m.cols = cols[i];
+    m.tile0 = t0;
+    m.n_rt = static_cast<uint32_t>((rows[i] + kTile - 1) / kTile);
+    m.n_ct = static_cast<uint32_t>((cols[i] + kTile - 1) / kTile);
+    t0 += static_cast<int64_t>(m.n_rt) * m.n_ct;
+  }
+  g.n_tiles = t0;
+  return true;
+}
+
+}  // namespace
+
+cudaError_t launch_amax_dual_ring(int n, const void* const* x, const int64_t* rows, const int64_t* cols,
+                                  const int64_t* ld, int g_r, int g_c, uint64_t seed, float* const* amax_r,
+                                  float* const* amax_c, cudaStream_t stream) {
+  if (n < 1 || n > kMaxDualMembers) return cudaErrorInvalidValue;
+  DualGroup g;
+  if (!make_group(g, n, x, rows, cols, ld)) return cudaErrorInvalidValue;
+  for (int i = 0; i < n; ++i) {
+    g.m[i].max_r = reinterpret_cast<unsigned int*>(amax_r[i]);
+    g.m[i].max_c = reinterpret_cast<unsigned int*>(amax_c[i]);
+  }
+  LaunchGeom geom;
+  cudaError_t e = launch_geometry(dual_amax_kernel, kDualThreads, kDualDynSmem, 1, &geom);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = g.n_tiles < int64_t(geom.sms) ? g.n_tiles : int64_t(geom.sms);
+  if (grid == 0) return cudaSuccess;
+  return launch_overlapped(dual_amax_kernel, static_cast<unsigned>(grid), kDualThreads, kDualDynSmem, stream, g, seed,
+                           g_r, g_c);
+}
+
 cudaError_t launch_amax_dual_mma(const void* x, int64_t rows, int64_t cols, int64_t ld, int g_r, int g_c,
                                  uint64_t seed, float* amax_r, float* amax_c, cudaStream_t stream) {
+  // the row view straight from the tile: the slot ring, a group of one
+  if (g_r == 0) return launch_amax_dual_ring(1, &x, &rows, &cols, &ld, g_r, g_c, seed, &amax_r, &amax_c, stream);
+  // both views rotated: the group kernel
   CUtensorMap map;
   if (!make_map(&map, x, rows, cols, ld)) return cudaErrorInvalidValue;
-  // both views rotated: the group kernel; the row view straight from the tile: the slot ring
-  const bool groups = g_r != 0;
-  auto kernel = groups ? dual_amax_group_kernel : dual_amax_kernel;
-  const int threads = groups ? kGrpThreads : kDualThreads;
-  const size_t smem = groups ? kGrpDynSmem : kDualDynSmem;
   LaunchGeom geom;
-  cudaError_t e = launch_geometry(kernel, threads, smem, 1, &geom);
+  cudaError_t e = launch_geometry(dual_amax_group_kernel, kGrpThreads, kGrpDynSmem, 1, &geom);
   if (e != cudaSuccess) return e;
-  const int sms = geom.sms;
   const int64_t n_tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
-  const int64_t grid = n_tiles < int64_t(sms) ? n_tiles : int64_t(sms);
+  const int64_t grid = n_tiles < int64_t(geom.sms) ? n_tiles : int64_t(geom.sms);
   if (grid == 0) return cudaSuccess;
-  return launch_overlapped(kernel, static_cast<unsigned>(grid), threads, smem, stream, map, rows, cols, seed, g_r, g_c,
-                           reinterpret_cast<unsigned int*>(amax_r), reinterpret_cast<unsigned int*>(amax_c));
+  return launch_overlapped(dual_amax_group_kernel, static_cast<unsigned>(grid), kGrpThreads, kGrpDynSmem, stream, map,
+                           rows, cols, seed, g_r, g_c, reinterpret_cast<unsigned int*>(amax_r),
+                           reinterpret_cast<unsigned int*>(amax_c));
 }
 
 namespace {
 
+// One launch for members a[0 .. n-1] (the same modes, groups, seed, stream
+// and tile order; each fused).
 template <int MODE_R, int G_R, int MODE_C, int G_C>
-cudaError_t launch_dual_quantize_t(const DualQuantArgs& a) {
-  CUtensorMap map;
-  if (!make_map(&map, a.x, a.rows, a.cols, a.ld)) return cudaErrorInvalidValue;
+cudaError_t launch_dual_quantize_t(const DualQuantArgs* a, int n) {
+  const void* x[kMaxDualMembers];
+  int64_t rows[kMaxDualMembers], cols[kMaxDualMembers], ld[kMaxDualMembers];
+  for (int i = 0; i < n; ++i) {
+    x[i] = a[i].x;
+    rows[i] = a[i].rows;
+    cols[i] = a[i].cols;
+    ld[i] = a[i].ld;
+  }
+  DualGroup g;
+  if (!make_group(g, n, x, rows, cols, ld)) return cudaErrorInvalidValue;
+  for (int i = 0; i < n; ++i) {
+    DualMember& m = g.m[i];
+    m.amax_r = a[i].amax_row;
+    m.amax_c = a[i].amax_col;
+    m.codes_r = a[i].codes_row;
+    m.scales_r = a[i].scales_row;
+    m.gscale_r = a[i].gscale_row;
+    m.codes_c = a[i].codes_col;
+    m.scales_c = a[i].scales_col;
+    m.gscale_c = a[i].gscale_col;
+  }
   auto kernel = dual_quantize_kernel<MODE_R, G_R, MODE_C, G_C>;
   LaunchGeom geom;
   cudaError_t e = launch_geometry(kernel, kDualThreads, kDualDynSmem, 1, &geom);
   if (e != cudaSuccess) return e;
-  const int64_t n_tiles = ((a.rows + kTile - 1) / kTile) * ((a.cols + kTile - 1) / kTile);
-  const int64_t grid = n_tiles < int64_t(geom.sms) ? n_tiles : int64_t(geom.sms);
+  const int64_t grid = g.n_tiles < int64_t(geom.sms) ? g.n_tiles : int64_t(geom.sms);
   if (grid == 0) return cudaSuccess;
-  return launch_overlapped(kernel, static_cast<unsigned>(grid), kDualThreads, kDualDynSmem, a.stream, map, a.rows,
-                           a.cols, a.seed, a.amax_row, a.amax_col, a.codes_row, a.scales_row, a.gscale_row,
-                           a.codes_col, a.scales_col, a.gscale_col, a.reverse);
+  return launch_overlapped(kernel, static_cast<unsigned>(grid), kDualThreads, kDualDynSmem, a[0].stream, g, a[0].seed,
+                           a[0].reverse);
 }
 
 template <int G>
-cudaError_t dispatch_dual_quantize(const DualQuantArgs& a) {
-  if (a.mode_row == kRTN && a.rht_group_row == 0) return launch_dual_quantize_t<kRTN, 0, kMSEDEN, G>(a);
-  return launch_dual_quantize_t<kMSEDEN, G, kMSEDEN, G>(a);
+cudaError_t dispatch_dual_quantize(const DualQuantArgs* a, int n) {
+  if (a[0].mode_row == kRTN && a[0].rht_group_row == 0) return launch_dual_quantize_t<kRTN, 0, kMSEDEN, G>(a, n);
+  return launch_dual_quantize_t<kMSEDEN, G, kMSEDEN, G>(a, n);
 }
 
 }  // namespace
@@ -1402,14 +1532,17 @@ bool dual_quantize_fused(const DualQuantArgs& a) {
   return a.mode_row == kMSEDEN && a.rht_group_row == g;
 }
 
-cudaError_t launch_quantize_dual_mma(const DualQuantArgs& a) {
-  switch (a.rht_group_col) {
-    case 16: return dispatch_dual_quantize<16>(a);
-    case 32: return dispatch_dual_quantize<32>(a);
-    case 64: return dispatch_dual_quantize<64>(a);
-    case 128: return dispatch_dual_quantize<128>(a);
+cudaError_t launch_quantize_dual_group(const DualQuantArgs* a, int n) {
+  if (n < 1 || n > kMaxDualMembers) return cudaErrorInvalidValue;
+  switch (a[0].rht_group_col) {
+    case 16: return dispatch_dual_quantize<16>(a, n);
+    case 32: return dispatch_dual_quantize<32>(a, n);
+    case 64: return dispatch_dual_quantize<64>(a, n);
+    case 128: return dispatch_dual_quantize<128>(a, n);
     default: return cudaErrorInvalidValue;
   }
 }
+
+cudaError_t launch_quantize_dual_mma(const DualQuantArgs& a) { return launch_quantize_dual_group(&a, 1); }
 
 }  // namespace nvfp4

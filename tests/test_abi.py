@@ -34,7 +34,8 @@ def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ["nvfp4_quantize", "nvfp4_dequantize", "nvfp4_rht", "nvfp4_amax", "nvfp4_workspace_bytes",
               "nvfp4_status_string", "nvfp4_encode_e2m1", "nvfp4_encode_e4m3", "nvfp4_quantize_noalloc",
-              "nvfp4_amax_dual", "nvfp4_gemm", "nvfp4_quantize_dual", "nvfp4_pack3", "nvfp4_unpack3"]:
+              "nvfp4_amax_dual", "nvfp4_gemm", "nvfp4_quantize_dual", "nvfp4_pack3", "nvfp4_unpack3",
+              "nvfp4_amax_dual_group", "nvfp4_quantize_dual_group"]:
         assert n in names
 
 
@@ -131,6 +132,46 @@ def test_quantize_dual_rejects(N):
     assert qd(N, outs=(FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE)) == ALIGN
     assert qd(N, x=FAKE + 8) == ALIGN
     assert qd(N, ar=FAKE + 2) == ALIGN
+
+
+def _group_args(n, shapes, amax=True):
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    ptrs = lambda vals: (P * n)(*vals)  # noqa: E731
+    return dict(x=ptrs([FAKE + 0x10000 * i for i in range(n)]), rows=(I64 * n)(*[s[0] for s in shapes]),
+                cols=(I64 * n)(*[s[1] for s in shapes]), ld=(I64 * n)(*[s[1] for s in shapes]),
+                a=ptrs([FAKE + 0x100 * i if amax else None for i in range(n)]),
+                o=[ptrs([FAKE + 0x1000 * (j + 1) + 0x40 * i for i in range(n)]) for j in range(6)])
+
+
+def test_group_calls_reject(N):
+    """The group calls check every member as the single calls do, before any
+    launch: a bad second member fails the whole call."""
+    good = (256, 256)
+    g = _group_args(2, [good, good])
+    ag = lambda n, g, gr=0, gc=128: N.nvfp4_amax_dual_group(n, g["x"], g["rows"], g["cols"], g["ld"], gr, gc, 0,  # noqa: E731
+                                                            g["a"], g["a"], None)
+    assert ag(0, g) == INVALID                      # no members
+    assert ag(65, g) == INVALID                     # more than NVFP4_MAX_GROUP
+    assert N.nvfp4_amax_dual_group(2, None, g["rows"], g["cols"], g["ld"], 0, 128, 0, g["a"], g["a"], None) == INVALID
+    assert ag(2, g, gc=48) == INVALID               # rotation group
+    bad = _group_args(2, [good, (256, 40)])         # second member: cols not a multiple of 16
+    assert ag(2, bad) == SHAPE
+    noamax = _group_args(2, [good, good], amax=False)
+    assert ag(2, noamax) == INVALID                 # outputs required
+
+    def qg(n, g, mr=0, gr=0, mc=2, gc=128):
+        o = g["o"]
+        return N.nvfp4_quantize_dual_group(n, g["x"], g["rows"], g["cols"], g["ld"], mr, gr, mc, gc, 0, g["a"],
+                                           g["a"], o[0], o[1], o[2], o[3], o[4], o[5], None)
+    assert qg(0, g) == INVALID
+    assert qg(65, g) == INVALID
+    assert qg(2, g, mr=12) == INVALID               # mode
+    assert qg(2, g, mr=2, gr=0) == UNSUPPORTED      # MS-EDEN needs the rotation
+    assert qg(2, bad) == SHAPE
+    assert qg(2, noamax) == INVALID                 # the row view's amax is required (not an MX mode)
+    mis = _group_args(2, [good, good])
+    mis["o"][0] = (ctypes.c_void_p * 2)(FAKE, FAKE + 4)  # second member's codes not 8-byte aligned
+    assert qg(2, mis) == ALIGN
 
 
 def test_pack3_rejects(N):

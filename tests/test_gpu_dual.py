@@ -98,3 +98,66 @@ def test_dual_empty():
     torch.cuda.synchronize()
     assert row[0].numel() == 0 and col[0].numel() == 0
     assert float(row[2].item()) == 1.0 and float(col[2].item()) == 1.0
+
+
+# ---------------------------------------------------------------- groups
+def _f32bits(t):
+    return t.detach().cpu().numpy().astype(np.float32).view(np.uint32)
+
+
+def _members(shapes, seed, pad=0):
+    g = torch.Generator().manual_seed(seed)
+    return [to_device((torch.randn(r, c, generator=g) * (0.1 + i)).to(torch.bfloat16), pad if i % 2 else 0)
+            for i, (r, c) in enumerate(shapes)]
+
+
+# Members of different shapes (ragged tiles, a padded row pitch, one too small
+# for the fused kernel, one empty), more of them than one launch takes.
+GROUP_SHAPES = [(384, 256), (256, 640), (400, 272), (64, 96), (0, 128), (512, 384)]
+
+
+@pytest.mark.parametrize("g_r,g_c", [(0, 128), (0, 16), (128, 128)])
+def test_amax_dual_group_equals_single_calls(g_r, g_c):
+    shapes = [(r, c) for r, c in GROUP_SHAPES if (r % g_c == 0 or r == 0) and (g_r == 0 or c % g_r == 0)]
+    xs = _members(shapes, 11, pad=8)
+    got = N.amax_dual_group(xs, g_r, g_c, seed=5)
+    for x, (ar, ac) in zip(xs, got):
+        wr, wc = N.amax_dual(x, g_r, g_c, seed=5)
+        torch.cuda.synchronize()
+        what = f"shape={tuple(x.shape)} groups=({g_r},{g_c})"
+        assert np.array_equal(_f32bits(ar), _f32bits(wr)), what + " row view"
+        assert np.array_equal(_f32bits(ac), _f32bits(wc)), what + " column view"
+
+
+@pytest.mark.parametrize("mode_r,g_r,mode_c,g_c", [(W.RTN, 0, W.MS_EDEN, 128), (W.MS_EDEN, 128, W.MS_EDEN, 128),
+                                                   (W.RTN, 0, W.MS_EDEN, 16), (W.SR, 0, W.IF4, 0)])
+def test_quantize_dual_group_equals_single_calls(mode_r, g_r, mode_c, g_c):
+    gc = g_c if g_c else 16
+    shapes = [(r, c) for r, c in GROUP_SHAPES if (r % gc == 0 or r == 0) and (g_r == 0 or c % g_r == 0)]
+    xs = _members(shapes, 12, pad=8)
+    amaxes = N.amax_dual_group(xs, g_r, g_c, seed=6)
+    outs = N.quantize_dual_group(xs, mode_r, g_r, mode_c, g_c, seed=6, amaxes=amaxes)
+    for x, (ar, ac), (row, col) in zip(xs, amaxes, outs):
+        wrow, wcol = N.quantize_dual(x, mode_r, g_r, mode_c, g_c, seed=6, amax_row=ar, amax_col=ac)
+        torch.cuda.synchronize()
+        what = f"shape={tuple(x.shape)} row=({mode_r},{g_r}) col=({mode_c},{g_c})"
+        assert_same(_host(row), _host(wrow), what + " row-wise")
+        assert_same(_host(col), _host(wcol), what + " transposed")
+
+
+def test_group_of_the_mlp_forward_operands():
+    """X and W of the MLP up-projection workload in one group: the step's
+    forward pair, at full size."""
+    wl = W.mlp_up()
+    t = wl.tensors(torch.device("cuda"))
+    xs = [t["x"], t["w"]]
+    amaxes = N.amax_dual_group(xs, 0, 128, wl.seed)
+    outs = N.quantize_dual_group(xs, W.RTN, 0, W.MS_EDEN, 128, wl.seed, amaxes=amaxes)
+    for x, (ar, ac), (row, col) in zip(xs, amaxes, outs):
+        wr, wc = N.amax_dual(x, 0, 128, wl.seed)
+        wrow, wcol = N.quantize_dual(x, W.RTN, 0, W.MS_EDEN, 128, wl.seed, amax_row=wr, amax_col=wc)
+        torch.cuda.synchronize()
+        assert np.array_equal(_f32bits(ar), _f32bits(wr)) and np.array_equal(_f32bits(ac), _f32bits(wc))
+        for got, want in ((row, wrow), (col, wcol)):
+            assert torch.equal(got[0], want[0]) and torch.equal(got[1], want[1])
+            assert np.array_equal(_f32bits(got[2]), _f32bits(want[2]))
