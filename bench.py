@@ -59,6 +59,8 @@ NCU_TRAFFIC = {
         472454400 + 224126976,
     ("65a6a919a9ff92ea", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
         472376576 + 223989760,
+    ("e67268332ab8fc9f", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
+        472720896 + 224553728,
 }
 
 

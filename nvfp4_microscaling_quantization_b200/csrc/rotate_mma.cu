@@ -1091,7 +1091,7 @@ static_assert(kDualDynSmem + sizeof(DualQuantShared) <= 227u * 1024u, "both-layo
 #define NVFP4_DUALQ_BAND_ROWS 1
 #endif
 
-template <int MODE_R, int G_R, int MODE_C, int G_C>
+template <int MODE_R, int G_R, int MODE_C, int G_C, bool MULTI>
 __global__ void __launch_bounds__(kDualThreads, 1)
 dual_quantize_kernel(const __grid_constant__ DualGroup grp, uint64_t seed, int reverse) {
   static_assert(G_C > 0, "the column view is rotated on the tensor cores");
@@ -1235,23 +1235,41 @@ dual_quantize_kernel(const __grid_constant__ DualGroup grp, uint64_t seed, int r
     asm volatile("bar.sync 1, %0;" ::"r"(kDualEpiWarps * 32) : "memory");
     const int64_t n_acc = my_tiles * kViews;
     const uint32_t r_in_tile = 32u * q + lane;
+    // a group of one (MULTI false): the member's constants once, before the
+    // loop; a larger group: looked up for each tile's member
+    const DualMember& m0 = grp.m[0];
+    const ScaleCtx sc_r0 = MULTI ? ScaleCtx{} : sh.sc[0][0], sc_c0 = MULTI ? ScaleCtx{} : sh.sc[0][1];
+    const bool r_codes16_0 = ((m0.cols / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(m0.codes_r) % 16) == 0;
+    const bool r_scales4_0 = ((m0.cols / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(m0.scales_r) % 4) == 0;
+    const bool c_codes16_0 = ((m0.rows / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(m0.codes_c) % 16) == 0;
+    const bool c_scales4_0 = ((m0.rows / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(m0.scales_c) % 4) == 0;
     for (int64_t j = slot; j < n_acc; j += kDualSlots) {
       const int64_t k = j / kViews;
       const int v = static_cast<int>(j % kViews);
       uint32_t rt, ct;
-      const int mi = group_tile(grp, dual_tile_index(k, n_tiles, reverse), band, rt, ct);
-      const DualMember& mb = grp.m[mi];
+      int mi = 0;
+      if constexpr (MULTI) {
+        mi = group_tile(grp, dual_tile_index(k, n_tiles, reverse), band, rt, ct);
+      } else {
+        const TileGrid tg{m0.n_rt, m0.n_ct, band};
+        tg.coords(dual_tile_index(k, n_tiles, reverse), rt, ct);
+      }
+      const DualMember& mb = MULTI ? grp.m[mi] : m0;
       const int64_t rows = mb.rows, cols = mb.cols;
-      const ScaleCtx sc_r = sh.sc[mi][0], sc_c = sh.sc[mi][1];
+      const ScaleCtx sc_r = MULTI ? sh.sc[mi][0] : sc_r0, sc_c = MULTI ? sh.sc[mi][1] : sc_c0;
       uint8_t* const codes_r = mb.codes_r;
       uint8_t* const scales_r = mb.scales_r;
       uint8_t* const codes_c = mb.codes_c;
       uint8_t* const scales_c = mb.scales_c;
       // row view: rows x cols; column view: cols x rows
-      const bool r_codes16 = ((cols / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes_r) % 16) == 0;
-      const bool r_scales4 = ((cols / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales_r) % 4) == 0;
-      const bool c_codes16 = ((rows / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes_c) % 16) == 0;
-      const bool c_scales4 = ((rows / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales_c) % 4) == 0;
+      const bool r_codes16 =
+          MULTI ? ((cols / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes_r) % 16) == 0 : r_codes16_0;
+      const bool r_scales4 =
+          MULTI ? ((cols / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales_r) % 4) == 0 : r_scales4_0;
+      const bool c_codes16 =
+          MULTI ? ((rows / 2) % 16) == 0 && (reinterpret_cast<uintptr_t>(codes_c) % 16) == 0 : c_codes16_0;
+      const bool c_scales4 =
+          MULTI ? ((rows / 16) % 4) == 0 && (reinterpret_cast<uintptr_t>(scales_c) % 4) == 0 : c_scales4_0;
       const bool r_blocks8 = ((cols / 16) % 8) == 0, c_blocks8 = ((rows / 16) % 8) == 0;
       if constexpr (kRowFromSmem) {
         const int s = static_cast<int>(k % kDualStages);
@@ -1506,7 +1524,8 @@ cudaError_t launch_dual_quantize_t(const DualQuantArgs* a, int n) {
     m.scales_c = a[i].scales_col;
     m.gscale_c = a[i].gscale_col;
   }
-  auto kernel = dual_quantize_kernel<MODE_R, G_R, MODE_C, G_C>;
+  auto kernel = n > 1 ? dual_quantize_kernel<MODE_R, G_R, MODE_C, G_C, true>
+                      : dual_quantize_kernel<MODE_R, G_R, MODE_C, G_C, false>;
   LaunchGeom geom;
   cudaError_t e = launch_geometry(kernel, kDualThreads, kDualDynSmem, 1, &geom);
   if (e != cudaSuccess) return e;
