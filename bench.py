@@ -61,6 +61,8 @@ NCU_TRAFFIC = {
         472376576 + 223989760,
     ("e67268332ab8fc9f", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
         472720896 + 224553728,
+    ("7abb43885c7454fa", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
+        472767744 + 224883968,
 }
 
 

@@ -7,8 +7,11 @@
  *     up iff U < (a - l) / (u - l); code = sign(y) << 3 | index, and a code of
  *     magnitude 0 is 0.  Evaluated in binary64, where a - l and the quotient
  *     by the power-of-two gap are exact.
- *     Kernel form (restated): a1 = min(max(a, RU(0.5 a + 0.5)), 6);
- *     t = 64 bits(a1) + ((~k << 12 & 0x0FFFF000) | 0x40000FC0) (mod 2^32);
+ *     Kernel form (restated): a1 = min(max(a, RU(0.5 a + 0.5)), 6); with
+ *     the draws of a pair in one word (low half: even element, high half:
+ *     odd) and h = word >> 16, t = 64 bits(a1) + 0x4FFFFFC0 + h 2^28 +
+ *     word (2^32 - 4096) for the even element and t = 64 bits(a1) +
+ *     0x4FFFFFC0 + h (2^32 - 4096) for the odd one (mod 2^32);
  *     v = (t & 0x7FFFFFFF) | (bits(y) & 0x80000000); the top nibbles of the
  *     eight v gathered into one word with byte permutes, then the sign of a
  *     zero magnitude cleared.
@@ -68,15 +71,18 @@ static uint32_t sr_rule(float y, uint32_t k) {
 /* the eight-element kernel form; k[i] = draw of element i, held as the
  * generator delivers it: word i/2, low half for even i, high for odd */
 static uint32_t sr_kernel8(const float* y, const uint32_t* k) {
-  uint32_t word[4], v[8];
-  for (int m = 0; m < 4; ++m) word[m] = k[2 * m] | (k[2 * m + 1] << 16);
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t k_at12 = (i & 1) ? (word[i >> 1] >> 4) : (word[i >> 1] << 12);
-    const uint32_t n = (~k_at12 & 0x0FFFF000u) | 0x40000FC0u;
-    const float a = fabsf(y[i]);
-    const float a1 = fminf(fmaxf(a, fma_up(a, 0.5f, 0.5f)), 6.0f);
-    const uint32_t t = to_bits(a1) * 64u + n;
-    v[i] = (t & 0x7FFFFFFFu) | (to_bits(y[i]) & 0x80000000u);
+  uint32_t v[8];
+  for (int m = 0; m < 4; ++m) {
+    const uint32_t word = k[2 * m] | (k[2 * m + 1] << 16);
+    const uint32_t h = word >> 16;
+    for (int j = 0; j < 2; ++j) {
+      const int i = 2 * m + j;
+      const float a = fabsf(y[i]);
+      const float a1 = fminf(fmaxf(a, fma_up(a, 0.5f, 0.5f)), 6.0f);
+      const uint32_t base = to_bits(a1) * 64u + 0x4FFFFFC0u;
+      const uint32_t t = j == 0 ? h * 0x10000000u + word * 0xFFFFF000u + base : h * 0xFFFFF000u + base;
+      v[i] = (t & 0x7FFFFFFFu) | (to_bits(y[i]) & 0x80000000u);
+    }
   }
   const uint32_t even = perm(perm(v[0], v[2], 0x0073u), perm(v[4], v[6], 0x7300u), 0x7610u);
   const uint32_t odd = perm(perm(v[1], v[3], 0x0073u), perm(v[5], v[7], 0x7300u), 0x7610u);
