@@ -63,6 +63,8 @@ NCU_TRAFFIC = {
         472720896 + 224553728,
     ("7abb43885c7454fa", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
         472767744 + 224883968,
+    ("8d52fa3e473e5908", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
+        472467456 + 224157952,
 }
 
 

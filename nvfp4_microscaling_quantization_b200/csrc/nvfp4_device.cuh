@@ -72,8 +72,19 @@ __device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) { return add2_rn(a
 // the multiplication that produced b.  (The packed add.rn.f32x2 is not safe
 // here: a GPU parity test of IF4 found a packed product and sum contracted
 // into one fused operation, skipping the product's rounding.)
-__device__ __forceinline__ float2 add2_after_mul(float2 a, float2 b) { return f2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y)); }
 __device__ __forceinline__ float2 sub2_after_mul(float2 a, float2 b) { return f2(__fsub_rn(a.x, b.x), __fsub_rn(a.y, b.y)); }
+// RN(a b) per lane as a fused multiply-add whose addend is -0 held in a
+// register the compiler cannot see through (nz, from ScaleCtx): exact, since
+// x + (-0) = x for every x, zeros included, and a product formed this way is
+// never merged with a sum that follows, so that sum can be the packed one.
+__device__ __forceinline__ float2 mul2_unmerged(float2 a, float2 b, float nz) { return fma2_rn(a, b, f2(nz, nz)); }
+// a - b per lane in one packed subtraction; b must not be a product that the
+// compiler could merge into it (see mul2_unmerged).
+__device__ __forceinline__ float2 sub2_packed(float2 a, float2 b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pack2(a)), "l"(pack2(b)));
+  return unpack2(d);
+}
 
 // max(|a|, |b|, |c|) in one three-input sm_100 max (exact; a NaN operand is
 // ignored as by fmaxf).
@@ -375,30 +386,54 @@ __device__ __forceinline__ uint32_t sign_nibbles8(const float* y) {
                                    __byte_perm(__float_as_uint(y[5]), __float_as_uint(y[7]), 0x7300u), 0x7610u);
   return ((even >> 4) & 0x08080808u) | (odd & 0x80808080u);
 }
-// s = min(RN(|t| + 1.5 2^23), 1.5 2^23 + 7): RNE(|t|) clamped to 7 in its low bits.
+// s = min(RN(|t| + 1.5 2^23), 1.5 2^23 + KMAX): RNE(|t|) clamped to KMAX
+// (7 for INT4, 3 for INT3) in its low bits.
+template <int KMAX = 7>
 __device__ __forceinline__ float int_magnitude_sum(float t) {
-  return fminf(__fadd_rn(fabsf(t), kRoundMagic), kRoundMagic + 7.0f);
+  return fminf(__fadd_rn(fabsf(t), kRoundMagic), kRoundMagic + static_cast<float>(KMAX));
 }
 
 // 3-bit elements, stored in nibbles (sign bit 3, magnitude code bits 0..1).
 // E2M0: magnitudes {0, 1, 2, 4}, nearest with ties to the even code (0.5 ->
-// 0, 1.5 -> 2, 3 -> 2), saturating at 4; zero is code 0.
-__device__ __forceinline__ uint32_t e2m0_nibble(float y) {
+// 0, 1.5 -> 2, 3 -> 2), saturating at 4; zero is code 0.  The rounding runs
+// on the bits of a1 = min(max(|y|, RU(0.5 + |y|/2)), 4), with no compares:
+// below 1, a1 = RU(0.5 + |y|/2) lies in [0.5, 1) and is above 0.75 iff
+// |y| > 0.5 (0.75 is a float, so the upward rounding keeps the comparison
+// exact); from 1 on, a1 = min(|y|, 4).  Adding 2^22 - 1 to the bits of a1,
+// plus one when its biased exponent is odd, carries into the exponent field
+// iff the mantissa is above one half, or exactly one half at an odd exponent:
+// the tie 1.5 (exponent 127) goes up and 3 (128) down, both to the even code
+// 2, and 0.75 (126, i.e. |y| = 0.5) down to code 0.  The exponent field of
+// the result is 126 + code, and its power of two is 2^(code - 1).
+__device__ __forceinline__ uint32_t e2m0_exponent_bits(float y) {
   const float a = fabsf(y);
-  const uint32_t m = (a > 0.5f ? 1u : 0u) + (a >= 1.5f ? 1u : 0u) + (a > 3.0f ? 1u : 0u);
-  return m == 0u ? 0u : (m | ((__float_as_uint(y) >> 28) & 8u));
+  const float a1 = fminf(fmaxf(a, __fmaf_ru(a, 0.5f, 0.5f)), 4.0f);
+  const uint32_t b = __float_as_uint(a1);
+  return b + 0x3FFFFFu + ((b >> 23) & 1u);
+}
+// |E2M0 value| from e2m0_exponent_bits: the power of two p in {0.5, 1, 2, 4},
+// then min(2p - 1, p) (exact), which is 0 for p = 0.5 (code 0) and p otherwise.
+__device__ __forceinline__ float e2m0_magnitude(uint32_t t) {
+  const float p = __uint_as_float(t & 0xFF800000u);
+  return fminf(__fmaf_rn(p, 2.0f, -1.0f), p);
+}
+// E2M0 codes of eight values from their e2m0_exponent_bits t_i: code_i =
+// (exponent field + 2) mod 4, which lands in bits 28..29 of 32 (t_i + 2^24)
+// = 32 t_i + 2^29 with bits 30..31 clear (exponent fields 126..129); the sign
+// of y_i goes into bit 31, the top nibbles are gathered with byte permutes,
+// and a zero code drops its sign.
+__device__ __forceinline__ uint32_t e2m0_nibbles8(const uint32_t* t, const float* y) {
+  uint32_t v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = (t[i] * 32u + 0x20000000u) | (__float_as_uint(y[i]) & 0x80000000u);
+  const uint32_t even = __byte_perm(__byte_perm(v[0], v[2], 0x0073u), __byte_perm(v[4], v[6], 0x7300u), 0x7610u);
+  const uint32_t odd = __byte_perm(__byte_perm(v[1], v[3], 0x0073u), __byte_perm(v[5], v[7], 0x7300u), 0x7610u);
+  return clear_negative_zero(((even >> 4) & 0x0F0F0F0Fu) | (odd & 0xF0F0F0F0u));
 }
 // signed E2M0 value of a nibble: 2^(m - 1) for m = 1..3
 __device__ __forceinline__ float e2m0_value(uint32_t c) {
   const uint32_t m = c & 3u;
   return m == 0u ? 0.0f : __uint_as_float(((126u + m) << 23) | ((c & 8u) << 28));
-}
-// INT3: k = clamp(RNE(t), -3, 3) as a sign-magnitude nibble (as int4_nibble)
-__device__ __forceinline__ float int3_level(float t) {
-  return fminf(fmaxf(__fsub_rn(__fadd_rn(t, kRoundMagic), kRoundMagic), -3.0f), 3.0f);
-}
-__device__ __forceinline__ uint32_t level_nibble(float k) {
-  return (__float_as_uint(__fadd_rn(fabsf(k), 8388608.0f)) & 7u) | ((__float_as_uint(k) >> 28) & 8u);
 }
 constexpr float kIF3K1 = 0.75f;            // RN(3/4)
 constexpr float kIF3K2 = 0x1.555556p+0f;   // RN(4/3)
@@ -418,44 +453,39 @@ struct BlockOut {
 // NVFP3 / NVINT3 / IF3 codes of one block of scaled values y under scale
 // byte S: E2M0, INT3, or (IF3) the option with the lower squared error in the
 // y domain (fmaf in element order, ties keep E2M0) with bit 7 set for INT3.
+// INT3 levels k = clamp(RNE(t), -3, 3) come from int_magnitude_sum<3>, their
+// signs from t's (NVINT3) or, for IF3, from the E2M0 codes: a nonzero level
+// needs |y| 3/4 >= 1/2, so |y| > 1/2, where the E2M0 code is nonzero and
+// carries the sign of y.  The errors use |y| - |v|, the same square as y - v.
 template <int MODE>
 __device__ __forceinline__ BlockOut block3_codes(const float* y, uint32_t S) {
-  BlockOut o{0u, 0u, S};
-  uint32_t f_lo = 0u, f_hi = 0u, i_lo = 0u, i_hi = 0u;
-  float eF = 0.0f, eI = 0.0f;
+  if constexpr (MODE == kNVINT3) {
+    uint32_t s[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    uint32_t cf = 0u, ci = 0u;
-    if constexpr (MODE == kNVINT3) {
-      cf = level_nibble(int3_level(y[i]));
-    } else {
-      cf = e2m0_nibble(y[i]);
-      if constexpr (MODE == kIF3) {
-        const float dF = __fsub_rn(y[i], e2m0_value(cf));
-        eF = __fmaf_rn(dF, dF, eF);
-        const float k = int3_level(__fmul_rn(y[i], kIF3K1));
-        const float dI = __fsub_rn(y[i], __fmul_rn(k, kIF3K2));
-        eI = __fmaf_rn(dI, dI, eI);
-        ci = level_nibble(k);
-      }
-    }
-    if (i < 8) {
-      f_lo |= cf << (4 * i);
-      i_lo |= ci << (4 * i);
-    } else {
-      f_hi |= cf << (4 * (i - 8));
-      i_hi |= ci << (4 * (i - 8));
-    }
-  }
-  if (MODE == kIF3 && eI < eF) {
-    o.lo = i_lo;
-    o.hi = i_hi;
-    o.scale = S | 0x80u;
+    for (int i = 0; i < 16; ++i) s[i] = __float_as_uint(int_magnitude_sum<3>(y[i]));
+    return BlockOut{int_nibbles8(s, sign_nibbles8(y)), int_nibbles8(s + 8, sign_nibbles8(y + 8)), S};
   } else {
-    o.lo = f_lo;
-    o.hi = f_hi;
+    uint32_t t[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) t[i] = e2m0_exponent_bits(y[i]);
+    const uint32_t f_lo = e2m0_nibbles8(t, y), f_hi = e2m0_nibbles8(t + 8, y + 8);
+    if constexpr (MODE == kIF3) {
+      uint32_t s[16];
+      float eF = 0.0f, eI = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float a = fabsf(y[i]);
+        const float dF = __fsub_rn(a, e2m0_magnitude(t[i]));
+        eF = __fmaf_rn(dF, dF, eF);
+        const float sI = int_magnitude_sum<3>(__fmul_rn(y[i], kIF3K1));
+        s[i] = __float_as_uint(sI);
+        const float dI = __fsub_rn(a, __fmul_rn(__fsub_rn(sI, kRoundMagic), kIF3K2));
+        eI = __fmaf_rn(dI, dI, eI);
+      }
+      if (eI < eF) return BlockOut{int_nibbles8(s, f_lo), int_nibbles8(s + 8, f_hi), S | 0x80u};
+    }
+    return BlockOut{f_lo, f_hi, S};
   }
-  return o;
 }
 
 
@@ -699,6 +729,7 @@ struct PairRng {
 // their round-to-nearest reciprocals for the division below.
 struct ScaleCtx {
   float s_g, q6, q4, r6, r4;
+  float nz;             // -0, derived from the amax loaded at run time (see mul2_unmerged)
   bool markstein;       // the reciprocal-based division is exact for every block
   const float4* tbl;    // per E4M3 code S: {dec(S), d = RN(dec(S) s_g), RN(1/d) or 0, 0}
 };
@@ -721,6 +752,10 @@ __device__ __forceinline__ ScaleCtx make_scale_ctx(float amax) {
   // a / q < 2^-12, where any value within an ulp gives the same (zero) E4M3
   // scale; outside that range the kernels divide with __fdiv_rn.
   c.markstein = c.q4 >= 0x1p-90f && c.q6 <= 0x1p100f;
+  // -0 for every amax >= 0 (for a negative amax +0, which changes nothing:
+  // RN(a b + 0) differs from RN(a b) only in the sign of a zero result, and
+  // every code of magnitude zero is stored unsigned)
+  c.nz = __uint_as_float((__float_as_uint(amax) & 0x80000000u) ^ 0x80000000u);
   return c;
 }
 
@@ -857,7 +892,7 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
       float2 e = f2(0.0f, 0.0f);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float2 diff = sub2_after_mul(z[i], mul2_rn(f2(va[i], vb[i]), d));
+        const float2 diff = sub2_packed(z[i], mul2_unmerged(f2(va[i], vb[i]), d, sc.nz));
         e = fma2_rn(diff, diff, e);
       }
       err[k] = e;
@@ -893,20 +928,18 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
     const uint32_t f = __float_as_uint(fmaxf(aa, ab)) >> 23;
     const uint32_t byte = f > 2u ? f - 2u : 0u;
     const float inv = __uint_as_float((254u - byte) << 23);
-    oa = BlockOut{0u, 0u, byte};
-    ob = BlockOut{0u, 0u, byte};
+    float ya[16], yb[16];
+    uint32_t ta[16], tb[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float2 y = mul2_rn(z[i], f2(inv, inv));
-      const uint32_t ca = e2m0_nibble(y.x), cb = e2m0_nibble(y.y);
-      if (i < 8) {
-        oa.lo |= ca << (4 * i);
-        ob.lo |= cb << (4 * i);
-      } else {
-        oa.hi |= ca << (4 * (i - 8));
-        ob.hi |= cb << (4 * (i - 8));
-      }
+      ya[i] = y.x;
+      yb[i] = y.y;
+      ta[i] = e2m0_exponent_bits(y.x);
+      tb[i] = e2m0_exponent_bits(y.y);
     }
+    oa = BlockOut{e2m0_nibbles8(ta, ya), e2m0_nibbles8(ta + 8, ya + 8), byte};
+    ob = BlockOut{e2m0_nibbles8(tb, yb), e2m0_nibbles8(tb + 8, yb + 8), byte};
     return;
   } else if constexpr (MODE == kNVINT4) {
     // q6 holds RN(7 s_g) for this mode (make_scale_ctx)
@@ -984,7 +1017,7 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
       float2 e = f2(0.0f, 0.0f);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float2 diff = sub2_after_mul(z[i], mul2_rn(f2(va[i], vb[i]), d));
+        const float2 diff = sub2_packed(z[i], mul2_unmerged(f2(va[i], vb[i]), d, sc.nz));
         e = fma2_rn(diff, diff, e);
       }
       if (e.x < best.x) {
@@ -1014,7 +1047,8 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
     float ya[16], yb[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const float2 y = mul2_rn(z[i], r);
+      // IF4 subtracts from y below: its product is kept unmerged
+      const float2 y = MODE == kIF4 ? mul2_unmerged(z[i], r, sc.nz) : mul2_rn(z[i], r);
       ya[i] = y.x;
       yb[i] = y.y;
     }
@@ -1059,7 +1093,7 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float2 y = f2(ya[i], yb[i]);
-        const float2 dF = sub2_after_mul(y, f2(va[i], vb[i]));
+        const float2 dF = sub2_packed(y, f2(va[i], vb[i]));
         eF = fma2_rn(dF, dF, eF);
         // the INT4 level k = clamp(RNE(y K1), -7, 7) through its magnitude:
         // |k| = s - 1.5 2^23 exactly, and |y| - |k| K2 = +-(y - k K2), the

@@ -215,7 +215,7 @@ quantize_tma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int6
     for (int k = 0; k < kStages; ++k) load(k);
   }
 
-  ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false, nullptr};
+  ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, -0.0f, false, nullptr};
   if constexpr (!AMAX_ONLY) {
     // the first loads are in flight: build the scale table meanwhile
     build_scale_table(scale_tbl, global_scale_of<MODE>(*amax), tid, kNT);

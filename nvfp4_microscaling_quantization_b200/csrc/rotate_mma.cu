@@ -321,7 +321,7 @@ rotate_mma_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_
     // memory requires): its thread owns one tile row, all 128 columns
     const uint32_t q = warp & 3u, grp = warp >> 2;
     grid_dependency_wait();
-    ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, false, nullptr};
+    ScaleCtx sc{1.0f, 6.0f, 4.0f, 1.0f / 6.0f, 0.25f, -0.0f, false, nullptr};
     if constexpr (KIND == kQuantize) {
       sc = make_scale_ctx<MODE>(*amax);
       // the scale table, built by the epilogue warps while the first tiles load

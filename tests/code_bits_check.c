@@ -15,12 +15,24 @@
  *     v = (t & 0x7FFFFFFF) | (bits(y) & 0x80000000); the top nibbles of the
  *     eight v gathered into one word with byte permutes, then the sign of a
  *     zero magnitude cleared.
- * (2) INT4 levels (NVINT4, and IF4's integer option).
- *     Rule: k = clamp(RNE(t), -7, 7) as a sign-magnitude nibble, never -0.
- *     Kernel form (restated): s = min(RN(|t| + 1.5 2^23), 1.5 2^23 + 7); the
+ * (2) INT4 and INT3 levels (NVINT4, IF4's integer option; NVINT3, IF3's).
+ *     Rule: k = clamp(RNE(t), -K, K) (K = 7, 3) as a sign-magnitude nibble,
+ *     never -0.
+ *     Kernel form (restated): s = min(RN(|t| + 1.5 2^23), 1.5 2^23 + K); the
  *     low bytes of eight s gathered into nibbles with byte permutes, the
  *     signs of the eight t added from their top bytes, then the sign of a
  *     zero magnitude cleared.
+ * (3) E2M0 codes and magnitudes (NVFP3, MXFP3, IF3's E2M0 option).
+ *     Rule: the nearest of {0, 1, 2, 4} to |y| (distances in binary64 from
+ *     min(|y|, 8), exact), a tie going to the even code index (0.5 -> 0,
+ *     1.5 -> 2, 3 -> 2); code = sign(y) << 3 | index, a zero index unsigned.
+ *     Kernel form (restated): a1 = min(max(|y|, RU(0.5 |y| + 0.5)), 4);
+ *     t = bits(a1) + 2^22 - 1 + ((bits(a1) >> 23) & 1); v = (32 t + 2^29) |
+ *     (bits(y) & 0x80000000); the top nibbles of eight v gathered as for SR,
+ *     then the sign of a zero index cleared; the magnitude is min(2p - 1, p)
+ *     with p the float of bits t & 0xFF800000.
+ *     Also checked: where RNE(RN(|y| 3/4)) >= 1 (a nonzero IF3 integer
+ *     level) the E2M0 index is nonzero, so it carries the sign of y.
  * Byte permute: byte n of perm(x, y, s) is byte (nibble n of s) of the
  * eight bytes y:x (x bytes 0..3, y bytes 4..7).
  * Build: cc -O2 -ffp-contract=off -fno-fast-math -frounding-math, linked with
@@ -171,19 +183,19 @@ int64_t sr_check(int64_t n_random, int variant, int64_t* checked) {
   return bad;
 }
 
-/* ------------------------------------------------------------------ INT4 */
-static uint32_t int4_rule(float t) {
+/* ------------------------------------------------------------ INT4, INT3 */
+static uint32_t int_rule(float t, int kmax) {
   double k = nearbyint((double)t);  /* ties to even (default rounding mode) */
-  if (k > 7.0) k = 7.0;
-  if (k < -7.0) k = -7.0;
+  if (k > kmax) k = kmax;
+  if (k < -kmax) k = -kmax;
   const int ki = (int)k;
   return ki == 0 ? 0u : ((uint32_t)(ki < 0 ? -ki : ki) | (ki < 0 ? 8u : 0u));
 }
 
-static uint32_t int4_kernel8(const float* t) {
+static uint32_t int_kernel8(const float* t, int kmax) {
   const float magic = 12582912.0f;  /* 1.5 2^23 */
   uint32_t s[8];
-  for (int i = 0; i < 8; ++i) s[i] = to_bits(fminf(fabsf(t[i]) + magic, magic + 7.0f));
+  for (int i = 0; i < 8; ++i) s[i] = to_bits(fminf(fabsf(t[i]) + magic, magic + (float)kmax));
   const uint32_t even = perm(perm(s[0], s[2], 0x0040u), perm(s[4], s[6], 0x4000u), 0x7610u);
   const uint32_t odd = perm(perm(s[1], s[3], 0x0040u), perm(s[5], s[7], 0x4000u), 0x7610u);
   const uint32_t se = perm(perm(to_bits(t[0]), to_bits(t[2]), 0x0073u), perm(to_bits(t[4]), to_bits(t[6]), 0x7300u), 0x7610u);
@@ -197,18 +209,18 @@ static uint32_t int4_kernel8(const float* t) {
  * (at 2^22 and above RN(|t| + 1.5 2^23) is past the clamp as well), and
  * random binary32 values in (-16, 16); eight per word in order.  Returns the
  * number of elements whose nibble differs from the rule. */
-int64_t int4_check(int64_t n_random, int variant, int64_t* checked) {
+static int64_t int_levels_check(int64_t n_random, int variant, int kmax, int64_t* checked) {
   int64_t bad = 0, n = 0;
   rng_state = 0xD1B54A32D192ED03ull;
   float vals[8];
   int nv = 0;
 #define FLUSH()                                                              \
   do {                                                                       \
-    uint32_t w = int4_kernel8(vals);                                         \
+    uint32_t w = int_kernel8(vals, kmax);                                    \
     if (variant == 1) w ^= 4u;                                               \
     for (int e = 0; e < nv; ++e) {                                           \
       ++n;                                                                   \
-      bad += ((w >> (4 * e)) & 0xFu) != int4_rule(vals[e]);                  \
+      bad += ((w >> (4 * e)) & 0xFu) != int_rule(vals[e], kmax);            \
     }                                                                        \
     nv = 0;                                                                  \
   } while (0)
@@ -226,6 +238,104 @@ int64_t int4_check(int64_t n_random, int variant, int64_t* checked) {
   for (uint32_t h = 0; h < 65536u; ++h) {
     const float t = from_bits(h << 16);
     if (isfinite(t)) PUSH(t);
+  }
+  for (int64_t r = 0; r < n_random; ++r) PUSH(from_bits((uint32_t)next64() & 0xC1FFFFFFu));
+  if (nv) {
+    while (nv < 8) vals[nv++] = 0.0f;
+    FLUSH();
+  }
+#undef PUSH
+#undef FLUSH
+  *checked = n;
+  return bad;
+}
+
+int64_t int4_check(int64_t n_random, int variant, int64_t* checked) {
+  return int_levels_check(n_random, variant, 7, checked);
+}
+int64_t int3_check(int64_t n_random, int variant, int64_t* checked) {
+  return int_levels_check(n_random, variant, 3, checked);
+}
+
+/* ------------------------------------------------------------------ E2M0 */
+static const double kE2m0[4] = {0.0, 1.0, 2.0, 4.0};
+
+static uint32_t e2m0_rule(float y) {
+  /* |y| capped at 8 (nearest value 4 either way) keeps the distances exact */
+  const double a = fmin(fabs((double)y), 8.0);
+  int best = 0;
+  for (int c = 1; c < 4; ++c) {
+    const double dc = fabs(a - kE2m0[c]), db = fabs(a - kE2m0[best]);
+    if (dc < db || (dc == db && (c & 1) == 0)) best = c;
+  }
+  return best == 0 ? 0u : ((uint32_t)best | (signbit(y) ? 8u : 0u));
+}
+
+static uint32_t e2m0_t(float y) {
+  const float a = fabsf(y);
+  const float a1 = fminf(fmaxf(a, fma_up(a, 0.5f, 0.5f)), 4.0f);
+  const uint32_t b = to_bits(a1);
+  return b + 0x3FFFFFu + ((b >> 23) & 1u);
+}
+
+static float e2m0_magnitude(uint32_t t) {
+  const float p = from_bits(t & 0xFF800000u);
+  volatile float q = fmaf(p, 2.0f, -1.0f);
+  return fminf(q, p);
+}
+
+static uint32_t e2m0_kernel8(const float* y) {
+  uint32_t v[8];
+  for (int i = 0; i < 8; ++i) v[i] = (e2m0_t(y[i]) * 32u + 0x20000000u) | (to_bits(y[i]) & 0x80000000u);
+  const uint32_t even = perm(perm(v[0], v[2], 0x0073u), perm(v[4], v[6], 0x7300u), 0x7610u);
+  const uint32_t odd = perm(perm(v[1], v[3], 0x0073u), perm(v[5], v[7], 0x7300u), 0x7610u);
+  return clear_negative_zero(((even >> 4) & 0x0F0F0F0Fu) | (odd & 0xF0F0F0F0u));
+}
+
+/* Values y: every finite bf16 value, the thresholds 0.5, 1.5, 3 and the
+ * saturation 4 with their binary32 neighbours (both signs), and random
+ * binary32 values in (-16, 16); eight per word.  Counts the elements whose
+ * code or magnitude differs from the rule, and those where a nonzero IF3
+ * integer level meets a zero E2M0 index (variant 1 flips one code bit per
+ * word, variant 2 takes the magnitude 0.5 for index 0). */
+int64_t e2m0_check(int64_t n_random, int variant, int64_t* checked) {
+  int64_t bad = 0, n = 0;
+  rng_state = 0x94D049BB133111EBull;
+  float vals[8];
+  int nv = 0;
+#define FLUSH()                                                              \
+  do {                                                                       \
+    uint32_t w = e2m0_kernel8(vals);                                         \
+    if (variant == 1) w ^= 1u;                                               \
+    for (int e = 0; e < nv; ++e) {                                           \
+      const uint32_t want = e2m0_rule(vals[e]);                              \
+      const uint32_t t = e2m0_t(vals[e]);                                    \
+      const float mag = variant == 2 ? from_bits(t & 0xFF800000u) : e2m0_magnitude(t); \
+      const float lvl = nearbyintf(fabsf(vals[e]) * 0.75f);                  \
+      ++n;                                                                   \
+      bad += ((w >> (4 * e)) & 0xFu) != want;                                \
+      bad += (double)mag != kE2m0[want & 3u];                                \
+      bad += lvl >= 1.0f && (want & 3u) == 0u;                               \
+    }                                                                        \
+    nv = 0;                                                                  \
+  } while (0)
+#define PUSH(x)                                                              \
+  do {                                                                       \
+    vals[nv++] = (x);                                                        \
+    if (nv == 8) FLUSH();                                                    \
+  } while (0)
+  static const float edges[] = {0.0f, 0.5f, 0.75f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  for (int k = 0; k < (int)(sizeof(edges) / sizeof(edges[0])); ++k) {
+    for (int sgn = 0; sgn < 2; ++sgn) {
+      const float x = sgn ? -edges[k] : edges[k];
+      PUSH(x);
+      PUSH(nextafterf(x, INFINITY));
+      PUSH(nextafterf(x, -INFINITY));
+    }
+  }
+  for (uint32_t h = 0; h < 65536u; ++h) {
+    const float y = from_bits(h << 16);
+    if (isfinite(y)) PUSH(y);
   }
   for (int64_t r = 0; r < n_random; ++r) PUSH(from_bits((uint32_t)next64() & 0xC1FFFFFFu));
   if (nv) {

@@ -1,6 +1,7 @@
 """The kernels' bit-level formation of codes, pinned on the CPU.
 
-Stochastic rounding onto E2M1 and the INT4 levels of NVINT4 and IF4 are
+Stochastic rounding onto E2M1, the INT4 levels of NVINT4 and IF4, the INT3
+levels of NVINT3 and IF3, and the E2M0 codes of NVFP3, MXFP3 and IF3 are
 formed in the kernels without conversion instructions: integer sums on the
 bits of the floats, and byte permutes that gather eight elements' nibbles
 into one code word.  tests/code_bits_check.c restates those sequences in C
@@ -8,10 +9,12 @@ and compares every element, bit for bit, with the rules written from their
 definitions: stochastic rounding goes up iff U < (a - l)/(u - l) (the
 palettes post, "The two corners, and what the palette does to them"), the
 INT4 level is clamp(RNE(t), -7, 7) as a sign-magnitude nibble (IF4 paper
-page, Table 1 and Figure 3).  Inputs: every finite bf16 value at the draws
-next to its decision point and at the extremes, in random word slots, plus
-random binary32 values; the ties, clamp edges and signed zeros of the INT4
-levels.  No difference is allowed.
+page, Table 1 and Figure 3), the INT3 level clamp(RNE(t), -3, 3), and E2M0
+the nearest of {0, 1, 2, 4} with ties to the even code (the same page's
+3-bit formats table lists E2M0 and INT3 elements).  Inputs: every finite
+bf16 value at the draws next to its decision point and at the extremes, in
+random word slots, plus random binary32 values; the ties, clamp edges and
+signed zeros of the integer levels and of E2M0.  No difference is allowed.
 """
 import ctypes
 import os
@@ -30,7 +33,7 @@ def checker():
     subprocess.run(["cc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-frounding-math", "-fPIC", "-shared",
                     os.path.join(HERE, "code_bits_check.c"), "-o", so, "-lm"], check=True)
     L = ctypes.CDLL(so)
-    for fn in (L.sr_check, L.int4_check):
+    for fn in (L.sr_check, L.int4_check, L.int3_check, L.e2m0_check):
         fn.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
         fn.restype = ctypes.c_int64
     return L
@@ -48,6 +51,12 @@ def test_planted_mistakes_are_caught(checker):
     assert bad > 100000 and n > 0
     bad, n = _run(checker.int4_check, 0, variant=1)
     assert bad > 1000 and n > 0
+    bad, n = _run(checker.int3_check, 0, variant=1)
+    assert bad > 1000 and n > 0
+    bad, n = _run(checker.e2m0_check, 0, variant=1)
+    assert bad > 1000 and n > 0
+    bad, n = _run(checker.e2m0_check, 0, variant=2)  # magnitude 0.5 kept for index 0
+    assert bad > 1000 and n > 0
 
 
 def test_stochastic_rounding_codes(checker):
@@ -60,3 +69,15 @@ def test_int4_level_codes(checker):
     bad, n = _run(checker.int4_check, 1 << 20)
     assert n > 1_000_000
     assert bad == 0, f"{bad} of {n} INT4 nibbles differ from the rule"
+
+
+def test_int3_level_codes(checker):
+    bad, n = _run(checker.int3_check, 1 << 20)
+    assert n > 1_000_000
+    assert bad == 0, f"{bad} of {n} INT3 nibbles differ from the rule"
+
+
+def test_e2m0_codes_and_magnitudes(checker):
+    bad, n = _run(checker.e2m0_check, 1 << 20)
+    assert n > 1_000_000
+    assert bad == 0, f"{bad} of {n} E2M0 codes, magnitudes or IF3 sign sources differ from the rule"
