@@ -65,6 +65,8 @@ NCU_TRAFFIC = {
         472767744 + 224883968,
     ("8d52fa3e473e5908", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
         472467456 + 224157952,
+    ("159b0bcef2cc77d9", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
+        472862976 + 224496384,
 }
 
 

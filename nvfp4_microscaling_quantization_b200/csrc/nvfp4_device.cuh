@@ -1095,11 +1095,14 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
         const float2 y = f2(ya[i], yb[i]);
         const float2 dF = sub2_packed(y, f2(va[i], vb[i]));
         eF = fma2_rn(dF, dF, eF);
-        // the INT4 level k = clamp(RNE(y K1), -7, 7) through its magnitude:
-        // |k| = s - 1.5 2^23 exactly, and |y| - |k| K2 = +-(y - k K2), the
-        // same square (k is 0 or has the sign of y)
-        const float2 t = mul2_rn(y, f2(kIF4K1, kIF4K1));
-        const float2 s2 = f2(int_magnitude_sum(t.x), int_magnitude_sum(t.y));
+        // the INT4 level k = clamp(RNE(y K1), -7, 7) through its magnitude
+        // |k| = s - 1.5 2^23, s = RN(RN(min(|y|, 6) K1) + 1.5 2^23): RN(6 K1)
+        // is 7 exactly and RN is monotone, so clamping |y| at 6 first clamps
+        // the level at 7 and the two-lane sum needs no clamp of its own; and
+        // |y| - |k| K2 = +-(y - k K2), the same square (k is 0 or has the
+        // sign of y)
+        const float2 yc = f2(fminf(fabsf(y.x), 6.0f), fminf(fabsf(y.y), 6.0f));
+        const float2 s2 = add2_rn(mul2_unmerged(yc, f2(kIF4K1, kIF4K1), sc.nz), f2(kRoundMagic, kRoundMagic));
         sa[i] = __float_as_uint(s2.x);
         sb[i] = __float_as_uint(s2.y);
         const float2 vi = mul2_rn(sub2_rn(s2, f2(kRoundMagic, kRoundMagic)), f2(kIF4K2, kIF4K2));

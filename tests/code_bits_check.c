@@ -22,6 +22,10 @@
  *     low bytes of eight s gathered into nibbles with byte permutes, the
  *     signs of the eight t added from their top bytes, then the sign of a
  *     zero magnitude cleared.
+ * (2b) IF4's INT4 level magnitude from y.
+ *     Rule: |k| = |clamp(RNE(RN(y K1)), -7, 7)| with K1 = RN(7/6).
+ *     Kernel form (restated): s = RN(RN(min(|y|, 6) K1) + 1.5 2^23), |k| =
+ *     the low byte of s (no clamp on s: RN(6 K1) = 7).
  * (3) E2M0 codes and magnitudes (NVFP3, MXFP3, IF3's E2M0 option).
  *     Rule: the nearest of {0, 1, 2, 4} to |y| (distances in binary64 from
  *     min(|y|, 8), exact), a tie going to the even code index (0.5 -> 0,
@@ -255,6 +259,63 @@ int64_t int4_check(int64_t n_random, int variant, int64_t* checked) {
 }
 int64_t int3_check(int64_t n_random, int variant, int64_t* checked) {
   return int_levels_check(n_random, variant, 3, checked);
+}
+
+/* ------------------------------------------------------- IF4 level from y */
+static const float kIF4K1 = 0x1.2aaaaap+0f; /* RN(7/6) */
+
+static uint32_t if4_level_rule(float y) {
+  volatile float t = y * kIF4K1;
+  double k = nearbyint((double)t);
+  if (k > 7.0) k = 7.0;
+  if (k < -7.0) k = -7.0;
+  return (uint32_t)fabs(k);
+}
+
+static uint32_t if4_level_kernel(float y) {
+  volatile float t = fminf(fabsf(y), 6.0f) * kIF4K1;
+  volatile float s = t + 12582912.0f;
+  return to_bits(s) & 0xFFu;
+}
+
+/* Values y: every finite bf16 value, the points where RN(y K1) is a tie
+ * (m + 1/2) / K1 with their binary32 neighbours, 6 and its neighbours, and
+ * random binary32 values in (-16, 16).  Variant 1 drops the clamp at 6. */
+int64_t if4_level_check(int64_t n_random, int variant, int64_t* checked) {
+  int64_t bad = 0, n = 0;
+  rng_state = 0x2545F4914F6CDD1Dull;
+#define CHECK(yv)                                                            \
+  do {                                                                       \
+    const float y_ = (yv);                                                   \
+    uint32_t got = if4_level_kernel(y_);                                     \
+    if (variant == 1) {                                                      \
+      volatile float t_ = fabsf(y_) * kIF4K1;                                \
+      volatile float s_ = t_ + 12582912.0f;                                  \
+      got = to_bits(s_) & 0xFFu;                                             \
+    }                                                                        \
+    ++n;                                                                     \
+    bad += got != if4_level_rule(y_);                                        \
+  } while (0)
+  for (uint32_t h = 0; h < 65536u; ++h) {
+    const float y = from_bits(h << 16);
+    if (isfinite(y)) CHECK(y);
+  }
+  for (int m = -8; m <= 8; ++m) {
+    const float y0 = (float)(((double)m + 0.5) / (double)kIF4K1);
+    float y = y0;
+    for (int d = 0; d < 4; ++d) y = nextafterf(y, -INFINITY);
+    for (int d = 0; d < 9; ++d, y = nextafterf(y, INFINITY)) CHECK(y);
+  }
+  for (int sgn = 0; sgn < 2; ++sgn) {
+    const float x = sgn ? -6.0f : 6.0f;
+    CHECK(x);
+    CHECK(nextafterf(x, INFINITY));
+    CHECK(nextafterf(x, -INFINITY));
+  }
+  for (int64_t r = 0; r < n_random; ++r) CHECK(from_bits((uint32_t)next64() & 0xC1FFFFFFu));
+#undef CHECK
+  *checked = n;
+  return bad;
 }
 
 /* ------------------------------------------------------------------ E2M0 */

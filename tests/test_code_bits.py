@@ -33,7 +33,7 @@ def checker():
     subprocess.run(["cc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-frounding-math", "-fPIC", "-shared",
                     os.path.join(HERE, "code_bits_check.c"), "-o", so, "-lm"], check=True)
     L = ctypes.CDLL(so)
-    for fn in (L.sr_check, L.int4_check, L.int3_check, L.e2m0_check):
+    for fn in (L.sr_check, L.int4_check, L.int3_check, L.e2m0_check, L.if4_level_check):
         fn.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
         fn.restype = ctypes.c_int64
     return L
@@ -56,6 +56,8 @@ def test_planted_mistakes_are_caught(checker):
     bad, n = _run(checker.e2m0_check, 0, variant=1)
     assert bad > 1000 and n > 0
     bad, n = _run(checker.e2m0_check, 0, variant=2)  # magnitude 0.5 kept for index 0
+    assert bad > 1000 and n > 0
+    bad, n = _run(checker.if4_level_check, 1 << 16, variant=1)  # no clamp of |y| at 6
     assert bad > 1000 and n > 0
 
 
@@ -81,3 +83,9 @@ def test_e2m0_codes_and_magnitudes(checker):
     bad, n = _run(checker.e2m0_check, 1 << 20)
     assert n > 1_000_000
     assert bad == 0, f"{bad} of {n} E2M0 codes, magnitudes or IF3 sign sources differ from the rule"
+
+
+def test_if4_integer_level_from_y(checker):
+    bad, n = _run(checker.if4_level_check, 1 << 20)
+    assert n > 1_000_000
+    assert bad == 0, f"{bad} of {n} IF4 integer levels differ from clamp(RNE(RN(y K1)), -7, 7)"
