@@ -246,6 +246,26 @@ def test_exhaustive_bf16_rtn_path():
             assert np.all(gpu[1][:n // 8] == 0x78)  # scale 256
 
 
+SATURATING_MODES = [(W.RTN, 0), (W.SR, 0), (W.MS_EDEN, 16), (W.MS_EDEN, 128), (W.IF4, 0), (W.IF4, 128),
+                    (W.FOUR_OVER_SIX, 0), (W.SR, 128), (W.SCALE_SEARCH, 0), (W.NVINT4, 0), (W.NVFP3, 0),
+                    (W.NVINT3, 0), (W.IF3, 0), (W.IF3, 128)]
+
+
+@pytest.mark.parametrize("mode,g", SATURATING_MODES)
+@pytest.mark.parametrize("layout", [W.ROWWISE, W.TRANSPOSED])
+def test_amax_far_below_the_tensor_maximum(mode, g, layout):
+    """A supplied tensor amax 1/64 of the true one: most block scales saturate at
+    448 and the scaled values run far past every grid, so the saturation of
+    E2M1 at 6, of E2M0 at 4, the clamps of the integer levels at 7 and 3, and
+    MS-EDEN's corrected scale at 448 all decide codes."""
+    gen = torch.Generator().manual_seed(41)
+    x = (torch.randn((128, 256), generator=gen) * 3.0).to(torch.bfloat16)
+    amax = float(x.float().abs().max()) / 64.0
+    gpu = compare_call(x, layout, mode, g, 77, amax=amax)
+    if mode not in (W.SCALE_SEARCH, W.FOUR_OVER_SIX):
+        assert np.mean((np.asarray(gpu[1]) & 0x7F) == 0x7E) > 0.5  # most scales saturated at 448
+
+
 def _neighbourhood(centres, radius):
     out = []
     for c in centres:
