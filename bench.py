@@ -805,8 +805,9 @@ def run_ours(args, world, rank, local):
             "workload": "mlp_up: one Llama-style MLP up-projection training step's tensors, "
                         "X 16384x4096 N(0,1), W 14336x4096 N(0,0.02^2), dY 16384x14336 Student-t3 std 1e-4",
             "calls": [c.call.name for c in calls],
-            "path": "per tensor: one tensor-amax pre-pass for both layouts (nvfp4_amax_dual), then both "
-                    "layouts' codes and scales from one read (nvfp4_quantize_dual), C ABI, one stream",
+            "path": "X and W together, then dY: one tensor-amax pre-pass for both layouts of every tensor of "
+                    "the group (nvfp4_amax_dual_group), then both layouts' codes and scales from one read of each "
+                    "(nvfp4_quantize_dual_group); 4 launches, C ABI, one stream",
             "timing": "the K steps captured once as one CUDA graph of the C-ABI launches (consecutive launches "
                       "adjacent, CUDA events at the step boundaries) and replayed once; per-launch times from a "
                       "second replay with an event between every two launches",
@@ -862,14 +863,15 @@ def run_e2e(args, calls, tensors, stream, device, world, bytes_per_step):
     inputs, the six calls, D2H of every output, all inside the timed region.
 
     Steps are pipelined the way a caller streaming tensors would run them: the
-    host-to-device copies (one stream) of step i overlap the device-to-host
-    copies (another stream) of step i-1, the kernels run on a third, and the
-    outputs are double-buffered so step i's kernels never overwrite what step
-    i-1 is still copying out."""
+    host-to-device copies (one stream) of step i overlap the kernels (a second
+    stream) of step i-1 and the device-to-host copies (a third) of step i-1;
+    inputs and outputs are double-buffered, so a step's copies never overwrite
+    what the previous step's kernels still read or its outputs still hold."""
     N = calls[0].N
     s_in, s_comp, s_out = (torch.cuda.Stream(device) for _ in range(3))
     sh = ctypes.c_void_p(s_comp.cuda_stream)
-    sets = [[Call(N, c.call, tensors[c.call.tensor], c.seed, sh) for c in calls] for _ in range(2)]
+    inputs = [tensors, {k: torch.empty_like(v) for k, v in tensors.items()}]
+    sets = [[Call(N, c.call, inputs[b][c.call.tensor], c.seed, sh) for c in calls] for b in range(2)]
     group_sets = [group_step_parts([TensorCalls(N, [c for c in cs if c.call.tensor == name])
                                     for name in dict.fromkeys(c.call.tensor for c in cs)]) for cs in sets]
     host_in = {k: v.cpu().pin_memory() for k, v in tensors.items()}
@@ -883,10 +885,10 @@ def run_e2e(args, calls, tensors, stream, device, world, bytes_per_step):
         ev = {k: [torch.cuda.Event() for _ in range(K)] for k in ("in", "comp", "out")}
         for i in range(K):
             b = i % 2
-            if i > 0:
-                s_in.wait_event(ev["comp"][i - 1])   # the inputs are free once the kernels are done
+            if i >= 2:
+                s_in.wait_event(ev["comp"][i - 2])   # input set b is free once step i-2's kernels are done
             with torch.cuda.stream(s_in):
-                for k, t in tensors.items():
+                for k, t in inputs[b].items():
                     t.copy_(host_in[k], non_blocking=True)
             ev["in"][i].record(s_in)
             s_comp.wait_event(ev["in"][i])
@@ -919,7 +921,7 @@ def run_e2e(args, calls, tensors, stream, device, world, bytes_per_step):
     return {"value": round(weak_scaling_value(bytes_per_step, K, world, secs), 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
             "ms_per_step": round(secs * 1e3 / K, 3),
-            "pipeline": "H2D of step i || D2H of step i-1 || kernels, outputs double-buffered"}
+            "pipeline": "H2D of step i || kernels and D2H of step i-1, inputs and outputs double-buffered"}
 
 
 # ------------------------------------------------------------------------ CPU oracle
