@@ -785,12 +785,14 @@ dual_amax_kernel(const __grid_constant__ DualGroup grp, uint64_t seed, int g_r, 
   }
 }
 
-// The same pre-pass when both views are rotated (dY of the backward pass),
+// The same pre-pass when both views are rotated with different group sizes,
 // in groups: two epilogue groups of eight warps, each owning two 128-column
 // accumulators (row view and column view of one tile, one commit for both);
 // warp (q, j) of a group reads lane quarter q of view j, 64 columns per load,
 // scales by c_g and reduces with a tree.  Measured faster than the slot ring
-// when every tile carries two MMAs; the results are identical.
+// when every tile carries two MMAs; the results are identical.  With one
+// group size for both views (dY of the backward pass) the pair kernel below
+// does the same work in half the MMA instructions.
 constexpr int kGrpStages = 5;     // A tiles in flight (each held until both MMAs are done)
 constexpr int kGrpGroups = 2;
 constexpr int kGrpEpiWarps = 8 * kGrpGroups;
@@ -1004,6 +1006,204 @@ dual_amax_group_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, i
   tc_fence_before_sync();
   __syncthreads();
   if (warp == kGrpMmaWarp) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+
+// ------------------------------------ both views rotated with one group size
+// Pairs of tiles: the rotation matrix is the A operand of every MMA and the
+// two tiles of a pair together the N = 256 B operand (an amax does not care
+// how D is laid out): D_row[n][r] = sum_k B[k][n] T[r][k] over the pair's 256
+// tile rows r (K-major B), D_col[n][c] = sum_r B[r][n] T[r][c] over its 256
+// tile columns c (MN-major B).  A stage holds a pair with its 64-column boxes
+// interleaved -- tile 0 box 0, tile 1 box 0, tile 0 box 1, tile 1 box 1 -- so
+// that both B operands have regular strides; a CTA's odd last tile is loaded
+// twice.  Half the MMA instructions of the group kernel for the same work,
+// and a quarter fewer operand bytes read from shared memory.
+constexpr int kPairStages = 3;
+constexpr uint32_t kPairBytes = 2 * kTileBytes;
+constexpr int kPairEpiWarps = 16;  // eight per view: lane quarter q, column half h
+constexpr int kPairThreads = (kPairEpiWarps + 2) * 32;
+constexpr int kPairProducerWarp = kPairEpiWarps, kPairMmaWarp = kPairEpiWarps + 1;
+constexpr size_t kPairDynSmem = kPairStages * kPairBytes + kTileBytes + 1024;
+
+struct PairDualShared {
+  uint64_t full[kPairStages];
+  uint64_t sfree[kPairStages];
+  uint64_t tfull[2];  // view v's accumulator holds the pair's result
+  uint64_t tfree[2];  // ... and has been loaded by the view's eight warps
+  uint32_t tmem_base;
+  uint32_t issued_a;
+  uint32_t issued_mma;
+  int abort_flag;
+  unsigned int warp_max[2][kPairEpiWarps];
+};
+static_assert(kPairDynSmem + sizeof(PairDualShared) <= 227u * 1024u, "pair pre-pass shared memory");
+
+__global__ void __launch_bounds__(kPairThreads, 1)
+dual_amax_pair_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols, uint64_t seed, int g,
+                      unsigned int* __restrict__ amax_r, unsigned int* __restrict__ amax_c) {
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ __align__(8) PairDualShared sh;
+  uint8_t* pairs = align_1024(dyn_smem);
+  uint8_t* bmat = pairs + kPairStages * kPairBytes;
+
+  const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
+  const PhiloxKey key = philox_key(seed);
+  const TileGrid tg{static_cast<uint32_t>((rows + kTile - 1) / kTile), static_cast<uint32_t>((cols + kTile - 1) / kTile),
+                    static_cast<uint32_t>(NVFP4_MMA_BAND_ROWS)};
+  const int64_t n_tiles = static_cast<int64_t>(tg.n_rt) * tg.n_ct;
+  const int64_t step = gridDim.x;
+  const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - blockIdx.x + step - 1) / step : 0;
+  const int64_t my_pairs = (my_tiles + 1) / 2;
+
+  if (tid == kPairProducerWarp * 32) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.sfree[s], 1);
+    }
+    for (int v = 0; v < 2; ++v) {
+      mbar_init(&sh.tfull[v], 1);
+      mbar_init(&sh.tfree[v], 8);
+    }
+    sh.issued_a = 0;
+    sh.issued_mma = 0;
+    sh.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kPairMmaWarp) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  allow_dependent_launch();
+  const uint32_t tmem_base = sh.tmem_base;
+  if (warp != kPairProducerWarp) {
+    const uint32_t bt = warp < kPairProducerWarp ? tid : tid - 32, nb = kPairThreads - 32;
+    build_rotation_b(bmat, key, bt, nb, g);
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 2, %0;" ::"r"(nb) : "memory");
+  }
+
+  if (warp == kPairProducerWarp) {
+    if (lane == 0) {
+      grid_dependency_wait();
+      prefetch_tensormap(&tmap);
+      for (int64_t p = 0; p < my_pairs; ++p) {
+        const int s = static_cast<int>(p % kPairStages);
+        const uint32_t u = static_cast<uint32_t>(p / kPairStages);
+        if (p >= kPairStages && !mbar_wait(&sh.sfree[s], (u - 1) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        if (*reinterpret_cast<volatile int*>(&sh.abort_flag)) break;
+        const int64_t t0 = blockIdx.x + 2 * p * step;
+        const int64_t t1 = 2 * p + 1 < my_tiles ? t0 + step : t0;
+        uint32_t rt0, ct0, rt1, ct1;
+        tg.coords(static_cast<uint32_t>(t0), rt0, ct0);
+        tg.coords(static_cast<uint32_t>(t1), rt1, ct1);
+        const int32_t x0 = static_cast<int32_t>(ct0 * kTile), y0 = static_cast<int32_t>(rt0 * kTile);
+        const int32_t x1 = static_cast<int32_t>(ct1 * kTile), y1 = static_cast<int32_t>(rt1 * kTile);
+        mbar_arrive_expect_tx(&sh.full[s], kPairBytes);
+        uint8_t* dst = pairs + s * kPairBytes;
+        tma_load_2d(dst, &tmap, x0, y0, &sh.full[s]);
+        tma_load_2d(dst + kBoxBytes, &tmap, x1, y1, &sh.full[s]);
+        tma_load_2d(dst + 2 * kBoxBytes, &tmap, x0 + 64, y0, &sh.full[s]);
+        tma_load_2d(dst + 3 * kBoxBytes, &tmap, x1 + 64, y1, &sh.full[s]);
+        sh.issued_a = (sh.issued_a & ~(0x101u << s)) | (1u << s) | ((u & 1u) << (8 + s));
+      }
+    }
+  } else if (warp == kPairMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_r = idesc_bf16_f32(kTile, 2 * kTile, 0u);
+      constexpr uint32_t idesc_c = idesc_bf16_f32(kTile, 2 * kTile, 0u) | (1u << 16);  // B MN-major
+      const uint32_t b_addr = smem_u32(bmat);
+      for (int64_t p = 0; p < my_pairs; ++p) {
+        const int s = static_cast<int>(p % kPairStages);
+        if (!mbar_wait(&sh.full[s], static_cast<uint32_t>(p / kPairStages) & 1u)) {
+          atomicExch(&sh.abort_flag, 1);
+          break;
+        }
+        const uint32_t pair_addr = smem_u32(pairs + s * kPairBytes);
+        bool ok = true;
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          if (p > 0 && !mbar_wait(&sh.tfree[v], static_cast<uint32_t>(p - 1) & 1u)) {
+            atomicExch(&sh.abort_flag, 1);
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t d = tmem_base + v * 256;
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(b_addr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
+            const uint64_t bdesc = v == 0 ? smem_desc_sw128(pair_addr + (kk >> 2) * 2 * kBoxBytes + (kk & 3) * 32, 16, 1024)
+                                          : smem_desc_sw128(pair_addr + kk * 2048, kBoxBytes, 1024);
+            umma_bf16(d, adesc, bdesc, v == 0 ? idesc_r : idesc_c, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&sh.tfull[v]);
+          sh.issued_mma = (sh.issued_mma & ~(0x101u << v)) | (1u << v) | ((static_cast<uint32_t>(p) & 1u) << (8 + v));
+        }
+        if (!ok) break;
+        umma_commit(&sh.sfree[s]);
+      }
+    }
+  } else {
+    const uint32_t v = warp >> 3, q = warp & 3u, h = (warp >> 2) & 1u;
+    grid_dependency_wait();
+    float m = 0.0f;
+    for (int64_t p = 0; p < my_pairs; ++p) {
+      if (!mbar_wait(&sh.tfull[v], static_cast<uint32_t>(p) & 1u)) {
+        atomicExch(&sh.abort_flag, 1);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t base = tmem_base + ((32u * q) << 16) + v * 256 + h * 128;
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        float vals[64];
+        tmem_ld64_wait(base + 64 * hh, vals);
+        if (hh == 1) {
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.tfree[v]);
+        }
+        m = absmax64(vals, m);
+      }
+    }
+    m = __fmul_rn(rht_scale_of(g), m);
+    const unsigned int bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
+    if (lane == 0) sh.warp_max[v][warp & 7u] = bits;
+  }
+
+  __syncthreads();
+  const bool failed = *reinterpret_cast<volatile int*>(&sh.abort_flag) != 0;
+  if (failed) {
+    if (tid == kPairProducerWarp * 32)
+      for (int s = 0; s < kPairStages; ++s)
+        if ((sh.issued_a >> s) & 1u) mbar_wait(&sh.full[s], (sh.issued_a >> (8 + s)) & 1u);
+    if (tid == kPairMmaWarp * 32)
+      for (int v = 0; v < 2; ++v)
+        if ((sh.issued_mma >> v) & 1u) mbar_wait(&sh.tfull[v], (sh.issued_mma >> (8 + v)) & 1u);
+  }
+  if (tid == 0) {
+    unsigned int mr = 0, mc = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      mr = max(mr, sh.warp_max[0][w]);
+      mc = max(mc, sh.warp_max[1][w]);
+    }
+    atomicMax(amax_r, failed ? 0x7FC00000u : mr);
+    atomicMax(amax_c, failed ? 0x7FC00000u : mc);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == kPairMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, 512);
   }
@@ -1483,10 +1683,21 @@ cudaError_t launch_amax_dual_mma(const void* x, int64_t rows, int64_t cols, int6
                                  uint64_t seed, float* amax_r, float* amax_c, cudaStream_t stream) {
   // the row view straight from the tile: the slot ring, a group of one
   if (g_r == 0) return launch_amax_dual_ring(1, &x, &rows, &cols, &ld, g_r, g_c, seed, &amax_r, &amax_c, stream);
-  // both views rotated: the group kernel
   CUtensorMap map;
   if (!make_map(&map, x, rows, cols, ld)) return cudaErrorInvalidValue;
   LaunchGeom geom;
+  if (g_r == g_c) {
+    // both views rotated with one group size: pairs of tiles per MMA
+    cudaError_t e = launch_geometry(dual_amax_pair_kernel, kPairThreads, kPairDynSmem, 1, &geom);
+    if (e != cudaSuccess) return e;
+    const int64_t n_tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
+    const int64_t grid = n_tiles < int64_t(geom.sms) ? n_tiles : int64_t(geom.sms);
+    if (grid == 0) return cudaSuccess;
+    return launch_overlapped(dual_amax_pair_kernel, static_cast<unsigned>(grid), kPairThreads, kPairDynSmem, stream,
+                             map, rows, cols, seed, g_r, reinterpret_cast<unsigned int*>(amax_r),
+                             reinterpret_cast<unsigned int*>(amax_c));
+  }
+  // both views rotated, different group sizes: the group kernel
   cudaError_t e = launch_geometry(dual_amax_group_kernel, kGrpThreads, kGrpDynSmem, 1, &geom);
   if (e != cudaSuccess) return e;
   const int64_t n_tiles = ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);

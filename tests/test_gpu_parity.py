@@ -378,6 +378,8 @@ def test_if4_int4_rounding_ties():
     ((256, 384), 128, 128), ((640, 384), 0, 128), ((384, 1280), 128, 0), ((512, 512), 16, 64),
     ((256, 256), 0, 0), ((1280, 896), 32, 128),
     ((96, 256), 32, 32),      # below one tensor-core tile: two single pre-passes
+    ((384, 19328), 128, 128),  # 453 tiles: CTAs with odd and even tile counts, several tile pairs each
+    ((1280, 896), 64, 64),
 ])
 def test_amax_dual_equals_two_single_passes(shape, g_row, g_col):
     """nvfp4_amax_dual (both layouts from one read) gives the two single-layout
