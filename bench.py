@@ -67,6 +67,8 @@ NCU_TRAFFIC = {
         472467456 + 224157952,
     ("159b0bcef2cc77d9", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
         472862976 + 224496384,
+    ("3bbcfdfa5970de20", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
+        472672000 + 224679936,
 }
 
 
