@@ -69,6 +69,8 @@ NCU_TRAFFIC = {
         472862976 + 224496384,
     ("3bbcfdfa5970de20", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
         472672000 + 224679936,
+    ("886b5cad3ef870ce", "quantize_dual dy (dy.rowwise.ms_eden.g128 + dy.transposed.ms_eden.g128)"):
+        472838144 + 224669440,
 }
 
 

@@ -721,7 +721,7 @@ __device__ __forceinline__ BlockOut quantize_block(const float* z, float s_g, co
 struct PairRng {
   PhiloxKey key;
   uint64_t elem_a, elem_b;  // view index of element 0 of block a / b (multiples of 16)
-  float u_a, u_b;           // scale uniforms of block a / b (MS-EDEN)
+  uint32_t k_a, k_b;        // 16-bit scale draws of block a / b (MS-EDEN): U = k 2^-16
 };
 
 // Per-launch constants of the block-scale step: the tensor scale s_g, the
@@ -784,29 +784,23 @@ __device__ __forceinline__ uint32_t e4m3x2_rne_sat(float a, float b) {
   return out;
 }
 
-// Two E4M3 codes (bits 0..7 and 8..15, each < 0x7F) -> two floats.
-__device__ __forceinline__ float2 e4m3x2_decode(uint32_t codes) {
-  uint32_t h2;
-  const uint16_t in = static_cast<uint16_t>(codes & 0x7F7Fu);
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
-  const __half2 p = *reinterpret_cast<const __half2*>(&h2);
-  return f2(__low2float(p), __high2float(p));
-}
-
-// Stochastic rounding of two t >= 0 onto E4M3, the two-lane form of e4m3_sr:
-// bits 0..7 for t.x with the uniform ua, bits 8..15 for t.y with ub.  Each
-// byte stays in 0..0x7F: the RNE code is lowered only when it decodes above
-// t (so it is nonzero), and 0x7E + 1 = 0x7F decodes to NaN, which never
-// rounds up.
-__device__ __forceinline__ uint32_t e4m3x2_sr(float2 t, float ua, float ub) {
-  uint32_t lo = e4m3x2_rne_sat(t.x, t.y);
-  const float2 d = e4m3x2_decode(lo);
-  lo -= (d.x > t.x ? 1u : 0u) + (d.y > t.y ? 0x100u : 0u);
-  const float2 l = e4m3x2_decode(lo);
-  const float2 h = e4m3x2_decode(lo + 0x0101u);
-  const float2 below = mul2_rn(f2(ua, ub), sub2_rn(h, l));  // exact: the gap is a power of two
-  const float2 above = sub2_after_mul(t, l);                   // exact (t is a rounded product)
-  return lo + (below.x < above.x ? 1u : 0u) + (below.y < above.y ? 0x100u : 0u);
+// Stochastic rounding of two t >= 0 onto E4M3 (the rule of e4m3_sr) with the
+// 16-bit draws ka, kb (U = k 2^-16): bits 0..7 for t.x, 8..15 for t.y, each in
+// 0..0x7E, on the bits of the floats.  a1 = min(max(t, RU(t/2 + 2^-7)), 448):
+// below 2^-6, E4M3's subnormal range (spacing 2^-9), a1 = RU(t/2 + 2^-7) lies
+// in [2^-7, 2^-6), whose three kept mantissa bits are floor(t / 2^-9) and whose
+// 20 bits below hold the fraction rounded upward on their grid (exact for a
+// comparison with the integer 16k); from 2^-6 on a1 = t, whose 20 bits below
+// the kept three are the fraction of its E4M3 interval.  Either way the code
+// is (exponent field << 3 | kept bits) - 960, and t goes up iff U < fraction
+// iff 16k < low20 iff low20 + 2^20 - 1 - 16k carries into the kept bits; 448
+// (0x7E, the largest finite code) has low20 = 0 and never goes up.
+__device__ __forceinline__ uint32_t e4m3x2_sr(float2 t, uint32_t ka, uint32_t kb) {
+  const float a = fminf(fmaxf(t.x, __fmaf_ru(t.x, 0.5f, 0x1p-7f)), 448.0f);
+  const float b = fminf(fmaxf(t.y, __fmaf_ru(t.y, 0.5f, 0x1p-7f)), 448.0f);
+  const uint32_t ca = ((__float_as_uint(a) + 0xFFFFFu - (ka << 4)) >> 20) - 960u;
+  const uint32_t cb = ((__float_as_uint(b) + 0xFFFFFu - (kb << 4)) >> 20) - 960u;
+  return ca | (cb << 8);
 }
 
 // Stochastic rounding of one block of 16 scaled values; elem = view index of element 0.
@@ -1076,7 +1070,7 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
       const float qa = __fdiv_rn(num.x, den.x), qb = __fdiv_rn(num.y, den.y);
       const float ca = (num.x > 0.0f && den.x > 0.0f) ? qa : 1.0f;
       const float cb = (num.y > 0.0f && den.y > 0.0f) ? qb : 1.0f;
-      const uint32_t S = e4m3x2_sr(mul2_rn(dS, f2(ca, cb)), rng.u_a, rng.u_b);
+      const uint32_t S = e4m3x2_sr(mul2_rn(dS, f2(ca, cb)), rng.k_a, rng.k_b);
       oa.scale = S & 0xFFu;
       ob.scale = S >> 8;
     } else {  // kIF4
@@ -1124,21 +1118,21 @@ __device__ __forceinline__ void quantize_pair(const float2 (&z)[16], const Scale
   }
 }
 
-// Scale uniforms of N consecutive view blocks b0 .. b0+N-1 (MS-EDEN): one
-// Philox call when they lie in one group of eight, two otherwise.
+// 16-bit scale draws of N consecutive view blocks b0 .. b0+N-1 (MS-EDEN):
+// one Philox call when they lie in one group of eight, two otherwise.
 template <int N>
-__device__ __forceinline__ void block_uniforms(PhiloxKey key, uint64_t b0, float (&u)[N]) {
+__device__ __forceinline__ void block_draws(PhiloxKey key, uint64_t b0, uint32_t (&k)[N]) {
   const uint32_t first = static_cast<uint32_t>(b0 & 7u);
   const uint4 w0 = philox_call(key, b0 >> 3, kTagBlock);
   if (first + N <= 8) {
 #pragma unroll
-    for (int k = 0; k < N; ++k) u[k] = uniform16(half_word(w0, first + k));
+    for (int j = 0; j < N; ++j) k[j] = half_word(w0, first + j);
   } else {
     const uint4 w1 = philox_call(key, (b0 >> 3) + 1, kTagBlock);
 #pragma unroll
-    for (int k = 0; k < N; ++k) {
-      const uint32_t i = first + k;
-      u[k] = uniform16(i < 8 ? half_word(w0, i) : half_word(w1, i - 8));
+    for (int j = 0; j < N; ++j) {
+      const uint32_t i = first + j;
+      k[j] = i < 8 ? half_word(w0, i) : half_word(w1, i - 8);
     }
   }
 }

@@ -49,12 +49,12 @@ __device__ __forceinline__ void quantize_store64(const float2 (&z)[2][16], const
                                                  int64_t vrow, int64_t vcol0, int64_t vcols, uint8_t* codes,
                                                  uint8_t* scales, bool codes_aligned16, bool scales_aligned4) {
   const uint64_t e0 = static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols) + static_cast<uint64_t>(vcol0);
-  float u[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  if constexpr (MODE == kMSEDEN) block_uniforms<4>(key, e0 >> 4, u);
+  uint32_t kd[4] = {0u, 0u, 0u, 0u};
+  if constexpr (MODE == kMSEDEN) block_draws<4>(key, e0 >> 4, kd);
   BlockOut o[4];
 #pragma unroll
   for (int p = 0; p < 2; ++p) {
-    const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, u[2 * p], u[2 * p + 1]};
+    const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, kd[2 * p], kd[2 * p + 1]};
     quantize_pair<MODE, TBL>(z[p], sc, rng, o[2 * p], o[2 * p + 1]);
   }
   store64(o, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);

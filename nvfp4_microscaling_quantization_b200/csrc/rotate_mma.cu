@@ -162,7 +162,7 @@ __device__ __forceinline__ void quantize_tmem_row(uint32_t taddr, uint64_t* free
                                                   bool scales_aligned4, uint8_t* codes, uint8_t* scales) {
   const uint32_t lane = threadIdx.x & 31u;
   const float2 c2 = f2(RhtConst<G>::c, RhtConst<G>::c);
-  // MS-EDEN scale uniforms: when a thread owns a whole 128-column row of the
+  // MS-EDEN scale draws: when a thread owns a whole 128-column row of the
   // tile and view rows hold whole groups of eight blocks, its eight blocks
   // take the eight draws of one Philox call
   uint4 wu = make_uint4(0u, 0u, 0u, 0u);
@@ -179,13 +179,13 @@ __device__ __forceinline__ void quantize_tmem_row(uint32_t taddr, uint64_t* free
     // one pair of blocks at a time: load 32 columns, quantize, then the next 32
     const bool valid = vrow < vrows && vcol0 < vcols;
     const uint64_t e0 = static_cast<uint64_t>(vrow) * static_cast<uint64_t>(vcols) + static_cast<uint64_t>(vcol0);
-    float u[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    uint32_t kd[4] = {0u, 0u, 0u, 0u};
     if constexpr (MODE == kMSEDEN) {
       if (row_blocks8) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b) u[b] = uniform16(half_word(wu, 4 * h + b));
+        for (int b = 0; b < 4; ++b) kd[b] = half_word(wu, 4 * h + b);
       } else {
-        block_uniforms<4>(key, e0 >> 4, u);
+        block_draws<4>(key, e0 >> 4, kd);
       }
     }
     BlockOut o[4];
@@ -201,7 +201,7 @@ __device__ __forceinline__ void quantize_tmem_row(uint32_t taddr, uint64_t* free
       float2 zp[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) zp[i] = mul2_rn(f2(v[2 * i], v[2 * i + 1]), c2);
-      const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, u[2 * p], u[2 * p + 1]};
+      const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, kd[2 * p], kd[2 * p + 1]};
       quantize_pair<MODE>(zp, sc, rng, o[2 * p], o[2 * p + 1]);
     }
     if (valid) store64(o, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);
@@ -1258,7 +1258,7 @@ __device__ __forceinline__ void quantize_smem_row(const uint8_t* tile, uint32_t 
         z[2 * i] = f2(a0, b0);
         z[2 * i + 1] = f2(a1, b1);
       }
-      const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, 0.0f, 0.0f};
+      const PairRng rng{key, e0 + 32 * p, e0 + 32 * p + 16, 0u, 0u};
       quantize_pair<MODE>(z, sc, rng, o[2 * p], o[2 * p + 1]);
     }
     if (valid) store64(o, vrow, vcol0, vcols, codes, scales, codes_aligned16, scales_aligned4);

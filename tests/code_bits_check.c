@@ -26,6 +26,12 @@
  *     Rule: |k| = |clamp(RNE(RN(y K1)), -7, 7)| with K1 = RN(7/6).
  *     Kernel form (restated): s = RN(RN(min(|y|, 6) K1) + 1.5 2^23), |k| =
  *     the low byte of s (no clamp on s: RN(6 K1) = 7).
+ * (2c) Stochastic rounding onto E4M3 (MS-EDEN's corrected scale t >= 0).
+ *     Rule: lo = the largest E4M3 value <= t (448 for t >= 448), hi the next;
+ *     with U = k 2^-16 the code goes up iff U (hi - lo) < t - lo (binary64,
+ *     exact).
+ *     Kernel form (restated): a1 = min(max(t, RU(t/2 + 2^-7)), 448); code =
+ *     ((bits(a1) + 2^20 - 1 - 16k) >> 20) - 960.
  * (3) E2M0 codes and magnitudes (NVFP3, MXFP3, IF3's E2M0 option).
  *     Rule: the nearest of {0, 1, 2, 4} to |y| (distances in binary64 from
  *     min(|y|, 8), exact), a tie going to the even code index (0.5 -> 0,
@@ -313,6 +319,69 @@ int64_t if4_level_check(int64_t n_random, int variant, int64_t* checked) {
     CHECK(nextafterf(x, -INFINITY));
   }
   for (int64_t r = 0; r < n_random; ++r) CHECK(from_bits((uint32_t)next64() & 0xC1FFFFFFu));
+#undef CHECK
+  *checked = n;
+  return bad;
+}
+
+/* ------------------------------------------------------------ E4M3 SR */
+static double e4m3_value(uint32_t c) {
+  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+  return e == 0 ? m * 0x1p-9 : (1.0 + m / 8.0) * ldexp(1.0, (int)e - 7);
+}
+
+static uint32_t e4m3_sr_rule(float t, uint32_t k) {
+  if (t >= 448.0f) return 0x7Eu;
+  uint32_t lo = 0;
+  while (lo + 1 < 0x7Fu && e4m3_value(lo + 1) <= (double)t) ++lo;
+  const double l = e4m3_value(lo), h = e4m3_value(lo + 1);
+  return (double)k * 0x1p-16 * (h - l) < (double)t - l ? lo + 1 : lo;
+}
+
+static uint32_t e4m3_sr_kernel(float t, uint32_t k) {
+  const float a1 = fminf(fmaxf(t, fma_up(t, 0.5f, 0x1p-7f)), 448.0f);
+  return ((to_bits(a1) + 0xFFFFFu - (k << 4)) >> 20) - 960u;
+}
+
+/* Values t: every E4M3 value and its binary32 neighbours, the decision point
+ * lo + k 2^-16 (hi - lo) of every interval at a stride of draws with its
+ * neighbours and the neighbouring draws, values past 448, and random binary32
+ * values in [0, 2^10).  Variant 1 drops the upward rounding of t/2 + 2^-7. */
+int64_t e4m3_sr_check(int64_t n_random, int variant, int64_t* checked) {
+  int64_t bad = 0, n = 0;
+  rng_state = 0x8C2F1E5A77D3B901ull;
+#define CHECK(tv, kv)                                                        \
+  do {                                                                       \
+    const float t_ = (tv);                                                   \
+    const uint32_t k_ = (kv);                                                \
+    uint32_t got = e4m3_sr_kernel(t_, k_);                                   \
+    if (variant == 1) {                                                      \
+      volatile float h_ = t_ * 0.5f;                                         \
+      volatile float g_ = h_ + 0x1p-7f;                                      \
+      const float a_ = fminf(fmaxf(t_, g_), 448.0f);                         \
+      got = ((to_bits(a_) + 0xFFFFFu - (k_ << 4)) >> 20) - 960u;             \
+    }                                                                        \
+    ++n;                                                                     \
+    bad += got != e4m3_sr_rule(t_, k_);                                      \
+  } while (0)
+  for (uint32_t c = 0; c < 0x7Fu; ++c) {
+    const float v = (float)e4m3_value(c);
+    const float ts[3] = {v, nextafterf(v, INFINITY), c ? nextafterf(v, -INFINITY) : v};
+    for (int i = 0; i < 3; ++i)
+      for (uint32_t k = 0; k < 65536u; k += 251u) CHECK(ts[i], k);
+  }
+  for (uint32_t c = 0; c < 0x7Eu; ++c) {
+    const double l = e4m3_value(c), h = e4m3_value(c + 1);
+    for (uint32_t k = 1; k < 65535u; k += 97u) {
+      const float t = (float)(l + k * 0x1p-16 * (h - l));
+      const float ts[3] = {t, nextafterf(t, INFINITY), nextafterf(t, -INFINITY)};
+      for (int i = 0; i < 3; ++i)
+        for (int d = -1; d <= 1; ++d) CHECK(ts[i], (uint32_t)((int)k + d));
+    }
+  }
+  for (float t = 448.0f; t < 1e30f; t *= 3.7f) CHECK(t, (uint32_t)(next64() & 0xFFFFu));
+  for (int64_t r = 0; r < n_random; ++r)
+    CHECK(from_bits((uint32_t)next64() & 0x447FFFFFu), (uint32_t)(next64() & 0xFFFFu));
 #undef CHECK
   *checked = n;
   return bad;

@@ -1,6 +1,7 @@
 """The kernels' bit-level formation of codes, pinned on the CPU.
 
-Stochastic rounding onto E2M1, the INT4 levels of NVINT4 and IF4, the INT3
+Stochastic rounding onto E2M1 and onto E4M3 (MS-EDEN's scale), the INT4
+levels of NVINT4 and IF4, the INT3
 levels of NVINT3 and IF3, and the E2M0 codes of NVFP3, MXFP3 and IF3 are
 formed in the kernels without conversion instructions: integer sums on the
 bits of the floats, and byte permutes that gather eight elements' nibbles
@@ -33,7 +34,7 @@ def checker():
     subprocess.run(["cc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-frounding-math", "-fPIC", "-shared",
                     os.path.join(HERE, "code_bits_check.c"), "-o", so, "-lm"], check=True)
     L = ctypes.CDLL(so)
-    for fn in (L.sr_check, L.int4_check, L.int3_check, L.e2m0_check, L.if4_level_check):
+    for fn in (L.sr_check, L.int4_check, L.int3_check, L.e2m0_check, L.if4_level_check, L.e4m3_sr_check):
         fn.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
         fn.restype = ctypes.c_int64
     return L
@@ -59,6 +60,8 @@ def test_planted_mistakes_are_caught(checker):
     assert bad > 1000 and n > 0
     bad, n = _run(checker.if4_level_check, 1 << 16, variant=1)  # no clamp of |y| at 6
     assert bad > 1000 and n > 0
+    bad, n = _run(checker.e4m3_sr_check, 1 << 16, variant=1)  # t/2 + 2^-7 rounded to nearest
+    assert bad > 100 and n > 0
 
 
 def test_stochastic_rounding_codes(checker):
@@ -89,3 +92,9 @@ def test_if4_integer_level_from_y(checker):
     bad, n = _run(checker.if4_level_check, 1 << 20)
     assert n > 1_000_000
     assert bad == 0, f"{bad} of {n} IF4 integer levels differ from clamp(RNE(RN(y K1)), -7, 7)"
+
+
+def test_e4m3_stochastic_scale_rounding(checker):
+    bad, n = _run(checker.e4m3_sr_check, 1 << 20)
+    assert n > 1_000_000
+    assert bad == 0, f"{bad} of {n} stochastically rounded E4M3 scales differ from the rule"
