@@ -80,7 +80,8 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--e2e-steps", type=int, default=None,
+                   help="steps of the end-to-end measurement (default: --steps)")
     p.add_argument("--cpu-sample-fraction", type=float, default=1.0 / 8,
                    help="fraction of each call's view rows the CPU baseline quantizes")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -912,7 +913,7 @@ def run_e2e(args, calls, tensors, stream, device, world, bytes_per_step):
 
     run(2)
     torch.cuda.synchronize(device)
-    K = max(args.e2e_steps, 1)
+    K = max(args.e2e_steps if args.e2e_steps is not None else args.steps, 1)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world, device.index)
     torch.cuda.synchronize(device)
